@@ -1,0 +1,171 @@
+// KV-injection attention on CUDA cores: the DeepspecContextAttention.attend
+// seam ("mlx-bun 0.2.0 -> 0.4.0" page 75): block queries attend, non-causally
+// and at scale 1.0, over the row's cached context keys followed by the
+// block's own keys. The storage-side split: context keys in chunks plus the
+// block keys as one more part, each reduced to (max, sum, weighted values),
+// then merged by the online-softmax rule.
+//
+// This is the path of the fp32 workload (no tensor cores at its 1e-4 bar).
+#include <float.h>
+#include <math.h>
+
+#include "internal.h"
+#include "common.cuh"
+
+namespace dspark {
+namespace {
+
+constexpr int KT = 16;            // keys per tile
+constexpr int kMaxO = 16;         // O elements per thread (G * hd <= 16 * 256)
+constexpr int kThreads = 256;
+
+// grid (A * nH, n_splits + 1); one CTA = one query head of one row over one key range.
+__global__ void __launch_bounds__(kThreads)
+attn_partial_kernel(AttnArgs a, int G, int nH, int nKv, int hd, int dtype) {
+    extern __shared__ float sm[];
+    float* qs = sm;                       // [G][hd]
+    float* ks = qs + G * hd;              // [KT][hd]
+    float* vs = ks + KT * hd;             // [KT][hd]
+    float* ps = vs + KT * hd;             // [G][KT]
+    float* mrow = ps + G * KT;            // [G]
+    float* lrow = mrow + G;               // [G]
+    float* alpha = lrow + G;              // [G]
+
+    const int b = blockIdx.x / nH, h = blockIdx.x % nH;
+    const int g = h / (nH / nKv);
+    const int split = blockIdx.y;
+    const int tid = threadIdx.x;
+
+    int len = a.len[b];
+    if (len < 0 || len > a.capacity) {
+        if (tid == 0) atomicOr(a.status, DSPARK_DEV_BAD_LENGTH);
+        len = min(max(len, 0), a.capacity);
+    }
+    int k0, k1;
+    const bool blk = split == a.n_splits;
+    if (blk) { k0 = 0; k1 = G; }
+    else { k0 = split * a.chunk; k1 = min(len, k0 + a.chunk); }
+
+    for (int e = tid; e < G * hd; e += kThreads) {
+        const int i = e / hd, d = e % hd;
+        qs[e] = load_any(a.q, (((int64_t)b * G + i) * nH + h) * hd + d, a.q_dtype);
+    }
+    for (int i = tid; i < G; i += kThreads) { mrow[i] = -INFINITY; lrow[i] = 0.f; }
+    float o[kMaxO];
+#pragma unroll
+    for (int c = 0; c < kMaxO; ++c) o[c] = 0.f;
+    __syncthreads();
+
+    for (int t0 = k0; t0 < k1; t0 += KT) {
+        const int nt = min(KT, k1 - t0);
+        for (int e = tid; e < KT * hd; e += kThreads) {
+            const int j = e / hd, d = e % hd;
+            float kv = 0.f, vv = 0.f;
+            if (j < nt) {
+                int64_t idx;
+                if (blk) {
+                    idx = (((int64_t)b * G + t0 + j) * nKv + g) * hd + d;
+                    kv = load_any(a.kb, idx, dtype); vv = load_any(a.vb, idx, dtype);
+                } else {
+                    idx = (((int64_t)b * a.capacity + t0 + j) * nKv + g) * hd + d;
+                    kv = load_any(a.kc, idx, dtype); vv = load_any(a.vc, idx, dtype);
+                }
+            }
+            ks[e] = kv; vs[e] = vv;
+        }
+        __syncthreads();
+        // scores
+        for (int e = tid; e < G * KT; e += kThreads) {
+            const int i = e / KT, j = e % KT;
+            float s = -INFINITY;
+            if (j < nt) {
+                s = 0.f;
+                for (int d = 0; d < hd; ++d) s = fmaf(qs[i * hd + d], ks[j * hd + d], s);
+            }
+            ps[e] = s;
+        }
+        __syncthreads();
+        // online softmax per query row
+        for (int i = tid; i < G; i += kThreads) {
+            float mx = mrow[i];
+            for (int j = 0; j < nt; ++j) mx = fmaxf(mx, ps[i * KT + j]);
+            const float al = expf(mrow[i] - mx);        // mrow = -inf on the first tile: 0
+            float l = lrow[i] * al;
+            for (int j = 0; j < KT; ++j) {
+                const float p = j < nt ? expf(ps[i * KT + j] - mx) : 0.f;
+                ps[i * KT + j] = p;
+                l += p;
+            }
+            mrow[i] = mx; lrow[i] = l; alpha[i] = al;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < kMaxO; ++c) {
+            const int e = tid + c * kThreads;
+            if (e < G * hd) {
+                const int i = e / hd, d = e % hd;
+                float acc = o[c] * alpha[i];
+                for (int j = 0; j < nt; ++j) acc = fmaf(ps[i * KT + j], vs[j * hd + d], acc);
+                o[c] = acc;
+            }
+        }
+        __syncthreads();
+    }
+
+    const int S1 = a.n_splits + 1;
+    const int64_t base = ((int64_t)blockIdx.x * S1 + split) * G;   // (b, h, split) major
+#pragma unroll
+    for (int c = 0; c < kMaxO; ++c) {
+        const int e = tid + c * kThreads;
+        if (e < G * hd) a.part_o[base * hd + e] = o[c];
+    }
+    for (int i = tid; i < G; i += kThreads) {
+        a.part_ml[(base + i) * 2] = mrow[i];
+        a.part_ml[(base + i) * 2 + 1] = lrow[i];
+    }
+}
+
+// grid (A * nH * G), block hd: merge the splits of one query row of one head.
+__global__ void attn_merge_kernel(AttnArgs a, int G, int nH, int hd) {
+    const int row = blockIdx.x;                 // ((b * nH) + h) * G + i
+    const int i = row % G, bh = row / G;
+    const int b = bh / nH, h = bh % nH;
+    const int d = threadIdx.x;
+    const int S1 = a.n_splits + 1;
+    float M = -INFINITY;
+    for (int s = 0; s < S1; ++s) M = fmaxf(M, a.part_ml[(((int64_t)bh * S1 + s) * G + i) * 2]);
+    float num = 0.f, den = 0.f;
+    for (int s = 0; s < S1; ++s) {
+        const int64_t base = ((int64_t)bh * S1 + s) * G + i;
+        const float m = a.part_ml[base * 2];
+        if (m == -INFINITY) continue;
+        const float w = expf(m - M);
+        den += w * a.part_ml[base * 2 + 1];
+        num += w * a.part_o[base * hd + d];
+    }
+    store_any(a.out, (((int64_t)b * G + i) * nH + h) * hd + d, a.out_dtype, num / den);
+}
+
+}  // namespace
+
+size_t attn_simt_smem(int G, int hd) {
+    return sizeof(float) * ((size_t)G * hd + 2 * (size_t)KT * hd + (size_t)G * KT + 3 * (size_t)G);
+}
+
+cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
+    const Dims& d = m->d;
+    const size_t smem = attn_simt_smem(d.gamma, d.hd);
+    static thread_local int configured_dev = -1;
+    if (configured_dev != m->device) {
+        cudaFuncSetAttribute(attn_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        configured_dev = m->device;
+    }
+    dim3 grid(a.A * d.nH, a.n_splits + 1);
+    attn_partial_kernel<<<grid, kThreads, smem, s>>>(a, d.gamma, d.nH, d.nKv, d.hd, d.dtype);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_merge_kernel<<<a.A * d.nH * d.gamma, d.hd, 0, s>>>(a, d.gamma, d.nH, d.hd);
+    return cudaGetLastError();
+}
+
+}  // namespace dspark

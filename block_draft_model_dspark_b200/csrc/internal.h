@@ -1,0 +1,169 @@
+// Internal declarations of libdspark (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+#include <string>
+#include <vector>
+
+#include "../../include/dspark.h"
+
+namespace dspark {
+
+using bf16 = __nv_bfloat16;
+
+// ---------------------------------------------------------------- errors
+void set_error(const std::string& msg);
+#define DSPARK_FAIL(code, msg)                 \
+    do {                                       \
+        ::dspark::set_error(msg);              \
+        return (code);                         \
+    } while (0)
+#define DSPARK_CUDA_CHECK(expr)                                                           \
+    do {                                                                                  \
+        cudaError_t e_ = (expr);                                                          \
+        if (e_ != cudaSuccess)                                                            \
+            DSPARK_FAIL(DSPARK_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e_)); \
+    } while (0)
+
+// A weight matrix as the kernels see it: dense T [n, k] (row stride k), or
+// affine 4-bit words [n, k/8] + bf16 scales/biases [n, k/group].
+struct MatRef {
+    const void* w = nullptr;
+    const bf16* scales = nullptr;
+    const bf16* biases = nullptr;
+    int64_t n = 0, k = 0;
+    bool quant = false;
+};
+
+// Device layout of everything dspark_model_create places in model_ws.
+struct ModelWs {
+    int32_t* status = nullptr;      // device status word (+ padding)
+    double* inv_freq = nullptr;     // [hd/2] RoPE inverse frequencies (0 = identity lane)
+    void* wqk = nullptr;            // per layer [(nH+nKv)*hd, H] (dense) or words
+    void* wgu = nullptr;            // per layer [2I, H]
+    void* wk_all = nullptr;         // [Lyr*nKv*hd, H]
+    bf16* wqk_s = nullptr; bf16* wqk_b = nullptr;   // quantized scales / biases of the stacks
+    bf16* wgu_s = nullptr; bf16* wgu_b = nullptr;
+    bf16* wk_all_s = nullptr; bf16* wk_all_b = nullptr;
+};
+
+constexpr int kMaxLayers = 64;
+struct LayerPtrs { const void* p[kMaxLayers]; };
+
+struct LayerRef {
+    MatRef qk, o, gu, down;   // qk = [Wq; Wk], gu = [Wg; Wu]
+    const void *q_norm, *k_norm, *in_norm, *post_attn_norm, *pre_ff_norm, *post_ff_norm, *layer_scalar;
+};
+
+struct Dims {
+    int H, Lyr, nH, nKv, hd, grp, I, V, gamma, mask_id, r;
+    int dtype;          // DSPARK_DTYPE_*
+    bool quant;
+    int group;
+    float eps, cap, conf_thr;
+    bool conf_head, conf_markov;
+    int conf_in;        // H (+ r)
+};
+
+}  // namespace dspark
+
+struct dspark_model {
+    dspark_config cfg;
+    dspark::Dims d;
+    dspark::ModelWs ws;
+    std::vector<dspark::LayerRef> layers;
+    dspark::MatRef embed, lm_head, w2, conf_proj, wk_all;
+    const void* w1 = nullptr;
+    const void* final_norm = nullptr;
+    const void* conf_bias = nullptr;
+    int device = 0;
+    int num_sms = 148;
+};
+
+namespace dspark {
+
+// ---------------------------------------------------------------- launch helpers
+// Each returns cudaGetLastError() of its launch.
+
+// SIMT GEMM: out[z][m][n] = sum_{k in split z} X[m,k] * W[n,k]  (fp32 partials),
+// or with softcap (splits must be 1): out[m][n] = cap*tanh(acc/cap) (cap > 0) or acc.
+cudaError_t launch_simt_gemm(const void* X, int64_t ldx, int x_dtype, int w_dtype, const MatRef& W, int group,
+                             int M, int N, int K, int splits, float* out, int64_t ldo, int64_t split_stride,
+                             bool softcap, float cap, cudaStream_t s);
+
+// Context K/V epilogue: raw fp32 [rows, Lyr*nKv*hd] (sum of `splits` partials
+// at split_stride) -> cache rows. Row r = b*Lrows + t is valid when t < n_b.
+struct KvDest {
+    void* k; void* v;
+    int64_t batch_stride;    // elements between batch rows   (= cap * nKv * hd)
+    int64_t layer_stride;    // elements between layers       (= batch * cap * nKv * hd)
+    int capacity;
+};
+struct RowsPlan {
+    int B, Lrows;            // rows are b*Lrows + t
+    int row0;                // first global row index (b*Lrows+t) held by this chunk
+    int nrows;               // rows in this chunk
+    const int32_t* n_valid;  // device [B] or null (all Lrows valid)
+    const int32_t* dst_row0; // device [B] cache row of t = 0, or null (0)
+    const int32_t* pos0;     // device [B] position of t = 0, or null (static_pos)
+    int static_pos;
+};
+cudaError_t launch_kv_epilogue(const dspark_model* m, const float* raw, int splits, int64_t split_stride,
+                               const RowsPlan& rp, const KvDest& dst, cudaStream_t s);
+cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStream_t s);
+
+// Activations of the round (x, q, attention output, gelu*up) are fp32 in the
+// workspace for both model dtypes; only the K/V cache and the block K/V are
+// stored in the model dtype.
+// Block embedding: h = embed[ids]*sqrt(H) (fp32 [M,H]); x = rms(h, w_in0) (fp32 [M,H]).
+cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, float* h, float* x,
+                         int32_t* status, cudaStream_t s);
+// q (fp32) and block k/v (model dtype) heads from the [Wq;Wk] GEMM partials.
+cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
+                               int A, const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s);
+// h += rms(o_proj partials, post_attn); x = rms(h, pre_ff).
+cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
+                              int M, float* h, float* x, cudaStream_t s);
+// act = gelu_tanh(g) * u  (fp32 [M, I]).
+cudaError_t launch_gu_epilogue(const dspark_model* m, const float* part, int splits, int64_t split_stride,
+                               int M, float* act, cudaStream_t s);
+// h = (h + rms(down partials, post_ff)) * layer_scalar; then x = rms(h, next gain)
+// (next gain = next layer's input norm, or the final norm).
+cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
+                                 int M, float* h, float* x, cudaStream_t s);
+
+// Attention: partial pass over context chunks + block keys, then merge.
+struct AttnArgs {
+    const void* q;  const void* kb; const void* vb;  // [A, G, nH, hd] / [A, G, nKv, hd]
+    int q_dtype, out_dtype;                          // DSPARK_DTYPE_* of q and out (kb, vb, cache: model dtype)
+    const void* kc; const void* vc;                  // cache of this layer: [batch, cap, nKv, hd]
+    const int32_t* len; int capacity;
+    void* out;                                       // [A, G, nH, hd]
+    float* part_o; float* part_ml;                   // workspace
+    int A, n_splits, chunk;                          // context splits of `chunk` keys (+1 block split)
+    int32_t* status;
+};
+
+// Markov walk step k: tokens[:,k] from U[:,k,:] + w2 . w1[prev]; prev updated.
+struct WalkArgs {
+    const float* U;            // [A, G, V]
+    int32_t* tokens;           // [A, G]
+    int32_t* prev;             // [A]
+    float* part_val; int32_t* part_idx;  // [nblk, A]
+    uint32_t* ticket;          // one counter, zero at entry
+    int A, nblk, step;
+    int32_t* status;
+};
+cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s);
+cudaError_t launch_walk_init(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V,
+                             int32_t* status, cudaStream_t s);
+// Confidence + lengths (hf = the final-normed hidden, fp32 [M, H]).
+cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const int32_t* anchors, const int32_t* tokens,
+                              int A, float* conf, int32_t* lengths, cudaStream_t s);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace dspark

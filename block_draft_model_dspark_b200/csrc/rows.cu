@@ -1,0 +1,310 @@
+// Row-wise kernels of the round: the block embedding, the fused epilogues
+// that follow each GEMM (norms, RoPE, residual adds, gelu, layer scalar),
+// the context K/V epilogue, and the confidence head with truncation.
+//
+// Each epilogue first sums the GEMM's split-K partials in split order (a
+// fixed order, so results do not depend on scheduling).
+#include <math.h>
+
+#include "internal.h"
+#include "common.cuh"
+
+namespace dspark {
+namespace {
+
+constexpr int kMaxPer = 16;   // columns per thread in the full-row kernels
+
+__device__ __forceinline__ float sum_splits(const float* part, int splits, int64_t stride, int64_t idx) {
+    float v = 0.f;
+    for (int s = 0; s < splits; ++s) v += part[s * stride + idx];
+    return v;
+}
+
+// One element W[n, j] of a (possibly 4-bit) matrix.
+__device__ __forceinline__ float mat_at(const MatRef& W, int dtype, int group, int64_t n, int64_t j) {
+    if (!W.quant) return load_any(W.w, n * W.k + j, dtype);
+    const uint32_t w = static_cast<const uint32_t*>(W.w)[n * (W.k / 8) + j / 8];
+    const int64_t g = n * (W.k / group) + j / group;
+    return fmaf(__bfloat162float(W.scales[g]), (float)((w >> (4 * (j % 8))) & 0xFu), __bfloat162float(W.biases[g]));
+}
+
+// ------------------------------------------------------------------ context K/V
+// grid (rows, Lyr*nKv), block hd/2: thread i owns the RoPE pair (i, i + hd/2).
+__global__ void kv_epilogue_kernel(const float* __restrict__ raw, int splits, int64_t split_stride, int N,
+                                   RowsPlan rp, KvDest dst, const double* __restrict__ inv_freq,
+                                   LayerPtrs k_norms, int nKv, int hd, float eps,
+                                   int dtype, int32_t* status) {
+    __shared__ float red[32];
+    const int r = blockIdx.x;
+    const int rg = rp.row0 + r;
+    const int b = rg / rp.Lrows, t = rg % rp.Lrows;
+    if (rp.n_valid && t >= rp.n_valid[b]) return;
+    const int dst_row = (rp.dst_row0 ? rp.dst_row0[b] : 0) + t;
+    if (dst_row < 0 || dst_row >= dst.capacity) {
+        if (threadIdx.x == 0) atomicOr(status, DSPARK_DEV_BAD_LENGTH);
+        return;
+    }
+    const int pos = (rp.pos0 ? rp.pos0[b] : rp.static_pos) + dst_row;
+    const int l = blockIdx.y / nKv, g = blockIdx.y % nKv;
+    const int half = hd / 2, i = threadIdx.x;
+    const int64_t col = (int64_t)blockIdx.y * hd;
+    const float x1 = sum_splits(raw, splits, split_stride, (int64_t)r * N + col + i);
+    const float x2 = sum_splits(raw, splits, split_stride, (int64_t)r * N + col + i + half);
+    const float ss = block_sum(x1 * x1 + x2 * x2, red);
+    const float rinv = rsqrtf(ss / (float)hd + eps);
+    const float v1 = x1 * rinv, v2 = x2 * rinv;
+    const void* wk = k_norms.p[l];
+    const float k1 = v1 * load_any(wk, i, dtype), k2 = v2 * load_any(wk, i + half, dtype);
+    float sn, cs;
+    rope_sincos(pos, inv_freq[i], &sn, &cs);
+    const int64_t o = (int64_t)l * dst.layer_stride + (int64_t)b * dst.batch_stride + ((int64_t)dst_row * nKv + g) * hd;
+    store_any(dst.v, o + i, dtype, v1);
+    store_any(dst.v, o + i + half, dtype, v2);
+    store_any(dst.k, o + i, dtype, k1 * cs - k2 * sn);
+    store_any(dst.k, o + i + half, dtype, k2 * cs + k1 * sn);
+}
+
+__global__ void commit_len_kernel(int32_t* len, const int32_t* n_new, int B) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < B) len[b] += n_new[b];
+}
+
+// ------------------------------------------------------------------ block embedding
+__global__ void embed_kernel(MatRef E, int dtype, int group, const int32_t* __restrict__ anchors, int gamma,
+                             int mask_id, int V, int H, float scale, const void* __restrict__ w_in,
+                             float eps, float* __restrict__ h, float* __restrict__ x, int32_t* status) {
+    __shared__ float red[32];
+    const int m = blockIdx.x;
+    const int b = m / gamma, t = m % gamma;
+    int id = t == 0 ? anchors[b] : mask_id;
+    if (id < 0 || id >= V) {
+        if (threadIdx.x == 0) atomicOr(status, DSPARK_DEV_BAD_TOKEN);
+        id = min(max(id, 0), V - 1);
+    }
+    float vals[kMaxPer];
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxPer; ++c) {
+        const int j = threadIdx.x + c * blockDim.x;
+        vals[c] = 0.f;
+        if (j < H) {
+            vals[c] = mat_at(E, dtype, group, id, j) * scale;
+            ss += vals[c] * vals[c];
+        }
+    }
+    ss = block_sum(ss, red);
+    const float rinv = rsqrtf(ss / (float)H + eps);
+#pragma unroll
+    for (int c = 0; c < kMaxPer; ++c) {
+        const int j = threadIdx.x + c * blockDim.x;
+        if (j < H) {
+            h[(int64_t)m * H + j] = vals[c];
+            x[(int64_t)m * H + j] = vals[c] * rinv * load_any(w_in, j, dtype);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ q / k / v heads
+// grid (M, nH + nKv), block hd/2.
+__global__ void qk_epilogue_kernel(const float* __restrict__ part, int splits, int64_t split_stride, int N,
+                                   int gamma, int nH, int nKv, int hd, const int32_t* __restrict__ block_pos,
+                                   const double* __restrict__ inv_freq, const void* __restrict__ q_norm,
+                                   const void* __restrict__ k_norm, float eps, int dtype,
+                                   float* __restrict__ q, void* __restrict__ kb, void* __restrict__ vb) {
+    __shared__ float red[32];
+    const int m = blockIdx.x, hh = blockIdx.y;
+    const int b = m / gamma, t = m % gamma;
+    const int pos = block_pos[b] + t;
+    const int half = hd / 2, i = threadIdx.x;
+    const int64_t col = (int64_t)hh * hd;
+    const float x1 = sum_splits(part, splits, split_stride, (int64_t)m * N + col + i);
+    const float x2 = sum_splits(part, splits, split_stride, (int64_t)m * N + col + i + half);
+    const float ss = block_sum(x1 * x1 + x2 * x2, red);
+    const float rinv = rsqrtf(ss / (float)hd + eps);
+    float y1 = x1 * rinv, y2 = x2 * rinv;
+    float sn, cs;
+    rope_sincos(pos, inv_freq[i], &sn, &cs);
+    if (hh < nH) {
+        y1 *= load_any(q_norm, i, dtype);
+        y2 *= load_any(q_norm, i + half, dtype);
+        const int64_t o = ((int64_t)m * nH + hh) * hd;
+        q[o + i] = y1 * cs - y2 * sn;
+        q[o + i + half] = y2 * cs + y1 * sn;
+    } else {
+        const int g = hh - nH;
+        const int64_t o = ((int64_t)m * nKv + g) * hd;
+        store_any(vb, o + i, dtype, y1);
+        store_any(vb, o + i + half, dtype, y2);
+        const float k1 = y1 * load_any(k_norm, i, dtype), k2 = y2 * load_any(k_norm, i + half, dtype);
+        store_any(kb, o + i, dtype, k1 * cs - k2 * sn);
+        store_any(kb, o + i + half, dtype, k2 * cs + k1 * sn);
+    }
+}
+
+// ------------------------------------------------------------------ o_proj / down epilogues
+// mode 0 (o_proj):  h += rms(sum, g1);            x = rms(h, g2)
+// mode 1 (down):    h = (h + rms(sum, g1)) * s;   x = rms(h, g2)   (+ hf32 = x when given)
+__global__ void residual_epilogue_kernel(const float* __restrict__ part, int splits, int64_t split_stride, int H,
+                                         const void* __restrict__ g1, const void* __restrict__ g2,
+                                         const void* __restrict__ scalar, int mode, float eps, int dtype,
+                                         float* __restrict__ h, float* __restrict__ x) {
+    __shared__ float red[32];
+    const int m = blockIdx.x;
+    float a[kMaxPer];
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxPer; ++c) {
+        const int j = threadIdx.x + c * blockDim.x;
+        a[c] = j < H ? sum_splits(part, splits, split_stride, (int64_t)m * H + j) : 0.f;
+        ss += a[c] * a[c];
+    }
+    ss = block_sum(ss, red);
+    const float r1 = rsqrtf(ss / (float)H + eps);
+    const float s = mode == 1 ? load_any(scalar, 0, dtype) : 1.f;
+    float ss2 = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxPer; ++c) {
+        const int j = threadIdx.x + c * blockDim.x;
+        if (j < H) {
+            const float nv = (h[(int64_t)m * H + j] + a[c] * r1 * load_any(g1, j, dtype)) * s;
+            h[(int64_t)m * H + j] = nv;
+            a[c] = nv;
+            ss2 += nv * nv;
+        }
+    }
+    ss2 = block_sum(ss2, red);
+    const float r2 = rsqrtf(ss2 / (float)H + eps);
+#pragma unroll
+    for (int c = 0; c < kMaxPer; ++c) {
+        const int j = threadIdx.x + c * blockDim.x;
+        if (j < H) {
+            x[(int64_t)m * H + j] = a[c] * r2 * load_any(g2, j, dtype);
+        }
+    }
+}
+
+__global__ void gu_epilogue_kernel(const float* __restrict__ part, int splits, int64_t split_stride, int M, int I,
+                                   float* __restrict__ act) {
+    const int64_t total = (int64_t)M * I;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = e / I, i = e % I;
+        const float g = sum_splits(part, splits, split_stride, m * 2 * I + i);
+        const float u = sum_splits(part, splits, split_stride, m * 2 * I + I + i);
+        act[e] = gelu_tanh(g) * u;
+    }
+}
+
+// ------------------------------------------------------------------ confidence + truncation
+// grid A, block 256: c[b,k] = sigmoid(proj . [hf(b,k) ; w1[prev]] + bias); lengths[b].
+__global__ void confidence_kernel(const float* __restrict__ hf32, MatRef P, int dtype, int group,
+                                  const void* __restrict__ w1, const void* __restrict__ bias,
+                                  const int32_t* __restrict__ anchors, const int32_t* __restrict__ tokens,
+                                  int gamma, int H, int r, int with_markov, int V, float thr, int has_head,
+                                  float* __restrict__ conf, int32_t* __restrict__ lengths) {
+    __shared__ float red[32];
+    const int b = blockIdx.x;
+    int len = gamma;
+    const float bz = has_head ? load_any(bias, 0, dtype) : 0.f;
+    for (int k = 0; has_head && k < gamma; ++k) {
+        int prev = k == 0 ? anchors[b] : tokens[b * gamma + k - 1];
+        prev = min(max(prev, 0), V - 1);
+        const int64_t m = (int64_t)b * gamma + k;
+        float z = 0.f;
+        for (int j = threadIdx.x; j < H; j += blockDim.x) z += hf32[m * H + j] * mat_at(P, dtype, group, 0, j);
+        if (with_markov)
+            for (int j = threadIdx.x; j < r; j += blockDim.x)
+                z += load_any(w1, (int64_t)prev * r + j, dtype) * mat_at(P, dtype, group, 0, H + j);
+        z = block_sum(z, red) + bz;
+        const float c = 1.f / (1.f + expf(-z));
+        if (threadIdx.x == 0) {
+            if (conf) conf[m] = c;
+            if (thr > 0.f && c < thr && len == gamma) len = k;
+        }
+    }
+    if (threadIdx.x == 0 && lengths) lengths[b] = len;
+}
+
+int row_threads(int H) {
+    int t = (H + kMaxPer - 1) / kMaxPer;
+    t = (t + 31) / 32 * 32;
+    return t < 32 ? 32 : t;
+}
+
+}  // namespace
+
+cudaError_t launch_kv_epilogue(const dspark_model* m, const float* raw, int splits, int64_t split_stride,
+                               const RowsPlan& rp, const KvDest& dst, cudaStream_t s) {
+    const Dims& d = m->d;
+    if (rp.nrows <= 0) return cudaSuccess;
+    LayerPtrs kn{};
+    for (int l = 0; l < d.Lyr; ++l) kn.p[l] = m->layers[l].k_norm;
+    dim3 grid(rp.nrows, d.Lyr * d.nKv);
+    kv_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(raw, splits, split_stride, d.Lyr * d.nKv * d.hd, rp, dst,
+                                                 m->ws.inv_freq, kn, d.nKv, d.hd, d.eps, d.dtype, m->ws.status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStream_t s) {
+    commit_len_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, n_new, B);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, float* h, float* x, int32_t* status,
+                         cudaStream_t s) {
+    const Dims& d = m->d;
+    embed_kernel<<<A * d.gamma, row_threads(d.H), 0, s>>>(m->embed, d.dtype, d.group, anchors, d.gamma, d.mask_id,
+                                                         d.V, d.H, sqrtf((float)d.H), m->layers[0].in_norm, d.eps,
+                                                         h, x, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
+                               int A, const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s) {
+    const Dims& d = m->d;
+    dim3 grid(A * d.gamma, d.nH + d.nKv);
+    qk_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(part, splits, split_stride, (d.nH + d.nKv) * d.hd, d.gamma, d.nH,
+                                                 d.nKv, d.hd, block_pos, m->ws.inv_freq, m->layers[layer].q_norm,
+                                                 m->layers[layer].k_norm, d.eps, d.dtype, q, kb, vb);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
+                              int M, float* h, float* x, cudaStream_t s) {
+    const Dims& d = m->d;
+    const LayerRef& L = m->layers[layer];
+    residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, splits, split_stride, d.H, L.post_attn_norm,
+                                                            L.pre_ff_norm, nullptr, 0, d.eps, d.dtype, h, x);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gu_epilogue(const dspark_model* m, const float* part, int splits, int64_t split_stride, int M,
+                               float* act, cudaStream_t s) {
+    const Dims& d = m->d;
+    const int64_t total = (int64_t)M * d.I;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 8 * m->num_sms) blocks = 8 * m->num_sms;
+    gu_epilogue_kernel<<<blocks, 256, 0, s>>>(part, splits, split_stride, M, d.I, act);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
+                                 int M, float* h, float* x, cudaStream_t s) {
+    const Dims& d = m->d;
+    const LayerRef& L = m->layers[layer];
+    const bool last = layer + 1 == d.Lyr;
+    const void* next = last ? m->final_norm : m->layers[layer + 1].in_norm;
+    residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, splits, split_stride, d.H, L.post_ff_norm, next,
+                                                            L.layer_scalar, 1, d.eps, d.dtype, h, x);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const int32_t* anchors, const int32_t* tokens,
+                              int A, float* conf, int32_t* lengths, cudaStream_t s) {
+    const Dims& d = m->d;
+    confidence_kernel<<<A, 256, 0, s>>>(hf32, m->conf_proj, d.dtype, d.group, m->w1, m->conf_bias, anchors, tokens,
+                                        d.gamma, d.H, d.r, d.conf_markov ? 1 : 0, d.V, d.conf_thr,
+                                        d.conf_head ? 1 : 0, d.conf_head ? conf : nullptr, lengths);
+    return cudaGetLastError();
+}
+
+}  // namespace dspark

@@ -1,0 +1,260 @@
+/*
+ * dspark.h -- C ABI of libdspark, the DSpark draft round on one B200 (sm_100a).
+ *
+ * The round is the one the "@mlx-bun/inference 0.0.0-stage -> 1.0.0" page
+ * defines in package/src/models/speculative/deepspec.ts (class
+ * DeepspecDrafter): context K/V projection (#projectContextKVRows), the
+ * backbone over the noise block with KV-injection attention
+ * (#forwardBackbone and the DeepspecContextAttention.attend seam of the
+ * "mlx-bun 0.2.0 -> 0.4.0" page 75), logits with softcap (#computeLogits),
+ * the VanillaMarkov walk (#markovStepBias / #selectStep), the confidence
+ * head (#confidence) and the confident-prefix truncation (draftRows).
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer argument named "device" is CUDA device memory the caller
+ *    allocated and owns; the library never allocates device memory. Pointers
+ *    named "host" are host memory, read during the call only.
+ *  - Row-major layouts; dims listed outermost first. "T" is the model's
+ *    storage dtype (dspark_config.dtype: fp32 or bf16).
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream); calls return once enqueued. Results are valid after the stream
+ *    reaches them.
+ *  - Return value: DSPARK_OK or a negative DSPARK_ERR_*; on error nothing was
+ *    enqueued and no output or cache was modified, and dspark_last_error()
+ *    (per host thread) says why. Arguments are validated before any launch.
+ *  - Device-side checks (token ids, cache lengths, bounded waits) record a
+ *    nonzero code in the model's device status word instead of faulting;
+ *    dspark_read_device_status() fetches and clears it.
+ */
+#ifndef DSPARK_H
+#define DSPARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSPARK_OK                    0
+#define DSPARK_ERR_INVALID_ARGUMENT (-1) /* null pointer, bad size, misaligned buffer */
+#define DSPARK_ERR_UNSUPPORTED      (-2) /* a config the drafter page refuses, or outside this build's shapes */
+#define DSPARK_ERR_CAPACITY         (-3) /* an append would pass the cache capacity */
+#define DSPARK_ERR_WORKSPACE        (-4) /* workspace smaller than the matching *_workspace_bytes() */
+#define DSPARK_ERR_CUDA             (-5) /* a CUDA runtime call or launch failed */
+#define DSPARK_ERR_DEVICE           (-6) /* a device-side check failed (see dspark_read_device_status) */
+
+/* Device status codes (bit flags, OR-ed by kernels). */
+#define DSPARK_DEV_BAD_TOKEN     1  /* an anchor or walked token outside [0, vocab) was clamped */
+#define DSPARK_DEV_BAD_LENGTH    2  /* a cache length above capacity was clamped */
+#define DSPARK_DEV_WAIT_TIMEOUT  4  /* a bounded device wait gave up */
+
+#define DSPARK_DTYPE_F32  0
+#define DSPARK_DTYPE_BF16 1
+
+/*
+ * Model configuration: the drafter's config.json keys (deepspec.ts,
+ * DeepspecConfig / readConfig), one int or float each. The three variants
+ * readConfig refuses are refused here too (DSPARK_ERR_UNSUPPORTED):
+ * attention_k_eq_v = 0, a non-vanilla Markov head with markov_rank > 0, and
+ * an activation other than gelu_pytorch_tanh.
+ */
+typedef struct dspark_config {
+    int32_t hidden_size;
+    int32_t num_hidden_layers;
+    int32_t num_attention_heads;
+    int32_t global_head_dim;               /* even, <= 256, multiple of 32 */
+    int32_t num_global_key_value_heads;    /* divides num_attention_heads */
+    int32_t intermediate_size;
+    int32_t vocab_size;
+    int32_t block_size;                    /* gamma */
+    int32_t mask_token_id;
+    int32_t markov_rank;                   /* 0 = no Markov head (plain argmax) */
+    int32_t attention_k_eq_v;              /* must be 1 */
+    int32_t markov_head_vanilla;           /* must be 1 when markov_rank > 0 */
+    int32_t hidden_activation_gelu_tanh;   /* must be 1 */
+    int32_t enable_confidence_head;
+    int32_t confidence_head_with_markov;
+    int32_t dtype;                         /* DSPARK_DTYPE_F32 or DSPARK_DTYPE_BF16 */
+    int32_t quant_bits;                    /* 0 = dense T weights; 4 = affine 4-bit (bf16 only) */
+    int32_t quant_group_size;              /* 64 when quant_bits == 4 */
+    float   rope_theta;
+    float   partial_rotary_factor;
+    float   rms_norm_eps;
+    float   final_logit_softcapping;       /* 0 = none (config null) */
+    float   confidence_threshold;          /* <= 0: no truncation, full gamma */
+} dspark_config;
+
+/*
+ * A matmul weight W [out, in] used as x @ W^T (deepspec.ts MatW), or a
+ * gather table [rows, dim] (TableW). Dense: `w` is T [out, in] and
+ * `scales`/`biases` are NULL. Affine 4-bit (MLX QuantizedLinear layout): `w`
+ * is uint32 [out, in/8] with input column 8*j + i in bits 4i..4i+3 of word
+ * j; `scales` and `biases` are bf16 [out, in/group]; weight = scale*code + bias.
+ * All device pointers, 16-byte aligned.
+ */
+typedef struct dspark_matrix {
+    const void* w;
+    const void* scales;
+    const void* biases;
+} dspark_matrix;
+
+/* One decoder layer's weights (deepspec.ts, interface Layer). Gains are T
+ * [hidden] or [head_dim]; layer_scalar is T [1]. */
+typedef struct dspark_layer_weights {
+    dspark_matrix q_proj;     /* [nH*hd, H] */
+    dspark_matrix k_proj;     /* [nKv*hd, H] */
+    dspark_matrix o_proj;     /* [H, nH*hd] */
+    dspark_matrix gate_proj;  /* [I, H] */
+    dspark_matrix up_proj;    /* [I, H] */
+    dspark_matrix down_proj;  /* [H, I] */
+    const void* q_norm;                      /* [hd] */
+    const void* k_norm;                      /* [hd] */
+    const void* input_layernorm;             /* [H] */
+    const void* post_attention_layernorm;    /* [H] */
+    const void* pre_feedforward_layernorm;   /* [H] */
+    const void* post_feedforward_layernorm;  /* [H] */
+    const void* layer_scalar;                /* [1] */
+} dspark_layer_weights;
+
+/* All weights (device pointers, caller-owned, read-only to the library). */
+typedef struct dspark_weights {
+    dspark_matrix embed_tokens;      /* table [V, H] */
+    dspark_matrix lm_head;           /* [V, H] */
+    dspark_matrix markov_w2;         /* [V, r] (unused when markov_rank == 0) */
+    dspark_matrix confidence_proj;   /* [1, H (+ r)] (unused without the confidence head) */
+    const void* markov_w1;           /* dense T table [V, r] */
+    const void* norm;                /* final norm gain, T [H] */
+    const void* confidence_bias;     /* T [1] */
+    const dspark_layer_weights* layers;  /* HOST array of num_hidden_layers entries */
+} dspark_weights;
+
+/*
+ * Per-request context K/V storage, owned by the caller (the drafter page's
+ * seam: "storage owns context validity"; deepspec.ts draftRows doc: the
+ * caller owns the cache's lifetime and the crop after the round).
+ * k, v: device T [num_hidden_layers][batch][capacity][nKv][hd]; row t of
+ * batch row b holds the K (normed, roped) / V (scale-less normed, unroped)
+ * of context row t. len: device int32 [batch], the valid rows per batch row.
+ * len_host: host int32 [batch], the library's host mirror of `len`, kept in
+ * step by dspark_append_context_kv; the caller sets both when it builds or
+ * crops a cache.
+ */
+typedef struct dspark_kv_cache {
+    void*    k;
+    void*    v;
+    int32_t* len;
+    int32_t* len_host;
+    int32_t  batch;
+    int32_t  capacity;
+} dspark_kv_cache;
+
+typedef struct dspark_model dspark_model;
+
+/* Bytes of device memory dspark_model_create needs for its stacked weight
+ * copies, RoPE table and status word; 0 for an invalid config. */
+size_t dspark_model_workspace_bytes(const dspark_config* cfg);
+
+/*
+ * Builds a model handle: validates `cfg` (readConfig's guards plus this
+ * build's shape limits), records the weight pointers, and writes into
+ * `model_ws` (device, >= dspark_model_workspace_bytes, 256-byte aligned,
+ * caller-owned, must outlive the model) the RoPE inverse-frequency table and
+ * the stacked [q_proj; k_proj], [gate_proj; up_proj] and all-layer k_proj
+ * copies the kernels read. Enqueues those copies on `stream`. The weights
+ * must stay valid and unchanged for the model's lifetime.
+ */
+int dspark_model_create(const dspark_config* cfg, const dspark_weights* weights,
+                        void* model_ws, size_t model_ws_bytes, void* stream,
+                        dspark_model** out_model);
+
+/* Frees the host-side handle (device memory stays the caller's). */
+int dspark_model_destroy(dspark_model* model);
+
+/* Scratch bytes dspark_project_context_kv / dspark_append_context_kv need
+ * for `rows` = B * L projected rows. */
+size_t dspark_project_workspace_bytes(const dspark_model* model, int64_t rows);
+
+/*
+ * Context K/V projection (deepspec.ts #projectContextKVRows; page 75
+ * projectContextKV). For every layer l, batch row b < B and context row
+ * t < L, with k_raw = hidden[b,t,:] @ k_proj_l^T viewed [nKv, hd]:
+ *   v[l,b,t] = k_raw / sqrt(mean(k_raw^2) + eps)            (v_norm, no rope)
+ *   k[l,b,t] = rope(v[l,b,t] * k_norm_l, position p)        (k_norm then rope)
+ * where p = static_pos + t when pos0 == NULL, else pos0[b] + t.
+ *   hidden  device T [B, L, H]
+ *   pos0    device int32 [B] or NULL
+ *   k_out, v_out  device T [num_hidden_layers][B][L][nKv][hd]
+ * (the dspark_kv_cache layout with capacity = L).
+ */
+int dspark_project_context_kv(const dspark_model* model, const void* hidden, int32_t B, int32_t L,
+                              int32_t static_pos, const int32_t* pos0,
+                              void* k_out, void* v_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Incremental context append (the drafter page's incremental cache:
+ * post-norm, post-rope context rows are per-row, so caching them equals
+ * recomputing them inside every round's concat). For batch row b, projects
+ * hidden[b, 0:n_new[b]] as above and writes cache rows [len_b, len_b +
+ * n_new[b]) at positions pos0[b] + len_b + t, then sets len[b] += n_new[b]
+ * on the device and in len_host.
+ *   hidden     device T [cache.batch, Lnew_max, H] (rows past n_new[b] are ignored)
+ *   n_new_host host int32 [cache.batch], each in [0, Lnew_max]
+ *   pos0       device int32 [cache.batch]: absolute position of cache row 0
+ * Fails with DSPARK_ERR_CAPACITY, before any launch, if len_host[b] +
+ * n_new[b] > capacity for some b.
+ */
+int dspark_append_context_kv(const dspark_model* model, const void* hidden, int32_t Lnew_max,
+                             const int32_t* n_new_host, const int32_t* pos0, dspark_kv_cache* cache,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Scratch bytes dspark_draft_rows / dspark_attend need for A rows whose
+ * context is at most max_ctx_len rows. */
+size_t dspark_draft_workspace_bytes(const dspark_model* model, int32_t A, int32_t max_ctx_len);
+
+/*
+ * One draft round for A rows (deepspec.ts draftRows). Row b drafts the block
+ * [anchors[b], mask x (gamma-1)] at positions block_pos[b] + t against its
+ * cached context rows [0, cache.len[b]) (cache batch row b; A <= cache.batch):
+ * backbone -> final norm -> U = softcap(lm_head(h)) -> for k = 0..gamma-1:
+ * tokens[b,k] = argmax_v(U[b,k,v] + markov_w2(markov_w1[prev])[v]) with prev =
+ * anchor then the previous token (lowest index on ties) -> conf[b,k] =
+ * sigmoid(proj([h_k ; markov_w1[prev_k]]) + bias) -> lengths[b] = first k with
+ * conf < threshold (threshold > 0), else gamma.
+ *   anchors    device int32 [A]       block_pos device int32 [A]
+ *   max_ctx_len  host upper bound of cache.len[b] over the A rows (<= capacity)
+ *   tokens     device int32 [A, gamma] (all gamma walked tokens; lengths says how many to keep)
+ *   conf       device float [A, gamma] or NULL (needs the confidence head)
+ *   lengths    device int32 [A]
+ *   base_logits device float [A, gamma, V] or NULL (the page's collectLogits)
+ */
+int dspark_draft_rows(const dspark_model* model, const dspark_kv_cache* cache,
+                      const int32_t* anchors, const int32_t* block_pos, int32_t A, int32_t max_ctx_len,
+                      int32_t* tokens, float* conf, int32_t* lengths, float* base_logits,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The attention seam alone (page 75, DeepspecContextAttention.attend and
+ * plainDeepspecContext): for batch row b < A and query head h, attends
+ * q[b,:,h,:] over keys [cache.k[layer,b,0:len_b,g] ++ k_blk[b,:,g]] and
+ * values [cache.v[layer,b,0:len_b,g] ++ v_blk[b,:,g]], g = h / (nH/nKv),
+ * non-causal, scale 1.0, softmax in fp32.
+ *   q   device T [A, gamma, nH, hd]     k_blk, v_blk device T [A, gamma, nKv, hd]
+ *   out device T [A, gamma, nH, hd]
+ */
+int dspark_attend(const dspark_model* model, int32_t layer, const dspark_kv_cache* cache,
+                  const void* q, const void* k_blk, const void* v_blk, void* out,
+                  int32_t A, int32_t max_ctx_len, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the device status bits in *status and
+ * clears them. */
+int dspark_read_device_status(const dspark_model* model, void* stream, int32_t* status);
+
+/* Last error message of the calling host thread ("" if none). */
+const char* dspark_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_H */

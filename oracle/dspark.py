@@ -31,7 +31,7 @@ import numpy as np
 
 __all__ = [
     "OracleWeights", "dequantize_affine4", "rope_wavelengths", "rms_norm", "apply_rope",
-    "gelu_tanh", "project_context_kv", "attention_weights", "attend_concat", "attend_split",
+    "gelu_tanh", "store_rounded", "project_context_kv", "attention_weights", "attend_concat", "attend_split",
     "embed_block", "decoder_layer", "backbone", "compute_logits", "markov_bias", "markov_walk", "teacher_forced_walk",
     "confidence", "prefix_length", "draft_rows", "block_ids",
 ]
@@ -170,13 +170,25 @@ def _sigmoid(z: np.ndarray) -> np.ndarray:
 # Stage 1: context K/V (``#projectContextKVRows``).
 # ---------------------------------------------------------------------------
 
+def store_rounded(x: np.ndarray, store_dtype: Optional[str]) -> np.ndarray:
+    """Round to the cache's storage dtype: the drafter keeps ContextKV rows in the
+    model dtype (``#rms`` casts back to it), so a bf16 model's cached K/V are
+    bf16 values. None / "fp32" / "fp64" keep the fp64 values."""
+    if store_dtype != "bf16":
+        return x
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
 def project_context_kv(W: OracleWeights, hidden, pos0: Sequence[int], lengths: Optional[Sequence[int]] = None,
-                       chunk: int = 8192) -> List[List[tuple]]:
+                       chunk: int = 8192, store_dtype: Optional[str] = None) -> List[List[tuple]]:
     """Per-layer context K/V of every row, ready to cache across rounds.
 
     For each layer: k_raw = hidden @ Wk^T viewed [L, nKv, hd];
     v = rms(k_raw, none) (attention_k_eq_v: v is k before the norms diverge,
     and gets no rope); k = rope(rms(k_raw, k_norm), pos0 + t).
+    ``store_dtype="bf16"`` returns the values the cache holds for a bf16
+    model (fp64 values rounded to bf16); the default keeps fp64.
     Returns ``out[b][layer] = (k [L_b, nKv, hd], v [L_b, nKv, hd])``.
     """
     m = W.m
@@ -198,8 +210,8 @@ def project_context_kv(W: OracleWeights, hidden, pos0: Sequence[int], lengths: O
                 k = rms_norm(k_raw, kn, m.rms_norm_eps)
                 pos = int(pos0[b]) + np.arange(lo, hi)
                 k = apply_rope(k.transpose(1, 0, 2), pos[None, :], wl).transpose(1, 0, 2)
-                ks.append(k)
-                vs.append(v)
+                ks.append(store_rounded(k, store_dtype))
+                vs.append(store_rounded(v, store_dtype))
             per_layer.append((np.concatenate(ks, 0) if ks else np.zeros((0, nKv, hd)),
                               np.concatenate(vs, 0) if vs else np.zeros((0, nKv, hd))))
         out.append(per_layer)

@@ -188,18 +188,25 @@ def quantize_affine4(w: torch.Tensor, group: int = 64):
     return words.contiguous(), scale.contiguous(), bias.contiguous()
 
 
-def make_weights(m: ModelShape, seed: int, literal: bool = False,
+def make_weights(m: ModelShape, seed: int, literal: bool = False, unit_attention_logits: bool = True,
                  markov_scale: float = 1.0) -> Dict[str, torch.Tensor]:
     """Seeded synthetic drafter weights on the CPU.
 
     Matmul, embedding, Markov and confidence weights are N(0, 0.02); RMSNorm
-    gains are 1 + N(0, 0.02) and layer_scalar is 1.0 (``literal=True`` draws
-    gains and layer_scalar as N(0, 0.02) too). ``markov_scale`` multiplies
-    both Markov tables (a test knob that makes the transition bias matter).
-    For ``quant_bits == 4`` each quantized matrix ``X`` is stored as
-    ``X.q`` (int32 words), ``X.scales``, ``X.biases`` instead of ``X``.
+    gains are 1 + N(0, 0.02) and layer_scalar is 1.0. The q_norm and k_norm
+    gains are further scaled by head_dim^(-1/4) (``unit_attention_logits``):
+    attention runs at scale 1.0 on QK-normed vectors, so gains of 1 give
+    logits of standard deviation sqrt(head_dim) and a near one-hot softmax
+    whose output, from the second layer on, hinges on the last bits of the
+    stored keys; the scaled gains give unit-variance logits, the temperature a
+    trained model has. ``literal=True`` instead draws every gain and the
+    layer scalar as N(0, 0.02). ``markov_scale`` multiplies both Markov
+    tables (a test knob that makes the transition bias matter). For
+    ``quant_bits == 4`` each quantized matrix ``X`` is stored as ``X.q``
+    (int32 words), ``X.scales``, ``X.biases`` instead of ``X``.
     """
     out: Dict[str, torch.Tensor] = {}
+    qk_scale = m.global_head_dim ** -0.25 if unit_attention_logits else 1.0
     for idx, (name, shape, kind) in enumerate(weight_names(m)):
         if kind == "mat":
             t = _draw(seed, idx, shape, std=0.02)
@@ -207,6 +214,8 @@ def make_weights(m: ModelShape, seed: int, literal: bool = False,
                 t.mul_(markov_scale)
         elif kind == "gain":
             t = _draw(seed, idx, shape, std=0.02) if literal else _draw(seed, idx, shape, std=0.02, mean=1.0)
+            if not literal and name.endswith(("q_norm", "k_norm")):
+                t.mul_(qk_scale)
         elif kind == "scalar":
             t = _draw(seed, idx, shape, std=0.02) if literal else torch.ones(shape)
         else:  # bias
@@ -290,7 +299,7 @@ def small_model(dtype: str = "bf16", quant_bits: int = 0, **kw) -> ModelShape:
     """A small Gemma-like drafter used by the fast parity tests (several tiles, ragged tails)."""
     base = dict(hidden_size=512, num_hidden_layers=2, num_attention_heads=8, global_head_dim=128,
                 num_global_key_value_heads=2, intermediate_size=1024, vocab_size=4096 + 64,
-                block_size=8, mask_token_id=4096 + 63, markov_rank=16, rope_theta=1e6,
+                block_size=8, mask_token_id=4096 + 63, markov_rank=64 if quant_bits else 16, rope_theta=1e6,
                 partial_rotary_factor=0.5, final_logit_softcapping=30.0, dtype=dtype,
                 quant_bits=quant_bits)
     base.update(kw)

@@ -1,0 +1,252 @@
+"""GPU parity: libdspark's kernels (through the C ABI) against the fp64 oracle.
+
+Small models here span several tiles and ragged tails in every dimension;
+the full-size workloads are in test_gpu_full_size.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dspark as O
+from synthetic import WORKLOADS, make_round_inputs, make_weights, small_model
+from parity_util import as_stored, assert_close, build, check_tokens, CONF_TOL, ensure_built
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    ensure_built()
+
+
+def _project_into_cache(model, hidden_cpu, lens, pos0, capacity=None):
+    """Cache of `capacity` rows per batch row with rows [0, lens[b]) appended at pos0[b]."""
+    import block_draft_model_dspark_b200 as dsp
+    B, L = hidden_cpu.shape[0], hidden_cpu.shape[1]
+    cache = dsp.KvCache(model, B, capacity or L)
+    cache.set_lengths([0] * B)
+    model.dspark_append_context_kv(cache, hidden_cpu.cuda(), [int(x) for x in lens],
+                                   torch.tensor(pos0, dtype=torch.int32, device="cuda"))
+    return cache
+
+
+def _check_cache_rows(cache, kv_oracle, lens, dtype):
+    k = cache.k.float().cpu().numpy()
+    v = cache.v.float().cpu().numpy()
+    for b, L in enumerate(lens):
+        for l in range(k.shape[0]):
+            assert_close(k[l, b, :L], kv_oracle[b][l][0], dtype, f"K layer {l} row {b}")
+            assert_close(v[l, b, :L], kv_oracle[b][l][1], dtype, f"V layer {l} row {b}")
+
+
+def _round_and_compare(shape, W, model, cache, kv_oracle, anchors, block_pos, lens, what):
+    A = len(anchors)
+    dev_anchors = torch.tensor(anchors, dtype=torch.int32, device="cuda")
+    dev_bpos = torch.tensor(block_pos, dtype=torch.int32, device="cuda")
+    out = model.draft(cache, dev_anchors, dev_bpos, max(lens) if len(lens) else 0)
+    torch.cuda.synchronize()
+    assert model.dspark_read_device_status() == 0
+    ref = O.draft_rows(W, as_stored(kv_oracle, shape.dtype), anchors, block_pos)
+    assert_close(out["base_logits"].cpu().numpy(), ref["base_logits"], shape.dtype, f"{what}: base logits")
+    gtok = out["tokens"].cpu().numpy().astype(np.int64)
+    checked, total = check_tokens(W, ref["base_logits"], anchors, gtok, f"{what}: tokens")
+    assert checked >= total // 2, f"{what}: too few decisive steps ({checked}/{total})"
+    if shape.enable_confidence_head:
+        conf_ref = O.confidence(W, ref["hidden"], anchors, gtok)
+        gconf = out["conf"].cpu().numpy()
+        assert np.max(np.abs(gconf - conf_ref)) <= CONF_TOL, f"{what}: confidence"
+        lens_gpu = out["lengths"].cpu().numpy()
+        for b in range(A):
+            assert lens_gpu[b] == O.prefix_length(gconf[b], shape.confidence_threshold, shape.block_size)
+    else:
+        assert (out["lengths"].cpu().numpy() == shape.block_size).all()
+    return out, ref
+
+
+# ----------------------------------------------------------------------------- the tiny fp32 workload
+
+def test_tiny_fp32_workload_round():
+    wl = WORKLOADS["tiny_fp32"]
+    m = wl.model
+    cpu, W, model = build(m, wl.seed)
+    inp = make_round_inputs(wl)
+    lens = inp["ctx_len"].tolist()
+    cache = _project_into_cache(model, inp["hidden"], lens, inp["pos0"].tolist())
+    kv = O.project_context_kv(W, inp["hidden"], inp["pos0"].tolist(), lengths=lens)
+    _check_cache_rows(cache, kv, lens, "fp32")
+    _round_and_compare(m, W, model, cache, kv, inp["anchors"].tolist(), inp["block_pos"].tolist(), lens, "tiny_fp32")
+
+
+def test_project_context_kv_static_and_dynamic_positions():
+    m = small_model(dtype="bf16")
+    cpu, W, model = build(m, 3)
+    import block_draft_model_dspark_b200 as dsp
+    hid = torch.randn(3, 70, m.hidden_size, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    for pos0 in (None, [5, 0, 9000]):
+        cache = dsp.KvCache(model, 3, 70)
+        model.dspark_project_context_kv(hid.cuda(), cache.k, cache.v,
+                                        pos0=None if pos0 is None else torch.tensor(pos0, dtype=torch.int32, device="cuda"),
+                                        static_pos=17)
+        torch.cuda.synchronize()
+        kv = O.project_context_kv(W, hid, pos0 if pos0 is not None else [17, 17, 17])
+        _check_cache_rows(cache, kv, [70, 70, 70], "bf16")
+
+
+# ----------------------------------------------------------------------------- attention seam
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_attend_matches_concat_sdpa(dtype):
+    m = small_model(dtype=dtype, block_size=8)
+    cpu, W, model = build(m, 5)
+    import block_draft_model_dspark_b200 as dsp
+    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    A, G, nH, nKv, hd = 4, m.block_size, m.num_attention_heads, m.num_global_key_value_heads, m.global_head_dim
+    lens = [0, 1, 333, 1000]
+    cap = 1003
+    g = torch.Generator().manual_seed(7)
+    cache = dsp.KvCache(model, A, cap)
+    cache.k.copy_((torch.randn(cache.k.shape, generator=g) * 0.6).to(tdt))
+    cache.v.copy_(torch.randn(cache.v.shape, generator=g).to(tdt))
+    cache.set_lengths(lens)
+    q = (torch.randn(A, G, nH, hd, generator=g) * 0.6).to(tdt)
+    kb = (torch.randn(A, G, nKv, hd, generator=g) * 0.6).to(tdt)
+    vb = torch.randn(A, G, nKv, hd, generator=g).to(tdt)
+    out = torch.empty(A, G, nH, hd, dtype=tdt, device="cuda")
+    for layer in range(m.num_hidden_layers):
+        model.dspark_attend(layer, cache, q.cuda(), kb.cuda(), vb.cuda(), out, max(lens))
+        torch.cuda.synchronize()
+        kc, vc = cache.k[layer].float().cpu().numpy(), cache.v[layer].float().cpu().numpy()
+        for b in range(A):
+            ref = O.attend_concat(q[b].double().numpy(), kc[b, :lens[b]], vc[b, :lens[b]], kb[b].double().numpy(),
+                                  vb[b].double().numpy())
+            assert_close(out[b].float().cpu().numpy(), ref, dtype, f"attend layer {layer} row {b}")
+
+
+# ----------------------------------------------------------------------------- whole rounds, small models
+
+@pytest.mark.parametrize("quant", [0, 4])
+def test_small_bf16_ragged_round(quant):
+    m = small_model(dtype="bf16", quant_bits=quant)
+    cpu, W, model = build(m, 11 + quant)
+    A = 3
+    lens = [37, 0, 200]
+    pos0 = [0, 50, 4000]
+    hid = torch.randn(A, 200, m.hidden_size, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    cache = _project_into_cache(model, hid, lens, pos0)
+    kv = O.project_context_kv(W, hid, pos0, lengths=lens)
+    _check_cache_rows(cache, kv, lens, "bf16")
+    anchors = [5, m.vocab_size - 2, 1234]
+    block_pos = [p + L for p, L in zip(pos0, lens)]
+    _round_and_compare(m, W, model, cache, kv, anchors, block_pos, lens, f"small bf16 q{quant}")
+
+
+def test_strong_markov_walk_and_threshold():
+    """Markov tables scaled so the transition bias reorders tokens; threshold 0.5 truncates."""
+    m = small_model(dtype="bf16", confidence_threshold=0.5)
+    cpu, W, model = build(m, 21, markov_scale=60.0)
+    A, lens, pos0 = 2, [64, 129], [0, 7]
+    hid = torch.randn(A, 129, m.hidden_size, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    cache = _project_into_cache(model, hid, lens, pos0)
+    kv = O.project_context_kv(W, hid, pos0, lengths=lens)
+    out, ref = _round_and_compare(m, W, model, cache, kv, [3, 4], [64, 136], lens, "strong markov")
+    # the bias matters: the walk differs from per-step argmax of U somewhere
+    assert (ref["tokens"] != np.argmax(ref["base_logits"], -1)).any()
+
+
+def test_rank0_no_confidence_head():
+    m = small_model(dtype="bf16", markov_rank=0, enable_confidence_head=False, confidence_head_with_markov=False)
+    cpu, W, model = build(m, 31)
+    lens, pos0 = [90], [3]
+    hid = torch.randn(1, 90, m.hidden_size, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    cache = _project_into_cache(model, hid, lens, pos0)
+    kv = O.project_context_kv(W, hid, pos0, lengths=lens)
+    _round_and_compare(m, W, model, cache, kv, [9], [93], lens, "rank 0")
+
+
+# ----------------------------------------------------------------------------- the incremental cache
+
+def test_append_equals_recompute_with_sentinels():
+    import block_draft_model_dspark_b200 as dsp
+    m = small_model(dtype="bf16")
+    cpu, W, model = build(m, 41)
+    B, cap = 3, 96
+    pos0 = torch.tensor([0, 100, 7], dtype=torch.int32, device="cuda")
+    cache = dsp.KvCache(model, B, cap)
+    sentinel = torch.tensor(-12345.0, dtype=torch.bfloat16)
+    cache.k.fill_(sentinel)
+    cache.v.fill_(sentinel)
+    cache.set_lengths([0, 0, 0])
+    g = torch.Generator().manual_seed(9)
+    rows = [[] for _ in range(B)]
+    sched = [[5, 1, 16], [16, 0, 3], [1, 16, 16], [7, 9, 0]]
+    for n_new in sched:
+        hid = torch.randn(B, 16, m.hidden_size, generator=g).to(torch.bfloat16)
+        model.dspark_append_context_kv(cache, hid.cuda(), n_new, pos0)
+        for b in range(B):
+            rows[b].append(hid[b, :n_new[b]])
+    torch.cuda.synchronize()
+    lens = [sum(s[b] for s in sched) for b in range(B)]
+    assert list(cache.len_host) == lens and cache.len.cpu().tolist() == lens
+    full = [torch.cat(r) for r in rows]
+    Lmax = max(lens)
+    hid_full = torch.zeros(B, Lmax, m.hidden_size, dtype=torch.bfloat16)
+    for b in range(B):
+        hid_full[b, :lens[b]] = full[b]
+    # recompute all rows at once on the GPU
+    ref = dsp.KvCache(model, B, Lmax)
+    model.dspark_project_context_kv(hid_full.cuda(), ref.k, ref.v, pos0=pos0)
+    torch.cuda.synchronize()
+    kv = O.project_context_kv(W, hid_full, pos0.cpu().tolist(), lengths=lens)
+    _check_cache_rows(cache, kv, lens, "bf16")
+    same = total = 0
+    for b in range(B):
+        a = cache.k[:, b, :lens[b]]
+        r = ref.k[:, b, :lens[b]]
+        same += int((a.view(torch.int16) == r.view(torch.int16)).sum())
+        total += a.numel()
+        # rows past len were never written
+        assert (cache.k[:, b, lens[b]:].view(torch.int16) == sentinel.view(torch.int16).item()).all()
+        assert (cache.v[:, b, lens[b]:].view(torch.int16) == sentinel.view(torch.int16).item()).all()
+    assert same / total > 0.99, f"append vs recompute: only {same}/{total} bf16 values bit-identical"
+
+
+def test_capacity_error_leaves_cache_untouched():
+    import block_draft_model_dspark_b200 as dsp
+    m = small_model(dtype="bf16")
+    cpu, W, model = build(m, 43)
+    cache = dsp.KvCache(model, 2, 20)
+    cache.k.zero_(); cache.v.zero_()
+    cache.set_lengths([10, 18])
+    k0 = cache.k.clone()
+    hid = torch.randn(2, 4, m.hidden_size).to(torch.bfloat16).cuda()
+    with pytest.raises(dsp.DsparkError) as ei:
+        model.dspark_append_context_kv(cache, hid, [4, 3], torch.zeros(2, dtype=torch.int32, device="cuda"))
+    assert ei.value.code == dsp.DSPARK_ERR_CAPACITY
+    torch.cuda.synchronize()
+    assert torch.equal(cache.k, k0) and list(cache.len_host) == [10, 18] and cache.len.cpu().tolist() == [10, 18]
+
+
+def test_workspace_too_small_and_bad_anchor_status():
+    import block_draft_model_dspark_b200 as dsp
+    m = small_model(dtype="bf16")
+    cpu, W, model = build(m, 47)
+    cache = dsp.KvCache(model, 1, 8)
+    cache.k.zero_(); cache.v.zero_()
+    cache.set_lengths([8])
+    anchors = torch.tensor([m.vocab_size + 5], dtype=torch.int32, device="cuda")
+    bpos = torch.tensor([8], dtype=torch.int32, device="cuda")
+    tok = torch.empty(1, m.block_size, dtype=torch.int32, device="cuda")
+    lens = torch.empty(1, dtype=torch.int32, device="cuda")
+    small = model.workspace(1024)
+    with pytest.raises(dsp.DsparkError) as ei:
+        model.dspark_draft_rows(cache, anchors, bpos, 8, tok, lens, ws=small)
+    assert ei.value.code == dsp.DSPARK_ERR_WORKSPACE
+    model.dspark_draft_rows(cache, anchors, bpos, 8, tok, lens)
+    assert model.dspark_read_device_status() & dsp.DSPARK_DEV_BAD_TOKEN
+    assert model.dspark_read_device_status() == 0     # read clears it
+    t = tok.cpu()
+    assert ((t >= 0) & (t < m.vocab_size)).all()

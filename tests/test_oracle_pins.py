@@ -478,3 +478,12 @@ def test_full_round_shapes_and_consistency():
     for b in range(A):
         assert out["lengths"][b] == O.prefix_length(out["conf"][b], 0.5, G)
     assert len(out["attention"]) == 2
+
+
+def test_store_rounded_is_round_to_nearest_even_bf16():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, -3.14159, 1e-3, 0.0])
+    got = O.store_rounded(x, "bf16")
+    # bf16 keeps 8 significant bits: 1 + 2^-8 is a tie -> even (1.0); 1 + 3*2^-9 rounds up to 1 + 2^-7
+    assert got[0] == 1.0 and got[1] == 1.0 and got[2] == 1.0 + 2 ** -7
+    assert abs(got[3] + 3.140625) < 1e-12
+    np.testing.assert_array_equal(O.store_rounded(x, None), x)
