@@ -84,7 +84,30 @@ _PROTOTYPES = {
                               c_size, c_vp]),
     "dspark_read_device_status": (c_i32, [c_vp, c_vp, c_i32p]),
     "dspark_last_error": (ctypes.c_char_p, []),
+    "dspark_kernel_launches": (ctypes.c_uint64, []),
+    "dspark_timer_enable": (c_i32, [c_i32]),
+    "dspark_timer_read": (c_i32, [c_i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
+                                  ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
 }
+
+DSPARK_TIMER_KINDS = {"gemm": 0, "lm_head": 1, "attention": 2, "walk": 3, "kv_project": 4, "rows": 5}
+
+
+def dspark_kernel_launches() -> int:
+    """Kernels libdspark has launched in this process."""
+    return int(get_lib().dspark_kernel_launches())
+
+
+def dspark_timer_enable(enable: bool) -> None:
+    _check(get_lib().dspark_timer_enable(1 if enable else 0))
+
+
+def dspark_timer_read(kind: str):
+    """(device ms, launches, algorithmic bytes, flops) summed over the timed launches of a kernel class."""
+    ms, n, by, fl = ctypes.c_double(), ctypes.c_int64(), ctypes.c_double(), ctypes.c_double()
+    _check(get_lib().dspark_timer_read(DSPARK_TIMER_KINDS[kind], ctypes.byref(ms), ctypes.byref(n),
+                                       ctypes.byref(by), ctypes.byref(fl)))
+    return ms.value, n.value, by.value, fl.value
 
 
 class DsparkError(RuntimeError):

@@ -437,6 +437,15 @@ static AttnArgs attn_args(const dspark_model* m, const DraftPlan& p, void* ws, c
     a.part_o = at<float>(ws, p.part_o); a.part_ml = at<float>(ws, p.part_ml);
     a.A = A; a.n_splits = p.attn_splits; a.chunk = p.attn_chunk;
     a.status = m->ws.status;
+    // algorithmic work: every valid context row's K and V once, the block K/V, q and out
+    double keys = (double)A * d.gamma;
+    if (c->len_host)
+        for (int b = 0; b < A; ++b) keys += c->len_host[b];
+    else
+        keys += (double)A * c->capacity;
+    const double qo = 2.0 * A * d.gamma * d.nH * d.hd * (io_dtype == DSPARK_DTYPE_F32 ? 4.0 : (double)es);
+    a.kv_bytes = keys * d.nKv * d.hd * 2.0 * es + qo;
+    a.flops = 4.0 * (double)d.nH * d.gamma * d.hd * keys;
     return a;
 }
 
@@ -498,8 +507,11 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
         wa.part_val = at<float>(ws, p.walk_val); wa.part_idx = at<int32_t>(ws, p.walk_idx);
         wa.ticket = at<uint32_t>(ws, p.ticket); wa.A = A; wa.nblk = p.walk_blocks; wa.status = m->ws.status;
         e = launch_walk_init(anchors, wa.prev, wa.ticket, A, d.V, m->ws.status, s);
+        const double w2b = d.r > 0 ? (d.quant ? (double)d.V * d.r * 0.5 + (double)d.V * (d.r / d.group) * 4.0
+                                              : (double)d.V * d.r * esize(d.dtype)) : 0.0;
         for (int k = 0; k < d.gamma && e == cudaSuccess; ++k) {
             wa.step = k;
+            KernelTimer t(DSPARK_TIMER_WALK, s, w2b + 4.0 * A * d.V, 2.0 * A * (double)d.V * d.r);
             e = launch_walk_step(m, wa, s);
         }
     }

@@ -163,8 +163,10 @@ cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a, cuda
     dim3 grid(a.A * d.nH, a.n_splits + 1);
     attn_partial_kernel<<<grid, kThreads, smem, s>>>(a, d.gamma, d.nH, d.nKv, d.hd, d.dtype);
     cudaError_t e = cudaGetLastError();
+    count_launches(1);
     if (e != cudaSuccess) return e;
     attn_merge_kernel<<<a.A * d.nH * d.gamma, d.hd, 0, s>>>(a, d.gamma, d.nH, d.hd);
+    count_launches(1);
     return cudaGetLastError();
 }
 

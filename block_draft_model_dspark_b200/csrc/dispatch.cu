@@ -26,14 +26,22 @@ int gemm_splits(const dspark_model* m, int M, int N, int K) {
     }
 }
 
+double weight_bytes(const dspark_model* m, int64_t N, int64_t K) {
+    if (m->d.quant) return (double)N * K * 0.5 + (double)N * (K / m->d.group) * 4.0;
+    return (double)N * K * (m->d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0);
+}
+
 cudaError_t run_gemm(const dspark_model* m, const void* X, int64_t ldx, const MatRef& W, int M, int N, int K,
                      int splits, float* out, cudaStream_t s) {
+    KernelTimer t(DSPARK_TIMER_GEMM, s, weight_bytes(m, N, K) + 4.0 * M * K + 4.0 * M * N, 2.0 * M * N * K);
     return launch_simt_gemm(X, ldx, DSPARK_DTYPE_F32, m->d.dtype, W, m->d.group, M, N, K, splits, out, N,
                             (int64_t)M * N, false, 0.f, s);
 }
 
 cudaError_t run_lm_head(const dspark_model* m, const void* x, int M, float* U, cudaStream_t s) {
     const Dims& d = m->d;
+    KernelTimer t(DSPARK_TIMER_LM_HEAD, s, weight_bytes(m, d.V, d.H) + 4.0 * M * d.H + 4.0 * M * d.V,
+                  2.0 * M * (double)d.V * d.H);
     return launch_simt_gemm(x, d.H, DSPARK_DTYPE_F32, d.dtype, m->lm_head, d.group, M, d.V, d.H, 1, U, d.V, 0, true,
                             d.cap, s);
 }
@@ -44,6 +52,9 @@ cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, c
                               float* raw, int splits, cudaStream_t s) {
     const Dims& d = m->d;
     const int N = d.Lyr * d.nKv * d.hd;
+    const double es = d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0;
+    KernelTimer t(DSPARK_TIMER_KV_PROJECT, s, weight_bytes(m, N, d.H) + es * nrows * d.H + 2.0 * es * nrows * N,
+                  2.0 * nrows * (double)N * d.H);
     cudaError_t e = launch_simt_gemm(X, d.H, d.dtype, d.dtype, m->wk_all, d.group, nrows, N, d.H, splits, raw, N,
                                      (int64_t)nrows * N, false, 0.f, s);
     if (e != cudaSuccess) return e;
@@ -51,6 +62,7 @@ cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, c
 }
 
 cudaError_t run_attention(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
+    KernelTimer t(DSPARK_TIMER_ATTENTION, s, a.kv_bytes, a.flops);
     return launch_attention_simt(m, a, s);
 }
 

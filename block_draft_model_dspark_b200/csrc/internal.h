@@ -145,6 +145,7 @@ struct AttnArgs {
     float* part_o; float* part_ml;                   // workspace
     int A, n_splits, chunk;                          // context splits of `chunk` keys (+1 block split)
     int32_t* status;
+    double kv_bytes, flops;                          // algorithmic work (for the timers)
 };
 
 // Markov walk step k: tokens[:,k] from U[:,k,:] + w2 . w1[prev]; prev updated.
@@ -165,5 +166,21 @@ cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const in
                               int A, float* conf, int32_t* lengths, cudaStream_t s);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Launch accounting (timing.cu): count_launches after each launch; a
+// KernelTimer in scope around a launch brackets it with events when timing is on.
+void count_launches(int n);
+class KernelTimer {
+  public:
+    KernelTimer(int kind, cudaStream_t s, double bytes, double flops);
+    ~KernelTimer();
+    KernelTimer(const KernelTimer&) = delete;
+    KernelTimer& operator=(const KernelTimer&) = delete;
+  private:
+    int kind_;
+    cudaStream_t s_;
+    double bytes_, flops_;
+    cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
 
 }  // namespace dspark

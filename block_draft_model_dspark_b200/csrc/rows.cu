@@ -241,11 +241,13 @@ cudaError_t launch_kv_epilogue(const dspark_model* m, const float* raw, int spli
     dim3 grid(rp.nrows, d.Lyr * d.nKv);
     kv_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(raw, splits, split_stride, d.Lyr * d.nKv * d.hd, rp, dst,
                                                  m->ws.inv_freq, kn, d.nKv, d.hd, d.eps, d.dtype, m->ws.status);
+    count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStream_t s) {
     commit_len_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, n_new, B);
+    count_launches(1);
     return cudaGetLastError();
 }
 
@@ -255,6 +257,7 @@ cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, f
     embed_kernel<<<A * d.gamma, row_threads(d.H), 0, s>>>(m->embed, d.dtype, d.group, anchors, d.gamma, d.mask_id,
                                                          d.V, d.H, sqrtf((float)d.H), m->layers[0].in_norm, d.eps,
                                                          h, x, status);
+    count_launches(1);
     return cudaGetLastError();
 }
 
@@ -265,6 +268,7 @@ cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const float* pa
     qk_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(part, splits, split_stride, (d.nH + d.nKv) * d.hd, d.gamma, d.nH,
                                                  d.nKv, d.hd, block_pos, m->ws.inv_freq, m->layers[layer].q_norm,
                                                  m->layers[layer].k_norm, d.eps, d.dtype, q, kb, vb);
+    count_launches(1);
     return cudaGetLastError();
 }
 
@@ -274,6 +278,7 @@ cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const float* par
     const LayerRef& L = m->layers[layer];
     residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, splits, split_stride, d.H, L.post_attn_norm,
                                                             L.pre_ff_norm, nullptr, 0, d.eps, d.dtype, h, x);
+    count_launches(1);
     return cudaGetLastError();
 }
 
@@ -284,6 +289,7 @@ cudaError_t launch_gu_epilogue(const dspark_model* m, const float* part, int spl
     int blocks = (int)((total + 255) / 256);
     if (blocks > 8 * m->num_sms) blocks = 8 * m->num_sms;
     gu_epilogue_kernel<<<blocks, 256, 0, s>>>(part, splits, split_stride, M, d.I, act);
+    count_launches(1);
     return cudaGetLastError();
 }
 
@@ -295,6 +301,7 @@ cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const float* 
     const void* next = last ? m->final_norm : m->layers[layer + 1].in_norm;
     residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, splits, split_stride, d.H, L.post_ff_norm, next,
                                                             L.layer_scalar, 1, d.eps, d.dtype, h, x);
+    count_launches(1);
     return cudaGetLastError();
 }
 
@@ -304,6 +311,7 @@ cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const in
     confidence_kernel<<<A, 256, 0, s>>>(hf32, m->conf_proj, d.dtype, d.group, m->w1, m->conf_bias, anchors, tokens,
                                         d.gamma, d.H, d.r, d.conf_markov ? 1 : 0, d.V, d.conf_thr,
                                         d.conf_head ? 1 : 0, d.conf_head ? conf : nullptr, lengths);
+    count_launches(1);
     return cudaGetLastError();
 }
 

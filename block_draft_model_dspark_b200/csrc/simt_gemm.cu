@@ -133,6 +133,7 @@ cudaError_t launch_simt_gemm(const void* X, int64_t ldx, int x_dtype, int w_dtyp
         if (xf) DSPARK_SIMT_LAUNCH(float, bf16, false); else DSPARK_SIMT_LAUNCH(bf16, bf16, false);
     }
 #undef DSPARK_SIMT_LAUNCH
+    count_launches(1);
     return cudaGetLastError();
 }
 

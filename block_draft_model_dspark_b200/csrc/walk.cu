@@ -108,12 +108,14 @@ walk_step_kernel(WalkArgs a, MatRef W2, const void* __restrict__ w1, int dtype, 
 cudaError_t launch_walk_init(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V, int32_t* status,
                              cudaStream_t s) {
     walk_init_kernel<<<(A + 127) / 128, 128, 0, s>>>(anchors, prev, ticket, A, V, status);
+    count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s) {
     const Dims& d = m->d;
     walk_step_kernel<<<a.nblk, kThreads, 0, s>>>(a, m->w2, m->w1, d.dtype, d.group, d.gamma, d.V, d.r);
+    count_launches(1);
     return cudaGetLastError();
 }
 

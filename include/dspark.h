@@ -253,6 +253,27 @@ int dspark_read_device_status(const dspark_model* model, void* stream, int32_t* 
 /* Last error message of the calling host thread ("" if none). */
 const char* dspark_last_error(void);
 
+/*
+ * Instrumentation (no counterpart on the pages; used by the benchmark).
+ * dspark_kernel_launches: number of CUDA kernels this library has launched in
+ * this process. dspark_timer_enable(1): from now on each launch of a kernel
+ * class below is bracketed by CUDA events on its stream (a few microseconds of
+ * host work per launch) and tagged with its algorithmic bytes and flops.
+ * dspark_timer_read: waits for the recorded events of `kind`, returns their
+ * summed device milliseconds, launch count, bytes and flops (either of the
+ * last two may be NULL), and forgets them.
+ */
+#define DSPARK_TIMER_GEMM        0  /* the layers' weight GEMMs: [q;k], o, [gate;up], down */
+#define DSPARK_TIMER_LM_HEAD     1  /* lm-head GEMM with softcap */
+#define DSPARK_TIMER_ATTENTION   2  /* KV-injection attention (partials + merge) */
+#define DSPARK_TIMER_WALK        3  /* Markov walk steps */
+#define DSPARK_TIMER_KV_PROJECT  4  /* context K/V projection GEMM + epilogue */
+#define DSPARK_TIMER_ROWS        5  /* embedding, norms/RoPE/residual epilogues, confidence */
+#define DSPARK_TIMER_KINDS       6
+uint64_t dspark_kernel_launches(void);
+int dspark_timer_enable(int enable);
+int dspark_timer_read(int kind, double* total_ms, int64_t* launches, double* bytes, double* flops);
+
 #ifdef __cplusplus
 }
 #endif
