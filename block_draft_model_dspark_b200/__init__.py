@@ -82,6 +82,8 @@ _PROTOTYPES = {
                                   c_vp, c_vp, c_size, c_vp]),
     "dspark_attend": (c_i32, [c_vp, c_i32, ctypes.POINTER(dspark_kv_cache), c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_vp,
                               c_size, c_vp]),
+    "dspark_attend_no_alloc": (c_i32, [c_vp, c_i32, ctypes.POINTER(dspark_kv_cache), c_vp, c_vp, c_vp, c_vp, c_i32,
+                                       c_i32, c_vp]),
     "dspark_read_device_status": (c_i32, [c_vp, c_vp, c_i32p]),
     "dspark_last_error": (ctypes.c_char_p, []),
     "dspark_kernel_launches": (ctypes.c_uint64, []),
@@ -326,6 +328,14 @@ class DsparkModel:
         _check(get_lib().dspark_attend(self.handle, layer, ctypes.byref(st), q.data_ptr(), k_blk.data_ptr(),
                                  v_blk.data_ptr(), out.data_ptr(), A, max_ctx_len, ws.data_ptr(), ws.numel(),
                                  _stream_ptr(stream)))
+
+    def dspark_attend_no_alloc(self, layer: int, cache: KvCache, q, k_blk, v_blk, out, max_ctx_len: int,
+                               stream=None):
+        """The attention seam with the library's static scratch: no workspace tensor is passed."""
+        A = int(q.shape[0])
+        st = cache.struct()
+        _check(get_lib().dspark_attend_no_alloc(self.handle, layer, ctypes.byref(st), q.data_ptr(), k_blk.data_ptr(),
+                                                v_blk.data_ptr(), out.data_ptr(), A, max_ctx_len, _stream_ptr(stream)))
 
     def dspark_read_device_status(self, stream=None) -> int:
         v = ctypes.c_int32(0)

@@ -246,6 +246,29 @@ int dspark_attend(const dspark_model* model, int32_t layer, const dspark_kv_cach
                   const void* q, const void* k_blk, const void* v_blk, void* out,
                   int32_t A, int32_t max_ctx_len, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * dspark_attend without a workspace argument: it computes exactly what
+ * dspark_attend computes (same kernels, same split plan), for callers that
+ * cannot provide device scratch memory -- a plugin whose host program owns
+ * the whole device pool and hands it only the tensors above, or a path that
+ * must not call cudaMalloc (which may synchronise the device). The pages have
+ * no counterpart to this entry point.
+ * Its scratch (the per-split softmax state) is a 16 MiB static device array
+ * inside libdspark, allocated on every GPU that loads the library and held
+ * until the process exits. Shapes whose state exceeds 16 MiB
+ * (A * nH * (context splits + 1) * gamma * (hd + 2) * 4 bytes) are refused
+ * with DSPARK_ERR_WORKSPACE before any launch. It allocates nothing. The first
+ * call on each device looks up the array's device address (a one-time
+ * runtime call): make that first call, with the model's device current,
+ * before any stream capture. Every call on a device shares the one array, so
+ * calls that overlap on the GPU (different streams or threads) race: issue
+ * them in order on one stream per device. No part of the array needs to
+ * start at zero: each call writes every slot before reading it.
+ */
+int dspark_attend_no_alloc(const dspark_model* model, int32_t layer, const dspark_kv_cache* cache,
+                           const void* q, const void* k_blk, const void* v_blk, void* out,
+                           int32_t A, int32_t max_ctx_len, void* stream);
+
 /* Synchronises `stream`, returns the device status bits in *status and
  * clears them. */
 int dspark_read_device_status(const dspark_model* model, void* stream, int32_t* status);
