@@ -144,8 +144,10 @@ struct Carve {
 };
 
 struct DraftPlan {
-    int M, S_qk, S_o, S_gu, S_down, S_max, attn_splits, attn_chunk, walk_blocks;
-    size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx, total;
+    int M, attn_splits, attn_chunk, walk_blocks;
+    bool pairs;   // GEMM inputs also kept as bf16 (hi, lo) pairs for the tensor-core GEMMs
+    size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx;
+    size_t x_hi, x_lo, ao_hi, ao_lo, act_hi, act_lo, total;
 };
 
 DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
@@ -153,12 +155,11 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     DraftPlan p{};
     p.M = A * d.gamma;
     const int Nqk = (d.nH + d.nKv) * d.hd;
-    p.S_qk = gemm_splits(m, p.M, Nqk, d.H);
-    p.S_o = gemm_splits(m, p.M, d.H, d.nH * d.hd);
-    p.S_gu = gemm_splits(m, p.M, 2 * d.I, d.H);
-    p.S_down = gemm_splits(m, p.M, d.H, d.I);
-    size_t part_elems = std::max({(size_t)p.S_qk * Nqk, (size_t)p.S_o * d.H, (size_t)p.S_gu * 2 * d.I,
-                                  (size_t)p.S_down * d.H}) * (size_t)p.M;
+    p.pairs = use_tensor_cores(m);
+    const size_t part_elems = std::max({gemm_part_elems(m, p.M, Nqk, d.H, p.pairs),
+                                        gemm_part_elems(m, p.M, d.H, d.nH * d.hd, p.pairs),
+                                        gemm_part_elems(m, p.M, 2 * d.I, d.H, p.pairs),
+                                        gemm_part_elems(m, p.M, d.H, d.I, p.pairs)});
     // attention: context chunks so that A * nH * splits covers the GPU ~2x
     int chunk = 64;
     int want = std::max(1, (2 * m->num_sms + A * d.nH - 1) / (A * d.nH));
@@ -185,6 +186,13 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.ticket = c.take(256);
     p.walk_val = c.take((size_t)p.walk_blocks * A * 4);
     p.walk_idx = c.take((size_t)p.walk_blocks * A * 4);
+    const size_t pb = p.pairs ? 2 : 0;
+    p.x_hi = c.take((size_t)p.M * d.H * pb);
+    p.x_lo = c.take((size_t)p.M * d.H * pb);
+    p.ao_hi = c.take((size_t)p.M * d.nH * d.hd * pb);
+    p.ao_lo = c.take((size_t)p.M * d.nH * d.hd * pb);
+    p.act_hi = c.take((size_t)p.M * d.I * pb);
+    p.act_lo = c.take((size_t)p.M * d.I * pb);
     p.total = c.off;
     return p;
 }
@@ -193,18 +201,19 @@ constexpr int64_t kProjectChunkRows = 16384;
 
 struct ProjectPlan {
     int64_t chunk_rows;
-    int S;
     size_t nvalid, raw, total;
 };
 ProjectPlan plan_project(const dspark_model* m, int64_t rows) {
     const Dims& d = m->d;
     ProjectPlan p{};
-    p.chunk_rows = std::min<int64_t>(std::max<int64_t>(rows, 1), kProjectChunkRows);
+    rows = std::max<int64_t>(rows, 1);
+    p.chunk_rows = std::min<int64_t>(rows, kProjectChunkRows);
     const int N = d.Lyr * d.nKv * d.hd;
-    p.S = gemm_splits(m, (int)p.chunk_rows, N, d.H);
+    size_t raw = gemm_part_elems(m, (int)p.chunk_rows, N, d.H, false);
+    if (rows % p.chunk_rows) raw = std::max(raw, gemm_part_elems(m, (int)(rows % p.chunk_rows), N, d.H, false));
     Carve c;
     p.nvalid = c.take(4096 * 4);
-    p.raw = project_needs_raw(m) ? c.take((size_t)p.S * p.chunk_rows * N * 4) : 0;
+    p.raw = c.take(raw * 4);
     p.total = c.off;
     return p;
 }
@@ -216,7 +225,6 @@ int project_rows(const dspark_model* m, const void* hidden, int B, int Lrows, co
                  const ProjectPlan& pp, cudaStream_t s) {
     const Dims& d = m->d;
     const int64_t rows = (int64_t)B * Lrows;
-    const int N = d.Lyr * d.nKv * d.hd;
     const size_t es = esize(d.dtype);
     for (int64_t r0 = 0; r0 < rows; r0 += pp.chunk_rows) {
         const int nr = (int)std::min<int64_t>(pp.chunk_rows, rows - r0);
@@ -224,10 +232,9 @@ int project_rows(const dspark_model* m, const void* hidden, int B, int Lrows, co
         rp.B = B; rp.Lrows = Lrows; rp.row0 = (int)r0; rp.nrows = nr; rp.n_valid = n_valid;
         rp.dst_row0 = dst_row0; rp.pos0 = pos0; rp.static_pos = static_pos;
         const void* X = static_cast<const char*>(hidden) + (size_t)r0 * d.H * es;
-        cudaError_t e = run_kv_projection(m, X, nr, rp, dst, at<float>(ws, pp.raw), pp.S, s);
+        cudaError_t e = run_kv_projection(m, X, nr, rp, dst, at<float>(ws, pp.raw), s);
         if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("context K/V projection launch: ") + cudaGetErrorString(e));
     }
-    (void)N;
     return DSPARK_OK;
 }
 
@@ -481,26 +488,36 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int M = p.M;
     float* h = at<float>(ws, p.h);
-    float* x = at<float>(ws, p.x);
     float* part = at<float>(ws, p.part);
     float* q = at<float>(ws, p.q); void* kb = at<void>(ws, p.kb); void* vb = at<void>(ws, p.vb);
-    float* ao = at<float>(ws, p.attn_out); float* act = at<float>(ws, p.act);
     float* U = base_logits ? base_logits : at<float>(ws, p.U);
+    ActBuf x, ao, act;
+    x.f32 = at<float>(ws, p.x); ao.f32 = at<float>(ws, p.attn_out); act.f32 = at<float>(ws, p.act);
+    if (p.pairs) {
+        x.hi = at<bf16>(ws, p.x_hi); x.lo = at<bf16>(ws, p.x_lo);
+        ao.hi = at<bf16>(ws, p.ao_hi); ao.lo = at<bf16>(ws, p.ao_lo);
+        act.hi = at<bf16>(ws, p.act_hi); act.lo = at<bf16>(ws, p.act_lo);
+    }
     const int Nqk = (d.nH + d.nKv) * d.hd;
+    PartView pv;
     cudaError_t e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
     for (int l = 0; l < d.Lyr && e == cudaSuccess; ++l) {
         const LayerRef& L = m->layers[l];
-        e = run_gemm(m, x, d.H, L.qk, M, Nqk, d.H, p.S_qk, part, s);
-        if (e == cudaSuccess) e = launch_qk_epilogue(m, l, part, p.S_qk, (int64_t)M * Nqk, A, block_pos, q, kb, vb, s);
-        if (e == cudaSuccess) e = run_attention(m, attn_args(m, p, ws, cache, l, A, q, kb, vb, ao, DSPARK_DTYPE_F32), s);
-        if (e == cudaSuccess) e = run_gemm(m, ao, d.nH * d.hd, L.o, M, d.H, d.nH * d.hd, p.S_o, part, s);
-        if (e == cudaSuccess) e = launch_o_epilogue(m, l, part, p.S_o, (int64_t)M * d.H, M, h, x, s);
-        if (e == cudaSuccess) e = run_gemm(m, x, d.H, L.gu, M, 2 * d.I, d.H, p.S_gu, part, s);
-        if (e == cudaSuccess) e = launch_gu_epilogue(m, part, p.S_gu, (int64_t)M * 2 * d.I, M, act, s);
-        if (e == cudaSuccess) e = run_gemm(m, act, d.I, L.down, M, d.H, d.I, p.S_down, part, s);
-        if (e == cudaSuccess) e = launch_down_epilogue(m, l, part, p.S_down, (int64_t)M * d.H, M, h, x, s);
+        e = run_gemm(m, x, L.qk, M, Nqk, d.H, part, &pv, s);
+        if (e == cudaSuccess) e = launch_qk_epilogue(m, l, pv, A, block_pos, q, kb, vb, s);
+        if (e == cudaSuccess) {
+            AttnArgs a = attn_args(m, p, ws, cache, l, A, q, kb, vb, ao.f32, DSPARK_DTYPE_F32);
+            a.out_hi = ao.hi; a.out_lo = ao.lo;
+            e = run_attention(m, a, s);
+        }
+        if (e == cudaSuccess) e = run_gemm(m, ao, L.o, M, d.H, d.nH * d.hd, part, &pv, s);
+        if (e == cudaSuccess) e = launch_o_epilogue(m, l, pv, M, h, x, s);
+        if (e == cudaSuccess) e = run_gemm(m, x, L.gu, M, 2 * d.I, d.H, part, &pv, s);
+        if (e == cudaSuccess) e = launch_gu_epilogue(m, pv, M, act, s);
+        if (e == cudaSuccess) e = run_gemm(m, act, L.down, M, d.H, d.I, part, &pv, s);
+        if (e == cudaSuccess) e = launch_down_epilogue(m, l, pv, M, h, x, s);
     }
-    if (e == cudaSuccess) e = run_lm_head(m, x, M, U, s);
+    if (e == cudaSuccess) e = run_lm_head(m, x, M, U, part, s);
     if (e == cudaSuccess) {
         WalkArgs wa{};
         wa.U = U; wa.tokens = tokens; wa.prev = at<int32_t>(ws, p.prev);
@@ -515,7 +532,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
             e = launch_walk_step(m, wa, s);
         }
     }
-    if (e == cudaSuccess) e = launch_confidence(m, x, anchors, tokens, A, conf, lengths, s);
+    if (e == cudaSuccess) e = launch_confidence(m, x.f32, anchors, tokens, A, conf, lengths, s);
     if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("draft round launch: ") + cudaGetErrorString(e));
     return DSPARK_OK;
 }

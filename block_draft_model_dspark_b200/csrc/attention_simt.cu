@@ -143,7 +143,14 @@ __global__ void attn_merge_kernel(AttnArgs a, int G, int nH, int hd) {
         den += w * a.part_ml[base * 2 + 1];
         num += w * a.part_o[base * hd + d];
     }
-    store_any(a.out, (((int64_t)b * G + i) * nH + h) * hd + d, a.out_dtype, num / den);
+    const int64_t o = (((int64_t)b * G + i) * nH + h) * hd + d;
+    const float v = num / den;
+    store_any(a.out, o, a.out_dtype, v);
+    if (a.out_hi) {
+        const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+        a.out_hi[o] = hv;
+        a.out_lo[o] = __float2bfloat16_rn(v - __bfloat162float(hv));
+    }
 }
 
 }  // namespace

@@ -1,5 +1,6 @@
-// Chooses the kernel for each contraction: CUDA-core paths for the fp32
-// model (whose 1e-4 bar excludes TF32), tensor-core paths for bf16.
+// Chooses the kernel for each contraction: tcgen05 tensor cores for bf16
+// weights; CUDA cores for the fp32 model (whose 1e-4 bar excludes TF32) and
+// for 4-bit weights (dequantized on load).
 #include <algorithm>
 
 #include "gemm.h"
@@ -9,16 +10,17 @@ namespace dspark {
 cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
 
 namespace {
+
 int simt_kps(int K, int S) {
     int kps = (K + S - 1) / S;
     return (kps + 31) / 32 * 32;
 }
-}  // namespace
 
-int gemm_splits(const dspark_model* m, int M, int N, int K) {
+// Split count of the CUDA-core GEMM: ~2 CTAs per SM, then the count the launch really produces.
+int simt_splits(const dspark_model* m, int M, int N, int K) {
     const int tiles = ((N + 63) / 64) * ((M + 63) / 64);
     int S = std::max(1, std::min((2 * m->num_sms + tiles - 1) / tiles, std::max(1, K / 128)));
-    for (;;) {   // the split count the launch will really produce
+    for (;;) {
         const int kps = simt_kps(K, S);
         const int z = (K + kps - 1) / kps;
         if (z == S) return S;
@@ -31,34 +33,69 @@ double weight_bytes(const dspark_model* m, int64_t N, int64_t K) {
     return (double)N * K * (m->d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0);
 }
 
-cudaError_t run_gemm(const dspark_model* m, const void* X, int64_t ldx, const MatRef& W, int M, int N, int K,
-                     int splits, float* out, cudaStream_t s) {
+}  // namespace
+
+bool use_tensor_cores(const dspark_model* m) { return m->d.dtype == DSPARK_DTYPE_BF16 && !m->d.quant; }
+
+size_t gemm_part_elems(const dspark_model* m, int M, int N, int K, bool act_pair) {
+    if (M <= 0) return 0;
+    if (use_tensor_cores(m)) return tc::gemm_partial_elems(tc::plan_gemm(m->num_sms, M, N, K, act_pair ? 2 : 1, false));
+    return (size_t)simt_splits(m, M, N, K) * M * N;
+}
+
+cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, int M, int N, int K, float* part,
+                     PartView* view, cudaStream_t s) {
     KernelTimer t(DSPARK_TIMER_GEMM, s, weight_bytes(m, N, K) + 4.0 * M * K + 4.0 * M * N, 2.0 * M * N * K);
-    return launch_simt_gemm(X, ldx, DSPARK_DTYPE_F32, m->d.dtype, W, m->d.group, M, N, K, splits, out, N,
+    *view = PartView{};
+    view->p = part;
+    if (use_tensor_cores(m)) {
+        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, 2, false);
+        view->mode = 1;
+        view->plan = p;
+        return tc::launch_gemm_tc(p, W.w, W.n, X.hi, X.lo, part, false, 0, 0.f, m->ws.status, s);
+    }
+    const int S = simt_splits(m, M, N, K);
+    view->mode = 0; view->S = S; view->stride = (int64_t)M * N; view->ld = N;
+    return launch_simt_gemm(X.f32, K, DSPARK_DTYPE_F32, m->d.dtype, W, m->d.group, M, N, K, S, part, N,
                             (int64_t)M * N, false, 0.f, s);
 }
 
-cudaError_t run_lm_head(const dspark_model* m, const void* x, int M, float* U, cudaStream_t s) {
+cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U, float* part, cudaStream_t s) {
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_LM_HEAD, s, weight_bytes(m, d.V, d.H) + 4.0 * M * d.H + 4.0 * M * d.V,
                   2.0 * M * (double)d.V * d.H);
-    return launch_simt_gemm(x, d.H, DSPARK_DTYPE_F32, d.dtype, m->lm_head, d.group, M, d.V, d.H, 1, U, d.V, 0, true,
-                            d.cap, s);
+    (void)part;
+    if (use_tensor_cores(m)) {
+        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, d.V, d.H, 2, true);
+        return tc::launch_gemm_tc(p, m->lm_head.w, d.V, x.hi, x.lo, U, true, d.V, d.cap, m->ws.status, s);
+    }
+    return launch_simt_gemm(x.f32, d.H, DSPARK_DTYPE_F32, d.dtype, m->lm_head, d.group, M, d.V, d.H, 1, U, d.V, 0,
+                            true, d.cap, s);
 }
 
-bool project_needs_raw(const dspark_model* m) { (void)m; return true; }
-
 cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, const RowsPlan& rp, const KvDest& dst,
-                              float* raw, int splits, cudaStream_t s) {
+                              float* raw, cudaStream_t s) {
     const Dims& d = m->d;
     const int N = d.Lyr * d.nKv * d.hd;
     const double es = d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0;
     KernelTimer t(DSPARK_TIMER_KV_PROJECT, s, weight_bytes(m, N, d.H) + es * nrows * d.H + 2.0 * es * nrows * N,
                   2.0 * nrows * (double)N * d.H);
-    cudaError_t e = launch_simt_gemm(X, d.H, d.dtype, d.dtype, m->wk_all, d.group, nrows, N, d.H, splits, raw, N,
-                                     (int64_t)nrows * N, false, 0.f, s);
+    PartView view{};
+    view.p = raw;
+    cudaError_t e;
+    if (use_tensor_cores(m)) {
+        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, nrows, N, d.H, 1, false);
+        view.mode = 1;
+        view.plan = p;
+        e = tc::launch_gemm_tc(p, m->wk_all.w, N, X, nullptr, raw, false, 0, 0.f, m->ws.status, s);
+    } else {
+        const int S = simt_splits(m, nrows, N, d.H);
+        view.mode = 0; view.S = S; view.stride = (int64_t)nrows * N; view.ld = N;
+        e = launch_simt_gemm(X, d.H, d.dtype, d.dtype, m->wk_all, d.group, nrows, N, d.H, S, raw, N,
+                             (int64_t)nrows * N, false, 0.f, s);
+    }
     if (e != cudaSuccess) return e;
-    return launch_kv_epilogue(m, raw, splits, (int64_t)nrows * N, rp, dst, s);
+    return launch_kv_epilogue(m, view, rp, dst, s);
 }
 
 cudaError_t run_attention(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {

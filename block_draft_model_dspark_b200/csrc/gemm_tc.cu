@@ -1,0 +1,333 @@
+// Tensor-core GEMM for sm_100a: out = X @ W^T with bf16 operands and fp32
+// accumulation in TMEM (deepspec.ts `matmulW`: x @ W^T for a Linear weight
+// stored [out, in]).
+//
+// Orientation ("swap-AB"): the weight supplies the MMA's 128-row A operand
+// (128 output features per tile) and the activation rows supply its N side
+// (BN = 16..256 columns), so a round with 16 activation rows still runs full
+// 128-row MMAs and streams each weight tile exactly once.
+//
+// Operands are staged by TMA with the 128-byte swizzle into a ring of
+// shared-memory stages. An fp32 activation enters as a bf16 pair (hi, lo =
+// x - hi): two MMAs per K slice accumulate both into the same fp32 tile, so
+// the activation keeps ~16 significant bits while the weight streams once.
+//
+// Roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// MMAs, warps 2-5 drain accumulators (TMEM lane quadrant = warp % 4).
+// Accumulators are double-buffered in TMEM so the epilogue of one tile
+// overlaps the MMAs of the next.
+//
+// Work split: the grid is persistent (at most one CTA per SM). In stream-K
+// mode the tiles' K-blocks form one sequence cut into equal contiguous
+// ranges, one per CTA; a CTA writes one fp32 partial tile per tile it
+// touches, and the consumer sums a tile's partials in CTA order (no
+// atomics: deterministic). In tile mode each CTA owns whole tiles
+// (round-robin) and the epilogue writes the result directly, optionally with
+// the final-logit softcap.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+#include <string>
+
+#include "internal.h"
+#include "gemm_tc.h"
+#include "tc_ptx.cuh"
+
+namespace dspark {
+namespace tc {
+namespace {
+
+constexpr int BM = 128;            // weight rows per tile (MMA M)
+constexpr int BK = 64;             // K elements per stage: one 128-byte swizzle row
+constexpr int kThreads = 192;
+constexpr int kABytes = BM * BK * 2;
+
+struct KParams {
+    GemmPlan p;
+    float* out;        // partial tiles [tile][P][BN][128], or result rows when `direct`
+    int64_t ldo;       // direct: row stride of `out`
+    float cap;         // direct: softcap (0 = none)
+    int direct;        // tile mode only: write out[m * ldo + n] instead of partial tiles
+    int32_t* status;
+};
+
+// Iterates the (tile, k-range) segments of one CTA, identically in every role.
+struct SegIter {
+    const GemmPlan& p;
+    int c;
+    int g, g1;      // stream-K: this CTA's remaining global K-block range
+    int t;          // tile mode: next tile
+    __device__ SegIter(const GemmPlan& p_, int c_) : p(p_), c(c_) {
+        g = p.streamk ? p.range_lo(c) : 0;
+        g1 = p.streamk ? p.range_lo(c + 1) : 0;
+        t = c;
+    }
+    __device__ bool next(int& tile, int& k0, int& k1, int& slot) {
+        if (p.streamk) {
+            if (g >= g1) return false;
+            tile = g / p.kb;
+            k0 = g - tile * p.kb;
+            k1 = min(p.kb, k0 + (g1 - g));
+            slot = c - p.cta_of(tile * p.kb);
+            g += k1 - k0;
+            return true;
+        }
+        if (t >= p.tiles) return false;
+        tile = t; k0 = 0; k1 = p.kb; slot = 0;
+        t += p.grid;
+        return true;
+    }
+};
+
+template <int NP>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX0,
+               const __grid_constant__ CUtensorMap tmX1, KParams kp) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const GemmPlan& p = kp.p;
+    const int BN = p.BN;
+    const int stages = p.stages;
+    const int b_bytes = BN * BK * 2;
+    const int stage_bytes = kABytes + NP * b_bytes;
+
+    // carve: [stages x (A, B0, B1)] then barriers
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + stages * stage_bytes);
+    uint64_t* empty = full + stages;
+    uint64_t* acc_full = empty + stages;      // [2]
+    uint64_t* acc_empty = acc_full + 2;       // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t tmem_cols = p.tmem_cols;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 128); }
+        *abort_flag = 0;
+        mbar_fence_init();
+        prefetch_tmap(&tmW); prefetch_tmap(&tmX0);
+        if (NP == 2) prefetch_tmap(&tmX1);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, tmem_cols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            SegIter it(p, blockIdx.x);
+            int tile, k0, k1, slot, n = 0;
+            bool ok = true;
+            while (ok && it.next(tile, k0, k1, slot)) {
+                const int nt = tile / p.n_mt, mt = tile % p.n_mt;
+                for (int kk = k0; kk < k1; ++kk, ++n) {
+                    const int s = n % stages;
+                    const uint32_t ph = (uint32_t)(n / stages) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, kp.status)) { ok = false; break; }
+                    uint8_t* st = base + s * stage_bytes;
+                    mbar_arrive_expect_tx(&full[s], stage_bytes);
+                    tma_load_2d(st, &tmW, &full[s], kk * BK, nt * BM);
+                    tma_load_2d(st + kABytes, &tmX0, &full[s], kk * BK, mt * BN);
+                    if (NP == 2) tma_load_2d(st + kABytes + b_bytes, &tmX1, &full[s], kk * BK, mt * BN);
+                }
+            }
+            // drain: the loads of the last `stages` slots complete before teardown
+            for (int d = 0; ok && d < stages && d < n; ++d) {
+                const int m = n - 1 - d;
+                if (!mbar_wait(&full[m % stages], (uint32_t)(m / stages) & 1u, abort_flag, kp.status)) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(BM, BN);
+            SegIter it(p, blockIdx.x);
+            int tile, k0, k1, slot, n = 0, seg = 0;
+            bool ok = true;
+            while (ok && it.next(tile, k0, k1, slot)) {
+                const int acc = seg & 1;
+                const uint32_t aph = (uint32_t)(seg >> 1) & 1u;
+                if (!mbar_wait(&acc_empty[acc], aph ^ 1u, abort_flag, kp.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kk = k0; kk < k1; ++kk, ++n) {
+                    const int s = n % stages;
+                    const uint32_t ph = (uint32_t)(n / stages) & 1u;
+                    if (!mbar_wait(&full[s], ph, abort_flag, kp.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(base + s * stage_bytes);
+                    const uint64_t adesc = sdesc_k_sw128(a_addr);
+#pragma unroll
+                    for (int part = 0; part < NP; ++part) {
+                        const uint64_t bdesc = sdesc_k_sw128(a_addr + kABytes + part * b_bytes);
+#pragma unroll
+                        for (int j = 0; j < BK / 16; ++j) {
+                            const uint32_t accum = (kk > k0 || part > 0 || j > 0) ? 1u : 0u;
+                            mma_bf16(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, accum);
+                        }
+                    }
+                    mma_commit(&empty[s]);          // frees the stage once these MMAs have read it
+                }
+                if (!ok) break;
+                mma_commit(&acc_full[acc]);         // the tile's accumulator is complete
+                ++seg;
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue (warps 2-5)
+        const int quad = warp & 3;
+        const int n_local = quad * 32 + lane;
+        SegIter it(p, blockIdx.x);
+        int tile, k0, k1, slot, seg = 0;
+        while (it.next(tile, k0, k1, slot)) {
+            const int acc = seg & 1;
+            const uint32_t aph = (uint32_t)(seg >> 1) & 1u;
+            if (!mbar_wait(&acc_full[acc], aph, abort_flag, kp.status)) break;
+            tc_fence_after();
+            const int nt = tile / p.n_mt, mt = tile % p.n_mt;
+            const int n = nt * BM + n_local;
+            const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld_x16(tbase + (uint32_t)c0, r);
+                tmem_ld_wait();
+                if (kp.direct) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int m = mt * BN + c0 + j;
+                        if (m < p.M && n < p.N) {
+                            float v = __uint_as_float(r[j]);
+                            if (kp.cap > 0.f) v = kp.cap * tanhf(v / kp.cap);
+                            kp.out[(int64_t)m * kp.ldo + n] = v;
+                        }
+                    }
+                } else {
+                    float* dst = kp.out + (((int64_t)tile * p.P + slot) * BN + c0) * BM + n_local;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) dst[(int64_t)j * BM] = __uint_as_float(r[j]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+            ++seg;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// Row-major bf16 [rows, cols] matrix, box of box_rows x 64 columns, 128-byte swizzle.
+bool make_tmap(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
+    if (!get_encoder()) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int tmem_cols_for(int BN) {
+    int c = 32;
+    while (c < 2 * BN) c <<= 1;
+    return c;
+}
+
+}  // namespace
+
+GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles) {
+    GemmPlan p{};
+    p.M = M; p.N = N; p.K = K; p.np = np;
+    const int m_pad = (M + 15) / 16 * 16;
+    p.BN = m_pad <= 256 ? m_pad : 256;
+    p.n_mt = (M + p.BN - 1) / p.BN;
+    p.n_nt = (N + BM - 1) / BM;
+    p.kb = K / BK;
+    p.tiles = p.n_mt * p.n_nt;
+    const int stage_bytes = kABytes + np * p.BN * BK * 2;
+    p.stages = std::max(2, std::min(8, (200 * 1024) / stage_bytes));
+    p.tmem_cols = tmem_cols_for(p.BN);
+    // tile mode when whole tiles balance the SMs to >= 90%, else stream-K
+    const int waves = (p.tiles + num_sms - 1) / num_sms;
+    const bool tiles_ok = force_tiles || (p.tiles >= num_sms && 10 * p.tiles >= 9 * waves * num_sms);
+    if (tiles_ok) {
+        p.mode = kModeTiles; p.streamk = 0;
+        p.grid = std::min(p.tiles, num_sms);
+        p.T = p.tiles * p.kb; p.G = p.grid; p.P = 1;
+    } else {
+        p.mode = kModePartials; p.streamk = 1;
+        p.T = p.tiles * p.kb;
+        p.G = std::min(p.T, num_sms);
+        p.grid = p.G;
+        int P = 1;
+        for (int t = 0; t < p.tiles; ++t) P = std::max(P, p.cta_of((t + 1) * p.kb - 1) - p.cta_of(t * p.kb) + 1);
+        p.P = P;
+    }
+    return p;
+}
+
+size_t gemm_partial_elems(const GemmPlan& p) {
+    return (size_t)p.tiles * p.P * p.BN * BM;
+}
+
+size_t gemm_smem_bytes(const GemmPlan& p) {
+    const int stage_bytes = kABytes + p.np * p.BN * BK * 2;
+    return (size_t)p.stages * stage_bytes + 1024 + 256;
+}
+
+cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, const void* X0, const void* X1,
+                           float* out, bool direct, int64_t ldo, float cap, int32_t* status, cudaStream_t s) {
+    if (direct && p.mode != kModeTiles) return cudaErrorInvalidValue;
+    CUtensorMap tw, tx0, tx1;
+    if (!make_tmap(&tw, W, w_rows, p.K, BM)) return cudaErrorInvalidValue;
+    if (!make_tmap(&tx0, X0, p.M, p.K, p.BN)) return cudaErrorInvalidValue;
+    if (p.np == 2) {
+        if (!make_tmap(&tx1, X1, p.M, p.K, p.BN)) return cudaErrorInvalidValue;
+    } else {
+        tx1 = tx0;
+    }
+    KParams kp{};
+    kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.status = status; kp.direct = direct ? 1 : 0;
+    const size_t smem = gemm_smem_bytes(p);
+    cudaError_t e;
+    if (p.np == 2) {
+        e = cudaFuncSetAttribute(gemm_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        gemm_tc_kernel<2><<<p.grid, kThreads, smem, s>>>(tw, tx0, tx1, kp);
+    } else {
+        e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        gemm_tc_kernel<1><<<p.grid, kThreads, smem, s>>>(tw, tx0, tx1, kp);
+    }
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace dspark

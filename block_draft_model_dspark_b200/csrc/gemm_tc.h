@@ -1,0 +1,42 @@
+// Plan and launch interface of the tcgen05 GEMM (gemm_tc.cu), and the view
+// the row epilogues use to sum its partial tiles.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace dspark {
+namespace tc {
+
+constexpr int kModeTiles = 0;      // whole tiles per CTA; result written directly
+constexpr int kModePartials = 1;   // stream-K; fp32 partial tiles [tile][P][BN][128]
+
+struct GemmPlan {
+    int M, N, K, np;       // out [M, N] = X [M, K] @ W [N, K]^T; np = 1 (bf16 X) or 2 (X as bf16 hi + lo)
+    int BN;                // activation rows per tile (MMA N)
+    int n_mt, n_nt;        // tiles along the activation rows and along the 128 weight rows
+    int kb;                // 64-wide K blocks
+    int tiles;             // n_mt * n_nt; tile index t = nt * n_mt + mt
+    int stages, tmem_cols;
+    int mode, streamk;
+    int grid;              // CTAs launched
+    int T, G, P;           // stream-K: K blocks in all tiles, CTAs, most CTAs touching one tile
+    // First global K block of CTA c (stream-K partition of T blocks over G CTAs).
+    __host__ __device__ int range_lo(int c) const { return (int)(((int64_t)c * T) / G); }
+    // The CTA whose range holds global K block g.
+    __host__ __device__ int cta_of(int g) const { return (int)((((int64_t)g + 1) * G - 1) / T); }
+};
+
+GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles);
+size_t gemm_partial_elems(const GemmPlan& p);
+size_t gemm_smem_bytes(const GemmPlan& p);
+// W: bf16 [w_rows >= N, K]; X0 (and X1 when np == 2): bf16 [M, K].
+// Writes `out` as fp32 tiles [tile][P][BN][128] (P = 1 in tile mode), or, when
+// `direct` (tile mode only), the result rows out[m * ldo + n] with the softcap
+// cap * tanh(v / cap) applied when cap > 0.
+cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, const void* X0, const void* X1,
+                           float* out, bool direct, int64_t ldo, float cap, int32_t* status, cudaStream_t s);
+
+}  // namespace tc
+}  // namespace dspark

@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "../../include/dspark.h"
+#include "gemm_tc.h"
 
 namespace dspark {
 
@@ -48,6 +49,39 @@ struct ModelWs {
     bf16* wqk_s = nullptr; bf16* wqk_b = nullptr;   // quantized scales / biases of the stacks
     bf16* wgu_s = nullptr; bf16* wgu_b = nullptr;
     bf16* wk_all_s = nullptr; bf16* wk_all_b = nullptr;
+};
+
+// A GEMM result as its consumers read it: out[m][n] is the sum of the GEMM's
+// partial tiles. mode 0: CUDA-core split-K partials [S][M][ld]; mode 1: the
+// tcgen05 GEMM's tiles [tile][P][BN][128] (stream-K: the tile's partials
+// come from consecutive CTAs, summed in CTA order).
+struct PartView {
+    const float* p = nullptr;
+    int mode = 0;
+    int S = 1; int64_t stride = 0, ld = 0;
+    tc::GemmPlan plan{};
+    __device__ __forceinline__ float sum(int64_t m, int64_t n) const {
+        float v = 0.f;
+        if (mode == 0) {
+            for (int s = 0; s < S; ++s) v += p[s * stride + m * ld + n];
+            return v;
+        }
+        const int BN = plan.BN;
+        const int mt = (int)(m / BN), ml = (int)(m % BN), nt = (int)(n >> 7), nl = (int)(n & 127);
+        const int t = nt * plan.n_mt + mt;
+        int cnt = 1;
+        if (plan.streamk) cnt = plan.cta_of(t * plan.kb + plan.kb - 1) - plan.cta_of(t * plan.kb) + 1;
+        const float* q = p + (((int64_t)t * plan.P) * BN + ml) * 128 + nl;
+        for (int s = 0; s < cnt; ++s) v += q[(int64_t)s * BN * 128];
+        return v;
+    }
+};
+
+// An fp32 activation and, for tensor-core GEMMs, its bf16 pair hi + lo.
+struct ActBuf {
+    float* f32 = nullptr;
+    bf16* hi = nullptr;
+    bf16* lo = nullptr;
 };
 
 constexpr int kMaxLayers = 64;
@@ -94,8 +128,8 @@ cudaError_t launch_simt_gemm(const void* X, int64_t ldx, int x_dtype, int w_dtyp
                              int M, int N, int K, int splits, float* out, int64_t ldo, int64_t split_stride,
                              bool softcap, float cap, cudaStream_t s);
 
-// Context K/V epilogue: raw fp32 [rows, Lyr*nKv*hd] (sum of `splits` partials
-// at split_stride) -> cache rows. Row r = b*Lrows + t is valid when t < n_b.
+// Context K/V epilogue: the K/V GEMM's result [rows, Lyr*nKv*hd] -> cache rows.
+// Row r = b*Lrows + t is valid when t < n_b.
 struct KvDest {
     void* k; void* v;
     int64_t batch_stride;    // elements between batch rows   (= cap * nKv * hd)
@@ -111,29 +145,29 @@ struct RowsPlan {
     const int32_t* pos0;     // device [B] position of t = 0, or null (static_pos)
     int static_pos;
 };
-cudaError_t launch_kv_epilogue(const dspark_model* m, const float* raw, int splits, int64_t split_stride,
-                               const RowsPlan& rp, const KvDest& dst, cudaStream_t s);
+cudaError_t launch_kv_epilogue(const dspark_model* m, const PartView& raw, const RowsPlan& rp, const KvDest& dst,
+                               cudaStream_t s);
 cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStream_t s);
 
 // Activations of the round (x, q, attention output, gelu*up) are fp32 in the
 // workspace for both model dtypes; only the K/V cache and the block K/V are
 // stored in the model dtype.
 // Block embedding: h = embed[ids]*sqrt(H) (fp32 [M,H]); x = rms(h, w_in0) (fp32 [M,H]).
-cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, float* h, float* x,
+cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, float* h, const ActBuf& x,
                          int32_t* status, cudaStream_t s);
 // q (fp32) and block k/v (model dtype) heads from the [Wq;Wk] GEMM partials.
-cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
-                               int A, const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s);
+cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const PartView& part, int A,
+                               const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s);
 // h += rms(o_proj partials, post_attn); x = rms(h, pre_ff).
-cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
-                              int M, float* h, float* x, cudaStream_t s);
+cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,
+                              const ActBuf& x, cudaStream_t s);
 // act = gelu_tanh(g) * u  (fp32 [M, I]).
-cudaError_t launch_gu_epilogue(const dspark_model* m, const float* part, int splits, int64_t split_stride,
-                               int M, float* act, cudaStream_t s);
+cudaError_t launch_gu_epilogue(const dspark_model* m, const PartView& part, int M, const ActBuf& act,
+                               cudaStream_t s);
 // h = (h + rms(down partials, post_ff)) * layer_scalar; then x = rms(h, next gain)
 // (next gain = next layer's input norm, or the final norm).
-cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
-                                 int M, float* h, float* x, cudaStream_t s);
+cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,
+                                 const ActBuf& x, cudaStream_t s);
 
 // Attention: partial pass over context chunks + block keys, then merge.
 struct AttnArgs {
@@ -142,6 +176,7 @@ struct AttnArgs {
     const void* kc; const void* vc;                  // cache of this layer: [batch, cap, nKv, hd]
     const int32_t* len; int capacity;
     void* out;                                       // [A, G, nH, hd]
+    bf16* out_hi; bf16* out_lo;                      // optional bf16 pair of out (fp32 out only)
     float* part_o; float* part_ml;                   // workspace
     int A, n_splits, chunk;                          // context splits of `chunk` keys (+1 block split)
     int32_t* status;

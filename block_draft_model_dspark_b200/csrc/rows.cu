@@ -2,8 +2,11 @@
 // that follow each GEMM (norms, RoPE, residual adds, gelu, layer scalar),
 // the context K/V epilogue, and the confidence head with truncation.
 //
-// Each epilogue first sums the GEMM's split-K partials in split order (a
-// fixed order, so results do not depend on scheduling).
+// Each epilogue reads its GEMM's result through a PartView, which sums the
+// GEMM's partial tiles in a fixed order (results do not depend on
+// scheduling). Activations that feed the next GEMM are written in fp32 and,
+// when the model has bf16 weights, also as a bf16 pair (hi, lo = v - hi) for
+// the tensor-core GEMM.
 #include <math.h>
 
 #include "internal.h"
@@ -14,10 +17,13 @@ namespace {
 
 constexpr int kMaxPer = 16;   // columns per thread in the full-row kernels
 
-__device__ __forceinline__ float sum_splits(const float* part, int splits, int64_t stride, int64_t idx) {
-    float v = 0.f;
-    for (int s = 0; s < splits; ++s) v += part[s * stride + idx];
-    return v;
+__device__ __forceinline__ void store_act(const ActBuf& a, int64_t i, float v) {
+    a.f32[i] = v;
+    if (a.hi) {
+        const bf16 h = __float2bfloat16_rn(v);
+        a.hi[i] = h;
+        a.lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
 }
 
 // One element W[n, j] of a (possibly 4-bit) matrix.
@@ -30,10 +36,8 @@ __device__ __forceinline__ float mat_at(const MatRef& W, int dtype, int group, i
 
 // ------------------------------------------------------------------ context K/V
 // grid (rows, Lyr*nKv), block hd/2: thread i owns the RoPE pair (i, i + hd/2).
-__global__ void kv_epilogue_kernel(const float* __restrict__ raw, int splits, int64_t split_stride, int N,
-                                   RowsPlan rp, KvDest dst, const double* __restrict__ inv_freq,
-                                   LayerPtrs k_norms, int nKv, int hd, float eps,
-                                   int dtype, int32_t* status) {
+__global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const double* __restrict__ inv_freq,
+                                   LayerPtrs k_norms, int nKv, int hd, float eps, int dtype, int32_t* status) {
     __shared__ float red[32];
     const int r = blockIdx.x;
     const int rg = rp.row0 + r;
@@ -48,8 +52,8 @@ __global__ void kv_epilogue_kernel(const float* __restrict__ raw, int splits, in
     const int l = blockIdx.y / nKv, g = blockIdx.y % nKv;
     const int half = hd / 2, i = threadIdx.x;
     const int64_t col = (int64_t)blockIdx.y * hd;
-    const float x1 = sum_splits(raw, splits, split_stride, (int64_t)r * N + col + i);
-    const float x2 = sum_splits(raw, splits, split_stride, (int64_t)r * N + col + i + half);
+    const float x1 = raw.sum(r, col + i);
+    const float x2 = raw.sum(r, col + i + half);
     const float ss = block_sum(x1 * x1 + x2 * x2, red);
     const float rinv = rsqrtf(ss / (float)hd + eps);
     const float v1 = x1 * rinv, v2 = x2 * rinv;
@@ -72,7 +76,7 @@ __global__ void commit_len_kernel(int32_t* len, const int32_t* n_new, int B) {
 // ------------------------------------------------------------------ block embedding
 __global__ void embed_kernel(MatRef E, int dtype, int group, const int32_t* __restrict__ anchors, int gamma,
                              int mask_id, int V, int H, float scale, const void* __restrict__ w_in,
-                             float eps, float* __restrict__ h, float* __restrict__ x, int32_t* status) {
+                             float eps, float* __restrict__ h, ActBuf x, int32_t* status) {
     __shared__ float red[32];
     const int m = blockIdx.x;
     const int b = m / gamma, t = m % gamma;
@@ -99,26 +103,25 @@ __global__ void embed_kernel(MatRef E, int dtype, int group, const int32_t* __re
         const int j = threadIdx.x + c * blockDim.x;
         if (j < H) {
             h[(int64_t)m * H + j] = vals[c];
-            x[(int64_t)m * H + j] = vals[c] * rinv * load_any(w_in, j, dtype);
+            store_act(x, (int64_t)m * H + j, vals[c] * rinv * load_any(w_in, j, dtype));
         }
     }
 }
 
 // ------------------------------------------------------------------ q / k / v heads
 // grid (M, nH + nKv), block hd/2.
-__global__ void qk_epilogue_kernel(const float* __restrict__ part, int splits, int64_t split_stride, int N,
-                                   int gamma, int nH, int nKv, int hd, const int32_t* __restrict__ block_pos,
-                                   const double* __restrict__ inv_freq, const void* __restrict__ q_norm,
-                                   const void* __restrict__ k_norm, float eps, int dtype,
-                                   float* __restrict__ q, void* __restrict__ kb, void* __restrict__ vb) {
+__global__ void qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, int hd,
+                                   const int32_t* __restrict__ block_pos, const double* __restrict__ inv_freq,
+                                   const void* __restrict__ q_norm, const void* __restrict__ k_norm, float eps,
+                                   int dtype, float* __restrict__ q, void* __restrict__ kb, void* __restrict__ vb) {
     __shared__ float red[32];
     const int m = blockIdx.x, hh = blockIdx.y;
     const int b = m / gamma, t = m % gamma;
     const int pos = block_pos[b] + t;
     const int half = hd / 2, i = threadIdx.x;
     const int64_t col = (int64_t)hh * hd;
-    const float x1 = sum_splits(part, splits, split_stride, (int64_t)m * N + col + i);
-    const float x2 = sum_splits(part, splits, split_stride, (int64_t)m * N + col + i + half);
+    const float x1 = part.sum(m, col + i);
+    const float x2 = part.sum(m, col + i + half);
     const float ss = block_sum(x1 * x1 + x2 * x2, red);
     const float rinv = rsqrtf(ss / (float)hd + eps);
     float y1 = x1 * rinv, y2 = x2 * rinv;
@@ -143,11 +146,10 @@ __global__ void qk_epilogue_kernel(const float* __restrict__ part, int splits, i
 
 // ------------------------------------------------------------------ o_proj / down epilogues
 // mode 0 (o_proj):  h += rms(sum, g1);            x = rms(h, g2)
-// mode 1 (down):    h = (h + rms(sum, g1)) * s;   x = rms(h, g2)   (+ hf32 = x when given)
-__global__ void residual_epilogue_kernel(const float* __restrict__ part, int splits, int64_t split_stride, int H,
-                                         const void* __restrict__ g1, const void* __restrict__ g2,
-                                         const void* __restrict__ scalar, int mode, float eps, int dtype,
-                                         float* __restrict__ h, float* __restrict__ x) {
+// mode 1 (down):    h = (h + rms(sum, g1)) * s;   x = rms(h, g2)
+__global__ void residual_epilogue_kernel(PartView part, int H, const void* __restrict__ g1,
+                                         const void* __restrict__ g2, const void* __restrict__ scalar, int mode,
+                                         float eps, int dtype, float* __restrict__ h, ActBuf x) {
     __shared__ float red[32];
     const int m = blockIdx.x;
     float a[kMaxPer];
@@ -155,7 +157,7 @@ __global__ void residual_epilogue_kernel(const float* __restrict__ part, int spl
 #pragma unroll
     for (int c = 0; c < kMaxPer; ++c) {
         const int j = threadIdx.x + c * blockDim.x;
-        a[c] = j < H ? sum_splits(part, splits, split_stride, (int64_t)m * H + j) : 0.f;
+        a[c] = j < H ? part.sum(m, j) : 0.f;
         ss += a[c] * a[c];
     }
     ss = block_sum(ss, red);
@@ -177,20 +179,17 @@ __global__ void residual_epilogue_kernel(const float* __restrict__ part, int spl
 #pragma unroll
     for (int c = 0; c < kMaxPer; ++c) {
         const int j = threadIdx.x + c * blockDim.x;
-        if (j < H) {
-            x[(int64_t)m * H + j] = a[c] * r2 * load_any(g2, j, dtype);
-        }
+        if (j < H) store_act(x, (int64_t)m * H + j, a[c] * r2 * load_any(g2, j, dtype));
     }
 }
 
-__global__ void gu_epilogue_kernel(const float* __restrict__ part, int splits, int64_t split_stride, int M, int I,
-                                   float* __restrict__ act) {
+__global__ void gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
     const int64_t total = (int64_t)M * I;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t m = e / I, i = e % I;
-        const float g = sum_splits(part, splits, split_stride, m * 2 * I + i);
-        const float u = sum_splits(part, splits, split_stride, m * 2 * I + I + i);
-        act[e] = gelu_tanh(g) * u;
+        const float g = part.sum(m, i);
+        const float u = part.sum(m, I + i);
+        store_act(act, e, gelu_tanh(g) * u);
     }
 }
 
@@ -232,15 +231,15 @@ int row_threads(int H) {
 
 }  // namespace
 
-cudaError_t launch_kv_epilogue(const dspark_model* m, const float* raw, int splits, int64_t split_stride,
-                               const RowsPlan& rp, const KvDest& dst, cudaStream_t s) {
+cudaError_t launch_kv_epilogue(const dspark_model* m, const PartView& raw, const RowsPlan& rp, const KvDest& dst,
+                               cudaStream_t s) {
     const Dims& d = m->d;
     if (rp.nrows <= 0) return cudaSuccess;
     LayerPtrs kn{};
     for (int l = 0; l < d.Lyr; ++l) kn.p[l] = m->layers[l].k_norm;
     dim3 grid(rp.nrows, d.Lyr * d.nKv);
-    kv_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(raw, splits, split_stride, d.Lyr * d.nKv * d.hd, rp, dst,
-                                                 m->ws.inv_freq, kn, d.nKv, d.hd, d.eps, d.dtype, m->ws.status);
+    kv_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(raw, rp, dst, m->ws.inv_freq, kn, d.nKv, d.hd, d.eps, d.dtype,
+                                                 m->ws.status);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -251,8 +250,8 @@ cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStr
     return cudaGetLastError();
 }
 
-cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, float* h, float* x, int32_t* status,
-                         cudaStream_t s) {
+cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, float* h, const ActBuf& x,
+                         int32_t* status, cudaStream_t s) {
     const Dims& d = m->d;
     embed_kernel<<<A * d.gamma, row_threads(d.H), 0, s>>>(m->embed, d.dtype, d.group, anchors, d.gamma, d.mask_id,
                                                          d.V, d.H, sqrtf((float)d.H), m->layers[0].in_norm, d.eps,
@@ -261,46 +260,46 @@ cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, f
     return cudaGetLastError();
 }
 
-cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
-                               int A, const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s) {
+cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const PartView& part, int A,
+                               const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s) {
     const Dims& d = m->d;
     dim3 grid(A * d.gamma, d.nH + d.nKv);
-    qk_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(part, splits, split_stride, (d.nH + d.nKv) * d.hd, d.gamma, d.nH,
-                                                 d.nKv, d.hd, block_pos, m->ws.inv_freq, m->layers[layer].q_norm,
-                                                 m->layers[layer].k_norm, d.eps, d.dtype, q, kb, vb);
+    qk_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(part, d.gamma, d.nH, d.nKv, d.hd, block_pos, m->ws.inv_freq,
+                                                 m->layers[layer].q_norm, m->layers[layer].k_norm, d.eps, d.dtype,
+                                                 q, kb, vb);
     count_launches(1);
     return cudaGetLastError();
 }
 
-cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
-                              int M, float* h, float* x, cudaStream_t s) {
+cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,
+                              const ActBuf& x, cudaStream_t s) {
     const Dims& d = m->d;
     const LayerRef& L = m->layers[layer];
-    residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, splits, split_stride, d.H, L.post_attn_norm,
-                                                            L.pre_ff_norm, nullptr, 0, d.eps, d.dtype, h, x);
+    residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, d.H, L.post_attn_norm, L.pre_ff_norm, nullptr, 0,
+                                                            d.eps, d.dtype, h, x);
     count_launches(1);
     return cudaGetLastError();
 }
 
-cudaError_t launch_gu_epilogue(const dspark_model* m, const float* part, int splits, int64_t split_stride, int M,
-                               float* act, cudaStream_t s) {
+cudaError_t launch_gu_epilogue(const dspark_model* m, const PartView& part, int M, const ActBuf& act,
+                               cudaStream_t s) {
     const Dims& d = m->d;
     const int64_t total = (int64_t)M * d.I;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 8 * m->num_sms) blocks = 8 * m->num_sms;
-    gu_epilogue_kernel<<<blocks, 256, 0, s>>>(part, splits, split_stride, M, d.I, act);
+    gu_epilogue_kernel<<<blocks, 256, 0, s>>>(part, M, d.I, act);
     count_launches(1);
     return cudaGetLastError();
 }
 
-cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const float* part, int splits, int64_t split_stride,
-                                 int M, float* h, float* x, cudaStream_t s) {
+cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,
+                                 const ActBuf& x, cudaStream_t s) {
     const Dims& d = m->d;
     const LayerRef& L = m->layers[layer];
     const bool last = layer + 1 == d.Lyr;
     const void* next = last ? m->final_norm : m->layers[layer + 1].in_norm;
-    residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, splits, split_stride, d.H, L.post_ff_norm, next,
-                                                            L.layer_scalar, 1, d.eps, d.dtype, h, x);
+    residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, d.H, L.post_ff_norm, next, L.layer_scalar, 1,
+                                                            d.eps, d.dtype, h, x);
     count_launches(1);
     return cudaGetLastError();
 }
