@@ -160,11 +160,7 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
                                         gemm_part_elems(m, p.M, d.H, d.nH * d.hd, p.pairs),
                                         gemm_part_elems(m, p.M, 2 * d.I, d.H, p.pairs),
                                         gemm_part_elems(m, p.M, d.H, d.I, p.pairs)});
-    // attention: context chunks so that A * nH * splits covers the GPU ~2x
-    int chunk = 64;
-    int want = std::max(1, (2 * m->num_sms + A * d.nH - 1) / (A * d.nH));
-    if (maxL > 0) chunk = std::max(64, (maxL + want - 1) / want);
-    chunk = (chunk + 15) / 16 * 16;
+    const int chunk = attention_key_chunk(m, A, maxL);
     p.attn_chunk = chunk;
     p.attn_splits = maxL > 0 ? (maxL + chunk - 1) / chunk : 0;
     p.walk_blocks = std::max(1, std::min(2 * m->num_sms, (d.V + 255) / 256));
@@ -440,7 +436,7 @@ static AttnArgs attn_args(const dspark_model* m, const DraftPlan& p, void* ws, c
     a.q_dtype = io_dtype; a.out_dtype = io_dtype;
     a.kc = static_cast<const char*>(c->k) + layer_bytes * layer;
     a.vc = static_cast<const char*>(c->v) + layer_bytes * layer;
-    a.len = c->len; a.capacity = c->capacity;
+    a.len = c->len; a.capacity = c->capacity; a.batch = c->batch;
     a.part_o = at<float>(ws, p.part_o); a.part_ml = at<float>(ws, p.part_ml);
     a.A = A; a.n_splits = p.attn_splits; a.chunk = p.attn_chunk;
     a.status = m->ws.status;

@@ -61,11 +61,8 @@ extern "C" int dspark_attend_no_alloc(const dspark_model* m, int32_t layer, cons
         DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "cache k / v must be 16-byte aligned");
     const Dims& d = m->d;
 
-    // The same split plan as dspark_attend: context chunks so that A * nH * splits covers the GPU ~2x.
-    int chunk = 64;
-    const int want = std::max(1, (2 * m->num_sms + A * d.nH - 1) / (A * d.nH));
-    if (max_ctx_len > 0) chunk = std::max(64, (max_ctx_len + want - 1) / want);
-    chunk = (chunk + 15) / 16 * 16;
+    // The same split plan as dspark_attend.
+    const int chunk = attention_key_chunk(m, A, max_ctx_len);
     const int splits = max_ctx_len > 0 ? (max_ctx_len + chunk - 1) / chunk : 0;
     const size_t parts = (size_t)A * d.nH * (size_t)(splits + 1) * d.gamma;
     const size_t o_bytes = align_up(parts * d.hd * sizeof(float), 256);
@@ -90,7 +87,7 @@ extern "C" int dspark_attend_no_alloc(const dspark_model* m, int32_t layer, cons
     a.q_dtype = d.dtype; a.out_dtype = d.dtype;
     a.kc = static_cast<const char*>(c->k) + layer_bytes * layer;
     a.vc = static_cast<const char*>(c->v) + layer_bytes * layer;
-    a.len = c->len; a.capacity = c->capacity;
+    a.len = c->len; a.capacity = c->capacity; a.batch = c->batch;
     // Every slot of both arrays is written by the partial pass before the merge
     // reads it, so nothing here needs clearing between calls.
     a.part_o = static_cast<float*>(scratch);

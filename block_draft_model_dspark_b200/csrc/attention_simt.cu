@@ -155,6 +155,8 @@ __global__ void attn_merge_kernel(AttnArgs a, int G, int nH, int hd) {
 
 }  // namespace
 
+cudaError_t launch_attention_merge(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
+
 size_t attn_simt_smem(int G, int hd) {
     return sizeof(float) * ((size_t)G * hd + 2 * (size_t)KT * hd + (size_t)G * KT + 3 * (size_t)G);
 }
@@ -172,6 +174,11 @@ cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a, cuda
     cudaError_t e = cudaGetLastError();
     count_launches(1);
     if (e != cudaSuccess) return e;
+    return launch_attention_merge(m, a, s);
+}
+
+cudaError_t launch_attention_merge(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
+    const Dims& d = m->d;
     attn_merge_kernel<<<a.A * d.nH * d.gamma, d.hd, 0, s>>>(a, d.gamma, d.nH, d.hd);
     count_launches(1);
     return cudaGetLastError();

@@ -8,6 +8,10 @@
 namespace dspark {
 
 cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
+namespace tc {
+bool attention_tc_supported(const dspark_model* m);
+cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
+}
 
 namespace {
 
@@ -36,6 +40,18 @@ double weight_bytes(const dspark_model* m, int64_t N, int64_t K) {
 }  // namespace
 
 bool use_tensor_cores(const dspark_model* m) { return m->d.dtype == DSPARK_DTYPE_BF16 && !m->d.quant; }
+
+int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len) {
+    // context chunks so that A * nKv (tensor cores) or A * nH (CUDA cores) CTAs per split cover the GPU ~2x
+    const Dims& d = m->d;
+    const bool tcore = tc::attention_tc_supported(m);
+    const int per_split = A * (tcore ? d.nKv : d.nH);
+    const int want = std::max(1, (2 * m->num_sms + per_split - 1) / per_split);
+    const int align = tcore ? 64 : 16;
+    int chunk = 64;
+    if (max_ctx_len > 0) chunk = std::max(64, (max_ctx_len + want - 1) / want);
+    return (chunk + align - 1) / align * align;
+}
 
 size_t gemm_part_elems(const dspark_model* m, int M, int N, int K, bool act_pair) {
     if (M <= 0) return 0;
@@ -100,6 +116,7 @@ cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, c
 
 cudaError_t run_attention(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
     KernelTimer t(DSPARK_TIMER_ATTENTION, s, a.kv_bytes, a.flops);
+    if (tc::attention_tc_supported(m)) return tc::launch_attention_tc(m, a, s);
     return launch_attention_simt(m, a, s);
 }
 

@@ -19,6 +19,8 @@ cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U,
 cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, const RowsPlan& rp, const KvDest& dst,
                               float* raw, cudaStream_t s);
 cudaError_t run_attention(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
+// Context keys per split of the attention for A rows of at most max_ctx_len keys.
+int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len);
 
 int gemm_prepare_model(dspark_model* m);
 void gemm_release_model(dspark_model* m);

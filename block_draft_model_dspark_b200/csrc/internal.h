@@ -174,7 +174,7 @@ struct AttnArgs {
     const void* q;  const void* kb; const void* vb;  // [A, G, nH, hd] / [A, G, nKv, hd]
     int q_dtype, out_dtype;                          // DSPARK_DTYPE_* of q and out (kb, vb, cache: model dtype)
     const void* kc; const void* vc;                  // cache of this layer: [batch, cap, nKv, hd]
-    const int32_t* len; int capacity;
+    const int32_t* len; int capacity, batch;         // cache lengths [batch], capacity, batch rows
     void* out;                                       // [A, G, nH, hd]
     bf16* out_hi; bf16* out_lo;                      // optional bf16 pair of out (fp32 out only)
     float* part_o; float* part_ml;                   // workspace
