@@ -322,11 +322,10 @@ def run_dspark(args, wl):
     h2d = h_rows.numel() * h_rows.element_size() + h_anc.numel() * 4 + h_bpos.numel() * 4 + crop_host.numel() * 4
     d2h = h_tok.numel() * 4 + h_len.numel() * 4 + h_conf.numel() * 4
 
-    # max over ranks
-    t = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, e2e_ms = t.tolist()
+    # the job's time is its slowest rank's
+    from block_draft_model_dspark_b200.sharding import max_over_ranks
+    ms_total = max_over_ranks(ms_total)
+    e2e_ms = max_over_ranks(e2e_ms)
 
     if rank == 0:
         tok_per_step = A * G * world

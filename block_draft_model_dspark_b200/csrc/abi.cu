@@ -46,7 +46,8 @@ int validate_config(const dspark_config* c, std::string* why) {
     if (c->mask_token_id < 0 || c->mask_token_id >= c->vocab_size) return fail(DSPARK_ERR_INVALID_ARGUMENT, "mask_token_id outside [0, vocab_size)");
     if (c->block_size < 1 || c->block_size > 32 || c->block_size * hd > 4096)
         return fail(DSPARK_ERR_UNSUPPORTED, "block_size must be in [1, 32] with block_size * head_dim <= 4096");
-    if (c->markov_rank < 0 || c->markov_rank > 256) return fail(DSPARK_ERR_UNSUPPORTED, "markov_rank must be in [0, 256]");
+    if (c->markov_rank != 0 && !(c->markov_rank >= 8 && c->markov_rank <= 256 && (c->markov_rank & (c->markov_rank - 1)) == 0))
+        return fail(DSPARK_ERR_UNSUPPORTED, "markov_rank must be 0 or a power of two in [8, 256]");
     if (c->quant_bits == 4 && c->markov_rank % 64) return fail(DSPARK_ERR_UNSUPPORTED, "quantized markov_w2 needs markov_rank % 64 == 0");
     if (c->enable_confidence_head && c->confidence_head_with_markov && c->markov_rank <= 0)
         return fail(DSPARK_ERR_INVALID_ARGUMENT, "confidence_head_with_markov requires markov_rank > 0");
@@ -163,7 +164,7 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     const int chunk = attention_key_chunk(m, A, maxL);
     p.attn_chunk = chunk;
     p.attn_splits = maxL > 0 ? (maxL + chunk - 1) / chunk : 0;
-    p.walk_blocks = std::max(1, std::min(2 * m->num_sms, (d.V + 255) / 256));
+    p.walk_blocks = walk_vocab_blocks(m->num_sms, d.V, d.r);
     Carve c;
     const size_t es = esize(d.dtype);
     p.h = c.take((size_t)p.M * d.H * 4);

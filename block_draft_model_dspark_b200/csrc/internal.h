@@ -194,6 +194,8 @@ struct WalkArgs {
     int32_t* status;
 };
 cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s);
+// Vocabulary slices (grid.x) of a walk step.
+int walk_vocab_blocks(int num_sms, int V, int r);
 cudaError_t launch_walk_init(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V,
                              int32_t* status, cudaStream_t s);
 // Confidence + lengths (hf = the final-normed hidden, fp32 [M, H]).

@@ -3,11 +3,14 @@
 //   bias_b[v] = markov_w2[v] . markov_w1[prev_b]        (rank-r GEMV over the vocabulary)
 //   tok_{b,k} = argmax_v (U[b,k,v] + bias_b[v])          (lowest index on ties)
 //   prev_b    = tok_{b,k}
-// The sum is taken in fp32. One launch per step: every CTA scans a slice of
-// the vocabulary for all rows and writes its (value, index) candidates; the
-// last CTA to finish (a ticket counter, not a value atomic) reduces the
-// candidates in CTA order and commits the step's tokens, so the result does
-// not depend on scheduling.
+// The sum is taken in fp32. One launch per step. A CTA owns a slice of the
+// vocabulary and up to kRowsPerCta batch rows: r/8 lanes share one W2 row
+// (each lane holds 8 of its values in registers, loaded once with 16-byte
+// coalesced loads) and apply it to every row's markov_w1[prev] (from shared
+// memory), so W2 streams once per step per kRowsPerCta rows. Each CTA writes
+// its (value, index) candidates; the last CTA to finish (a ticket counter,
+// not a value atomic) reduces them in CTA order and commits the step's
+// tokens, so the result does not depend on scheduling.
 #include <math.h>
 
 #include "internal.h"
@@ -17,14 +20,9 @@ namespace dspark {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kRowsPerCta = 8;       // batch rows per CTA (grid.y covers the rest)
 constexpr int kMaxRank = 256;
-
-__device__ __forceinline__ float w2_at(const MatRef& W, int dtype, int group, int64_t v, int j) {
-    if (!W.quant) return load_any(W.w, v * W.k + j, dtype);
-    const uint32_t w = static_cast<const uint32_t*>(W.w)[v * (W.k / 8) + j / 8];
-    const int64_t g = v * (W.k / group) + j / group;
-    return fmaf(__bfloat162float(W.scales[g]), (float)((w >> (4 * (j % 8))) & 0xFu), __bfloat162float(W.biases[g]));
-}
 
 __global__ void walk_init_kernel(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V,
                                  int32_t* status) {
@@ -40,57 +38,106 @@ __global__ void walk_init_kernel(const int32_t* anchors, int32_t* prev, uint32_t
     }
 }
 
+// Eight consecutive markov_w2 values W2[v, c8 .. c8+7] as fp32.
+__device__ __forceinline__ void load_w2_8(const MatRef& W, int dtype, int group, int64_t v, int c8, int r,
+                                          float w[8]) {
+    if (W.quant) {
+        dequant8(static_cast<const uint32_t*>(W.w), W.scales, W.biases, v, c8, r, group, w);
+    } else if (dtype == DSPARK_DTYPE_F32) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(W.w) + v * r + c8);
+        const float4 a = p[0], b = p[1];
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    } else {
+        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const bf16*>(W.w) + v * r + c8);
+        const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { w[2 * j] = __uint_as_float(q[j] << 16); w[2 * j + 1] = __uint_as_float(q[j] & 0xffff0000u); }
+    }
+}
+
+// grid (vocabulary slices, ceil(A / kRowsPerCta)).
 __global__ void __launch_bounds__(kThreads)
-walk_step_kernel(WalkArgs a, MatRef W2, const void* __restrict__ w1, int dtype, int group, int G, int V, int r) {
-    __shared__ float e[kMaxRank];
-    __shared__ float rv[32];
-    __shared__ int ri[32];
+walk_step_kernel(WalkArgs a, MatRef W2, const void* __restrict__ w1, int dtype, int group, int G, int V, int r,
+                 int per) {
+    __shared__ float e[kRowsPerCta][kMaxRank];
+    __shared__ float rv[kWarps][kRowsPerCta];
+    __shared__ int ri[kWarps][kRowsPerCta];
     __shared__ bool last;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int per = (V + gridDim.x - 1) / gridDim.x;
+    const int b0 = blockIdx.y * kRowsPerCta;
+    const int nb = min(kRowsPerCta, a.A - b0);
     const int v0 = blockIdx.x * per, v1 = min(V, v0 + per);
 
-    for (int b = 0; b < a.A; ++b) {
-        const int pb = a.prev[b];
-        for (int j = tid; j < r; j += kThreads) e[j] = load_any(w1, (int64_t)pb * r + j, dtype);
-        __syncthreads();
-        float best = -INFINITY;
-        int bi = 0x7fffffff;
-        const float* Urow = a.U + ((int64_t)b * G + a.step) * V;
-        for (int v = v0 + tid; v < v1; v += kThreads) {
-            float s = Urow[v];
-            float bias = 0.f;
-            for (int j = 0; j < r; ++j) bias = fmaf(e[j], w2_at(W2, dtype, group, v, j), bias);
-            s += bias;
-            argmax_merge(best, bi, s, v);
+    for (int i = tid; i < nb * r; i += kThreads) {
+        const int bb = i / r, j = i % r;
+        e[bb][j] = load_any(w1, (int64_t)a.prev[b0 + bb] * r + j, dtype);
+    }
+    __syncthreads();
+
+    // lanes per W2 row (r/8, a power of two <= 32) and rows per warp step
+    const int lpr = r > 0 ? r / 8 : 1;
+    const int rpw = 32 / lpr;
+    const int c8 = (lane % lpr) * 8;
+    const bool leader = (lane % lpr) == 0;
+    float best[kRowsPerCta];
+    int bidx[kRowsPerCta];
+#pragma unroll
+    for (int bb = 0; bb < kRowsPerCta; ++bb) { best[bb] = -INFINITY; bidx[bb] = 0x7fffffff; }
+
+    for (int vbase = v0 + wid * rpw; vbase < v1; vbase += kWarps * rpw) {     // warp-uniform
+        const int v = vbase + lane / lpr;
+        const bool live = v < v1;
+        float w[8];
+        if (r > 0 && live) load_w2_8(W2, dtype, group, v, c8, r, w);
+        else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[j] = 0.f;
         }
-        warp_argmax(best, bi);
-        if (lane == 0) { rv[wid] = best; ri[wid] = bi; }
-        __syncthreads();
-        if (wid == 0) {
-            best = lane < kThreads / 32 ? rv[lane] : -INFINITY;
-            bi = lane < kThreads / 32 ? ri[lane] : 0x7fffffff;
-            warp_argmax(best, bi);
-            if (lane == 0) {
-                a.part_val[(int64_t)blockIdx.x * a.A + b] = best;
-                a.part_idx[(int64_t)blockIdx.x * a.A + b] = bi;
+#pragma unroll
+        for (int bb = 0; bb < kRowsPerCta; ++bb) {
+            if (bb >= nb) break;
+            float part = 0.f;
+            if (r > 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) part = fmaf(w[j], e[bb][c8 + j], part);
+                for (int o = lpr / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            }
+            if (leader && live) {
+                const float s = a.U[((int64_t)(b0 + bb) * G + a.step) * V + v] + part;
+                argmax_merge(best[bb], bidx[bb], s, v);
             }
         }
-        __syncthreads();
+    }
+#pragma unroll
+    for (int bb = 0; bb < kRowsPerCta; ++bb) {
+        if (bb >= nb) break;
+        float bv = best[bb];
+        int bi = bidx[bb];
+        warp_argmax(bv, bi);
+        if (lane == 0) { rv[wid][bb] = bv; ri[wid][bb] = bi; }
+    }
+    __syncthreads();
+    if (tid < nb) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int w = 0; w < kWarps; ++w) argmax_merge(bv, bi, rv[w][tid], ri[w][tid]);
+        a.part_val[(int64_t)blockIdx.x * a.A + b0 + tid] = bv;
+        a.part_idx[(int64_t)blockIdx.x * a.A + b0 + tid] = bi;
     }
 
     // ticket: the last CTA reduces all candidates in CTA order
     __threadfence();
-    if (tid == 0) last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (tid == 0) last = atomicAdd(a.ticket, 1u) == gridDim.x * gridDim.y - 1;
     __syncthreads();
     if (!last) return;
     __threadfence();
-    for (int b = wid; b < a.A; b += kThreads / 32) {
-        float best = -INFINITY;
+    for (int b = wid; b < a.A; b += kWarps) {
+        float bv = -INFINITY;
         int bi = 0x7fffffff;
         for (int c = lane; c < (int)gridDim.x; c += 32)
-            argmax_merge(best, bi, a.part_val[(int64_t)c * a.A + b], a.part_idx[(int64_t)c * a.A + b]);
-        warp_argmax(best, bi);
+            argmax_merge(bv, bi, a.part_val[(int64_t)c * a.A + b], a.part_idx[(int64_t)c * a.A + b]);
+        warp_argmax(bv, bi);
         if (lane == 0) {
             if (bi < 0 || bi >= V) {            // only if a row was all NaN
                 atomicOr(a.status, DSPARK_DEV_BAD_TOKEN);
@@ -105,6 +152,14 @@ walk_step_kernel(WalkArgs a, MatRef W2, const void* __restrict__ w1, int dtype, 
 
 }  // namespace
 
+int walk_vocab_blocks(int num_sms, int V, int r) {
+    const int rpw = r > 0 ? 32 / (r / 8) : 32;
+    const int rows_per_iter = kWarps * rpw;
+    const int want = 2 * num_sms;
+    const int cap = (V + rows_per_iter * 4 - 1) / (rows_per_iter * 4);   // >= 4 warp steps per CTA
+    return cap < 1 ? 1 : (want < cap ? want : cap);
+}
+
 cudaError_t launch_walk_init(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V, int32_t* status,
                              cudaStream_t s) {
     walk_init_kernel<<<(A + 127) / 128, 128, 0, s>>>(anchors, prev, ticket, A, V, status);
@@ -114,7 +169,9 @@ cudaError_t launch_walk_init(const int32_t* anchors, int32_t* prev, uint32_t* ti
 
 cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s) {
     const Dims& d = m->d;
-    walk_step_kernel<<<a.nblk, kThreads, 0, s>>>(a, m->w2, m->w1, d.dtype, d.group, d.gamma, d.V, d.r);
+    const int per = (d.V + a.nblk - 1) / a.nblk;
+    dim3 grid(a.nblk, (a.A + kRowsPerCta - 1) / kRowsPerCta);
+    walk_step_kernel<<<grid, kThreads, 0, s>>>(a, m->w2, m->w1, d.dtype, d.group, d.gamma, d.V, d.r, per);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -63,13 +63,13 @@ typedef struct dspark_config {
     int32_t hidden_size;
     int32_t num_hidden_layers;
     int32_t num_attention_heads;
-    int32_t global_head_dim;               /* even, <= 256, multiple of 32 */
+    int32_t global_head_dim;               /* 64, 128, 192 or 256 */
     int32_t num_global_key_value_heads;    /* divides num_attention_heads */
     int32_t intermediate_size;
     int32_t vocab_size;
     int32_t block_size;                    /* gamma */
     int32_t mask_token_id;
-    int32_t markov_rank;                   /* 0 = no Markov head (plain argmax) */
+    int32_t markov_rank;                   /* 0 = no Markov head (plain argmax); else a power of two in [8, 256] */
     int32_t attention_k_eq_v;              /* must be 1 */
     int32_t markov_head_vanilla;           /* must be 1 when markov_rank > 0 */
     int32_t hidden_activation_gelu_tanh;   /* must be 1 */
