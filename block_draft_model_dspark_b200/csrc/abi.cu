@@ -148,7 +148,7 @@ struct DraftPlan {
     int M, attn_splits, attn_chunk, walk_blocks;
     bool pairs;   // GEMM inputs also kept as bf16 (hi, lo) pairs for the tensor-core GEMMs
     size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx;
-    size_t x_hi, x_lo, ao_hi, ao_lo, act_hi, act_lo, total;
+    size_t x_hi, x_lo, ao_hi, ao_lo, act_hi, act_lo, conf, total;
 };
 
 DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
@@ -190,6 +190,7 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.ao_lo = c.take((size_t)p.M * d.nH * d.hd * pb);
     p.act_hi = c.take((size_t)p.M * d.I * pb);
     p.act_lo = c.take((size_t)p.M * d.I * pb);
+    p.conf = c.take((size_t)p.M * 4);
     p.total = c.off;
     return p;
 }
@@ -529,7 +530,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
             e = launch_walk_step(m, wa, s);
         }
     }
-    if (e == cudaSuccess) e = launch_confidence(m, x.f32, anchors, tokens, A, conf, lengths, s);
+    if (e == cudaSuccess) e = launch_confidence(m, x.f32, anchors, tokens, A, conf ? conf : at<float>(ws, p.conf), lengths, s);
     if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("draft round launch: ") + cudaGetErrorString(e));
     return DSPARK_OK;
 }

@@ -133,15 +133,18 @@ __global__ void attn_merge_kernel(AttnArgs a, int G, int nH, int hd) {
     const int d = threadIdx.x;
     const int S1 = a.n_splits + 1;
     float M = -INFINITY;
+#pragma unroll 8
     for (int s = 0; s < S1; ++s) M = fmaxf(M, a.part_ml[(((int64_t)bh * S1 + s) * G + i) * 2]);
     float num = 0.f, den = 0.f;
+#pragma unroll 8
     for (int s = 0; s < S1; ++s) {
         const int64_t base = ((int64_t)bh * S1 + s) * G + i;
         const float m = a.part_ml[base * 2];
-        if (m == -INFINITY) continue;
-        const float w = expf(m - M);
-        den += w * a.part_ml[base * 2 + 1];
-        num += w * a.part_o[base * hd + d];
+        const float l = a.part_ml[base * 2 + 1];
+        const float o = m == -INFINITY ? 0.f : a.part_o[base * hd + d];
+        const float w = m == -INFINITY ? 0.f : expf(m - M);
+        den += w * l;
+        num += w * o;
     }
     const int64_t o = (((int64_t)b * G + i) * nH + h) * hd + d;
     const float v = num / den;

@@ -48,8 +48,11 @@ int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len) {
     const int per_split = A * (tcore ? d.nKv : d.nH);
     const int want = std::max(1, (2 * m->num_sms + per_split - 1) / per_split);
     const int align = tcore ? 64 : 16;
-    int chunk = 64;
-    if (max_ctx_len > 0) chunk = std::max(64, (max_ctx_len + want - 1) / want);
+    // tensor cores: >= 4 key tiles per split, so a split's partial output (q rows x hd fp32)
+    // stays below half of the K/V bytes it reads
+    const int min_chunk = tcore ? 256 : 64;
+    int chunk = min_chunk;
+    if (max_ctx_len > 0) chunk = std::max(min_chunk, (max_ctx_len + want - 1) / want);
     return (chunk + align - 1) / align * align;
 }
 

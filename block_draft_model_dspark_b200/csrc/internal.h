@@ -51,6 +51,8 @@ struct ModelWs {
     bf16* wk_all_s = nullptr; bf16* wk_all_b = nullptr;
 };
 
+constexpr int kMaxPartials = 12;   // partial tiles a consumer loads at once
+
 // A GEMM result as its consumers read it: out[m][n] is the sum of the GEMM's
 // partial tiles. mode 0: CUDA-core split-K partials [S][M][ld]; mode 1: the
 // tcgen05 GEMM's tiles [tile][P][BN][128] (stream-K: the tile's partials
@@ -72,7 +74,12 @@ struct PartView {
         int cnt = 1;
         if (plan.streamk) cnt = plan.cta_of(t * plan.kb + plan.kb - 1) - plan.cta_of(t * plan.kb) + 1;
         const float* q = p + (((int64_t)t * plan.P) * BN + ml) * 128 + nl;
-        for (int s = 0; s < cnt; ++s) v += q[(int64_t)s * BN * 128];
+        float x[kMaxPartials];
+#pragma unroll
+        for (int s = 0; s < kMaxPartials; ++s) x[s] = s < cnt ? q[(int64_t)s * BN * 128] : 0.f;   // loads in flight together
+#pragma unroll
+        for (int s = 0; s < kMaxPartials; ++s) v += x[s];                                        // summed in CTA order
+        for (int s = kMaxPartials; s < cnt; ++s) v += q[(int64_t)s * BN * 128];
         return v;
     }
 };

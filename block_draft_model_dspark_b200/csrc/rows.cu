@@ -194,37 +194,46 @@ __global__ void gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
 }
 
 // ------------------------------------------------------------------ confidence + truncation
-// grid A, block 256: c[b,k] = sigmoid(proj . [hf(b,k) ; w1[prev]] + bias); lengths[b].
+// grid A * gamma, block 256: c[b,k] = sigmoid(proj . [hf(b,k) ; w1[prev_k]] + bias),
+// prev_0 = anchor, prev_k = tokens[b, k-1].
 __global__ void confidence_kernel(const float* __restrict__ hf32, MatRef P, int dtype, int group,
                                   const void* __restrict__ w1, const void* __restrict__ bias,
                                   const int32_t* __restrict__ anchors, const int32_t* __restrict__ tokens,
-                                  int gamma, int H, int r, int with_markov, int V, float thr, int has_head,
-                                  float* __restrict__ conf, int32_t* __restrict__ lengths) {
+                                  int gamma, int H, int r, int with_markov, int V, float* __restrict__ conf) {
     __shared__ float red[32];
-    const int b = blockIdx.x;
-    int len = gamma;
-    const float bz = has_head ? load_any(bias, 0, dtype) : 0.f;
-    for (int k = 0; has_head && k < gamma; ++k) {
-        int prev = k == 0 ? anchors[b] : tokens[b * gamma + k - 1];
-        prev = min(max(prev, 0), V - 1);
-        const int64_t m = (int64_t)b * gamma + k;
-        float z = 0.f;
-        for (int j = threadIdx.x; j < H; j += blockDim.x) z += hf32[m * H + j] * mat_at(P, dtype, group, 0, j);
-        if (with_markov)
-            for (int j = threadIdx.x; j < r; j += blockDim.x)
-                z += load_any(w1, (int64_t)prev * r + j, dtype) * mat_at(P, dtype, group, 0, H + j);
-        z = block_sum(z, red) + bz;
-        const float c = 1.f / (1.f + expf(-z));
-        if (threadIdx.x == 0) {
-            if (conf) conf[m] = c;
-            if (thr > 0.f && c < thr && len == gamma) len = k;
-        }
-    }
-    if (threadIdx.x == 0 && lengths) lengths[b] = len;
+    const int m = blockIdx.x;
+    const int b = m / gamma, k = m % gamma;
+    int prev = k == 0 ? anchors[b] : tokens[b * gamma + k - 1];
+    prev = min(max(prev, 0), V - 1);
+    float z = 0.f;
+    for (int j = threadIdx.x; j < H; j += blockDim.x) z += hf32[(int64_t)m * H + j] * mat_at(P, dtype, group, 0, j);
+    if (with_markov)
+        for (int j = threadIdx.x; j < r; j += blockDim.x)
+            z += load_any(w1, (int64_t)prev * r + j, dtype) * mat_at(P, dtype, group, 0, H + j);
+    z = block_sum(z, red) + load_any(bias, 0, dtype);
+    if (threadIdx.x == 0) conf[m] = 1.f / (1.f + expf(-z));
 }
 
+// lengths[b] = first k with conf < thr (thr > 0), else gamma (no head: gamma).
+__global__ void lengths_kernel(const float* __restrict__ conf, int A, int gamma, float thr, int has_head,
+                               int32_t* __restrict__ lengths) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= A) return;
+    int len = gamma;
+    if (has_head && thr > 0.f)
+        for (int k = 0; k < gamma; ++k)
+            if (conf[(int64_t)b * gamma + k] < thr) { len = k; break; }
+    lengths[b] = len;
+}
+
+// Threads of a full-row kernel: enough that each holds at most kMaxPer
+// columns, about 8 columns per thread, and at most 512 (the kernels use up
+// to ~80 registers a thread; 512 x 80 fits a block's register file).
 int row_threads(int H) {
-    int t = (H + kMaxPer - 1) / kMaxPer;
+    int t = (H + 7) / 8;
+    const int need = (H + kMaxPer - 1) / kMaxPer;
+    if (t > 512) t = 512;
+    if (t < need) t = need;
     t = (t + 31) / 32 * 32;
     return t < 32 ? 32 : t;
 }
@@ -307,9 +316,15 @@ cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const PartVie
 cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const int32_t* anchors, const int32_t* tokens,
                               int A, float* conf, int32_t* lengths, cudaStream_t s) {
     const Dims& d = m->d;
-    confidence_kernel<<<A, 256, 0, s>>>(hf32, m->conf_proj, d.dtype, d.group, m->w1, m->conf_bias, anchors, tokens,
-                                        d.gamma, d.H, d.r, d.conf_markov ? 1 : 0, d.V, d.conf_thr,
-                                        d.conf_head ? 1 : 0, d.conf_head ? conf : nullptr, lengths);
+    if (d.conf_head) {
+        confidence_kernel<<<A * d.gamma, 256, 0, s>>>(hf32, m->conf_proj, d.dtype, d.group, m->w1, m->conf_bias,
+                                                      anchors, tokens, d.gamma, d.H, d.r, d.conf_markov ? 1 : 0, d.V,
+                                                      conf);
+        count_launches(1);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    lengths_kernel<<<(A + 127) / 128, 128, 0, s>>>(conf, A, d.gamma, d.conf_thr, d.conf_head ? 1 : 0, lengths);
     count_launches(1);
     return cudaGetLastError();
 }

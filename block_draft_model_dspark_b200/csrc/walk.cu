@@ -84,27 +84,36 @@ walk_step_kernel(WalkArgs a, MatRef W2, const void* __restrict__ w1, int dtype, 
 #pragma unroll
     for (int bb = 0; bb < kRowsPerCta; ++bb) { best[bb] = -INFINITY; bidx[bb] = 0x7fffffff; }
 
-    for (int vbase = v0 + wid * rpw; vbase < v1; vbase += kWarps * rpw) {     // warp-uniform
-        const int v = vbase + lane / lpr;
-        const bool live = v < v1;
-        float w[8];
-        if (r > 0 && live) load_w2_8(W2, dtype, group, v, c8, r, w);
-        else {
+    constexpr int U = 4;                                   // row groups in flight per lane
+    const int stride = kWarps * rpw;
+    for (int vbase = v0 + wid * rpw; vbase < v1; vbase += U * stride) {     // warp-uniform
+        int vv[U];
+        float w[U][8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) w[j] = 0.f;
+        for (int u = 0; u < U; ++u) {
+            vv[u] = vbase + u * stride + lane / lpr;
+            if (r > 0 && vv[u] < v1) load_w2_8(W2, dtype, group, vv[u], c8, r, w[u]);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[u][j] = 0.f;
+            }
         }
 #pragma unroll
         for (int bb = 0; bb < kRowsPerCta; ++bb) {
             if (bb >= nb) break;
-            float part = 0.f;
-            if (r > 0) {
+            const float* Urow = a.U + ((int64_t)(b0 + bb) * G + a.step) * V;
+            float uv[U];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) part = fmaf(w[j], e[bb][c8 + j], part);
-                for (int o = lpr / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            }
-            if (leader && live) {
-                const float s = a.U[((int64_t)(b0 + bb) * G + a.step) * V + v] + part;
-                argmax_merge(best[bb], bidx[bb], s, v);
+            for (int u = 0; u < U; ++u) uv[u] = (leader && vv[u] < v1) ? Urow[vv[u]] : 0.f;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                float part = 0.f;
+                if (r > 0) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) part = fmaf(w[u][j], e[bb][c8 + j], part);
+                    for (int o = lpr / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                }
+                if (leader && vv[u] < v1) argmax_merge(best[bb], bidx[bb], uv[u] + part, vv[u]);
             }
         }
     }
