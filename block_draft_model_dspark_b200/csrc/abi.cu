@@ -148,7 +148,7 @@ struct DraftPlan {
     int M, attn_splits, attn_chunk, walk_blocks;
     bool pairs;   // GEMM inputs also kept as bf16 (hi, lo) pairs for the tensor-core GEMMs
     size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx;
-    size_t x_hi, x_lo, ao_hi, ao_lo, act_hi, act_lo, conf, total;
+    size_t x_hi, x_lo, ao_hi, ao_lo, act_hi, act_lo, conf, gscr, gscr_bytes, total;
 };
 
 DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
@@ -157,14 +157,17 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.M = A * d.gamma;
     const int Nqk = (d.nH + d.nKv) * d.hd;
     p.pairs = use_tensor_cores(m);
-    const size_t part_elems = std::max({gemm_part_elems(m, p.M, Nqk, d.H, p.pairs),
-                                        gemm_part_elems(m, p.M, d.H, d.nH * d.hd, p.pairs),
-                                        gemm_part_elems(m, p.M, 2 * d.I, d.H, p.pairs),
-                                        gemm_part_elems(m, p.M, d.H, d.I, p.pairs)});
+    const size_t part_elems = std::max({gemm_out_elems(m, p.M, Nqk, d.H), gemm_out_elems(m, p.M, d.H, d.nH * d.hd),
+                                        gemm_out_elems(m, p.M, 2 * d.I, d.H), gemm_out_elems(m, p.M, d.H, d.I)});
+    p.gscr_bytes = std::max({gemm_scratch_bytes(m, p.M, Nqk, d.H, p.pairs),
+                             gemm_scratch_bytes(m, p.M, d.H, d.nH * d.hd, p.pairs),
+                             gemm_scratch_bytes(m, p.M, 2 * d.I, d.H, p.pairs),
+                             gemm_scratch_bytes(m, p.M, d.H, d.I, p.pairs)});
     const int chunk = attention_key_chunk(m, A, maxL);
     p.attn_chunk = chunk;
     p.attn_splits = maxL > 0 ? (maxL + chunk - 1) / chunk : 0;
-    p.walk_blocks = walk_vocab_blocks(m->num_sms, d.V, d.r);
+    p.walk_blocks = walk_persistent_supported(m, A) ? walk_persistent_blocks(m)
+                                                    : walk_vocab_blocks(m->num_sms, d.V, d.r, d.dtype, d.quant);
     Carve c;
     const size_t es = esize(d.dtype);
     p.h = c.take((size_t)p.M * d.H * 4);
@@ -181,8 +184,8 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.part_ml = c.take((size_t)A * d.nH * S1 * d.gamma * 2 * 4);
     p.prev = c.take((size_t)A * 4);
     p.ticket = c.take(256);
-    p.walk_val = c.take((size_t)p.walk_blocks * A * 4);
-    p.walk_idx = c.take((size_t)p.walk_blocks * A * 4);
+    p.walk_val = c.take((size_t)2 * p.walk_blocks * A * 4);     // two step-parity buffers (persistent walk)
+    p.walk_idx = c.take((size_t)2 * p.walk_blocks * A * 4);
     const size_t pb = p.pairs ? 2 : 0;
     p.x_hi = c.take((size_t)p.M * d.H * pb);
     p.x_lo = c.take((size_t)p.M * d.H * pb);
@@ -191,6 +194,7 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.act_hi = c.take((size_t)p.M * d.I * pb);
     p.act_lo = c.take((size_t)p.M * d.I * pb);
     p.conf = c.take((size_t)p.M * 4);
+    p.gscr = c.take(p.gscr_bytes);
     p.total = c.off;
     return p;
 }
@@ -199,7 +203,7 @@ constexpr int64_t kProjectChunkRows = 16384;
 
 struct ProjectPlan {
     int64_t chunk_rows;
-    size_t nvalid, raw, total;
+    size_t nvalid, raw, gscr, gscr_bytes, total;
 };
 ProjectPlan plan_project(const dspark_model* m, int64_t rows) {
     const Dims& d = m->d;
@@ -207,11 +211,16 @@ ProjectPlan plan_project(const dspark_model* m, int64_t rows) {
     rows = std::max<int64_t>(rows, 1);
     p.chunk_rows = std::min<int64_t>(rows, kProjectChunkRows);
     const int N = d.Lyr * d.nKv * d.hd;
-    size_t raw = gemm_part_elems(m, (int)p.chunk_rows, N, d.H, false);
-    if (rows % p.chunk_rows) raw = std::max(raw, gemm_part_elems(m, (int)(rows % p.chunk_rows), N, d.H, false));
+    size_t raw = gemm_out_elems(m, (int)p.chunk_rows, N, d.H);
+    p.gscr_bytes = gemm_scratch_bytes(m, (int)p.chunk_rows, N, d.H, false);
+    if (rows % p.chunk_rows) {
+        raw = std::max(raw, gemm_out_elems(m, (int)(rows % p.chunk_rows), N, d.H));
+        p.gscr_bytes = std::max(p.gscr_bytes, gemm_scratch_bytes(m, (int)(rows % p.chunk_rows), N, d.H, false));
+    }
     Carve c;
     p.nvalid = c.take(4096 * 4);
     p.raw = c.take(raw * 4);
+    p.gscr = c.take(p.gscr_bytes);
     p.total = c.off;
     return p;
 }
@@ -224,13 +233,16 @@ int project_rows(const dspark_model* m, const void* hidden, int B, int Lrows, co
     const Dims& d = m->d;
     const int64_t rows = (int64_t)B * Lrows;
     const size_t es = esize(d.dtype);
+    const GemmScratch sc = gemm_scratch_at(at<void>(ws, pp.gscr), pp.gscr_bytes);
+    cudaError_t e0 = gemm_scratch_reset(sc, pp.gscr_bytes, s);
+    if (e0 != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("GEMM scratch reset: ") + cudaGetErrorString(e0));
     for (int64_t r0 = 0; r0 < rows; r0 += pp.chunk_rows) {
         const int nr = (int)std::min<int64_t>(pp.chunk_rows, rows - r0);
         RowsPlan rp{};
         rp.B = B; rp.Lrows = Lrows; rp.row0 = (int)r0; rp.nrows = nr; rp.n_valid = n_valid;
         rp.dst_row0 = dst_row0; rp.pos0 = pos0; rp.static_pos = static_pos;
         const void* X = static_cast<const char*>(hidden) + (size_t)r0 * d.H * es;
-        cudaError_t e = run_kv_projection(m, X, nr, rp, dst, at<float>(ws, pp.raw), s);
+        cudaError_t e = run_kv_projection(m, X, nr, rp, dst, at<float>(ws, pp.raw), sc, s);
         if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("context K/V projection launch: ") + cudaGetErrorString(e));
     }
     return DSPARK_OK;
@@ -498,36 +510,45 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     }
     const int Nqk = (d.nH + d.nKv) * d.hd;
     PartView pv;
-    cudaError_t e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
+    const GemmScratch sc = gemm_scratch_at(at<void>(ws, p.gscr), p.gscr_bytes);
+    cudaError_t e = gemm_scratch_reset(sc, p.gscr_bytes, s);
+    // the persistent walk's grid-barrier counter
+    if (e == cudaSuccess) e = cudaMemsetAsync(at<uint32_t>(ws, p.ticket), 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
     for (int l = 0; l < d.Lyr && e == cudaSuccess; ++l) {
         const LayerRef& L = m->layers[l];
-        e = run_gemm(m, x, L.qk, M, Nqk, d.H, part, &pv, s);
+        e = run_gemm(m, x, L.qk, M, Nqk, d.H, part, sc, &pv, s);
         if (e == cudaSuccess) e = launch_qk_epilogue(m, l, pv, A, block_pos, q, kb, vb, s);
         if (e == cudaSuccess) {
             AttnArgs a = attn_args(m, p, ws, cache, l, A, q, kb, vb, ao.f32, DSPARK_DTYPE_F32);
             a.out_hi = ao.hi; a.out_lo = ao.lo;
             e = run_attention(m, a, s);
         }
-        if (e == cudaSuccess) e = run_gemm(m, ao, L.o, M, d.H, d.nH * d.hd, part, &pv, s);
+        if (e == cudaSuccess) e = run_gemm(m, ao, L.o, M, d.H, d.nH * d.hd, part, sc, &pv, s);
         if (e == cudaSuccess) e = launch_o_epilogue(m, l, pv, M, h, x, s);
-        if (e == cudaSuccess) e = run_gemm(m, x, L.gu, M, 2 * d.I, d.H, part, &pv, s);
+        if (e == cudaSuccess) e = run_gemm(m, x, L.gu, M, 2 * d.I, d.H, part, sc, &pv, s);
         if (e == cudaSuccess) e = launch_gu_epilogue(m, pv, M, act, s);
-        if (e == cudaSuccess) e = run_gemm(m, act, L.down, M, d.H, d.I, part, &pv, s);
+        if (e == cudaSuccess) e = run_gemm(m, act, L.down, M, d.H, d.I, part, sc, &pv, s);
         if (e == cudaSuccess) e = launch_down_epilogue(m, l, pv, M, h, x, s);
     }
-    if (e == cudaSuccess) e = run_lm_head(m, x, M, U, part, s);
+    if (e == cudaSuccess) e = run_lm_head(m, x, M, U, s);
     if (e == cudaSuccess) {
         WalkArgs wa{};
         wa.U = U; wa.tokens = tokens; wa.prev = at<int32_t>(ws, p.prev);
         wa.part_val = at<float>(ws, p.walk_val); wa.part_idx = at<int32_t>(ws, p.walk_idx);
         wa.ticket = at<uint32_t>(ws, p.ticket); wa.A = A; wa.nblk = p.walk_blocks; wa.status = m->ws.status;
-        e = launch_walk_init(anchors, wa.prev, wa.ticket, A, d.V, m->ws.status, s);
         const double w2b = d.r > 0 ? (d.quant ? (double)d.V * d.r * 0.5 + (double)d.V * (d.r / d.group) * 4.0
                                               : (double)d.V * d.r * esize(d.dtype)) : 0.0;
-        for (int k = 0; k < d.gamma && e == cudaSuccess; ++k) {
-            wa.step = k;
-            KernelTimer t(DSPARK_TIMER_WALK, s, w2b + 4.0 * A * d.V, 2.0 * A * (double)d.V * d.r);
-            e = launch_walk_step(m, wa, s);
+        if (walk_persistent_supported(m, A)) {
+            KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
+            e = launch_walk_persistent(m, U, anchors, tokens, wa.part_val, wa.part_idx, wa.ticket, A, s);
+        } else {
+            e = launch_walk_init(anchors, wa.prev, wa.ticket, A, d.V, m->ws.status, s);
+            for (int k = 0; k < d.gamma && e == cudaSuccess; ++k) {
+                wa.step = k;
+                KernelTimer t(DSPARK_TIMER_WALK, s, w2b + 4.0 * A * d.V, 2.0 * A * (double)d.V * d.r);
+                e = launch_walk_step(m, wa, s);
+            }
         }
     }
     if (e == cudaSuccess) e = launch_confidence(m, x.f32, anchors, tokens, A, conf ? conf : at<float>(ws, p.conf), lengths, s);

@@ -31,6 +31,8 @@ attn_partial_kernel(AttnArgs a, int G, int nH, int nKv, int hd, int dtype) {
     float* lrow = mrow + G;               // [G]
     float* alpha = lrow + G;              // [G]
 
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.x / nH, h = blockIdx.x % nH;
     const int g = h / (nH / nKv);
     const int split = blockIdx.y;
@@ -127,6 +129,8 @@ attn_partial_kernel(AttnArgs a, int G, int nH, int nKv, int hd, int dtype) {
 
 // grid (A * nH * G), block hd: merge the splits of one query row of one head.
 __global__ void attn_merge_kernel(AttnArgs a, int G, int nH, int hd) {
+    pdl_trigger();
+    pdl_wait();
     const int row = blockIdx.x;                 // ((b * nH) + h) * G + i
     const int i = row % G, bh = row / G;
     const int b = bh / nH, h = bh % nH;
@@ -173,18 +177,14 @@ cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a, cuda
         configured_dev = m->device;
     }
     dim3 grid(a.A * d.nH, a.n_splits + 1);
-    attn_partial_kernel<<<grid, kThreads, smem, s>>>(a, d.gamma, d.nH, d.nKv, d.hd, d.dtype);
-    cudaError_t e = cudaGetLastError();
-    count_launches(1);
+    cudaError_t e = launch_pdl(attn_partial_kernel, grid, dim3(kThreads), smem, s, a, d.gamma, d.nH, d.nKv, d.hd, d.dtype);
     if (e != cudaSuccess) return e;
     return launch_attention_merge(m, a, s);
 }
 
 cudaError_t launch_attention_merge(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
     const Dims& d = m->d;
-    attn_merge_kernel<<<a.A * d.nH * d.gamma, d.hd, 0, s>>>(a, d.gamma, d.nH, d.hd);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_pdl(attn_merge_kernel, dim3(a.A * d.nH * d.gamma), dim3(d.hd), 0, s, a, d.gamma, d.nH, d.hd);
 }
 
 }  // namespace dspark

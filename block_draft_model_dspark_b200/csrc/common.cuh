@@ -8,6 +8,15 @@
 
 namespace dspark {
 
+// Programmatic dependent launch: every kernel of the library is launched so
+// that it may start while its predecessor in the stream is still running.
+// pdl_trigger lets the next kernel start launching; pdl_wait blocks until the
+// predecessor grid has completed and its memory is visible. A kernel reads
+// nothing its predecessors wrote (and writes nothing they read) before
+// pdl_wait; only constant data (weights) may be touched earlier.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 template <typename T> __device__ __forceinline__ T from_f(float x);

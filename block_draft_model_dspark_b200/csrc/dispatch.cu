@@ -15,6 +15,8 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
 
 namespace {
 
+constexpr size_t kTicketBytes = (size_t)tc::kMaxTickets * 4;
+
 int simt_kps(int K, int S) {
     int kps = (K + S - 1) / S;
     return (kps + 31) / 32 * 32;
@@ -56,44 +58,63 @@ int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len) {
     return (chunk + align - 1) / align * align;
 }
 
-size_t gemm_part_elems(const dspark_model* m, int M, int N, int K, bool act_pair) {
+size_t gemm_out_elems(const dspark_model* m, int M, int N, int K) {
     if (M <= 0) return 0;
-    if (use_tensor_cores(m)) return tc::gemm_partial_elems(tc::plan_gemm(m->num_sms, M, N, K, act_pair ? 2 : 1, false));
+    if (use_tensor_cores(m)) return (size_t)M * N;
     return (size_t)simt_splits(m, M, N, K) * M * N;
 }
 
-cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, int M, int N, int K, float* part,
-                     PartView* view, cudaStream_t s) {
+size_t gemm_scratch_bytes(const dspark_model* m, int M, int N, int K, bool act_pair) {
+    if (M <= 0 || !use_tensor_cores(m)) return 0;
+    const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, act_pair ? 2 : 1, false);
+    return p.streamk ? kTicketBytes + tc::gemm_partial_elems(p) * 4 : 0;
+}
+
+// Tickets first, sized for the largest tile count any plan uses (a tile is at
+// least 128 x 16 of the result, so out elements / 2048 bounds it).
+GemmScratch gemm_scratch_at(void* base, size_t bytes) {
+    GemmScratch sc;
+    if (!base || bytes == 0) return sc;
+    sc.tickets = static_cast<uint32_t*>(base);
+    sc.part = reinterpret_cast<float*>(static_cast<char*>(base) + kTicketBytes);
+    return sc;
+}
+
+cudaError_t gemm_scratch_reset(const GemmScratch& sc, size_t bytes, cudaStream_t s) {
+    if (!sc.tickets || bytes == 0) return cudaSuccess;
+    return cudaMemsetAsync(sc.tickets, 0, kTicketBytes, s);
+}
+
+cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, int M, int N, int K, float* out,
+                     const GemmScratch& sc, PartView* view, cudaStream_t s) {
     KernelTimer t(DSPARK_TIMER_GEMM, s, weight_bytes(m, N, K) + 4.0 * M * K + 4.0 * M * N, 2.0 * M * N * K);
     *view = PartView{};
-    view->p = part;
+    view->p = out;
     if (use_tensor_cores(m)) {
         const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, 2, false);
-        view->mode = 1;
-        view->plan = p;
-        return tc::launch_gemm_tc(p, W.w, W.n, X.hi, X.lo, part, false, 0, 0.f, m->ws.status, s);
+        view->S = 1; view->stride = (int64_t)M * N; view->ld = N;
+        return tc::launch_gemm_tc(p, W.w, W.n, X.hi, X.lo, out, N, 0.f, sc.part, sc.tickets, m->ws.status, s);
     }
     const int S = simt_splits(m, M, N, K);
-    view->mode = 0; view->S = S; view->stride = (int64_t)M * N; view->ld = N;
-    return launch_simt_gemm(X.f32, K, DSPARK_DTYPE_F32, m->d.dtype, W, m->d.group, M, N, K, S, part, N,
+    view->S = S; view->stride = (int64_t)M * N; view->ld = N;
+    return launch_simt_gemm(X.f32, K, DSPARK_DTYPE_F32, m->d.dtype, W, m->d.group, M, N, K, S, out, N,
                             (int64_t)M * N, false, 0.f, s);
 }
 
-cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U, float* part, cudaStream_t s) {
+cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U, cudaStream_t s) {
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_LM_HEAD, s, weight_bytes(m, d.V, d.H) + 4.0 * M * d.H + 4.0 * M * d.V,
                   2.0 * M * (double)d.V * d.H);
-    (void)part;
     if (use_tensor_cores(m)) {
         const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, d.V, d.H, 2, true);
-        return tc::launch_gemm_tc(p, m->lm_head.w, d.V, x.hi, x.lo, U, true, d.V, d.cap, m->ws.status, s);
+        return tc::launch_gemm_tc(p, m->lm_head.w, d.V, x.hi, x.lo, U, d.V, d.cap, nullptr, nullptr, m->ws.status, s);
     }
     return launch_simt_gemm(x.f32, d.H, DSPARK_DTYPE_F32, d.dtype, m->lm_head, d.group, M, d.V, d.H, 1, U, d.V, 0,
                             true, d.cap, s);
 }
 
 cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, const RowsPlan& rp, const KvDest& dst,
-                              float* raw, cudaStream_t s) {
+                              float* raw, const GemmScratch& sc, cudaStream_t s) {
     const Dims& d = m->d;
     const int N = d.Lyr * d.nKv * d.hd;
     const double es = d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0;
@@ -104,12 +125,11 @@ cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, c
     cudaError_t e;
     if (use_tensor_cores(m)) {
         const tc::GemmPlan p = tc::plan_gemm(m->num_sms, nrows, N, d.H, 1, false);
-        view.mode = 1;
-        view.plan = p;
-        e = tc::launch_gemm_tc(p, m->wk_all.w, N, X, nullptr, raw, false, 0, 0.f, m->ws.status, s);
+        view.S = 1; view.stride = (int64_t)nrows * N; view.ld = N;
+        e = tc::launch_gemm_tc(p, m->wk_all.w, N, X, nullptr, raw, N, 0.f, sc.part, sc.tickets, m->ws.status, s);
     } else {
         const int S = simt_splits(m, nrows, N, d.H);
-        view.mode = 0; view.S = S; view.stride = (int64_t)nrows * N; view.ld = N;
+        view.S = S; view.stride = (int64_t)nrows * N; view.ld = N;
         e = launch_simt_gemm(X, d.H, d.dtype, d.dtype, m->wk_all, d.group, nrows, N, d.H, S, raw, N,
                              (int64_t)nrows * N, false, 0.f, s);
     }

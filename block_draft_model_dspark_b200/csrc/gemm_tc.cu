@@ -32,6 +32,7 @@
 #include <string>
 
 #include "internal.h"
+#include "common.cuh"
 #include "gemm_tc.h"
 #include "tc_ptx.cuh"
 
@@ -43,13 +44,19 @@ constexpr int BM = 128;            // weight rows per tile (MMA M)
 constexpr int BK = 64;             // K elements per stage: one 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kABytes = BM * BK * 2;
+constexpr int kMaxStages = 12;
+constexpr int kSmemLimit = 227 * 1024;   // dynamic shared memory a CTA may opt into
+// alignment slack + full/empty barriers per stage + 4 accumulator barriers,
+// the TMEM slot and the abort/last flags
+constexpr int kSmemExtra(int stages) { return 1024 + 16 * stages + 32 + 16 + 64; }
 
 struct KParams {
     GemmPlan p;
-    float* out;        // partial tiles [tile][P][BN][128], or result rows when `direct`
-    int64_t ldo;       // direct: row stride of `out`
-    float cap;         // direct: softcap (0 = none)
-    int direct;        // tile mode only: write out[m * ldo + n] instead of partial tiles
+    float* out;        // result rows out[m * ldo + n]
+    int64_t ldo;
+    float cap;         // softcap of the result (0 = none)
+    float* part;       // stream-K partial tiles [tile][P][BN][128]
+    uint32_t* tickets; // stream-K: one counter per tile, zero between launches
     int32_t* status;
 };
 
@@ -99,7 +106,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     uint64_t* acc_full = empty + stages;      // [2]
     uint64_t* acc_empty = acc_full + 2;       // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort, [1] last-CTA flag
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t tmem_cols = p.tmem_cols;
@@ -117,10 +124,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // TMEM is held: the next kernel in the stream may begin launching (it
+    // waits for this grid before touching what this grid writes).
+    pdl_trigger();
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
+            // The weights do not depend on the previous kernel: the first
+            // `stages` weight tiles are requested before waiting for it, so
+            // the weight stream starts while the producer of X drains.
+            int n_pre = 0;
+            {
+                SegIter it(p, blockIdx.x);
+                int tile, k0, k1, slot;
+                while (n_pre < stages && it.next(tile, k0, k1, slot)) {
+                    const int nt = tile / p.n_mt;
+                    for (int kk = k0; kk < k1 && n_pre < stages; ++kk, ++n_pre) {
+                        mbar_arrive_expect_tx(&full[n_pre], stage_bytes);
+                        tma_load_2d(base + n_pre * stage_bytes, &tmW, &full[n_pre], kk * BK, nt * BM);
+                    }
+                }
+            }
+            pdl_wait();
             SegIter it(p, blockIdx.x);
             int tile, k0, k1, slot, n = 0;
             bool ok = true;
@@ -128,23 +154,34 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 const int nt = tile / p.n_mt, mt = tile % p.n_mt;
                 for (int kk = k0; kk < k1; ++kk, ++n) {
                     const int s = n % stages;
-                    const uint32_t ph = (uint32_t)(n / stages) & 1u;
-                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, kp.status)) { ok = false; break; }
                     uint8_t* st = base + s * stage_bytes;
-                    mbar_arrive_expect_tx(&full[s], stage_bytes);
-                    tma_load_2d(st, &tmW, &full[s], kk * BK, nt * BM);
+                    if (n >= n_pre) {
+                        const uint32_t ph = (uint32_t)(n / stages) & 1u;
+                        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, kp.status)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&full[s], stage_bytes);
+                        tma_load_2d(st, &tmW, &full[s], kk * BK, nt * BM);
+                    }
                     tma_load_2d(st + kABytes, &tmX0, &full[s], kk * BK, mt * BN);
                     if (NP == 2) tma_load_2d(st + kABytes + b_bytes, &tmX1, &full[s], kk * BK, mt * BN);
                 }
             }
-            // drain: the loads of the last `stages` slots complete before teardown
-            for (int d = 0; ok && d < stages && d < n; ++d) {
+            // drain: the loads of the last `stages` slots (every issued slot
+            // has its X loads too, since no wait precedes them) complete
+            // before teardown, also after an abort (bounded)
+            const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
+            for (int d = 0; d < stages && d < n; ++d) {
                 const int m = n - 1 - d;
-                if (!mbar_wait(&full[m % stages], (uint32_t)(m / stages) & 1u, abort_flag, kp.status)) break;
+                if (!mbar_wait_until(&full[m % stages], (uint32_t)(m / stages) & 1u, deadline)) {
+                    atomicOr(kp.status, DSPARK_DEV_WAIT_TIMEOUT);
+                    break;
+                }
             }
+        } else {
+            pdl_wait();
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
+        pdl_wait();
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(BM, BN);
             SegIter it(p, blockIdx.x);
@@ -181,23 +218,33 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         }
     } else {
         // ---------------------------------------------------------- epilogue (warps 2-5)
+        // A tile computed whole by this CTA is written straight to `out`. A
+        // stream-K tile shared by `cnt` CTAs is written as this CTA's partial;
+        // the last of them to finish (ticket counter; nobody waits) sums the
+        // tile's partials in CTA order and writes `out`.
+        pdl_wait();
         const int quad = warp & 3;
         const int n_local = quad * 32 + lane;
+        volatile int* s_last = abort_flag + 1;
         SegIter it(p, blockIdx.x);
         int tile, k0, k1, slot, seg = 0;
         while (it.next(tile, k0, k1, slot)) {
             const int acc = seg & 1;
             const uint32_t aph = (uint32_t)(seg >> 1) & 1u;
-            if (!mbar_wait(&acc_full[acc], aph, abort_flag, kp.status)) break;
+            mbar_wait(&acc_full[acc], aph, abort_flag, kp.status);
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // the group leaves together if any wait gave up
+            if (*abort_flag) break;
             tc_fence_after();
             const int nt = tile / p.n_mt, mt = tile % p.n_mt;
             const int n = nt * BM + n_local;
+            const int cnt = p.streamk ? p.cta_of(tile * p.kb + p.kb - 1) - p.cta_of(tile * p.kb) + 1 : 1;
             const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+            float* part_tile = kp.part + ((int64_t)tile * p.P * BN) * BM + n_local;
             for (int c0 = 0; c0 < BN; c0 += 16) {
                 uint32_t r[16];
                 tmem_ld_x16(tbase + (uint32_t)c0, r);
                 tmem_ld_wait();
-                if (kp.direct) {
+                if (cnt == 1) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int m = mt * BN + c0 + j;
@@ -208,7 +255,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                         }
                     }
                 } else {
-                    float* dst = kp.out + (((int64_t)tile * p.P + slot) * BN + c0) * BM + n_local;
+                    float* dst = part_tile + ((int64_t)slot * BN + c0) * BM;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) dst[(int64_t)j * BM] = __uint_as_float(r[j]);
                 }
@@ -216,6 +263,40 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             tc_fence_before();
             mbar_arrive(&acc_empty[acc]);
             ++seg;
+            if (cnt > 1) {
+                asm volatile("bar.sync 1, 128;" ::: "memory");          // this CTA's partial is written
+                if (threadIdx.x == 64) {
+                    __threadfence();
+                    *s_last = atomicAdd(&kp.tickets[tile], 1u) == (uint32_t)(cnt - 1);
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (*s_last) {
+                    __threadfence();
+                    for (int j0 = 0; j0 < BN; j0 += 16) {        // 16 rows of loads in flight per partial
+                        float v[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                        for (int s2 = 0; s2 < cnt; ++s2) {
+                            const float* src = part_tile + ((int64_t)s2 * BN + j0) * BM;
+                            float x[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) x[j] = src[(int64_t)j * BM];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) v[j] += x[j];     // partials summed in CTA order
+                        }
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int m = mt * BN + j0 + j;
+                            if (m < p.M && n < p.N) {
+                                float y = v[j];
+                                if (kp.cap > 0.f) y = kp.cap * tanhf(y / kp.cap);
+                                kp.out[(int64_t)m * kp.ldo + n] = y;
+                            }
+                        }
+                    }
+                    if (threadIdx.x == 64) kp.tickets[tile] = 0u;
+                }
+            }
         }
     }
 
@@ -270,8 +351,10 @@ GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles) {
     p.n_nt = (N + BM - 1) / BM;
     p.kb = K / BK;
     p.tiles = p.n_mt * p.n_nt;
+    // as many stages as shared memory holds: the bytes in flight per SM are
+    // what sustains the weight stream at HBM latency under load
     const int stage_bytes = kABytes + np * p.BN * BK * 2;
-    p.stages = std::max(2, std::min(8, (200 * 1024) / stage_bytes));
+    p.stages = std::max(2, std::min(kMaxStages, (kSmemLimit - kSmemExtra(kMaxStages)) / stage_bytes));
     p.tmem_cols = tmem_cols_for(p.BN);
     // tile mode when whole tiles balance the SMs to >= 90%, else stream-K
     const int waves = (p.tiles + num_sms - 1) / num_sms;
@@ -293,17 +376,18 @@ GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles) {
 }
 
 size_t gemm_partial_elems(const GemmPlan& p) {
-    return (size_t)p.tiles * p.P * p.BN * BM;
+    return p.streamk ? (size_t)p.tiles * p.P * p.BN * BM : 0;
 }
 
 size_t gemm_smem_bytes(const GemmPlan& p) {
     const int stage_bytes = kABytes + p.np * p.BN * BK * 2;
-    return (size_t)p.stages * stage_bytes + 1024 + 256;
+    return (size_t)p.stages * stage_bytes + kSmemExtra(p.stages);
 }
 
 cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, const void* X0, const void* X1,
-                           float* out, bool direct, int64_t ldo, float cap, int32_t* status, cudaStream_t s) {
-    if (direct && p.mode != kModeTiles) return cudaErrorInvalidValue;
+                           float* out, int64_t ldo, float cap, float* part, uint32_t* tickets, int32_t* status,
+                           cudaStream_t s) {
+    if (p.streamk && (!part || !tickets || p.tiles > kMaxTickets)) return cudaErrorInvalidValue;
     CUtensorMap tw, tx0, tx1;
     if (!make_tmap(&tw, W, w_rows, p.K, BM)) return cudaErrorInvalidValue;
     if (!make_tmap(&tx0, X0, p.M, p.K, p.BN)) return cudaErrorInvalidValue;
@@ -313,20 +397,12 @@ cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, con
         tx1 = tx0;
     }
     KParams kp{};
-    kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.status = status; kp.direct = direct ? 1 : 0;
+    kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.status = status; kp.part = part; kp.tickets = tickets;
     const size_t smem = gemm_smem_bytes(p);
-    cudaError_t e;
-    if (p.np == 2) {
-        e = cudaFuncSetAttribute(gemm_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        gemm_tc_kernel<2><<<p.grid, kThreads, smem, s>>>(tw, tx0, tx1, kp);
-    } else {
-        e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        gemm_tc_kernel<1><<<p.grid, kThreads, smem, s>>>(tw, tx0, tx1, kp);
-    }
-    count_launches(1);
-    return cudaGetLastError();
+    void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, KParams) = p.np == 2 ? gemm_tc_kernel<2> : gemm_tc_kernel<1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3(p.grid), dim3(kThreads), smem, s, tw, tx0, tx1, kp);
 }
 
 }  // namespace tc

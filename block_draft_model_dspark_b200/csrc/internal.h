@@ -51,35 +51,18 @@ struct ModelWs {
     bf16* wk_all_s = nullptr; bf16* wk_all_b = nullptr;
 };
 
-constexpr int kMaxPartials = 12;   // partial tiles a consumer loads at once
-
-// A GEMM result as its consumers read it: out[m][n] is the sum of the GEMM's
-// partial tiles. mode 0: CUDA-core split-K partials [S][M][ld]; mode 1: the
-// tcgen05 GEMM's tiles [tile][P][BN][128] (stream-K: the tile's partials
-// come from consecutive CTAs, summed in CTA order).
+// A GEMM result as its consumers read it: out[m][n] is the sum, in slice
+// order, of S split-K slices [S][M][ld] (S = 1 for the tensor-core GEMM,
+// which reduces its stream-K partials itself). Consumers load slice 0 of
+// all their elements first (at), then add the other slices, so one round of
+// memory latency covers a whole row.
 struct PartView {
     const float* p = nullptr;
-    int mode = 0;
     int S = 1; int64_t stride = 0, ld = 0;
-    tc::GemmPlan plan{};
+    __device__ __forceinline__ float at(int s, int64_t m, int64_t n) const { return p[s * stride + m * ld + n]; }
     __device__ __forceinline__ float sum(int64_t m, int64_t n) const {
-        float v = 0.f;
-        if (mode == 0) {
-            for (int s = 0; s < S; ++s) v += p[s * stride + m * ld + n];
-            return v;
-        }
-        const int BN = plan.BN;
-        const int mt = (int)(m / BN), ml = (int)(m % BN), nt = (int)(n >> 7), nl = (int)(n & 127);
-        const int t = nt * plan.n_mt + mt;
-        int cnt = 1;
-        if (plan.streamk) cnt = plan.cta_of(t * plan.kb + plan.kb - 1) - plan.cta_of(t * plan.kb) + 1;
-        const float* q = p + (((int64_t)t * plan.P) * BN + ml) * 128 + nl;
-        float x[kMaxPartials];
-#pragma unroll
-        for (int s = 0; s < kMaxPartials; ++s) x[s] = s < cnt ? q[(int64_t)s * BN * 128] : 0.f;   // loads in flight together
-#pragma unroll
-        for (int s = 0; s < kMaxPartials; ++s) v += x[s];                                        // summed in CTA order
-        for (int s = kMaxPartials; s < cnt; ++s) v += q[(int64_t)s * BN * 128];
+        float v = at(0, m, n);
+        for (int s = 1; s < S; ++s) v += at(s, m, n);
         return v;
     }
 };
@@ -201,8 +184,13 @@ struct WalkArgs {
     int32_t* status;
 };
 cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s);
+// The whole walk in one cooperative launch (one CTA per SM, bounded grid barriers).
+bool walk_persistent_supported(const dspark_model* m, int A);
+int walk_persistent_blocks(const dspark_model* m);
+cudaError_t launch_walk_persistent(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
+                                   float* cand_val, int32_t* cand_idx, uint32_t* arrivals, int A, cudaStream_t s);
 // Vocabulary slices (grid.x) of a walk step.
-int walk_vocab_blocks(int num_sms, int V, int r);
+int walk_vocab_blocks(int num_sms, int V, int r, int dtype, bool quant);
 cudaError_t launch_walk_init(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V,
                              int32_t* status, cudaStream_t s);
 // Confidence + lengths (hf = the final-normed hidden, fp32 [M, H]).
@@ -210,6 +198,27 @@ cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const in
                               int A, float* conf, int32_t* lengths, cudaStream_t s);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Launches a kernel with programmatic stream serialization (it may begin
+// before its predecessor in the stream ends; see pdl_wait in common.cuh) and
+// counts it.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void count_launches(int n);
+    count_launches(1);
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 // Launch accounting (timing.cu): count_launches after each launch; a
 // KernelTimer in scope around a launch brackets it with events when timing is on.

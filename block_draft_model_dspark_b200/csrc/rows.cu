@@ -39,6 +39,8 @@ __device__ __forceinline__ float mat_at(const MatRef& W, int dtype, int group, i
 __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const double* __restrict__ inv_freq,
                                    LayerPtrs k_norms, int nKv, int hd, float eps, int dtype, int32_t* status) {
     __shared__ float red[32];
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     const int rg = rp.row0 + r;
     const int b = rg / rp.Lrows, t = rg % rp.Lrows;
@@ -52,8 +54,8 @@ __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const 
     const int l = blockIdx.y / nKv, g = blockIdx.y % nKv;
     const int half = hd / 2, i = threadIdx.x;
     const int64_t col = (int64_t)blockIdx.y * hd;
-    const float x1 = raw.sum(r, col + i);
-    const float x2 = raw.sum(r, col + i + half);
+    float x1 = raw.at(0, r, col + i), x2 = raw.at(0, r, col + i + half);
+    for (int sl = 1; sl < raw.S; ++sl) { x1 += raw.at(sl, r, col + i); x2 += raw.at(sl, r, col + i + half); }
     const float ss = block_sum(x1 * x1 + x2 * x2, red);
     const float rinv = rsqrtf(ss / (float)hd + eps);
     const float v1 = x1 * rinv, v2 = x2 * rinv;
@@ -69,15 +71,19 @@ __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const 
 }
 
 __global__ void commit_len_kernel(int32_t* len, const int32_t* n_new, int B) {
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b < B) len[b] += n_new[b];
 }
 
 // ------------------------------------------------------------------ block embedding
-__global__ void embed_kernel(MatRef E, int dtype, int group, const int32_t* __restrict__ anchors, int gamma,
+__global__ void __launch_bounds__(512) embed_kernel(MatRef E, int dtype, int group, const int32_t* __restrict__ anchors, int gamma,
                              int mask_id, int V, int H, float scale, const void* __restrict__ w_in,
                              float eps, float* __restrict__ h, ActBuf x, int32_t* status) {
     __shared__ float red[32];
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x;
     const int b = m / gamma, t = m % gamma;
     int id = t == 0 ? anchors[b] : mask_id;
@@ -115,13 +121,15 @@ __global__ void qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, in
                                    const void* __restrict__ q_norm, const void* __restrict__ k_norm, float eps,
                                    int dtype, float* __restrict__ q, void* __restrict__ kb, void* __restrict__ vb) {
     __shared__ float red[32];
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x, hh = blockIdx.y;
     const int b = m / gamma, t = m % gamma;
     const int pos = block_pos[b] + t;
     const int half = hd / 2, i = threadIdx.x;
     const int64_t col = (int64_t)hh * hd;
-    const float x1 = part.sum(m, col + i);
-    const float x2 = part.sum(m, col + i + half);
+    float x1 = part.at(0, m, col + i), x2 = part.at(0, m, col + i + half);
+    for (int sl = 1; sl < part.S; ++sl) { x1 += part.at(sl, m, col + i); x2 += part.at(sl, m, col + i + half); }
     const float ss = block_sum(x1 * x1 + x2 * x2, red);
     const float rinv = rsqrtf(ss / (float)hd + eps);
     float y1 = x1 * rinv, y2 = x2 * rinv;
@@ -147,48 +155,70 @@ __global__ void qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, in
 // ------------------------------------------------------------------ o_proj / down epilogues
 // mode 0 (o_proj):  h += rms(sum, g1);            x = rms(h, g2)
 // mode 1 (down):    h = (h + rms(sum, g1)) * s;   x = rms(h, g2)
-__global__ void residual_epilogue_kernel(PartView part, int H, const void* __restrict__ g1,
+template <int PER>
+__global__ void __launch_bounds__(512) residual_epilogue_kernel(PartView part, int H, const void* __restrict__ g1,
                                          const void* __restrict__ g2, const void* __restrict__ scalar, int mode,
                                          float eps, int dtype, float* __restrict__ h, ActBuf x) {
     __shared__ float red[32];
+    pdl_trigger();
     const int m = blockIdx.x;
-    float a[kMaxPer];
+    float a[PER], hv[PER], w1v[PER], w2v[PER];
+    // the gains are weights: loaded while the producing GEMM drains
+#pragma unroll
+    for (int c = 0; c < PER; ++c) {
+        const int j = threadIdx.x + c * blockDim.x;
+        const bool in = j < H;
+        w1v[c] = in ? load_any(g1, j, dtype) : 0.f;
+        w2v[c] = in ? load_any(g2, j, dtype) : 0.f;
+    }
+    const float s = mode == 1 ? load_any(scalar, 0, dtype) : 1.f;
+    pdl_wait();
+    // every activation load of the row first: one round of memory latency
+#pragma unroll
+    for (int c = 0; c < PER; ++c) {
+        const int j = threadIdx.x + c * blockDim.x;
+        const bool in = j < H;
+        a[c] = in ? part.at(0, m, j) : 0.f;
+        hv[c] = in ? h[(int64_t)m * H + j] : 0.f;
+    }
+    for (int sl = 1; sl < part.S; ++sl) {
+#pragma unroll
+        for (int c = 0; c < PER; ++c) {
+            const int j = threadIdx.x + c * blockDim.x;
+            if (j < H) a[c] += part.at(sl, m, j);
+        }
+    }
     float ss = 0.f;
 #pragma unroll
-    for (int c = 0; c < kMaxPer; ++c) {
-        const int j = threadIdx.x + c * blockDim.x;
-        a[c] = j < H ? part.sum(m, j) : 0.f;
-        ss += a[c] * a[c];
-    }
+    for (int c = 0; c < PER; ++c) ss += a[c] * a[c];
     ss = block_sum(ss, red);
     const float r1 = rsqrtf(ss / (float)H + eps);
-    const float s = mode == 1 ? load_any(scalar, 0, dtype) : 1.f;
     float ss2 = 0.f;
 #pragma unroll
-    for (int c = 0; c < kMaxPer; ++c) {
-        const int j = threadIdx.x + c * blockDim.x;
-        if (j < H) {
-            const float nv = (h[(int64_t)m * H + j] + a[c] * r1 * load_any(g1, j, dtype)) * s;
-            h[(int64_t)m * H + j] = nv;
-            a[c] = nv;
-            ss2 += nv * nv;
-        }
+    for (int c = 0; c < PER; ++c) {
+        hv[c] = (hv[c] + a[c] * r1 * w1v[c]) * s;
+        ss2 += hv[c] * hv[c];
     }
     ss2 = block_sum(ss2, red);
     const float r2 = rsqrtf(ss2 / (float)H + eps);
 #pragma unroll
-    for (int c = 0; c < kMaxPer; ++c) {
+    for (int c = 0; c < PER; ++c) {
         const int j = threadIdx.x + c * blockDim.x;
-        if (j < H) store_act(x, (int64_t)m * H + j, a[c] * r2 * load_any(g2, j, dtype));
+        if (j < H) {
+            h[(int64_t)m * H + j] = hv[c];
+            store_act(x, (int64_t)m * H + j, hv[c] * r2 * w2v[c]);
+        }
     }
 }
 
 __global__ void gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t total = (int64_t)M * I;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t m = e / I, i = e % I;
-        const float g = part.sum(m, i);
-        const float u = part.sum(m, I + i);
+        float g = part.at(0, m, i), u = part.at(0, m, I + i);
+        for (int sl = 1; sl < part.S; ++sl) { g += part.at(sl, m, i); u += part.at(sl, m, I + i); }
         store_act(act, e, gelu_tanh(g) * u);
     }
 }
@@ -201,6 +231,8 @@ __global__ void confidence_kernel(const float* __restrict__ hf32, MatRef P, int 
                                   const int32_t* __restrict__ anchors, const int32_t* __restrict__ tokens,
                                   int gamma, int H, int r, int with_markov, int V, float* __restrict__ conf) {
     __shared__ float red[32];
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x;
     const int b = m / gamma, k = m % gamma;
     int prev = k == 0 ? anchors[b] : tokens[b * gamma + k - 1];
@@ -217,6 +249,8 @@ __global__ void confidence_kernel(const float* __restrict__ hf32, MatRef P, int 
 // lengths[b] = first k with conf < thr (thr > 0), else gamma (no head: gamma).
 __global__ void lengths_kernel(const float* __restrict__ conf, int A, int gamma, float thr, int has_head,
                                int32_t* __restrict__ lengths) {
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= A) return;
     int len = gamma;
@@ -229,6 +263,24 @@ __global__ void lengths_kernel(const float* __restrict__ conf, int A, int gamma,
 // Threads of a full-row kernel: enough that each holds at most kMaxPer
 // columns, about 8 columns per thread, and at most 512 (the kernels use up
 // to ~80 registers a thread; 512 x 80 fits a block's register file).
+// Columns per thread (template argument of the full-row kernels) for a row
+// of H spread over row_threads(H) threads.
+int row_per(int H, int threads) {
+    const int per = (H + threads - 1) / threads;
+    return per <= 4 ? 4 : per <= 8 ? 8 : kMaxPer;
+}
+
+template <int PER>
+cudaError_t launch_residual(const PartView& part, int M, int H, const void* g1, const void* g2, const void* scalar,
+                            int mode, float eps, int dtype, float* h, const ActBuf& x, int threads, cudaStream_t s) {
+    return launch_pdl(residual_epilogue_kernel<PER>, dim3(M), dim3(threads), 0, s, part, H, g1, g2, scalar, mode, eps,
+                      dtype, h, x);
+}
+
+cudaError_t launch_residual_any(const PartView& part, int M, int H, const void* g1, const void* g2,
+                                const void* scalar, int mode, float eps, int dtype, float* h, const ActBuf& x,
+                                cudaStream_t s);
+
 int row_threads(int H) {
     int t = (H + 7) / 8;
     const int need = (H + kMaxPer - 1) / kMaxPer;
@@ -236,6 +288,17 @@ int row_threads(int H) {
     if (t < need) t = need;
     t = (t + 31) / 32 * 32;
     return t < 32 ? 32 : t;
+}
+
+cudaError_t launch_residual_any(const PartView& part, int M, int H, const void* g1, const void* g2,
+                                const void* scalar, int mode, float eps, int dtype, float* h, const ActBuf& x,
+                                cudaStream_t s) {
+    const int t = row_threads(H);
+    switch (row_per(H, t)) {
+        case 4: return launch_residual<4>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, t, s);
+        case 8: return launch_residual<8>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, t, s);
+        default: return launch_residual<kMaxPer>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, t, s);
+    }
 }
 
 }  // namespace
@@ -247,86 +310,71 @@ cudaError_t launch_kv_epilogue(const dspark_model* m, const PartView& raw, const
     LayerPtrs kn{};
     for (int l = 0; l < d.Lyr; ++l) kn.p[l] = m->layers[l].k_norm;
     dim3 grid(rp.nrows, d.Lyr * d.nKv);
-    kv_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(raw, rp, dst, m->ws.inv_freq, kn, d.nKv, d.hd, d.eps, d.dtype,
-                                                 m->ws.status);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_pdl(kv_epilogue_kernel, grid, dim3(d.hd / 2), 0, s, raw, rp, dst, m->ws.inv_freq, kn, d.nKv, d.hd,
+                      d.eps, d.dtype, m->ws.status);
 }
 
 cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStream_t s) {
-    commit_len_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, n_new, B);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_pdl(commit_len_kernel, dim3((B + 127) / 128), dim3(128), 0, s, len, n_new, B);
 }
 
 cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, float* h, const ActBuf& x,
                          int32_t* status, cudaStream_t s) {
     const Dims& d = m->d;
-    embed_kernel<<<A * d.gamma, row_threads(d.H), 0, s>>>(m->embed, d.dtype, d.group, anchors, d.gamma, d.mask_id,
-                                                         d.V, d.H, sqrtf((float)d.H), m->layers[0].in_norm, d.eps,
-                                                         h, x, status);
-    count_launches(1);
-    return cudaGetLastError();
+    KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
+    return launch_pdl(embed_kernel, dim3(A * d.gamma), dim3(row_threads(d.H)), 0, s, m->embed, d.dtype, d.group, anchors,
+                      d.gamma, d.mask_id, d.V, d.H, sqrtf((float)d.H), m->layers[0].in_norm, d.eps, h, x, status);
 }
 
 cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const PartView& part, int A,
                                const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s) {
     const Dims& d = m->d;
+    KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
     dim3 grid(A * d.gamma, d.nH + d.nKv);
-    qk_epilogue_kernel<<<grid, d.hd / 2, 0, s>>>(part, d.gamma, d.nH, d.nKv, d.hd, block_pos, m->ws.inv_freq,
-                                                 m->layers[layer].q_norm, m->layers[layer].k_norm, d.eps, d.dtype,
-                                                 q, kb, vb);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_pdl(qk_epilogue_kernel, grid, dim3(d.hd / 2), 0, s, part, d.gamma, d.nH, d.nKv, d.hd, block_pos,
+                      m->ws.inv_freq, m->layers[layer].q_norm, m->layers[layer].k_norm, d.eps, d.dtype, q, kb, vb);
 }
 
 cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,
                               const ActBuf& x, cudaStream_t s) {
     const Dims& d = m->d;
+    KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
     const LayerRef& L = m->layers[layer];
-    residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, d.H, L.post_attn_norm, L.pre_ff_norm, nullptr, 0,
-                                                            d.eps, d.dtype, h, x);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_residual_any(part, M, d.H, L.post_attn_norm, L.pre_ff_norm, nullptr, 0, d.eps, d.dtype, h, x, s);
 }
 
 cudaError_t launch_gu_epilogue(const dspark_model* m, const PartView& part, int M, const ActBuf& act,
                                cudaStream_t s) {
     const Dims& d = m->d;
+    KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
     const int64_t total = (int64_t)M * d.I;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 8 * m->num_sms) blocks = 8 * m->num_sms;
-    gu_epilogue_kernel<<<blocks, 256, 0, s>>>(part, M, d.I, act);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_pdl(gu_epilogue_kernel, dim3(blocks), dim3(256), 0, s, part, M, d.I, act);
 }
 
 cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,
                                  const ActBuf& x, cudaStream_t s) {
     const Dims& d = m->d;
+    KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
     const LayerRef& L = m->layers[layer];
     const bool last = layer + 1 == d.Lyr;
     const void* next = last ? m->final_norm : m->layers[layer + 1].in_norm;
-    residual_epilogue_kernel<<<M, row_threads(d.H), 0, s>>>(part, d.H, L.post_ff_norm, next, L.layer_scalar, 1,
-                                                            d.eps, d.dtype, h, x);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_residual_any(part, M, d.H, L.post_ff_norm, next, L.layer_scalar, 1, d.eps, d.dtype, h, x, s);
 }
 
 cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const int32_t* anchors, const int32_t* tokens,
                               int A, float* conf, int32_t* lengths, cudaStream_t s) {
     const Dims& d = m->d;
+    KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
     if (d.conf_head) {
-        confidence_kernel<<<A * d.gamma, 256, 0, s>>>(hf32, m->conf_proj, d.dtype, d.group, m->w1, m->conf_bias,
-                                                      anchors, tokens, d.gamma, d.H, d.r, d.conf_markov ? 1 : 0, d.V,
-                                                      conf);
-        count_launches(1);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(confidence_kernel, dim3(A * d.gamma), dim3(256), 0, s, hf32, m->conf_proj, d.dtype,
+                                   d.group, m->w1, m->conf_bias, anchors, tokens, d.gamma, d.H, d.r,
+                                   d.conf_markov ? 1 : 0, d.V, conf);
         if (e != cudaSuccess) return e;
     }
-    lengths_kernel<<<(A + 127) / 128, 128, 0, s>>>(conf, A, d.gamma, d.conf_thr, d.conf_head ? 1 : 0, lengths);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_pdl(lengths_kernel, dim3((A + 127) / 128), dim3(128), 0, s, conf, A, d.gamma, d.conf_thr,
+                      d.conf_head ? 1 : 0, lengths);
 }
 
 }  // namespace dspark

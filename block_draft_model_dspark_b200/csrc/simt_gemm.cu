@@ -45,6 +45,8 @@ simt_gemm_kernel(const TX* __restrict__ X, int64_t ldx, const void* __restrict__
                  int64_t split_stride, int softcap, float cap) {
     __shared__ float Xs[BK][BM + 4];
     __shared__ float Ws[BK][BN + 4];
+    pdl_trigger();
+    pdl_wait();
     const int tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
     const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
@@ -122,9 +124,10 @@ cudaError_t launch_simt_gemm(const void* X, int64_t ldx, int x_dtype, int w_dtyp
     const int z = (K + kps - 1) / kps;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, z);
 #define DSPARK_SIMT_LAUNCH(TX, TW, Q)                                                                     \
-    simt_gemm_kernel<TX, TW, Q><<<grid, 256, 0, s>>>(static_cast<const TX*>(X), ldx, W.w, W.scales, W.biases, \
-                                                     group, M, N, K, kps, out, ldo, split_stride, softcap, cap)
+    e = launch_pdl(simt_gemm_kernel<TX, TW, Q>, grid, dim3(256), 0, s, static_cast<const TX*>(X), ldx, W.w,   \
+                   W.scales, W.biases, group, M, N, K, kps, out, ldo, split_stride, (int)softcap, cap)
     const bool xf = x_dtype == DSPARK_DTYPE_F32;
+    cudaError_t e;
     if (W.quant) {
         if (xf) DSPARK_SIMT_LAUNCH(float, bf16, true); else DSPARK_SIMT_LAUNCH(bf16, bf16, true);
     } else if (w_dtype == DSPARK_DTYPE_F32) {
@@ -133,8 +136,7 @@ cudaError_t launch_simt_gemm(const void* X, int64_t ldx, int x_dtype, int w_dtyp
         if (xf) DSPARK_SIMT_LAUNCH(float, bf16, false); else DSPARK_SIMT_LAUNCH(bf16, bf16, false);
     }
 #undef DSPARK_SIMT_LAUNCH
-    count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace dspark

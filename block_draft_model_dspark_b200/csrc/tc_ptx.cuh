@@ -70,6 +70,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Waits for the phase of `parity` until the global timer passes `deadline`,
+// whatever other roles did; for draining copies in flight before exit.
+__device__ __forceinline__ bool mbar_wait_until(uint64_t* bar, uint32_t parity, uint64_t deadline) {
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && global_timer_ns() > deadline) return false;
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 // 2-D tiled load of box {x, y} at coordinates (x = innermost element index,
 // y = row) into shared memory, completing `bytes` on the mbarrier.
@@ -176,6 +185,14 @@ __device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t smem_addr, uint32_t 
            | ((uint64_t)(1024 >> 4) << 32)
            | ((uint64_t)1 << 46)
            | ((uint64_t)2 << 61);
+}
+
+// 1-D bulk copy global -> shared of `bytes` (both addresses 16-byte aligned,
+// bytes a multiple of 16), completing on the mbarrier.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 
 // 3-D tiled TMA load (coordinates innermost first).
