@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--impl", default="dspark", choices=["dspark", "reference"])
     ap.add_argument("--workload", default="single_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None, choices=[None, "attention"],
+                    help="time one seam alone instead of the round (prints a case line, not the bench line)")
     return ap.parse_args()
 
 
@@ -343,7 +345,7 @@ def run_dspark(args, wl):
         ms_per_step = ms_total / args.steps
         value = tok_per_step / (ms_per_step / 1e3)
         hbm, tf_burst, tf_sust, peak_kind = measured_peaks()
-        # the dominant kernel class by device time
+        # the dominant kernel (one kernel shape per timer class) by device time
         dom = max(kinds, key=lambda k: kinds[k]["ms"])
         dk = kinds[dom]
         per_launch_ms = dk["ms"] / max(dk["launches"], 1)
@@ -389,10 +391,61 @@ def run_dspark(args, wl):
         dist.destroy_process_group()
 
 
+def run_attention_case(args, wl):
+    """The KV-injection attention seam alone (dspark_attend) at a workload's
+    attention shape and context lengths: one layer's cache, random bf16 K/V.
+    Prints one JSON line with the achieved K/V bandwidth (not the bench line)."""
+    import torch
+    import block_draft_model_dspark_b200 as dsp
+    from block_draft_model_dspark_b200 import build as libbuild
+    from synthetic import make_weights, round_meta
+    libbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    m0 = wl.model
+    # only the attention dimensions matter to the seam: a 1-layer model with small other sizes
+    m = m0.replace(num_hidden_layers=1, hidden_size=256, intermediate_size=256, vocab_size=1024, mask_token_id=1023,
+                   markov_rank=8, quant_bits=0)
+    model = dsp.DsparkModel(m, {k: v.to(dev) for k, v in make_weights(m, wl.seed).items()})
+    lens = [int(x) for x in round_meta(wl)[0].tolist()]
+    A, G, nH, nKv, hd = wl.rows, m.block_size, m.num_attention_heads, m.num_global_key_value_heads, m.global_head_dim
+    L = max(lens)
+    cache = dsp.KvCache(model, A, L)
+    g = torch.Generator(device=dev).manual_seed(wl.seed)
+    cache.k.copy_(torch.randn(cache.k.shape, generator=g, device=dev, dtype=torch.float32).to(cache.k.dtype))
+    cache.v.copy_(torch.randn(cache.v.shape, generator=g, device=dev, dtype=torch.float32).to(cache.v.dtype))
+    cache.set_lengths(lens)
+    q = torch.randn(A, G, nH, hd, generator=g, device=dev).to(torch.bfloat16)
+    kb = torch.randn(A, G, nKv, hd, generator=g, device=dev).to(torch.bfloat16)
+    vb = torch.randn(A, G, nKv, hd, generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty(A, G, nH, hd, device=dev, dtype=torch.bfloat16)
+    ws = model.workspace(model.draft_workspace_bytes(A, L))
+    for _ in range(max(args.warmup, 3)):
+        model.dspark_attend(0, cache, q, kb, vb, out, L, ws=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        model.dspark_attend(0, cache, q, kb, vb, out, L, ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / args.steps * 1e3
+    kv_bytes = sum(lens[b] + G for b in range(A)) * nKv * hd * 2 * 2 + 2 * A * G * nH * hd * 2
+    hbm = measured_peaks()[0]
+    gbs = kv_bytes / (us * 1e-6) / 1e9
+    print(json.dumps({"case": "attention", "workload": wl.name, "A": A, "ctx_lens": lens, "heads": [nH, nKv, hd],
+                      "us_per_call": us, "algorithmic_bytes": kv_bytes, "GB_per_s": gbs, "hbm_peak_GB_per_s": hbm,
+                      "frac": gbs / hbm, "calls": args.steps, "note": "attention partials + merge kernel; "
+                      "cache larger than L2 when its bytes exceed 126 MB"}), flush=True)
+
+
 def main():
     args = parse()
     from synthetic import WORKLOADS
     wl = WORKLOADS[args.workload]
+    if args.case == "attention":
+        run_attention_case(args, wl)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
     else:

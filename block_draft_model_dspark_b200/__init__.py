@@ -92,7 +92,8 @@ _PROTOTYPES = {
                                   ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
 }
 
-DSPARK_TIMER_KINDS = {"gemm": 0, "lm_head": 1, "attention": 2, "walk": 3, "kv_project": 4, "rows": 5}
+DSPARK_TIMER_KINDS = {"gemm_qk": 0, "lm_head": 1, "attention": 2, "walk": 3, "kv_project": 4, "rows": 5,
+                      "gemm_o": 6, "gemm_gu": 7, "gemm_down": 8}
 
 
 def dspark_kernel_launches() -> int:

@@ -517,18 +517,18 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     if (e == cudaSuccess) e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
     for (int l = 0; l < d.Lyr && e == cudaSuccess; ++l) {
         const LayerRef& L = m->layers[l];
-        e = run_gemm(m, x, L.qk, M, Nqk, d.H, part, sc, &pv, s);
+        e = run_gemm(m, x, L.qk, M, Nqk, d.H, part, sc, &pv, DSPARK_TIMER_GEMM_QK, s);
         if (e == cudaSuccess) e = launch_qk_epilogue(m, l, pv, A, block_pos, q, kb, vb, s);
         if (e == cudaSuccess) {
             AttnArgs a = attn_args(m, p, ws, cache, l, A, q, kb, vb, ao.f32, DSPARK_DTYPE_F32);
             a.out_hi = ao.hi; a.out_lo = ao.lo;
             e = run_attention(m, a, s);
         }
-        if (e == cudaSuccess) e = run_gemm(m, ao, L.o, M, d.H, d.nH * d.hd, part, sc, &pv, s);
+        if (e == cudaSuccess) e = run_gemm(m, ao, L.o, M, d.H, d.nH * d.hd, part, sc, &pv, DSPARK_TIMER_GEMM_O, s);
         if (e == cudaSuccess) e = launch_o_epilogue(m, l, pv, M, h, x, s);
-        if (e == cudaSuccess) e = run_gemm(m, x, L.gu, M, 2 * d.I, d.H, part, sc, &pv, s);
+        if (e == cudaSuccess) e = run_gemm(m, x, L.gu, M, 2 * d.I, d.H, part, sc, &pv, DSPARK_TIMER_GEMM_GU, s);
         if (e == cudaSuccess) e = launch_gu_epilogue(m, pv, M, act, s);
-        if (e == cudaSuccess) e = run_gemm(m, act, L.down, M, d.H, d.I, part, sc, &pv, s);
+        if (e == cudaSuccess) e = run_gemm(m, act, L.down, M, d.H, d.I, part, sc, &pv, DSPARK_TIMER_GEMM_DOWN, s);
         if (e == cudaSuccess) e = launch_down_epilogue(m, l, pv, M, h, x, s);
     }
     if (e == cudaSuccess) e = run_lm_head(m, x, M, U, s);
@@ -539,7 +539,10 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
         wa.ticket = at<uint32_t>(ws, p.ticket); wa.A = A; wa.nblk = p.walk_blocks; wa.status = m->ws.status;
         const double w2b = d.r > 0 ? (d.quant ? (double)d.V * d.r * 0.5 + (double)d.V * (d.r / d.group) * 4.0
                                               : (double)d.V * d.r * esize(d.dtype)) : 0.0;
-        if (walk_persistent_supported(m, A)) {
+        if (tc::walk_tc_supported(m, A)) {
+            KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
+            e = tc::launch_walk_tc(m, U, anchors, tokens, wa.part_val, wa.part_idx, wa.ticket, A, s);
+        } else if (walk_persistent_supported(m, A)) {
             KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
             e = launch_walk_persistent(m, U, anchors, tokens, wa.part_val, wa.part_idx, wa.ticket, A, s);
         } else {

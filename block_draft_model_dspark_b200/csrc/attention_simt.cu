@@ -127,6 +127,8 @@ attn_partial_kernel(AttnArgs a, int G, int nH, int nKv, int hd, int dtype) {
     }
 }
 
+constexpr int kMergeBatch = 32;      // splits a merge thread loads at once
+
 // grid (A * nH * G), block hd: merge the splits of one query row of one head.
 __global__ void attn_merge_kernel(AttnArgs a, int G, int nH, int hd) {
     pdl_trigger();
@@ -135,20 +137,41 @@ __global__ void attn_merge_kernel(AttnArgs a, int G, int nH, int hd) {
     const int i = row % G, bh = row / G;
     const int b = bh / nH, h = bh % nH;
     const int d = threadIdx.x;
-    const int S1 = a.n_splits + 1;
-    float M = -INFINITY;
-#pragma unroll 8
-    for (int s = 0; s < S1; ++s) M = fmaxf(M, a.part_ml[(((int64_t)bh * S1 + s) * G + i) * 2]);
+    const int S1 = a.S1;
     float num = 0.f, den = 0.f;
+    if (S1 <= kMergeBatch) {
+        // every split's (max, sum, O) in flight at once: one round of memory latency
+        float mv[kMergeBatch], lv[kMergeBatch], ov[kMergeBatch];
+#pragma unroll
+        for (int s = 0; s < kMergeBatch; ++s) {
+            const int64_t base = ((int64_t)bh * S1 + s) * G + i;
+            mv[s] = s < S1 ? a.part_ml[base * 2] : -INFINITY;
+            lv[s] = s < S1 ? a.part_ml[base * 2 + 1] : 0.f;
+            ov[s] = s < S1 ? a.part_o[base * hd + d] : 0.f;
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < kMergeBatch; ++s) M = fmaxf(M, mv[s]);
+#pragma unroll
+        for (int s = 0; s < kMergeBatch; ++s) {
+            const float w = mv[s] == -INFINITY ? 0.f : expf(mv[s] - M);   // empty splits carry no weight
+            den += w * lv[s];
+            num += w * (mv[s] == -INFINITY ? 0.f : ov[s]);
+        }
+    } else {
+        float M = -INFINITY;
 #pragma unroll 8
-    for (int s = 0; s < S1; ++s) {
-        const int64_t base = ((int64_t)bh * S1 + s) * G + i;
-        const float m = a.part_ml[base * 2];
-        const float l = a.part_ml[base * 2 + 1];
-        const float o = m == -INFINITY ? 0.f : a.part_o[base * hd + d];
-        const float w = m == -INFINITY ? 0.f : expf(m - M);
-        den += w * l;
-        num += w * o;
+        for (int s = 0; s < S1; ++s) M = fmaxf(M, a.part_ml[(((int64_t)bh * S1 + s) * G + i) * 2]);
+#pragma unroll 8
+        for (int s = 0; s < S1; ++s) {
+            const int64_t base = ((int64_t)bh * S1 + s) * G + i;
+            const float m = a.part_ml[base * 2];
+            const float l = a.part_ml[base * 2 + 1];
+            const float o = m == -INFINITY ? 0.f : a.part_o[base * hd + d];
+            const float w = m == -INFINITY ? 0.f : expf(m - M);
+            den += w * l;
+            num += w * o;
+        }
     }
     const int64_t o = (((int64_t)b * G + i) * nH + h) * hd + d;
     const float v = num / den;
@@ -168,7 +191,9 @@ size_t attn_simt_smem(int G, int hd) {
     return sizeof(float) * ((size_t)G * hd + 2 * (size_t)KT * hd + (size_t)G * KT + 3 * (size_t)G);
 }
 
-cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
+cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a_in, cudaStream_t s) {
+    AttnArgs a = a_in;
+    a.S1 = a.n_splits + 1;                      // context splits + the block split
     const Dims& d = m->d;
     const size_t smem = attn_simt_smem(d.gamma, d.hd);
     static thread_local int configured_dev = -1;

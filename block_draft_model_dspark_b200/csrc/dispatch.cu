@@ -10,6 +10,7 @@ namespace dspark {
 cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
 namespace tc {
 bool attention_tc_supported(const dspark_model* m);
+int attention_tc_key_tile();
 cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
 }
 
@@ -48,11 +49,14 @@ int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len) {
     const Dims& d = m->d;
     const bool tcore = tc::attention_tc_supported(m);
     const int per_split = A * (tcore ? d.nKv : d.nH);
-    const int want = std::max(1, (2 * m->num_sms + per_split - 1) / per_split);
-    const int align = tcore ? 64 : 16;
-    // tensor cores: >= 4 key tiles per split, so a split's partial output (q rows x hd fp32)
-    // stays below half of the K/V bytes it reads
-    const int min_chunk = tcore ? 256 : 64;
+    // tensor cores: one CTA per SM (a CTA holds ~225 KB of shared memory), so one wave
+    // of A * nKv * splits CTAs; CUDA cores: ~2 waves
+    const int want = tcore ? std::max(1, m->num_sms / per_split)
+                           : std::max(1, (2 * m->num_sms + per_split - 1) / per_split);
+    const int align = tcore ? tc::attention_tc_key_tile() : 16;
+    // tensor cores: >= 4 key tiles per split (each split also pays a Q tile load and
+    // writes a 128-row partial O)
+    const int min_chunk = tcore ? 4 * tc::attention_tc_key_tile() : 64;
     int chunk = min_chunk;
     if (max_ctx_len > 0) chunk = std::max(min_chunk, (max_ctx_len + want - 1) / want);
     return (chunk + align - 1) / align * align;
@@ -86,8 +90,8 @@ cudaError_t gemm_scratch_reset(const GemmScratch& sc, size_t bytes, cudaStream_t
 }
 
 cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, int M, int N, int K, float* out,
-                     const GemmScratch& sc, PartView* view, cudaStream_t s) {
-    KernelTimer t(DSPARK_TIMER_GEMM, s, weight_bytes(m, N, K) + 4.0 * M * K + 4.0 * M * N, 2.0 * M * N * K);
+                     const GemmScratch& sc, PartView* view, int timer_kind, cudaStream_t s) {
+    KernelTimer t(timer_kind, s, weight_bytes(m, N, K) + 4.0 * M * K + 4.0 * M * N, 2.0 * M * N * K);
     *view = PartView{};
     view->p = out;
     if (use_tensor_cores(m)) {

@@ -23,7 +23,7 @@ GemmScratch gemm_scratch_at(void* base, size_t bytes);
 cudaError_t gemm_scratch_reset(const GemmScratch& sc, size_t bytes, cudaStream_t s);
 // out = X @ W^T for an activation X (fp32, or its bf16 pair on tensor cores); *view reads the result.
 cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, int M, int N, int K, float* out,
-                     const GemmScratch& sc, PartView* view, cudaStream_t s);
+                     const GemmScratch& sc, PartView* view, int timer_kind, cudaStream_t s);
 // U[m][v] = softcap(x[m] . lm_head[v]) in fp32 (no cap when final_logit_softcapping == 0).
 cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U, cudaStream_t s);
 // Context K/V of `nrows` rows of the caller's hidden X (model dtype) into `dst`.

@@ -34,6 +34,7 @@
 #include "internal.h"
 #include "common.cuh"
 #include "gemm_tc.h"
+#include "tmap.h"
 #include "tc_ptx.cuh"
 
 namespace dspark {
@@ -183,7 +184,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         // ---------------------------------------------------------- MMA issuer
         pdl_wait();
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(BM, BN);
+            // hi and lo in one MMA when both fit in N <= 256: the X_lo rows sit right
+            // after the X_hi rows in the stage, so [X_hi; X_lo] is one B operand of
+            // 2 BN rows and the two products land in adjacent accumulator columns
+            const bool fused = NP == 2 && p.acc_cols == 2 * BN;
+            const uint32_t idesc = idesc_bf16(BM, fused ? 2 * BN : BN);
             SegIter it(p, blockIdx.x);
             int tile, k0, k1, slot, n = 0, seg = 0;
             bool ok = true;
@@ -192,7 +197,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 const uint32_t aph = (uint32_t)(seg >> 1) & 1u;
                 if (!mbar_wait(&acc_empty[acc], aph ^ 1u, abort_flag, kp.status)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_cols);
                 for (int kk = k0; kk < k1; ++kk, ++n) {
                     const int s = n % stages;
                     const uint32_t ph = (uint32_t)(n / stages) & 1u;
@@ -201,7 +206,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     const uint32_t a_addr = smem_u32(base + s * stage_bytes);
                     const uint64_t adesc = sdesc_k_sw128(a_addr);
 #pragma unroll
-                    for (int part = 0; part < NP; ++part) {
+                    for (int part = 0; part < (fused ? 1 : NP); ++part) {
                         const uint64_t bdesc = sdesc_k_sw128(a_addr + kABytes + part * b_bytes);
 #pragma unroll
                         for (int j = 0; j < BK / 16; ++j) {
@@ -238,12 +243,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             const int nt = tile / p.n_mt, mt = tile % p.n_mt;
             const int n = nt * BM + n_local;
             const int cnt = p.streamk ? p.cta_of(tile * p.kb + p.kb - 1) - p.cta_of(tile * p.kb) + 1 : 1;
-            const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+            const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * p.acc_cols);
             float* part_tile = kp.part + ((int64_t)tile * p.P * BN) * BM + n_local;
+            const bool split_acc = p.acc_cols == 2 * BN;       // X_hi and X_lo products in separate columns
             for (int c0 = 0; c0 < BN; c0 += 16) {
                 uint32_t r[16];
                 tmem_ld_x16(tbase + (uint32_t)c0, r);
-                tmem_ld_wait();
+                if (split_acc) {
+                    uint32_t r2[16];
+                    tmem_ld_x16(tbase + (uint32_t)(BN + c0), r2);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
+                } else {
+                    tmem_ld_wait();
+                }
                 if (cnt == 1) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
@@ -321,6 +335,8 @@ bool get_encoder() {
     return g_encode != nullptr;
 }
 
+}  // namespace
+
 // Row-major bf16 [rows, cols] matrix, box of box_rows x 64 columns, 128-byte swizzle.
 bool make_tmap(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
     if (!get_encoder()) return false;
@@ -334,9 +350,12 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t cols, int
     return r == CUDA_SUCCESS;
 }
 
-int tmem_cols_for(int BN) {
+namespace {
+
+// Two accumulator buffers of acc_cols columns each.
+int tmem_cols_for(int acc_cols) {
     int c = 32;
-    while (c < 2 * BN) c <<= 1;
+    while (c < 2 * acc_cols) c <<= 1;
     return c;
 }
 
@@ -355,7 +374,10 @@ GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles) {
     // what sustains the weight stream at HBM latency under load
     const int stage_bytes = kABytes + np * p.BN * BK * 2;
     p.stages = std::max(2, std::min(kMaxStages, (kSmemLimit - kSmemExtra(kMaxStages)) / stage_bytes));
-    p.tmem_cols = tmem_cols_for(p.BN);
+    // the tensor core takes as long for an MMA of N = 16 as for N = 256: with a
+    // bf16 pair activation, hi and lo go through one MMA of N = 2 BN when it fits
+    p.acc_cols = (np == 2 && 2 * p.BN <= 256) ? 2 * p.BN : p.BN;
+    p.tmem_cols = tmem_cols_for(p.acc_cols);
     // tile mode when whole tiles balance the SMs to >= 90%, else stream-K
     const int waves = (p.tiles + num_sms - 1) / num_sms;
     const bool tiles_ok = force_tiles || (p.tiles >= num_sms && 10 * p.tiles >= 9 * waves * num_sms);

@@ -20,6 +20,7 @@ struct GemmPlan {
     int kb;                // 64-wide K blocks
     int tiles;             // n_mt * n_nt; tile index t = nt * n_mt + mt
     int stages, tmem_cols;
+    int acc_cols;          // TMEM columns per accumulator: 2 BN when X_hi and X_lo products share one MMA
     int mode, streamk;
     int grid;              // CTAs launched
     int T, G, P;           // stream-K: K blocks in all tiles, CTAs, most CTAs touching one tile

@@ -168,7 +168,8 @@ struct AttnArgs {
     void* out;                                       // [A, G, nH, hd]
     bf16* out_hi; bf16* out_lo;                      // optional bf16 pair of out (fp32 out only)
     float* part_o; float* part_ml;                   // workspace
-    int A, n_splits, chunk;                          // context splits of `chunk` keys (+1 block split)
+    int A, n_splits, chunk;                          // context splits of `chunk` keys
+    int S1;                                          // partial slots per (b, h): set by the kernel path
     int32_t* status;
     double kv_bytes, flops;                          // algorithmic work (for the timers)
 };
@@ -185,6 +186,12 @@ struct WalkArgs {
 };
 cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s);
 // The whole walk in one cooperative launch (one CTA per SM, bounded grid barriers).
+namespace tc {
+// Markov walk with the bias on tensor cores (walk_tc.cu).
+bool walk_tc_supported(const dspark_model* m, int A);
+cudaError_t launch_walk_tc(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
+                           float* cand_val, int32_t* cand_idx, uint32_t* arrivals, int A, cudaStream_t s);
+}  // namespace tc
 bool walk_persistent_supported(const dspark_model* m, int A);
 int walk_persistent_blocks(const dspark_model* m);
 cudaError_t launch_walk_persistent(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,

@@ -286,13 +286,16 @@ const char* dspark_last_error(void);
  * summed device milliseconds, launch count, bytes and flops (either of the
  * last two may be NULL), and forgets them.
  */
-#define DSPARK_TIMER_GEMM        0  /* the layers' weight GEMMs: [q;k], o, [gate;up], down */
+#define DSPARK_TIMER_GEMM_QK     0  /* per layer: x @ [q_proj; k_proj]^T */
 #define DSPARK_TIMER_LM_HEAD     1  /* lm-head GEMM with softcap */
 #define DSPARK_TIMER_ATTENTION   2  /* KV-injection attention (partials + merge) */
-#define DSPARK_TIMER_WALK        3  /* Markov walk steps */
+#define DSPARK_TIMER_WALK        3  /* Markov walk */
 #define DSPARK_TIMER_KV_PROJECT  4  /* context K/V projection GEMM + epilogue */
 #define DSPARK_TIMER_ROWS        5  /* embedding, norms/RoPE/residual epilogues, confidence */
-#define DSPARK_TIMER_KINDS       6
+#define DSPARK_TIMER_GEMM_O      6  /* per layer: attention out @ o_proj^T */
+#define DSPARK_TIMER_GEMM_GU     7  /* per layer: x @ [gate; up]^T */
+#define DSPARK_TIMER_GEMM_DOWN   8  /* per layer: gelu(gate) * up @ down^T */
+#define DSPARK_TIMER_KINDS       9
 uint64_t dspark_kernel_launches(void);
 int dspark_timer_enable(int enable);
 int dspark_timer_read(int kind, double* total_ms, int64_t* launches, double* bytes, double* flops);

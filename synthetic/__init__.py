@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "ModelShape", "Workload", "WORKLOADS", "workload", "make_weights",
-    "make_round_inputs", "make_append_schedule", "quantize_affine4", "weight_names",
+    "make_round_inputs", "round_meta", "make_append_schedule", "quantize_affine4", "weight_names",
     "QUANTIZED_MATRICES",
 ]
 
@@ -228,16 +228,9 @@ def make_weights(m: ModelShape, seed: int, literal: bool = False, unit_attention
     return out
 
 
-def make_round_inputs(w: Workload, rows: Optional[List[int]] = None) -> Dict[str, torch.Tensor]:
-    """Context hiddens, positions, lengths and anchors of one draft round.
-
-    Returns CPU tensors: ``hidden`` [A, Lmax, H] (rows past a row's length are
-    padding drawn like the rest), ``ctx_len`` [A] int32, ``pos0`` [A] int32
-    (absolute position of context row 0), ``block_pos`` [A] int32 (= pos0 +
-    ctx_len: the block follows the context), ``anchors`` [A] int32 uniform in
-    [0, V-1). ``rows`` selects a subset of the A rows (same values as in the
-    full draw), for checking sampled rows of a large workload.
-    """
+def round_meta(w: Workload):
+    """Per-row context lengths, start positions and anchors of a round
+    (int64 CPU tensors [A]); the first draws of make_round_inputs."""
     m = w.model
     A = w.rows
     g = torch.Generator(device="cpu")
@@ -251,6 +244,22 @@ def make_round_inputs(w: Workload, rows: Optional[List[int]] = None) -> Dict[str
     else:
         pos0 = torch.zeros(A, dtype=torch.int64)
     anchors = torch.randint(0, m.vocab_size - 1, (A,), generator=g, dtype=torch.int64)
+    return lens, pos0, anchors
+
+
+def make_round_inputs(w: Workload, rows: Optional[List[int]] = None) -> Dict[str, torch.Tensor]:
+    """Context hiddens, positions, lengths and anchors of one draft round.
+
+    Returns CPU tensors: ``hidden`` [A, Lmax, H] (rows past a row's length are
+    padding drawn like the rest), ``ctx_len`` [A] int32, ``pos0`` [A] int32
+    (absolute position of context row 0), ``block_pos`` [A] int32 (= pos0 +
+    ctx_len: the block follows the context), ``anchors`` [A] int32 uniform in
+    [0, V-1). ``rows`` selects a subset of the A rows (same values as in the
+    full draw), for checking sampled rows of a large workload.
+    """
+    m = w.model
+    A = w.rows
+    lens, pos0, anchors = round_meta(w)
     sel = list(range(A)) if rows is None else list(rows)
     Lmax = int(lens[sel].max()) if w.ragged_min > 0 else w.ctx_len
     hid = []

@@ -157,6 +157,24 @@ def test_strong_markov_walk_and_threshold():
     assert (ref["tokens"] != np.argmax(ref["base_logits"], -1)).any()
 
 
+@pytest.mark.parametrize("A", [1, 8, 9])
+def test_rank64_markov_walk(A):
+    """markov_rank 64 with a strong bias: the tensor-core walk (A <= 8) and the
+    CUDA-core persistent walk (A = 9) against the oracle's teacher-forced walk."""
+    m = small_model(dtype="bf16", markov_rank=64)
+    cpu, W, model = build(m, 41, markov_scale=30.0)
+    g = torch.Generator().manual_seed(40 + A)
+    lens = [int(x) for x in torch.randint(1, 97, (A,), generator=g)]
+    pos0 = [int(x) for x in torch.randint(0, 500, (A,), generator=g)]
+    hid = torch.randn(A, max(lens), m.hidden_size, generator=g).to(torch.bfloat16)
+    cache = _project_into_cache(model, hid, lens, pos0)
+    kv = O.project_context_kv(W, hid, pos0, lengths=lens)
+    anchors = [int(x) for x in torch.randint(0, m.vocab_size - 1, (A,), generator=g)]
+    block_pos = [p + L for p, L in zip(pos0, lens)]
+    out, ref = _round_and_compare(m, W, model, cache, kv, anchors, block_pos, lens, f"rank 64, A={A}")
+    assert (ref["tokens"] != np.argmax(ref["base_logits"], -1)).any()
+
+
 def test_rank0_no_confidence_head():
     m = small_model(dtype="bf16", markov_rank=0, enable_confidence_head=False, confidence_head_with_markov=False)
     cpu, W, model = build(m, 31)
