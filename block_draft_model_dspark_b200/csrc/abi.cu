@@ -147,7 +147,7 @@ struct Carve {
 struct DraftPlan {
     int M, attn_splits, attn_chunk, walk_blocks;
     bool pairs;   // GEMM inputs also kept as bf16 (hi, lo) pairs for the tensor-core GEMMs
-    size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx;
+    size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx, walk_keys;
     size_t x_hi, x_lo, ao_hi, ao_lo, act_hi, act_lo, conf, gscr, gscr_bytes, total;
 };
 
@@ -184,6 +184,7 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.part_ml = c.take((size_t)A * d.nH * S1 * d.gamma * 2 * 4);
     p.prev = c.take((size_t)A * 4);
     p.ticket = c.take(256);
+    p.walk_keys = c.take((size_t)d.gamma * A * 8);              // tensor-core walk: per (step, row) maximum
     p.walk_val = c.take((size_t)2 * p.walk_blocks * A * 4);     // two step-parity buffers (persistent walk)
     p.walk_idx = c.take((size_t)2 * p.walk_blocks * A * 4);
     const size_t pb = p.pairs ? 2 : 0;
@@ -514,6 +515,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     cudaError_t e = gemm_scratch_reset(sc, p.gscr_bytes, s);
     // the persistent walk's grid-barrier counter
     if (e == cudaSuccess) e = cudaMemsetAsync(at<uint32_t>(ws, p.ticket), 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(at<void>(ws, p.walk_keys), 0, (size_t)d.gamma * A * 8, s);
     if (e == cudaSuccess) e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
     for (int l = 0; l < d.Lyr && e == cudaSuccess; ++l) {
         const LayerRef& L = m->layers[l];
@@ -541,7 +543,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
                                               : (double)d.V * d.r * esize(d.dtype)) : 0.0;
         if (tc::walk_tc_supported(m, A)) {
             KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
-            e = tc::launch_walk_tc(m, U, anchors, tokens, wa.part_val, wa.part_idx, wa.ticket, A, s);
+            e = tc::launch_walk_tc(m, U, anchors, tokens, at<unsigned long long>(ws, p.walk_keys), wa.ticket, A, s);
         } else if (walk_persistent_supported(m, A)) {
             KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
             e = launch_walk_persistent(m, U, anchors, tokens, wa.part_val, wa.part_idx, wa.ticket, A, s);

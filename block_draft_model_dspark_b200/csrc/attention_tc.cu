@@ -21,13 +21,16 @@
 // are in flight while tile t is converted and multiplied; per 64 keys at
 // hd = 256 the tensor cores run 16 (S) + 4 (P V) MMAs.
 //
-// Warp roles (288 threads): warps 0-3 run the softmax, warps 4-7 convert K
-// and V tiles (and zero the rows past the last key: stale cache bytes could be
-// NaN, and P = 0 times NaN still poisons the accumulator), warp 8 issues TMA
-// loads and MMAs. The pipeline overlaps the next K tile's load, conversion and
-// S product with the current tile's softmax, and the next V tile with the
-// current P V product. Every wait is bounded.
-// Shared memory at hd = 256: Q 64 KB, K 2 x 32 KB, V 2 x 32 KB, P 16 KB.
+// Warp roles (544 threads): warps 0-7 run the softmax, two threads per query
+// row (warps w and w + 4 share TMEM lanes 32 (w % 4) ..; each takes 32 of the
+// tile's 64 columns and half of O's columns; the row max is exchanged through
+// shared memory), warps 8-15 convert K and V tiles (and zero the rows past the
+// last key: stale cache bytes could be NaN, and P = 0 times NaN still poisons
+// the accumulator), warp 16 issues TMA loads and MMAs. K, V and P have two
+// slots each and S two TMEM buffers, so tile t + 1's load, conversion and S
+// product and tile t - 1's P V product all overlap tile t's softmax; the
+// softmax waits for P V of tile t - 1 only to rescale O (rare). Every wait is
+// bounded. Shared memory at hd = 256: Q 64 KB, K, V 2 x 32 KB each, P 2 x 16 KB.
 //
 // The CTA writes its unnormalised O with (max, sum) per query row: the split
 // layout the merge kernel reads. The last split of each (b, g) also takes the
@@ -50,10 +53,10 @@ cudaError_t launch_attention_merge(const dspark_model* m, const AttnArgs& a, cud
 namespace tc {
 namespace {
 
-constexpr int kThreads = 288;
-constexpr int kSoftThreads = 128;    // warps 0-3
-constexpr int kConvThreads = 128;    // warps 4-7
-constexpr int kIssuerWarp = 8;
+constexpr int kThreads = 544;
+constexpr int kSoftThreads = 256;    // warps 0-7
+constexpr int kConvThreads = 256;    // warps 8-15
+constexpr int kIssuerWarp = 16;
 constexpr int KT = 64;               // keys per tile
 constexpr int QROWS = 128;           // MMA M
 constexpr float kRescale = 5.0f;     // natural-log headroom before the running max is raised
@@ -88,6 +91,13 @@ __device__ __forceinline__ void convert_tile(uint8_t* tile, int nsub, int nvalid
     }
 }
 
+// A bounded mbarrier wait whose outcome is the same in every lane of the warp
+// (the softmax warps run warp-collective tcgen05.ld and votes after it).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status) {
+    const bool w = mbar_wait(bar, parity, abort_flag, status);
+    return __all_sync(0xffffffffu, w);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb, AttnTcParams P) {
@@ -98,18 +108,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     uint8_t* sQ = base;                                   // nsub x [128 rows x 128 B] fp16
     uint8_t* sK = sQ + nsub * QROWS * 128;                // 2 slots x tile
     uint8_t* sV = sK + 2 * tile_sz;                       // 2 slots x tile
-    uint8_t* sP = sV + 2 * tile_sz;                       // [128 rows x 128 B]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + QROWS * 128);
+    uint8_t* sP = sV + 2 * tile_sz;                       // 2 slots x [128 rows x 128 B]
+    float* red = reinterpret_cast<float*>(sP + 2 * QROWS * 128);   // [2 halves][128 rows] row maxima / sums
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * QROWS);
     uint64_t* kfull = bars + 0;      // [2] K tile landed in the slot (TMA)
     uint64_t* vfull = bars + 2;      // [2] V tile landed in the slot (TMA)
     uint64_t* kready = bars + 4;     // [2] K tile of the slot converted (128 arrivals)
     uint64_t* vready = bars + 6;     // [2] V tile of the slot converted (128 arrivals)
     uint64_t* sdone = bars + 8;      // [2] S product of the tile in that buffer done (its K slot free)
     uint64_t* sfree = bars + 10;     // [2] softmax has read the S buffer (128 arrivals)
-    uint64_t* pready = bars + 12;    // P written (128 arrivals)
-    uint64_t* odone = bars + 13;     // P V product done (its V slot and P free, O settled)
-    uint64_t* spare = bars + 14;     // teardown: MMAs in flight after an abort
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+    uint64_t* pready = bars + 12;    // [2] P slot written (256 arrivals)
+    uint64_t* odone = bars + 14;     // [2] P V product of the tile in that P slot done (its V slot free, O settled)
+    uint64_t* spare = bars + 16;     // teardown: MMAs in flight after an abort
+    uint64_t* xw = bars + 17;        // row-max exchange: both halves wrote (256 arrivals)
+    uint64_t* xr = bars + 18;        // row-max exchange: both halves read (256 arrivals)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -125,7 +138,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         }
         mbar_init(&sdone[0], 1); mbar_init(&sdone[1], 1);
         mbar_init(&sfree[0], kSoftThreads); mbar_init(&sfree[1], kSoftThreads);
-        mbar_init(pready, kSoftThreads); mbar_init(odone, 1); mbar_init(spare, 1);
+        mbar_init(&pready[0], kSoftThreads); mbar_init(&pready[1], kSoftThreads);
+        mbar_init(&odone[0], 1); mbar_init(&odone[1], 1); mbar_init(spare, 1);
+        mbar_init(xw, kSoftThreads); mbar_init(xr, kSoftThreads);
         *abort_flag = 0;
         mbar_fence_init();
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmKb); prefetch_tmap(&tmVb);
@@ -209,45 +224,69 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 load(sK + t * tile_sz, &kfull[t], false, t); ++nk[t];
                 load(sV + t * tile_sz, &vfull[t], true, t); ++nv[t];
             }
+            // Loads wait only for their slot to be free; the issuer never blocks on them:
+            // every wait below keeps issuing the loads whose slot has come free.
+            int kn = min(2, nt), vn = min(2, nt);             // next K / V tile to load
+            int qk_issued = 0, pv_issued = 0;                 // S / P V products issued
+            auto service = [&]() {
+                // K(kn) into slot kn % 2 once S(kn - 2) has read it
+                while (kn < nt && kn - 2 < qk_issued && mbar_try_wait(&sdone[kn & 1], (uint32_t)((kn - 2) >> 1) & 1u)) {
+                    load(sK + (kn & 1) * tile_sz, &kfull[kn & 1], false, kn); ++nk[kn & 1]; ++kn;
+                }
+                // V(vn) into slot vn % 2 once P(vn - 2) V(vn - 2) has read it
+                while (vn < nt && vn - 2 < pv_issued && mbar_try_wait(&odone[vn & 1], (uint32_t)((vn - 2) >> 1) & 1u)) {
+                    load(sV + (vn & 1) * tile_sz, &vfull[vn & 1], true, vn); ++nv[vn & 1]; ++vn;
+                }
+            };
+            auto wait_serving = [&](uint64_t* bar, uint32_t parity) -> bool {
+                const uint64_t t0w = global_timer_ns();
+                while (!mbar_try_wait(bar, parity)) {
+                    service();
+                    if (*abort_flag) return false;
+                    if (global_timer_ns() - t0w > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        atomicOr(P.status, DSPARK_DEV_WAIT_TIMEOUT);
+                        return false;
+                    }
+                }
+                return true;
+            };
+            const uint32_t qa = smem_u32(sQ);
             for (int t = 0; t <= nt && ok; ++t) {
                 const int sl = t & 1;
                 if (t < nt) {
                     // S(t) = Q K(t)^T into buffer t % 2
-                    if (!mbar_wait(&kready[sl], (uint32_t)(t >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
-                    if (t >= 2 && !mbar_wait(&sfree[sl], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+                    if (!wait_serving(&kready[sl], (uint32_t)(t >> 1) & 1u)) { ok = false; break; }
+                    if (t >= 2 && !wait_serving(&sfree[sl], (uint32_t)((t - 2) >> 1) & 1u)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK + sl * tile_sz);
+                    const uint32_t ka = smem_u32(sK + sl * tile_sz);
+                    const uint32_t d = tmem + (uint32_t)(sl * KT);
+#pragma unroll 4
                     for (int j = 0; j < hd / 16; ++j) {
                         const uint64_t ad = sdesc_k_sw128(qa + (j >> 2) * QROWS * 128 + (j & 3) * 32);
                         const uint64_t bd = sdesc_k_sw128(ka + (j >> 2) * KT * 128 + (j & 3) * 32);
-                        mma_bf16(tmem + (uint32_t)(sl * KT), ad, bd, idesc_qk, j > 0 ? 1u : 0u);
+                        mma_bf16(d, ad, bd, idesc_qk, j > 0 ? 1u : 0u);
                     }
                     mma_commit(&sdone[sl]);
+                    qk_issued = t + 1;
                 }
                 if (t >= 1) {
                     // O += P(t-1) V(t-1)
                     const int u = t - 1;
-                    if (!mbar_wait(pready, (uint32_t)u & 1u, abort_flag, P.status) ||
-                        !mbar_wait(&vready[u & 1], (uint32_t)(u >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+                    if (!wait_serving(&pready[u & 1], (uint32_t)(u >> 1) & 1u) ||
+                        !wait_serving(&vready[u & 1], (uint32_t)(u >> 1) & 1u)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t pa = smem_u32(sP), va = smem_u32(sV + (u & 1) * tile_sz);
+                    const uint32_t pa = smem_u32(sP + (u & 1) * QROWS * 128), va = smem_u32(sV + (u & 1) * tile_sz);
+#pragma unroll
                     for (int j = 0; j < KT / 16; ++j) {
                         const uint64_t ad = sdesc_k_sw128(pa + j * 32);
                         const uint64_t bd = sdesc_mn_sw128(va + j * 2048, KT * 128);
                         mma_bf16(tO, ad, bd, idesc_pv, (u > 0 || j > 0) ? 1u : 0u);
                     }
-                    mma_commit(odone);
+                    mma_commit(&odone[u & 1]);
+                    pv_issued = u + 1;
                 }
-                if (t + 2 < nt) {
-                    // K(t+2) into slot t % 2 once S(t) has read it
-                    if (!mbar_wait(&sdone[sl], (uint32_t)(t >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
-                    load(sK + sl * tile_sz, &kfull[sl], false, t + 2); ++nk[sl];
-                }
-                if (t >= 1 && t + 1 < nt) {
-                    // V(t+1) into slot (t+1) % 2 once P(t-1) V(t-1) has read it
-                    if (!mbar_wait(odone, (uint32_t)(t - 1) & 1u, abort_flag, P.status)) { ok = false; break; }
-                    load(sV + ((t + 1) & 1) * tile_sz, &vfull[(t + 1) & 1], true, t + 1); ++nv[(t + 1) & 1];
-                }
+                service();
             }
             // teardown after an abort: copies and MMAs in flight land first (bounded)
             if (!ok) {
@@ -262,7 +301,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 if (!drained) atomicOr(P.status, DSPARK_DEV_WAIT_TIMEOUT);
             }
         }
-    } else if (warp >= 4) {
+    } else if (warp >= kSoftThreads / 32) {
         // ------------------------------------------------------------ converters
         const int ct = tid - kSoftThreads;
         for (int t = 0; t < nt && ok; ++t) {
@@ -280,84 +319,105 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             mbar_arrive(&vready[sl]);
         }
     } else {
-        // ------------------------------------------------------------ softmax (thread = query row)
-        const int r = tid;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        float m_run = -INFINITY, l_run = 0.f;
+        // ------------------------------------------------------------ softmax (two threads per query row)
+        const int r = tid & (QROWS - 1);                   // query row = TMEM lane
+        const int half = tid >> 7;                         // S columns [32 half, +32), O columns [hd/2 half, +hd/2)
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const int oc0 = half * (hd / 2);
+        float m_run = -INFINITY, l_run = 0.f;              // l_run: this half's columns
         for (int t = 0; t < nt && ok; ++t) {
             int row, nvalid; bool blk;
             tile_rows(t, &row, &nvalid, &blk);
-            const uint32_t tS = tmem + (uint32_t)((t & 1) * KT) + lane_off;
-            if (!mbar_wait(&sdone[t & 1], (uint32_t)(t >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+            const int sl = t & 1;
+            const uint32_t tS = tmem + (uint32_t)(sl * KT) + lane_off + (uint32_t)(half * 32);
+            const int cbase = half * 32;                   // first key of this thread's columns
+            if (!warp_wait(&sdone[sl], (uint32_t)(t >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
-            float mx = -INFINITY;
-            for (int c = 0; c < KT; c += 16) {
-                uint32_t u[16];
-                tmem_ld_x16(tS + c, u);
-                tmem_ld_wait();
+            uint32_t u0[16], u1[16];
+            tmem_ld_x16(tS, u0);
+            tmem_ld_x16(tS + 16, u1);
+            tmem_ld_wait();
+            float sv[32];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) if (c + j < nvalid) mx = fmaxf(mx, __uint_as_float(u[j]));
+            for (int j = 0; j < 16; ++j) { sv[j] = __uint_as_float(u0[j]); sv[16 + j] = __uint_as_float(u1[j]); }
+            if (nvalid < KT) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) if (cbase + j >= nvalid) sv[j] = -INFINITY;
             }
-            // P(t-1) V(t-1) must be done before O is rescaled and P rewritten
-            if (t >= 1 && !mbar_wait(odone, (uint32_t)(t - 1) & 1u, abort_flag, P.status)) { ok = false; break; }
-            tc_fence_after();
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, sv[j]);
+            // exchange with the other half of the row (mbarriers: every wait stays bounded)
+            if (t >= 1 && !warp_wait(xr, (uint32_t)(t - 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+            red[half * QROWS + r] = mx;
+            mbar_arrive(xw);
+            if (!warp_wait(xw, (uint32_t)t & 1u, abort_flag, P.status)) { ok = false; break; }
+            mx = fmaxf(mx, red[(half ^ 1) * QROWS + r]);
+            mbar_arrive(xr);
             const bool need = t > 0 && mx > m_run + kRescale;
             if (t == 0) m_run = mx;
             if (__any_sync(0xffffffffu, need)) {
+                // O holds tiles up to t - 1 at the old max: P(t-1) V(t-1) must have landed
+                if (t >= 1 && !warp_wait(&odone[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+                tc_fence_after();
                 const float f = need ? __expf(m_run - mx) : 1.f;
                 if (need) { l_run *= f; m_run = mx; }
-                for (int c = 0; c < hd; c += 16) {
+                for (int c = 0; c < hd / 2; c += 16) {
                     uint32_t u[16];
-                    tmem_ld_x16(tO + lane_off + c, u);
+                    tmem_ld_x16(tO + lane_off + (uint32_t)(oc0 + c), u);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * f);
-                    tmem_st_x16(tO + lane_off + c, u);
+                    tmem_st_x16(tO + lane_off + (uint32_t)(oc0 + c), u);
                 }
                 tmem_st_wait();
             }
+            // P slot t % 2 was last read by P(t-2) V(t-2)
+            if (t >= 2 && !warp_wait(&odone[sl], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
             float lsum = 0.f;
-            for (int c = 0; c < KT; c += 16) {
-                uint32_t u[16];
-                tmem_ld_x16(tS + c, u);
-                tmem_ld_wait();
-                float p[16];
+            uint8_t* pslot = sP + sl * QROWS * 128;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    p[j] = c + j < nvalid ? __expf(__uint_as_float(u[j]) - m_run) : 0.f;
-                    lsum += p[j];
-                }
+            for (int q = 0; q < 4; ++q) {                  // four 16-byte chunks of 8 keys
+                float p[8];
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int k = c + hf * 8;                 // first key of this 16-byte chunk
-                    const int off = r * 128 + (((k >> 3) ^ (r & 7)) * 16);
-                    *reinterpret_cast<uint4*>(sP + off) =
-                        make_uint4(pack_half2(p[hf * 8 + 0], p[hf * 8 + 1]), pack_half2(p[hf * 8 + 2], p[hf * 8 + 3]),
-                                   pack_half2(p[hf * 8 + 4], p[hf * 8 + 5]), pack_half2(p[hf * 8 + 6], p[hf * 8 + 7]));
-                }
+                for (int j = 0; j < 8; ++j) { p[j] = __expf(sv[q * 8 + j] - m_run); lsum += p[j]; }
+                const int chunk = (cbase >> 3) + q;
+                *reinterpret_cast<uint4*>(pslot + r * 128 + ((chunk ^ (r & 7)) * 16)) =
+                    make_uint4(pack_half2(p[0], p[1]), pack_half2(p[2], p[3]), pack_half2(p[4], p[5]), pack_half2(p[6], p[7]));
             }
             l_run += lsum;
             tc_fence_before();
-            mbar_arrive(&sfree[t & 1]);                        // S buffer read
+            mbar_arrive(&sfree[sl]);                           // S buffer read
             fence_async_shared();
-            mbar_arrive(pready);                               // P written
+            mbar_arrive(&pready[sl]);                          // P written
         }
         // ---- this split's state: unnormalised O and (max, sum) per query row
         const bool any = nt > 0;
-        if (any && ok && !mbar_wait(odone, (uint32_t)(nt - 1) & 1u, abort_flag, P.status)) ok = false;
+        if (any && ok && !warp_wait(&odone[(nt - 1) & 1], (uint32_t)((nt - 1) >> 1) & 1u, abort_flag, P.status)) ok = false;
         tc_fence_after();
-        if (r < nq) {
+        // the row's sum = both halves' sums (same running max): one more exchange
+        float l_tot = l_run;
+        if (any && ok) {
+            if (!warp_wait(xr, (uint32_t)(nt - 1) & 1u, abort_flag, P.status)) ok = false;
+            if (ok) {
+                red[half * QROWS + r] = l_run;
+                mbar_arrive(xw);
+                if (!warp_wait(xw, (uint32_t)nt & 1u, abort_flag, P.status)) ok = false;
+                else l_tot = l_run + red[(half ^ 1) * QROWS + r];
+            }
+        }
+        if (r < nq && half == 0) {
             const int i = r / P.grp, h = g * P.grp + r % P.grp;
             const int64_t prow = ((int64_t)(b * P.nH + h) * P.S1 + split) * P.G + i;
             P.part_ml[prow * 2] = any ? m_run : -INFINITY;
-            P.part_ml[prow * 2 + 1] = any ? l_run : 0.f;
+            P.part_ml[prow * 2 + 1] = any ? l_tot : 0.f;
         }
         if (any && ok) {
             const int i = r / P.grp, h = g * P.grp + r % P.grp;
-            float* dst = P.part_o + (((int64_t)(b * P.nH + h) * P.S1 + split) * P.G + i) * hd;
-            for (int c = 0; c < hd; c += 16) {
+            float* dst = P.part_o + (((int64_t)(b * P.nH + h) * P.S1 + split) * P.G + i) * hd + oc0;
+            for (int c = 0; c < hd / 2; c += 16) {
                 uint32_t u[16];
-                tmem_ld_x16(tO + lane_off + c, u);
+                tmem_ld_x16(tO + lane_off + (uint32_t)(oc0 + c), u);
                 tmem_ld_wait();
                 if (r < nq) {
 #pragma unroll
@@ -398,8 +458,9 @@ bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd
 
 size_t attn_tc_smem(int hd) {
     const int nsub = hd / 64;
-    // Q, K (2 slots), V (2 slots), P, then 15 barriers + TMEM slot + abort flag; 1 KB alignment slack
-    return (size_t)nsub * QROWS * 128 + 4 * (size_t)nsub * KT * 128 + QROWS * 128 + 192 + 1024;
+    // Q, K (2 slots), V (2 slots), P (2 slots), row maxima, then 17 barriers + TMEM slot + abort
+    // flag; 1 KB alignment slack
+    return (size_t)nsub * QROWS * 128 + 4 * (size_t)nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 192 + 1024;
 }
 
 }  // namespace

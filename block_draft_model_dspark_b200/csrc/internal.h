@@ -190,7 +190,7 @@ namespace tc {
 // Markov walk with the bias on tensor cores (walk_tc.cu).
 bool walk_tc_supported(const dspark_model* m, int A);
 cudaError_t launch_walk_tc(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
-                           float* cand_val, int32_t* cand_idx, uint32_t* arrivals, int A, cudaStream_t s);
+                           unsigned long long* keys, uint32_t* arrivals, int A, cudaStream_t s);
 }  // namespace tc
 bool walk_persistent_supported(const dspark_model* m, int A);
 int walk_persistent_blocks(const dspark_model* m);

@@ -13,8 +13,10 @@
 // products are exact in fp32, so the bias differs from a CUDA-core sum only
 // in the order of its fp32 additions. Then one thread per (tile row, b)
 // adds U[b, k, v] and keeps a running argmax; warp and CTA reductions give
-// one candidate per row b, and a grid barrier (bounded wait) lets every CTA
-// reduce all candidates in CTA order and agree on the step's token.
+// one candidate per row b, folded into one 64-bit key per (step, row) with an
+// atomic maximum (the value's bits made order-preserving, then the
+// complemented index: the largest value, lowest index on ties), and after a
+// grid barrier (bounded wait) every CTA reads the step's token from it.
 //
 // markov_w2 does not change during the walk: most of the CTA's tiles are
 // TMA-loaded once and stay in shared memory; the rest (at most 2 * kSlots)
@@ -46,9 +48,8 @@ struct WtcArgs {
     const int32_t* anchors;    // [A]
     const bf16* w1;            // markov_w1 [V, 64]
     int32_t* tokens;           // [A, G]
-    float* cand_val;           // [2][grid][A]
-    int32_t* cand_idx;         // [2][grid][A]
     uint32_t* arrivals;        // grid-barrier counter, zero at entry
+    unsigned long long* keys;  // [G][A] packed (value, index) maxima of each step, zero at entry
     int A, G, V;
     int tiles_total;           // ceil(V / 128)
     int res_max;               // resident tiles a CTA may hold
@@ -62,6 +63,16 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// (value, index) as one 64-bit key whose unsigned maximum is the largest
+// value with the lowest index: the value's bits made order-preserving, then
+// the complemented index. NaN maps to 0 and never wins.
+__device__ __forceinline__ unsigned long long pack_key(float v, int idx) {
+    const uint32_t u = __float_as_uint(v);
+    uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    if (v != v) ord = 0u;
+    return ((unsigned long long)ord << 32) | (unsigned long long)(~(uint32_t)idx);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -94,7 +105,7 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
 
     if (tid == 0) {
         s_fail = 0;
-        for (int i = 0; i < 2 + 2 * kSlots; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 2 + 2 * kSlots; ++i) mbar_init(&bars[i], i == 1 ? 2 : 1);   // bar_mma: two issuers
         mbar_fence_init();
         prefetch_tmap(&tmW2);
         // markov_w2 is a weight: requested before waiting on the previous kernel
@@ -154,16 +165,27 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
             for (int b = 0; b < kRows; ++b)
                 uval[i][b] = (t < nt && b < A && v < V) ? __ldcs(a.U + ((int64_t)b * G + step) * V + v) : 0.f;
         }
-        // ---- bias tiles on the tensor cores (one thread)
+        // ---- bias tiles on the tensor cores: two issuing threads (warps 0 and 1) share
+        // the resident tiles; thread 0 also runs the streamed ones
+        const int half_res = nres / 2;
+        auto mma_tile = [&](const uint8_t* src, int t) {
+            const uint64_t adesc = sdesc_k_sw128(smem_u32(src));
+            const uint64_t bdesc = sdesc_k_sw128(smem_u32(sE));
+            const uint32_t d = tmem + (uint32_t)(t * kN);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) mma_bf16(d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, j > 0 ? 1u : 0u);
+        };
+        if (tid == 32) {
+            tc_fence_after();
+            if (step == 0 && !mbar_wait(bar_res, 0u, abort_flag, a.status)) ok = false;
+            if (ok) {
+                tc_fence_after();
+                for (int t = half_res; t < nres; ++t) mma_tile(sRes + t * kTileBytes, t);
+                mma_commit(bar_mma);
+            }
+        }
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t bdesc = sdesc_k_sw128(smem_u32(sE));
-            auto mma_tile = [&](const uint8_t* src, int t) {
-                const uint64_t adesc = sdesc_k_sw128(smem_u32(src));
-                for (int j = 0; j < 4; ++j)
-                    mma_bf16(tmem + (uint32_t)(t * kN), adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
-                             j > 0 ? 1u : 0u);
-            };
             const int q0 = step * ns, q1 = q0 + ns;
             const int q_pre = min(q_load, q1);         // streamed tiles already requested
             for (int q = q0; q < q_pre && ok; ++q) {
@@ -180,7 +202,7 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
             }
             if (ok && step == 0 && !mbar_wait(bar_res, 0u, abort_flag, a.status)) ok = false;
             if (ok) tc_fence_after();
-            for (int t = 0; ok && t < nres; ++t) mma_tile(sRes + t * kTileBytes, t);
+            for (int t = 0; ok && t < half_res; ++t) mma_tile(sRes + t * kTileBytes, t);
             for (int q = q_pre; ok && q < q1; ++q) {
                 if (!mbar_wait(&full[q % kSlots], (uint32_t)(q / kSlots) & 1u, abort_flag, a.status)) { ok = false; break; }
                 tc_fence_after();
@@ -225,14 +247,11 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
             if (lane == 0) { rv[warp][b] = bv; ri[warp][b] = bi; }
         }
         __syncthreads();
-        float* cval = a.cand_val + (size_t)(step & 1) * nblk * A;
-        int32_t* cidx = a.cand_idx + (size_t)(step & 1) * nblk * A;
         if (tid < A) {
             float bv = -INFINITY;
             int bi = 0x7fffffff;
             for (int w = 0; w < kWarps; ++w) argmax_merge(bv, bi, rv[w][tid], ri[w][tid]);
-            cval[(size_t)blockIdx.x * A + tid] = bv;
-            cidx[(size_t)blockIdx.x * A + tid] = bi;
+            if (bi != 0x7fffffff) atomicMax(&a.keys[(size_t)step * A + tid], pack_key(bv, bi));
         }
         __syncthreads();
         // ---- grid barrier (bounded), then every CTA reduces all candidates in CTA order
@@ -250,20 +269,16 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
         }
         __syncthreads();
         if (s_fail) { ok = false; break; }
-        for (int b = warp; b < A; b += kWarps) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int c = lane; c < nblk; c += 32)
-                argmax_merge(bv, bi, __ldcg(&cval[(size_t)c * A + b]), __ldcg(&cidx[(size_t)c * A + b]));
-            warp_argmax(bv, bi);
-            if (lane == 0) {
-                if (bi < 0 || bi >= V) {               // only if a row was all NaN
-                    if (blockIdx.x == 0) atomicOr(a.status, DSPARK_DEV_BAD_TOKEN);
-                    bi = 0;
-                }
-                prev[b] = bi;
-                if (blockIdx.x == 0) a.tokens[b * G + step] = bi;
+        // the step's maximum over all CTAs is one 64-bit word per row
+        if (tid < A) {
+            const unsigned long long key = __ldcg(&a.keys[(size_t)step * A + tid]);
+            int bi = (int)~(uint32_t)(key & 0xffffffffull);
+            if ((key >> 32) == 0ull || bi < 0 || bi >= V) {   // only if a row was all NaN
+                if (blockIdx.x == 0) atomicOr(a.status, DSPARK_DEV_BAD_TOKEN);
+                bi = 0;
             }
+            prev[tid] = bi;
+            if (blockIdx.x == 0) a.tokens[tid * G + step] = bi;
         }
         __syncthreads();
     }
@@ -306,13 +321,13 @@ bool walk_tc_supported(const dspark_model* m, int A) {
 }
 
 cudaError_t launch_walk_tc(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
-                           float* cand_val, int32_t* cand_idx, uint32_t* arrivals, int A, cudaStream_t s) {
+                           unsigned long long* keys, uint32_t* arrivals, int A, cudaStream_t s) {
     const Dims& d = m->d;
     CUtensorMap tw;
     if (!make_tmap(&tw, m->w2.w, d.V, 64, 128)) return cudaErrorInvalidValue;
     WtcArgs wa{};
     wa.U = U; wa.anchors = anchors; wa.w1 = static_cast<const bf16*>(m->w1); wa.tokens = tokens;
-    wa.cand_val = cand_val; wa.cand_idx = cand_idx; wa.arrivals = arrivals;
+    wa.keys = keys; wa.arrivals = arrivals;
     wa.A = A; wa.G = d.gamma; wa.V = d.V;
     wa.tiles_total = (d.V + 127) / 128;
     wa.res_max = resident_tiles();
