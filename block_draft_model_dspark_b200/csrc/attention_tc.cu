@@ -21,12 +21,13 @@
 // are in flight while tile t is converted and multiplied; per 64 keys at
 // hd = 256 the tensor cores run 16 (S) + 4 (P V) MMAs.
 //
-// Warp roles (544 threads): warps 0-7 run the softmax, two threads per query
+// Warp roles (576 threads): warps 0-7 run the softmax, two threads per query
 // row (warps w and w + 4 share TMEM lanes 32 (w % 4) ..; each takes 32 of the
 // tile's 64 columns and half of O's columns; the row max is exchanged through
 // shared memory), warps 8-15 convert K and V tiles (and zero the rows past the
 // last key: stale cache bytes could be NaN, and P = 0 times NaN still poisons
-// the accumulator), warp 16 issues TMA loads and MMAs. K, V and P have two
+// the accumulator), warp 16 issues the S products and K loads, warp 17 the
+// P V products and V loads. K, V and P have two
 // slots each and S two TMEM buffers, so tile t + 1's load, conversion and S
 // product and tile t - 1's P V product all overlap tile t's softmax; the
 // softmax waits for P V of tile t - 1 only to rescale O (rare). Every wait is
@@ -53,10 +54,10 @@ cudaError_t launch_attention_merge(const dspark_model* m, const AttnArgs& a, cud
 namespace tc {
 namespace {
 
-constexpr int kThreads = 544;
+constexpr int kThreads = 576;
 constexpr int kSoftThreads = 256;    // warps 0-7
 constexpr int kConvThreads = 256;    // warps 8-15
-constexpr int kIssuerWarp = 16;
+constexpr int kIssuerWarp = 16;      // S products and K loads; warp 17: P V products and V loads
 constexpr int KT = 64;               // keys per tile
 constexpr int QROWS = 128;           // MMA M
 constexpr float kRescale = 5.0f;     // natural-log headroom before the running max is raised
@@ -76,14 +77,25 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 
 // bf16 -> fp16 in place over a tile of `nsub` sub-tiles [KT rows x 128 B] by
 // the converter threads; rows >= nvalid become zeros.
+// Each thread owns 16-byte chunks ct, ct + kConvThreads, ...; all its loads
+// are issued before the first conversion (one round of shared-memory latency).
 __device__ __forceinline__ void convert_tile(uint8_t* tile, int nsub, int nvalid, int ct) {
+    constexpr int kPer = 4 * KT * 8 / kConvThreads;    // chunks per thread at nsub = 4
     const int n16 = nsub * KT * 8;
     uint4* p = reinterpret_cast<uint4*>(tile);
-    for (int i = ct; i < n16; i += kConvThreads) {
+    uint4 u[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = ct + k * kConvThreads;
+        u[k] = i < n16 ? p[i] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = ct + k * kConvThreads;
+        if (i >= n16) break;
         const int row = (i >> 3) % KT;
         if (row >= nvalid) { p[i] = make_uint4(0u, 0u, 0u, 0u); continue; }
-        const uint4 u = p[i];
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
         uint32_t o[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) o[j] = pack_half2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
@@ -91,10 +103,32 @@ __device__ __forceinline__ void convert_tile(uint8_t* tile, int nsub, int nvalid
     }
 }
 
+// Bounded mbarrier wait by polling (no suspension): for the short waits on the
+// softmax's critical path, where a wake-up delay would add to every tile.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicOr(status, DSPARK_DEV_WAIT_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
 // A bounded mbarrier wait whose outcome is the same in every lane of the warp
 // (the softmax warps run warp-collective tcgen05.ld and votes after it).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status) {
     const bool w = mbar_wait(bar, parity, abort_flag, status);
+    return __all_sync(0xffffffffu, w);
+}
+__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status) {
+    const bool w = mbar_wait_spin(bar, parity, abort_flag, status);
     return __all_sync(0xffffffffu, w);
 }
 
@@ -122,7 +156,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     uint64_t* spare = bars + 16;     // teardown: MMAs in flight after an abort
     uint64_t* xw = bars + 17;        // row-max exchange: both halves wrote (256 arrivals)
     uint64_t* xr = bars + 18;        // row-max exchange: both halves read (256 arrivals)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+    uint64_t* spare2 = bars + 19;    // teardown of the P V issuer
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -140,7 +175,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         mbar_init(&sfree[0], kSoftThreads); mbar_init(&sfree[1], kSoftThreads);
         mbar_init(&pready[0], kSoftThreads); mbar_init(&pready[1], kSoftThreads);
         mbar_init(&odone[0], 1); mbar_init(&odone[1], 1); mbar_init(spare, 1);
-        mbar_init(xw, kSoftThreads); mbar_init(xr, kSoftThreads);
+        mbar_init(xw, kSoftThreads); mbar_init(xr, kSoftThreads); mbar_init(spare2, 1);
         *abort_flag = 0;
         mbar_fence_init();
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmKb); prefetch_tmap(&tmVb);
@@ -207,9 +242,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     const uint32_t tO = tmem + 2 * KT;                    // O: columns [128, 128 + hd); S buffers at 0 and 64
     bool ok = true;
 
-    if (warp == kIssuerWarp) {
-        // ------------------------------------------------------------ issuer
+    if (warp >= kIssuerWarp) {
+        // ------------------------------------------------------------ issuers
+        // warp 16: S = Q K^T and the K loads; warp 17: O += P V and the V loads.
+        // Each waits only for what its own products need; a load waits only for its
+        // slot to be free, and every wait keeps issuing the loads that can go.
         if (lane == 0) {
+            const bool is_qk = warp == kIssuerWarp;
             auto load = [&](uint8_t* dst, uint64_t* bar, bool v_tile, int t) {
                 int row, nvalid; bool blk;
                 tile_rows(t, &row, &nvalid, &blk);
@@ -217,25 +256,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 mbar_arrive_expect_tx(bar, tile_bytes);
                 for (int sb = 0; sb < nsub; ++sb) tma_load_3d(dst + sb * KT * 128, m, bar, sb * 64, g, row);
             };
-            const uint32_t idesc_qk = idesc_f16(QROWS, KT, 0);
-            const uint32_t idesc_pv = idesc_f16(QROWS, hd, 1);
-            int nk[2] = {0, 0}, nv[2] = {0, 0};               // loads issued per slot
-            for (int t = 0; t < 2 && t < nt; ++t) {
-                load(sK + t * tile_sz, &kfull[t], false, t); ++nk[t];
-                load(sV + t * tile_sz, &vfull[t], true, t); ++nv[t];
-            }
-            // Loads wait only for their slot to be free; the issuer never blocks on them:
-            // every wait below keeps issuing the loads whose slot has come free.
-            int kn = min(2, nt), vn = min(2, nt);             // next K / V tile to load
-            int qk_issued = 0, pv_issued = 0;                 // S / P V products issued
+            uint8_t* buf = is_qk ? sK : sV;
+            uint64_t* fullb = is_qk ? kfull : vfull;
+            uint64_t* doneb = is_qk ? sdone : odone;          // completion of the product that read a slot
+            int nl[2] = {0, 0};                               // loads issued per slot
+            for (int t = 0; t < 2 && t < nt; ++t) { load(buf + t * tile_sz, &fullb[t], !is_qk, t); ++nl[t]; }
+            int ln = min(2, nt);                              // next tile to load
+            int issued = 0;                                   // products issued
             auto service = [&]() {
-                // K(kn) into slot kn % 2 once S(kn - 2) has read it
-                while (kn < nt && kn - 2 < qk_issued && mbar_try_wait(&sdone[kn & 1], (uint32_t)((kn - 2) >> 1) & 1u)) {
-                    load(sK + (kn & 1) * tile_sz, &kfull[kn & 1], false, kn); ++nk[kn & 1]; ++kn;
-                }
-                // V(vn) into slot vn % 2 once P(vn - 2) V(vn - 2) has read it
-                while (vn < nt && vn - 2 < pv_issued && mbar_try_wait(&odone[vn & 1], (uint32_t)((vn - 2) >> 1) & 1u)) {
-                    load(sV + (vn & 1) * tile_sz, &vfull[vn & 1], true, vn); ++nv[vn & 1]; ++vn;
+                while (ln < nt && ln - 2 < issued && mbar_try_wait(&doneb[ln & 1], (uint32_t)((ln - 2) >> 1) & 1u)) {
+                    load(buf + (ln & 1) * tile_sz, &fullb[ln & 1], !is_qk, ln); ++nl[ln & 1]; ++ln;
                 }
             };
             auto wait_serving = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -251,53 +281,54 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 }
                 return true;
             };
+            const uint32_t idesc_qk = idesc_f16(QROWS, KT, 0);
+            const uint32_t idesc_pv = idesc_f16(QROWS, hd, 1);
             const uint32_t qa = smem_u32(sQ);
-            for (int t = 0; t <= nt && ok; ++t) {
+            for (int t = 0; t < nt && ok; ++t) {
                 const int sl = t & 1;
-                if (t < nt) {
+                if (is_qk) {
                     // S(t) = Q K(t)^T into buffer t % 2
                     if (!wait_serving(&kready[sl], (uint32_t)(t >> 1) & 1u)) { ok = false; break; }
                     if (t >= 2 && !wait_serving(&sfree[sl], (uint32_t)((t - 2) >> 1) & 1u)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t ka = smem_u32(sK + sl * tile_sz);
                     const uint32_t d = tmem + (uint32_t)(sl * KT);
-#pragma unroll 4
-                    for (int j = 0; j < hd / 16; ++j) {
-                        const uint64_t ad = sdesc_k_sw128(qa + (j >> 2) * QROWS * 128 + (j & 3) * 32);
-                        const uint64_t bd = sdesc_k_sw128(ka + (j >> 2) * KT * 128 + (j & 3) * 32);
-                        mma_bf16(d, ad, bd, idesc_qk, j > 0 ? 1u : 0u);
+                    // descriptors advance by address / 16: constants per unrolled slice
+                    const uint64_t ad0 = sdesc_k_sw128(qa);
+                    const uint64_t bd0 = sdesc_k_sw128(smem_u32(sK + sl * tile_sz));
+                    mma_bf16(d, ad0, bd0, idesc_qk, 0u);
+#pragma unroll
+                    for (int j = 1; j < 16; ++j) {
+                        if (j >= hd / 16) break;
+                        const uint64_t aoff = (uint64_t)(((j >> 2) * QROWS * 128 + (j & 3) * 32) >> 4);
+                        const uint64_t boff = (uint64_t)(((j >> 2) * KT * 128 + (j & 3) * 32) >> 4);
+                        mma_bf16(d, ad0 + aoff, bd0 + boff, idesc_qk, 1u);
                     }
                     mma_commit(&sdone[sl]);
-                    qk_issued = t + 1;
-                }
-                if (t >= 1) {
-                    // O += P(t-1) V(t-1)
-                    const int u = t - 1;
-                    if (!wait_serving(&pready[u & 1], (uint32_t)(u >> 1) & 1u) ||
-                        !wait_serving(&vready[u & 1], (uint32_t)(u >> 1) & 1u)) { ok = false; break; }
+                } else {
+                    // O += P(t) V(t)
+                    if (!wait_serving(&pready[sl], (uint32_t)(t >> 1) & 1u) ||
+                        !wait_serving(&vready[sl], (uint32_t)(t >> 1) & 1u)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t pa = smem_u32(sP + (u & 1) * QROWS * 128), va = smem_u32(sV + (u & 1) * tile_sz);
+                    const uint64_t ad0 = sdesc_k_sw128(smem_u32(sP + sl * QROWS * 128));
+                    const uint64_t bd0 = sdesc_mn_sw128(smem_u32(sV + sl * tile_sz), KT * 128);
 #pragma unroll
-                    for (int j = 0; j < KT / 16; ++j) {
-                        const uint64_t ad = sdesc_k_sw128(pa + j * 32);
-                        const uint64_t bd = sdesc_mn_sw128(va + j * 2048, KT * 128);
-                        mma_bf16(tO, ad, bd, idesc_pv, (u > 0 || j > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&odone[u & 1]);
-                    pv_issued = u + 1;
+                    for (int j = 0; j < KT / 16; ++j)
+                        mma_bf16(tO, ad0 + (uint64_t)((j * 32) >> 4), bd0 + (uint64_t)((j * 2048) >> 4), idesc_pv,
+                                 (t > 0 || j > 0) ? 1u : 0u);
+                    mma_commit(&odone[sl]);
                 }
+                issued = t + 1;
                 service();
             }
             // teardown after an abort: copies and MMAs in flight land first (bounded)
             if (!ok) {
                 const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
                 bool drained = true;
-                for (int i = 0; i < 2; ++i) {
-                    if (drained && nk[i] > 0) drained = mbar_wait_until(&kfull[i], (uint32_t)(nk[i] - 1) & 1u, deadline);
-                    if (drained && nv[i] > 0) drained = mbar_wait_until(&vfull[i], (uint32_t)(nv[i] - 1) & 1u, deadline);
-                }
-                mma_commit(spare);
-                if (drained) drained = mbar_wait_until(spare, 0u, deadline);
+                for (int i = 0; i < 2; ++i)
+                    if (drained && nl[i] > 0) drained = mbar_wait_until(&fullb[i], (uint32_t)(nl[i] - 1) & 1u, deadline);
+                uint64_t* sp = is_qk ? spare : spare2;
+                mma_commit(sp);
+                if (drained) drained = mbar_wait_until(sp, 0u, deadline);
                 if (!drained) atomicOr(P.status, DSPARK_DEV_WAIT_TIMEOUT);
             }
         }
@@ -344,14 +375,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 #pragma unroll
                 for (int j = 0; j < 32; ++j) if (cbase + j >= nvalid) sv[j] = -INFINITY;
             }
-            float mx = -INFINITY;
+            float mt[16];                                   // tree maximum: 5 dependent steps, not 32
 #pragma unroll
-            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, sv[j]);
+            for (int j = 0; j < 16; ++j) mt[j] = fmaxf(sv[j], sv[16 + j]);
+#pragma unroll
+            for (int w = 8; w > 0; w >>= 1) {
+#pragma unroll
+                for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
+            }
+            float mx = mt[0];
             // exchange with the other half of the row (mbarriers: every wait stays bounded)
-            if (t >= 1 && !warp_wait(xr, (uint32_t)(t - 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+            if (t >= 1 && !warp_wait_spin(xr, (uint32_t)(t - 1) & 1u, abort_flag, P.status)) { ok = false; break; }
             red[half * QROWS + r] = mx;
             mbar_arrive(xw);
-            if (!warp_wait(xw, (uint32_t)t & 1u, abort_flag, P.status)) { ok = false; break; }
+            if (!warp_wait_spin(xw, (uint32_t)t & 1u, abort_flag, P.status)) { ok = false; break; }
             mx = fmaxf(mx, red[(half ^ 1) * QROWS + r]);
             mbar_arrive(xr);
             const bool need = t > 0 && mx > m_run + kRescale;
@@ -374,17 +411,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             }
             // P slot t % 2 was last read by P(t-2) V(t-2)
             if (t >= 2 && !warp_wait(&odone[sl], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
-            float lsum = 0.f;
+            float ls[8];                                    // sums in 8 independent chains
+#pragma unroll
+            for (int j = 0; j < 8; ++j) ls[j] = 0.f;
             uint8_t* pslot = sP + sl * QROWS * 128;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {                  // four 16-byte chunks of 8 keys
                 float p[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) { p[j] = __expf(sv[q * 8 + j] - m_run); lsum += p[j]; }
+                for (int j = 0; j < 8; ++j) { p[j] = __expf(sv[q * 8 + j] - m_run); ls[j] += p[j]; }
                 const int chunk = (cbase >> 3) + q;
                 *reinterpret_cast<uint4*>(pslot + r * 128 + ((chunk ^ (r & 7)) * 16)) =
                     make_uint4(pack_half2(p[0], p[1]), pack_half2(p[2], p[3]), pack_half2(p[4], p[5]), pack_half2(p[6], p[7]));
             }
+            const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
             l_run += lsum;
             tc_fence_before();
             mbar_arrive(&sfree[sl]);                           // S buffer read
@@ -458,7 +498,7 @@ bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd
 
 size_t attn_tc_smem(int hd) {
     const int nsub = hd / 64;
-    // Q, K (2 slots), V (2 slots), P (2 slots), row maxima, then 17 barriers + TMEM slot + abort
+    // Q, K (2 slots), V (2 slots), P (2 slots), row maxima, then 20 barriers + TMEM slot + abort
     // flag; 1 KB alignment slack
     return (size_t)nsub * QROWS * 128 + 4 * (size_t)nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 192 + 1024;
 }
