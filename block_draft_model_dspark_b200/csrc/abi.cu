@@ -188,12 +188,13 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.walk_val = c.take((size_t)2 * p.walk_blocks * A * 4);     // two step-parity buffers (persistent walk)
     p.walk_idx = c.take((size_t)2 * p.walk_blocks * A * 4);
     const size_t pb = p.pairs ? 2 : 0;
-    p.x_hi = c.take((size_t)p.M * d.H * pb);
-    p.x_lo = c.take((size_t)p.M * d.H * pb);
-    p.ao_hi = c.take((size_t)p.M * d.nH * d.hd * pb);
-    p.ao_lo = c.take((size_t)p.M * d.nH * d.hd * pb);
-    p.act_hi = c.take((size_t)p.M * d.I * pb);
-    p.act_lo = c.take((size_t)p.M * d.I * pb);
+    // each bf16 pair as one [2][M][K] block (lo right after hi): the GEMM loads both with one TMA
+    p.x_hi = c.take(2 * (size_t)p.M * d.H * pb);
+    p.x_lo = p.x_hi + (size_t)p.M * d.H * pb;
+    p.ao_hi = c.take(2 * (size_t)p.M * d.nH * d.hd * pb);
+    p.ao_lo = p.ao_hi + (size_t)p.M * d.nH * d.hd * pb;
+    p.act_hi = c.take(2 * (size_t)p.M * d.I * pb);
+    p.act_lo = p.act_hi + (size_t)p.M * d.I * pb;
     p.conf = c.take((size_t)p.M * 4);
     p.gscr = c.take(p.gscr_bytes);
     p.total = c.off;

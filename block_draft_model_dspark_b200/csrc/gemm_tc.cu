@@ -9,8 +9,18 @@
 //
 // Operands are staged by TMA with the 128-byte swizzle into a ring of
 // shared-memory stages. An fp32 activation enters as a bf16 pair (hi, lo =
-// x - hi): two MMAs per K slice accumulate both into the same fp32 tile, so
-// the activation keeps ~16 significant bits while the weight streams once.
+// x - hi), stored as one [2][M][K] block: when 2 BN <= 256 the pair is one B
+// operand of 2 BN rows and one MMA per K slice produces both products in
+// adjacent accumulator columns (summed in the epilogue), else two MMAs per
+// slice accumulate into the same columns. The activation keeps ~16
+// significant bits while the weight streams once.
+//
+// A stage spans KSUB = 2 K blocks of 64 when K allows: one TMA request brings
+// the stage's 2 x 16 KB of weights (a 3-D map whose third dimension steps
+// 128 bytes along K) and one brings its activation rows (hi and lo, both K
+// blocks). A single producer thread issues every request, and its issue
+// rate, not HBM, bounded the weight stream at one request per 4 KB of X or
+// 16 KB of W.
 //
 // Roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
 // MMAs, warps 2-5 drain accumulators (TMEM lane quadrant = warp % 4).
@@ -42,9 +52,9 @@ namespace tc {
 namespace {
 
 constexpr int BM = 128;            // weight rows per tile (MMA M)
-constexpr int BK = 64;             // K elements per stage: one 128-byte swizzle row
+constexpr int BK = 64;             // K elements per K block: one 128-byte swizzle row
 constexpr int kThreads = 192;
-constexpr int kABytes = BM * BK * 2;
+constexpr int kABytes = BM * BK * 2;   // one K block of weights (16 KB)
 constexpr int kMaxStages = 12;
 constexpr int kSmemLimit = 227 * 1024;   // dynamic shared memory a CTA may opt into
 // alignment slack + full/empty barriers per stage + 4 accumulator barriers,
@@ -89,18 +99,19 @@ struct SegIter {
     }
 };
 
-template <int NP>
+// KSUB K blocks per stage; stage layout [KSUB x W block][KSUB x (NP x BN rows of X)].
+template <int NP, int KSUB>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX0,
-               const __grid_constant__ CUtensorMap tmX1, KParams kp) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, KParams kp) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const GemmPlan& p = kp.p;
     const int BN = p.BN;
     const int stages = p.stages;
-    const int b_bytes = BN * BK * 2;
-    const int stage_bytes = kABytes + NP * b_bytes;
+    const int b_bytes = BN * BK * 2;                // one K block of one activation part
+    const int x_bytes = NP * b_bytes;               // one K block of the activation (hi and lo)
+    const int stage_bytes = KSUB * (kABytes + x_bytes);
 
-    // carve: [stages x (A, B0, B1)] then barriers
+    // carve: [stages x (W blocks, X blocks)] then barriers
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(base + stages * stage_bytes);
     uint64_t* empty = full + stages;
@@ -117,8 +128,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 128); }
         *abort_flag = 0;
         mbar_fence_init();
-        prefetch_tmap(&tmW); prefetch_tmap(&tmX0);
-        if (NP == 2) prefetch_tmap(&tmX1);
+        prefetch_tmap(&tmW); prefetch_tmap(&tmX);
     }
     if (warp == 1) tmem_alloc(tmem_slot, tmem_cols);
     tc_fence_before();
@@ -132,6 +142,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
+            // one request per stage for the weights, one for the activation
+            auto load_w = [&](uint8_t* dst, uint64_t* bar, int kk, int nt) {
+                if (KSUB == 1) tma_load_2d(dst, &tmW, bar, kk * BK, nt * BM);
+                else tma_load_3d(dst, &tmW, bar, 0, nt * BM, kk * KSUB);
+            };
+            auto load_x = [&](uint8_t* dst, uint64_t* bar, int kk, int mt) {
+                if (NP == 1 && KSUB == 1) tma_load_2d(dst, &tmX, bar, kk * BK, mt * BN);
+                else if (NP == 1) tma_load_3d(dst, &tmX, bar, 0, mt * BN, kk * KSUB);
+                else if (KSUB == 1) tma_load_3d(dst, &tmX, bar, kk * BK, mt * BN, 0);
+                else tma_load_4d(dst, &tmX, bar, 0, mt * BN, 0, kk * KSUB);
+            };
             // The weights do not depend on the previous kernel: the first
             // `stages` weight tiles are requested before waiting for it, so
             // the weight stream starts while the producer of X drains.
@@ -143,7 +164,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     const int nt = tile / p.n_mt;
                     for (int kk = k0; kk < k1 && n_pre < stages; ++kk, ++n_pre) {
                         mbar_arrive_expect_tx(&full[n_pre], stage_bytes);
-                        tma_load_2d(base + n_pre * stage_bytes, &tmW, &full[n_pre], kk * BK, nt * BM);
+                        load_w(base + n_pre * stage_bytes, &full[n_pre], kk, nt);
                     }
                 }
             }
@@ -160,10 +181,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                         const uint32_t ph = (uint32_t)(n / stages) & 1u;
                         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, kp.status)) { ok = false; break; }
                         mbar_arrive_expect_tx(&full[s], stage_bytes);
-                        tma_load_2d(st, &tmW, &full[s], kk * BK, nt * BM);
+                        load_w(st, &full[s], kk, nt);
                     }
-                    tma_load_2d(st + kABytes, &tmX0, &full[s], kk * BK, mt * BN);
-                    if (NP == 2) tma_load_2d(st + kABytes + b_bytes, &tmX1, &full[s], kk * BK, mt * BN);
+                    load_x(st + KSUB * kABytes, &full[s], kk, mt);
                 }
             }
             // drain: the loads of the last `stages` slots (every issued slot
@@ -203,15 +223,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     const uint32_t ph = (uint32_t)(n / stages) & 1u;
                     if (!mbar_wait(&full[s], ph, abort_flag, kp.status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(base + s * stage_bytes);
-                    const uint64_t adesc = sdesc_k_sw128(a_addr);
+                    const uint32_t st_addr = smem_u32(base + s * stage_bytes);
 #pragma unroll
-                    for (int part = 0; part < (fused ? 1 : NP); ++part) {
-                        const uint64_t bdesc = sdesc_k_sw128(a_addr + kABytes + part * b_bytes);
+                    for (int sub = 0; sub < KSUB; ++sub) {
+                        const uint64_t adesc = sdesc_k_sw128(st_addr + sub * kABytes);
+                        const uint32_t x_addr = st_addr + KSUB * kABytes + sub * x_bytes;
 #pragma unroll
-                        for (int j = 0; j < BK / 16; ++j) {
-                            const uint32_t accum = (kk > k0 || part > 0 || j > 0) ? 1u : 0u;
-                            mma_bf16(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, accum);
+                        for (int part = 0; part < (fused ? 1 : NP); ++part) {
+                            const uint64_t bdesc = sdesc_k_sw128(x_addr + part * b_bytes);
+#pragma unroll
+                            for (int j = 0; j < BK / 16; ++j) {
+                                const uint32_t accum = (kk > k0 || sub > 0 || part > 0 || j > 0) ? 1u : 0u;
+                                mma_bf16(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, accum);
+                            }
                         }
                     }
                     mma_commit(&empty[s]);          // frees the stage once these MMAs have read it
@@ -352,6 +376,48 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t cols, int
 
 namespace {
 
+bool encode(CUtensorMap* tm, int rank, const void* ptr, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+    if (!get_encoder()) return false;
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Weights [rows, K]: KSUB = 1 -> 2-D box {64, 128}; KSUB = 2 -> 3-D view
+// {64, rows, K / 64} (the third dimension steps 128 bytes along K), box
+// {64, 128, 2}: shared layout [K block][row][64].
+bool make_wmap(CUtensorMap* tm, const void* W, int64_t rows, int64_t K, int ksub) {
+    if (ksub == 1) return make_tmap(tm, W, rows, K, BM);
+    const cuuint64_t dims[3] = {(cuuint64_t)BK, (cuuint64_t)rows, (cuuint64_t)(K / BK)};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)BK * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)BM, (cuuint32_t)ksub};
+    return encode(tm, 3, W, dims, strides, box);
+}
+
+// Activation [np][M][K] (np = 2: hi then lo, adjacent): shared layout
+// [K block][part][row][64] for a box of BN rows.
+bool make_xmap(CUtensorMap* tm, const void* X, int64_t M, int64_t K, int BN, int np, int ksub) {
+    if (np == 1 && ksub == 1) return make_tmap(tm, X, M, K, BN);
+    if (np == 1) {
+        const cuuint64_t dims[3] = {(cuuint64_t)BK, (cuuint64_t)M, (cuuint64_t)(K / BK)};
+        const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)BK * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)BN, (cuuint32_t)ksub};
+        return encode(tm, 3, X, dims, strides, box);
+    }
+    if (ksub == 1) {
+        const cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)M, 2};
+        const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)M * K * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)BN, 2};
+        return encode(tm, 3, X, dims, strides, box);
+    }
+    const cuuint64_t dims[4] = {(cuuint64_t)BK, (cuuint64_t)M, 2, (cuuint64_t)(K / BK)};
+    const cuuint64_t strides[3] = {(cuuint64_t)K * 2, (cuuint64_t)M * K * 2, (cuuint64_t)BK * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)BK, (cuuint32_t)BN, 2, (cuuint32_t)ksub};
+    return encode(tm, 4, X, dims, strides, box);
+}
+
 // Two accumulator buffers of acc_cols columns each.
 int tmem_cols_for(int acc_cols) {
     int c = 32;
@@ -368,12 +434,15 @@ GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles) {
     p.BN = m_pad <= 256 ? m_pad : 256;
     p.n_mt = (M + p.BN - 1) / p.BN;
     p.n_nt = (N + BM - 1) / BM;
-    p.kb = K / BK;
     p.tiles = p.n_mt * p.n_nt;
     // as many stages as shared memory holds: the bytes in flight per SM are
-    // what sustains the weight stream at HBM latency under load
-    const int stage_bytes = kABytes + np * p.BN * BK * 2;
-    p.stages = std::max(2, std::min(kMaxStages, (kSmemLimit - kSmemExtra(kMaxStages)) / stage_bytes));
+    // what sustains the weight stream at HBM latency under load; two K blocks
+    // per stage (half the TMA requests) when K allows and >= 3 stages still fit
+    auto stage_bytes_for = [&](int ksub) { return ksub * (kABytes + np * p.BN * BK * 2); };
+    const int avail = kSmemLimit - kSmemExtra(kMaxStages);
+    p.ksub = (K % (2 * BK) == 0 && avail / stage_bytes_for(2) >= 3) ? 2 : 1;
+    p.kb = K / (BK * p.ksub);
+    p.stages = std::max(2, std::min(kMaxStages, avail / stage_bytes_for(p.ksub)));
     // the tensor core takes as long for an MMA of N = 16 as for N = 256: with a
     // bf16 pair activation, hi and lo go through one MMA of N = 2 BN when it fits
     p.acc_cols = (np == 2 && 2 * p.BN <= 256) ? 2 * p.BN : p.BN;
@@ -402,7 +471,7 @@ size_t gemm_partial_elems(const GemmPlan& p) {
 }
 
 size_t gemm_smem_bytes(const GemmPlan& p) {
-    const int stage_bytes = kABytes + p.np * p.BN * BK * 2;
+    const int stage_bytes = p.ksub * (kABytes + p.np * p.BN * BK * 2);
     return (size_t)p.stages * stage_bytes + kSmemExtra(p.stages);
 }
 
@@ -410,21 +479,21 @@ cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, con
                            float* out, int64_t ldo, float cap, float* part, uint32_t* tickets, int32_t* status,
                            cudaStream_t s) {
     if (p.streamk && (!part || !tickets || p.tiles > kMaxTickets)) return cudaErrorInvalidValue;
-    CUtensorMap tw, tx0, tx1;
-    if (!make_tmap(&tw, W, w_rows, p.K, BM)) return cudaErrorInvalidValue;
-    if (!make_tmap(&tx0, X0, p.M, p.K, p.BN)) return cudaErrorInvalidValue;
-    if (p.np == 2) {
-        if (!make_tmap(&tx1, X1, p.M, p.K, p.BN)) return cudaErrorInvalidValue;
-    } else {
-        tx1 = tx0;
-    }
+    // the bf16 pair must be one [2][M][K] block (lo right after hi)
+    if (p.np == 2 && static_cast<const char*>(X1) != static_cast<const char*>(X0) + (size_t)p.M * p.K * 2)
+        return cudaErrorInvalidValue;
+    CUtensorMap tw, tx;
+    if (!make_wmap(&tw, W, w_rows, p.K, p.ksub)) return cudaErrorInvalidValue;
+    if (!make_xmap(&tx, X0, p.M, p.K, p.BN, p.np, p.ksub)) return cudaErrorInvalidValue;
     KParams kp{};
     kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.status = status; kp.part = part; kp.tickets = tickets;
     const size_t smem = gemm_smem_bytes(p);
-    void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, KParams) = p.np == 2 ? gemm_tc_kernel<2> : gemm_tc_kernel<1>;
+    void (*kern)(CUtensorMap, CUtensorMap, KParams) =
+        p.np == 2 ? (p.ksub == 2 ? gemm_tc_kernel<2, 2> : gemm_tc_kernel<2, 1>)
+                  : (p.ksub == 2 ? gemm_tc_kernel<1, 2> : gemm_tc_kernel<1, 1>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(p.grid), dim3(kThreads), smem, s, tw, tx0, tx1, kp);
+    return launch_pdl(kern, dim3(p.grid), dim3(kThreads), smem, s, tw, tx, kp);
 }
 
 }  // namespace tc

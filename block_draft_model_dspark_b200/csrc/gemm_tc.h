@@ -17,7 +17,8 @@ struct GemmPlan {
     int M, N, K, np;       // out [M, N] = X [M, K] @ W [N, K]^T; np = 1 (bf16 X) or 2 (X as bf16 hi + lo)
     int BN;                // activation rows per tile (MMA N)
     int n_mt, n_nt;        // tiles along the activation rows and along the 128 weight rows
-    int kb;                // 64-wide K blocks
+    int ksub;              // 64-wide K blocks per stage (1 or 2)
+    int kb;                // stages along K: K / (64 ksub)
     int tiles;             // n_mt * n_nt; tile index t = nt * n_mt + mt
     int stages, tmem_cols;
     int acc_cols;          // TMEM columns per accumulator: 2 BN when X_hi and X_lo products share one MMA
