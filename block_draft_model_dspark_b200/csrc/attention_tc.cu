@@ -254,7 +254,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 tile_rows(t, &row, &nvalid, &blk);
                 const CUtensorMap* m = blk ? (v_tile ? &tmVb : &tmKb) : (v_tile ? &tmV : &tmK);
                 mbar_arrive_expect_tx(bar, tile_bytes);
-                for (int sb = 0; sb < nsub; ++sb) tma_load_3d(dst + sb * KT * 128, m, bar, sb * 64, g, row);
+                tma_load_4d(dst, m, bar, 0, row, g, 0);     // the whole tile in one request
             };
             uint8_t* buf = is_qk ? sK : sV;
             uint64_t* fullb = is_qk ? kfull : vfull;
@@ -477,7 +477,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 PFN_cuTensorMapEncodeTiled_v12000 g_enc = nullptr;
 std::once_flag g_enc_once;
 
-// 3-D map over a bf16 [rows, nKv, hd] tensor; box {64, 1, KT}, 128-byte swizzle.
+// Map over a bf16 [rows, nKv, hd] tensor; 128-byte swizzle.
 bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd) {
     std::call_once(g_enc_once, [] {
         void* fn = nullptr;
@@ -487,11 +487,13 @@ bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd
             g_enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     });
     if (!g_enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)hd, (cuuint64_t)nKv, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)hd * 2, (cuuint64_t)nKv * hd * 2};
-    cuuint32_t box[3] = {64, 1, (cuuint32_t)KT};   // KT <= 256
-    cuuint32_t estr[3] = {1, 1, 1};
-    return g_enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+    // 4-D view {64 dims, rows, kv heads, hd / 64 chunks (128 bytes apart)}: one request brings a whole
+    // tile, laid out [chunk][key][64] = nsub K-major sub-tiles of KT rows
+    cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)nKv, (cuuint64_t)(hd / 64)};
+    cuuint64_t strides[3] = {(cuuint64_t)nKv * hd * 2, (cuuint64_t)hd * 2, 128};
+    cuuint32_t box[4] = {64, (cuuint32_t)KT, 1, (cuuint32_t)(hd / 64)};   // KT <= 256
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return g_enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
