@@ -165,9 +165,9 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
             for (int b = 0; b < kRows; ++b)
                 uval[i][b] = (t < nt && b < A && v < V) ? __ldcs(a.U + ((int64_t)b * G + step) * V + v) : 0.f;
         }
-        // ---- bias tiles on the tensor cores: two issuing threads (warps 0 and 1) share
-        // the resident tiles; thread 0 also runs the streamed ones
-        const int half_res = nres / 2;
+        // ---- bias tiles on the tensor cores: two issuing threads. Thread 32 runs every
+        // resident tile while thread 0 runs the streamed ones, whose mid-step reload
+        // latency then hides behind thread 32's MMAs.
         auto mma_tile = [&](const uint8_t* src, int t) {
             const uint64_t adesc = sdesc_k_sw128(smem_u32(src));
             const uint64_t bdesc = sdesc_k_sw128(smem_u32(sE));
@@ -180,7 +180,7 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
             if (step == 0 && !mbar_wait(bar_res, 0u, abort_flag, a.status)) ok = false;
             if (ok) {
                 tc_fence_after();
-                for (int t = half_res; t < nres; ++t) mma_tile(sRes + t * kTileBytes, t);
+                for (int t = 0; t < nres; ++t) mma_tile(sRes + t * kTileBytes, t);
                 mma_commit(bar_mma);
             }
         }
@@ -200,9 +200,6 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
                 if (!mbar_wait(&freed[qp % kSlots], (uint32_t)(qp / kSlots) & 1u, abort_flag, a.status)) { ok = false; break; }
                 load_q(q_load);
             }
-            if (ok && step == 0 && !mbar_wait(bar_res, 0u, abort_flag, a.status)) ok = false;
-            if (ok) tc_fence_after();
-            for (int t = 0; ok && t < half_res; ++t) mma_tile(sRes + t * kTileBytes, t);
             for (int q = q_pre; ok && q < q1; ++q) {
                 if (!mbar_wait(&full[q % kSlots], (uint32_t)(q / kSlots) & 1u, abort_flag, a.status)) { ok = false; break; }
                 tc_fence_after();
@@ -237,6 +234,17 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
                 if (b < A && v < V) argmax_merge(best[b], bidx[b], uval[i][b] + __uint_as_float(r[b]), v);
         }
         tc_fence_before();
+        // the next step's U rows of this thread into L2 while the step's reduction runs
+        if (step + 1 < G) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = group + 4 * i;
+                const int v = (t0 + t) * 128 + row;
+                if (t < nt && v < V)
+                    for (int b = 0; b < A; ++b)
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.U + ((int64_t)b * G + step + 1) * V + v));
+            }
+        }
         // ---- candidates of this CTA
 #pragma unroll
         for (int b = 0; b < kRows; ++b) {
@@ -251,7 +259,11 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
             float bv = -INFINITY;
             int bi = 0x7fffffff;
             for (int w = 0; w < kWarps; ++w) argmax_merge(bv, bi, rv[w][tid], ri[w][tid]);
-            if (bi != 0x7fffffff) atomicMax(&a.keys[(size_t)step * A + tid], pack_key(bv, bi));
+            if (bi != 0x7fffffff) {
+                atomicMax(&a.keys[(size_t)step * A + tid], pack_key(bv, bi));
+                // the winner's markov_w1 row is the next step's operand: have it in L2
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.w1 + (int64_t)bi * 64));
+            }
         }
         __syncthreads();
         // ---- grid barrier (bounded), then every CTA reduces all candidates in CTA order
