@@ -236,8 +236,6 @@ int project_rows(const dspark_model* m, const void* hidden, int B, int Lrows, co
     const int64_t rows = (int64_t)B * Lrows;
     const size_t es = esize(d.dtype);
     const GemmScratch sc = gemm_scratch_at(at<void>(ws, pp.gscr), pp.gscr_bytes);
-    cudaError_t e0 = gemm_scratch_reset(sc, pp.gscr_bytes, s);
-    if (e0 != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("GEMM scratch reset: ") + cudaGetErrorString(e0));
     for (int64_t r0 = 0; r0 < rows; r0 += pp.chunk_rows) {
         const int nr = (int)std::min<int64_t>(pp.chunk_rows, rows - r0);
         RowsPlan rp{};
@@ -513,9 +511,8 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     const int Nqk = (d.nH + d.nKv) * d.hd;
     PartView pv;
     const GemmScratch sc = gemm_scratch_at(at<void>(ws, p.gscr), p.gscr_bytes);
-    cudaError_t e = gemm_scratch_reset(sc, p.gscr_bytes, s);
     // the persistent walk's grid-barrier counter
-    if (e == cudaSuccess) e = cudaMemsetAsync(at<uint32_t>(ws, p.ticket), 0, sizeof(uint32_t), s);
+    cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, p.ticket), 0, sizeof(uint32_t), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(at<void>(ws, p.walk_keys), 0, (size_t)d.gamma * A * 8, s);
     if (e == cudaSuccess) e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
     for (int l = 0; l < d.Lyr && e == cudaSuccess; ++l) {

@@ -185,9 +185,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM is held: the next kernel may begin launching; q, the lengths and
-    // the caches come from earlier kernels
-    pdl_trigger();
+    // q, the lengths and the caches come from earlier kernels. No
+    // pdl_trigger: the merge launches as these CTAs exit (see gemm_tc.cu)
     pdl_wait();
 
     int len = P.len[b];

@@ -13,9 +13,25 @@ namespace dspark {
 // pdl_trigger lets the next kernel start launching; pdl_wait blocks until the
 // predecessor grid has completed and its memory is visible. A kernel reads
 // nothing its predecessors wrote (and writes nothing they read) before
-// pdl_wait; only constant data (weights) may be touched earlier.
+// pdl_wait; only constant data (weights) may be touched earlier. The short
+// row kernels trigger at once (the GEMM after them then streams its first
+// weight tiles early); the long kernels (GEMMs, attention, walk) do not
+// trigger, so their consumers launch as they exit instead of waiting beside them.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Thread-block cluster: all threads of every CTA of the cluster meet (release /
+// acquire), and a 32-bit shared-memory word of CTA `rank` of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster_f32(const float* local, int rank) {
+    uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local)), ra;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -16,8 +16,6 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
 
 namespace {
 
-constexpr size_t kTicketBytes = (size_t)tc::kMaxTickets * 4;
-
 int simt_kps(int K, int S) {
     int kps = (K + S - 1) / S;
     return (kps + 31) / 32 * 32;
@@ -71,36 +69,43 @@ size_t gemm_out_elems(const dspark_model* m, int M, int N, int K) {
 size_t gemm_scratch_bytes(const dspark_model* m, int M, int N, int K, bool act_pair) {
     if (M <= 0 || !use_tensor_cores(m)) return 0;
     const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, act_pair ? 2 : 1, false);
-    return p.streamk ? kTicketBytes + tc::gemm_partial_elems(p) * 4 : 0;
+    return tc::gemm_partial_elems(p) * 4;
 }
 
-// Tickets first, sized for the largest tile count any plan uses (a tile is at
-// least 128 x 16 of the result, so out elements / 2048 bounds it).
 GemmScratch gemm_scratch_at(void* base, size_t bytes) {
     GemmScratch sc;
-    if (!base || bytes == 0) return sc;
-    sc.tickets = static_cast<uint32_t*>(base);
-    sc.part = reinterpret_cast<float*>(static_cast<char*>(base) + kTicketBytes);
+    if (base && bytes) sc.part = static_cast<float*>(base);
     return sc;
 }
 
-cudaError_t gemm_scratch_reset(const GemmScratch& sc, size_t bytes, cudaStream_t s) {
-    if (!sc.tickets || bytes == 0) return cudaSuccess;
-    return cudaMemsetAsync(sc.tickets, 0, kTicketBytes, s);
+namespace {
+
+// The view of a tensor-core GEMM's result: the partial tiles of a stream-K
+// plan, else the plain [M, N] result.
+void tc_view(const tc::GemmPlan& p, float* out, const GemmScratch& sc, PartView* v) {
+    *v = PartView{};
+    if (p.streamk) {
+        v->mode = 1; v->p = sc.part;
+        v->BN = p.BN; v->n_mt = p.n_mt; v->kb = p.kb; v->P = p.P; v->T = p.T; v->G = p.G;
+        v->wide = (int64_t)p.T * p.G >= ((int64_t)1 << 32);
+    } else {
+        v->p = out; v->S = 1; v->stride = (int64_t)p.M * p.N; v->ld = p.N;
+    }
 }
+
+}  // namespace
 
 cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, int M, int N, int K, float* out,
                      const GemmScratch& sc, PartView* view, int timer_kind, cudaStream_t s) {
     KernelTimer t(timer_kind, s, weight_bytes(m, N, K) + 4.0 * M * K + 4.0 * M * N, 2.0 * M * N * K);
-    *view = PartView{};
-    view->p = out;
     if (use_tensor_cores(m)) {
         const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, 2, false);
-        view->S = 1; view->stride = (int64_t)M * N; view->ld = N;
-        return tc::launch_gemm_tc(p, W.w, W.n, X.hi, X.lo, out, N, 0.f, sc.part, sc.tickets, m->ws.status, s);
+        tc_view(p, out, sc, view);
+        return tc::launch_gemm_tc(p, W.w, W.n, X.hi, X.lo, out, N, 0.f, sc.part, m->ws.status, s);
     }
     const int S = simt_splits(m, M, N, K);
-    view->S = S; view->stride = (int64_t)M * N; view->ld = N;
+    *view = PartView{};
+    view->p = out; view->S = S; view->stride = (int64_t)M * N; view->ld = N;
     return launch_simt_gemm(X.f32, K, DSPARK_DTYPE_F32, m->d.dtype, W, m->d.group, M, N, K, S, out, N,
                             (int64_t)M * N, false, 0.f, s);
 }
@@ -111,7 +116,7 @@ cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U,
                   2.0 * M * (double)d.V * d.H);
     if (use_tensor_cores(m)) {
         const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, d.V, d.H, 2, true);
-        return tc::launch_gemm_tc(p, m->lm_head.w, d.V, x.hi, x.lo, U, d.V, d.cap, nullptr, nullptr, m->ws.status, s);
+        return tc::launch_gemm_tc(p, m->lm_head.w, d.V, x.hi, x.lo, U, d.V, d.cap, nullptr, m->ws.status, s);
     }
     return launch_simt_gemm(x.f32, d.H, DSPARK_DTYPE_F32, d.dtype, m->lm_head, d.group, M, d.V, d.H, 1, U, d.V, 0,
                             true, d.cap, s);
@@ -129,8 +134,8 @@ cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, c
     cudaError_t e;
     if (use_tensor_cores(m)) {
         const tc::GemmPlan p = tc::plan_gemm(m->num_sms, nrows, N, d.H, 1, false);
-        view.S = 1; view.stride = (int64_t)nrows * N; view.ld = N;
-        e = tc::launch_gemm_tc(p, m->wk_all.w, N, X, nullptr, raw, N, 0.f, sc.part, sc.tickets, m->ws.status, s);
+        tc_view(p, raw, sc, &view);
+        e = tc::launch_gemm_tc(p, m->wk_all.w, N, X, nullptr, raw, N, 0.f, sc.part, m->ws.status, s);
     } else {
         const int S = simt_splits(m, nrows, N, d.H);
         view.S = S; view.stride = (int64_t)nrows * N; view.ld = N;

@@ -8,19 +8,16 @@ namespace dspark {
 // Tensor-core (tcgen05) path: bf16 dense weights. CUDA-core path: the fp32
 // model (its 1e-4 bar excludes TF32) and 4-bit weights.
 bool use_tensor_cores(const dspark_model* m);
-// Scratch of the tensor-core GEMM's stream-K tiles: partial tiles and one
-// ticket per tile. The tickets must be zero before the first GEMM of an API
-// call (gemm_scratch_reset); each GEMM leaves them zero.
+// Scratch of the tensor-core GEMM's stream-K partial tiles, read back by the
+// consumer through its PartView.
 struct GemmScratch {
     float* part = nullptr;
-    uint32_t* tickets = nullptr;
 };
 // fp32 elements of the result buffer run_gemm / run_kv_projection write for an
-// [M, K] x [N, K]^T product, and bytes of GemmScratch it needs (tickets first).
+// [M, K] x [N, K]^T product, and bytes of GemmScratch it needs.
 size_t gemm_out_elems(const dspark_model* m, int M, int N, int K);
 size_t gemm_scratch_bytes(const dspark_model* m, int M, int N, int K, bool act_pair);
 GemmScratch gemm_scratch_at(void* base, size_t bytes);
-cudaError_t gemm_scratch_reset(const GemmScratch& sc, size_t bytes, cudaStream_t s);
 // out = X @ W^T for an activation X (fp32, or its bf16 pair on tensor cores); *view reads the result.
 cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, int M, int N, int K, float* out,
                      const GemmScratch& sc, PartView* view, int timer_kind, cudaStream_t s);

@@ -30,10 +30,10 @@
 // Work split: the grid is persistent (at most one CTA per SM). In stream-K
 // mode the tiles' K-blocks form one sequence cut into equal contiguous
 // ranges, one per CTA; a CTA writes one fp32 partial tile per tile it
-// touches, and the consumer sums a tile's partials in CTA order (no
-// atomics: deterministic). In tile mode each CTA owns whole tiles
-// (round-robin) and the epilogue writes the result directly, optionally with
-// the final-logit softcap.
+// touches, and the consuming kernel sums a tile's partials in CTA order (no
+// atomics, no wait between CTAs: deterministic). In tile mode each CTA owns
+// whole tiles (round-robin) and the epilogue writes the result directly,
+// optionally with the final-logit softcap.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -67,7 +67,6 @@ struct KParams {
     int64_t ldo;
     float cap;         // softcap of the result (0 = none)
     float* part;       // stream-K partial tiles [tile][P][BN][128]
-    uint32_t* tickets; // stream-K: one counter per tile, zero between launches
     int32_t* status;
 };
 
@@ -135,9 +134,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // TMEM is held: the next kernel in the stream may begin launching (it
-    // waits for this grid before touching what this grid writes).
-    pdl_trigger();
+    // No pdl_trigger: the consumer is launched as these CTAs exit. CTAs of a
+    // consumer launched at the GEMM's start would sit in griddepcontrol.wait
+    // for the whole GEMM, and kernels running beside such waiting CTAs were
+    // measured to take ~3x longer over their memory phase.
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
@@ -247,14 +247,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         }
     } else {
         // ---------------------------------------------------------- epilogue (warps 2-5)
-        // A tile computed whole by this CTA is written straight to `out`. A
-        // stream-K tile shared by `cnt` CTAs is written as this CTA's partial;
-        // the last of them to finish (ticket counter; nobody waits) sums the
-        // tile's partials in CTA order and writes `out`.
+        // Tile mode: the result goes straight to `out` (with the softcap). Stream-K:
+        // each CTA writes its partial of every tile it touches into that tile's slot
+        // (slot = CTA - first CTA of the tile); the consumer kernel sums a tile's
+        // partials in slot order (PartView), so no CTA waits for another and the
+        // GEMM ends as soon as its last MMA has drained.
         pdl_wait();
         const int quad = warp & 3;
         const int n_local = quad * 32 + lane;
-        volatile int* s_last = abort_flag + 1;
         SegIter it(p, blockIdx.x);
         int tile, k0, k1, slot, seg = 0;
         while (it.next(tile, k0, k1, slot)) {
@@ -266,7 +266,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             tc_fence_after();
             const int nt = tile / p.n_mt, mt = tile % p.n_mt;
             const int n = nt * BM + n_local;
-            const int cnt = p.streamk ? p.cta_of(tile * p.kb + p.kb - 1) - p.cta_of(tile * p.kb) + 1 : 1;
             const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * p.acc_cols);
             float* part_tile = kp.part + ((int64_t)tile * p.P * BN) * BM + n_local;
             const bool split_acc = p.acc_cols == 2 * BN;       // X_hi and X_lo products in separate columns
@@ -282,7 +281,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 } else {
                     tmem_ld_wait();
                 }
-                if (cnt == 1) {
+                if (!p.streamk) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int m = mt * BN + c0 + j;
@@ -301,40 +300,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             tc_fence_before();
             mbar_arrive(&acc_empty[acc]);
             ++seg;
-            if (cnt > 1) {
-                asm volatile("bar.sync 1, 128;" ::: "memory");          // this CTA's partial is written
-                if (threadIdx.x == 64) {
-                    __threadfence();
-                    *s_last = atomicAdd(&kp.tickets[tile], 1u) == (uint32_t)(cnt - 1);
-                }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (*s_last) {
-                    __threadfence();
-                    for (int j0 = 0; j0 < BN; j0 += 16) {        // 16 rows of loads in flight per partial
-                        float v[16];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) v[j] = 0.f;
-                        for (int s2 = 0; s2 < cnt; ++s2) {
-                            const float* src = part_tile + ((int64_t)s2 * BN + j0) * BM;
-                            float x[16];
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) x[j] = src[(int64_t)j * BM];
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) v[j] += x[j];     // partials summed in CTA order
-                        }
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int m = mt * BN + j0 + j;
-                            if (m < p.M && n < p.N) {
-                                float y = v[j];
-                                if (kp.cap > 0.f) y = kp.cap * tanhf(y / kp.cap);
-                                kp.out[(int64_t)m * kp.ldo + n] = y;
-                            }
-                        }
-                    }
-                    if (threadIdx.x == 64) kp.tickets[tile] = 0u;
-                }
-            }
         }
     }
 
@@ -476,9 +441,8 @@ size_t gemm_smem_bytes(const GemmPlan& p) {
 }
 
 cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, const void* X0, const void* X1,
-                           float* out, int64_t ldo, float cap, float* part, uint32_t* tickets, int32_t* status,
-                           cudaStream_t s) {
-    if (p.streamk && (!part || !tickets || p.tiles > kMaxTickets)) return cudaErrorInvalidValue;
+                           float* out, int64_t ldo, float cap, float* part, int32_t* status, cudaStream_t s) {
+    if (p.streamk && !part) return cudaErrorInvalidValue;
     // the bf16 pair must be one [2][M][K] block (lo right after hi)
     if (p.np == 2 && static_cast<const char*>(X1) != static_cast<const char*>(X0) + (size_t)p.M * p.K * 2)
         return cudaErrorInvalidValue;
@@ -486,7 +450,7 @@ cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, con
     if (!make_wmap(&tw, W, w_rows, p.K, p.ksub)) return cudaErrorInvalidValue;
     if (!make_xmap(&tx, X0, p.M, p.K, p.BN, p.np, p.ksub)) return cudaErrorInvalidValue;
     KParams kp{};
-    kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.status = status; kp.part = part; kp.tickets = tickets;
+    kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.status = status; kp.part = part;
     const size_t smem = gemm_smem_bytes(p);
     void (*kern)(CUtensorMap, CUtensorMap, KParams) =
         p.np == 2 ? (p.ksub == 2 ? gemm_tc_kernel<2, 2> : gemm_tc_kernel<2, 1>)

@@ -9,7 +9,6 @@
 namespace dspark {
 namespace tc {
 
-constexpr int kMaxTickets = 16384;  // stream-K tiles per launch (stream-K is chosen for few tiles)
 constexpr int kModeTiles = 0;      // whole tiles per CTA; result written directly
 constexpr int kModePartials = 1;   // stream-K; fp32 partial tiles [tile][P][BN][128]
 
@@ -32,18 +31,16 @@ struct GemmPlan {
 };
 
 GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles);
-// fp32 scratch elements of the stream-K partial tiles (0 in tile mode) and tile tickets.
+// fp32 scratch elements of the stream-K partial tiles (0 in tile mode).
 size_t gemm_partial_elems(const GemmPlan& p);
-inline size_t gemm_ticket_count(const GemmPlan& p) { return p.streamk ? (size_t)p.tiles : 0; }
 size_t gemm_smem_bytes(const GemmPlan& p);
 // W: bf16 [w_rows >= N, K]; X0 (and X1 when np == 2): bf16 [M, K].
 // Writes the fp32 result out[m * ldo + n] for m < M, n < N, with the softcap
-// cap * tanh(v / cap) when cap > 0. Stream-K plans also need `part`
-// (gemm_partial_elems floats) and `tickets` (gemm_ticket_count counters,
-// zero before the first launch; each launch leaves them zero).
+// cap * tanh(v / cap) when cap > 0, in tile mode. A stream-K plan writes
+// its partial tiles to `part` (gemm_partial_elems floats) instead, and the
+// consumer sums them (PartView mode 1); `out` is then untouched.
 cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, const void* X0, const void* X1,
-                           float* out, int64_t ldo, float cap, float* part, uint32_t* tickets, int32_t* status,
-                           cudaStream_t s);
+                           float* out, int64_t ldo, float cap, float* part, int32_t* status, cudaStream_t s);
 
 }  // namespace tc
 }  // namespace dspark

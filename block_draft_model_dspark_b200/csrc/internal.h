@@ -51,20 +51,59 @@ struct ModelWs {
     bf16* wk_all_s = nullptr; bf16* wk_all_b = nullptr;
 };
 
-// A GEMM result as its consumers read it: out[m][n] is the sum, in slice
-// order, of S split-K slices [S][M][ld] (S = 1 for the tensor-core GEMM,
-// which reduces its stream-K partials itself). Consumers load slice 0 of
-// all their elements first (at), then add the other slices, so one round of
-// memory latency covers a whole row.
+constexpr int kMaxPartials = 8;    // partials a consumer keeps in flight per element
+
+// A GEMM result as its consumers read it. mode 0: out[m][n] is the sum, in
+// slice order, of S split-K slices [S][M][ld] (S = 1: a plain result).
+// mode 1: the tensor-core GEMM's stream-K partial tiles [tile][P][BN][128]
+// (tile = (n / 128) * n_mt + m / BN); the tile's cnt partials come from
+// consecutive CTAs and are summed in CTA order. load() issues every partial
+// load of one element, finish() adds them: callers load all their elements
+// first, so one round of memory latency covers a row.
 struct PartView {
     const float* p = nullptr;
-    int S = 1; int64_t stride = 0, ld = 0;
-    __device__ __forceinline__ float at(int s, int64_t m, int64_t n) const { return p[s * stride + m * ld + n]; }
-    __device__ __forceinline__ float sum(int64_t m, int64_t n) const {
-        float v = at(0, m, n);
-        for (int s = 1; s < S; ++s) v += at(s, m, n);
+    int mode = 0;
+    int S = 1; int64_t stride = 0, ld = 0;     // mode 0
+    int BN = 16, n_mt = 1, kb = 1, P = 1;      // mode 1
+    int T = 1, G = 1;                          // mode 1: stream-K partition (K blocks, CTAs)
+    int wide = 0;                              // mode 1: T * G needs 64-bit arithmetic
+    struct Pending {
+        float x[kMaxPartials];
+        int cnt;
+        const float* rest;                     // partials beyond kMaxPartials (rare)
+    };
+    // the CTA whose K range holds global K block g (32-bit division unless T * G >= 2^32)
+    __device__ __forceinline__ int cta_of(int g) const {
+        if (wide) return (int)((((int64_t)g + 1) * G - 1) / T);
+        return (int)((((uint32_t)g + 1u) * (uint32_t)G - 1u) / (uint32_t)T);
+    }
+    __device__ __forceinline__ Pending load(int64_t m, int64_t n) const {
+        Pending q;
+        if (mode == 0) {
+#pragma unroll
+            for (int s = 0; s < kMaxPartials; ++s) q.x[s] = s < S ? p[s * stride + m * ld + n] : 0.f;
+            q.cnt = S; q.rest = p + m * ld + n;
+            return q;
+        }
+        const int mi = (int)m, ni = (int)n;
+        const int mt = mi / BN, ml = mi - mt * BN, nt = ni >> 7, nl = ni & 127;
+        const int tile = nt * n_mt + mt;
+        q.cnt = cta_of(tile * kb + kb - 1) - cta_of(tile * kb) + 1;
+        const float* base = p + (((int64_t)tile * P) * BN + ml) * 128 + nl;
+#pragma unroll
+        for (int s = 0; s < kMaxPartials; ++s) q.x[s] = s < q.cnt ? base[(int64_t)s * BN * 128] : 0.f;
+        q.rest = base;
+        return q;
+    }
+    __device__ __forceinline__ float finish(const Pending& q) const {
+        float v = q.x[0];
+#pragma unroll
+        for (int s = 1; s < kMaxPartials; ++s) v += q.x[s];      // in slot order; absent slots are +0
+        const int64_t step = mode == 0 ? stride : (int64_t)BN * 128;
+        for (int s = kMaxPartials; s < q.cnt; ++s) v += q.rest[s * step];
         return v;
     }
+    __device__ __forceinline__ float sum(int64_t m, int64_t n) const { return finish(load(m, n)); }
 };
 
 // An fp32 activation and, for tensor-core GEMMs, its bf16 pair hi + lo.
@@ -222,6 +261,29 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    void count_launches(int n);
+    count_launches(1);
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// launch_pdl with clusters of `cluster_x` CTAs along x (gridDim.x a multiple of it).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, int cluster_x, size_t smem,
+                               cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     void count_launches(int n);
     count_launches(1);
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);

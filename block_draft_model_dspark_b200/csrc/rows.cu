@@ -9,6 +9,8 @@
 // the tensor-core GEMM.
 #include <math.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "common.cuh"
 
@@ -54,8 +56,8 @@ __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const 
     const int l = blockIdx.y / nKv, g = blockIdx.y % nKv;
     const int half = hd / 2, i = threadIdx.x;
     const int64_t col = (int64_t)blockIdx.y * hd;
-    float x1 = raw.at(0, r, col + i), x2 = raw.at(0, r, col + i + half);
-    for (int sl = 1; sl < raw.S; ++sl) { x1 += raw.at(sl, r, col + i); x2 += raw.at(sl, r, col + i + half); }
+    const PartView::Pending q1 = raw.load(r, col + i), q2 = raw.load(r, col + i + half);
+    const float x1 = raw.finish(q1), x2 = raw.finish(q2);
     const float ss = block_sum(x1 * x1 + x2 * x2, red);
     const float rinv = rsqrtf(ss / (float)hd + eps);
     const float v1 = x1 * rinv, v2 = x2 * rinv;
@@ -128,8 +130,8 @@ __global__ void qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, in
     const int pos = block_pos[b] + t;
     const int half = hd / 2, i = threadIdx.x;
     const int64_t col = (int64_t)hh * hd;
-    float x1 = part.at(0, m, col + i), x2 = part.at(0, m, col + i + half);
-    for (int sl = 1; sl < part.S; ++sl) { x1 += part.at(sl, m, col + i); x2 += part.at(sl, m, col + i + half); }
+    const PartView::Pending q1 = part.load(m, col + i), q2 = part.load(m, col + i + half);
+    const float x1 = part.finish(q1), x2 = part.finish(q2);
     const float ss = block_sum(x1 * x1 + x2 * x2, red);
     const float rinv = rsqrtf(ss / (float)hd + eps);
     float y1 = x1 * rinv, y2 = x2 * rinv;
@@ -155,43 +157,72 @@ __global__ void qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, in
 // ------------------------------------------------------------------ o_proj / down epilogues
 // mode 0 (o_proj):  h += rms(sum, g1);            x = rms(h, g2)
 // mode 1 (down):    h = (h + rms(sum, g1)) * s;   x = rms(h, g2)
+//
+// grid (C, M) with clusters of C CTAs along x: the C CTAs of a row split its
+// columns (CTA c owns [c * span, (c + 1) * span), span = blockDim.x * PER) and
+// add up the row's two sums of squares through distributed shared memory, in
+// rank order, so every CTA gets the same totals. Few rows (a draft block)
+// thereby still spread over many SMs.
+
+// Sum of v over the block, then over the cluster's C CTAs (rank order). `slot`
+// is this CTA's shared word for the exchange; callers end with cluster_sync()
+// before exiting so no CTA leaves while another still reads its slot.
+__device__ __forceinline__ float cluster_row_sum(float v, float* red, float* slot, int C) {
+    v = block_sum(v, red);
+    if (C == 1) return v;
+    if (threadIdx.x == 0) *slot = v;
+    cluster_sync();
+    float t = 0.f;
+    for (int r = 0; r < C; ++r) t += ld_cluster_f32(slot, r);
+    return t;
+}
+
 template <int PER>
 __global__ void __launch_bounds__(512) residual_epilogue_kernel(PartView part, int H, const void* __restrict__ g1,
                                          const void* __restrict__ g2, const void* __restrict__ scalar, int mode,
                                          float eps, int dtype, float* __restrict__ h, ActBuf x) {
     __shared__ float red[32];
+    __shared__ float xch[2];
     pdl_trigger();
-    const int m = blockIdx.x;
+    const int C = gridDim.x;
+    const int m = blockIdx.y;
+    const int j0 = blockIdx.x * blockDim.x * PER + threadIdx.x;
     float a[PER], hv[PER], w1v[PER], w2v[PER];
     // the gains are weights: loaded while the producing GEMM drains
 #pragma unroll
     for (int c = 0; c < PER; ++c) {
-        const int j = threadIdx.x + c * blockDim.x;
+        const int j = j0 + c * blockDim.x;
         const bool in = j < H;
         w1v[c] = in ? load_any(g1, j, dtype) : 0.f;
         w2v[c] = in ? load_any(g2, j, dtype) : 0.f;
     }
     const float s = mode == 1 ? load_any(scalar, 0, dtype) : 1.f;
     pdl_wait();
-    // every activation load of the row first: one round of memory latency
+    // the activation loads go out in groups of 4 columns (each with all its
+    // partials): one or two rounds of memory latency at bounded registers
 #pragma unroll
     for (int c = 0; c < PER; ++c) {
-        const int j = threadIdx.x + c * blockDim.x;
-        const bool in = j < H;
-        a[c] = in ? part.at(0, m, j) : 0.f;
-        hv[c] = in ? h[(int64_t)m * H + j] : 0.f;
+        const int j = j0 + c * blockDim.x;
+        hv[c] = j < H ? h[(int64_t)m * H + j] : 0.f;
     }
-    for (int sl = 1; sl < part.S; ++sl) {
 #pragma unroll
-        for (int c = 0; c < PER; ++c) {
-            const int j = threadIdx.x + c * blockDim.x;
-            if (j < H) a[c] += part.at(sl, m, j);
+    for (int c0 = 0; c0 < PER; c0 += 4) {
+        PartView::Pending q[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int j = j0 + (c0 + c) * blockDim.x;
+            q[c] = part.load(m, j < H ? j : 0);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int j = j0 + (c0 + c) * blockDim.x;
+            a[c0 + c] = j < H ? part.finish(q[c]) : 0.f;
         }
     }
     float ss = 0.f;
 #pragma unroll
     for (int c = 0; c < PER; ++c) ss += a[c] * a[c];
-    ss = block_sum(ss, red);
+    ss = cluster_row_sum(ss, red, &xch[0], C);
     const float r1 = rsqrtf(ss / (float)H + eps);
     float ss2 = 0.f;
 #pragma unroll
@@ -199,16 +230,17 @@ __global__ void __launch_bounds__(512) residual_epilogue_kernel(PartView part, i
         hv[c] = (hv[c] + a[c] * r1 * w1v[c]) * s;
         ss2 += hv[c] * hv[c];
     }
-    ss2 = block_sum(ss2, red);
+    ss2 = cluster_row_sum(ss2, red, &xch[1], C);
     const float r2 = rsqrtf(ss2 / (float)H + eps);
 #pragma unroll
     for (int c = 0; c < PER; ++c) {
-        const int j = threadIdx.x + c * blockDim.x;
+        const int j = j0 + c * blockDim.x;
         if (j < H) {
             h[(int64_t)m * H + j] = hv[c];
             store_act(x, (int64_t)m * H + j, hv[c] * r2 * w2v[c]);
         }
     }
+    if (C > 1) cluster_sync();
 }
 
 __global__ void gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
@@ -217,8 +249,8 @@ __global__ void gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
     const int64_t total = (int64_t)M * I;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t m = e / I, i = e % I;
-        float g = part.at(0, m, i), u = part.at(0, m, I + i);
-        for (int sl = 1; sl < part.S; ++sl) { g += part.at(sl, m, i); u += part.at(sl, m, I + i); }
+        const PartView::Pending qg = part.load(m, i), qu = part.load(m, I + i);
+        const float g = part.finish(qg), u = part.finish(qu);
         store_act(act, e, gelu_tanh(g) * u);
     }
 }
@@ -272,14 +304,11 @@ int row_per(int H, int threads) {
 
 template <int PER>
 cudaError_t launch_residual(const PartView& part, int M, int H, const void* g1, const void* g2, const void* scalar,
-                            int mode, float eps, int dtype, float* h, const ActBuf& x, int threads, cudaStream_t s) {
-    return launch_pdl(residual_epilogue_kernel<PER>, dim3(M), dim3(threads), 0, s, part, H, g1, g2, scalar, mode, eps,
-                      dtype, h, x);
+                            int mode, float eps, int dtype, float* h, const ActBuf& x, int C, int threads,
+                            cudaStream_t s) {
+    return launch_pdl_cluster(residual_epilogue_kernel<PER>, dim3(C, M), dim3(threads), C, 0, s, part, H, g1, g2,
+                              scalar, mode, eps, dtype, h, x);
 }
-
-cudaError_t launch_residual_any(const PartView& part, int M, int H, const void* g1, const void* g2,
-                                const void* scalar, int mode, float eps, int dtype, float* h, const ActBuf& x,
-                                cudaStream_t s);
 
 int row_threads(int H) {
     int t = (H + 7) / 8;
@@ -290,14 +319,26 @@ int row_threads(int H) {
     return t < 32 ? 32 : t;
 }
 
+// Rows of a full-row epilogue spread over a cluster of C CTAs (C a power of
+// two, at most 8) while M * C stays under about one CTA per SM and each CTA
+// keeps >= 256 columns.
+int residual_cluster(int M, int H, int num_sms) {
+    int C = 1;
+    while (C < 8 && M * C * 2 <= num_sms && H / (C * 2) >= 256) C *= 2;
+    return C;
+}
+
 cudaError_t launch_residual_any(const PartView& part, int M, int H, const void* g1, const void* g2,
                                 const void* scalar, int mode, float eps, int dtype, float* h, const ActBuf& x,
-                                cudaStream_t s) {
-    const int t = row_threads(H);
-    switch (row_per(H, t)) {
-        case 4: return launch_residual<4>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, t, s);
-        case 8: return launch_residual<8>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, t, s);
-        default: return launch_residual<kMaxPer>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, t, s);
+                                int num_sms, cudaStream_t s) {
+    const int C = residual_cluster(M, H, num_sms);
+    const int Hc = (H + C - 1) / C;                 // columns per CTA
+    // split rows: ~4 columns a thread (each load group of 4 covers the CTA's columns)
+    const int t = C > 1 ? std::min(512, std::max(32, ((Hc + 3) / 4 + 31) / 32 * 32)) : row_threads(Hc);
+    switch (row_per(Hc, t)) {
+        case 4: return launch_residual<4>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, C, t, s);
+        case 8: return launch_residual<8>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, C, t, s);
+        default: return launch_residual<kMaxPer>(part, M, H, g1, g2, scalar, mode, eps, dtype, h, x, C, t, s);
     }
 }
 
@@ -340,7 +381,7 @@ cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const PartView& 
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
     const LayerRef& L = m->layers[layer];
-    return launch_residual_any(part, M, d.H, L.post_attn_norm, L.pre_ff_norm, nullptr, 0, d.eps, d.dtype, h, x, s);
+    return launch_residual_any(part, M, d.H, L.post_attn_norm, L.pre_ff_norm, nullptr, 0, d.eps, d.dtype, h, x, m->num_sms, s);
 }
 
 cudaError_t launch_gu_epilogue(const dspark_model* m, const PartView& part, int M, const ActBuf& act,
@@ -360,7 +401,7 @@ cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const PartVie
     const LayerRef& L = m->layers[layer];
     const bool last = layer + 1 == d.Lyr;
     const void* next = last ? m->final_norm : m->layers[layer + 1].in_norm;
-    return launch_residual_any(part, M, d.H, L.post_ff_norm, next, L.layer_scalar, 1, d.eps, d.dtype, h, x, s);
+    return launch_residual_any(part, M, d.H, L.post_ff_norm, next, L.layer_scalar, 1, d.eps, d.dtype, h, x, m->num_sms, s);
 }
 
 cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const int32_t* anchors, const int32_t* tokens,

@@ -117,7 +117,7 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
-    pdl_trigger();
+    // no pdl_trigger: the confidence kernel launches as the walk exits
     pdl_wait();
 
     // streamed tiles: load q (counted over all steps) goes to slot q % kSlots
