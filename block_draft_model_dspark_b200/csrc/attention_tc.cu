@@ -204,32 +204,62 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         else { *row = b * P.G; *nvalid = P.G; *blk = true; }
     };
 
-    // Q tile (all warps): fp16, 128-byte swizzle; rows past the queries are zero
-    for (int row = warp; row < QROWS; row += kThreads / 32) {
-        for (int cd = 0; cd < hd; cd += 256) {
-            const int d = cd + lane * 8;
-            if (d >= hd) continue;
-            float v[8];
-            if (row < nq) {
-                const int i = row / P.grp, h = g * P.grp + row % P.grp;
-                const int64_t off = (((int64_t)b * P.G + i) * P.nH + h) * hd + d;
-                if (P.q_dtype == DSPARK_DTYPE_F32) {
-                    const float4 a0 = *reinterpret_cast<const float4*>(static_cast<const float*>(P.q) + off);
-                    const float4 a1 = *reinterpret_cast<const float4*>(static_cast<const float*>(P.q) + off + 4);
-                    v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w; v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
-                } else {
-                    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(P.q) + off);
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    // The first two K and V tiles do not depend on Q: their loads go out
+    // before the Q tile is built, so they land while it is.
+    const uint32_t tile_bytes = (uint32_t)nsub * KT * 128;
+    if ((warp == kIssuerWarp || warp == kIssuerWarp + 1) && lane == 0) {
+        const bool v_tile = warp != kIssuerWarp;
+        for (int t = 0; t < 2 && t < nt; ++t) {
+            int row, nvalid; bool blk;
+            tile_rows(t, &row, &nvalid, &blk);
+            const CUtensorMap* m = blk ? (v_tile ? &tmVb : &tmKb) : (v_tile ? &tmV : &tmK);
+            uint64_t* bar = v_tile ? &vfull[t] : &kfull[t];
+            mbar_arrive_expect_tx(bar, tile_bytes);
+            tma_load_4d((v_tile ? sV : sK) + t * tile_sz, m, bar, 0, row, g, 0);
+        }
+    }
+
+    // Q tile (all warps): fp16, 128-byte swizzle; rows past the queries are zero.
+    // Each thread's rows are loaded kQBatch at a time before any is converted:
+    // a few rounds of memory latency instead of one per row.
+    constexpr int kQBatch = 4;
+    for (int cd = 0; cd < hd; cd += 256) {
+        const int d = cd + lane * 8;
+        const int sub = d / 64, chunk = (d % 64) / 8;
+        for (int row0 = warp; row0 < QROWS; row0 += kQBatch * (kThreads / 32)) {
+            float v[kQBatch][8];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) { v[2 * j] = __uint_as_float(w[j] << 16); v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u); }
+            for (int k = 0; k < kQBatch; ++k) {
+                const int row = row0 + k * (kThreads / 32);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[k][j] = 0.f;
+                if (row < nq && d < hd) {
+                    const int i = row / P.grp, h = g * P.grp + row % P.grp;
+                    const int64_t off = (((int64_t)b * P.G + i) * P.nH + h) * hd + d;
+                    if (P.q_dtype == DSPARK_DTYPE_F32) {
+                        const float4 a0 = *reinterpret_cast<const float4*>(static_cast<const float*>(P.q) + off);
+                        const float4 a1 = *reinterpret_cast<const float4*>(static_cast<const float*>(P.q) + off + 4);
+                        v[k][0] = a0.x; v[k][1] = a0.y; v[k][2] = a0.z; v[k][3] = a0.w;
+                        v[k][4] = a1.x; v[k][5] = a1.y; v[k][6] = a1.z; v[k][7] = a1.w;
+                    } else {
+                        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(P.q) + off);
+                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            v[k][2 * j] = __uint_as_float(w[j] << 16);
+                            v[k][2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+                        }
+                    }
                 }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = 0.f;
             }
-            const int sub = d / 64, chunk = (d % 64) / 8;
-            *reinterpret_cast<uint4*>(sQ + sub * QROWS * 128 + row * 128 + ((chunk ^ (row & 7)) * 16)) =
-                make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]), pack_half2(v[4], v[5]), pack_half2(v[6], v[7]));
+#pragma unroll
+            for (int k = 0; k < kQBatch; ++k) {
+                const int row = row0 + k * (kThreads / 32);
+                if (row < QROWS && d < hd)
+                    *reinterpret_cast<uint4*>(sQ + sub * QROWS * 128 + row * 128 + ((chunk ^ (row & 7)) * 16)) =
+                        make_uint4(pack_half2(v[k][0], v[k][1]), pack_half2(v[k][2], v[k][3]),
+                                   pack_half2(v[k][4], v[k][5]), pack_half2(v[k][6], v[k][7]));
+            }
         }
     }
     fence_async_shared();
@@ -237,7 +267,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
 
-    const uint32_t tile_bytes = (uint32_t)nsub * KT * 128;
     const uint32_t tO = tmem + 2 * KT;                    // O: columns [128, 128 + hd); S buffers at 0 and 64
     bool ok = true;
 
@@ -259,7 +288,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             uint64_t* fullb = is_qk ? kfull : vfull;
             uint64_t* doneb = is_qk ? sdone : odone;          // completion of the product that read a slot
             int nl[2] = {0, 0};                               // loads issued per slot
-            for (int t = 0; t < 2 && t < nt; ++t) { load(buf + t * tile_sz, &fullb[t], !is_qk, t); ++nl[t]; }
+            for (int t = 0; t < 2 && t < nt; ++t) ++nl[t];    // tiles 0 and 1: issued before the Q tile
             int ln = min(2, nt);                              // next tile to load
             int issued = 0;                                   // products issued
             auto service = [&]() {
@@ -454,15 +483,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         if (any && ok) {
             const int i = r / P.grp, h = g * P.grp + r % P.grp;
             float* dst = P.part_o + (((int64_t)(b * P.nH + h) * P.S1 + split) * P.G + i) * hd + oc0;
-            for (int c = 0; c < hd / 2; c += 16) {
-                uint32_t u[16];
-                tmem_ld_x16(tO + lane_off + (uint32_t)(oc0 + c), u);
+            // 32 columns per TMEM wait: half the waits, stores of 128 contiguous bytes
+            for (int c = 0; c < hd / 2; c += 32) {
+                uint32_t u[2][16];
+                tmem_ld_x16(tO + lane_off + (uint32_t)(oc0 + c), u[0]);
+                tmem_ld_x16(tO + lane_off + (uint32_t)(oc0 + c + 16), u[1]);
                 tmem_ld_wait();
                 if (r < nq) {
 #pragma unroll
-                    for (int j = 0; j < 16; j += 4)
-                        *reinterpret_cast<float4*>(dst + c + j) = make_float4(__uint_as_float(u[j]), __uint_as_float(u[j + 1]),
-                                                                              __uint_as_float(u[j + 2]), __uint_as_float(u[j + 3]));
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(dst + c + j) =
+                            make_float4(__uint_as_float(u[j >> 4][j & 15]), __uint_as_float(u[j >> 4][(j & 15) + 1]),
+                                        __uint_as_float(u[j >> 4][(j & 15) + 2]), __uint_as_float(u[j >> 4][(j & 15) + 3]));
                 }
             }
         }
