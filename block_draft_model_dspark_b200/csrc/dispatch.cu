@@ -52,9 +52,11 @@ int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len) {
     const int want = tcore ? std::max(1, m->num_sms / per_split)
                            : std::max(1, (2 * m->num_sms + per_split - 1) / per_split);
     const int align = tcore ? tc::attention_tc_key_tile() : 16;
-    // tensor cores: >= 4 key tiles per split (each split also pays a Q tile load and
-    // writes a 128-row partial O)
-    const int min_chunk = tcore ? 4 * tc::attention_tc_key_tile() : 64;
+    // tensor cores: >= 2 key tiles per split (each split also pays a Q tile load and
+    // writes a 128-row partial O that the merge reads back). At one 4096-key row,
+    // attention + merge per layer measured 30.0 us with 4 tiles per split, 27.7 with
+    // 2 and 28.3 with 1 (more, smaller partials shift the time into the merge).
+    const int min_chunk = tcore ? 2 * tc::attention_tc_key_tile() : 64;
     int chunk = min_chunk;
     if (max_ctx_len > 0) chunk = std::max(min_chunk, (max_ctx_len + want - 1) / want);
     return (chunk + align - 1) / align * align;
