@@ -11,7 +11,7 @@ Source page: "@mlx-bun/inference 0.0.0-stage -> 1.0.0",
 plus "mlx-bun 0.2.0 -> 0.4.0" page 75 for ``plainDeepspecContext`` and
 ``projectContextKV``. Method names below are the page's.
 
-Readings where the page leaves a step open (each also listed in the design doc):
+Readings where the page leaves a step open:
   * RoPE pairs lane i with lane i + hd/2 (rotate-half, the HF
     ``apply_rotary_pos_emb`` convention the page says it was checked against);
     angle = position / wavelength, wavelength = theta^(2k/hd) for
