@@ -58,7 +58,7 @@ constexpr int kABytes = BM * BK * 2;   // one K block of weights (16 KB)
 constexpr int kMaxStages = 12;
 constexpr int kSmemLimit = 227 * 1024;   // dynamic shared memory a CTA may opt into
 // alignment slack + full/empty barriers per stage + 4 accumulator barriers,
-// the TMEM slot and the abort/last flags
+// the TMEM slot and the abort flag (plus one spare word)
 constexpr int kSmemExtra(int stages) { return 1024 + 16 * stages + 32 + 16 + 64; }
 
 struct KParams {
@@ -117,7 +117,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     uint64_t* acc_full = empty + stages;      // [2]
     uint64_t* acc_empty = acc_full + 2;       // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort, [1] last-CTA flag
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // set when a wait gives up
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t tmem_cols = p.tmem_cols;
