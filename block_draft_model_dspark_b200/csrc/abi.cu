@@ -79,7 +79,7 @@ MatBytes mat_bytes(const Dims& d, int64_t n, int64_t k) {
 }
 
 struct ModelLayout {
-    size_t status, inv_freq, wqk, wqk_s, wqk_b, wgu, wgu_s, wgu_b, wk, wk_s, wk_b, total;
+    size_t status, inv_freq, wqk, wqk_s, wqk_b, wgu, wgu_s, wgu_b, wk, wk_s, wk_b, w2norm, w1max, total;
     MatBytes qk, gu, kall;
 };
 ModelLayout model_layout(const Dims& d) {
@@ -100,6 +100,10 @@ ModelLayout model_layout(const Dims& d) {
     L.wk = take(L.kall.w);
     L.wk_s = take(L.kall.s);
     L.wk_b = take(L.kall.s);
+    // markov norm bounds of the pruned walk
+    const bool prune = walk_prune_model_supported(d);
+    L.w2norm = take(prune ? sizeof(float) * (size_t)d.V : 0);
+    L.w1max = take(prune ? sizeof(uint32_t) : 0);
     L.total = o;
     return L;
 }
@@ -149,6 +153,8 @@ struct DraftPlan {
     bool pairs;   // GEMM inputs also kept as bf16 (hi, lo) pairs for the tensor-core GEMMs
     size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx, walk_keys;
     size_t x_hi, x_lo, ao_hi, ao_lo, act_hi, act_lo, conf, gscr, gscr_bytes, total;
+    bool prune;          // pruned walk ahead of the tensor-core walk
+    size_t prune_words, prune_list;   // [T | cnt][M] + fail, and the candidate lists
 };
 
 DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
@@ -185,6 +191,9 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.prev = c.take((size_t)A * 4);
     p.ticket = c.take(256);
     p.walk_keys = c.take((size_t)d.gamma * A * 8);              // tensor-core walk: per (step, row) maximum
+    p.prune = m->ws.w2norm != nullptr && tc::walk_tc_supported(m, A);
+    p.prune_words = c.take(p.prune ? (size_t)p.M * 8 + 4 : 0);
+    p.prune_list = c.take(p.prune ? (size_t)p.M * kPruneCap * 4 : 0);
     p.walk_val = c.take((size_t)2 * p.walk_blocks * A * 4);     // two step-parity buffers (persistent walk)
     p.walk_idx = c.take((size_t)2 * p.walk_blocks * A * 4);
     const size_t pb = p.pairs ? 2 : 0;
@@ -353,6 +362,17 @@ int dspark_model_create(const dspark_config* cfg, const dspark_weights* w, void*
     m->w1 = w->markov_w1;
     m->final_norm = w->norm;
     m->conf_bias = w->confidence_bias;
+    // norm bounds of the pruned walk: once per model, from the weights as given
+    if (walk_prune_model_supported(d) && aligned16(m->w1) && aligned16(m->w2.w)) {
+        m->ws.w2norm = reinterpret_cast<float*>(base + L.w2norm);
+        m->ws.w1max_bits = reinterpret_cast<uint32_t*>(base + L.w1max);
+        e = launch_markov_norms(m, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) {
+            delete m;
+            DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("markov norm bounds: ") + cudaGetErrorString(e));
+        }
+    }
     rc = gemm_prepare_model(m);
     if (rc != DSPARK_OK) { delete m; return rc; }
     *out = m;
@@ -514,6 +534,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     // the persistent walk's grid-barrier counter
     cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, p.ticket), 0, sizeof(uint32_t), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(at<void>(ws, p.walk_keys), 0, (size_t)d.gamma * A * 8, s);
+    if (e == cudaSuccess && p.prune) e = cudaMemsetAsync(at<void>(ws, p.prune_words), 0, (size_t)M * 8 + 4, s);
     if (e == cudaSuccess) e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
     for (int l = 0; l < d.Lyr && e == cudaSuccess; ++l) {
         const LayerRef& L = m->layers[l];
@@ -540,8 +561,20 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
         const double w2b = d.r > 0 ? (d.quant ? (double)d.V * d.r * 0.5 + (double)d.V * (d.r / d.group) * 4.0
                                               : (double)d.V * d.r * esize(d.dtype)) : 0.0;
         if (tc::walk_tc_supported(m, A)) {
+            const int* skip = nullptr;
+            if (p.prune) {
+                PruneScratch ps;
+                ps.T = at<uint32_t>(ws, p.prune_words);
+                ps.cnt = at<int>(ws, p.prune_words + (size_t)M * 4);
+                ps.fail = at<int>(ws, p.prune_words + (size_t)M * 8);
+                ps.list = at<int>(ws, p.prune_list);
+                KernelTimer t(DSPARK_TIMER_WALK, s, 2.0 * 4.0 * A * d.gamma * (double)d.V, 0.0);
+                e = launch_walk_prune(m, U, anchors, tokens, A, ps, s);
+                skip = ps.fail;
+            }
             KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
-            e = tc::launch_walk_tc(m, U, anchors, tokens, at<unsigned long long>(ws, p.walk_keys), wa.ticket, A, s);
+            if (e == cudaSuccess)
+                e = tc::launch_walk_tc(m, U, anchors, tokens, at<unsigned long long>(ws, p.walk_keys), wa.ticket, skip, A, s);
         } else if (walk_persistent_supported(m, A)) {
             KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
             e = launch_walk_persistent(m, U, anchors, tokens, wa.part_val, wa.part_idx, wa.ticket, A, s);

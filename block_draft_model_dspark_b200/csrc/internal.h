@@ -49,6 +49,8 @@ struct ModelWs {
     bf16* wqk_s = nullptr; bf16* wqk_b = nullptr;   // quantized scales / biases of the stacks
     bf16* wgu_s = nullptr; bf16* wgu_b = nullptr;
     bf16* wk_all_s = nullptr; bf16* wk_all_b = nullptr;
+    float* w2norm = nullptr;        // [V] |markov_w2[v]| upper bounds (pruned walk; NULL when not eligible)
+    uint32_t* w1max_bits = nullptr; // max_p |markov_w1[p]| upper bound, as float bits
 };
 
 constexpr int kMaxPartials = 8;    // partials a consumer keeps in flight per element
@@ -226,11 +228,25 @@ struct WalkArgs {
 cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s);
 // The whole walk in one cooperative launch (one CTA per SM, bounded grid barriers).
 namespace tc {
-// Markov walk with the bias on tensor cores (walk_tc.cu).
+// Markov walk with the bias on tensor cores (walk_tc.cu). With `skip` non-NULL the
+// kernel returns at once when *skip == 0 (the pruned walk already wrote the tokens).
 bool walk_tc_supported(const dspark_model* m, int A);
 cudaError_t launch_walk_tc(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
-                           unsigned long long* keys, uint32_t* arrivals, int A, cudaStream_t s);
+                           unsigned long long* keys, uint32_t* arrivals, const int* skip, int A, cudaStream_t s);
 }  // namespace tc
+// Exact pruning of the walk (walk_prune.cu): candidate lists from norm bounds, then
+// the walk over the candidates; *fail = 1 hands the round to the full walk.
+constexpr int kPruneCap = 256;      // candidates a position may keep (one thread each)
+struct PruneScratch {
+    uint32_t* T = nullptr;          // [M] ordered max of U - B |w2|, zero at entry
+    int* cnt = nullptr;             // [M] candidate counts, zero at entry
+    int* fail = nullptr;            // one word, zero at entry
+    int* list = nullptr;            // [M][kPruneCap]
+};
+bool walk_prune_model_supported(const Dims& d);
+cudaError_t launch_markov_norms(const dspark_model* m, cudaStream_t s);
+cudaError_t launch_walk_prune(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens, int A,
+                              const PruneScratch& ps, cudaStream_t s);
 bool walk_persistent_supported(const dspark_model* m, int A);
 int walk_persistent_blocks(const dspark_model* m);
 cudaError_t launch_walk_persistent(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,

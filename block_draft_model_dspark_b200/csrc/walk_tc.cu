@@ -54,6 +54,7 @@ struct WtcArgs {
     int tiles_total;           // ceil(V / 128)
     int res_max;               // resident tiles a CTA may hold
     int32_t* status;
+    const int* skip;           // non-NULL: return at once when *skip == 0 (tokens already written)
 };
 
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
@@ -85,6 +86,10 @@ walk_tc_kernel(const __grid_constant__ CUtensorMap tmW2, WtcArgs a) {
     __shared__ uint32_t tmem_slot;
     __shared__ int s_fail;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // the pruned walk has written this round's tokens: every CTA reads the same
+    // word (its writer completed before this stream-ordered launch) and leaves
+    // before touching TMEM, barriers or memory
+    if (a.skip && *a.skip == 0) return;
     const int A = a.A, G = a.G, V = a.V;
     const int nblk = gridDim.x;
     // this CTA's tiles [t0, t1) of the vocabulary
@@ -333,7 +338,7 @@ bool walk_tc_supported(const dspark_model* m, int A) {
 }
 
 cudaError_t launch_walk_tc(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
-                           unsigned long long* keys, uint32_t* arrivals, int A, cudaStream_t s) {
+                           unsigned long long* keys, uint32_t* arrivals, const int* skip, int A, cudaStream_t s) {
     const Dims& d = m->d;
     CUtensorMap tw;
     if (!make_tmap(&tw, m->w2.w, d.V, 64, 128)) return cudaErrorInvalidValue;
@@ -344,6 +349,7 @@ cudaError_t launch_walk_tc(const dspark_model* m, const float* U, const int32_t*
     wa.tiles_total = (d.V + 127) / 128;
     wa.res_max = resident_tiles();
     wa.status = m->ws.status;
+    wa.skip = skip;
     const int nblk = m->num_sms;
     const int per = (wa.tiles_total + nblk - 1) / nblk;
     const int nres = std::min(per, wa.res_max);

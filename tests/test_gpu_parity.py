@@ -175,6 +175,26 @@ def test_rank64_markov_walk(A):
     assert (ref["tokens"] != np.argmax(ref["base_logits"], -1)).any()
 
 
+def test_pruned_markov_walk():
+    """markov_rank 64 with a moderate bias (markov_scale 3): every position keeps
+    16-192 candidates under the norm bound, so the pruned walk decides the tokens
+    (the strong-bias case above overflows the lists and exercises the fallback to
+    the full walk); the bias changes the argmax at some positions."""
+    m = small_model(dtype="bf16", markov_rank=64)
+    cpu, W, model = build(m, 43, markov_scale=3.0)
+    A = 4
+    g = torch.Generator().manual_seed(70 + A)
+    lens = [int(x) for x in torch.randint(1, 97, (A,), generator=g)]
+    pos0 = [int(x) for x in torch.randint(0, 500, (A,), generator=g)]
+    hid = torch.randn(A, max(lens), m.hidden_size, generator=g).to(torch.bfloat16)
+    cache = _project_into_cache(model, hid, lens, pos0)
+    kv = O.project_context_kv(W, hid, pos0, lengths=lens)
+    anchors = [int(x) for x in torch.randint(0, m.vocab_size - 1, (A,), generator=g)]
+    block_pos = [p + L for p, L in zip(pos0, lens)]
+    out, ref = _round_and_compare(m, W, model, cache, kv, anchors, block_pos, lens, "pruned walk, A=4")
+    assert (ref["tokens"] != np.argmax(ref["base_logits"], -1)).any()
+
+
 def test_rank0_no_confidence_head():
     m = small_model(dtype="bf16", markov_rank=0, enable_confidence_head=False, confidence_head_with_markov=False)
     cpu, W, model = build(m, 31)
