@@ -152,7 +152,8 @@ typedef struct dspark_kv_cache {
 typedef struct dspark_model dspark_model;
 
 /* Bytes of device memory dspark_model_create needs for its stacked weight
- * copies, RoPE table and status word; 0 for an invalid config. */
+ * copies, RoPE table, status word and (bf16, markov_rank 64) the Markov norm
+ * bounds; 0 for an invalid config. */
 size_t dspark_model_workspace_bytes(const dspark_config* cfg);
 
 /*
@@ -161,8 +162,10 @@ size_t dspark_model_workspace_bytes(const dspark_config* cfg);
  * `model_ws` (device, >= dspark_model_workspace_bytes, 256-byte aligned,
  * caller-owned, must outlive the model) the RoPE inverse-frequency table and
  * the stacked [q_proj; k_proj], [gate_proj; up_proj] and all-layer k_proj
- * copies the kernels read. Enqueues those copies on `stream`. The weights
- * must stay valid and unchanged for the model's lifetime.
+ * copies the kernels read, and for bf16 weights with markov_rank 64 the
+ * bounds |markov_w2[v]| and max_p |markov_w1[p]| that let dspark_draft_rows
+ * prune the walk exactly. Enqueues this work on `stream` and waits for it. The
+ * weights must stay valid and unchanged for the model's lifetime.
  */
 int dspark_model_create(const dspark_config* cfg, const dspark_weights* weights,
                         void* model_ws, size_t model_ws_bytes, void* stream,
