@@ -568,11 +568,16 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
                 ps.cnt = at<int>(ws, p.prune_words + (size_t)M * 4);
                 ps.fail = at<int>(ws, p.prune_words + (size_t)M * 8);
                 ps.list = at<int>(ws, p.prune_list);
+                // algorithmic bytes: the two scans of U
                 KernelTimer t(DSPARK_TIMER_WALK, s, 2.0 * 4.0 * A * d.gamma * (double)d.V, 0.0);
                 e = launch_walk_prune(m, U, anchors, tokens, A, ps, s);
                 skip = ps.fail;
             }
-            KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
+            // with the pruned walk ahead, the full walk runs only when a candidate list
+            // overflowed: its work is then not counted (it usually returns at once)
+            const bool full_counted = skip == nullptr;
+            KernelTimer t(DSPARK_TIMER_WALK, s, full_counted ? d.gamma * (w2b + 4.0 * A * d.V) : 0.0,
+                          full_counted ? 2.0 * d.gamma * A * (double)d.V * d.r : 0.0);
             if (e == cudaSuccess)
                 e = tc::launch_walk_tc(m, U, anchors, tokens, at<unsigned long long>(ws, p.walk_keys), wa.ticket, skip, A, s);
         } else if (walk_persistent_supported(m, A)) {
