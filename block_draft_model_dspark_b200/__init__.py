@@ -30,6 +30,7 @@ DSPARK_ERR_DEVICE = -6
 DSPARK_DEV_BAD_TOKEN = 1
 DSPARK_DEV_BAD_LENGTH = 2
 DSPARK_DEV_WAIT_TIMEOUT = 4
+DSPARK_DEV_CAPACITY = 8
 DSPARK_DTYPE_F32 = 0
 DSPARK_DTYPE_BF16 = 1
 
@@ -75,7 +76,7 @@ _PROTOTYPES = {
     "dspark_model_destroy": (c_i32, [c_vp]),
     "dspark_project_workspace_bytes": (c_size, [c_vp, ctypes.c_int64]),
     "dspark_project_context_kv": (c_i32, [c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
-    "dspark_append_context_kv": (c_i32, [c_vp, c_vp, c_i32, c_i32p, c_vp, ctypes.POINTER(dspark_kv_cache), c_vp,
+    "dspark_append_context_kv": (c_i32, [c_vp, c_vp, c_i32, c_vp, c_vp, ctypes.POINTER(dspark_kv_cache), c_vp,
                                          c_size, c_vp]),
     "dspark_draft_workspace_bytes": (c_size, [c_vp, c_i32, c_i32]),
     "dspark_draft_rows": (c_i32, [c_vp, ctypes.POINTER(dspark_kv_cache), c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp,
@@ -84,6 +85,7 @@ _PROTOTYPES = {
                               c_size, c_vp]),
     "dspark_attend_no_alloc": (c_i32, [c_vp, c_i32, ctypes.POINTER(dspark_kv_cache), c_vp, c_vp, c_vp, c_vp, c_i32,
                                        c_i32, c_vp]),
+    "dspark_debug_attention_dump": (c_i32, [c_vp, c_vp, c_size]),
     "dspark_read_device_status": (c_i32, [c_vp, c_vp, c_i32p]),
     "dspark_last_error": (ctypes.c_char_p, []),
     "dspark_kernel_launches": (ctypes.c_uint64, []),
@@ -305,13 +307,18 @@ class DsparkModel:
                                              k_out.data_ptr(), v_out.data_ptr(), ws.data_ptr(), ws.numel(),
                                              _stream_ptr(stream)))
 
-    def dspark_append_context_kv(self, cache: KvCache, hidden, n_new: Sequence[int], pos0, ws=None, stream=None):
+    def dspark_append_context_kv(self, cache: KvCache, hidden, n_new, pos0, ws=None, stream=None):
+        """Appends hidden[b, :n_new[b]] to row b of `cache`. ``n_new`` is an int32 tensor on the
+        model's device (a sequence of ints is copied there first); the counts are validated on
+        the device (a refused append sets DSPARK_DEV_CAPACITY in the device status)."""
+        import torch
         B, Lnew = cache.batch, int(hidden.shape[1])
-        n = (ctypes.c_int32 * B)(*[int(x) for x in n_new])
+        if not torch.is_tensor(n_new):
+            n_new = torch.tensor([int(x) for x in n_new], dtype=torch.int32).to(self.device, non_blocking=False)
         ws = ws if ws is not None else self.workspace(self.project_workspace_bytes(B * Lnew))
         st = cache.struct()
-        _check(get_lib().dspark_append_context_kv(self.handle, hidden.data_ptr(), Lnew, n, pos0.data_ptr(), ctypes.byref(st),
-                                            ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
+        _check(get_lib().dspark_append_context_kv(self.handle, hidden.data_ptr(), Lnew, n_new.data_ptr(), pos0.data_ptr(),
+                                                  ctypes.byref(st), ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
 
     def dspark_draft_rows(self, cache: KvCache, anchors, block_pos, max_ctx_len: int, tokens, lengths, conf=None,
                           base_logits=None, ws=None, stream=None):
@@ -337,6 +344,12 @@ class DsparkModel:
         st = cache.struct()
         _check(get_lib().dspark_attend_no_alloc(self.handle, layer, ctypes.byref(st), q.data_ptr(), k_blk.data_ptr(),
                                                 v_blk.data_ptr(), out.data_ptr(), A, max_ctx_len, _stream_ptr(stream)))
+
+    def dspark_debug_attention_dump(self, dst) -> None:
+        """Per-layer attention outputs of later rounds into `dst` (fp32 CUDA tensor
+        [layers, A, gamma, nH, hd]); None turns the dump off."""
+        _check(get_lib().dspark_debug_attention_dump(self.handle, _ptr(dst),
+                                                     0 if dst is None else dst.numel() * dst.element_size()))
 
     def dspark_read_device_status(self, stream=None) -> int:
         v = ctypes.c_int32(0)

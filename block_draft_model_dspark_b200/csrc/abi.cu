@@ -211,10 +211,11 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
 }
 
 constexpr int64_t kProjectChunkRows = 16384;
+constexpr int kMaxAppendBatch = 4096;    // cache batch rows an append handles
 
 struct ProjectPlan {
     int64_t chunk_rows;
-    size_t nvalid, raw, gscr, gscr_bytes, total;
+    size_t nvalid, row0, raw, gscr, gscr_bytes, total;
 };
 ProjectPlan plan_project(const dspark_model* m, int64_t rows) {
     const Dims& d = m->d;
@@ -229,7 +230,8 @@ ProjectPlan plan_project(const dspark_model* m, int64_t rows) {
         p.gscr_bytes = std::max(p.gscr_bytes, gemm_scratch_bytes(m, (int)(rows % p.chunk_rows), N, d.H, false));
     }
     Carve c;
-    p.nvalid = c.take(4096 * 4);
+    p.nvalid = c.take(kMaxAppendBatch * 4);
+    p.row0 = c.take(kMaxAppendBatch * 4);
     p.raw = c.take(raw * 4);
     p.gscr = c.take(p.gscr_bytes);
     p.total = c.off;
@@ -410,39 +412,35 @@ int dspark_project_context_kv(const dspark_model* m, const void* hidden, int32_t
     return project_rows(m, hidden, B, L, nullptr, nullptr, pos0, static_pos, dst, ws, pp, static_cast<cudaStream_t>(stream));
 }
 
-int dspark_append_context_kv(const dspark_model* m, const void* hidden, int32_t Lnew_max, const int32_t* n_new_host,
+int dspark_append_context_kv(const dspark_model* m, const void* hidden, int32_t Lnew_max, const int32_t* n_new,
                              const int32_t* pos0, dspark_kv_cache* cache, void* ws, size_t ws_bytes, void* stream) {
     if (!m || !cache) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "model and cache must be non-NULL");
     const int B = cache->batch;
-    if (B <= 0 || B > 4096) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "cache.batch must be in [1, 4096]");
-    if (Lnew_max < 0) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "Lnew_max must be >= 0");
-    if (!n_new_host || !pos0 || !cache->len || !cache->len_host || !cache->k || !cache->v)
-        DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "n_new_host, pos0 and the cache's k, v, len, len_host must be non-NULL");
-    int total = 0;
-    for (int b = 0; b < B; ++b) {
-        const int n = n_new_host[b], len = cache->len_host[b];
-        if (n < 0 || n > Lnew_max) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "n_new[" + std::to_string(b) + "] outside [0, Lnew_max]");
-        if (len < 0 || (int64_t)len + n > cache->capacity)
-            DSPARK_FAIL(DSPARK_ERR_CAPACITY, "append would pass the cache capacity at row " + std::to_string(b));
-        total += n;
-    }
-    if (total == 0) return DSPARK_OK;
+    if (B <= 0 || B > kMaxAppendBatch) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "cache.batch must be in [1, 4096]");
+    if (Lnew_max < 0 || Lnew_max > cache->capacity) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "Lnew_max must be in [0, cache.capacity]");
+    if ((int64_t)B * Lnew_max > (int64_t)1 << 30) DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "batch * Lnew_max above 2^30 rows");
+    if (!n_new || !pos0 || !cache->len || !cache->k || !cache->v)
+        DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "n_new, pos0 and the cache's k, v, len must be non-NULL");
+    if (!aligned16(cache->k) || !aligned16(cache->v)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "cache k / v must be 16-byte aligned");
+    if (Lnew_max == 0) return DSPARK_OK;
     if (!hidden || !ws || !aligned16(hidden)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "hidden and ws must be non-NULL, 16-byte aligned");
     const ProjectPlan pp = plan_project(m, (int64_t)B * Lnew_max);
     if (ws_bytes < pp.total) DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "ws smaller than dspark_project_workspace_bytes(): " + std::to_string(pp.total));
     const Dims& d = m->d;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* nvalid = at<int32_t>(ws, pp.nvalid);
-    DSPARK_CUDA_CHECK(cudaMemcpyAsync(nvalid, n_new_host, sizeof(int32_t) * B, cudaMemcpyHostToDevice, s));
+    int32_t* row0 = at<int32_t>(ws, pp.row0);
+    // the counts live on the device: validate them there (a refused append writes nothing)
+    cudaError_t e = launch_append_check(n_new, cache->len, B, Lnew_max, cache->capacity, nvalid, row0, m->ws.status, s);
+    if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("append check: ") + cudaGetErrorString(e));
     KvDest dst{};
     dst.k = cache->k; dst.v = cache->v; dst.capacity = cache->capacity;
     dst.batch_stride = (int64_t)cache->capacity * d.nKv * d.hd;
     dst.layer_stride = (int64_t)B * dst.batch_stride;
-    int rc = project_rows(m, hidden, B, Lnew_max, nvalid, cache->len, pos0, 0, dst, ws, pp, s);
+    int rc = project_rows(m, hidden, B, Lnew_max, nvalid, row0, pos0, 0, dst, ws, pp, s);
     if (rc != DSPARK_OK) return rc;
-    cudaError_t e = launch_commit_len(cache->len, nvalid, B, s);
+    e = launch_commit_len(cache->len, nvalid, B, s);
     if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("append commit: ") + cudaGetErrorString(e));
-    for (int b = 0; b < B; ++b) cache->len_host[b] += n_new_host[b];
     return DSPARK_OK;
 }
 
@@ -515,6 +513,9 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     const DraftPlan p = plan_draft(m, A, max_ctx_len);
     if (ws_bytes < p.total) DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "ws smaller than dspark_draft_workspace_bytes(): " + std::to_string(p.total));
     const Dims& d = m->d;
+    const size_t dump_layer = (size_t)A * d.gamma * d.nH * d.hd * sizeof(float);
+    if (m->attn_dump && m->attn_dump_bytes < dump_layer * d.Lyr)
+        DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "attention dump smaller than num_hidden_layers * A * gamma * nH * hd floats");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int M = p.M;
     float* h = at<float>(ws, p.h);
@@ -545,6 +546,9 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
             a.out_hi = ao.hi; a.out_lo = ao.lo;
             e = run_attention(m, a, s);
         }
+        if (e == cudaSuccess && m->attn_dump)
+            e = cudaMemcpyAsync(reinterpret_cast<char*>(m->attn_dump) + dump_layer * l, ao.f32, dump_layer,
+                                cudaMemcpyDeviceToDevice, s);
         if (e == cudaSuccess) e = run_gemm(m, ao, L.o, M, d.H, d.nH * d.hd, part, sc, &pv, DSPARK_TIMER_GEMM_O, s);
         if (e == cudaSuccess) e = launch_o_epilogue(m, l, pv, M, h, x, s);
         if (e == cudaSuccess) e = run_gemm(m, x, L.gu, M, 2 * d.I, d.H, part, sc, &pv, DSPARK_TIMER_GEMM_GU, s);
@@ -594,6 +598,14 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     }
     if (e == cudaSuccess) e = launch_confidence(m, x.f32, anchors, tokens, A, conf ? conf : at<float>(ws, p.conf), lengths, s);
     if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("draft round launch: ") + cudaGetErrorString(e));
+    return DSPARK_OK;
+}
+
+int dspark_debug_attention_dump(dspark_model* m, float* dst, size_t bytes) {
+    if (!m) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "model is NULL");
+    if (dst && (reinterpret_cast<uintptr_t>(dst) & 15u)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "dst must be 16-byte aligned");
+    m->attn_dump = dst;
+    m->attn_dump_bytes = dst ? bytes : 0;
     return DSPARK_OK;
 }
 

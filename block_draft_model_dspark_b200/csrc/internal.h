@@ -146,6 +146,8 @@ struct dspark_model {
     const void* conf_bias = nullptr;
     int device = 0;
     int num_sms = 148;
+    float* attn_dump = nullptr;      // test-facing per-layer attention dump (dspark_debug_attention_dump)
+    size_t attn_dump_bytes = 0;
 };
 
 namespace dspark {
@@ -178,6 +180,11 @@ struct RowsPlan {
 };
 cudaError_t launch_kv_epilogue(const dspark_model* m, const PartView& raw, const RowsPlan& rp, const KvDest& dst,
                                cudaStream_t s);
+// Validates an append's device counts (0 <= n_new[b] <= Lnew_max, len[b] + n_new[b] <= capacity);
+// writes the counts to use (all 0 when any row fails, with DSPARK_DEV_CAPACITY set) and a
+// snapshot of len as each row's first destination row.
+cudaError_t launch_append_check(const int32_t* n_new, const int32_t* len, int B, int Lnew_max, int capacity,
+                                int32_t* nvalid, int32_t* row0, int32_t* status, cudaStream_t s);
 cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStream_t s);
 
 // Activations of the round (x, q, attention output, gelu*up) are fp32 in the

@@ -72,6 +72,35 @@ __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const 
     store_any(dst.k, o + i + half, dtype, k2 * cs + k1 * sn);
 }
 
+// The append's device-side validation (the accepted-row counts come from the
+// caller's device memory, so the host cannot check them): every row must have
+// 0 <= n_new[b] <= Lnew_max and len[b] + n_new[b] <= capacity. If any row
+// fails, the whole append is refused -- every count becomes 0, so the
+// epilogue writes no cache row and the commit adds nothing -- and
+// DSPARK_DEV_CAPACITY is recorded. One CTA; row0[b] snapshots len[b], the
+// cache row where row b's new rows start.
+constexpr int kCheckThreads = 1024;
+__global__ void __launch_bounds__(kCheckThreads) append_check_kernel(const int32_t* __restrict__ n_new,
+                                                                     const int32_t* __restrict__ len, int B,
+                                                                     int Lnew_max, int capacity,
+                                                                     int32_t* __restrict__ nvalid,
+                                                                     int32_t* __restrict__ row0,
+                                                                     int32_t* __restrict__ status) {
+    pdl_trigger();
+    pdl_wait();
+    int bad = 0;
+    for (int b = threadIdx.x; b < B; b += kCheckThreads) {
+        const int n = n_new[b], l = len[b];
+        if (n < 0 || n > Lnew_max || l < 0 || (int64_t)l + n > capacity) bad = 1;
+    }
+    bad = __syncthreads_or(bad);
+    for (int b = threadIdx.x; b < B; b += kCheckThreads) {
+        nvalid[b] = bad ? 0 : n_new[b];
+        row0[b] = len[b];
+    }
+    if (bad && threadIdx.x == 0) atomicOr(status, DSPARK_DEV_CAPACITY);
+}
+
 __global__ void commit_len_kernel(int32_t* len, const int32_t* n_new, int B) {
     pdl_trigger();
     pdl_wait();
@@ -353,6 +382,12 @@ cudaError_t launch_kv_epilogue(const dspark_model* m, const PartView& raw, const
     dim3 grid(rp.nrows, d.Lyr * d.nKv);
     return launch_pdl(kv_epilogue_kernel, grid, dim3(d.hd / 2), 0, s, raw, rp, dst, m->ws.inv_freq, kn, d.nKv, d.hd,
                       d.eps, d.dtype, m->ws.status);
+}
+
+cudaError_t launch_append_check(const int32_t* n_new, const int32_t* len, int B, int Lnew_max, int capacity,
+                                int32_t* nvalid, int32_t* row0, int32_t* status, cudaStream_t s) {
+    return launch_pdl(append_check_kernel, dim3(1), dim3(kCheckThreads), 0, s, n_new, len, B, Lnew_max, capacity,
+                      nvalid, row0, status);
 }
 
 cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStream_t s) {

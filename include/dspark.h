@@ -39,7 +39,7 @@ extern "C" {
 #define DSPARK_OK                    0
 #define DSPARK_ERR_INVALID_ARGUMENT (-1) /* null pointer, bad size, misaligned buffer */
 #define DSPARK_ERR_UNSUPPORTED      (-2) /* a config the drafter page refuses, or outside this build's shapes */
-#define DSPARK_ERR_CAPACITY         (-3) /* an append would pass the cache capacity */
+#define DSPARK_ERR_CAPACITY         (-3) /* reserved: appends are validated on the device (DSPARK_DEV_CAPACITY) */
 #define DSPARK_ERR_WORKSPACE        (-4) /* workspace smaller than the matching *_workspace_bytes() */
 #define DSPARK_ERR_CUDA             (-5) /* a CUDA runtime call or launch failed */
 #define DSPARK_ERR_DEVICE           (-6) /* a device-side check failed (see dspark_read_device_status) */
@@ -48,6 +48,7 @@ extern "C" {
 #define DSPARK_DEV_BAD_TOKEN     1  /* an anchor or walked token outside [0, vocab) was clamped */
 #define DSPARK_DEV_BAD_LENGTH    2  /* a cache length above capacity was clamped */
 #define DSPARK_DEV_WAIT_TIMEOUT  4  /* a bounded device wait gave up */
+#define DSPARK_DEV_CAPACITY      8  /* an append was refused on the device (a count outside [0, Lnew_max] or past capacity) */
 
 #define DSPARK_DTYPE_F32  0
 #define DSPARK_DTYPE_BF16 1
@@ -135,10 +136,13 @@ typedef struct dspark_weights {
  * caller owns the cache's lifetime and the crop after the round).
  * k, v: device T [num_hidden_layers][batch][capacity][nKv][hd]; row t of
  * batch row b holds the K (normed, roped) / V (scale-less normed, unroped)
- * of context row t. len: device int32 [batch], the valid rows per batch row.
- * len_host: host int32 [batch], the library's host mirror of `len`, kept in
- * step by dspark_append_context_kv; the caller sets both when it builds or
- * crops a cache.
+ * of context row t. len: device int32 [batch], the valid rows per batch row;
+ * the caller sets it when it builds or crops a cache (a crop is a smaller
+ * len: rows past len are never read), dspark_append_context_kv advances it.
+ * len_host: optional host int32 [batch] (may be NULL), the caller's own
+ * host copy of len when it keeps one. The library never writes it and reads
+ * it only to count the attention's algorithmic bytes for the instrumentation
+ * timers below.
  */
 typedef struct dspark_kv_cache {
     void*    k;
@@ -197,18 +201,25 @@ int dspark_project_context_kv(const dspark_model* model, const void* hidden, int
 /*
  * Incremental context append (the drafter page's incremental cache:
  * post-norm, post-rope context rows are per-row, so caching them equals
- * recomputing them inside every round's concat). For batch row b, projects
+ * recomputing them inside every round's concat; deepspec.ts draftRows doc:
+ * the caller owns the cache and its crop). For batch row b, projects
  * hidden[b, 0:n_new[b]] as above and writes cache rows [len_b, len_b +
- * n_new[b]) at positions pos0[b] + len_b + t, then sets len[b] += n_new[b]
- * on the device and in len_host.
+ * n_new[b]) at positions pos0[b] + len_b + t, then sets len[b] += n_new[b],
+ * all on the device (the accepted-row counts come out of verification on the
+ * device; no host round trip is needed between verifying and appending).
  *   hidden     device T [cache.batch, Lnew_max, H] (rows past n_new[b] are ignored)
- *   n_new_host host int32 [cache.batch], each in [0, Lnew_max]
+ *   n_new      device int32 [cache.batch]
+ *   Lnew_max   host: the largest count the caller may pass, in [0, capacity]
  *   pos0       device int32 [cache.batch]: absolute position of cache row 0
- * Fails with DSPARK_ERR_CAPACITY, before any launch, if len_host[b] +
- * n_new[b] > capacity for some b.
+ * The counts are validated on the device before any row is written: if any
+ * row has n_new[b] outside [0, Lnew_max] or len[b] + n_new[b] > capacity,
+ * the whole append is refused -- no cache row and no len changes -- and
+ * DSPARK_DEV_CAPACITY is set in the device status word (read it with
+ * dspark_read_device_status). Host-side argument errors return before any
+ * launch. cache.batch <= 4096.
  */
 int dspark_append_context_kv(const dspark_model* model, const void* hidden, int32_t Lnew_max,
-                             const int32_t* n_new_host, const int32_t* pos0, dspark_kv_cache* cache,
+                             const int32_t* n_new, const int32_t* pos0, dspark_kv_cache* cache,
                              void* ws, size_t ws_bytes, void* stream);
 
 /* Scratch bytes dspark_draft_rows / dspark_attend need for A rows whose
@@ -271,6 +282,17 @@ int dspark_attend(const dspark_model* model, int32_t layer, const dspark_kv_cach
 int dspark_attend_no_alloc(const dspark_model* model, int32_t layer, const dspark_kv_cache* cache,
                            const void* q, const void* k_blk, const void* v_blk, void* out,
                            int32_t A, int32_t max_ctx_len, void* stream);
+
+/*
+ * Test-facing dump of every layer's attention output (the parity check of the
+ * DeepspecContextAttention.attend seam inside a round, page 75). While `dst`
+ * is non-NULL, every later dspark_draft_rows call on `model` also copies each
+ * layer's attention output, fp32 [num_hidden_layers][A][gamma][nH][hd], into
+ * `dst` (device, at least `bytes`; a round whose A needs more fails with
+ * DSPARK_ERR_WORKSPACE before any launch). dst = NULL turns the dump off. The
+ * copies run on the round's stream; they slow the round down.
+ */
+int dspark_debug_attention_dump(dspark_model* model, float* dst, size_t bytes);
 
 /* Synchronises `stream`, returns the device status bits in *status and
  * clears them. */

@@ -228,7 +228,7 @@ def test_append_equals_recompute_with_sentinels():
             rows[b].append(hid[b, :n_new[b]])
     torch.cuda.synchronize()
     lens = [sum(s[b] for s in sched) for b in range(B)]
-    assert list(cache.len_host) == lens and cache.len.cpu().tolist() == lens
+    assert cache.len.cpu().tolist() == lens
     full = [torch.cat(r) for r in rows]
     Lmax = max(lens)
     hid_full = torch.zeros(B, Lmax, m.hidden_size, dtype=torch.bfloat16)
@@ -252,20 +252,31 @@ def test_append_equals_recompute_with_sentinels():
     assert same / total > 0.99, f"append vs recompute: only {same}/{total} bf16 values bit-identical"
 
 
-def test_capacity_error_leaves_cache_untouched():
+def test_refused_append_leaves_cache_untouched():
+    """The accepted-row counts live on the device, so the append validates them there: a count
+    past the capacity (or outside [0, Lnew_max]) refuses the whole append, writes no cache row,
+    leaves len unchanged and sets DSPARK_DEV_CAPACITY; the next valid append goes through."""
     import block_draft_model_dspark_b200 as dsp
     m = small_model(dtype="bf16")
     cpu, W, model = build(m, 43)
     cache = dsp.KvCache(model, 2, 20)
     cache.k.zero_(); cache.v.zero_()
     cache.set_lengths([10, 18])
-    k0 = cache.k.clone()
+    k0, v0 = cache.k.clone(), cache.v.clone()
     hid = torch.randn(2, 4, m.hidden_size).to(torch.bfloat16).cuda()
-    with pytest.raises(dsp.DsparkError) as ei:
-        model.dspark_append_context_kv(cache, hid, [4, 3], torch.zeros(2, dtype=torch.int32, device="cuda"))
-    assert ei.value.code == dsp.DSPARK_ERR_CAPACITY
-    torch.cuda.synchronize()
-    assert torch.equal(cache.k, k0) and list(cache.len_host) == [10, 18] and cache.len.cpu().tolist() == [10, 18]
+    pos0 = torch.zeros(2, dtype=torch.int32, device="cuda")
+    for bad in ([4, 3], [1, -1], [5, 0]):          # past capacity; a negative count; above Lnew_max = 4
+        model.dspark_append_context_kv(cache, hid, torch.tensor(bad, dtype=torch.int32, device="cuda"), pos0)
+        assert model.dspark_read_device_status() == dsp.DSPARK_DEV_CAPACITY, bad
+        assert torch.equal(cache.k, k0) and torch.equal(cache.v, v0) and cache.len.cpu().tolist() == [10, 18], bad
+    model.dspark_append_context_kv(cache, hid, torch.tensor([4, 2], dtype=torch.int32, device="cuda"), pos0)
+    assert model.dspark_read_device_status() == 0
+    assert cache.len.cpu().tolist() == [14, 20]
+    assert not torch.equal(cache.k, k0)
+    with pytest.raises(dsp.DsparkError) as ei:      # host-side argument check: Lnew_max above the capacity
+        model.dspark_append_context_kv(cache, torch.zeros(2, 21, m.hidden_size, dtype=torch.bfloat16, device="cuda"),
+                                       torch.zeros(2, dtype=torch.int32, device="cuda"), pos0)
+    assert ei.value.code == dsp.DSPARK_ERR_INVALID_ARGUMENT
 
 
 def test_workspace_too_small_and_bad_anchor_status():
