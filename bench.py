@@ -536,10 +536,11 @@ def run_attention_case(args, wl):
     cache.k.copy_(torch.randn(cache.k.shape, generator=g, device=dev, dtype=torch.float32).to(cache.k.dtype))
     cache.v.copy_(torch.randn(cache.v.shape, generator=g, device=dev, dtype=torch.float32).to(cache.v.dtype))
     cache.set_lengths(lens)
-    q = torch.randn(A, G, nH, hd, generator=g, device=dev).to(torch.bfloat16)
-    kb = torch.randn(A, G, nKv, hd, generator=g, device=dev).to(torch.bfloat16)
-    vb = torch.randn(A, G, nKv, hd, generator=g, device=dev).to(torch.bfloat16)
-    out = torch.empty(A, G, nH, hd, device=dev, dtype=torch.bfloat16)
+    kvt = model.kv_torch_dtype
+    q = torch.randn(A, G, nH, hd, generator=g, device=dev).to(kvt)
+    kb = torch.randn(A, G, nKv, hd, generator=g, device=dev).to(kvt)
+    vb = torch.randn(A, G, nKv, hd, generator=g, device=dev).to(kvt)
+    out = torch.empty(A, G, nH, hd, device=dev, dtype=kvt)
     ws = model.workspace(model.draft_workspace_bytes(A, L))
     for _ in range(max(args.warmup, 3)):
         model.dspark_attend(0, cache, q, kb, vb, out, L, ws=ws)

@@ -31,8 +31,10 @@ DSPARK_DEV_BAD_TOKEN = 1
 DSPARK_DEV_BAD_LENGTH = 2
 DSPARK_DEV_WAIT_TIMEOUT = 4
 DSPARK_DEV_CAPACITY = 8
+DSPARK_DEV_RANGE = 16
 DSPARK_DTYPE_F32 = 0
 DSPARK_DTYPE_BF16 = 1
+DSPARK_DTYPE_F16 = 2
 
 c_i32, c_f32, c_vp, c_size = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 c_i32p = ctypes.POINTER(ctypes.c_int32)
@@ -70,6 +72,7 @@ class dspark_kv_cache(ctypes.Structure):
 
 
 _PROTOTYPES = {
+    "dspark_kv_dtype": (c_i32, [ctypes.POINTER(dspark_config)]),
     "dspark_model_workspace_bytes": (c_size, [ctypes.POINTER(dspark_config)]),
     "dspark_model_create": (c_i32, [ctypes.POINTER(dspark_config), ctypes.POINTER(dspark_weights), c_vp, c_size, c_vp,
                                     ctypes.POINTER(c_vp)]),
@@ -86,6 +89,8 @@ _PROTOTYPES = {
     "dspark_attend_no_alloc": (c_i32, [c_vp, c_i32, ctypes.POINTER(dspark_kv_cache), c_vp, c_vp, c_vp, c_vp, c_i32,
                                        c_i32, c_vp]),
     "dspark_debug_attention_dump": (c_i32, [c_vp, c_vp, c_size]),
+    "dspark_debug_logit_stats": (c_i32, [c_vp, c_vp, c_size]),
+    "dspark_debug_wait_probe": (c_i32, [c_vp, c_i32, c_vp]),
     "dspark_read_device_status": (c_i32, [c_vp, c_vp, c_i32p]),
     "dspark_last_error": (ctypes.c_char_p, []),
     "dspark_kernel_launches": (ctypes.c_uint64, []),
@@ -204,14 +209,15 @@ def _matrix(tensors: Dict, name: str) -> dspark_matrix:
 
 
 class KvCache:
-    """Caller-owned context K/V (``dspark_kv_cache``): k, v [Lyr, batch, capacity, nKv, hd], len [batch]."""
+    """Caller-owned context K/V (``dspark_kv_cache``): k, v [Lyr, batch, capacity, nKv, hd] in the
+    model's KV dtype (``dspark_kv_dtype``: fp16 for a bf16 model), len [batch]."""
 
     def __init__(self, model: "DsparkModel", batch: int, capacity: int, k=None, v=None):
         import torch
         s = model.shape
         shp = (s.num_hidden_layers, batch, capacity, s.num_global_key_value_heads, s.global_head_dim)
-        self.k = k if k is not None else torch.empty(shp, dtype=model.torch_dtype, device=model.device)
-        self.v = v if v is not None else torch.empty(shp, dtype=model.torch_dtype, device=model.device)
+        self.k = k if k is not None else torch.empty(shp, dtype=model.kv_torch_dtype, device=model.device)
+        self.v = v if v is not None else torch.empty(shp, dtype=model.kv_torch_dtype, device=model.device)
         self.len = torch.zeros(batch, dtype=torch.int32, device=model.device)
         self.len_host = (ctypes.c_int32 * batch)()
         self.batch, self.capacity = batch, capacity
@@ -249,6 +255,11 @@ class DsparkModel:
         self.device = next(iter(tensors.values())).device
         self.torch_dtype = torch.float32 if shape.dtype == "fp32" else torch.bfloat16
         self.cfg = make_config(shape)
+        kvd = get_lib().dspark_kv_dtype(ctypes.byref(self.cfg))
+        if kvd < 0:
+            raise DsparkError(DSPARK_ERR_UNSUPPORTED, "invalid config")
+        # element type of caches, projected K/V and the attention seam's tensors
+        self.kv_torch_dtype = {DSPARK_DTYPE_F32: torch.float32, DSPARK_DTYPE_F16: torch.float16}[kvd]
         L = shape.num_hidden_layers
         self._layers = (dspark_layer_weights * L)()
         for i in range(L):
@@ -350,6 +361,17 @@ class DsparkModel:
         [layers, A, gamma, nH, hd]); None turns the dump off."""
         _check(get_lib().dspark_debug_attention_dump(self.handle, _ptr(dst),
                                                      0 if dst is None else dst.numel() * dst.element_size()))
+
+    def dspark_debug_logit_stats(self, dst) -> None:
+        """Per-position logit statistics of later rounds into `dst` (a CUDA tensor of
+        A * gamma * 16 bytes: float max, float logsumexp, int32 argmax, int32 candidates);
+        None turns the dump off."""
+        _check(get_lib().dspark_debug_logit_stats(self.handle, _ptr(dst),
+                                                  0 if dst is None else dst.numel() * dst.element_size()))
+
+    def dspark_debug_wait_probe(self, limit_us: int, stream=None) -> None:
+        """Enqueues a bounded device wait that nothing satisfies (it gives up after limit_us)."""
+        _check(get_lib().dspark_debug_wait_probe(self.handle, int(limit_us), _stream_ptr(stream)))
 
     def dspark_read_device_status(self, stream=None) -> int:
         v = ctypes.c_int32(0)

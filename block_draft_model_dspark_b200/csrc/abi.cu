@@ -64,7 +64,8 @@ Dims make_dims(const dspark_config* c) {
     d.H = c->hidden_size; d.Lyr = c->num_hidden_layers; d.nH = c->num_attention_heads;
     d.nKv = c->num_global_key_value_heads; d.hd = c->global_head_dim; d.grp = d.nH / d.nKv;
     d.I = c->intermediate_size; d.V = c->vocab_size; d.gamma = c->block_size; d.mask_id = c->mask_token_id;
-    d.r = c->markov_rank; d.dtype = c->dtype; d.quant = c->quant_bits == 4; d.group = d.quant ? c->quant_group_size : 64;
+    d.r = c->markov_rank; d.dtype = c->dtype; d.quant = c->quant_bits == 4;
+    d.kv_dtype = c->dtype == DSPARK_DTYPE_BF16 ? DSPARK_DTYPE_F16 : DSPARK_DTYPE_F32; d.group = d.quant ? c->quant_group_size : 64;
     d.eps = c->rms_norm_eps; d.cap = c->final_logit_softcapping; d.conf_thr = c->confidence_threshold;
     d.conf_head = c->enable_confidence_head != 0; d.conf_markov = c->confidence_head_with_markov != 0;
     d.conf_in = d.H + (d.conf_markov ? d.r : 0);
@@ -81,6 +82,12 @@ MatBytes mat_bytes(const Dims& d, int64_t n, int64_t k) {
 struct ModelLayout {
     size_t status, inv_freq, wqk, wqk_s, wqk_b, wgu, wgu_s, wgu_b, wk, wk_s, wk_b, w2norm, w1max, total;
     MatBytes qk, gu, kall;
+    // 4-bit models: the packed copies the tensor-core GEMM reads (per layer where stacked per layer)
+    size_t pk_qk, pk_o, pk_gu, pk_down, pk_lm, pk_k;
+    size_t pk_qk_b, pk_o_b, pk_gu_b, pk_down_b;       // bytes of one layer's copy
+    // dense bf16 models: fp16 copies of o_proj, down_proj (per layer) and the lm-head (the
+    // [q; k] and [gate; up] stacks are fp16 too; the all-layer k_proj stays bf16)
+    size_t h_o, h_down, h_lm, h_o_b, h_down_b;
 };
 ModelLayout model_layout(const Dims& d) {
     ModelLayout L{};
@@ -88,9 +95,23 @@ ModelLayout model_layout(const Dims& d) {
     auto take = [&](size_t bytes) { size_t at = o; o += align_up(bytes, 256); return at; };
     L.status = take(256);
     L.inv_freq = take(sizeof(double) * (size_t)(d.hd / 2));
-    L.qk = mat_bytes(d, (int64_t)(d.nH + d.nKv) * d.hd, d.H);
-    L.gu = mat_bytes(d, 2 * (int64_t)d.I, d.H);
-    L.kall = mat_bytes(d, (int64_t)d.Lyr * d.nKv * d.hd, d.H);
+    // dense: stacked [q_proj; k_proj], [gate; up] and all layers' k_proj; 4-bit: packed copies instead
+    if (!d.quant) {
+        L.qk = mat_bytes(d, (int64_t)(d.nH + d.nKv) * d.hd, d.H);
+        L.gu = mat_bytes(d, 2 * (int64_t)d.I, d.H);
+        L.kall = mat_bytes(d, (int64_t)d.Lyr * d.nKv * d.hd, d.H);
+    } else {
+        L.pk_qk_b = tc::q4_packed_bytes((int64_t)(d.nH + d.nKv) * d.hd, d.H);
+        L.pk_o_b = tc::q4_packed_bytes(d.H, (int64_t)d.nH * d.hd);
+        L.pk_gu_b = tc::q4_packed_bytes(2 * (int64_t)d.I, d.H);
+        L.pk_down_b = tc::q4_packed_bytes(d.H, d.I);
+        L.pk_qk = take(L.pk_qk_b * d.Lyr);
+        L.pk_o = take(L.pk_o_b * d.Lyr);
+        L.pk_gu = take(L.pk_gu_b * d.Lyr);
+        L.pk_down = take(L.pk_down_b * d.Lyr);
+        L.pk_lm = take(tc::q4_packed_bytes(d.V, d.H));
+        L.pk_k = take(tc::q4_packed_bytes((int64_t)d.Lyr * d.nKv * d.hd, d.H));
+    }
     L.wqk = take(L.qk.w * d.Lyr);
     L.wqk_s = take(L.qk.s * d.Lyr);
     L.wqk_b = take(L.qk.s * d.Lyr);
@@ -100,6 +121,13 @@ ModelLayout model_layout(const Dims& d) {
     L.wk = take(L.kall.w);
     L.wk_s = take(L.kall.s);
     L.wk_b = take(L.kall.s);
+    if (!d.quant && d.dtype == DSPARK_DTYPE_BF16) {
+        L.h_o_b = align_up((size_t)d.H * d.nH * d.hd * 2, 256);
+        L.h_down_b = align_up((size_t)d.H * d.I * 2, 256);
+        L.h_o = take(L.h_o_b * d.Lyr);
+        L.h_down = take(L.h_down_b * d.Lyr);
+        L.h_lm = take((size_t)d.V * d.H * 2);
+    }
     // markov norm bounds of the pruned walk
     const bool prune = walk_prune_model_supported(d);
     L.w2norm = take(prune ? sizeof(float) * (size_t)d.V : 0);
@@ -150,11 +178,15 @@ struct Carve {
 
 struct DraftPlan {
     int M, attn_splits, attn_chunk, walk_blocks;
-    bool pairs;   // GEMM inputs also kept as bf16 (hi, lo) pairs for the tensor-core GEMMs
+    int attn_tc_grid;    // tensor-core attention: CTAs (0: the CUDA-core split plan)
+    size_t attn_plan;    // its work plan (ints)
+    bool tc;      // tensor-core GEMMs: the inputs are also kept in fp16 (hi)
+    bool pairs;   // ... and as the fp16 pair (hi, lo)
     size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx, walk_keys;
     size_t x_hi, x_lo, ao_hi, ao_lo, act_hi, act_lo, conf, gscr, gscr_bytes, total;
-    bool prune;          // pruned walk ahead of the tensor-core walk
-    size_t prune_words, prune_list;   // [T | cnt][M] + fail, and the candidate lists
+    int n_vt;            // 128-entry vocabulary tiles of the logit statistics
+    size_t st_mx, st_arg, st_se, st_lo, st_hi;     // tile statistics [n_vt][M] each
+    size_t prune_cnt, prune_fail, prune_list;      // candidate counts [M], fail word, lists [M][kPruneCap]
 };
 
 DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
@@ -162,20 +194,22 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     DraftPlan p{};
     p.M = A * d.gamma;
     const int Nqk = (d.nH + d.nKv) * d.hd;
-    p.pairs = use_tensor_cores(m);
+    p.tc = use_tensor_cores(m);
+    p.pairs = act_pair(m, p.M);
+    const GemmFormat gf = round_gemm_format(m, p.M);
     const size_t part_elems = std::max({gemm_out_elems(m, p.M, Nqk, d.H), gemm_out_elems(m, p.M, d.H, d.nH * d.hd),
                                         gemm_out_elems(m, p.M, 2 * d.I, d.H), gemm_out_elems(m, p.M, d.H, d.I)});
-    p.gscr_bytes = std::max({gemm_scratch_bytes(m, p.M, Nqk, d.H, p.pairs),
-                             gemm_scratch_bytes(m, p.M, d.H, d.nH * d.hd, p.pairs),
-                             gemm_scratch_bytes(m, p.M, 2 * d.I, d.H, p.pairs),
-                             gemm_scratch_bytes(m, p.M, d.H, d.I, p.pairs)});
+    p.gscr_bytes = std::max({gemm_scratch_bytes(m, p.M, Nqk, d.H, gf),
+                             gemm_scratch_bytes(m, p.M, d.H, d.nH * d.hd, gf),
+                             gemm_scratch_bytes(m, p.M, 2 * d.I, d.H, gf),
+                             gemm_scratch_bytes(m, p.M, d.H, d.I, gf)});
     const int chunk = attention_key_chunk(m, A, maxL);
     p.attn_chunk = chunk;
     p.attn_splits = maxL > 0 ? (maxL + chunk - 1) / chunk : 0;
     p.walk_blocks = walk_persistent_supported(m, A) ? walk_persistent_blocks(m)
                                                     : walk_vocab_blocks(m->num_sms, d.V, d.r, d.dtype, d.quant);
     Carve c;
-    const size_t es = esize(d.dtype);
+    const size_t es = esize(d.kv_dtype);
     p.h = c.take((size_t)p.M * d.H * 4);
     p.x = c.take((size_t)p.M * d.H * 4);
     p.part = c.take(part_elems * 4);
@@ -185,25 +219,43 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.attn_out = c.take((size_t)p.M * d.nH * d.hd * 4);
     p.act = c.take((size_t)p.M * d.I * 4);
     p.U = c.take((size_t)p.M * d.V * 4);
-    const size_t S1 = (size_t)p.attn_splits + 1;
-    p.part_o = c.take((size_t)A * d.nH * S1 * d.gamma * d.hd * 4);
-    p.part_ml = c.take((size_t)A * d.nH * S1 * d.gamma * 2 * 4);
+    if (tc::attention_tc_supported(m)) {
+        // one partial slot per CTA of the plan: independent of the context lengths
+        p.attn_tc_grid = tc::attention_tc_grid(m, A);
+        const size_t slot_f = tc::attention_tc_partial_floats(m, p.attn_tc_grid);
+        p.part_o = c.take(slot_f / (d.hd + 2) * d.hd * 4);
+        p.part_ml = c.take(slot_f / (d.hd + 2) * 2 * 4);
+        p.attn_plan = c.take(tc::attention_tc_plan_ints(m, A, p.attn_tc_grid) * 4);
+    } else {
+        const size_t S1 = (size_t)p.attn_splits + 1;
+        p.part_o = c.take((size_t)A * d.nH * S1 * d.gamma * d.hd * 4);
+        p.part_ml = c.take((size_t)A * d.nH * S1 * d.gamma * 2 * 4);
+        p.attn_plan = c.take(0);
+    }
     p.prev = c.take((size_t)A * 4);
     p.ticket = c.take(256);
     p.walk_keys = c.take((size_t)d.gamma * A * 8);              // tensor-core walk: per (step, row) maximum
-    p.prune = m->ws.w2norm != nullptr && tc::walk_tc_supported(m, A);
-    p.prune_words = c.take(p.prune ? (size_t)p.M * 8 + 4 : 0);
-    p.prune_list = c.take(p.prune ? (size_t)p.M * kPruneCap * 4 : 0);
+    p.n_vt = (d.V + 127) / 128;
+    const size_t st = (size_t)p.n_vt * p.M * 4;
+    const bool bounds = d.r > 0;
+    p.st_mx = c.take(st);
+    p.st_arg = c.take(st);
+    p.st_se = c.take(st);
+    p.st_lo = c.take(bounds ? st : 0);
+    p.st_hi = c.take(bounds ? st : 0);
+    p.prune_cnt = c.take((size_t)p.M * 4);
+    p.prune_fail = c.take(4);
+    p.prune_list = c.take(bounds ? (size_t)p.M * kPruneCap * 4 : 0);
     p.walk_val = c.take((size_t)2 * p.walk_blocks * A * 4);     // two step-parity buffers (persistent walk)
     p.walk_idx = c.take((size_t)2 * p.walk_blocks * A * 4);
-    const size_t pb = p.pairs ? 2 : 0;
-    // each bf16 pair as one [2][M][K] block (lo right after hi): the GEMM loads both with one TMA
-    p.x_hi = c.take(2 * (size_t)p.M * d.H * pb);
-    p.x_lo = p.x_hi + (size_t)p.M * d.H * pb;
-    p.ao_hi = c.take(2 * (size_t)p.M * d.nH * d.hd * pb);
-    p.ao_lo = p.ao_hi + (size_t)p.M * d.nH * d.hd * pb;
-    p.act_hi = c.take(2 * (size_t)p.M * d.I * pb);
-    p.act_lo = p.act_hi + (size_t)p.M * d.I * pb;
+    // each fp16 form as one [parts][M][K] block (lo right after hi): the GEMM loads both with one TMA
+    const size_t fb = p.tc ? 2 : 0, parts = p.pairs ? 2 : 1;
+    p.x_hi = c.take(parts * (size_t)p.M * d.H * fb);
+    p.x_lo = p.x_hi + (size_t)p.M * d.H * fb;
+    p.ao_hi = c.take(parts * (size_t)p.M * d.nH * d.hd * fb);
+    p.ao_lo = p.ao_hi + (size_t)p.M * d.nH * d.hd * fb;
+    p.act_hi = c.take(parts * (size_t)p.M * d.I * fb);
+    p.act_lo = p.act_hi + (size_t)p.M * d.I * fb;
     p.conf = c.take((size_t)p.M * 4);
     p.gscr = c.take(p.gscr_bytes);
     p.total = c.off;
@@ -215,7 +267,7 @@ constexpr int kMaxAppendBatch = 4096;    // cache batch rows an append handles
 
 struct ProjectPlan {
     int64_t chunk_rows;
-    size_t nvalid, row0, raw, gscr, gscr_bytes, total;
+    size_t nvalid, row0, raw, gscr, gscr_bytes, x16, total;
 };
 ProjectPlan plan_project(const dspark_model* m, int64_t rows) {
     const Dims& d = m->d;
@@ -224,16 +276,18 @@ ProjectPlan plan_project(const dspark_model* m, int64_t rows) {
     p.chunk_rows = std::min<int64_t>(rows, kProjectChunkRows);
     const int N = d.Lyr * d.nKv * d.hd;
     size_t raw = gemm_out_elems(m, (int)p.chunk_rows, N, d.H);
-    p.gscr_bytes = gemm_scratch_bytes(m, (int)p.chunk_rows, N, d.H, false);
+    const GemmFormat pf = project_gemm_format(m);
+    p.gscr_bytes = gemm_scratch_bytes(m, (int)p.chunk_rows, N, d.H, pf);
     if (rows % p.chunk_rows) {
         raw = std::max(raw, gemm_out_elems(m, (int)(rows % p.chunk_rows), N, d.H));
-        p.gscr_bytes = std::max(p.gscr_bytes, gemm_scratch_bytes(m, (int)(rows % p.chunk_rows), N, d.H, false));
+        p.gscr_bytes = std::max(p.gscr_bytes, gemm_scratch_bytes(m, (int)(rows % p.chunk_rows), N, d.H, pf));
     }
     Carve c;
     p.nvalid = c.take(kMaxAppendBatch * 4);
     p.row0 = c.take(kMaxAppendBatch * 4);
     p.raw = c.take(raw * 4);
     p.gscr = c.take(p.gscr_bytes);
+    p.x16 = c.take(d.quant ? (size_t)p.chunk_rows * d.H * 2 : 0);   // 4-bit models: a chunk's rows in fp16
     p.total = c.off;
     return p;
 }
@@ -253,7 +307,7 @@ int project_rows(const dspark_model* m, const void* hidden, int B, int Lrows, co
         rp.B = B; rp.Lrows = Lrows; rp.row0 = (int)r0; rp.nrows = nr; rp.n_valid = n_valid;
         rp.dst_row0 = dst_row0; rp.pos0 = pos0; rp.static_pos = static_pos;
         const void* X = static_cast<const char*>(hidden) + (size_t)r0 * d.H * es;
-        cudaError_t e = run_kv_projection(m, X, nr, rp, dst, at<float>(ws, pp.raw), sc, s);
+        cudaError_t e = run_kv_projection(m, X, nr, rp, dst, at<float>(ws, pp.raw), sc, at<void>(ws, pp.x16), s);
         if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("context K/V projection launch: ") + cudaGetErrorString(e));
     }
     return DSPARK_OK;
@@ -267,6 +321,12 @@ using namespace dspark;
 extern "C" {
 
 const char* dspark_last_error(void) { return g_error.c_str(); }
+
+int32_t dspark_kv_dtype(const dspark_config* cfg) {
+    std::string why;
+    if (validate_config(cfg, &why) != DSPARK_OK) return -1;
+    return make_dims(cfg).kv_dtype;
+}
 
 size_t dspark_model_workspace_bytes(const dspark_config* cfg) {
     std::string why;
@@ -337,16 +397,61 @@ int dspark_model_create(const dspark_config* cfg, const dspark_weights* w, void*
         const MatRef mk = make_ref(lw.k_proj, (int64_t)d.nKv * d.hd, d.H, q);
         const MatRef mg = make_ref(lw.gate_proj, d.I, d.H, q);
         const MatRef mu = make_ref(lw.up_proj, d.I, d.H, q);
-        e = copy_rows(d, mq, qkw, qks, qkb, 0, s);
-        if (e == cudaSuccess) e = copy_rows(d, mk, qkw, qks, qkb, (int64_t)d.nH * d.hd, s);
-        if (e == cudaSuccess) e = copy_rows(d, mg, guw, gus, gub, 0, s);
-        if (e == cudaSuccess) e = copy_rows(d, mu, guw, gus, gub, d.I, s);
-        if (e == cudaSuccess)
-            e = copy_rows(d, mk, base + L.wk, at<bf16>(base, L.wk_s), at<bf16>(base, L.wk_b), (int64_t)l * d.nKv * d.hd, s);
-        R.qk = stacked_ref(d, qkw, qks, qkb, Nqk, d.H);
-        R.gu = stacked_ref(d, guw, gus, gub, 2 * (int64_t)d.I, d.H);
         R.o = make_ref(lw.o_proj, d.H, (int64_t)d.nH * d.hd, q);
         R.down = make_ref(lw.down_proj, d.H, d.I, q);
+        if (!q && d.dtype == DSPARK_DTYPE_F32) {
+            // fp32: stacked copies for the CUDA-core GEMM
+            e = copy_rows(d, mq, qkw, qks, qkb, 0, s);
+            if (e == cudaSuccess) e = copy_rows(d, mk, qkw, qks, qkb, (int64_t)d.nH * d.hd, s);
+            if (e == cudaSuccess) e = copy_rows(d, mg, guw, gus, gub, 0, s);
+            if (e == cudaSuccess) e = copy_rows(d, mu, guw, gus, gub, d.I, s);
+            if (e == cudaSuccess)
+                e = copy_rows(d, mk, base + L.wk, at<bf16>(base, L.wk_s), at<bf16>(base, L.wk_b), (int64_t)l * d.nKv * d.hd, s);
+            R.qk = stacked_ref(d, qkw, qks, qkb, Nqk, d.H);
+            R.gu = stacked_ref(d, guw, gus, gub, 2 * (int64_t)d.I, d.H);
+        } else if (!q) {
+            // bf16: fp16 copies for the tensor-core GEMMs (exact inside fp16's range; a weight
+            // outside it fails the model's creation), stacked where the GEMM is; the all-layer
+            // k_proj stays bf16 for the context projection of the caller's bf16 rows
+            int32_t* ovf = m->ws.status + 1;
+            const size_t qrow = (size_t)d.H * 2;
+            char* qk16 = static_cast<char*>(qkw);
+            char* gu16 = static_cast<char*>(guw);
+            void* o16 = base + L.h_o + L.h_o_b * l;
+            void* dn16 = base + L.h_down + L.h_down_b * l;
+            e = tc::f16_copy(mq.w, mq.n * d.H, qk16, ovf, s);
+            if (e == cudaSuccess) e = tc::f16_copy(mk.w, mk.n * d.H, qk16 + (size_t)mq.n * qrow, ovf, s);
+            if (e == cudaSuccess) e = tc::f16_copy(mg.w, mg.n * d.H, gu16, ovf, s);
+            if (e == cudaSuccess) e = tc::f16_copy(mu.w, mu.n * d.H, gu16 + (size_t)mg.n * qrow, ovf, s);
+            if (e == cudaSuccess) e = tc::f16_copy(R.o.w, R.o.n * R.o.k, o16, ovf, s);
+            if (e == cudaSuccess) e = tc::f16_copy(R.down.w, R.down.n * R.down.k, dn16, ovf, s);
+            if (e == cudaSuccess)
+                e = copy_rows(d, mk, base + L.wk, at<bf16>(base, L.wk_s), at<bf16>(base, L.wk_b), (int64_t)l * d.nKv * d.hd, s);
+            R.qk = stacked_ref(d, nullptr, nullptr, nullptr, Nqk, d.H);
+            R.gu = stacked_ref(d, nullptr, nullptr, nullptr, 2 * (int64_t)d.I, d.H);
+            R.qk.w16 = qkw; R.gu.w16 = guw; R.o.w16 = o16; R.down.w16 = dn16;
+        } else {
+            // the packed copies the tensor-core GEMM streams (stacked where the GEMM is)
+            auto piece = [](const MatRef& r, int64_t row0) {
+                tc::Q4Piece pc{};
+                pc.w = static_cast<const uint32_t*>(r.w); pc.s = r.scales; pc.b = r.biases; pc.row0 = row0; pc.rows = r.n;
+                return pc;
+            };
+            void* pqk = base + L.pk_qk + L.pk_qk_b * l;
+            void* po = base + L.pk_o + L.pk_o_b * l;
+            void* pgu = base + L.pk_gu + L.pk_gu_b * l;
+            void* pdn = base + L.pk_down + L.pk_down_b * l;
+            const tc::Q4Piece qk2[2] = {piece(mq, 0), piece(mk, (int64_t)d.nH * d.hd)};
+            const tc::Q4Piece gu2[2] = {piece(mg, 0), piece(mu, d.I)};
+            const tc::Q4Piece o1 = piece(R.o, 0), d1 = piece(R.down, 0);
+            e = tc::q4_pack(qk2, 2, Nqk, d.H, pqk, s);
+            if (e == cudaSuccess) e = tc::q4_pack(&o1, 1, d.H, (int64_t)d.nH * d.hd, po, s);
+            if (e == cudaSuccess) e = tc::q4_pack(gu2, 2, 2 * (int64_t)d.I, d.H, pgu, s);
+            if (e == cudaSuccess) e = tc::q4_pack(&d1, 1, d.H, d.I, pdn, s);
+            R.qk = stacked_ref(d, nullptr, nullptr, nullptr, Nqk, d.H);
+            R.gu = stacked_ref(d, nullptr, nullptr, nullptr, 2 * (int64_t)d.I, d.H);
+            R.qk.packed = pqk; R.gu.packed = pgu; R.o.packed = po; R.down.packed = pdn;
+        }
         R.q_norm = lw.q_norm; R.k_norm = lw.k_norm; R.in_norm = lw.input_layernorm;
         R.post_attn_norm = lw.post_attention_layernorm; R.pre_ff_norm = lw.pre_feedforward_layernorm;
         R.post_ff_norm = lw.post_feedforward_layernorm; R.layer_scalar = lw.layer_scalar;
@@ -359,13 +464,50 @@ int dspark_model_create(const dspark_config* cfg, const dspark_weights* w, void*
     m->wk_all = stacked_ref(d, base + L.wk, at<bf16>(base, L.wk_s), at<bf16>(base, L.wk_b), (int64_t)d.Lyr * d.nKv * d.hd, d.H);
     m->embed = make_ref(w->embed_tokens, d.V, d.H, q);
     m->lm_head = make_ref(w->lm_head, d.V, d.H, q);
+    if (!q && d.dtype == DSPARK_DTYPE_BF16) {
+        e = tc::f16_copy(m->lm_head.w, (int64_t)d.V * d.H, base + L.h_lm, m->ws.status + 1, s);
+        int32_t ovf = 0;
+        if (e == cudaSuccess) e = cudaMemcpyAsync(&ovf, m->ws.status + 1, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) {
+            delete m;
+            DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("fp16 weight copies: ") + cudaGetErrorString(e));
+        }
+        if (ovf) {
+            delete m;
+            DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "a bf16 weight lies outside fp16's range (|w| > 65504): the tensor-core "
+                                                "GEMMs read fp16 copies of the weights");
+        }
+        m->lm_head.w16 = base + L.h_lm;
+    }
+    if (q) {
+        // packed copies of the lm-head and of all layers' k_proj (one context projection GEMM)
+        std::vector<tc::Q4Piece> kp(d.Lyr);
+        for (int l = 0; l < d.Lyr; ++l) {
+            const MatRef mk = make_ref(w->layers[l].k_proj, (int64_t)d.nKv * d.hd, d.H, q);
+            kp[l].w = static_cast<const uint32_t*>(mk.w); kp[l].s = mk.scales; kp[l].b = mk.biases;
+            kp[l].row0 = (int64_t)l * d.nKv * d.hd; kp[l].rows = mk.n;
+        }
+        tc::Q4Piece lm{};
+        lm.w = static_cast<const uint32_t*>(m->lm_head.w); lm.s = m->lm_head.scales; lm.b = m->lm_head.biases;
+        lm.row0 = 0; lm.rows = d.V;
+        e = tc::q4_pack(kp.data(), d.Lyr, (int64_t)d.Lyr * d.nKv * d.hd, d.H, base + L.pk_k, s);
+        if (e == cudaSuccess) e = tc::q4_pack(&lm, 1, d.V, d.H, base + L.pk_lm, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) {
+            delete m;
+            DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("4-bit weight packing: ") + cudaGetErrorString(e));
+        }
+        m->wk_all.packed = base + L.pk_k;
+        m->lm_head.packed = base + L.pk_lm;
+    }
     if (d.r > 0) m->w2 = make_ref(w->markov_w2, d.V, d.r, q);
     if (d.conf_head) m->conf_proj = make_ref(w->confidence_proj, 1, d.conf_in, q);
     m->w1 = w->markov_w1;
     m->final_norm = w->norm;
     m->conf_bias = w->confidence_bias;
     // norm bounds of the pruned walk: once per model, from the weights as given
-    if (walk_prune_model_supported(d) && aligned16(m->w1) && aligned16(m->w2.w)) {
+    if (walk_prune_model_supported(d)) {
         m->ws.w2norm = reinterpret_cast<float*>(base + L.w2norm);
         m->ws.w1max_bits = reinterpret_cast<uint32_t*>(base + L.w1max);
         e = launch_markov_norms(m, s);
@@ -375,15 +517,12 @@ int dspark_model_create(const dspark_config* cfg, const dspark_weights* w, void*
             DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("markov norm bounds: ") + cudaGetErrorString(e));
         }
     }
-    rc = gemm_prepare_model(m);
-    if (rc != DSPARK_OK) { delete m; return rc; }
     *out = m;
     return DSPARK_OK;
 }
 
 int dspark_model_destroy(dspark_model* m) {
     if (!m) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "model is NULL");
-    gemm_release_model(m);
     delete m;
     return DSPARK_OK;
 }
@@ -461,7 +600,7 @@ static int check_cache(const dspark_model* m, const dspark_kv_cache* c, int A, i
 static AttnArgs attn_args(const dspark_model* m, const DraftPlan& p, void* ws, const dspark_kv_cache* c, int layer, int A,
                           const void* q, const void* kb, const void* vb, void* out, int io_dtype) {
     const Dims& d = m->d;
-    const size_t es = esize(d.dtype);
+    const size_t es = esize(d.kv_dtype);
     const size_t layer_bytes = (size_t)c->batch * c->capacity * d.nKv * d.hd * es;
     AttnArgs a{};
     a.q = q; a.kb = kb; a.vb = vb; a.out = out;
@@ -470,6 +609,7 @@ static AttnArgs attn_args(const dspark_model* m, const DraftPlan& p, void* ws, c
     a.vc = static_cast<const char*>(c->v) + layer_bytes * layer;
     a.len = c->len; a.capacity = c->capacity; a.batch = c->batch;
     a.part_o = at<float>(ws, p.part_o); a.part_ml = at<float>(ws, p.part_ml);
+    a.plan = p.attn_tc_grid ? at<int>(ws, p.attn_plan) : nullptr; a.tc_grid = p.attn_tc_grid;
     a.A = A; a.n_splits = p.attn_splits; a.chunk = p.attn_chunk;
     a.status = m->ws.status;
     // algorithmic work: every valid context row's K and V once, the block K/V, q and out
@@ -494,7 +634,7 @@ int dspark_attend(const dspark_model* m, int32_t layer, const dspark_kv_cache* c
     if (!q || !k_blk || !v_blk || !out || !ws) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "q, k_blk, v_blk, out and ws must be non-NULL");
     const DraftPlan p = plan_draft(m, A, max_ctx_len);
     if (ws_bytes < p.total) DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "ws smaller than dspark_draft_workspace_bytes(): " + std::to_string(p.total));
-    const AttnArgs a = attn_args(m, p, ws, cache, layer, A, q, k_blk, v_blk, out, m->d.dtype);
+    const AttnArgs a = attn_args(m, p, ws, cache, layer, A, q, k_blk, v_blk, out, m->d.kv_dtype);
     cudaError_t e = run_attention(m, a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
     return DSPARK_OK;
@@ -516,6 +656,8 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     const size_t dump_layer = (size_t)A * d.gamma * d.nH * d.hd * sizeof(float);
     if (m->attn_dump && m->attn_dump_bytes < dump_layer * d.Lyr)
         DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "attention dump smaller than num_hidden_layers * A * gamma * nH * hd floats");
+    if (m->logit_dump && m->logit_dump_bytes < (size_t)A * d.gamma * sizeof(LogitRowStat))
+        DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "logit statistics dump smaller than A * gamma * 16 bytes");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int M = p.M;
     float* h = at<float>(ws, p.h);
@@ -524,10 +666,11 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     float* U = base_logits ? base_logits : at<float>(ws, p.U);
     ActBuf x, ao, act;
     x.f32 = at<float>(ws, p.x); ao.f32 = at<float>(ws, p.attn_out); act.f32 = at<float>(ws, p.act);
+    if (p.tc) {
+        x.hi = at<__half>(ws, p.x_hi); ao.hi = at<__half>(ws, p.ao_hi); act.hi = at<__half>(ws, p.act_hi);
+    }
     if (p.pairs) {
-        x.hi = at<bf16>(ws, p.x_hi); x.lo = at<bf16>(ws, p.x_lo);
-        ao.hi = at<bf16>(ws, p.ao_hi); ao.lo = at<bf16>(ws, p.ao_lo);
-        act.hi = at<bf16>(ws, p.act_hi); act.lo = at<bf16>(ws, p.act_lo);
+        x.lo = at<__half>(ws, p.x_lo); ao.lo = at<__half>(ws, p.ao_lo); act.lo = at<__half>(ws, p.act_lo);
     }
     const int Nqk = (d.nH + d.nKv) * d.hd;
     PartView pv;
@@ -535,7 +678,6 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     // the persistent walk's grid-barrier counter
     cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, p.ticket), 0, sizeof(uint32_t), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(at<void>(ws, p.walk_keys), 0, (size_t)d.gamma * A * 8, s);
-    if (e == cudaSuccess && p.prune) e = cudaMemsetAsync(at<void>(ws, p.prune_words), 0, (size_t)M * 8 + 4, s);
     if (e == cudaSuccess) e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
     for (int l = 0; l < d.Lyr && e == cudaSuccess; ++l) {
         const LayerRef& L = m->layers[l];
@@ -544,6 +686,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
         if (e == cudaSuccess) {
             AttnArgs a = attn_args(m, p, ws, cache, l, A, q, kb, vb, ao.f32, DSPARK_DTYPE_F32);
             a.out_hi = ao.hi; a.out_lo = ao.lo;
+            a.plan_ready = l > 0;           // every layer attends over the same lengths
             e = run_attention(m, a, s);
         }
         if (e == cudaSuccess && m->attn_dump)
@@ -556,43 +699,42 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
         if (e == cudaSuccess) e = run_gemm(m, act, L.down, M, d.H, d.I, part, sc, &pv, DSPARK_TIMER_GEMM_DOWN, s);
         if (e == cudaSuccess) e = launch_down_epilogue(m, l, pv, M, h, x, s);
     }
-    if (e == cudaSuccess) e = run_lm_head(m, x, M, U, s);
+    TileStats ts;
+    ts.mx = at<float>(ws, p.st_mx); ts.arg = at<int>(ws, p.st_arg); ts.se = at<float>(ws, p.st_se);
+    if (d.r > 0) { ts.lo = at<float>(ws, p.st_lo); ts.hi = at<float>(ws, p.st_hi); }
+    ts.M = M; ts.n_tiles = p.n_vt;
+    if (e == cudaSuccess) e = run_lm_head(m, x, M, U, ts, s);
     if (e == cudaSuccess) {
-        WalkArgs wa{};
-        wa.U = U; wa.tokens = tokens; wa.prev = at<int32_t>(ws, p.prev);
-        wa.part_val = at<float>(ws, p.walk_val); wa.part_idx = at<int32_t>(ws, p.walk_idx);
-        wa.ticket = at<uint32_t>(ws, p.ticket); wa.A = A; wa.nblk = p.walk_blocks; wa.status = m->ws.status;
-        const double w2b = d.r > 0 ? (d.quant ? (double)d.V * d.r * 0.5 + (double)d.V * (d.r / d.group) * 4.0
-                                              : (double)d.V * d.r * esize(d.dtype)) : 0.0;
-        if (tc::walk_tc_supported(m, A)) {
-            const int* skip = nullptr;
-            if (p.prune) {
-                PruneScratch ps;
-                ps.T = at<uint32_t>(ws, p.prune_words);
-                ps.cnt = at<int>(ws, p.prune_words + (size_t)M * 4);
-                ps.fail = at<int>(ws, p.prune_words + (size_t)M * 8);
-                ps.list = at<int>(ws, p.prune_list);
-                // algorithmic bytes: the two scans of U
-                KernelTimer t(DSPARK_TIMER_WALK, s, 2.0 * 4.0 * A * d.gamma * (double)d.V, 0.0);
-                e = launch_walk_prune(m, U, anchors, tokens, A, ps, s);
-                skip = ps.fail;
-            }
-            // with the pruned walk ahead, the full walk runs only when a candidate list
-            // overflowed: its work is then not counted (it usually returns at once)
-            const bool full_counted = skip == nullptr;
-            KernelTimer t(DSPARK_TIMER_WALK, s, full_counted ? d.gamma * (w2b + 4.0 * A * d.V) : 0.0,
-                          full_counted ? 2.0 * d.gamma * A * (double)d.V * d.r : 0.0);
-            if (e == cudaSuccess)
-                e = tc::launch_walk_tc(m, U, anchors, tokens, at<unsigned long long>(ws, p.walk_keys), wa.ticket, skip, A, s);
-        } else if (walk_persistent_supported(m, A)) {
-            KernelTimer t(DSPARK_TIMER_WALK, s, d.gamma * (w2b + 4.0 * A * d.V), 2.0 * d.gamma * A * (double)d.V * d.r);
-            e = launch_walk_persistent(m, U, anchors, tokens, wa.part_val, wa.part_idx, wa.ticket, A, s);
-        } else {
-            e = launch_walk_init(anchors, wa.prev, wa.ticket, A, d.V, m->ws.status, s);
-            for (int k = 0; k < d.gamma && e == cudaSuccess; ++k) {
-                wa.step = k;
-                KernelTimer t(DSPARK_TIMER_WALK, s, w2b + 4.0 * A * d.V, 2.0 * A * (double)d.V * d.r);
-                e = launch_walk_step(m, wa, s);
+        // exact pruning: candidate lists from the tile statistics, then the walk over them
+        PruneScratch ps;
+        ps.cnt = at<int>(ws, p.prune_cnt); ps.fail = at<int>(ws, p.prune_fail); ps.list = at<int>(ws, p.prune_list);
+        LogitRowStat* row_out = static_cast<LogitRowStat*>(m->logit_dump);
+        {
+            // algorithmic bytes: the tile statistics (the candidate tiles' U rows depend on the data)
+            KernelTimer t(DSPARK_TIMER_WALK, s, (double)p.n_vt * M * (d.r > 0 ? 20.0 : 12.0), 0.0);
+            e = launch_walk_prune(m, U, ts, anchors, tokens, A, ps, row_out, s);
+        }
+        if (e == cudaSuccess && d.r > 0) {
+            // the full walk runs only when a candidate list overflowed (it returns at once
+            // otherwise), so its work is not counted
+            const int* skip = ps.fail;
+            KernelTimer t(DSPARK_TIMER_WALK, s, 0.0, 0.0);
+            WalkArgs wa{};
+            wa.U = U; wa.tokens = tokens; wa.prev = at<int32_t>(ws, p.prev);
+            wa.part_val = at<float>(ws, p.walk_val); wa.part_idx = at<int32_t>(ws, p.walk_idx);
+            wa.ticket = at<uint32_t>(ws, p.ticket); wa.A = A; wa.nblk = p.walk_blocks; wa.status = m->ws.status;
+            wa.skip = skip;
+            if (tc::walk_tc_supported(m, A)) {
+                e = tc::launch_walk_tc(m, U, anchors, tokens, at<unsigned long long>(ws, p.walk_keys), wa.ticket, skip,
+                                       A, s);
+            } else if (walk_persistent_supported(m, A)) {
+                e = launch_walk_persistent(m, U, anchors, tokens, wa.part_val, wa.part_idx, wa.ticket, skip, A, s);
+            } else {
+                e = launch_walk_init(anchors, wa.prev, wa.ticket, A, d.V, m->ws.status, skip, s);
+                for (int k = 0; k < d.gamma && e == cudaSuccess; ++k) {
+                    wa.step = k;
+                    e = launch_walk_step(m, wa, s);
+                }
             }
         }
     }
@@ -606,6 +748,14 @@ int dspark_debug_attention_dump(dspark_model* m, float* dst, size_t bytes) {
     if (dst && (reinterpret_cast<uintptr_t>(dst) & 15u)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "dst must be 16-byte aligned");
     m->attn_dump = dst;
     m->attn_dump_bytes = dst ? bytes : 0;
+    return DSPARK_OK;
+}
+
+int dspark_debug_logit_stats(dspark_model* m, void* dst, size_t bytes) {
+    if (!m) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "model is NULL");
+    if (dst && (reinterpret_cast<uintptr_t>(dst) & 15u)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "dst must be 16-byte aligned");
+    m->logit_dump = dst;
+    m->logit_dump_bytes = dst ? bytes : 0;
     return DSPARK_OK;
 }
 

@@ -127,59 +127,70 @@ attn_partial_kernel(AttnArgs a, int G, int nH, int nKv, int hd, int dtype) {
     }
 }
 
-constexpr int kMergeBatch = 32;      // splits a merge thread loads at once
+constexpr int kMergeWarps = 8;       // query rows per merge CTA (one warp each)
 
-// grid (A * nH * G), block hd: merge the splits of one query row of one head.
-__global__ void attn_merge_kernel(AttnArgs a, int G, int nH, int hd) {
+// One warp per query row (b, h, i): the splits' (max, sum) pairs are read by
+// lane s (loops over 32 splits at a time), the weights w_s = exp(m_s - M)
+// combine the unnormalised outputs, lane l owning the 4-column groups l, l + 32,
+// ... of the row (float4 loads). Empty splits (m = -inf) weigh nothing.
+__global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(AttnArgs a, int G, int nH, int hd, int rows) {
     pdl_trigger();
     pdl_wait();
-    const int row = blockIdx.x;                 // ((b * nH) + h) * G + i
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);   // ((b * nH) + h) * G + i
+    if (row >= rows) return;
     const int i = row % G, bh = row / G;
     const int b = bh / nH, h = bh % nH;
-    const int d = threadIdx.x;
     const int S1 = a.S1;
-    float num = 0.f, den = 0.f;
-    if (S1 <= kMergeBatch) {
-        // every split's (max, sum, O) in flight at once: one round of memory latency
-        float mv[kMergeBatch], lv[kMergeBatch], ov[kMergeBatch];
+    // the row maximum over the splits
+    float M = -INFINITY;
+    for (int s = lane; s < S1; s += 32) M = fmaxf(M, a.part_ml[(((int64_t)bh * S1 + s) * G + i) * 2]);
 #pragma unroll
-        for (int s = 0; s < kMergeBatch; ++s) {
-            const int64_t base = ((int64_t)bh * S1 + s) * G + i;
-            mv[s] = s < S1 ? a.part_ml[base * 2] : -INFINITY;
-            lv[s] = s < S1 ? a.part_ml[base * 2 + 1] : 0.f;
-            ov[s] = s < S1 ? a.part_o[base * hd + d] : 0.f;
-        }
-        float M = -INFINITY;
-#pragma unroll
-        for (int s = 0; s < kMergeBatch; ++s) M = fmaxf(M, mv[s]);
-#pragma unroll
-        for (int s = 0; s < kMergeBatch; ++s) {
-            const float w = mv[s] == -INFINITY ? 0.f : expf(mv[s] - M);   // empty splits carry no weight
-            den += w * lv[s];
-            num += w * (mv[s] == -INFINITY ? 0.f : ov[s]);
-        }
-    } else {
-        float M = -INFINITY;
-#pragma unroll 8
-        for (int s = 0; s < S1; ++s) M = fmaxf(M, a.part_ml[(((int64_t)bh * S1 + s) * G + i) * 2]);
-#pragma unroll 8
-        for (int s = 0; s < S1; ++s) {
-            const int64_t base = ((int64_t)bh * S1 + s) * G + i;
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const int ng = hd / 4;                      // float4 groups of the row
+    float4 num[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    float den = 0.f;
+    for (int s0 = 0; s0 < S1; s0 += 32) {
+        float ws = 0.f, ls = 0.f;
+        if (s0 + lane < S1) {
+            const int64_t base = ((int64_t)bh * S1 + s0 + lane) * G + i;
             const float m = a.part_ml[base * 2];
-            const float l = a.part_ml[base * 2 + 1];
-            const float o = m == -INFINITY ? 0.f : a.part_o[base * hd + d];
-            const float w = m == -INFINITY ? 0.f : expf(m - M);
-            den += w * l;
-            num += w * o;
+            ls = a.part_ml[base * 2 + 1];
+            ws = m == -INFINITY ? 0.f : __expf(m - M);
+        }
+        const int cnt = min(32, S1 - s0);
+        for (int t = 0; t < cnt; ++t) {
+            const float w = __shfl_sync(0xffffffffu, ws, t);
+            den += w * __shfl_sync(0xffffffffu, ls, t);
+            if (w == 0.f) continue;                 // uniform: an empty split
+            const float* o = a.part_o + (((int64_t)bh * S1 + s0 + t) * G + i) * hd;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int g4 = lane + q * 32;
+                if (g4 < ng) {
+                    const float4 v = reinterpret_cast<const float4*>(o)[g4];
+                    num[q].x += w * v.x; num[q].y += w * v.y; num[q].z += w * v.z; num[q].w += w * v.w;
+                }
+            }
         }
     }
-    const int64_t o = (((int64_t)b * G + i) * nH + h) * hd + d;
-    const float v = num / den;
-    store_any(a.out, o, a.out_dtype, v);
-    if (a.out_hi) {
-        const __nv_bfloat16 hv = __float2bfloat16_rn(v);
-        a.out_hi[o] = hv;
-        a.out_lo[o] = __float2bfloat16_rn(v - __bfloat162float(hv));
+    const float inv = 1.f / den;
+    const int64_t ob = (((int64_t)b * G + i) * nH + h) * hd;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int g4 = lane + q * 32;
+        if (g4 >= ng) continue;
+        const float v[4] = {num[q].x * inv, num[q].y * inv, num[q].z * inv, num[q].w * inv};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int64_t o = ob + g4 * 4 + c;
+            store_any(a.out, o, a.out_dtype, v[c]);
+            if (a.out_hi) {
+                const __half hv = __float2half_rn(v[c]);
+                a.out_hi[o] = hv;
+                if (a.out_lo) a.out_lo[o] = __float2half_rn(v[c] - __half2float(hv));
+            }
+        }
     }
 }
 
@@ -202,14 +213,17 @@ cudaError_t launch_attention_simt(const dspark_model* m, const AttnArgs& a_in, c
         configured_dev = m->device;
     }
     dim3 grid(a.A * d.nH, a.n_splits + 1);
-    cudaError_t e = launch_pdl(attn_partial_kernel, grid, dim3(kThreads), smem, s, a, d.gamma, d.nH, d.nKv, d.hd, d.dtype);
+    cudaError_t e = launch_pdl(attn_partial_kernel, grid, dim3(kThreads), smem, s, a, d.gamma, d.nH, d.nKv, d.hd,
+                               d.kv_dtype);
     if (e != cudaSuccess) return e;
     return launch_attention_merge(m, a, s);
 }
 
 cudaError_t launch_attention_merge(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
     const Dims& d = m->d;
-    return launch_pdl(attn_merge_kernel, dim3(a.A * d.nH * d.gamma), dim3(d.hd), 0, s, a, d.gamma, d.nH, d.hd);
+    const int rows = a.A * d.nH * d.gamma;
+    return launch_pdl(attn_merge_kernel, dim3((rows + kMergeWarps - 1) / kMergeWarps), dim3(kMergeWarps * 32), 0, s, a,
+                      d.gamma, d.nH, d.hd, rows);
 }
 
 }  // namespace dspark

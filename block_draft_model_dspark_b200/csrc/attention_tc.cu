@@ -4,13 +4,14 @@
 // and at scale 1.0, over the row's cached context keys followed by the
 // block's own keys; GQA maps query head h to kv head h / (nH / nKv).
 //
-// One CTA = (row b, kv head g, key split). Its query tile is the 128-row MMA
+// One CTA = a range of key tiles of one item (row b, kv head g), as the plan
+// kernel assigns them from the device-side lengths (ragged rows get CTAs in
+// proportion to their tiles; every CTA runs in one wave). Its query tile is the 128-row MMA
 // side: the grp * gamma queries of the heads that share kv head g (row r =
 // query i * grp + head-in-group). Key tiles of KT = 64 rows are TMA-loaded
-// from the bf16 cache (3-D maps pick kv head g out of [rows, nKv, hd]) and
-// converted in place to fp16, so both MMAs run as kind::f16 with fp16
-// operands: q and the probabilities P keep an 11-bit mantissa (bf16 has 8)
-// and the bf16 keys and values convert exactly.
+// from the fp16 cache (4-D maps pick kv head g out of [rows, nKv, hd]) and
+// multiplied as they land: both MMAs run as kind::f16 with fp16 operands (q
+// and the probabilities P keep an 11-bit significand; the cache holds fp16).
 //   S = Q K^T  -> TMEM, two 64-column buffers (tile t in buffer t % 2)
 //   softmax    -> one thread per query row (TMEM lane = row); the running max
 //                 is raised only when a tile's max exceeds it by more than
@@ -18,23 +19,24 @@
 //   O += P V   -> TMEM (hd columns), P fp16 from shared memory (K-major,
 //                 128-byte swizzle), V as an MN-major operand
 // K and V tiles have two shared-memory slots each, so the loads of tile t + 2
-// are in flight while tile t is converted and multiplied; per 64 keys at
-// hd = 256 the tensor cores run 16 (S) + 4 (P V) MMAs.
+// are in flight while tile t is multiplied; per 64 keys at hd = 256 the
+// tensor cores run 16 (S) + 4 (P V) MMAs.
 //
-// Warp roles (576 threads): warps 0-7 run the softmax, two threads per query
+// Warp roles (352 threads): warps 0-7 run the softmax, two threads per query
 // row (warps w and w + 4 share TMEM lanes 32 (w % 4) ..; each takes 32 of the
 // tile's 64 columns and half of O's columns; the row max is exchanged through
-// shared memory), warps 8-15 convert K and V tiles (and zero the rows past the
-// last key: stale cache bytes could be NaN, and P = 0 times NaN still poisons
-// the accumulator), warp 16 issues the S products and K loads, warp 17 the
-// P V products and V loads. K, V and P have two
-// slots each and S two TMEM buffers, so tile t + 1's load, conversion and S
-// product and tile t - 1's P V product all overlap tile t's softmax; the
-// softmax waits for P V of tile t - 1 only to rescale O (rare). Every wait is
-// bounded. Shared memory at hd = 256: Q 64 KB, K, V 2 x 32 KB each, P 2 x 16 KB.
+// shared memory), warp 8 issues the S products and K loads, warp 9 the P V
+// products and V loads, and warp 10 zeroes the V rows past the last key of a
+// partial tile before its product (stale cache rows may hold any bits, and
+// P = 0 times NaN still poisons the accumulator; K needs no fix: those S
+// columns are masked to -inf). K, V and P have two slots each and S two TMEM
+// buffers, so tile t + 1's load and S product and tile t - 1's P V product all
+// overlap tile t's softmax; the softmax waits for P V of tile t - 1 only to
+// rescale O (rare). Every wait is bounded. Shared memory at hd = 256: Q 64 KB,
+// K, V 2 x 32 KB each, P 2 x 16 KB.
 //
-// The CTA writes its unnormalised O with (max, sum) per query row: the split
-// layout the merge kernel reads. The last split of each (b, g) also takes the
+// The CTA writes its unnormalised O with (max, sum) per query row into its own
+// slot, which the merge kernel combines per item. The last range of each (b, g) also takes the
 // block's own keys, as one more tile.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -49,57 +51,129 @@
 
 namespace dspark {
 
-cudaError_t launch_attention_merge(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
-
 namespace tc {
 namespace {
 
-constexpr int kThreads = 576;
+constexpr int kThreads = 352;
 constexpr int kSoftThreads = 256;    // warps 0-7
-constexpr int kConvThreads = 256;    // warps 8-15
-constexpr int kIssuerWarp = 16;      // S products and K loads; warp 17: P V products and V loads
+constexpr int kIssuerWarp = 8;       // S products and K loads; warp 9: P V products and V loads
+constexpr int kFixWarp = 10;         // zeroes the V rows past the last key of a partial tile
 constexpr int KT = 64;               // keys per tile
+constexpr int kSlots = 3;            // shared-memory slots of K tiles, and of V tiles (loads in flight)
+constexpr int kQCol = 2 * KT + 256;  // TMEM columns: S buffers [0, 2 KT), O [2 KT, 2 KT + hd), Q from 384
 constexpr int QROWS = 128;           // MMA M
 constexpr float kRescale = 5.0f;     // natural-log headroom before the running max is raised
 
 struct AttnTcParams {
-    int A, G, nH, nKv, grp, hd, capacity, S1, chunk, q_dtype;
-    const void* q;                   // [A, G, nH, hd] (fp32 or bf16)
+    int A, G, nH, nKv, grp, hd, capacity, q_dtype;
+    const void* q;                   // [A, G, nH, hd] (fp32 or fp16)
     const int32_t* len;
-    float* part_o; float* part_ml;
+    float* part_o; float* part_ml;   // one slot per CTA: [CTA][128 rows][hd] and [CTA][128 rows][2]
+    const int* cta_item;             // [grid] the (row, kv head) item of each CTA (-1: idle)
+    const int* cta_t0; const int* cta_t1;   // [grid] its tile range within the item
     int32_t* status;
 };
+
+// The work plan (one CTA, device lengths): item i = (row b, kv head g) has n_i =
+// ceil(len_b / KT) context tiles plus the block tile. The smallest q with
+// sum_i ceil(n_i / q) <= grid splits item i into k_i = ceil(n_i / q) equal
+// tile ranges, one CTA each (all CTAs in one wave, none above q tiles);
+// item_cta0 is the exclusive prefix sum of k_i (the CTAs, and partial slots,
+// of item i are item_cta0[i] .. item_cta0[i + 1] - 1).
+constexpr int kPlanThreads = 1024;
+__device__ __forceinline__ int plan_tiles(const int32_t* len, int b, int capacity) {
+    const int L = min(max(len[b], 0), capacity);
+    return (L + KT - 1) / KT + 1;
+}
+__device__ __forceinline__ int block_sum_int(int v, int* red) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if (lane == 0) red[wid] = v;
+    __syncthreads();
+    int t = 0;
+    for (int w = 0; w < kPlanThreads / 32; ++w) t += red[w];
+    return t;
+}
+__global__ void __launch_bounds__(kPlanThreads) attn_plan_kernel(const int32_t* __restrict__ len, int A, int nKv,
+                                                                 int capacity, int grid, int* __restrict__ cta_item,
+                                                                 int* __restrict__ cta_t0, int* __restrict__ cta_t1,
+                                                                 int* __restrict__ item_cta0) {
+    __shared__ int red[kPlanThreads / 32];
+    __shared__ int s_base;
+    pdl_trigger();
+    pdl_wait();
+    const int tid = threadIdx.x, n_items = A * nKv;
+    int mx = 1;
+    for (int i = tid; i < n_items; i += kPlanThreads) mx = max(mx, plan_tiles(len, i / nKv, capacity));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    __syncthreads();
+    if ((tid & 31) == 0) red[tid >> 5] = mx;
+    __syncthreads();
+    mx = 1;
+    for (int w = 0; w < kPlanThreads / 32; ++w) mx = max(mx, red[w]);
+    // the smallest q (tiles per CTA) whose splits fit the grid (q = mx needs n_items <= grid
+    // CTAs), at least 2: a CTA also builds its query tile and writes a 128-row partial
+    // state, and one tile per CTA measured slower at a single 4096-key row
+    int lo = min(2, mx), hi = mx;
+    while (lo < hi) {
+        const int mid = (lo + hi) / 2;
+        int cnt = 0;
+        for (int i = tid; i < n_items; i += kPlanThreads) cnt += (plan_tiles(len, i / nKv, capacity) + mid - 1) / mid;
+        cnt = block_sum_int(cnt, red);
+        if (cnt <= grid) hi = mid; else lo = mid + 1;
+    }
+    const int q = lo;
+    // exclusive scan of k_i over the items, in chunks of kPlanThreads
+    if (tid == 0) s_base = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < n_items; i0 += kPlanThreads) {
+        const int i = i0 + tid;
+        const int n = i < n_items ? plan_tiles(len, i / nKv, capacity) : 0;
+        const int k = i < n_items ? (n + q - 1) / q : 0;
+        int x = k;                                        // inclusive scan within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if ((tid & 31) >= o) x += y;
+        }
+        __syncthreads();
+        if ((tid & 31) == 31) red[tid >> 5] = x;
+        __syncthreads();
+        int wbase = 0;
+        for (int w = 0; w < (tid >> 5); ++w) wbase += red[w];
+        const int excl = s_base + wbase + x - k;
+        if (i < n_items) {
+            item_cta0[i] = excl;
+            // the item's k ranges of n tiles: range j is [j n / k, (j + 1) n / k)
+            for (int j = 0; j < k; ++j) {
+                cta_item[excl + j] = i;
+                cta_t0[excl + j] = (int)((int64_t)j * n / k);
+                cta_t1[excl + j] = (int)((int64_t)(j + 1) * n / k);
+            }
+        }
+        __syncthreads();
+        if (tid == kPlanThreads - 1) s_base = excl + k;
+        __syncthreads();
+    }
+    const int total = s_base;
+    if (tid == 0) item_cta0[n_items] = total;
+    for (int c = total + tid; c < grid; c += kPlanThreads) { cta_item[c] = -1; cta_t0[c] = 0; cta_t1[c] = 0; }
+}
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
     const __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// bf16 -> fp16 in place over a tile of `nsub` sub-tiles [KT rows x 128 B] by
-// the converter threads; rows >= nvalid become zeros.
-// Each thread owns 16-byte chunks ct, ct + kConvThreads, ...; all its loads
-// are issued before the first conversion (one round of shared-memory latency).
-__device__ __forceinline__ void convert_tile(uint8_t* tile, int nsub, int nvalid, int ct) {
-    constexpr int kPer = 4 * KT * 8 / kConvThreads;    // chunks per thread at nsub = 4
-    const int n16 = nsub * KT * 8;
-    uint4* p = reinterpret_cast<uint4*>(tile);
-    uint4 u[kPer];
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-        const int i = ct + k * kConvThreads;
-        u[k] = i < n16 ? p[i] : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-        const int i = ct + k * kConvThreads;
-        if (i >= n16) break;
-        const int row = (i >> 3) % KT;
-        if (row >= nvalid) { p[i] = make_uint4(0u, 0u, 0u, 0u); continue; }
-        const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
-        uint32_t o[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) o[j] = pack_half2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
-        p[i] = make_uint4(o[0], o[1], o[2], o[3]);
+// Zeroes rows [nvalid, KT) of a V tile of `nsub` sub-tiles [KT rows x 128 B] (one warp).
+__device__ __forceinline__ void zero_tail(uint8_t* tile, int nsub, int nvalid, int lane) {
+    const int per_sub = (KT - nvalid) * 8;          // 16-byte chunks past the last key, per sub-tile
+    for (int c = lane; c < nsub * per_sub; c += 32) {
+        const int sub = c / per_sub, r = c % per_sub;
+        reinterpret_cast<uint4*>(tile + sub * KT * 128 + nvalid * 128)[r] = make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
@@ -139,37 +213,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     const int hd = P.hd, nsub = hd / 64;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tile_sz = nsub * KT * 128;                  // one K or V tile: nsub x [64 keys x 128 B]
-    uint8_t* sQ = base;                                   // nsub x [128 rows x 128 B] fp16
-    uint8_t* sK = sQ + nsub * QROWS * 128;                // 2 slots x tile
-    uint8_t* sV = sK + 2 * tile_sz;                       // 2 slots x tile
-    uint8_t* sP = sV + 2 * tile_sz;                       // 2 slots x [128 rows x 128 B]
+    uint8_t* sK = base;                                   // kSlots x tile
+    uint8_t* sV = sK + kSlots * tile_sz;                  // kSlots x tile
+    uint8_t* sP = sV + kSlots * tile_sz;                  // 2 slots x [128 rows x 128 B]
     float* red = reinterpret_cast<float*>(sP + 2 * QROWS * 128);   // [2 halves][128 rows] row maxima / sums
     uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * QROWS);
-    uint64_t* kfull = bars + 0;      // [2] K tile landed in the slot (TMA)
-    uint64_t* vfull = bars + 2;      // [2] V tile landed in the slot (TMA)
-    uint64_t* kready = bars + 4;     // [2] K tile of the slot converted (128 arrivals)
-    uint64_t* vready = bars + 6;     // [2] V tile of the slot converted (128 arrivals)
-    uint64_t* sdone = bars + 8;      // [2] S product of the tile in that buffer done (its K slot free)
-    uint64_t* sfree = bars + 10;     // [2] softmax has read the S buffer (128 arrivals)
-    uint64_t* pready = bars + 12;    // [2] P slot written (256 arrivals)
-    uint64_t* odone = bars + 14;     // [2] P V product of the tile in that P slot done (its V slot free, O settled)
-    uint64_t* spare = bars + 16;     // teardown: MMAs in flight after an abort
-    uint64_t* xw = bars + 17;        // row-max exchange: both halves wrote (256 arrivals)
-    uint64_t* xr = bars + 18;        // row-max exchange: both halves read (256 arrivals)
-    uint64_t* spare2 = bars + 19;    // teardown of the P V issuer
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+    uint64_t* kfull = bars + 0;                // [kSlots] K tile landed in the slot (TMA)
+    uint64_t* vfull = kfull + kSlots;          // [kSlots] V tile landed in the slot (TMA)
+    uint64_t* vready = vfull + kSlots;         // [kSlots] V tile of the slot ready for its product (1 arrival)
+    uint64_t* kfree = vready + kSlots;         // [kSlots] the S product that read the K slot is done
+    uint64_t* vfree = kfree + kSlots;          // [kSlots] the P V product that read the V slot is done
+    uint64_t* sdone = vfree + kSlots;          // [2] S product of the tile in that buffer done
+    uint64_t* sfree = sdone + 2;               // [2] softmax has read the S buffer (256 arrivals)
+    uint64_t* pready = sfree + 2;              // [2] P slot written (256 arrivals)
+    uint64_t* odone = pready + 2;              // [2] P V product of the tile in that P slot done (O settled)
+    uint64_t* spare = odone + 2;               // teardown: MMAs in flight after an abort
+    uint64_t* xw = spare + 1;                  // row-max exchange: both halves wrote (256 arrivals)
+    uint64_t* xr = xw + 1;                     // row-max exchange: both halves read (256 arrivals)
+    uint64_t* spare2 = xr + 1;                 // teardown of the P V issuer
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(spare2 + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x;                            // b * nKv + g
-    const int b = bh / P.nKv, g = bh % P.nKv;
-    const int split = blockIdx.y;
     const int nq = P.grp * P.G;
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&kfull[i], 1); mbar_init(&vfull[i], 1);
-            mbar_init(&kready[i], kConvThreads); mbar_init(&vready[i], kConvThreads);
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(&kfull[i], 1); mbar_init(&vfull[i], 1); mbar_init(&vready[i], 1);
+            mbar_init(&kfree[i], 1); mbar_init(&vfree[i], 1);
         }
         mbar_init(&sdone[0], 1); mbar_init(&sdone[1], 1);
         mbar_init(&sfree[0], kSoftThreads); mbar_init(&sfree[1], kSoftThreads);
@@ -189,27 +260,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     // pdl_trigger: the merge launches as these CTAs exit (see gemm_tc.cu)
     pdl_wait();
 
+    // this CTA's work: tiles [t_lo, t_hi) of item (b, g) (the plan's); an idle CTA has none
+    const int slot = blockIdx.x;
+    const int item = P.cta_item[slot];
+    const int b = item >= 0 ? item / P.nKv : 0, g = item >= 0 ? item % P.nKv : 0;
+    const int t_lo = item >= 0 ? P.cta_t0[slot] : 0, t_hi = item >= 0 ? P.cta_t1[slot] : 0;
     int len = P.len[b];
     if (len < 0 || len > P.capacity) {
         if (tid == 0) atomicOr(P.status, DSPARK_DEV_BAD_LENGTH);
         len = min(max(len, 0), P.capacity);
     }
-    // this split's context keys [c0, c1), then (last split) the block's G keys
-    const int c0 = min(len, split * P.chunk), c1 = min(len, c0 + P.chunk);
-    const bool has_blk = split == P.S1 - 1;
-    const int n_ctx = (c1 - c0 + KT - 1) / KT;
-    const int nt = n_ctx + (has_blk ? 1 : 0);
+    // the item's tiles: ceil(len / KT) context tiles of KT keys, then the block's G keys
+    const int n_ctx_all = (len + KT - 1) / KT;
+    const int nt = t_hi - t_lo;
     auto tile_rows = [&](int t, int* row, int* nvalid, bool* blk) {
-        if (t < n_ctx) { *row = b * P.capacity + c0 + t * KT; *nvalid = min(KT, c1 - (c0 + t * KT)); *blk = false; }
+        const int u = t_lo + t;
+        if (u < n_ctx_all) { *row = b * P.capacity + u * KT; *nvalid = min(KT, len - u * KT); *blk = false; }
         else { *row = b * P.G; *nvalid = P.G; *blk = true; }
     };
 
-    // The first two K and V tiles do not depend on Q: their loads go out
+    // The first kSlots K and V tiles do not depend on Q: their loads go out
     // before the Q tile is built, so they land while it is.
     const uint32_t tile_bytes = (uint32_t)nsub * KT * 128;
     if ((warp == kIssuerWarp || warp == kIssuerWarp + 1) && lane == 0) {
         const bool v_tile = warp != kIssuerWarp;
-        for (int t = 0; t < 2 && t < nt; ++t) {
+        for (int t = 0; t < kSlots && t < nt; ++t) {
             int row, nvalid; bool blk;
             tile_rows(t, &row, &nvalid, &blk);
             const CUtensorMap* m = blk ? (v_tile ? &tmVb : &tmKb) : (v_tile ? &tmV : &tmK);
@@ -219,50 +294,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         }
     }
 
-    // Q tile (all warps): fp16, 128-byte swizzle; rows past the queries are zero.
-    // Each thread's rows are loaded kQBatch at a time before any is converted:
-    // a few rounds of memory latency instead of one per row.
-    constexpr int kQBatch = 4;
-    for (int cd = 0; cd < hd; cd += 256) {
-        const int d = cd + lane * 8;
-        const int sub = d / 64, chunk = (d % 64) / 8;
-        for (int row0 = warp; row0 < QROWS; row0 += kQBatch * (kThreads / 32)) {
-            float v[kQBatch][8];
+    // Q tile in tensor memory (the S product's A operand): TMEM lane r holds query
+    // row r, two fp16 values per 32-bit column from column kQCol; rows past the
+    // queries are zero. The softmax threads write it, thread (r, half) the row's
+    // half of the head dimensions, 16 columns per tcgen05.st.
+    if (tid < kSoftThreads) {
+        const int r = tid & (QROWS - 1), half = tid >> 7;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const int d0 = half * (hd / 2);
+        const int i = r / P.grp, h = g * P.grp + r % P.grp;
+        const int64_t off = (((int64_t)b * P.G + i) * P.nH + h) * hd + d0;
+        for (int c0 = 0; c0 < hd / 4; c0 += 16) {           // 16 columns = 32 dimensions
+            uint32_t w[16];
 #pragma unroll
-            for (int k = 0; k < kQBatch; ++k) {
-                const int row = row0 + k * (kThreads / 32);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[k][j] = 0.f;
-                if (row < nq && d < hd) {
-                    const int i = row / P.grp, h = g * P.grp + row % P.grp;
-                    const int64_t off = (((int64_t)b * P.G + i) * P.nH + h) * hd + d;
+            for (int j = 0; j < 16; ++j) {
+                float x0 = 0.f, x1 = 0.f;
+                if (r < nq) {
+                    const int d = 2 * (c0 + j);
                     if (P.q_dtype == DSPARK_DTYPE_F32) {
-                        const float4 a0 = *reinterpret_cast<const float4*>(static_cast<const float*>(P.q) + off);
-                        const float4 a1 = *reinterpret_cast<const float4*>(static_cast<const float*>(P.q) + off + 4);
-                        v[k][0] = a0.x; v[k][1] = a0.y; v[k][2] = a0.z; v[k][3] = a0.w;
-                        v[k][4] = a1.x; v[k][5] = a1.y; v[k][6] = a1.z; v[k][7] = a1.w;
+                        const float2 f = *reinterpret_cast<const float2*>(static_cast<const float*>(P.q) + off + d);
+                        x0 = f.x; x1 = f.y;
                     } else {
-                        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(P.q) + off);
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            v[k][2 * j] = __uint_as_float(w[j] << 16);
-                            v[k][2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-                        }
+                        // fp16 queries (the attention seam)
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(static_cast<const __half*>(P.q) + off + d));
+                        x0 = f.x; x1 = f.y;
                     }
                 }
+                w[j] = pack_half2(x0, x1);
             }
-#pragma unroll
-            for (int k = 0; k < kQBatch; ++k) {
-                const int row = row0 + k * (kThreads / 32);
-                if (row < QROWS && d < hd)
-                    *reinterpret_cast<uint4*>(sQ + sub * QROWS * 128 + row * 128 + ((chunk ^ (row & 7)) * 16)) =
-                        make_uint4(pack_half2(v[k][0], v[k][1]), pack_half2(v[k][2], v[k][3]),
-                                   pack_half2(v[k][4], v[k][5]), pack_half2(v[k][6], v[k][7]));
-            }
+            tmem_st_x16(tmem + (uint32_t)(kQCol + half * (hd / 4) + c0) + lane_off, w);
         }
+        tmem_st_wait();
     }
-    fence_async_shared();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -270,9 +333,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     const uint32_t tO = tmem + 2 * KT;                    // O: columns [128, 128 + hd); S buffers at 0 and 64
     bool ok = true;
 
-    if (warp >= kIssuerWarp) {
+    if (warp == kIssuerWarp || warp == kIssuerWarp + 1) {
         // ------------------------------------------------------------ issuers
-        // warp 16: S = Q K^T and the K loads; warp 17: O += P V and the V loads.
+        // warp 8: S = Q K^T and the K loads; warp 9: O += P V and the V loads.
         // Each waits only for what its own products need; a load waits only for its
         // slot to be free, and every wait keeps issuing the loads that can go.
         if (lane == 0) {
@@ -286,14 +349,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             };
             uint8_t* buf = is_qk ? sK : sV;
             uint64_t* fullb = is_qk ? kfull : vfull;
-            uint64_t* doneb = is_qk ? sdone : odone;          // completion of the product that read a slot
-            int nl[2] = {0, 0};                               // loads issued per slot
-            for (int t = 0; t < 2 && t < nt; ++t) ++nl[t];    // tiles 0 and 1: issued before the Q tile
-            int ln = min(2, nt);                              // next tile to load
+            uint64_t* freeb = is_qk ? kfree : vfree;          // completion of the product that read a slot
+            int nl[kSlots] = {};                              // loads issued per slot
+            for (int t = 0; t < kSlots && t < nt; ++t) ++nl[t];   // issued before the Q tile
+            int ln = min(kSlots, nt);                         // next tile to load
             int issued = 0;                                   // products issued
+            // tile ln goes into slot ln % kSlots once the product of tile ln - kSlots (the
+            // slot's previous tile, phase (ln - kSlots) / kSlots of its barrier) is done
             auto service = [&]() {
-                while (ln < nt && ln - 2 < issued && mbar_try_wait(&doneb[ln & 1], (uint32_t)((ln - 2) >> 1) & 1u)) {
-                    load(buf + (ln & 1) * tile_sz, &fullb[ln & 1], !is_qk, ln); ++nl[ln & 1]; ++ln;
+                while (ln < nt && ln - kSlots < issued &&
+                       mbar_try_wait(&freeb[ln % kSlots], (uint32_t)((ln - kSlots) / kSlots) & 1u)) {
+                    load(buf + (ln % kSlots) * tile_sz, &fullb[ln % kSlots], !is_qk, ln);
+                    ++nl[ln % kSlots];
+                    ++ln;
                 }
             };
             auto wait_serving = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -311,39 +379,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             };
             const uint32_t idesc_qk = idesc_f16(QROWS, KT, 0);
             const uint32_t idesc_pv = idesc_f16(QROWS, hd, 1);
-            const uint32_t qa = smem_u32(sQ);
+            const uint32_t qa = tmem + (uint32_t)kQCol;      // Q in tensor memory: 8 columns per 16-wide K slice
             for (int t = 0; t < nt && ok; ++t) {
-                const int sl = t & 1;
+                const int sl = t & 1;                             // S buffer / P slot
+                const int ks = t % kSlots;                        // K / V slot
+                const uint32_t kph = (uint32_t)(t / kSlots) & 1u;
                 if (is_qk) {
                     // S(t) = Q K(t)^T into buffer t % 2
-                    if (!wait_serving(&kready[sl], (uint32_t)(t >> 1) & 1u)) { ok = false; break; }
+                    if (!wait_serving(&kfull[ks], kph)) { ok = false; break; }
                     if (t >= 2 && !wait_serving(&sfree[sl], (uint32_t)((t - 2) >> 1) & 1u)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d = tmem + (uint32_t)(sl * KT);
                     // descriptors advance by address / 16: constants per unrolled slice
-                    const uint64_t ad0 = sdesc_k_sw128(qa);
-                    const uint64_t bd0 = sdesc_k_sw128(smem_u32(sK + sl * tile_sz));
-                    mma_bf16(d, ad0, bd0, idesc_qk, 0u);
+                    const uint64_t bd0 = sdesc_k_sw128(smem_u32(sK + ks * tile_sz));
+                    mma_f16_ts(d, qa, bd0, idesc_qk, 0u);
 #pragma unroll
                     for (int j = 1; j < 16; ++j) {
                         if (j >= hd / 16) break;
-                        const uint64_t aoff = (uint64_t)(((j >> 2) * QROWS * 128 + (j & 3) * 32) >> 4);
                         const uint64_t boff = (uint64_t)(((j >> 2) * KT * 128 + (j & 3) * 32) >> 4);
-                        mma_bf16(d, ad0 + aoff, bd0 + boff, idesc_qk, 1u);
+                        mma_f16_ts(d, qa + (uint32_t)(8 * j), bd0 + boff, idesc_qk, 1u);
                     }
                     mma_commit(&sdone[sl]);
+                    mma_commit(&kfree[ks]);
                 } else {
                     // O += P(t) V(t)
-                    if (!wait_serving(&pready[sl], (uint32_t)(t >> 1) & 1u) ||
-                        !wait_serving(&vready[sl], (uint32_t)(t >> 1) & 1u)) { ok = false; break; }
+                    if (!wait_serving(&pready[sl], (uint32_t)(t >> 1) & 1u) || !wait_serving(&vready[ks], kph)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint64_t ad0 = sdesc_k_sw128(smem_u32(sP + sl * QROWS * 128));
-                    const uint64_t bd0 = sdesc_mn_sw128(smem_u32(sV + sl * tile_sz), KT * 128);
+                    const uint64_t bd0 = sdesc_mn_sw128(smem_u32(sV + ks * tile_sz), KT * 128);
 #pragma unroll
                     for (int j = 0; j < KT / 16; ++j)
                         mma_bf16(tO, ad0 + (uint64_t)((j * 32) >> 4), bd0 + (uint64_t)((j * 2048) >> 4), idesc_pv,
                                  (t > 0 || j > 0) ? 1u : 0u);
                     mma_commit(&odone[sl]);
+                    mma_commit(&vfree[ks]);
                 }
                 issued = t + 1;
                 service();
@@ -352,7 +424,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             if (!ok) {
                 const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
                 bool drained = true;
-                for (int i = 0; i < 2; ++i)
+                for (int i = 0; i < kSlots; ++i)
                     if (drained && nl[i] > 0) drained = mbar_wait_until(&fullb[i], (uint32_t)(nl[i] - 1) & 1u, deadline);
                 uint64_t* sp = is_qk ? spare : spare2;
                 mma_commit(sp);
@@ -360,22 +432,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 if (!drained) atomicOr(P.status, DSPARK_DEV_WAIT_TIMEOUT);
             }
         }
-    } else if (warp >= kSoftThreads / 32) {
-        // ------------------------------------------------------------ converters
-        const int ct = tid - kSoftThreads;
+    } else if (warp == kFixWarp) {
+        // ------------------------------------------------------------ V tails
         for (int t = 0; t < nt && ok; ++t) {
             int row, nvalid; bool blk;
             tile_rows(t, &row, &nvalid, &blk);
-            const int sl = t & 1;
-            const uint32_t ph = (uint32_t)(t >> 1) & 1u;
-            if (!mbar_wait(&kfull[sl], ph, abort_flag, P.status)) { ok = false; break; }
-            convert_tile(sK + sl * tile_sz, nsub, nvalid, ct);
-            fence_async_shared();
-            mbar_arrive(&kready[sl]);
-            if (!mbar_wait(&vfull[sl], ph, abort_flag, P.status)) { ok = false; break; }
-            convert_tile(sV + sl * tile_sz, nsub, nvalid, ct);
-            fence_async_shared();
-            mbar_arrive(&vready[sl]);
+            const int ks = t % kSlots;
+            if (!warp_wait(&vfull[ks], (uint32_t)(t / kSlots) & 1u, abort_flag, P.status)) { ok = false; break; }
+            if (nvalid < KT) {
+                zero_tail(sV + ks * tile_sz, nsub, nvalid, lane);
+                fence_async_shared();               // the P V product reads the tile through the async proxy
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&vready[ks]);
         }
     } else {
         // ------------------------------------------------------------ softmax (two threads per query row)
@@ -459,7 +528,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             fence_async_shared();
             mbar_arrive(&pready[sl]);                          // P written
         }
-        // ---- this split's state: unnormalised O and (max, sum) per query row
+        // ---- this range's state: unnormalised O and (max, sum) per query row
         const bool any = nt > 0;
         if (any && ok && !warp_wait(&odone[(nt - 1) & 1], (uint32_t)((nt - 1) >> 1) & 1u, abort_flag, P.status)) ok = false;
         tc_fence_after();
@@ -475,14 +544,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             }
         }
         if (r < nq && half == 0) {
-            const int i = r / P.grp, h = g * P.grp + r % P.grp;
-            const int64_t prow = ((int64_t)(b * P.nH + h) * P.S1 + split) * P.G + i;
+            const int64_t prow = (int64_t)slot * QROWS + r;
             P.part_ml[prow * 2] = any ? m_run : -INFINITY;
             P.part_ml[prow * 2 + 1] = any ? l_tot : 0.f;
         }
         if (any && ok) {
-            const int i = r / P.grp, h = g * P.grp + r % P.grp;
-            float* dst = P.part_o + (((int64_t)(b * P.nH + h) * P.S1 + split) * P.G + i) * hd + oc0;
+            float* dst = P.part_o + ((int64_t)slot * QROWS + r) * hd + oc0;
             // 32 columns per TMEM wait: half the waits, stores of 128 contiguous bytes
             for (int c = 0; c < hd / 2; c += 32) {
                 uint32_t u[2][16];
@@ -531,12 +598,94 @@ bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd
 
 size_t attn_tc_smem(int hd) {
     const int nsub = hd / 64;
-    // Q, K (2 slots), V (2 slots), P (2 slots), row maxima, then 20 barriers + TMEM slot + abort
-    // flag; 1 KB alignment slack
-    return (size_t)nsub * QROWS * 128 + 4 * (size_t)nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 192 + 1024;
+    // K and V (kSlots each), P (2 slots), row maxima, then the barriers (5 kSlots + 12),
+    // the TMEM slot and the abort flag; 1 KB alignment slack
+    return 2 * (size_t)kSlots * nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 8 * (5 * kSlots + 12) + 16 + 1024;
 }
 
 }  // namespace
+
+// One warp per output row (b, h, i): the item's slots item_cta0[item] ..
+// item_cta0[item + 1] - 1, row r = i * grp + h % grp of each; the weights
+// w_s = exp(m_s - M) combine the unnormalised outputs (lane l owns the 4-column
+// groups l, l + 32 of the row). Slots of empty ranges (m = -inf) weigh nothing.
+constexpr int kMergeWarps = 8;
+constexpr int kMergeBatch = 16;      // slots a merge lane loads at once
+__global__ void __launch_bounds__(kMergeWarps * 32) attn_tc_merge_kernel(AttnArgs a, const int* __restrict__ item_cta0,
+                                                                         int G, int nH, int nKv, int hd, int rows) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);   // ((b * nH) + h) * G + i
+    if (row >= rows) return;
+    const int i = row % G, bh = row / G;
+    const int b = bh / nH, h = bh % nH;
+    const int grp = nH / nKv;
+    const int item = b * nKv + h / grp, r = i * grp + h % grp;
+    const int s0 = item_cta0[item], s1 = item_cta0[item + 1];
+    float M = -INFINITY;
+    for (int s = s0 + lane; s < s1; s += 32) M = fmaxf(M, a.part_ml[((int64_t)s * QROWS + r) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const int ng = hd / 4;
+    float4 num[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    float den = 0.f;
+    for (int sb = s0; sb < s1; sb += 32) {
+        float ws = 0.f, ls = 0.f;
+        if (sb + lane < s1) {
+            const int64_t base = (int64_t)(sb + lane) * QROWS + r;
+            const float m = a.part_ml[base * 2];
+            ls = a.part_ml[base * 2 + 1];
+            ws = m == -INFINITY ? 0.f : __expf(m - M);
+        }
+        const int cnt = min(32, s1 - sb);
+        // kMergeBatch slots' loads in flight at once, then their weighted sum in slot order
+        for (int t0 = 0; t0 < cnt; t0 += kMergeBatch) {
+            float4 v[kMergeBatch][2];
+#pragma unroll
+            for (int u = 0; u < kMergeBatch; ++u) {
+                const float* o = a.part_o + ((int64_t)(sb + t0 + u) * QROWS + r) * hd;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int g4 = lane + q * 32;
+                    v[u][q] = (t0 + u < cnt && g4 < ng) ? reinterpret_cast<const float4*>(o)[g4]
+                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kMergeBatch; ++u) {
+                const float w = __shfl_sync(0xffffffffu, ws, (t0 + u) & 31);
+                const float l = __shfl_sync(0xffffffffu, ls, (t0 + u) & 31);
+                if (t0 + u >= cnt) break;
+                den += w * l;
+                if (w == 0.f) continue;                // uniform: an empty range (its O slot is not written)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    num[q].x += w * v[u][q].x; num[q].y += w * v[u][q].y;
+                    num[q].z += w * v[u][q].z; num[q].w += w * v[u][q].w;
+                }
+            }
+        }
+    }
+    const float inv = 1.f / den;
+    const int64_t ob = (((int64_t)b * G + i) * nH + h) * hd;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int g4 = lane + q * 32;
+        if (g4 >= ng) continue;
+        const float v[4] = {num[q].x * inv, num[q].y * inv, num[q].z * inv, num[q].w * inv};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int64_t o = ob + g4 * 4 + c;
+            store_any(a.out, o, a.out_dtype, v[c]);
+            if (a.out_hi) {
+                const __half hv = __float2half_rn(v[c]);
+                a.out_hi[o] = hv;
+                if (a.out_lo) a.out_lo[o] = __float2half_rn(v[c] - __half2float(hv));
+            }
+        }
+    }
+}
 
 bool attention_tc_supported(const dspark_model* m) {
     const Dims& d = m->d;
@@ -545,27 +694,46 @@ bool attention_tc_supported(const dspark_model* m) {
 
 int attention_tc_key_tile() { return KT; }
 
-cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a_in, cudaStream_t s) {
-    AttnArgs a = a_in;
-    a.S1 = std::max(1, a.n_splits);             // the last context split also takes the block keys
+int attention_tc_grid(const dspark_model* m, int A) { return std::max(m->num_sms, A * m->d.nKv); }
+
+size_t attention_tc_plan_ints(const dspark_model* m, int A, int grid) {
+    return 3 * (size_t)grid + (size_t)A * m->d.nKv + 1;
+}
+
+size_t attention_tc_partial_floats(const dspark_model* m, int grid) { return (size_t)grid * QROWS * (m->d.hd + 2); }
+
+cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
     const Dims& d = m->d;
+    if (!a.plan || a.tc_grid < std::max(1, a.A * d.nKv)) return cudaErrorInvalidValue;
     CUtensorMap tk, tv, tkb, tvb;
     const int64_t cache_rows = (int64_t)a.batch * a.capacity;   // all rows of this layer's cache
     if (!make_kv_map(&tk, a.kc, cache_rows, d.nKv, d.hd) || !make_kv_map(&tv, a.vc, cache_rows, d.nKv, d.hd) ||
         !make_kv_map(&tkb, a.kb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
         !make_kv_map(&tvb, a.vb, (int64_t)a.A * d.gamma, d.nKv, d.hd))
         return cudaErrorInvalidValue;
+    const int grid = a.tc_grid;
+    int* cta_item = a.plan;
+    int* cta_t0 = cta_item + grid;
+    int* cta_t1 = cta_t0 + grid;
+    int* item_cta0 = cta_t1 + grid;
+    cudaError_t e = cudaSuccess;
+    if (!a.plan_ready)      // the plan depends only on the lengths: a round computes it for its first layer
+        e = launch_pdl(attn_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, a.len, a.A, d.nKv, a.capacity, grid,
+                       cta_item, cta_t0, cta_t1, item_cta0);
+    if (e != cudaSuccess) return e;
     AttnTcParams P{};
     P.A = a.A; P.G = d.gamma; P.nH = d.nH; P.nKv = d.nKv; P.grp = d.grp; P.hd = d.hd; P.capacity = a.capacity;
-    P.S1 = a.S1; P.chunk = a.chunk; P.q_dtype = a.q_dtype; P.q = a.q; P.len = a.len;
+    P.q_dtype = a.q_dtype; P.q = a.q; P.len = a.len;
     P.part_o = a.part_o; P.part_ml = a.part_ml; P.status = a.status;
+    P.cta_item = cta_item; P.cta_t0 = cta_t0; P.cta_t1 = cta_t1;
     const size_t smem = attn_tc_smem(d.hd);
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.A * d.nKv, a.S1);
-    e = launch_pdl(attn_tc_kernel, grid, dim3(kThreads), smem, s, tk, tv, tkb, tvb, P);
+    e = launch_pdl(attn_tc_kernel, dim3(grid), dim3(kThreads), smem, s, tk, tv, tkb, tvb, P);
     if (e != cudaSuccess) return e;
-    return launch_attention_merge(m, a, s);
+    const int rows = a.A * d.nH * d.gamma;
+    return launch_pdl(attn_tc_merge_kernel, dim3((rows + kMergeWarps - 1) / kMergeWarps), dim3(kMergeWarps * 32), 0, s,
+                      a, item_cta0, d.gamma, d.nH, d.nKv, d.hd, rows);
 }
 
 }  // namespace tc

@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace dspark {
@@ -39,12 +40,16 @@ template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
-// Loads element i of a T array whose dtype is chosen at run time.
+// Loads element i of an array whose dtype (DSPARK_DTYPE_F32 0, BF16 1, F16 2)
+// is chosen at run time.
 __device__ __forceinline__ float load_any(const void* p, int64_t i, int dtype) {
-    return dtype == 0 ? static_cast<const float*>(p)[i] : __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+    if (dtype == 0) return static_cast<const float*>(p)[i];
+    if (dtype == 2) return __half2float(static_cast<const __half*>(p)[i]);
+    return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
 }
 __device__ __forceinline__ void store_any(void* p, int64_t i, int dtype, float v) {
     if (dtype == 0) static_cast<float*>(p)[i] = v;
+    else if (dtype == 2) static_cast<__half*>(p)[i] = __float2half_rn(v);
     else static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
 }
 

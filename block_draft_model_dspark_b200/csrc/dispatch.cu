@@ -1,6 +1,6 @@
 // Chooses the kernel for each contraction: tcgen05 tensor cores for bf16
-// weights; CUDA cores for the fp32 model (whose 1e-4 bar excludes TF32) and
-// for 4-bit weights (dequantized on load).
+// models (dense bf16 weights, or 4-bit weights dequantized to 16 bits in shared
+// memory); CUDA cores for the fp32 model, whose 1e-4 bar excludes TF32.
 #include <algorithm>
 
 #include "gemm.h"
@@ -12,7 +12,7 @@ namespace tc {
 bool attention_tc_supported(const dspark_model* m);
 int attention_tc_key_tile();
 cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaStream_t s);
-}
+}  // namespace tc
 
 namespace {
 
@@ -40,7 +40,16 @@ double weight_bytes(const dspark_model* m, int64_t N, int64_t K) {
 
 }  // namespace
 
-bool use_tensor_cores(const dspark_model* m) { return m->d.dtype == DSPARK_DTYPE_BF16 && !m->d.quant; }
+bool use_tensor_cores(const dspark_model* m) { return m->d.dtype == DSPARK_DTYPE_BF16; }
+
+bool act_pair(const dspark_model* m, int M) { return use_tensor_cores(m) && !m->d.quant && M <= kPairMaxRows; }
+
+GemmFormat round_gemm_format(const dspark_model* m, int M) {
+    if (m->d.quant) return {1, tc::kWQ4AsF16};
+    return {act_pair(m, M) ? 2 : 1, tc::kWF16};
+}
+
+GemmFormat project_gemm_format(const dspark_model* m) { return {1, m->d.quant ? tc::kWQ4AsF16 : tc::kWBf16}; }
 
 int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len) {
     // context chunks so that A * nKv (tensor cores) or A * nH (CUDA cores) CTAs per split cover the GPU ~2x
@@ -68,9 +77,9 @@ size_t gemm_out_elems(const dspark_model* m, int M, int N, int K) {
     return (size_t)simt_splits(m, M, N, K) * M * N;
 }
 
-size_t gemm_scratch_bytes(const dspark_model* m, int M, int N, int K, bool act_pair) {
+size_t gemm_scratch_bytes(const dspark_model* m, int M, int N, int K, const GemmFormat& f) {
     if (M <= 0 || !use_tensor_cores(m)) return 0;
-    const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, act_pair ? 2 : 1, false);
+    const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, f.np, false, false, f.wfmt);
     return tc::gemm_partial_elems(p) * 4;
 }
 
@@ -101,9 +110,11 @@ cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, in
                      const GemmScratch& sc, PartView* view, int timer_kind, cudaStream_t s) {
     KernelTimer t(timer_kind, s, weight_bytes(m, N, K) + 4.0 * M * K + 4.0 * M * N, 2.0 * M * N * K);
     if (use_tensor_cores(m)) {
-        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, 2, false);
+        const GemmFormat f = round_gemm_format(m, M);
+        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, f.np, false, false, f.wfmt);
         tc_view(p, out, sc, view);
-        return tc::launch_gemm_tc(p, W.w, W.n, X.hi, X.lo, out, N, 0.f, sc.part, m->ws.status, s);
+        const void* w = m->d.quant ? W.packed : W.w16;
+        return tc::launch_gemm_tc(p, w, W.n, X.hi, X.lo, out, N, 0.f, sc.part, m->ws.status, s);
     }
     const int S = simt_splits(m, M, N, K);
     *view = PartView{};
@@ -112,20 +123,34 @@ cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, in
                             (int64_t)M * N, false, 0.f, s);
 }
 
-cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U, cudaStream_t s) {
+cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U, const TileStats& ts, cudaStream_t s) {
     const Dims& d = m->d;
-    KernelTimer t(DSPARK_TIMER_LM_HEAD, s, weight_bytes(m, d.V, d.H) + 4.0 * M * d.H + 4.0 * M * d.V,
-                  2.0 * M * (double)d.V * d.H);
+    const float* w2norm = d.r > 0 ? m->ws.w2norm : nullptr;
     if (use_tensor_cores(m)) {
-        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, d.V, d.H, 2, true);
-        return tc::launch_gemm_tc(p, m->lm_head.w, d.V, x.hi, x.lo, U, d.V, d.cap, nullptr, m->ws.status, s);
+        // the logit statistics come out of the epilogue
+        KernelTimer t(DSPARK_TIMER_LM_HEAD, s, weight_bytes(m, d.V, d.H) + 4.0 * M * d.H + 4.0 * M * d.V,
+                      2.0 * M * (double)d.V * d.H);
+        const GemmFormat f = round_gemm_format(m, M);
+        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, d.V, d.H, f.np, true, true, f.wfmt);
+        const void* w = d.quant ? m->lm_head.packed : m->lm_head.w16;
+        return tc::launch_gemm_tc(p, w, d.V, x.hi, x.lo, U, d.V, d.cap, nullptr, m->ws.status, s, &ts, w2norm,
+                                  m->ws.w1max_bits);
     }
-    return launch_simt_gemm(x.f32, d.H, DSPARK_DTYPE_F32, d.dtype, m->lm_head, d.group, M, d.V, d.H, 1, U, d.V, 0,
-                            true, d.cap, s);
+    cudaError_t e;
+    {
+        KernelTimer t(DSPARK_TIMER_LM_HEAD, s, weight_bytes(m, d.V, d.H) + 4.0 * M * d.H + 4.0 * M * d.V,
+                      2.0 * M * (double)d.V * d.H);
+        e = launch_simt_gemm(x.f32, d.H, DSPARK_DTYPE_F32, d.dtype, m->lm_head, d.group, M, d.V, d.H, 1, U, d.V, 0,
+                             true, d.cap, s);
+    }
+    if (e != cudaSuccess) return e;
+    // a scan of U gives the same statistics
+    KernelTimer t(DSPARK_TIMER_ROWS, s, 4.0 * M * d.V, 0.0);
+    return launch_tile_stats(m, U, M, ts, s);
 }
 
 cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, const RowsPlan& rp, const KvDest& dst,
-                              float* raw, const GemmScratch& sc, cudaStream_t s) {
+                              float* raw, const GemmScratch& sc, void* x16, cudaStream_t s) {
     const Dims& d = m->d;
     const int N = d.Lyr * d.nKv * d.hd;
     const double es = d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0;
@@ -135,9 +160,18 @@ cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, c
     view.p = raw;
     cudaError_t e;
     if (use_tensor_cores(m)) {
-        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, nrows, N, d.H, 1, false);
+        const GemmFormat f = project_gemm_format(m);
+        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, nrows, N, d.H, f.np, false, false, f.wfmt);
         tc_view(p, raw, sc, &view);
-        e = tc::launch_gemm_tc(p, m->wk_all.w, N, X, nullptr, raw, N, 0.f, sc.part, m->ws.status, s);
+        if (d.quant) {
+            // 4-bit k_proj is dequantized to fp16 (bf16 would round every weight to 8 bits and
+            // move the cached K/V by about one bf16 unit): the caller's bf16 rows become fp16
+            e = tc::f16_copy(X, (int64_t)nrows * d.H, x16, m->ws.status, s, DSPARK_DEV_RANGE);
+            if (e != cudaSuccess) return e;
+            X = x16;
+        }
+        e = tc::launch_gemm_tc(p, d.quant ? m->wk_all.packed : m->wk_all.w, N, X, nullptr, raw, N, 0.f, sc.part,
+                               m->ws.status, s);
     } else {
         const int S = simt_splits(m, nrows, N, d.H);
         view.S = S; view.stride = (int64_t)nrows * N; view.ld = N;
@@ -154,7 +188,5 @@ cudaError_t run_attention(const dspark_model* m, const AttnArgs& a, cudaStream_t
     return launch_attention_simt(m, a, s);
 }
 
-int gemm_prepare_model(dspark_model* m) { (void)m; return DSPARK_OK; }
-void gemm_release_model(dspark_model* m) { (void)m; }
 
 }  // namespace dspark

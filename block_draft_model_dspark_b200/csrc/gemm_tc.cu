@@ -22,8 +22,10 @@
 // rate, not HBM, bounded the weight stream at one request per 4 KB of X or
 // 16 KB of W.
 //
-// Roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
-// MMAs, warps 2-5 drain accumulators (TMEM lane quadrant = warp % 4).
+// Roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// MMAs, warps 2-9 drain accumulators (TMEM lane quadrant = warp % 4; warps w
+// and w + 4 take alternate 16-column chunks); with 4-bit weights warps 2-5
+// drain and warps 6-9 dequantize the weight tiles.
 // Accumulators are double-buffered in TMEM so the epilogue of one tile
 // overlaps the MMAs of the next.
 //
@@ -36,6 +38,8 @@
 // optionally with the final-logit softcap.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <string.h>
 
 #include <algorithm>
 #include <mutex>
@@ -46,6 +50,7 @@
 #include "gemm_tc.h"
 #include "tmap.h"
 #include "tc_ptx.cuh"
+#include "logit_stats.cuh"
 
 namespace dspark {
 namespace tc {
@@ -53,21 +58,43 @@ namespace {
 
 constexpr int BM = 128;            // weight rows per tile (MMA M)
 constexpr int BK = 64;             // K elements per K block: one 128-byte swizzle row
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;      // TMA, MMA and four epilogue warps
+constexpr int kConvThreads = 128;  // the weight-transform warps (one weight row each)
+// Epilogue warps: eight (two per TMEM lane quadrant, taking alternate 16-column
+// chunks) for the 16-bit weight formats, whose drain of softcapped logits and
+// their statistics otherwise outlasted a tile's MMAs; four beside the 4-bit
+// dequantizing warps.
+__host__ __device__ constexpr int epi_warps_for(int wfmt) { return wfmt == kWQ4AsF16 ? 4 : 8; }
 constexpr int kABytes = BM * BK * 2;   // one K block of weights (16 KB)
+// threads of a launch: the weight-transform formats add the converter warps (warps 6-9)
+__host__ __device__ constexpr int threads_for(int wfmt) {
+    return 64 + 32 * epi_warps_for(wfmt) + (wfmt == kWQ4AsF16 ? kConvThreads : 0);
+}
 constexpr int kMaxStages = 12;
 constexpr int kSmemLimit = 227 * 1024;   // dynamic shared memory a CTA may opt into
 // alignment slack + full/empty barriers per stage + 4 accumulator barriers,
 // the TMEM slot and the abort flag (plus one spare word)
-constexpr int kSmemExtra(int stages) { return 1024 + 16 * stages + 32 + 16 + 64; }
+constexpr int kSmemExtra(int stages) { return 1024 + 24 * stages + 32 + 16 + 64; }
+// shared memory of the epilogue's logit statistics: [4 warps][BN] WarpStat
+constexpr int kStatBytes(int BN) { return 4 * BN * (int)sizeof(WarpStat); }
 
 struct KParams {
     GemmPlan p;
     float* out;        // result rows out[m * ldo + n]
     int64_t ldo;
     float cap;         // softcap of the result (0 = none)
+    float cap_inv;     // 1 / cap
     float* part;       // stream-K partial tiles [tile][P][BN][128]
     int32_t* status;
+    TileStats stats;               // tile mode: per (128-row weight tile, activation row) logit statistics
+    const float* w2norm;           // with stats: |markov_w2[n]| bounds (NULL: no lo / hi)
+    const uint32_t* w1max_bits;    // max_p |markov_w1[p]| as float bits
+    const void* wq4;               // kWQ4*: the packed 4-bit blocks [tile][K block]
+};
+
+struct Q4Pieces {
+    Q4Piece p[kMaxQ4Pieces];
+    int n;
 };
 
 // Iterates the (tile, k-range) segments of one CTA, identically in every role.
@@ -98,17 +125,53 @@ struct SegIter {
     }
 };
 
-// KSUB K blocks per stage; stage layout [KSUB x W block][KSUB x (NP x BN rows of X)].
-template <int NP, int KSUB>
-__global__ void __launch_bounds__(kThreads, 1)
+// Eight 4-bit codes of one 32-bit word (code j in bits 4j..4j+3) dequantized to
+// scale * code + bias with one rounding, as 8 fp16 in element order. Each code
+// becomes the exact fp16 value 1024 + code by OR-ing it under a fixed exponent;
+// subtracting 1024 is exact, and the fused multiply-add rounds once.
+__device__ __forceinline__ uint4 q4x8_dequant(uint32_t w, uint32_t s2, uint32_t b2) {
+    const uint32_t magic = 0x64006400u;     // 1024.0 in both halves
+    uint32_t v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t t = ((w >> (4 * k)) & 0x000F000Fu) | magic;   // codes k (low half) and k + 4 (high half)
+        const __half2 c = __hsub2(*reinterpret_cast<const __half2*>(&t), *reinterpret_cast<const __half2*>(&magic));
+        const __half2 r = __hfma2(c, *reinterpret_cast<const __half2*>(&s2), *reinterpret_cast<const __half2*>(&b2));
+        v[k] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+    // v[k] holds elements (k, k + 4): regroup to (0,1) (2,3) (4,5) (6,7)
+    return make_uint4(__byte_perm(v[0], v[1], 0x5410), __byte_perm(v[2], v[3], 0x5410),
+                      __byte_perm(v[0], v[1], 0x7632), __byte_perm(v[2], v[3], 0x7632));
+}
+
+// tanh by the hardware's approximation (relative error about 2^-11): the
+// final-logit softcap cap * tanh(x / cap) then stays within 5e-4 |U| of the exact
+// value, far inside the logits' 2e-2 relative bar, at one instruction per logit.
+__device__ __forceinline__ float tanh_fast(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// KSUB K blocks per stage; stage layout [KSUB x W block][KSUB x (NP x BN rows of X)]
+// [the packed 4-bit blocks, for WFMT kWQ4*]. WFMT: the weight format and the MMA's
+// operand type (gemm_tc.h).
+template <int NP, int KSUB, int WFMT>
+__global__ void __launch_bounds__(threads_for(WFMT), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, KParams kp) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
+    constexpr bool kQ4 = WFMT == kWQ4AsF16;
+    constexpr bool kConv = kQ4;                     // the 4-bit formats have the dequantizing warps
+    constexpr int kEpi = epi_warps_for(WFMT);       // epilogue warps 2 .. 2 + kEpi - 1
     const GemmPlan& p = kp.p;
     const int BN = p.BN;
     const int stages = p.stages;
     const int b_bytes = BN * BK * 2;                // one K block of one activation part
     const int x_bytes = NP * b_bytes;               // one K block of the activation (hi and lo)
-    const int stage_bytes = KSUB * (kABytes + x_bytes);
+    const int raw_off = KSUB * (kABytes + x_bytes); // packed 4-bit blocks of the stage
+    const int stage_bytes = raw_off + (kQ4 ? q4_raw_bytes(KSUB) : 0);
+    // bytes the TMA / bulk copies of one stage bring
+    const uint32_t tx_bytes = (uint32_t)(KSUB * ((kQ4 ? kQ4BlockBytes : kABytes) + x_bytes));
 
     // carve: [stages x (W blocks, X blocks)] then barriers
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,18 +179,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     uint64_t* empty = full + stages;
     uint64_t* acc_full = empty + stages;      // [2]
     uint64_t* acc_empty = acc_full + 2;       // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    uint64_t* conv = acc_empty + 2;           // [stages] the stage's weights are in MMA operand form
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(conv + stages);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // set when a wait gives up
+    WarpStat* stat_sm = reinterpret_cast<WarpStat*>(tmem_slot + 16);              // [4 warps][BN] (with stats)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t tmem_cols = p.tmem_cols;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 128); }
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1); mbar_init(&empty[s], 1);
+            if (kConv) mbar_init(&conv[s], kConvThreads);
+        }
+        for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 32 * kEpi); }
         *abort_flag = 0;
         mbar_fence_init();
-        prefetch_tmap(&tmW); prefetch_tmap(&tmX);
+        if (!kQ4) prefetch_tmap(&tmW);       // packed 4-bit weights come by bulk copy (no weight map)
+        prefetch_tmap(&tmX);
     }
     if (warp == 1) tmem_alloc(tmem_slot, tmem_cols);
     tc_fence_before();
@@ -144,8 +213,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         if (lane == 0) {
             // one request per stage for the weights, one for the activation
             auto load_w = [&](uint8_t* dst, uint64_t* bar, int kk, int nt) {
-                if (KSUB == 1) tma_load_2d(dst, &tmW, bar, kk * BK, nt * BM);
-                else tma_load_3d(dst, &tmW, bar, 0, nt * BM, kk * KSUB);
+                if (kQ4) {
+                    // the tile's packed blocks [nt][K block] are contiguous: one bulk copy per stage
+                    const uint8_t* src = static_cast<const uint8_t*>(kp.wq4) +
+                                         ((int64_t)nt * (p.kb * KSUB) + (int64_t)kk * KSUB) * kQ4BlockBytes;
+                    bulk_load(dst + raw_off, src, (uint32_t)(KSUB * kQ4BlockBytes), bar);
+                } else if (KSUB == 1) {
+                    tma_load_2d(dst, &tmW, bar, kk * BK, nt * BM);
+                } else {
+                    tma_load_3d(dst, &tmW, bar, 0, nt * BM, kk * KSUB);
+                }
             };
             auto load_x = [&](uint8_t* dst, uint64_t* bar, int kk, int mt) {
                 if (NP == 1 && KSUB == 1) tma_load_2d(dst, &tmX, bar, kk * BK, mt * BN);
@@ -163,7 +240,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 while (n_pre < stages && it.next(tile, k0, k1, slot)) {
                     const int nt = tile / p.n_mt;
                     for (int kk = k0; kk < k1 && n_pre < stages; ++kk, ++n_pre) {
-                        mbar_arrive_expect_tx(&full[n_pre], stage_bytes);
+                        mbar_arrive_expect_tx(&full[n_pre], tx_bytes);
                         load_w(base + n_pre * stage_bytes, &full[n_pre], kk, nt);
                     }
                 }
@@ -180,7 +257,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     if (n >= n_pre) {
                         const uint32_t ph = (uint32_t)(n / stages) & 1u;
                         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, kp.status)) { ok = false; break; }
-                        mbar_arrive_expect_tx(&full[s], stage_bytes);
+                        mbar_arrive_expect_tx(&full[s], tx_bytes);
                         load_w(st, &full[s], kk, nt);
                     }
                     load_x(st + KSUB * kABytes, &full[s], kk, mt);
@@ -208,7 +285,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             // after the X_hi rows in the stage, so [X_hi; X_lo] is one B operand of
             // 2 BN rows and the two products land in adjacent accumulator columns
             const bool fused = NP == 2 && p.acc_cols == 2 * BN;
-            const uint32_t idesc = idesc_bf16(BM, fused ? 2 * BN : BN);
+            constexpr bool kF16 = WFMT == kWF16 || WFMT == kWQ4AsF16;
+            const uint32_t idesc = kF16 ? idesc_f16(BM, fused ? 2 * BN : BN, 0) : idesc_bf16(BM, fused ? 2 * BN : BN);
+            uint64_t* ready = kConv ? conv : full;          // the converters' barrier when they transform W
             SegIter it(p, blockIdx.x);
             int tile, k0, k1, slot, n = 0, seg = 0;
             bool ok = true;
@@ -221,7 +300,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 for (int kk = k0; kk < k1; ++kk, ++n) {
                     const int s = n % stages;
                     const uint32_t ph = (uint32_t)(n / stages) & 1u;
-                    if (!mbar_wait(&full[s], ph, abort_flag, kp.status)) { ok = false; break; }
+                    if (!mbar_wait(&ready[s], ph, abort_flag, kp.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t st_addr = smem_u32(base + s * stage_bytes);
 #pragma unroll
@@ -245,6 +324,48 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 ++seg;
             }
         }
+    } else if (kConv && warp >= 2 + kEpi) {
+        // ---------------------------------------------------------- weight dequantization (warps 6-9)
+        // Thread i owns weight row i of the tile: per K block it turns the packed
+        // 4-bit codes into the MMA operand (128 bytes, 128-byte swizzle: 16-byte chunk c
+        // of row i at chunk c ^ (i & 7)), then the stage's barrier counts it.
+        pdl_wait();
+        const int i = threadIdx.x - (64 + 32 * kEpi);
+        SegIter it(p, blockIdx.x);
+        int tile, k0, k1, slot, n = 0;
+        bool ok = true;
+        while (ok && it.next(tile, k0, k1, slot)) {
+            for (int kk = k0; kk < k1; ++kk, ++n) {
+                const int s = n % stages;
+                if (!mbar_wait(&full[s], (uint32_t)(n / stages) & 1u, abort_flag, kp.status)) { ok = false; break; }
+                uint8_t* st = base + s * stage_bytes;
+#pragma unroll
+                for (int sub = 0; sub < KSUB; ++sub) {
+                    uint8_t* wrow = st + sub * kABytes + i * 128;
+                    {
+                        // packed block: words [128 rows][8], scales [128], biases [128] (bf16)
+                        const uint8_t* blk = st + raw_off + sub * kQ4BlockBytes;
+                        const uint4 w0 = reinterpret_cast<const uint4*>(blk + i * 32)[0];
+                        const uint4 w1 = reinterpret_cast<const uint4*>(blk + i * 32)[1];
+                        const uint16_t sb = reinterpret_cast<const uint16_t*>(blk + BM * 32)[i];
+                        const uint16_t bb = reinterpret_cast<const uint16_t*>(blk + BM * 32 + BM * 2)[i];
+                        // bf16 scale and bias as fp16 (exact inside fp16's normal range)
+                        const __half hs = __float2half_rn(__uint_as_float((uint32_t)sb << 16));
+                        const __half hb = __float2half_rn(__uint_as_float((uint32_t)bb << 16));
+                        const uint16_t us = *reinterpret_cast<const uint16_t*>(&hs);
+                        const uint16_t ub = *reinterpret_cast<const uint16_t*>(&hb);
+                        const uint32_t s2 = (uint32_t)us | ((uint32_t)us << 16);
+                        const uint32_t b2 = (uint32_t)ub | ((uint32_t)ub << 16);
+                        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            reinterpret_cast<uint4*>(wrow)[c ^ (i & 7)] = q4x8_dequant(ws[c], s2, b2);
+                    }
+                }
+                fence_async_shared();            // the MMA reads these through the async proxy
+                mbar_arrive(&conv[s]);
+            }
+        }
     } else {
         // ---------------------------------------------------------- epilogue (warps 2-5)
         // Tile mode: the result goes straight to `out` (with the softcap). Stream-K:
@@ -255,21 +376,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         pdl_wait();
         const int quad = warp & 3;
         const int n_local = quad * 32 + lane;
+        const int grp = (warp - 2) >> 2;                  // column group: chunks grp, grp + kEpi / 4, ...
+        const bool with_stats = kp.stats.mx != nullptr && !p.streamk;
+        const bool bounds = with_stats && kp.w2norm != nullptr;
+        const float Bw1 = bounds ? __uint_as_float(*kp.w1max_bits) : 0.f;
         SegIter it(p, blockIdx.x);
         int tile, k0, k1, slot, seg = 0;
         while (it.next(tile, k0, k1, slot)) {
             const int acc = seg & 1;
             const uint32_t aph = (uint32_t)(seg >> 1) & 1u;
-            mbar_wait(&acc_full[acc], aph, abort_flag, kp.status);
-            asm volatile("bar.sync 1, 128;" ::: "memory");   // the group leaves together if any wait gave up
-            if (*abort_flag) break;
+            const bool got = mbar_wait(&acc_full[acc], aph, abort_flag, kp.status);
+            // the group leaves together if any wait gave up
+            if (named_barrier_or(1, 32 * kEpi, !got || *abort_flag != 0)) break;
             tc_fence_after();
             const int nt = tile / p.n_mt, mt = tile % p.n_mt;
             const int n = nt * BM + n_local;
             const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * p.acc_cols);
             float* part_tile = kp.part + ((int64_t)tile * p.P * BN) * BM + n_local;
             const bool split_acc = p.acc_cols == 2 * BN;       // X_hi and X_lo products in separate columns
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = 16 * grp; c0 < BN; c0 += 16 * (kEpi / 4)) {
                 uint32_t r[16];
                 tmem_ld_x16(tbase + (uint32_t)c0, r);
                 if (split_acc) {
@@ -282,14 +407,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     tmem_ld_wait();
                 }
                 if (!p.streamk) {
+                    float u[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int m = mt * BN + c0 + j;
-                        if (m < p.M && n < p.N) {
-                            float v = __uint_as_float(r[j]);
-                            if (kp.cap > 0.f) v = kp.cap * tanhf(v / kp.cap);
-                            kp.out[(int64_t)m * kp.ldo + n] = v;
-                        }
+                        float v = __uint_as_float(r[j]);
+                        if (kp.cap > 0.f) v = kp.cap * tanh_fast(v * kp.cap_inv);
+                        u[j] = n < p.N ? v : -INFINITY;
+                        if (m < p.M && n < p.N) kp.out[(int64_t)m * kp.ldo + n] = v;
+                    }
+                    if (with_stats) {
+                        // the 16 positions (columns) over this warp's 32 entries at once
+                        const float bw = bounds && n < p.N ? Bw1 * kp.w2norm[n] : 0.f;
+                        const WarpStat w = warp_logit_stat16(u, n, bw, bounds, kp.cap);
+                        if ((lane & 1) == 0) stat_sm[quad * BN + c0 + warp_stat16_col(lane)] = w;
                     }
                 } else {
                     float* dst = part_tile + ((int64_t)slot * BN + c0) * BM;
@@ -299,6 +430,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             }
             tc_fence_before();
             mbar_arrive(&acc_empty[acc]);
+            if (with_stats) {
+                // the four warps' results of every position of the tile, merged in warp order
+                asm volatile("bar.sync 2, %0;" ::"r"(32 * kEpi) : "memory");
+                const int tid_e = threadIdx.x - 64;
+                for (int c = tid_e; c < BN; c += 32 * kEpi) {
+                    const int m = mt * BN + c;
+                    if (m < p.M) {
+                        const WarpStat q4[4] = {stat_sm[c], stat_sm[BN + c], stat_sm[2 * BN + c], stat_sm[3 * BN + c]};
+                        store_tile_stat(kp.stats, nt, m, q4);
+                    }
+                }
+            }
             ++seg;
         }
     }
@@ -392,9 +535,10 @@ int tmem_cols_for(int acc_cols) {
 
 }  // namespace
 
-GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles) {
+GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles, bool stats, int wfmt) {
     GemmPlan p{};
-    p.M = M; p.N = N; p.K = K; p.np = np;
+    p.M = M; p.N = N; p.K = K; p.np = np; p.stats = stats ? 1 : 0; p.wfmt = wfmt;
+    const bool q4 = wfmt == kWQ4AsF16;
     const int m_pad = (M + 15) / 16 * 16;
     p.BN = m_pad <= 256 ? m_pad : 256;
     p.n_mt = (M + p.BN - 1) / p.BN;
@@ -403,8 +547,10 @@ GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles) {
     // as many stages as shared memory holds: the bytes in flight per SM are
     // what sustains the weight stream at HBM latency under load; two K blocks
     // per stage (half the TMA requests) when K allows and >= 3 stages still fit
-    auto stage_bytes_for = [&](int ksub) { return ksub * (kABytes + np * p.BN * BK * 2); };
-    const int avail = kSmemLimit - kSmemExtra(kMaxStages);
+    auto stage_bytes_for = [&](int ksub) {
+        return ksub * (kABytes + np * p.BN * BK * 2) + (q4 ? q4_raw_bytes(ksub) : 0);
+    };
+    const int avail = kSmemLimit - kSmemExtra(kMaxStages) - (stats ? kStatBytes(p.BN) : 0);
     p.ksub = (K % (2 * BK) == 0 && avail / stage_bytes_for(2) >= 3) ? 2 : 1;
     p.kb = K / (BK * p.ksub);
     p.stages = std::max(2, std::min(kMaxStages, avail / stage_bytes_for(p.ksub)));
@@ -436,28 +582,126 @@ size_t gemm_partial_elems(const GemmPlan& p) {
 }
 
 size_t gemm_smem_bytes(const GemmPlan& p) {
-    const int stage_bytes = p.ksub * (kABytes + p.np * p.BN * BK * 2);
-    return (size_t)p.stages * stage_bytes + kSmemExtra(p.stages);
+    const bool q4 = p.wfmt == kWQ4AsF16;
+    const int stage_bytes = p.ksub * (kABytes + p.np * p.BN * BK * 2) + (q4 ? q4_raw_bytes(p.ksub) : 0);
+    return (size_t)p.stages * stage_bytes + kSmemExtra(p.stages) + (p.stats ? kStatBytes(p.BN) : 0);
+}
+
+namespace {
+
+template <int NP, int KSUB>
+void* pick_kernel(int wfmt) {
+    switch (wfmt) {
+        case kWF16: return (void*)gemm_tc_kernel<NP, KSUB, kWF16>;
+        case kWQ4AsF16: return (void*)gemm_tc_kernel<NP, KSUB, kWQ4AsF16>;
+        default: return (void*)gemm_tc_kernel<NP, KSUB, kWBf16>;
+    }
+}
+
+// Packs one 128-row tile x one K block per CTA; thread i copies row i.
+__global__ void __launch_bounds__(128) q4_pack_kernel(Q4Pieces pcs, int64_t n, int64_t k, uint8_t* __restrict__ dst) {
+    pdl_trigger();
+    pdl_wait();
+    const int64_t t = blockIdx.x;
+    const int kb = blockIdx.y, KB = (int)(k / 64), i = threadIdx.x;
+    const int64_t row = t * 128 + i;
+    uint8_t* blk = dst + ((int64_t)t * KB + kb) * kQ4BlockBytes;
+    uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+    uint16_t sv = 0, bv = 0;
+    if (row < n) {
+        for (int q = 0; q < pcs.n; ++q) {
+            const Q4Piece& pc = pcs.p[q];
+            if (row >= pc.row0 && row < pc.row0 + pc.rows) {
+                const int64_t r = row - pc.row0;
+                const uint4* src = reinterpret_cast<const uint4*>(pc.w + r * (k / 8) + (int64_t)kb * 8);
+                w0 = src[0];
+                w1 = src[1];
+                sv = reinterpret_cast<const uint16_t*>(pc.s)[r * KB + kb];
+                bv = reinterpret_cast<const uint16_t*>(pc.b)[r * KB + kb];
+                break;
+            }
+        }
+    }
+    reinterpret_cast<uint4*>(blk + i * 32)[0] = w0;
+    reinterpret_cast<uint4*>(blk + i * 32)[1] = w1;
+    reinterpret_cast<uint16_t*>(blk + 128 * 32)[i] = sv;
+    reinterpret_cast<uint16_t*>(blk + 128 * 32 + 128 * 2)[i] = bv;
+}
+
+}  // namespace
+
+namespace {
+
+// bf16 -> fp16, eight values per thread (n a multiple of 8); flags values outside fp16's range.
+__global__ void f16_copy_kernel(const uint4* __restrict__ src, int64_t n8, uint4* __restrict__ dst,
+                                int32_t* __restrict__ overflow, int32_t bits) {
+    pdl_trigger();
+    pdl_wait();
+    bool bad = false;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 u = src[i];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xffff0000u);
+            bad |= !(fabsf(a) <= 65504.f) || !(fabsf(b) <= 65504.f);
+            const __half2 h = __floats2half2_rn(a, b);
+            o[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (bad) atomicOr(overflow, bits);
+}
+
+}  // namespace
+
+cudaError_t f16_copy(const void* src, int64_t n, void* dst, int32_t* overflow, cudaStream_t s, int32_t bits) {
+    if (n % 8 || (reinterpret_cast<uintptr_t>(src) & 15u) || (reinterpret_cast<uintptr_t>(dst) & 15u))
+        return cudaErrorInvalidValue;
+    const int64_t n8 = n / 8;
+    const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, 148 * 8);
+    return launch_pdl(f16_copy_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, s, static_cast<const uint4*>(src), n8,
+                      static_cast<uint4*>(dst), overflow, bits);
+}
+
+cudaError_t q4_pack(const Q4Piece* pieces, int npieces, int64_t n, int64_t k, void* dst, cudaStream_t s) {
+    if (npieces < 1 || npieces > kMaxQ4Pieces || k % 64 != 0 || n <= 0) return cudaErrorInvalidValue;
+    Q4Pieces pcs{};
+    pcs.n = npieces;
+    for (int q = 0; q < npieces; ++q) pcs.p[q] = pieces[q];
+    const dim3 grid((unsigned)((n + 127) / 128), (unsigned)(k / 64));
+    return launch_pdl(q4_pack_kernel, grid, dim3(128), 0, s, pcs, n, k, static_cast<uint8_t*>(dst));
 }
 
 cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, const void* X0, const void* X1,
-                           float* out, int64_t ldo, float cap, float* part, int32_t* status, cudaStream_t s) {
+                           float* out, int64_t ldo, float cap, float* part, int32_t* status, cudaStream_t s,
+                           const TileStats* stats, const float* w2norm, const uint32_t* w1max_bits) {
+    if (stats && (p.streamk || !p.stats)) return cudaErrorInvalidValue;
     if (p.streamk && !part) return cudaErrorInvalidValue;
+    const bool q4 = p.wfmt == kWQ4AsF16;
+    if (q4 && p.np != 1) return cudaErrorInvalidValue;
     // the bf16 pair must be one [2][M][K] block (lo right after hi)
     if (p.np == 2 && static_cast<const char*>(X1) != static_cast<const char*>(X0) + (size_t)p.M * p.K * 2)
         return cudaErrorInvalidValue;
+    if (q4 && (reinterpret_cast<uintptr_t>(W) & 15u)) return cudaErrorInvalidValue;
     CUtensorMap tw, tx;
-    if (!make_wmap(&tw, W, w_rows, p.K, p.ksub)) return cudaErrorInvalidValue;
+    memset(&tw, 0, sizeof(tw));
+    // packed 4-bit weights come by bulk copy: the weight map is unused
+    if (!q4 && !make_wmap(&tw, W, w_rows, p.K, p.ksub)) return cudaErrorInvalidValue;
     if (!make_xmap(&tx, X0, p.M, p.K, p.BN, p.np, p.ksub)) return cudaErrorInvalidValue;
     KParams kp{};
-    kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.status = status; kp.part = part;
+    kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.cap_inv = cap > 0.f ? 1.f / cap : 0.f;
+    kp.status = status; kp.part = part;
+    kp.wq4 = q4 ? W : nullptr;
+    if (stats) { kp.stats = *stats; kp.w2norm = w2norm; kp.w1max_bits = w1max_bits; }
     const size_t smem = gemm_smem_bytes(p);
-    void (*kern)(CUtensorMap, CUtensorMap, KParams) =
-        p.np == 2 ? (p.ksub == 2 ? gemm_tc_kernel<2, 2> : gemm_tc_kernel<2, 1>)
-                  : (p.ksub == 2 ? gemm_tc_kernel<1, 2> : gemm_tc_kernel<1, 1>);
+    void* kern = p.np == 2 ? (p.ksub == 2 ? pick_kernel<2, 2>(p.wfmt) : pick_kernel<2, 1>(p.wfmt))
+                           : (p.ksub == 2 ? pick_kernel<1, 2>(p.wfmt) : pick_kernel<1, 1>(p.wfmt));
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(p.grid), dim3(kThreads), smem, s, tw, tx, kp);
+    return launch_pdl(reinterpret_cast<void (*)(CUtensorMap, CUtensorMap, KParams)>(kern), dim3(p.grid),
+                      dim3(threads_for(p.wfmt)), smem, s, tw, tx, kp);
 }
 
 }  // namespace tc

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 #include <stddef.h>
 #include <string>
@@ -10,6 +11,7 @@
 
 #include "../../include/dspark.h"
 #include "gemm_tc.h"
+#include "logit_stats.cuh"
 
 namespace dspark {
 
@@ -37,11 +39,13 @@ struct MatRef {
     const bf16* biases = nullptr;
     int64_t n = 0, k = 0;
     bool quant = false;
+    const void* packed = nullptr;   // 4-bit GEMM weights: the packed copy the tensor-core GEMM reads
+    const void* w16 = nullptr;      // dense bf16 GEMM weights: the fp16 copy the tensor-core GEMM reads
 };
 
 // Device layout of everything dspark_model_create places in model_ws.
 struct ModelWs {
-    int32_t* status = nullptr;      // device status word (+ padding)
+    int32_t* status = nullptr;      // device status word (+ padding; status[1]: fp16-copy overflow flag)
     double* inv_freq = nullptr;     // [hd/2] RoPE inverse frequencies (0 = identity lane)
     void* wqk = nullptr;            // per layer [(nH+nKv)*hd, H] (dense) or words
     void* wgu = nullptr;            // per layer [2I, H]
@@ -106,13 +110,56 @@ struct PartView {
         return v;
     }
     __device__ __forceinline__ float sum(int64_t m, int64_t n) const { return finish(load(m, n)); }
+
+    // Four consecutive columns n .. n + 3 of row m (n % 4 == 0; mode 1: within one
+    // 128-column block, so they share a tile), each the sum of its partials in order.
+    static constexpr int kMax4 = 4;            // partials load4 keeps in flight (more are read in finish4)
+    struct Pending4 {
+        float4 x[kMax4];
+        int cnt;
+        const float* rest;
+        int64_t step;
+    };
+    __device__ __forceinline__ Pending4 load4(int m, int64_t n) const {
+        Pending4 q;
+        const float* base;
+        if (mode == 0) {
+            q.cnt = S; q.step = stride;
+            base = p + (int64_t)m * ld + n;
+        } else {
+            const int mt = m / BN, ml = m - mt * BN, nt = (int)(n >> 7), nl = (int)(n & 127);
+            const int tile = nt * n_mt + mt;
+            q.cnt = cta_of(tile * kb + kb - 1) - cta_of(tile * kb) + 1;
+            q.step = (int64_t)BN * 128;
+            base = p + (((int64_t)tile * P) * BN + ml) * 128 + nl;
+        }
+#pragma unroll
+        for (int s = 0; s < kMax4; ++s)
+            q.x[s] = s < q.cnt ? *reinterpret_cast<const float4*>(base + s * q.step) : make_float4(0.f, 0.f, 0.f, 0.f);
+        q.rest = base;
+        return q;
+    }
+    __device__ __forceinline__ float4 finish4(const Pending4& q) const {
+        float4 v = q.x[0];
+#pragma unroll
+        for (int s = 1; s < kMax4; ++s) { v.x += q.x[s].x; v.y += q.x[s].y; v.z += q.x[s].z; v.w += q.x[s].w; }
+        for (int s = kMax4; s < q.cnt; ++s) {
+            const float4 t = *reinterpret_cast<const float4*>(q.rest + s * q.step);
+            v.x += t.x; v.y += t.y; v.z += t.z; v.w += t.w;
+        }
+        return v;
+    }
 };
 
-// An fp32 activation and, for tensor-core GEMMs, its bf16 pair hi + lo.
+// An fp32 activation and the fp16 form its tensor-core GEMM reads: hi =
+// fp16(x), and for the pair form also lo = fp16(x - hi) (dense weights at up
+// to 128 activation rows, where both parts go through one MMA and the pair
+// costs nothing); with more rows (the MMAs bound the GEMM) and with 4-bit
+// weights, hi alone. hi and lo are one [2][M][K] block (lo right after hi).
 struct ActBuf {
     float* f32 = nullptr;
-    bf16* hi = nullptr;
-    bf16* lo = nullptr;
+    __half* hi = nullptr;
+    __half* lo = nullptr;
 };
 
 constexpr int kMaxLayers = 64;
@@ -125,7 +172,8 @@ struct LayerRef {
 
 struct Dims {
     int H, Lyr, nH, nKv, hd, grp, I, V, gamma, mask_id, r;
-    int dtype;          // DSPARK_DTYPE_*
+    int dtype;          // DSPARK_DTYPE_* of the weights and gains
+    int kv_dtype;       // DSPARK_DTYPE_* of the context and block K/V (fp16 for bf16 models)
     bool quant;
     int group;
     float eps, cap, conf_thr;
@@ -148,6 +196,8 @@ struct dspark_model {
     int num_sms = 148;
     float* attn_dump = nullptr;      // test-facing per-layer attention dump (dspark_debug_attention_dump)
     size_t attn_dump_bytes = 0;
+    void* logit_dump = nullptr;      // test-facing per-position logit statistics (dspark_debug_logit_stats)
+    size_t logit_dump_bytes = 0;
 };
 
 namespace dspark {
@@ -210,13 +260,15 @@ cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const PartVie
 // Attention: partial pass over context chunks + block keys, then merge.
 struct AttnArgs {
     const void* q;  const void* kb; const void* vb;  // [A, G, nH, hd] / [A, G, nKv, hd]
-    int q_dtype, out_dtype;                          // DSPARK_DTYPE_* of q and out (kb, vb, cache: model dtype)
+    int q_dtype, out_dtype;                          // DSPARK_DTYPE_* of q and out (kb, vb, cache: the KV dtype)
     const void* kc; const void* vc;                  // cache of this layer: [batch, cap, nKv, hd]
     const int32_t* len; int capacity, batch;         // cache lengths [batch], capacity, batch rows
     void* out;                                       // [A, G, nH, hd]
-    bf16* out_hi; bf16* out_lo;                      // optional bf16 pair of out (fp32 out only)
+    __half* out_hi; __half* out_lo;                  // optional fp16 form of out (fp32 out only; lo may be NULL)
     float* part_o; float* part_ml;                   // workspace
-    int A, n_splits, chunk;                          // context splits of `chunk` keys
+    int* plan; int tc_grid;                          // tensor cores: the work plan's ints and the CTAs
+    bool plan_ready;                                 // the plan was computed for these lengths already
+    int A, n_splits, chunk;                          // CUDA cores: context splits of `chunk` keys
     int S1;                                          // partial slots per (b, h): set by the kernel path
     int32_t* status;
     double kv_bytes, flops;                          // algorithmic work (for the timers)
@@ -231,6 +283,7 @@ struct WalkArgs {
     uint32_t* ticket;          // one counter, zero at entry
     int A, nblk, step;
     int32_t* status;
+    const int* skip;           // non-NULL: the step returns at once when *skip == 0
 };
 cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s);
 // The whole walk in one cooperative launch (one CTA per SM, bounded grid barriers).
@@ -241,27 +294,39 @@ bool walk_tc_supported(const dspark_model* m, int A);
 cudaError_t launch_walk_tc(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
                            unsigned long long* keys, uint32_t* arrivals, const int* skip, int A, cudaStream_t s);
 }  // namespace tc
-// Exact pruning of the walk (walk_prune.cu): candidate lists from norm bounds, then
-// the walk over the candidates; *fail = 1 hands the round to the full walk.
-constexpr int kPruneCap = 256;      // candidates a position may keep (one thread each)
+// Exact pruning of the walk (walk_prune.cu): candidate lists from norm bounds and the
+// lm-head's tile statistics, then the walk over the candidates; *fail = 1 hands the
+// round to the full walk.
+constexpr int kPruneCap = 1024;     // candidates a position may keep
 struct PruneScratch {
-    uint32_t* T = nullptr;          // [M] ordered max of U - B |w2|, zero at entry
-    int* cnt = nullptr;             // [M] candidate counts, zero at entry
-    int* fail = nullptr;            // one word, zero at entry
+    int* cnt = nullptr;             // [M] candidate counts
+    int* fail = nullptr;            // one word (cleared by the candidate kernel)
     int* list = nullptr;            // [M][kPruneCap]
+};
+// Per-position logit telemetry (dspark_debug_logit_stats): 16 bytes.
+struct LogitRowStat {
+    float max;
+    float lse;
+    int32_t argmax;
+    int32_t candidates;
 };
 bool walk_prune_model_supported(const Dims& d);
 cudaError_t launch_markov_norms(const dspark_model* m, cudaStream_t s);
-cudaError_t launch_walk_prune(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens, int A,
-                              const PruneScratch& ps, cudaStream_t s);
+// The tile statistics of U by a scan (lm-heads that do not produce them in their epilogue).
+cudaError_t launch_tile_stats(const dspark_model* m, const float* U, int M, const TileStats& ts, cudaStream_t s);
+// Candidate lists (and with markov_rank 0 the tokens), then the pruned walk.
+cudaError_t launch_walk_prune(const dspark_model* m, const float* U, const TileStats& ts, const int32_t* anchors,
+                              int32_t* tokens, int A, const PruneScratch& ps, LogitRowStat* row_out, cudaStream_t s);
 bool walk_persistent_supported(const dspark_model* m, int A);
 int walk_persistent_blocks(const dspark_model* m);
+// With `skip` non-NULL the kernel returns at once when *skip == 0 (the pruned walk wrote the tokens).
 cudaError_t launch_walk_persistent(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
-                                   float* cand_val, int32_t* cand_idx, uint32_t* arrivals, int A, cudaStream_t s);
+                                   float* cand_val, int32_t* cand_idx, uint32_t* arrivals, const int* skip, int A,
+                                   cudaStream_t s);
 // Vocabulary slices (grid.x) of a walk step.
 int walk_vocab_blocks(int num_sms, int V, int r, int dtype, bool quant);
 cudaError_t launch_walk_init(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V,
-                             int32_t* status, cudaStream_t s);
+                             int32_t* status, const int* skip, cudaStream_t s);
 // Confidence + lengths (hf = the final-normed hidden, fp32 [M, H]).
 cudaError_t launch_confidence(const dspark_model* m, const float* hf32, const int32_t* anchors, const int32_t* tokens,
                               int A, float* conf, int32_t* lengths, cudaStream_t s);

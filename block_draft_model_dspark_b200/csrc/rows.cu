@@ -5,8 +5,8 @@
 // Each epilogue reads its GEMM's result through a PartView, which sums the
 // GEMM's partial tiles in a fixed order (results do not depend on
 // scheduling). Activations that feed the next GEMM are written in fp32 and,
-// when the model has bf16 weights, also as a bf16 pair (hi, lo = v - hi) for
-// the tensor-core GEMM.
+// for the tensor-core GEMMs of a bf16 model, also in fp16 (hi = fp16(v), and
+// for the pair form lo = fp16(v - hi)).
 #include <math.h>
 
 #include <algorithm>
@@ -22,9 +22,29 @@ constexpr int kMaxPer = 16;   // columns per thread in the full-row kernels
 __device__ __forceinline__ void store_act(const ActBuf& a, int64_t i, float v) {
     a.f32[i] = v;
     if (a.hi) {
-        const bf16 h = __float2bfloat16_rn(v);
+        const __half h = __float2half_rn(v);
         a.hi[i] = h;
-        a.lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+        if (a.lo) a.lo[i] = __float2half_rn(v - __half2float(h));
+    }
+}
+
+// Four consecutive activation values at i .. i + 3 (i % 4 == 0).
+__device__ __forceinline__ void store_act4(const ActBuf& a, int64_t i, float4 v) {
+    *reinterpret_cast<float4*>(a.f32 + i) = v;
+    if (a.hi) {
+        const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+        uint2 hv;
+        hv.x = *reinterpret_cast<const uint32_t*>(&h01);
+        hv.y = *reinterpret_cast<const uint32_t*>(&h23);
+        *reinterpret_cast<uint2*>(a.hi + i) = hv;
+        if (a.lo) {
+            const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+            const __half2 l01 = __floats2half2_rn(v.x - f01.x, v.y - f01.y), l23 = __floats2half2_rn(v.z - f23.x, v.w - f23.y);
+            uint2 lv;
+            lv.x = *reinterpret_cast<const uint32_t*>(&l01);
+            lv.y = *reinterpret_cast<const uint32_t*>(&l23);
+            *reinterpret_cast<uint2*>(a.lo + i) = lv;
+        }
     }
 }
 
@@ -39,7 +59,8 @@ __device__ __forceinline__ float mat_at(const MatRef& W, int dtype, int group, i
 // ------------------------------------------------------------------ context K/V
 // grid (rows, Lyr*nKv), block hd/2: thread i owns the RoPE pair (i, i + hd/2).
 __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const double* __restrict__ inv_freq,
-                                   LayerPtrs k_norms, int nKv, int hd, float eps, int dtype, int32_t* status) {
+                                   LayerPtrs k_norms, int nKv, int hd, float eps, int dtype, int kv_dtype,
+                                   int32_t* status) {
     __shared__ float red[32];
     pdl_trigger();
     pdl_wait();
@@ -66,10 +87,10 @@ __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const 
     float sn, cs;
     rope_sincos(pos, inv_freq[i], &sn, &cs);
     const int64_t o = (int64_t)l * dst.layer_stride + (int64_t)b * dst.batch_stride + ((int64_t)dst_row * nKv + g) * hd;
-    store_any(dst.v, o + i, dtype, v1);
-    store_any(dst.v, o + i + half, dtype, v2);
-    store_any(dst.k, o + i, dtype, k1 * cs - k2 * sn);
-    store_any(dst.k, o + i + half, dtype, k2 * cs + k1 * sn);
+    store_any(dst.v, o + i, kv_dtype, v1);
+    store_any(dst.v, o + i + half, kv_dtype, v2);
+    store_any(dst.k, o + i, kv_dtype, k1 * cs - k2 * sn);
+    store_any(dst.k, o + i + half, kv_dtype, k2 * cs + k1 * sn);
 }
 
 // The append's device-side validation (the accepted-row counts come from the
@@ -146,40 +167,64 @@ __global__ void __launch_bounds__(512) embed_kernel(MatRef E, int dtype, int gro
 }
 
 // ------------------------------------------------------------------ q / k / v heads
-// grid (M, nH + nKv), block hd/2.
-__global__ void qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, int hd,
-                                   const int32_t* __restrict__ block_pos, const double* __restrict__ inv_freq,
-                                   const void* __restrict__ q_norm, const void* __restrict__ k_norm, float eps,
-                                   int dtype, float* __restrict__ q, void* __restrict__ kb, void* __restrict__ vb) {
-    __shared__ float red[32];
+// grid (M, ceil((nH + nKv) / 4)), block 128: one warp per head; lane l owns the
+// RoPE pairs (i, i + hd/2) for i = l, l + 32, ... < hd/2.
+constexpr int kQkHeadsPerCta = 4;
+constexpr int kQkMaxPairs = 4;                // hd/2 / 32 for hd <= 256
+__global__ void __launch_bounds__(32 * kQkHeadsPerCta)
+qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, int hd, const int32_t* __restrict__ block_pos,
+                   const double* __restrict__ inv_freq, const void* __restrict__ q_norm,
+                   const void* __restrict__ k_norm, float eps, int dtype, int kv_dtype, float* __restrict__ q,
+                   void* __restrict__ kb, void* __restrict__ vb) {
     pdl_trigger();
     pdl_wait();
-    const int m = blockIdx.x, hh = blockIdx.y;
+    const int m = blockIdx.x, lane = threadIdx.x & 31;
+    const int hh = blockIdx.y * kQkHeadsPerCta + (threadIdx.x >> 5);
+    if (hh >= nH + nKv) return;
     const int b = m / gamma, t = m % gamma;
     const int pos = block_pos[b] + t;
-    const int half = hd / 2, i = threadIdx.x;
+    const int half = hd / 2, np = half / 32;      // pairs per lane
     const int64_t col = (int64_t)hh * hd;
-    const PartView::Pending q1 = part.load(m, col + i), q2 = part.load(m, col + i + half);
-    const float x1 = part.finish(q1), x2 = part.finish(q2);
-    const float ss = block_sum(x1 * x1 + x2 * x2, red);
+    PartView::Pending p1[kQkMaxPairs], p2[kQkMaxPairs];
+#pragma unroll
+    for (int e = 0; e < kQkMaxPairs; ++e) {
+        if (e < np) {
+            p1[e] = part.load(m, col + lane + 32 * e);
+            p2[e] = part.load(m, col + lane + 32 * e + half);
+        }
+    }
+    float x1[kQkMaxPairs], x2[kQkMaxPairs];
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < kQkMaxPairs; ++e) {
+        x1[e] = e < np ? part.finish(p1[e]) : 0.f;
+        x2[e] = e < np ? part.finish(p2[e]) : 0.f;
+        ss += x1[e] * x1[e] + x2[e] * x2[e];
+    }
+    ss = warp_sum(ss);
     const float rinv = rsqrtf(ss / (float)hd + eps);
-    float y1 = x1 * rinv, y2 = x2 * rinv;
-    float sn, cs;
-    rope_sincos(pos, inv_freq[i], &sn, &cs);
-    if (hh < nH) {
-        y1 *= load_any(q_norm, i, dtype);
-        y2 *= load_any(q_norm, i + half, dtype);
-        const int64_t o = ((int64_t)m * nH + hh) * hd;
-        q[o + i] = y1 * cs - y2 * sn;
-        q[o + i + half] = y2 * cs + y1 * sn;
-    } else {
-        const int g = hh - nH;
-        const int64_t o = ((int64_t)m * nKv + g) * hd;
-        store_any(vb, o + i, dtype, y1);
-        store_any(vb, o + i + half, dtype, y2);
-        const float k1 = y1 * load_any(k_norm, i, dtype), k2 = y2 * load_any(k_norm, i + half, dtype);
-        store_any(kb, o + i, dtype, k1 * cs - k2 * sn);
-        store_any(kb, o + i + half, dtype, k2 * cs + k1 * sn);
+#pragma unroll
+    for (int e = 0; e < kQkMaxPairs; ++e) {
+        if (e >= np) break;
+        const int i = lane + 32 * e;
+        float y1 = x1[e] * rinv, y2 = x2[e] * rinv;
+        float sn, cs;
+        rope_sincos(pos, inv_freq[i], &sn, &cs);
+        if (hh < nH) {
+            y1 *= load_any(q_norm, i, dtype);
+            y2 *= load_any(q_norm, i + half, dtype);
+            const int64_t o = ((int64_t)m * nH + hh) * hd;
+            q[o + i] = y1 * cs - y2 * sn;
+            q[o + i + half] = y2 * cs + y1 * sn;
+        } else {
+            const int g = hh - nH;
+            const int64_t o = ((int64_t)m * nKv + g) * hd;
+            store_any(vb, o + i, kv_dtype, y1);
+            store_any(vb, o + i + half, kv_dtype, y2);
+            const float k1 = y1 * load_any(k_norm, i, dtype), k2 = y2 * load_any(k_norm, i + half, dtype);
+            store_any(kb, o + i, kv_dtype, k1 * cs - k2 * sn);
+            store_any(kb, o + i + half, kv_dtype, k2 * cs + k1 * sn);
+        }
     }
 }
 
@@ -210,42 +255,49 @@ template <int PER>
 __global__ void __launch_bounds__(512) residual_epilogue_kernel(PartView part, int H, const void* __restrict__ g1,
                                          const void* __restrict__ g2, const void* __restrict__ scalar, int mode,
                                          float eps, int dtype, float* __restrict__ h, ActBuf x) {
+    constexpr int G4 = PER / 4;                  // float4 groups per thread
     __shared__ float red[32];
     __shared__ float xch[2];
     pdl_trigger();
     const int C = gridDim.x;
     const int m = blockIdx.y;
-    const int j0 = blockIdx.x * blockDim.x * PER + threadIdx.x;
+    // this thread's columns: 4 consecutive ones per group, groups blockDim.x * 4 apart
+    const int j0 = blockIdx.x * blockDim.x * PER + threadIdx.x * 4;
     float a[PER], hv[PER], w1v[PER], w2v[PER];
     // the gains are weights: loaded while the producing GEMM drains
 #pragma unroll
-    for (int c = 0; c < PER; ++c) {
-        const int j = j0 + c * blockDim.x;
-        const bool in = j < H;
-        w1v[c] = in ? load_any(g1, j, dtype) : 0.f;
-        w2v[c] = in ? load_any(g2, j, dtype) : 0.f;
+    for (int g = 0; g < G4; ++g) {
+        const int j = j0 + g * blockDim.x * 4;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const bool in = j + c < H;
+            w1v[g * 4 + c] = in ? load_any(g1, j + c, dtype) : 0.f;
+            w2v[g * 4 + c] = in ? load_any(g2, j + c, dtype) : 0.f;
+        }
     }
     const float s = mode == 1 ? load_any(scalar, 0, dtype) : 1.f;
     pdl_wait();
-    // the activation loads go out in groups of 4 columns (each with all its
-    // partials): one or two rounds of memory latency at bounded registers
+    // the activation loads go out two groups at a time (each with all its partials):
+    // a round of memory latency per two groups at bounded registers
+    constexpr int kBatch = G4 < 2 ? G4 : 2;
 #pragma unroll
-    for (int c = 0; c < PER; ++c) {
-        const int j = j0 + c * blockDim.x;
-        hv[c] = j < H ? h[(int64_t)m * H + j] : 0.f;
-    }
+    for (int g0 = 0; g0 < G4; g0 += kBatch) {
+        PartView::Pending4 q[kBatch];
 #pragma unroll
-    for (int c0 = 0; c0 < PER; c0 += 4) {
-        PartView::Pending q[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int j = j0 + (c0 + c) * blockDim.x;
-            q[c] = part.load(m, j < H ? j : 0);
+        for (int gb = 0; gb < kBatch; ++gb) {
+            const int g = g0 + gb;
+            const int j = j0 + g * blockDim.x * 4;
+            const bool in = j < H;
+            q[gb] = part.load4(m, in ? j : 0);
+            const float4 hh = in ? *reinterpret_cast<const float4*>(h + (int64_t)m * H + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            hv[g * 4] = hh.x; hv[g * 4 + 1] = hh.y; hv[g * 4 + 2] = hh.z; hv[g * 4 + 3] = hh.w;
         }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int j = j0 + (c0 + c) * blockDim.x;
-            a[c0 + c] = j < H ? part.finish(q[c]) : 0.f;
+        for (int gb = 0; gb < kBatch; ++gb) {
+            const int g = g0 + gb;
+            const int j = j0 + g * blockDim.x * 4;
+            const float4 v = j < H ? part.finish4(q[gb]) : make_float4(0.f, 0.f, 0.f, 0.f);
+            a[g * 4] = v.x; a[g * 4 + 1] = v.y; a[g * 4 + 2] = v.z; a[g * 4 + 3] = v.w;
         }
     }
     float ss = 0.f;
@@ -262,26 +314,28 @@ __global__ void __launch_bounds__(512) residual_epilogue_kernel(PartView part, i
     ss2 = cluster_row_sum(ss2, red, &xch[1], C);
     const float r2 = rsqrtf(ss2 / (float)H + eps);
 #pragma unroll
-    for (int c = 0; c < PER; ++c) {
-        const int j = j0 + c * blockDim.x;
+    for (int g = 0; g < G4; ++g) {
+        const int j = j0 + g * blockDim.x * 4;
         if (j < H) {
-            h[(int64_t)m * H + j] = hv[c];
-            store_act(x, (int64_t)m * H + j, hv[c] * r2 * w2v[c]);
+            const int64_t o = (int64_t)m * H + j;
+            *reinterpret_cast<float4*>(h + o) = make_float4(hv[g * 4], hv[g * 4 + 1], hv[g * 4 + 2], hv[g * 4 + 3]);
+            store_act4(x, o, make_float4(hv[g * 4] * r2 * w2v[g * 4], hv[g * 4 + 1] * r2 * w2v[g * 4 + 1],
+                                         hv[g * 4 + 2] * r2 * w2v[g * 4 + 2], hv[g * 4 + 3] * r2 * w2v[g * 4 + 3]));
         }
     }
     if (C > 1) cluster_sync();
 }
 
-__global__ void gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
+__global__ void __launch_bounds__(256) gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
     pdl_trigger();
     pdl_wait();
-    const int64_t total = (int64_t)M * I;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = e / I, i = e % I;
-        const PartView::Pending qg = part.load(m, i), qu = part.load(m, I + i);
-        const float g = part.finish(qg), u = part.finish(qu);
-        store_act(act, e, gelu_tanh(g) * u);
-    }
+    const int m = blockIdx.y;
+    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (i >= I) return;
+    const PartView::Pending4 qg = part.load4(m, i), qu = part.load4(m, I + i);
+    const float4 g = part.finish4(qg), u = part.finish4(qu);
+    store_act4(act, (int64_t)m * I + i,
+               make_float4(gelu_tanh(g.x) * u.x, gelu_tanh(g.y) * u.y, gelu_tanh(g.z) * u.z, gelu_tanh(g.w) * u.w));
 }
 
 // ------------------------------------------------------------------ confidence + truncation
@@ -381,7 +435,7 @@ cudaError_t launch_kv_epilogue(const dspark_model* m, const PartView& raw, const
     for (int l = 0; l < d.Lyr; ++l) kn.p[l] = m->layers[l].k_norm;
     dim3 grid(rp.nrows, d.Lyr * d.nKv);
     return launch_pdl(kv_epilogue_kernel, grid, dim3(d.hd / 2), 0, s, raw, rp, dst, m->ws.inv_freq, kn, d.nKv, d.hd,
-                      d.eps, d.dtype, m->ws.status);
+                      d.eps, d.dtype, d.kv_dtype, m->ws.status);
 }
 
 cudaError_t launch_append_check(const int32_t* n_new, const int32_t* len, int B, int Lnew_max, int capacity,
@@ -406,9 +460,10 @@ cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const PartView&
                                const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s) {
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
-    dim3 grid(A * d.gamma, d.nH + d.nKv);
-    return launch_pdl(qk_epilogue_kernel, grid, dim3(d.hd / 2), 0, s, part, d.gamma, d.nH, d.nKv, d.hd, block_pos,
-                      m->ws.inv_freq, m->layers[layer].q_norm, m->layers[layer].k_norm, d.eps, d.dtype, q, kb, vb);
+    dim3 grid(A * d.gamma, (d.nH + d.nKv + kQkHeadsPerCta - 1) / kQkHeadsPerCta);
+    return launch_pdl(qk_epilogue_kernel, grid, dim3(32 * kQkHeadsPerCta), 0, s, part, d.gamma, d.nH, d.nKv, d.hd,
+                      block_pos, m->ws.inv_freq, m->layers[layer].q_norm, m->layers[layer].k_norm, d.eps, d.dtype,
+                      d.kv_dtype, q, kb, vb);
 }
 
 cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,
@@ -423,10 +478,8 @@ cudaError_t launch_gu_epilogue(const dspark_model* m, const PartView& part, int 
                                cudaStream_t s) {
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
-    const int64_t total = (int64_t)M * d.I;
-    int blocks = (int)((total + 255) / 256);
-    if (blocks > 8 * m->num_sms) blocks = 8 * m->num_sms;
-    return launch_pdl(gu_epilogue_kernel, dim3(blocks), dim3(256), 0, s, part, M, d.I, act);
+    const dim3 grid((unsigned)((d.I / 4 + 255) / 256), (unsigned)M);
+    return launch_pdl(gu_epilogue_kernel, grid, dim3(256), 0, s, part, M, d.I, act);
 }
 
 cudaError_t launch_down_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,

@@ -31,9 +31,10 @@ constexpr int kMaxChunks = 16;
 constexpr int kStageBytes = 96 * 1024;
 
 __global__ void walk_init_kernel(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V,
-                                 int32_t* status) {
+                                 int32_t* status, const int* skip) {
     pdl_trigger();
     pdl_wait();
+    if (skip && *skip == 0) return;      // the pruned walk wrote the tokens
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b == 0) *ticket = 0u;
     if (b < A) {
@@ -102,6 +103,15 @@ walk_step_kernel(WalkArgs a, MatRef W2, const void* __restrict__ w1, int dtype, 
         }
     }
     pdl_wait();          // markov_w2 is requested above; prev comes from the previous step
+    if (a.skip && *a.skip == 0) {
+        // the pruned walk wrote the tokens: only the copies in flight must land before exit (bounded)
+        if (STAGED && tid == 0) {
+            const uint64_t deadline = tc::global_timer_ns() + tc::kWaitLimitNs;
+            for (int c = 0; c < nchunks; ++c)
+                if (!tc::mbar_wait_until(&bars[c], 0u, deadline)) { atomicOr(a.status, DSPARK_DEV_WAIT_TIMEOUT); break; }
+        }
+        return;
+    }
     for (int i = tid; i < nb * r; i += kThreads) {
         const int bb = i / r, j = i % r;
         e[bb][j] = load_any(w1, (int64_t)a.prev[b0 + bb] * r + j, dtype);
@@ -235,8 +245,9 @@ int walk_vocab_blocks(int num_sms, int V, int r, int dtype, bool quant) {
 }
 
 cudaError_t launch_walk_init(const int32_t* anchors, int32_t* prev, uint32_t* ticket, int A, int V, int32_t* status,
-                             cudaStream_t s) {
-    return launch_pdl(walk_init_kernel, dim3((A + 127) / 128), dim3(128), 0, s, anchors, prev, ticket, A, V, status);
+                             const int* skip, cudaStream_t s) {
+    return launch_pdl(walk_init_kernel, dim3((A + 127) / 128), dim3(128), 0, s, anchors, prev, ticket, A, V, status,
+                      skip);
 }
 
 cudaError_t launch_walk_step(const dspark_model* m, const WalkArgs& a, cudaStream_t s) {

@@ -55,6 +55,7 @@ struct PWalkArgs {
     // staged variant: shared-memory layout (byte offsets) and resident rows
     int staged, R, off_u, off_res, off_ring, off_bars;
     int32_t* status;
+    const int* skip;           // non-NULL: return at once when *skip == 0 (tokens already written)
 };
 
 __device__ __forceinline__ void w2_load8(const MatRef& W, int dtype, int group, int64_t v, int c8, int r, float w[8]) {
@@ -169,6 +170,7 @@ walk_persistent_kernel(PWalkArgs a, MatRef W2, const void* __restrict__ w1) {
     __shared__ float rv[kWarps][8];
     __shared__ int ri[kWarps][8];
     __shared__ int s_fail;
+    if (a.skip && *a.skip == 0) return;   // uniform: every CTA reads the same word
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int G = a.G, V = a.V, r = a.r, A = a.A;
     const int nblk = gridDim.x;
@@ -424,7 +426,8 @@ bool walk_persistent_supported(const dspark_model* m, int A) {
 int walk_persistent_blocks(const dspark_model* m) { return m->num_sms; }
 
 cudaError_t launch_walk_persistent(const dspark_model* m, const float* U, const int32_t* anchors, int32_t* tokens,
-                                   float* cand_val, int32_t* cand_idx, uint32_t* arrivals, int A, cudaStream_t s) {
+                                   float* cand_val, int32_t* cand_idx, uint32_t* arrivals, const int* skip, int A,
+                                   cudaStream_t s) {
     const Dims& d = m->d;
     const int nblk = walk_persistent_blocks(m);
     PWalkArgs pa{};
@@ -432,6 +435,7 @@ cudaError_t launch_walk_persistent(const dspark_model* m, const float* U, const 
     pa.arrivals = arrivals; pa.A = A; pa.G = d.gamma; pa.V = d.V; pa.r = d.r; pa.dtype = d.dtype; pa.group = d.group;
     pa.per = (int)round_up((size_t)(d.V + nblk - 1) / nblk, 4);
     pa.status = m->ws.status;
+    pa.skip = skip;
     const Layout L = plan_layout(m, A, pa.per, U);
     pa.staged = L.staged ? 1 : 0;
     pa.R = L.R; pa.off_u = L.off_u; pa.off_res = L.off_res; pa.off_ring = L.off_ring; pa.off_bars = L.off_bars;

@@ -49,9 +49,11 @@ extern "C" {
 #define DSPARK_DEV_BAD_LENGTH    2  /* a cache length above capacity was clamped */
 #define DSPARK_DEV_WAIT_TIMEOUT  4  /* a bounded device wait gave up */
 #define DSPARK_DEV_CAPACITY      8  /* an append was refused on the device (a count outside [0, Lnew_max] or past capacity) */
+#define DSPARK_DEV_RANGE        16  /* a 4-bit model's context row held a value outside fp16's range (|x| > 65504) */
 
 #define DSPARK_DTYPE_F32  0
 #define DSPARK_DTYPE_BF16 1
+#define DSPARK_DTYPE_F16  2   /* the context K/V of bf16 models (dspark_kv_dtype) */
 
 /*
  * Model configuration: the drafter's config.json keys (deepspec.ts,
@@ -131,10 +133,22 @@ typedef struct dspark_weights {
 } dspark_weights;
 
 /*
+ * Element type "KV" of the context K/V (caches, the projection's outputs, the
+ * attention seam's tensors): DSPARK_DTYPE_F16 for a bf16 model, DSPARK_DTYPE_F32
+ * for an fp32 one; -1 for an invalid config. The drafter page keeps ContextKV
+ * rows in the model dtype; here a bf16 model's rows are fp16 instead (same two
+ * bytes per element): the keys and values are RMS-normed (|x| <= sqrt(head_dim)
+ * times the k_norm gain), where fp16's 11-bit significand holds them more
+ * precisely than bf16's 8 bits, and the tensor cores multiply fp16 queries and
+ * probabilities with them without converting any cache tile.
+ */
+int32_t dspark_kv_dtype(const dspark_config* cfg);
+
+/*
  * Per-request context K/V storage, owned by the caller (the drafter page's
  * seam: "storage owns context validity"; deepspec.ts draftRows doc: the
  * caller owns the cache's lifetime and the crop after the round).
- * k, v: device T [num_hidden_layers][batch][capacity][nKv][hd]; row t of
+ * k, v: device KV [num_hidden_layers][batch][capacity][nKv][hd]; row t of
  * batch row b holds the K (normed, roped) / V (scale-less normed, unroped)
  * of context row t. len: device int32 [batch], the valid rows per batch row;
  * the caller sets it when it builds or crops a cache (a crop is a smaller
@@ -191,7 +205,7 @@ size_t dspark_project_workspace_bytes(const dspark_model* model, int64_t rows);
  * where p = static_pos + t when pos0 == NULL, else pos0[b] + t.
  *   hidden  device T [B, L, H]
  *   pos0    device int32 [B] or NULL
- *   k_out, v_out  device T [num_hidden_layers][B][L][nKv][hd]
+ *   k_out, v_out  device KV [num_hidden_layers][B][L][nKv][hd]
  * (the dspark_kv_cache layout with capacity = L).
  */
 int dspark_project_context_kv(const dspark_model* model, const void* hidden, int32_t B, int32_t L,
@@ -253,28 +267,35 @@ int dspark_draft_rows(const dspark_model* model, const dspark_kv_cache* cache,
  * q[b,:,h,:] over keys [cache.k[layer,b,0:len_b,g] ++ k_blk[b,:,g]] and
  * values [cache.v[layer,b,0:len_b,g] ++ v_blk[b,:,g]], g = h / (nH/nKv),
  * non-causal, scale 1.0, softmax in fp32.
- *   q   device T [A, gamma, nH, hd]     k_blk, v_blk device T [A, gamma, nKv, hd]
- *   out device T [A, gamma, nH, hd]
+ *   q   device KV [A, gamma, nH, hd]    k_blk, v_blk device KV [A, gamma, nKv, hd]
+ *   out device KV [A, gamma, nH, hd]      (KV: dspark_kv_dtype)
  */
 int dspark_attend(const dspark_model* model, int32_t layer, const dspark_kv_cache* cache,
                   const void* q, const void* k_blk, const void* v_blk, void* out,
                   int32_t A, int32_t max_ctx_len, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * dspark_attend without a workspace argument: it computes exactly what
- * dspark_attend computes (same kernels, same split plan), for callers that
+ * dspark_attend without a workspace argument: it computes what dspark_attend
+ * computes, with the same kernels (a bf16 model's call may split the keys
+ * over fewer CTAs, so results can differ in the last bits), for callers that
  * cannot provide device scratch memory -- a plugin whose host program owns
  * the whole device pool and hands it only the tensors above, or a path that
  * must not call cudaMalloc (which may synchronise the device). The pages have
  * no counterpart to this entry point.
- * Its scratch (the per-split softmax state) is a 16 MiB static device array
- * inside libdspark, allocated on every GPU that loads the library and held
- * until the process exits. Shapes whose state exceeds 16 MiB
- * (A * nH * (context splits + 1) * gamma * (hd + 2) * 4 bytes) are refused
- * with DSPARK_ERR_WORKSPACE before any launch. It allocates nothing. The first
+ * Its scratch (the per-split softmax state and, for a bf16 model, the
+ * work plan) is a 16 MiB static device array inside libdspark, allocated on
+ * every GPU that loads the library and held until the process exits. A bf16
+ * model's call uses at most as many CTAs as that array holds partial states
+ * of 128 x (hd + 2) floats (at hd = 256, 126; fewer CTAs only lengthen the
+ * call), and is refused with DSPARK_ERR_WORKSPACE before any launch when A *
+ * nKv exceeds that; an fp32 model's call needs A * nH * (context splits + 1)
+ * * gamma * (hd + 2) * 4 bytes and is refused above 16 MiB. It allocates nothing. The first
  * call on each device looks up the array's device address (a one-time
- * runtime call): make that first call, with the model's device current,
- * before any stream capture. Every call on a device shares the one array, so
+ * runtime call) and keeps it for the process: make that first call, with the
+ * model's device current, before any stream capture, and do not use this entry
+ * point on a device whose context the process has reset (cudaDeviceReset)
+ * since then: the kept address would not belong to the new context. Every
+ * call on a device shares the one array, so
  * calls that overlap on the GPU (different streams or threads) race: issue
  * them in order on one stream per device. No part of the array needs to
  * start at zero: each call writes every slot before reading it.
@@ -293,6 +314,30 @@ int dspark_attend_no_alloc(const dspark_model* model, int32_t layer, const dspar
  * copies run on the round's stream; they slow the round down.
  */
 int dspark_debug_attention_dump(dspark_model* model, float* dst, size_t bytes);
+
+/*
+ * Test-facing dump of the per-position statistics of the logits U (the
+ * lm-head epilogue's per-tile max / argmax / sum of exponentials, merged per
+ * position; deepspec.ts #computeLogits). While `dst` is non-NULL, every later
+ * dspark_draft_rows call on `model` writes, for each position (row b, step k)
+ * in [A][gamma] order, 16 bytes: float max_v U[b,k,v]; float logsumexp_v
+ * U[b,k,v]; int32 lowest argmax; int32 candidates the Markov walk's exact
+ * pruning kept (above 1024: the full walk decided). `dst` is device memory of
+ * at least `bytes` (a round needing more than A * gamma * 16 bytes fails with
+ * DSPARK_ERR_WORKSPACE before any launch); dst = NULL turns the dump off.
+ */
+int dspark_debug_logit_stats(dspark_model* model, void* dst, size_t bytes);
+
+/*
+ * Test-facing probe of the device-side failure detection (no counterpart on
+ * the pages). Every wait inside the library's kernels is bounded: when it runs
+ * out it records DSPARK_DEV_WAIT_TIMEOUT in the model's status word and the
+ * kernel returns instead of hanging. This enqueues one small kernel that runs
+ * the same bounded wait on an mbarrier nothing ever arrives on, giving up after
+ * `limit_us` microseconds (1 .. 2,000,000), so a test can read the status and
+ * check that the next call runs normally. Faults nothing.
+ */
+int dspark_debug_wait_probe(const dspark_model* model, int32_t limit_us, void* stream);
 
 /* Synchronises `stream`, returns the device status bits in *status and
  * clears them. */

@@ -171,9 +171,13 @@ def _sigmoid(z: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 def store_rounded(x: np.ndarray, store_dtype: Optional[str]) -> np.ndarray:
-    """Round to the cache's storage dtype: the drafter keeps ContextKV rows in the
-    model dtype (``#rms`` casts back to it), so a bf16 model's cached K/V are
-    bf16 values. None / "fp32" / "fp64" keep the fp64 values."""
+    """Round to the cache's storage type (round to nearest even): cached K/V rows
+    hold values of that type, which every later round reads. The drafter keeps
+    ContextKV rows in the model dtype (``#rms`` casts back to it): "bf16" for its
+    bf16 models; "fp16" is the two-byte type with an 11-bit significand.
+    None / "fp32" / "fp64" keep the fp64 values."""
+    if store_dtype == "fp16":
+        return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
     if store_dtype != "bf16":
         return x
     import torch

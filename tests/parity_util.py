@@ -14,8 +14,8 @@ Tolerances (from the round's parity bar):
   * confidences: |delta| <= 1e-3, with the GPU's tokens as the previous tokens.
 
 The cache rows are compared with the oracle's fp64 K/V; the round itself is
-compared with the oracle run on the K/V as the cache stores them (bf16 for
-a bf16 model: the drafter keeps ContextKV in the model dtype).
+compared with the oracle run on the K/V as the cache stores them (fp16 rows
+for a bf16 model, fp32 for fp32: dspark_kv_dtype).
 """
 from __future__ import annotations
 
@@ -70,9 +70,15 @@ def check_tokens(W, U_oracle, anchors, gpu_tokens, what="tokens"):
     return int(decisive.sum()), int(decisive.size)
 
 
+def cache_store(dtype: str) -> str:
+    """Storage type of a model's K/V cache: fp16 rows for a bf16 model (dspark_kv_dtype), fp32 for fp32."""
+    return "fp16" if dtype == "bf16" else dtype
+
+
 def as_stored(kv_rows, dtype: str):
-    """The oracle's fp64 context K/V as the cache stores them (bf16 models keep bf16 rows)."""
-    return [[(O.store_rounded(k, dtype), O.store_rounded(v, dtype)) for (k, v) in row] for row in kv_rows]
+    """The oracle's fp64 context K/V as the cache of a `dtype` model stores them."""
+    store = cache_store(dtype)
+    return [[(O.store_rounded(k, store), O.store_rounded(v, store)) for (k, v) in row] for row in kv_rows]
 
 
 def ensure_built():

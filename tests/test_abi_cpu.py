@@ -45,9 +45,10 @@ def test_workspace_bytes_and_refusals(dsp):
     lib = dsp.get_lib()
     good = _cfg(dsp)
     n = lib.dspark_model_workspace_bytes(ctypes.byref(good))
-    # stacked [Wq;Wk] + [Wg;Wu] + all-layer k_proj, bf16; the pruned walk's |markov_w2| bounds
-    # (fp32 per vocabulary entry); RoPE table, status and padding under 64 KB
-    stacks = 2 * 3840 * (4 * (4608 + 30720) + 4 * 512)
+    # fp16 copies of every round GEMM's weights ([Wq;Wk], [Wg;Wu], o_proj and down_proj per layer,
+    # the lm-head), the all-layer k_proj in bf16; the pruned walk's |markov_w2| bounds (fp32 per
+    # vocabulary entry); RoPE table, status and padding under 64 KB
+    stacks = 2 * 3840 * (4 * (4608 + 30720 + 4096 + 15360) + 262144 + 4 * 512)
     norms = 4 * 262144
     assert stacks + norms <= n <= stacks + norms + (64 << 10)
     for bad in (dict(attention_k_eq_v=0), dict(markov_head_vanilla=0), dict(hidden_activation_gelu_tanh=0),

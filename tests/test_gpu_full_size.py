@@ -44,7 +44,15 @@ def _check_kv(cache, kv_rows, sample, lens, dtype, name, rows_to_check=None):
             assert_close(v[l], kv_rows[i][l][1][idx], dtype, f"{name}: V layer {l} row {b}")
 
 
-@pytest.mark.parametrize("name,sample", [("single_bf16", [0]), ("ragged_bf16", [0, 17]), ("quant4_bf16", [0, 63])])
+def _ragged_extremes():
+    """Row 0 plus the rows with the shortest and the longest context of the ragged workload."""
+    from synthetic import round_meta
+    lens = round_meta(WORKLOADS["ragged_bf16"])[0]
+    return sorted({0, int(lens.argmin()), int(lens.argmax())})
+
+
+@pytest.mark.parametrize("name,sample", [("single_bf16", [0]), ("ragged_bf16", _ragged_extremes()),
+                                         ("quant4_bf16", [0, 63])])
 def test_full_size_round(name, sample):
     import block_draft_model_dspark_b200 as dsp
     wl = WORKLOADS[name]

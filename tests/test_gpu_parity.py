@@ -103,7 +103,7 @@ def test_attend_matches_concat_sdpa(dtype):
     m = small_model(dtype=dtype, block_size=8)
     cpu, W, model = build(m, 5)
     import block_draft_model_dspark_b200 as dsp
-    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    tdt = model.kv_torch_dtype              # the seam's tensors are in the KV dtype (fp16 for a bf16 model)
     A, G, nH, nKv, hd = 4, m.block_size, m.num_attention_heads, m.num_global_key_value_heads, m.global_head_dim
     lens = [0, 1, 333, 1000]
     cap = 1003
@@ -214,7 +214,7 @@ def test_append_equals_recompute_with_sentinels():
     B, cap = 3, 96
     pos0 = torch.tensor([0, 100, 7], dtype=torch.int32, device="cuda")
     cache = dsp.KvCache(model, B, cap)
-    sentinel = torch.tensor(-12345.0, dtype=torch.bfloat16)
+    sentinel = torch.tensor(-12345.0, dtype=cache.k.dtype)
     cache.k.fill_(sentinel)
     cache.v.fill_(sentinel)
     cache.set_lengths([0, 0, 0])
@@ -299,3 +299,101 @@ def test_workspace_too_small_and_bad_anchor_status():
     assert model.dspark_read_device_status() == 0     # read clears it
     t = tok.cpu()
     assert ((t >= 0) & (t < m.vocab_size)).all()
+
+
+# ----------------------------------------------------------------------------- in-round dumps
+
+def test_attention_dump_every_layer_and_logit_stats():
+    """Each layer's attention output inside a round (the attend seam on the round's own
+    activations) and the per-position logit statistics of the lm-head epilogue, against the
+    oracle's round."""
+    m = small_model(dtype="bf16")
+    cpu, W, model = build(m, 61)
+    A, lens, pos0 = 3, [40, 0, 150], [0, 9, 300]
+    hid = torch.randn(A, 150, m.hidden_size, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    cache = _project_into_cache(model, hid, lens, pos0)
+    kv = O.project_context_kv(W, hid, pos0, lengths=lens)
+    anchors, block_pos = [7, 11, m.vocab_size - 2], [p + L for p, L in zip(pos0, lens)]
+    G, nH, hd, L = m.block_size, m.num_attention_heads, m.global_head_dim, m.num_hidden_layers
+    dump = torch.full((L, A, G, nH, hd), float("nan"), dtype=torch.float32, device="cuda")
+    stats = torch.zeros(A * G * 4, dtype=torch.int32, device="cuda")
+    model.dspark_debug_attention_dump(dump)
+    model.dspark_debug_logit_stats(stats)
+    try:
+        out = model.draft(cache, torch.tensor(anchors, dtype=torch.int32, device="cuda"),
+                          torch.tensor(block_pos, dtype=torch.int32, device="cuda"), max(lens))
+        torch.cuda.synchronize()
+    finally:
+        model.dspark_debug_attention_dump(None)
+        model.dspark_debug_logit_stats(None)
+    ref = O.draft_rows(W, as_stored(kv, "bf16"), anchors, block_pos, keep_attention=True)
+    for l in range(L):
+        assert_close(dump[l].cpu().numpy(), ref["attention"][l], "bf16", f"attention dump layer {l}")
+    st = stats.view(A * G, 4).cpu()
+    fmax = st[:, 0].view(torch.float32).numpy().reshape(A, G)
+    flse = st[:, 1].view(torch.float32).numpy().reshape(A, G)
+    farg = st[:, 2].numpy().reshape(A, G)
+    ncand = st[:, 3].numpy().reshape(A, G)
+    U = ref["base_logits"]
+    umax = U.max(-1)
+    lse = umax + np.log(np.exp(U - umax[..., None]).sum(-1))
+    assert_close(fmax, umax, "bf16", "row max")
+    assert_close(flse, lse, "bf16", "row logsumexp")
+    srt = np.sort(U, -1)
+    decisive = (srt[..., -1] - srt[..., -2]) > 1e-2
+    assert (farg[decisive] == U.argmax(-1)[decisive]).all(), "row argmax"
+    assert (ncand >= 1).all() and (ncand <= 1024).all(), ncand
+    # the dumps stay off once cleared: a round with them off does not touch the buffers
+    dump.fill_(0.0)
+    model.draft(cache, torch.tensor(anchors, dtype=torch.int32, device="cuda"),
+                torch.tensor(block_pos, dtype=torch.int32, device="cuda"), max(lens))
+    torch.cuda.synchronize()
+    assert float(dump.abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("scale", [3.0, 30.0])
+def test_walk_above_64_rows(scale):
+    """A = 65 request rows: with a moderate bias the pruned walk decides every position; with a
+    strong one the candidate lists overflow and the per-step full walk (the A > 64 path) runs."""
+    m = small_model(dtype="bf16", markov_rank=64, num_hidden_layers=1)
+    cpu, W, model = build(m, 71, markov_scale=scale)
+    A = 65
+    g = torch.Generator().manual_seed(72)
+    lens = [int(x) for x in torch.randint(1, 33, (A,), generator=g)]
+    pos0 = [int(x) for x in torch.randint(0, 500, (A,), generator=g)]
+    hid = torch.randn(A, max(lens), m.hidden_size, generator=g).to(torch.bfloat16)
+    cache = _project_into_cache(model, hid, lens, pos0)
+    kv = O.project_context_kv(W, hid, pos0, lengths=lens)
+    anchors = [int(x) for x in torch.randint(0, m.vocab_size - 1, (A,), generator=g)]
+    block_pos = [p + L for p, L in zip(pos0, lens)]
+    stats = torch.zeros(A * m.block_size * 4, dtype=torch.int32, device="cuda")
+    model.dspark_debug_logit_stats(stats)
+    try:
+        out, ref = _round_and_compare(m, W, model, cache, kv, anchors, block_pos, lens, f"A=65, markov scale {scale}")
+    finally:
+        model.dspark_debug_logit_stats(None)
+    ncand = stats.view(-1, 4)[:, 3].cpu().numpy()
+    if scale == 3.0:
+        assert (ncand <= 1024).all(), "the pruned walk should decide every position"
+    else:
+        assert (ncand > 1024).any(), "the strong bias should overflow a list and run the full walk"
+    assert (ref["tokens"] != np.argmax(ref["base_logits"], -1)).any()
+
+
+# ----------------------------------------------------------------------------- failure detection
+
+def test_bounded_wait_times_out_and_context_stays_usable():
+    """A device wait that nothing satisfies gives up after its limit, records
+    DSPARK_DEV_WAIT_TIMEOUT, and the next round on the same context is correct."""
+    import block_draft_model_dspark_b200 as dsp
+    m = small_model(dtype="bf16")
+    cpu, W, model = build(m, 81)
+    model.dspark_debug_wait_probe(50_000)                   # 50 ms
+    torch.cuda.synchronize()
+    assert model.dspark_read_device_status() == dsp.DSPARK_DEV_WAIT_TIMEOUT
+    assert model.dspark_read_device_status() == 0
+    lens, pos0 = [33, 70], [0, 5]
+    hid = torch.randn(2, 70, m.hidden_size, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16)
+    cache = _project_into_cache(model, hid, lens, pos0)
+    kv = O.project_context_kv(W, hid, pos0, lengths=lens)
+    _round_and_compare(m, W, model, cache, kv, [1, 2], [33, 75], lens, "round after a wait timeout")

@@ -487,3 +487,15 @@ def test_store_rounded_is_round_to_nearest_even_bf16():
     assert got[0] == 1.0 and got[1] == 1.0 and got[2] == 1.0 + 2 ** -7
     assert abs(got[3] + 3.140625) < 1e-12
     np.testing.assert_array_equal(O.store_rounded(x, None), x)
+
+
+def test_store_rounded_is_round_to_nearest_even_fp16():
+    """fp16 keeps 11 significant bits: hand-worked ties and the subnormal spacing 2^-24."""
+    x = np.array([1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11, 2049.0, 2051.0, -3.14159, 2 ** -24 * 1.5, 70000.0])
+    got = O.store_rounded(x, "fp16")
+    assert got[0] == 1.0                          # a tie -> even
+    assert got[1] == 1.0 + 2 ** -9                # 1 + 3 * 2^-11 -> up to 1 + 4 * 2^-11
+    assert got[2] == 2048.0 and got[3] == 2052.0  # spacing 2 above 2048: ties to even
+    assert got[4] == -3.140625                    # -3.14159 -> nearest multiple of 2^-9
+    assert got[5] == 2 ** -23                     # subnormals: a multiple of 2^-24, tie -> even
+    assert np.isinf(got[6])                       # past 65504
