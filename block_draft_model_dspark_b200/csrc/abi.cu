@@ -179,7 +179,7 @@ struct Carve {
 struct DraftPlan {
     int M, attn_splits, attn_chunk, walk_blocks;
     int attn_tc_grid;    // tensor-core attention: CTAs (0: the CUDA-core split plan)
-    size_t attn_plan;    // its work plan (ints)
+    size_t attn_items;   // its per-item (first slot, slots) for the merge (ints)
     bool tc;      // tensor-core GEMMs: the inputs are also kept in fp16 (hi)
     bool pairs;   // ... and as the fp16 pair (hi, lo)
     size_t h, x, part, q, kb, vb, attn_out, act, U, part_o, part_ml, prev, ticket, walk_val, walk_idx, walk_keys;
@@ -213,7 +213,7 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
     p.h = c.take((size_t)p.M * d.H * 4);
     p.x = c.take((size_t)p.M * d.H * 4);
     p.part = c.take(part_elems * 4);
-    p.q = c.take((size_t)p.M * d.nH * d.hd * 4);
+    p.q = c.take((size_t)p.M * d.nH * d.hd * es);    // the attention's queries, in the KV dtype
     p.kb = c.take((size_t)p.M * d.nKv * d.hd * es);
     p.vb = c.take((size_t)p.M * d.nKv * d.hd * es);
     p.attn_out = c.take((size_t)p.M * d.nH * d.hd * 4);
@@ -225,12 +225,12 @@ DraftPlan plan_draft(const dspark_model* m, int A, int maxL) {
         const size_t slot_f = tc::attention_tc_partial_floats(m, p.attn_tc_grid);
         p.part_o = c.take(slot_f / (d.hd + 2) * d.hd * 4);
         p.part_ml = c.take(slot_f / (d.hd + 2) * 2 * 4);
-        p.attn_plan = c.take(tc::attention_tc_plan_ints(m, A, p.attn_tc_grid) * 4);
+        p.attn_items = c.take(tc::attention_tc_item_ints(m, A) * 4);
     } else {
         const size_t S1 = (size_t)p.attn_splits + 1;
         p.part_o = c.take((size_t)A * d.nH * S1 * d.gamma * d.hd * 4);
         p.part_ml = c.take((size_t)A * d.nH * S1 * d.gamma * 2 * 4);
-        p.attn_plan = c.take(0);
+        p.attn_items = c.take(0);
     }
     p.prev = c.take((size_t)A * 4);
     p.ticket = c.take(256);
@@ -598,18 +598,18 @@ static int check_cache(const dspark_model* m, const dspark_kv_cache* c, int A, i
 }
 
 static AttnArgs attn_args(const dspark_model* m, const DraftPlan& p, void* ws, const dspark_kv_cache* c, int layer, int A,
-                          const void* q, const void* kb, const void* vb, void* out, int io_dtype) {
+                          const void* q, const void* kb, const void* vb, void* out, int q_dtype, int out_dtype) {
     const Dims& d = m->d;
     const size_t es = esize(d.kv_dtype);
     const size_t layer_bytes = (size_t)c->batch * c->capacity * d.nKv * d.hd * es;
     AttnArgs a{};
     a.q = q; a.kb = kb; a.vb = vb; a.out = out;
-    a.q_dtype = io_dtype; a.out_dtype = io_dtype;
+    a.q_dtype = q_dtype; a.out_dtype = out_dtype;
     a.kc = static_cast<const char*>(c->k) + layer_bytes * layer;
     a.vc = static_cast<const char*>(c->v) + layer_bytes * layer;
     a.len = c->len; a.capacity = c->capacity; a.batch = c->batch;
     a.part_o = at<float>(ws, p.part_o); a.part_ml = at<float>(ws, p.part_ml);
-    a.plan = p.attn_tc_grid ? at<int>(ws, p.attn_plan) : nullptr; a.tc_grid = p.attn_tc_grid;
+    a.item_slots = p.attn_tc_grid ? at<int>(ws, p.attn_items) : nullptr; a.tc_grid = p.attn_tc_grid;
     a.A = A; a.n_splits = p.attn_splits; a.chunk = p.attn_chunk;
     a.status = m->ws.status;
     // algorithmic work: every valid context row's K and V once, the block K/V, q and out
@@ -618,7 +618,7 @@ static AttnArgs attn_args(const dspark_model* m, const DraftPlan& p, void* ws, c
         for (int b = 0; b < A; ++b) keys += c->len_host[b];
     else
         keys += (double)A * c->capacity;
-    const double qo = 2.0 * A * d.gamma * d.nH * d.hd * (io_dtype == DSPARK_DTYPE_F32 ? 4.0 : (double)es);
+    const double qo = (double)A * d.gamma * d.nH * d.hd * (esize(q_dtype) + esize(out_dtype));
     a.kv_bytes = keys * d.nKv * d.hd * 2.0 * es + qo;
     a.flops = 4.0 * (double)d.nH * d.gamma * d.hd * keys;
     return a;
@@ -632,9 +632,11 @@ int dspark_attend(const dspark_model* m, int32_t layer, const dspark_kv_cache* c
     if (rc) DSPARK_FAIL(rc, why);
     if (layer < 0 || layer >= m->d.Lyr) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "layer out of range");
     if (!q || !k_blk || !v_blk || !out || !ws) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "q, k_blk, v_blk, out and ws must be non-NULL");
+    if (!aligned16(q) || !aligned16(k_blk) || !aligned16(v_blk) || !aligned16(out) || !aligned16(ws))
+        DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "q, k_blk, v_blk, out and ws must be 16-byte aligned");
     const DraftPlan p = plan_draft(m, A, max_ctx_len);
     if (ws_bytes < p.total) DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "ws smaller than dspark_draft_workspace_bytes(): " + std::to_string(p.total));
-    const AttnArgs a = attn_args(m, p, ws, cache, layer, A, q, k_blk, v_blk, out, m->d.kv_dtype);
+    const AttnArgs a = attn_args(m, p, ws, cache, layer, A, q, k_blk, v_blk, out, m->d.kv_dtype, m->d.kv_dtype);
     cudaError_t e = run_attention(m, a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
     return DSPARK_OK;
@@ -662,7 +664,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     const int M = p.M;
     float* h = at<float>(ws, p.h);
     float* part = at<float>(ws, p.part);
-    float* q = at<float>(ws, p.q); void* kb = at<void>(ws, p.kb); void* vb = at<void>(ws, p.vb);
+    void* q = at<void>(ws, p.q); void* kb = at<void>(ws, p.kb); void* vb = at<void>(ws, p.vb);
     float* U = base_logits ? base_logits : at<float>(ws, p.U);
     ActBuf x, ao, act;
     x.f32 = at<float>(ws, p.x); ao.f32 = at<float>(ws, p.attn_out); act.f32 = at<float>(ws, p.act);
@@ -684,9 +686,8 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
         e = run_gemm(m, x, L.qk, M, Nqk, d.H, part, sc, &pv, DSPARK_TIMER_GEMM_QK, s);
         if (e == cudaSuccess) e = launch_qk_epilogue(m, l, pv, A, block_pos, q, kb, vb, s);
         if (e == cudaSuccess) {
-            AttnArgs a = attn_args(m, p, ws, cache, l, A, q, kb, vb, ao.f32, DSPARK_DTYPE_F32);
+            AttnArgs a = attn_args(m, p, ws, cache, l, A, q, kb, vb, ao.f32, d.kv_dtype, DSPARK_DTYPE_F32);
             a.out_hi = ao.hi; a.out_lo = ao.lo;
-            a.plan_ready = l > 0;           // every layer attends over the same lengths
             e = run_attention(m, a, s);
         }
         if (e == cudaSuccess && m->attn_dump)

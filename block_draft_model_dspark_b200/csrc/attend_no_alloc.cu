@@ -59,6 +59,9 @@ extern "C" int dspark_attend_no_alloc(const dspark_model* m, int32_t layer, cons
     if (!q || !k_blk || !v_blk || !out) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "q, k_blk, v_blk and out must be non-NULL");
     if ((reinterpret_cast<uintptr_t>(c->k) | reinterpret_cast<uintptr_t>(c->v)) & 15u)
         DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "cache k / v must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_blk) | reinterpret_cast<uintptr_t>(v_blk) |
+         reinterpret_cast<uintptr_t>(out)) & 15u)
+        DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "q, k_blk, v_blk and out must be 16-byte aligned");
     const Dims& d = m->d;
 
     // The split plan of dspark_attend; on tensor cores with at most as many CTAs (one
@@ -67,11 +70,11 @@ extern "C" int dspark_attend_no_alloc(const dspark_model* m, int32_t layer, cons
     const int chunk = attention_key_chunk(m, A, max_ctx_len);
     const int splits = max_ctx_len > 0 ? (max_ctx_len + chunk - 1) / chunk : 0;
     int grid = 0;
-    size_t o_bytes, ml_bytes, plan_bytes = 0;
+    size_t o_bytes, ml_bytes, items_bytes = 0;
     if (tcore) {
         const size_t slot_bytes = (size_t)128 * (d.hd + 2) * sizeof(float);
         grid = tc::attention_tc_grid(m, A);
-        const size_t fixed = align_up(tc::attention_tc_plan_ints(m, A, grid) * 4, 256) + 512;
+        const size_t fixed = align_up(tc::attention_tc_item_ints(m, A) * 4, 256) + 512;
         const int fit = (int)((kNoAllocScratchBytes - std::min(fixed, kNoAllocScratchBytes)) / slot_bytes);
         grid = std::min(grid, fit);
         if (grid < A * d.nKv)
@@ -80,14 +83,14 @@ extern "C" int dspark_attend_no_alloc(const dspark_model* m, int32_t layer, cons
                                               "with a caller workspace");
         o_bytes = align_up((size_t)grid * 128 * d.hd * sizeof(float), 256);
         ml_bytes = align_up((size_t)grid * 128 * 2 * sizeof(float), 256);
-        plan_bytes = align_up(tc::attention_tc_plan_ints(m, A, grid) * 4, 256);
+        items_bytes = align_up(tc::attention_tc_item_ints(m, A) * 4, 256);
     } else {
         const size_t parts = (size_t)A * d.nH * (size_t)(splits + 1) * d.gamma;
         o_bytes = align_up(parts * d.hd * sizeof(float), 256);
         ml_bytes = align_up(parts * 2 * sizeof(float), 256);
     }
-    if (o_bytes + ml_bytes + plan_bytes > kNoAllocScratchBytes)
-        DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "attention state needs " + std::to_string(o_bytes + ml_bytes + plan_bytes) +
+    if (o_bytes + ml_bytes + items_bytes > kNoAllocScratchBytes)
+        DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "attention state needs " + std::to_string(o_bytes + ml_bytes + items_bytes) +
                                               " bytes, above the 16 MiB static scratch of dspark_attend_no_alloc; "
                                               "use dspark_attend with a caller workspace");
 
@@ -107,11 +110,11 @@ extern "C" int dspark_attend_no_alloc(const dspark_model* m, int32_t layer, cons
     a.kc = static_cast<const char*>(c->k) + layer_bytes * layer;
     a.vc = static_cast<const char*>(c->v) + layer_bytes * layer;
     a.len = c->len; a.capacity = c->capacity; a.batch = c->batch;
-    // Every slot the merge reads is written earlier in the same call (the plan, then
-    // each CTA's partial state), so nothing here needs clearing between calls.
+    // Every slot (and per-item record) a merge reads is written earlier in the same
+    // call, so nothing here needs clearing between calls.
     a.part_o = static_cast<float*>(scratch);
     a.part_ml = reinterpret_cast<float*>(static_cast<char*>(scratch) + o_bytes);
-    a.plan = tcore ? reinterpret_cast<int*>(static_cast<char*>(scratch) + o_bytes + ml_bytes) : nullptr;
+    a.item_slots = tcore ? reinterpret_cast<int*>(static_cast<char*>(scratch) + o_bytes + ml_bytes) : nullptr;
     a.tc_grid = grid;
     a.A = A; a.n_splits = splits; a.chunk = chunk;
     a.status = m->ws.status;

@@ -4,40 +4,41 @@
 // and at scale 1.0, over the row's cached context keys followed by the
 // block's own keys; GQA maps query head h to kv head h / (nH / nKv).
 //
-// One CTA = a range of key tiles of one item (row b, kv head g), as the plan
-// kernel assigns them from the device-side lengths (ragged rows get CTAs in
-// proportion to their tiles; every CTA runs in one wave). Its query tile is the 128-row MMA
-// side: the grp * gamma queries of the heads that share kv head g (row r =
-// query i * grp + head-in-group). Key tiles of KT = 64 rows are TMA-loaded
-// from the fp16 cache (4-D maps pick kv head g out of [rows, nKv, hd]) and
-// multiplied as they land: both MMAs run as kind::f16 with fp16 operands (q
-// and the probabilities P keep an 11-bit significand; the cache holds fp16).
+// One CTA = a range of key tiles of one item (row b, kv head g), as the work
+// plan assigns them from the device-side lengths (ragged rows get CTAs in
+// proportion to their tiles; every CTA runs in one wave); every CTA computes
+// the plan itself from the lengths, so no plan kernel precedes it. Its query tile is the
+// 128-row MMA side: the grp * gamma queries of the heads that share kv head g
+// (row r = query i * grp + head-in-group), in tensor memory as the S product's
+// A operand (two fp16 values per 32-bit column). Key tiles of KT = 64 rows are
+// TMA-loaded from the fp16 cache (4-D maps pick kv head g out of [rows, nKv,
+// hd]) and multiplied as they land: both MMAs run as kind::f16 with fp16
+// operands (q and the probabilities P keep an 11-bit significand).
 //   S = Q K^T  -> TMEM, two 64-column buffers (tile t in buffer t % 2)
 //   softmax    -> one thread per query row (TMEM lane = row); the running max
 //                 is raised only when a tile's max exceeds it by more than
 //                 kRescale, so O is rarely rescaled in TMEM
 //   O += P V   -> TMEM (hd columns), P fp16 from shared memory (K-major,
 //                 128-byte swizzle), V as an MN-major operand
-// K and V tiles have two shared-memory slots each, so the loads of tile t + 2
-// are in flight while tile t is multiplied; per 64 keys at hd = 256 the
-// tensor cores run 16 (S) + 4 (P V) MMAs.
+// TMEM columns: S buffers [0, 128), O [128, 128 + hd), Q [384, 384 + hd / 2).
+// K and V tiles have kSlots = 3 shared-memory slots each, so three tiles' loads
+// are in flight; per 64 keys at hd = 256 the tensor cores run 16 (S) + 4 (P V) MMAs.
 //
-// Warp roles (352 threads): warps 0-7 run the softmax, two threads per query
-// row (warps w and w + 4 share TMEM lanes 32 (w % 4) ..; each takes 32 of the
-// tile's 64 columns and half of O's columns; the row max is exchanged through
-// shared memory), warp 8 issues the S products and K loads, warp 9 the P V
-// products and V loads, and warp 10 zeroes the V rows past the last key of a
-// partial tile before its product (stale cache rows may hold any bits, and
-// P = 0 times NaN still poisons the accumulator; K needs no fix: those S
-// columns are masked to -inf). K, V and P have two slots each and S two TMEM
-// buffers, so tile t + 1's load and S product and tile t - 1's P V product all
-// overlap tile t's softmax; the softmax waits for P V of tile t - 1 only to
-// rescale O (rare). Every wait is bounded. Shared memory at hd = 256: Q 64 KB,
-// K, V 2 x 32 KB each, P 2 x 16 KB.
+// Warp roles (224 threads): warps 0-3 run the softmax, one thread per query
+// row (TMEM lane), all 64 columns of a tile, no exchange between threads; warp 4
+// issues the S products and K loads, warp 5 the P V products and V loads, and
+// warp 6 zeroes the V rows past the last key of a partial tile before its
+// product (stale cache rows may hold any bits, and P = 0 times NaN still
+// poisons the accumulator; K needs no fix: those S columns are masked to
+// -inf). Tile t + 1's S product and tile t - 1's P V product overlap tile t's
+// softmax; the softmax waits for P V of tile t - 1 only to rescale O (rare).
+// Every wait is bounded. Shared memory at hd = 256: K, V 3 x 32 KB each, P 2 x 16 KB.
 //
-// The CTA writes its unnormalised O with (max, sum) per query row into its own
-// slot, which the merge kernel combines per item. The last range of each (b, g) also takes the
-// block's own keys, as one more tile.
+// An item on one CTA writes its output straight from tensor memory. Otherwise
+// each CTA writes its unnormalised O with (max, sum) per query row into its own
+// slot, and the merge kernel (one warp per output row, over the whole GPU)
+// combines the item's slots in slot order. The last range of each (b, g) also
+// takes the block's own keys, as one more tile.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -54,118 +55,198 @@ namespace dspark {
 namespace tc {
 namespace {
 
-constexpr int kThreads = 352;
-constexpr int kSoftThreads = 256;    // warps 0-7
-constexpr int kIssuerWarp = 8;       // S products and K loads; warp 9: P V products and V loads
-constexpr int kFixWarp = 10;         // zeroes the V rows past the last key of a partial tile
+constexpr int kThreads = 224;
+constexpr int kSoftThreads = 128;    // warps 0-3: one thread per query row
+constexpr int kIssuerWarp = 4;       // S products and K loads; warp 5: P V products and V loads
+constexpr int kFixWarp = 6;          // zeroes the V rows past the last key of a partial tile
 constexpr int KT = 64;               // keys per tile
 constexpr int kSlots = 3;            // shared-memory slots of K tiles, and of V tiles (loads in flight)
 constexpr int kQCol = 2 * KT + 256;  // TMEM columns: S buffers [0, 2 KT), O [2 KT, 2 KT + hd), Q from 384
 constexpr int QROWS = 128;           // MMA M
-constexpr float kRescale = 5.0f;     // natural-log headroom before the running max is raised
+// Natural-log headroom before the running max is raised: P = exp(s - m_run) stays
+// below e^10 = 22026, inside fp16's range (65504) at fp16's relative precision.
+constexpr float kRescale = 10.0f;
 
 struct AttnTcParams {
-    int A, G, nH, nKv, grp, hd, capacity, q_dtype;
-    const void* q;                   // [A, G, nH, hd] (fp32 or fp16)
+    int A, G, nH, nKv, grp, hd, capacity, q_dtype, grid;
+    const void* q;                   // [A, G, nH, hd] fp16
     const int32_t* len;
     float* part_o; float* part_ml;   // one slot per CTA: [CTA][128 rows][hd] and [CTA][128 rows][2]
-    const int* cta_item;             // [grid] the (row, kv head) item of each CTA (-1: idle)
-    const int* cta_t0; const int* cta_t1;   // [grid] its tile range within the item
+    int* item_slots;                 // [A * nKv][2]: the item's first slot and its number of slots
+    void* out; int out_dtype;        // [A, G, nH, hd] fp32 or fp16
+    __half* out_hi; __half* out_lo;  // optional fp16 pair of the output (the next GEMM's input)
     int32_t* status;
 };
 
-// The work plan (one CTA, device lengths): item i = (row b, kv head g) has n_i =
-// ceil(len_b / KT) context tiles plus the block tile. The smallest q with
+// The work plan (device lengths): item i = (row b, kv head g) has n_i =
+// ceil(len_b / KT) context tiles plus the block tile. The smallest q >= 2 with
 // sum_i ceil(n_i / q) <= grid splits item i into k_i = ceil(n_i / q) equal
-// tile ranges, one CTA each (all CTAs in one wave, none above q tiles);
-// item_cta0 is the exclusive prefix sum of k_i (the CTAs, and partial slots,
-// of item i are item_cta0[i] .. item_cta0[i + 1] - 1).
-constexpr int kPlanThreads = 1024;
+// tile ranges, one CTA each (all CTAs in one wave, none above q tiles; a CTA
+// also builds its query tile and writes a 128-row state, so q = 1 does not
+// pay); the CTAs of item i are the exclusive prefix sum of k_i onwards.
 __device__ __forceinline__ int plan_tiles(const int32_t* len, int b, int capacity) {
     const int L = min(max(len[b], 0), capacity);
     return (L + KT - 1) / KT + 1;
 }
-__device__ __forceinline__ int block_sum_int(int v, int* red) {
+constexpr int kWarps = kThreads / 32;
+// Sum (or maximum) over the block; `buf` holds kWarps ints and callers
+// alternate two buffers, so one barrier per reduction suffices.
+__device__ __forceinline__ int block_reduce_int(int v, int* buf, bool is_max) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = 16; o > 0; o >>= 1) {
+        const int y = __shfl_xor_sync(0xffffffffu, v, o);
+        v = is_max ? max(v, y) : v + y;
+    }
+    if (lane == 0) buf[wid] = v;
     __syncthreads();
-    if (lane == 0) red[wid] = v;
-    __syncthreads();
-    int t = 0;
-    for (int w = 0; w < kPlanThreads / 32; ++w) t += red[w];
+    int t = is_max ? buf[0] : 0;
+    for (int w = is_max ? 1 : 0; w < kWarps; ++w) t = is_max ? max(t, buf[w]) : t + buf[w];
     return t;
 }
-__global__ void __launch_bounds__(kPlanThreads) attn_plan_kernel(const int32_t* __restrict__ len, int A, int nKv,
-                                                                 int capacity, int grid, int* __restrict__ cta_item,
-                                                                 int* __restrict__ cta_t0, int* __restrict__ cta_t1,
-                                                                 int* __restrict__ item_cta0) {
-    __shared__ int red[kPlanThreads / 32];
-    __shared__ int s_base;
-    pdl_trigger();
-    pdl_wait();
-    const int tid = threadIdx.x, n_items = A * nKv;
+struct CtaWork {
+    int item;        // -1: idle
+    int t0, t1;      // tile range within the item
+    int s0, k;       // the item's first CTA (slot) and its number of CTAs
+};
+// This CTA's share of the plan, by all threads of the block (every CTA
+// computes the same plan). `sh` holds 2 kWarps + 5 ints of shared memory.
+__device__ CtaWork cta_work(const int32_t* __restrict__ len, int A, int nKv, int capacity, int grid, int slot,
+                            int* sh) {
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int n_items = A * nKv;
+    int* res = sh + 2 * kWarps;                      // item, index within the item, n, k, first slot
+    if (tid == 0) res[0] = -1;                       // ordered before the scan by the reductions' barriers
+    int nb = 0;
     int mx = 1;
-    for (int i = tid; i < n_items; i += kPlanThreads) mx = max(mx, plan_tiles(len, i / nKv, capacity));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    __syncthreads();
-    if ((tid & 31) == 0) red[tid >> 5] = mx;
-    __syncthreads();
-    mx = 1;
-    for (int w = 0; w < kPlanThreads / 32; ++w) mx = max(mx, red[w]);
-    // the smallest q (tiles per CTA) whose splits fit the grid (q = mx needs n_items <= grid
-    // CTAs), at least 2: a CTA also builds its query tile and writes a 128-row partial
-    // state, and one tile per CTA measured slower at a single 4096-key row
+    for (int i = tid; i < n_items; i += kThreads) mx = max(mx, plan_tiles(len, i / nKv, capacity));
+    mx = block_reduce_int(mx, sh + (nb++ & 1) * kWarps, true);
     int lo = min(2, mx), hi = mx;
     while (lo < hi) {
         const int mid = (lo + hi) / 2;
         int cnt = 0;
-        for (int i = tid; i < n_items; i += kPlanThreads) cnt += (plan_tiles(len, i / nKv, capacity) + mid - 1) / mid;
-        cnt = block_sum_int(cnt, red);
+        for (int i = tid; i < n_items; i += kThreads) cnt += (plan_tiles(len, i / nKv, capacity) + mid - 1) / mid;
+        cnt = block_reduce_int(cnt, sh + (nb++ & 1) * kWarps, false);
         if (cnt <= grid) hi = mid; else lo = mid + 1;
     }
     const int q = lo;
-    // exclusive scan of k_i over the items, in chunks of kPlanThreads
-    if (tid == 0) s_base = 0;
-    __syncthreads();
-    for (int i0 = 0; i0 < n_items; i0 += kPlanThreads) {
+    int base = 0;                                    // CTAs of the items before this chunk
+    for (int i0 = 0; i0 < n_items; i0 += kThreads) {
         const int i = i0 + tid;
         const int n = i < n_items ? plan_tiles(len, i / nKv, capacity) : 0;
         const int k = i < n_items ? (n + q - 1) / q : 0;
-        int x = k;                                        // inclusive scan within the warp
+        int x = k;                                   // inclusive scan within the warp
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if ((tid & 31) >= o) x += y;
+            if (lane >= o) x += y;
         }
+        int* wb = sh + (nb++ & 1) * kWarps;
+        if (lane == 31) wb[wid] = x;
         __syncthreads();
-        if ((tid & 31) == 31) red[tid >> 5] = x;
-        __syncthreads();
-        int wbase = 0;
-        for (int w = 0; w < (tid >> 5); ++w) wbase += red[w];
-        const int excl = s_base + wbase + x - k;
-        if (i < n_items) {
-            item_cta0[i] = excl;
-            // the item's k ranges of n tiles: range j is [j n / k, (j + 1) n / k)
-            for (int j = 0; j < k; ++j) {
-                cta_item[excl + j] = i;
-                cta_t0[excl + j] = (int)((int64_t)j * n / k);
-                cta_t1[excl + j] = (int)((int64_t)(j + 1) * n / k);
-            }
+        int wbase = 0, tot = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            if (w < wid) wbase += wb[w];
+            tot += wb[w];
         }
-        __syncthreads();
-        if (tid == kPlanThreads - 1) s_base = excl + k;
-        __syncthreads();
+        const int excl = base + wbase + x - k;
+        if (i < n_items && slot >= excl && slot < excl + k) {
+            res[0] = i; res[1] = slot - excl; res[2] = n; res[3] = k; res[4] = excl;
+        }
+        base += tot;                                 // the same in every thread
+        if (base > slot) break;
     }
-    const int total = s_base;
-    if (tid == 0) item_cta0[n_items] = total;
-    for (int c = total + tid; c < grid; c += kPlanThreads) { cta_item[c] = -1; cta_t0[c] = 0; cta_t1[c] = 0; }
+    __syncthreads();
+    CtaWork w{res[0], 0, 0, 0, 0};
+    if (w.item >= 0) {
+        const int j = res[1], n = res[2], k = res[3];
+        w.t0 = (int)((int64_t)j * n / k);
+        w.t1 = (int)((int64_t)(j + 1) * n / k);
+        w.s0 = res[4];
+        w.k = k;
+    }
+    return w;
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
     const __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Four consecutive outputs at element o of the output (fp32 or fp16) and of its
+// optional fp16 pair hi = fp16(v), lo = fp16(v - hi).
+__device__ __forceinline__ void store_out4(const AttnTcParams& P, int64_t o, float4 v) {
+    const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+    uint2 hv;
+    hv.x = *reinterpret_cast<const uint32_t*>(&h01);
+    hv.y = *reinterpret_cast<const uint32_t*>(&h23);
+    if (P.out_dtype == DSPARK_DTYPE_F32) *reinterpret_cast<float4*>(static_cast<float*>(P.out) + o) = v;
+    else *reinterpret_cast<uint2*>(static_cast<__half*>(P.out) + o) = hv;
+    if (P.out_hi) {
+        *reinterpret_cast<uint2*>(P.out_hi + o) = hv;
+        if (P.out_lo) {
+            const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+            uint2 lv;
+            lv.x = pack_half2(v.x - f01.x, v.y - f01.y);
+            lv.y = pack_half2(v.z - f23.x, v.w - f23.y);
+            *reinterpret_cast<uint2*>(P.out_lo + o) = lv;
+        }
+    }
+}
+
+// Row r of item (b, g) combined over the item's k slots s0 .. s0 + k - 1 (one
+// warp): weights w_s = exp(m_s - M); lane l owns the 4-column groups l, l + 32.
+constexpr int kMergeBatch = 8;       // slots whose rows a lane loads at once
+__device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, int r, int64_t out_row) {
+    const int lane = threadIdx.x & 31, ng = P.hd / 4;
+    float M = -INFINITY;
+    for (int s = lane; s < k; s += 32) M = fmaxf(M, P.part_ml[((int64_t)(s0 + s) * QROWS + r) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float4 num[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    float den = 0.f;
+    for (int sb = 0; sb < k; sb += 32) {
+        float ws = 0.f, ls = 0.f;
+        if (sb + lane < k) {
+            const int64_t base = (int64_t)(s0 + sb + lane) * QROWS + r;
+            const float m = P.part_ml[base * 2];
+            ls = P.part_ml[base * 2 + 1];
+            ws = m == -INFINITY ? 0.f : __expf(m - M);
+        }
+        const int cnt = min(32, k - sb);
+        for (int t0 = 0; t0 < cnt; t0 += kMergeBatch) {
+            float4 v[kMergeBatch][2];
+#pragma unroll
+            for (int u = 0; u < kMergeBatch; ++u) {
+                const float4* o = reinterpret_cast<const float4*>(P.part_o + ((int64_t)(s0 + sb + t0 + u) * QROWS + r) * P.hd);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int g4 = lane + q * 32;
+                    v[u][q] = (t0 + u < cnt && g4 < ng) ? o[g4] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kMergeBatch; ++u) {
+                const float w = __shfl_sync(0xffffffffu, ws, (t0 + u) & 31);
+                const float l = __shfl_sync(0xffffffffu, ls, (t0 + u) & 31);
+                if (t0 + u >= cnt) break;
+                den += w * l;
+                if (w == 0.f) continue;                // uniform: an empty range
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    num[q].x += w * v[u][q].x; num[q].y += w * v[u][q].y;
+                    num[q].z += w * v[u][q].z; num[q].w += w * v[u][q].w;
+                }
+            }
+        }
+    }
+    const float inv = 1.f / den;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int g4 = lane + q * 32;
+        if (g4 < ng)
+            store_out4(P, out_row + g4 * 4, make_float4(num[q].x * inv, num[q].y * inv, num[q].z * inv, num[q].w * inv));
+    }
 }
 
 // Zeroes rows [nvalid, KT) of a V tile of `nsub` sub-tiles [KT rows x 128 B] (one warp).
@@ -216,7 +297,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     uint8_t* sK = base;                                   // kSlots x tile
     uint8_t* sV = sK + kSlots * tile_sz;                  // kSlots x tile
     uint8_t* sP = sV + kSlots * tile_sz;                  // 2 slots x [128 rows x 128 B]
-    float* red = reinterpret_cast<float*>(sP + 2 * QROWS * 128);   // [2 halves][128 rows] row maxima / sums
+    int* red = reinterpret_cast<int*>(sP + 2 * QROWS * 128);      // plan scratch (2 kWarps + 5 ints), last-CTA flag
     uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * QROWS);
     uint64_t* kfull = bars + 0;                // [kSlots] K tile landed in the slot (TMA)
     uint64_t* vfull = kfull + kSlots;          // [kSlots] V tile landed in the slot (TMA)
@@ -228,9 +309,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     uint64_t* pready = sfree + 2;              // [2] P slot written (256 arrivals)
     uint64_t* odone = pready + 2;              // [2] P V product of the tile in that P slot done (O settled)
     uint64_t* spare = odone + 2;               // teardown: MMAs in flight after an abort
-    uint64_t* xw = spare + 1;                  // row-max exchange: both halves wrote (256 arrivals)
-    uint64_t* xr = xw + 1;                     // row-max exchange: both halves read (256 arrivals)
-    uint64_t* spare2 = xr + 1;                 // teardown of the P V issuer
+    uint64_t* spare2 = spare + 1;              // teardown of the P V issuer
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(spare2 + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -245,8 +324,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         mbar_init(&sdone[0], 1); mbar_init(&sdone[1], 1);
         mbar_init(&sfree[0], kSoftThreads); mbar_init(&sfree[1], kSoftThreads);
         mbar_init(&pready[0], kSoftThreads); mbar_init(&pready[1], kSoftThreads);
-        mbar_init(&odone[0], 1); mbar_init(&odone[1], 1); mbar_init(spare, 1);
-        mbar_init(xw, kSoftThreads); mbar_init(xr, kSoftThreads); mbar_init(spare2, 1);
+        mbar_init(&odone[0], 1); mbar_init(&odone[1], 1); mbar_init(spare, 1); mbar_init(spare2, 1);
         *abort_flag = 0;
         mbar_fence_init();
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmKb); prefetch_tmap(&tmVb);
@@ -257,14 +335,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // q, the lengths and the caches come from earlier kernels. No
-    // pdl_trigger: the merge launches as these CTAs exit (see gemm_tc.cu)
+    // pdl_trigger: the next kernel launches as these CTAs exit (see gemm_tc.cu)
     pdl_wait();
 
-    // this CTA's work: tiles [t_lo, t_hi) of item (b, g) (the plan's); an idle CTA has none
+    // this CTA's work: tiles [t_lo, t_hi) of item (b, g); an idle CTA has none
     const int slot = blockIdx.x;
-    const int item = P.cta_item[slot];
+    const CtaWork W = cta_work(P.len, P.A, P.nKv, P.capacity, P.grid, slot, red);
+    const int item = W.item;
     const int b = item >= 0 ? item / P.nKv : 0, g = item >= 0 ? item % P.nKv : 0;
-    const int t_lo = item >= 0 ? P.cta_t0[slot] : 0, t_hi = item >= 0 ? P.cta_t1[slot] : 0;
+    const int t_lo = W.t0, t_hi = W.t1;
     int len = P.len[b];
     if (len < 0 || len > P.capacity) {
         if (tid == 0) atomicOr(P.status, DSPARK_DEV_BAD_LENGTH);
@@ -279,9 +358,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         else { *row = b * P.G; *nvalid = P.G; *blk = true; }
     };
 
+    const uint32_t tile_bytes = (uint32_t)nsub * KT * 128;
     // The first kSlots K and V tiles do not depend on Q: their loads go out
     // before the Q tile is built, so they land while it is.
-    const uint32_t tile_bytes = (uint32_t)nsub * KT * 128;
     if ((warp == kIssuerWarp || warp == kIssuerWarp + 1) && lane == 0) {
         const bool v_tile = warp != kIssuerWarp;
         for (int t = 0; t < kSlots && t < nt; ++t) {
@@ -299,30 +378,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     // queries are zero. The softmax threads write it, thread (r, half) the row's
     // half of the head dimensions, 16 columns per tcgen05.st.
     if (tid < kSoftThreads) {
-        const int r = tid & (QROWS - 1), half = tid >> 7;
+        // fp16 queries: thread r writes row r, hd / 8 contiguous 16-byte chunks (4 columns
+        // each), loaded 16 at a time before their stores
+        const int r = tid;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int d0 = half * (hd / 2);
         const int i = r / P.grp, h = g * P.grp + r % P.grp;
-        const int64_t off = (((int64_t)b * P.G + i) * P.nH + h) * hd + d0;
-        for (int c0 = 0; c0 < hd / 4; c0 += 16) {           // 16 columns = 32 dimensions
-            uint32_t w[16];
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(P.q) +
+                                                          (((int64_t)b * P.G + i) * P.nH + h) * hd);
+        const int n16 = hd / 8;                               // 16-byte chunks of the row (<= 32)
+        for (int cb = 0; cb < n16; cb += 16) {
+            uint4 u[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                float x0 = 0.f, x1 = 0.f;
-                if (r < nq) {
-                    const int d = 2 * (c0 + j);
-                    if (P.q_dtype == DSPARK_DTYPE_F32) {
-                        const float2 f = *reinterpret_cast<const float2*>(static_cast<const float*>(P.q) + off + d);
-                        x0 = f.x; x1 = f.y;
-                    } else {
-                        // fp16 queries (the attention seam)
-                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(static_cast<const __half*>(P.q) + off + d));
-                        x0 = f.x; x1 = f.y;
-                    }
-                }
-                w[j] = pack_half2(x0, x1);
+            for (int c = 0; c < 16; ++c) u[c] = (cb + c < n16 && r < nq) ? src[cb + c] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int c0 = 0; c0 < 16; c0 += 4) {              // 4 chunks = 16 columns per tcgen05.st
+                if (cb + c0 >= n16) break;
+                const uint32_t w[16] = {u[c0].x, u[c0].y, u[c0].z, u[c0].w, u[c0 + 1].x, u[c0 + 1].y, u[c0 + 1].z,
+                                        u[c0 + 1].w, u[c0 + 2].x, u[c0 + 2].y, u[c0 + 2].z, u[c0 + 2].w,
+                                        u[c0 + 3].x, u[c0 + 3].y, u[c0 + 3].z, u[c0 + 3].w};
+                tmem_st_x16(tmem + (uint32_t)(kQCol + 4 * (cb + c0)) + lane_off, w);
             }
-            tmem_st_x16(tmem + (uint32_t)(kQCol + half * (hd / 4) + c0) + lane_off, w);
         }
         tmem_st_wait();
     }
@@ -447,47 +522,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             if (lane == 0) mbar_arrive(&vready[ks]);
         }
     } else {
-        // ------------------------------------------------------------ softmax (two threads per query row)
-        const int r = tid & (QROWS - 1);                   // query row = TMEM lane
-        const int half = tid >> 7;                         // S columns [32 half, +32), O columns [hd/2 half, +hd/2)
+        // ------------------------------------------------------------ softmax (one thread per query row)
+        const int r = tid;                                 // query row = TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int oc0 = half * (hd / 2);
-        float m_run = -INFINITY, l_run = 0.f;              // l_run: this half's columns
+        float m_run = -INFINITY, l_run = 0.f;
         for (int t = 0; t < nt && ok; ++t) {
             int row, nvalid; bool blk;
             tile_rows(t, &row, &nvalid, &blk);
             const int sl = t & 1;
-            const uint32_t tS = tmem + (uint32_t)(sl * KT) + lane_off + (uint32_t)(half * 32);
-            const int cbase = half * 32;                   // first key of this thread's columns
-            if (!warp_wait(&sdone[sl], (uint32_t)(t >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+            const uint32_t tS = tmem + (uint32_t)(sl * KT) + lane_off;
+            // S(t) is on the critical path: poll (no suspension)
+            if (!warp_wait_spin(&sdone[sl], (uint32_t)(t >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
-            uint32_t u0[16], u1[16];
-            tmem_ld_x16(tS, u0);
-            tmem_ld_x16(tS + 16, u1);
-            tmem_ld_wait();
-            float sv[32];
+            uint32_t u[4][16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) { sv[j] = __uint_as_float(u0[j]); sv[16 + j] = __uint_as_float(u1[j]); }
+            for (int c = 0; c < 4; ++c) tmem_ld_x16(tS + (uint32_t)(16 * c), u[c]);
+            tmem_ld_wait();
+            float sv[KT];
+#pragma unroll
+            for (int j = 0; j < KT; ++j) sv[j] = __uint_as_float(u[j >> 4][j & 15]);
             if (nvalid < KT) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) if (cbase + j >= nvalid) sv[j] = -INFINITY;
+                for (int j = 0; j < KT; ++j) if (j >= nvalid) sv[j] = -INFINITY;
             }
-            float mt[16];                                   // tree maximum: 5 dependent steps, not 32
+            float mt[32];                                   // tree maximum: 6 dependent steps, not 64
 #pragma unroll
-            for (int j = 0; j < 16; ++j) mt[j] = fmaxf(sv[j], sv[16 + j]);
+            for (int j = 0; j < 32; ++j) mt[j] = fmaxf(sv[j], sv[32 + j]);
 #pragma unroll
-            for (int w = 8; w > 0; w >>= 1) {
+            for (int w = 16; w > 0; w >>= 1) {
 #pragma unroll
                 for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
             }
-            float mx = mt[0];
-            // exchange with the other half of the row (mbarriers: every wait stays bounded)
-            if (t >= 1 && !warp_wait_spin(xr, (uint32_t)(t - 1) & 1u, abort_flag, P.status)) { ok = false; break; }
-            red[half * QROWS + r] = mx;
-            mbar_arrive(xw);
-            if (!warp_wait_spin(xw, (uint32_t)t & 1u, abort_flag, P.status)) { ok = false; break; }
-            mx = fmaxf(mx, red[(half ^ 1) * QROWS + r]);
-            mbar_arrive(xr);
+            const float mx = mt[0];
             const bool need = t > 0 && mx > m_run + kRescale;
             if (t == 0) m_run = mx;
             if (__any_sync(0xffffffffu, need)) {
@@ -496,72 +562,90 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 tc_fence_after();
                 const float f = need ? __expf(m_run - mx) : 1.f;
                 if (need) { l_run *= f; m_run = mx; }
-                for (int c = 0; c < hd / 2; c += 16) {
-                    uint32_t u[16];
-                    tmem_ld_x16(tO + lane_off + (uint32_t)(oc0 + c), u);
+                for (int c = 0; c < hd; c += 32) {            // 32 columns per TMEM round trip
+                    uint32_t o[2][16];
+                    tmem_ld_x16(tO + lane_off + (uint32_t)c, o[0]);
+                    tmem_ld_x16(tO + lane_off + (uint32_t)(c + 16), o[1]);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * f);
-                    tmem_st_x16(tO + lane_off + (uint32_t)(oc0 + c), u);
+                    for (int j = 0; j < 32; ++j) o[j >> 4][j & 15] = __float_as_uint(__uint_as_float(o[j >> 4][j & 15]) * f);
+                    tmem_st_x16(tO + lane_off + (uint32_t)c, o[0]);
+                    tmem_st_x16(tO + lane_off + (uint32_t)(c + 16), o[1]);
                 }
                 tmem_st_wait();
             }
             // P slot t % 2 was last read by P(t-2) V(t-2)
-            if (t >= 2 && !warp_wait(&odone[sl], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+            if (t >= 2 && !warp_wait_spin(&odone[sl], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
             float ls[8];                                    // sums in 8 independent chains
 #pragma unroll
             for (int j = 0; j < 8; ++j) ls[j] = 0.f;
             uint8_t* pslot = sP + sl * QROWS * 128;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {                  // four 16-byte chunks of 8 keys
+            for (int q = 0; q < 8; ++q) {                  // eight 16-byte chunks of 8 keys
                 float p[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) { p[j] = __expf(sv[q * 8 + j] - m_run); ls[j] += p[j]; }
-                const int chunk = (cbase >> 3) + q;
-                *reinterpret_cast<uint4*>(pslot + r * 128 + ((chunk ^ (r & 7)) * 16)) =
+                *reinterpret_cast<uint4*>(pslot + r * 128 + ((q ^ (r & 7)) * 16)) =
                     make_uint4(pack_half2(p[0], p[1]), pack_half2(p[2], p[3]), pack_half2(p[4], p[5]), pack_half2(p[6], p[7]));
             }
-            const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-            l_run += lsum;
+            l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
             tc_fence_before();
             mbar_arrive(&sfree[sl]);                           // S buffer read
             fence_async_shared();
             mbar_arrive(&pready[sl]);                          // P written
         }
-        // ---- this range's state: unnormalised O and (max, sum) per query row
+        // ---- this range's result
         const bool any = nt > 0;
         if (any && ok && !warp_wait(&odone[(nt - 1) & 1], (uint32_t)((nt - 1) >> 1) & 1u, abort_flag, P.status)) ok = false;
         tc_fence_after();
-        // the row's sum = both halves' sums (same running max): one more exchange
-        float l_tot = l_run;
-        if (any && ok) {
-            if (!warp_wait(xr, (uint32_t)(nt - 1) & 1u, abort_flag, P.status)) ok = false;
-            if (ok) {
-                red[half * QROWS + r] = l_run;
-                mbar_arrive(xw);
-                if (!warp_wait(xw, (uint32_t)nt & 1u, abort_flag, P.status)) ok = false;
-                else l_tot = l_run + red[(half ^ 1) * QROWS + r];
-            }
-        }
-        if (r < nq && half == 0) {
-            const int64_t prow = (int64_t)slot * QROWS + r;
-            P.part_ml[prow * 2] = any ? m_run : -INFINITY;
-            P.part_ml[prow * 2 + 1] = any ? l_tot : 0.f;
-        }
-        if (any && ok) {
-            float* dst = P.part_o + ((int64_t)slot * QROWS + r) * hd + oc0;
-            // 32 columns per TMEM wait: half the waits, stores of 128 contiguous bytes
-            for (int c = 0; c < hd / 2; c += 32) {
-                uint32_t u[2][16];
-                tmem_ld_x16(tO + lane_off + (uint32_t)(oc0 + c), u[0]);
-                tmem_ld_x16(tO + lane_off + (uint32_t)(oc0 + c + 16), u[1]);
-                tmem_ld_wait();
-                if (r < nq) {
+        if (W.k == 1) {
+            // the item's only CTA: the normalised output straight from tensor memory
+            if (tid == 0) { P.item_slots[2 * item] = W.s0; P.item_slots[2 * item + 1] = 1; }
+            const int64_t out_row = (((int64_t)b * P.G + r / P.grp) * P.nH + g * P.grp + r % P.grp) * hd;
+            if (any && ok) {
+                const float inv = 1.f / l_run;
+                for (int c = 0; c < hd; c += 32) {
+                    uint32_t o[2][16];
+                    tmem_ld_x16(tO + lane_off + (uint32_t)c, o[0]);
+                    tmem_ld_x16(tO + lane_off + (uint32_t)(c + 16), o[1]);
+                    tmem_ld_wait();
+                    if (r < nq) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4*>(dst + c + j) =
-                            make_float4(__uint_as_float(u[j >> 4][j & 15]), __uint_as_float(u[j >> 4][(j & 15) + 1]),
-                                        __uint_as_float(u[j >> 4][(j & 15) + 2]), __uint_as_float(u[j >> 4][(j & 15) + 3]));
+                        for (int j = 0; j < 32; j += 4)
+                            store_out4(P, out_row + c + j,
+                                       make_float4(__uint_as_float(o[j >> 4][j & 15]) * inv,
+                                                   __uint_as_float(o[j >> 4][(j & 15) + 1]) * inv,
+                                                   __uint_as_float(o[j >> 4][(j & 15) + 2]) * inv,
+                                                   __uint_as_float(o[j >> 4][(j & 15) + 3]) * inv));
+                    }
+                }
+            }
+        } else if (item >= 0) {
+            // unnormalised O and (max, sum) per query row into this CTA's slot
+            if (tid == 0 && W.t0 == 0) {                      // the item's first CTA tells the merge its slots
+                P.item_slots[2 * item] = W.s0;
+                P.item_slots[2 * item + 1] = W.k;
+            }
+            if (r < nq) {
+                const int64_t prow = (int64_t)slot * QROWS + r;
+                P.part_ml[prow * 2] = any ? m_run : -INFINITY;
+                P.part_ml[prow * 2 + 1] = any ? l_run : 0.f;
+            }
+            if (any && ok) {
+                float* dst = P.part_o + ((int64_t)slot * QROWS + r) * hd;
+                // 32 columns per TMEM wait: half the waits, stores of 128 contiguous bytes
+                for (int c = 0; c < hd; c += 32) {
+                    uint32_t o[2][16];
+                    tmem_ld_x16(tO + lane_off + (uint32_t)c, o[0]);
+                    tmem_ld_x16(tO + lane_off + (uint32_t)(c + 16), o[1]);
+                    tmem_ld_wait();
+                    if (r < nq) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4*>(dst + c + j) =
+                                make_float4(__uint_as_float(o[j >> 4][j & 15]), __uint_as_float(o[j >> 4][(j & 15) + 1]),
+                                            __uint_as_float(o[j >> 4][(j & 15) + 2]), __uint_as_float(o[j >> 4][(j & 15) + 3]));
+                    }
                 }
             }
         }
@@ -586,7 +670,8 @@ bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd
     });
     if (!g_enc) return false;
     // 4-D view {64 dims, rows, kv heads, hd / 64 chunks (128 bytes apart)}: one request brings a whole
-    // tile, laid out [chunk][key][64] = nsub K-major sub-tiles of KT rows
+    // tile, laid out [chunk][key][64] = nsub K-major sub-tiles of KT rows (one 32 KB request
+    // measured faster than eight of 8 keys each)
     cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)nKv, (cuuint64_t)(hd / 64)};
     cuuint64_t strides[3] = {(cuuint64_t)nKv * hd * 2, (cuuint64_t)hd * 2, 128};
     cuuint32_t box[4] = {64, (cuuint32_t)KT, 1, (cuuint32_t)(hd / 64)};   // KT <= 256
@@ -598,94 +683,29 @@ bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd
 
 size_t attn_tc_smem(int hd) {
     const int nsub = hd / 64;
-    // K and V (kSlots each), P (2 slots), row maxima, then the barriers (5 kSlots + 12),
-    // the TMEM slot and the abort flag; 1 KB alignment slack
-    return 2 * (size_t)kSlots * nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 8 * (5 * kSlots + 12) + 16 + 1024;
+    // K and V (kSlots each), P (2 slots), the plan scratch, then the barriers
+    // (5 kSlots + 10), the TMEM slot and the abort flag; 1 KB alignment slack
+    return 2 * (size_t)kSlots * nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 8 * (5 * kSlots + 10) + 16 + 1024;
+}
+
+
+// One warp per output row (b, h, i) of the items on more than one CTA (an item
+// on one CTA wrote its output itself).
+constexpr int kMergeWarps = 8;
+__global__ void __launch_bounds__(kMergeWarps * 32) attn_tc_merge_kernel(AttnTcParams P, int rows) {
+    pdl_trigger();
+    pdl_wait();
+    const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);   // ((b * nH) + h) * G + i
+    if (row >= rows) return;
+    const int i = row % P.G, bh = row / P.G;
+    const int b = bh / P.nH, h = bh % P.nH;
+    const int item = b * P.nKv + h / P.grp;
+    const int k = P.item_slots[2 * item + 1];
+    if (k <= 1) return;
+    merge_row(P, P.item_slots[2 * item], k, i * P.grp + h % P.grp, (((int64_t)b * P.G + i) * P.nH + h) * P.hd);
 }
 
 }  // namespace
-
-// One warp per output row (b, h, i): the item's slots item_cta0[item] ..
-// item_cta0[item + 1] - 1, row r = i * grp + h % grp of each; the weights
-// w_s = exp(m_s - M) combine the unnormalised outputs (lane l owns the 4-column
-// groups l, l + 32 of the row). Slots of empty ranges (m = -inf) weigh nothing.
-constexpr int kMergeWarps = 8;
-constexpr int kMergeBatch = 16;      // slots a merge lane loads at once
-__global__ void __launch_bounds__(kMergeWarps * 32) attn_tc_merge_kernel(AttnArgs a, const int* __restrict__ item_cta0,
-                                                                         int G, int nH, int nKv, int hd, int rows) {
-    pdl_trigger();
-    pdl_wait();
-    const int lane = threadIdx.x & 31;
-    const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);   // ((b * nH) + h) * G + i
-    if (row >= rows) return;
-    const int i = row % G, bh = row / G;
-    const int b = bh / nH, h = bh % nH;
-    const int grp = nH / nKv;
-    const int item = b * nKv + h / grp, r = i * grp + h % grp;
-    const int s0 = item_cta0[item], s1 = item_cta0[item + 1];
-    float M = -INFINITY;
-    for (int s = s0 + lane; s < s1; s += 32) M = fmaxf(M, a.part_ml[((int64_t)s * QROWS + r) * 2]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const int ng = hd / 4;
-    float4 num[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-    float den = 0.f;
-    for (int sb = s0; sb < s1; sb += 32) {
-        float ws = 0.f, ls = 0.f;
-        if (sb + lane < s1) {
-            const int64_t base = (int64_t)(sb + lane) * QROWS + r;
-            const float m = a.part_ml[base * 2];
-            ls = a.part_ml[base * 2 + 1];
-            ws = m == -INFINITY ? 0.f : __expf(m - M);
-        }
-        const int cnt = min(32, s1 - sb);
-        // kMergeBatch slots' loads in flight at once, then their weighted sum in slot order
-        for (int t0 = 0; t0 < cnt; t0 += kMergeBatch) {
-            float4 v[kMergeBatch][2];
-#pragma unroll
-            for (int u = 0; u < kMergeBatch; ++u) {
-                const float* o = a.part_o + ((int64_t)(sb + t0 + u) * QROWS + r) * hd;
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int g4 = lane + q * 32;
-                    v[u][q] = (t0 + u < cnt && g4 < ng) ? reinterpret_cast<const float4*>(o)[g4]
-                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kMergeBatch; ++u) {
-                const float w = __shfl_sync(0xffffffffu, ws, (t0 + u) & 31);
-                const float l = __shfl_sync(0xffffffffu, ls, (t0 + u) & 31);
-                if (t0 + u >= cnt) break;
-                den += w * l;
-                if (w == 0.f) continue;                // uniform: an empty range (its O slot is not written)
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    num[q].x += w * v[u][q].x; num[q].y += w * v[u][q].y;
-                    num[q].z += w * v[u][q].z; num[q].w += w * v[u][q].w;
-                }
-            }
-        }
-    }
-    const float inv = 1.f / den;
-    const int64_t ob = (((int64_t)b * G + i) * nH + h) * hd;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const int g4 = lane + q * 32;
-        if (g4 >= ng) continue;
-        const float v[4] = {num[q].x * inv, num[q].y * inv, num[q].z * inv, num[q].w * inv};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int64_t o = ob + g4 * 4 + c;
-            store_any(a.out, o, a.out_dtype, v[c]);
-            if (a.out_hi) {
-                const __half hv = __float2half_rn(v[c]);
-                a.out_hi[o] = hv;
-                if (a.out_lo) a.out_lo[o] = __float2half_rn(v[c] - __half2float(hv));
-            }
-        }
-    }
-}
 
 bool attention_tc_supported(const dspark_model* m) {
     const Dims& d = m->d;
@@ -696,44 +716,36 @@ int attention_tc_key_tile() { return KT; }
 
 int attention_tc_grid(const dspark_model* m, int A) { return std::max(m->num_sms, A * m->d.nKv); }
 
-size_t attention_tc_plan_ints(const dspark_model* m, int A, int grid) {
-    return 3 * (size_t)grid + (size_t)A * m->d.nKv + 1;
-}
+size_t attention_tc_item_ints(const dspark_model* m, int A) { return 2 * (size_t)A * m->d.nKv; }
 
 size_t attention_tc_partial_floats(const dspark_model* m, int grid) { return (size_t)grid * QROWS * (m->d.hd + 2); }
 
 cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaStream_t s) {
     const Dims& d = m->d;
-    if (!a.plan || a.tc_grid < std::max(1, a.A * d.nKv)) return cudaErrorInvalidValue;
+    if (!a.item_slots || a.tc_grid < std::max(1, a.A * d.nKv) || a.q_dtype != DSPARK_DTYPE_F16 ||
+        (a.out_dtype != DSPARK_DTYPE_F32 && a.out_dtype != DSPARK_DTYPE_F16))
+        return cudaErrorInvalidValue;
     CUtensorMap tk, tv, tkb, tvb;
     const int64_t cache_rows = (int64_t)a.batch * a.capacity;   // all rows of this layer's cache
     if (!make_kv_map(&tk, a.kc, cache_rows, d.nKv, d.hd) || !make_kv_map(&tv, a.vc, cache_rows, d.nKv, d.hd) ||
         !make_kv_map(&tkb, a.kb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
         !make_kv_map(&tvb, a.vb, (int64_t)a.A * d.gamma, d.nKv, d.hd))
         return cudaErrorInvalidValue;
-    const int grid = a.tc_grid;
-    int* cta_item = a.plan;
-    int* cta_t0 = cta_item + grid;
-    int* cta_t1 = cta_t0 + grid;
-    int* item_cta0 = cta_t1 + grid;
-    cudaError_t e = cudaSuccess;
-    if (!a.plan_ready)      // the plan depends only on the lengths: a round computes it for its first layer
-        e = launch_pdl(attn_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, a.len, a.A, d.nKv, a.capacity, grid,
-                       cta_item, cta_t0, cta_t1, item_cta0);
-    if (e != cudaSuccess) return e;
     AttnTcParams P{};
     P.A = a.A; P.G = d.gamma; P.nH = d.nH; P.nKv = d.nKv; P.grp = d.grp; P.hd = d.hd; P.capacity = a.capacity;
-    P.q_dtype = a.q_dtype; P.q = a.q; P.len = a.len;
-    P.part_o = a.part_o; P.part_ml = a.part_ml; P.status = a.status;
-    P.cta_item = cta_item; P.cta_t0 = cta_t0; P.cta_t1 = cta_t1;
+    P.q_dtype = a.q_dtype; P.grid = a.tc_grid; P.q = a.q; P.len = a.len;
+    P.part_o = a.part_o; P.part_ml = a.part_ml; P.item_slots = a.item_slots; P.status = a.status;
+    P.out = a.out; P.out_dtype = a.out_dtype; P.out_hi = a.out_hi; P.out_lo = a.out_lo;
     const size_t smem = attn_tc_smem(d.hd);
-    e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attn_tc_kernel, dim3(grid), dim3(kThreads), smem, s, tk, tv, tkb, tvb, P);
+    e = launch_pdl(attn_tc_kernel, dim3(a.tc_grid), dim3(kThreads), smem, s, tk, tv, tkb, tvb, P);
     if (e != cudaSuccess) return e;
+    // with at least as many items as CTAs every item is on one CTA: nothing to merge
+    if (a.A * d.nKv >= a.tc_grid) return cudaSuccess;
     const int rows = a.A * d.nH * d.gamma;
-    return launch_pdl(attn_tc_merge_kernel, dim3((rows + kMergeWarps - 1) / kMergeWarps), dim3(kMergeWarps * 32), 0, s,
-                      a, item_cta0, d.gamma, d.nH, d.nKv, d.hd, rows);
+    return launch_pdl(attn_tc_merge_kernel, dim3((rows + kMergeWarps - 1) / kMergeWarps), dim3(kMergeWarps * 32), 0,
+                      s, P, rows);
 }
 
 }  // namespace tc

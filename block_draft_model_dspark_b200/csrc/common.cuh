@@ -88,8 +88,9 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
 __device__ __forceinline__ void rope_sincos(int pos, double inv_freq, float* s, float* c) {
     if (inv_freq == 0.0) { *s = 0.f; *c = 1.f; return; }
     const double two_pi = 6.283185307179586476925286766559;
+    const double inv_two_pi = 0.15915494309189533576888376337251;
     double a = (double)pos * inv_freq;
-    a -= floor(a / two_pi) * two_pi;
+    a -= floor(a * inv_two_pi) * two_pi;        // within an ulp of [0, 2 pi) either way the turn count rounds
     sincosf((float)a, s, c);
 }
 

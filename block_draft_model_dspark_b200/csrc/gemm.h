@@ -47,7 +47,7 @@ bool attention_tc_supported(const dspark_model* m);
 // Tensor-core attention: CTAs of a call for A rows, ints of its work plan and floats of its
 // per-CTA partial state (one slot of 128 rows x (head_dim + 2) per CTA).
 int attention_tc_grid(const dspark_model* m, int A);
-size_t attention_tc_plan_ints(const dspark_model* m, int A, int grid);
+size_t attention_tc_item_ints(const dspark_model* m, int A);
 size_t attention_tc_partial_floats(const dspark_model* m, int grid);
 }  // namespace tc
 

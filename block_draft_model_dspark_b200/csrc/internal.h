@@ -243,9 +243,9 @@ cudaError_t launch_commit_len(int32_t* len, const int32_t* n_new, int B, cudaStr
 // Block embedding: h = embed[ids]*sqrt(H) (fp32 [M,H]); x = rms(h, w_in0) (fp32 [M,H]).
 cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, float* h, const ActBuf& x,
                          int32_t* status, cudaStream_t s);
-// q (fp32) and block k/v (model dtype) heads from the [Wq;Wk] GEMM partials.
+// q and block k/v heads (all in the KV dtype) from the [Wq;Wk] GEMM partials.
 cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const PartView& part, int A,
-                               const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s);
+                               const int32_t* block_pos, void* q, void* kb, void* vb, cudaStream_t s);
 // h += rms(o_proj partials, post_attn); x = rms(h, pre_ff).
 cudaError_t launch_o_epilogue(const dspark_model* m, int layer, const PartView& part, int M, float* h,
                               const ActBuf& x, cudaStream_t s);
@@ -266,8 +266,7 @@ struct AttnArgs {
     void* out;                                       // [A, G, nH, hd]
     __half* out_hi; __half* out_lo;                  // optional fp16 form of out (fp32 out only; lo may be NULL)
     float* part_o; float* part_ml;                   // workspace
-    int* plan; int tc_grid;                          // tensor cores: the work plan's ints and the CTAs
-    bool plan_ready;                                 // the plan was computed for these lengths already
+    int* item_slots; int tc_grid;                    // tensor cores: per-item (first slot, slots) and the CTAs
     int A, n_splits, chunk;                          // CUDA cores: context splits of `chunk` keys
     int S1;                                          // partial slots per (b, h): set by the kernel path
     int32_t* status;

@@ -167,63 +167,67 @@ __global__ void __launch_bounds__(512) embed_kernel(MatRef E, int dtype, int gro
 }
 
 // ------------------------------------------------------------------ q / k / v heads
-// grid (M, ceil((nH + nKv) / 4)), block 128: one warp per head; lane l owns the
-// RoPE pairs (i, i + hd/2) for i = l, l + 32, ... < hd/2.
-constexpr int kQkHeadsPerCta = 4;
+// grid (M), block kQkWarps warps: the row's RoPE angles (hd/2 of them, one
+// position) are computed once into shared memory, then one warp per head (heads
+// warp, warp + kQkWarps, ...); lane l owns the RoPE pairs (i, i + hd/2) for
+// i = l, l + 32, ... < hd/2.
+constexpr int kQkWarps = 8;
 constexpr int kQkMaxPairs = 4;                // hd/2 / 32 for hd <= 256
-__global__ void __launch_bounds__(32 * kQkHeadsPerCta)
+__global__ void __launch_bounds__(32 * kQkWarps)
 qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, int hd, const int32_t* __restrict__ block_pos,
                    const double* __restrict__ inv_freq, const void* __restrict__ q_norm,
-                   const void* __restrict__ k_norm, float eps, int dtype, int kv_dtype, float* __restrict__ q,
+                   const void* __restrict__ k_norm, float eps, int dtype, int kv_dtype, void* __restrict__ q,
                    void* __restrict__ kb, void* __restrict__ vb) {
+    __shared__ float s_sin[128], s_cos[128];
     pdl_trigger();
     pdl_wait();
-    const int m = blockIdx.x, lane = threadIdx.x & 31;
-    const int hh = blockIdx.y * kQkHeadsPerCta + (threadIdx.x >> 5);
-    if (hh >= nH + nKv) return;
+    const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int b = m / gamma, t = m % gamma;
     const int pos = block_pos[b] + t;
     const int half = hd / 2, np = half / 32;      // pairs per lane
-    const int64_t col = (int64_t)hh * hd;
-    PartView::Pending p1[kQkMaxPairs], p2[kQkMaxPairs];
+    for (int i = threadIdx.x; i < half; i += blockDim.x) rope_sincos(pos, inv_freq[i], &s_sin[i], &s_cos[i]);
+    __syncthreads();
+    for (int hh = warp; hh < nH + nKv; hh += kQkWarps) {
+        const int64_t col = (int64_t)hh * hd;
+        PartView::Pending p1[kQkMaxPairs], p2[kQkMaxPairs];
 #pragma unroll
-    for (int e = 0; e < kQkMaxPairs; ++e) {
-        if (e < np) {
-            p1[e] = part.load(m, col + lane + 32 * e);
-            p2[e] = part.load(m, col + lane + 32 * e + half);
+        for (int e = 0; e < kQkMaxPairs; ++e) {
+            if (e < np) {
+                p1[e] = part.load(m, col + lane + 32 * e);
+                p2[e] = part.load(m, col + lane + 32 * e + half);
+            }
         }
-    }
-    float x1[kQkMaxPairs], x2[kQkMaxPairs];
-    float ss = 0.f;
+        float x1[kQkMaxPairs], x2[kQkMaxPairs];
+        float ss = 0.f;
 #pragma unroll
-    for (int e = 0; e < kQkMaxPairs; ++e) {
-        x1[e] = e < np ? part.finish(p1[e]) : 0.f;
-        x2[e] = e < np ? part.finish(p2[e]) : 0.f;
-        ss += x1[e] * x1[e] + x2[e] * x2[e];
-    }
-    ss = warp_sum(ss);
-    const float rinv = rsqrtf(ss / (float)hd + eps);
+        for (int e = 0; e < kQkMaxPairs; ++e) {
+            x1[e] = e < np ? part.finish(p1[e]) : 0.f;
+            x2[e] = e < np ? part.finish(p2[e]) : 0.f;
+            ss += x1[e] * x1[e] + x2[e] * x2[e];
+        }
+        ss = warp_sum(ss);
+        const float rinv = rsqrtf(ss / (float)hd + eps);
 #pragma unroll
-    for (int e = 0; e < kQkMaxPairs; ++e) {
-        if (e >= np) break;
-        const int i = lane + 32 * e;
-        float y1 = x1[e] * rinv, y2 = x2[e] * rinv;
-        float sn, cs;
-        rope_sincos(pos, inv_freq[i], &sn, &cs);
-        if (hh < nH) {
-            y1 *= load_any(q_norm, i, dtype);
-            y2 *= load_any(q_norm, i + half, dtype);
-            const int64_t o = ((int64_t)m * nH + hh) * hd;
-            q[o + i] = y1 * cs - y2 * sn;
-            q[o + i + half] = y2 * cs + y1 * sn;
-        } else {
-            const int g = hh - nH;
-            const int64_t o = ((int64_t)m * nKv + g) * hd;
-            store_any(vb, o + i, kv_dtype, y1);
-            store_any(vb, o + i + half, kv_dtype, y2);
-            const float k1 = y1 * load_any(k_norm, i, dtype), k2 = y2 * load_any(k_norm, i + half, dtype);
-            store_any(kb, o + i, kv_dtype, k1 * cs - k2 * sn);
-            store_any(kb, o + i + half, kv_dtype, k2 * cs + k1 * sn);
+        for (int e = 0; e < kQkMaxPairs; ++e) {
+            if (e >= np) break;
+            const int i = lane + 32 * e;
+            float y1 = x1[e] * rinv, y2 = x2[e] * rinv;
+            const float sn = s_sin[i], cs = s_cos[i];
+            if (hh < nH) {
+                y1 *= load_any(q_norm, i, dtype);
+                y2 *= load_any(q_norm, i + half, dtype);
+                const int64_t o = ((int64_t)m * nH + hh) * hd;
+                store_any(q, o + i, kv_dtype, y1 * cs - y2 * sn);          // the attention's query type
+                store_any(q, o + i + half, kv_dtype, y2 * cs + y1 * sn);
+            } else {
+                const int g = hh - nH;
+                const int64_t o = ((int64_t)m * nKv + g) * hd;
+                store_any(vb, o + i, kv_dtype, y1);
+                store_any(vb, o + i + half, kv_dtype, y2);
+                const float k1 = y1 * load_any(k_norm, i, dtype), k2 = y2 * load_any(k_norm, i + half, dtype);
+                store_any(kb, o + i, kv_dtype, k1 * cs - k2 * sn);
+                store_any(kb, o + i + half, kv_dtype, k2 * cs + k1 * sn);
+            }
         }
     }
 }
@@ -457,11 +461,10 @@ cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, f
 }
 
 cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const PartView& part, int A,
-                               const int32_t* block_pos, float* q, void* kb, void* vb, cudaStream_t s) {
+                               const int32_t* block_pos, void* q, void* kb, void* vb, cudaStream_t s) {
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
-    dim3 grid(A * d.gamma, (d.nH + d.nKv + kQkHeadsPerCta - 1) / kQkHeadsPerCta);
-    return launch_pdl(qk_epilogue_kernel, grid, dim3(32 * kQkHeadsPerCta), 0, s, part, d.gamma, d.nH, d.nKv, d.hd,
+    return launch_pdl(qk_epilogue_kernel, dim3(A * d.gamma), dim3(32 * kQkWarps), 0, s, part, d.gamma, d.nH, d.nKv, d.hd,
                       block_pos, m->ws.inv_freq, m->layers[layer].q_norm, m->layers[layer].k_norm, d.eps, d.dtype,
                       d.kv_dtype, q, kb, vb);
 }

@@ -180,10 +180,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 // with the 128-byte swizzle: rows of 128 bytes (64 bf16), 8-row groups 1024
 // bytes apart. The tile must start on a 1024-byte boundary; advancing the
 // start address by 32 bytes selects the next 16-element K slice.
-__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t smem_addr) {
+__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t smem_addr, uint32_t sbo = 1024) {
     return (uint64_t)((smem_addr >> 4) & 0x3FFFu)   // start address
            | ((uint64_t)1 << 16)                     // leading byte offset (unused for swizzled K-major)
-           | ((uint64_t)(1024 >> 4) << 32)           // stride byte offset: 8 rows x 128 B
+           | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32)  // stride byte offset: between groups of 8 rows x 128 B
            | ((uint64_t)1 << 46)                     // descriptor version (sm_100)
            | ((uint64_t)2 << 61);                    // layout: 128-byte swizzle
 }
@@ -223,10 +223,10 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int b_mn_major) {
 // Descriptor of an MN-major operand laid out by TMA with the 128-byte swizzle:
 // 64-element (128-byte) rows along N, one row per K index, 8-row groups 1024
 // bytes apart (stride byte offset); successive 64-element N chunks `lbo` bytes apart.
-__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t smem_addr, uint32_t lbo) {
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo = 1024) {
     return (uint64_t)((smem_addr >> 4) & 0x3FFFu)
            | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16)
-           | ((uint64_t)(1024 >> 4) << 32)
+           | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32)
            | ((uint64_t)1 << 46)
            | ((uint64_t)2 << 61);
 }

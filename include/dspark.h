@@ -269,6 +269,8 @@ int dspark_draft_rows(const dspark_model* model, const dspark_kv_cache* cache,
  * non-causal, scale 1.0, softmax in fp32.
  *   q   device KV [A, gamma, nH, hd]    k_blk, v_blk device KV [A, gamma, nKv, hd]
  *   out device KV [A, gamma, nH, hd]      (KV: dspark_kv_dtype)
+ * q, k_blk, v_blk, out and ws must be 16-byte aligned (DSPARK_ERR_INVALID_ARGUMENT
+ * otherwise, before any launch); the same holds for dspark_attend_no_alloc.
  */
 int dspark_attend(const dspark_model* model, int32_t layer, const dspark_kv_cache* cache,
                   const void* q, const void* k_blk, const void* v_blk, void* out,
@@ -283,7 +285,7 @@ int dspark_attend(const dspark_model* model, int32_t layer, const dspark_kv_cach
  * must not call cudaMalloc (which may synchronise the device). The pages have
  * no counterpart to this entry point.
  * Its scratch (the per-split softmax state and, for a bf16 model, the
- * work plan) is a 16 MiB static device array inside libdspark, allocated on
+ * per-item slot records) is a 16 MiB static device array inside libdspark, allocated on
  * every GPU that loads the library and held until the process exits. A bf16
  * model's call uses at most as many CTAs as that array holds partial states
  * of 128 x (hd + 2) floats (at hd = 256, 126; fewer CTAs only lengthen the

@@ -126,6 +126,73 @@ def test_attend_matches_concat_sdpa(dtype):
             assert_close(out[b].float().cpu().numpy(), ref, dtype, f"attend layer {layer} row {b}")
 
 
+@pytest.mark.parametrize("slope", [0.25, -0.25])
+def test_attend_rising_and_falling_logits(slope):
+    """Logits that rise along the keys by 16 per 64-key tile (every tile raises the
+    running maximum past the kernel's rescale headroom, so the output state is
+    rescaled at every tile, and the block's keys rise further), and the mirror case
+    (the first tile holds the maximum: never rescaled). q . k_j = slope * j exactly
+    in fp16 (k_j = j / 16 in head dimension 0, q = 4 slope there)."""
+    import block_draft_model_dspark_b200 as dsp
+    m = small_model(dtype="bf16", block_size=8)
+    cpu, W, model = build(m, 5)
+    tdt = model.kv_torch_dtype
+    A, G, nH, nKv, hd = 3, m.block_size, m.num_attention_heads, m.num_global_key_value_heads, m.global_head_dim
+    lens = [1000, 64, 7]
+    cap = 1000
+    g = torch.Generator().manual_seed(17)
+    cache = dsp.KvCache(model, A, cap)
+    k = torch.zeros(cache.k.shape)
+    v = torch.randn(cache.v.shape, generator=g)
+    for b in range(A):
+        k[:, b, :, :, 0] = (torch.arange(cap, dtype=torch.float32) / 16.0)[None, :, None]
+    cache.k.copy_(k.to(tdt))
+    cache.v.copy_(v.to(tdt))
+    cache.set_lengths(lens)
+    q = torch.zeros(A, G, nH, hd)
+    q[..., 0] = 4.0 * slope
+    kb = torch.zeros(A, G, nKv, hd)
+    for b in range(A):
+        kb[b, :, :, 0] = ((lens[b] + torch.arange(G, dtype=torch.float32)) / 16.0)[:, None]
+    vb = torch.randn(A, G, nKv, hd, generator=g)
+    q, kb, vb = q.to(tdt), kb.to(tdt), vb.to(tdt)
+    out = torch.empty(A, G, nH, hd, dtype=tdt, device="cuda")
+    model.dspark_attend(0, cache, q.cuda(), kb.cuda(), vb.cuda(), out, max(lens))
+    torch.cuda.synchronize()
+    assert model.dspark_read_device_status() == 0
+    kc, vc = cache.k[0].float().cpu().numpy(), cache.v[0].float().cpu().numpy()
+    for b in range(A):
+        ref = O.attend_concat(q[b].double().numpy(), kc[b, :lens[b]], vc[b, :lens[b]], kb[b].double().numpy(),
+                              vb[b].double().numpy())
+        assert_close(out[b].float().cpu().numpy(), ref, "bf16", f"attend slope {slope} row {b}")
+
+
+def test_attend_refuses_misaligned_buffers():
+    """The seam's vector loads and stores need 16-byte aligned q, k_blk, v_blk and
+    out: both entry points refuse a misaligned one before any launch."""
+    import block_draft_model_dspark_b200 as dsp
+    m = small_model(dtype="bf16", block_size=8)
+    cpu, W, model = build(m, 5)
+    tdt = model.kv_torch_dtype
+    A, G, nH, nKv, hd = 2, m.block_size, m.num_attention_heads, m.num_global_key_value_heads, m.global_head_dim
+    cache = dsp.KvCache(model, A, 64)
+    cache.k.zero_(); cache.v.zero_()
+    cache.set_lengths([10, 64])
+    q = torch.zeros(A, G, nH, hd, dtype=tdt, device="cuda")
+    kb = torch.zeros(A, G, nKv, hd, dtype=tdt, device="cuda")
+    vb = torch.zeros_like(kb)
+    n = A * G * nH * hd
+    flat = torch.zeros(n + 8, dtype=tdt, device="cuda")
+    bad = flat[1:1 + n].view(A, G, nH, hd)                 # 2 bytes past a 256-byte boundary
+    for call in (model.dspark_attend, model.dspark_attend_no_alloc):
+        for args in ((bad, kb, vb, q.clone()), (q, kb, vb, bad)):
+            with pytest.raises(dsp.DsparkError) as ei:
+                call(0, cache, *args, 64)
+            assert ei.value.code == dsp.DSPARK_ERR_INVALID_ARGUMENT
+    torch.cuda.synchronize()
+    assert model.dspark_read_device_status() == 0
+
+
 # ----------------------------------------------------------------------------- whole rounds, small models
 
 @pytest.mark.parametrize("quant", [0, 4])
