@@ -109,33 +109,61 @@ struct CtaWork {
     int t0, t1;      // tile range within the item
     int s0, k;       // the item's first CTA (slot) and its number of CTAs
 };
-// This CTA's share of the plan, by all threads of the block (every CTA
-// computes the same plan). `sh` holds 2 kWarps + 5 ints of shared memory.
+// ceil(n / q) for 0 <= n, 1 <= q below 2^20, from a float reciprocal of q
+// (off by at most one before the correction).
+__device__ __forceinline__ int ceil_div_small(int n, int q, float rq) {
+    const int a = n + q - 1;
+    int c = __float2int_rz((float)a * rq);
+    if (c * q > a) --c;
+    else if ((c + 1) * q <= a) ++c;
+    return c;
+}
+// This CTA's share of the plan, by all threads of the block (every CTA computes
+// the same plan). Items (b, g) of one row b have the same n_b, so the plan works
+// on rows: n_b cached in `ncache` (A ints of shared memory), the smallest
+// feasible q found by testing up to kThreads candidates at once (each thread
+// sums nKv * ceil(n_b / q) over the rows for its candidate; two rounds at most
+// for n up to kThreads^2), then a scan of k_b over the rows places the CTA.
+// `sh` holds 2 kWarps + 5 ints.
 __device__ CtaWork cta_work(const int32_t* __restrict__ len, int A, int nKv, int capacity, int grid, int slot,
-                            int* sh) {
+                            int* sh, int* ncache) {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int n_items = A * nKv;
     int* res = sh + 2 * kWarps;                      // item, index within the item, n, k, first slot
-    if (tid == 0) res[0] = -1;                       // ordered before the scan by the reductions' barriers
+    if (tid == 0) res[0] = -1;                       // ordered before the scan by the barriers below
     int nb = 0;
     int mx = 1;
-    for (int i = tid; i < n_items; i += kThreads) mx = max(mx, plan_tiles(len, i / nKv, capacity));
-    mx = block_reduce_int(mx, sh + (nb++ & 1) * kWarps, true);
-    int lo = min(2, mx), hi = mx;
-    while (lo < hi) {
-        const int mid = (lo + hi) / 2;
-        int cnt = 0;
-        for (int i = tid; i < n_items; i += kThreads) cnt += (plan_tiles(len, i / nKv, capacity) + mid - 1) / mid;
-        cnt = block_reduce_int(cnt, sh + (nb++ & 1) * kWarps, false);
-        if (cnt <= grid) hi = mid; else lo = mid + 1;
+    for (int b = tid; b < A; b += kThreads) {
+        const int n = plan_tiles(len, b, capacity);
+        ncache[b] = n;
+        mx = max(mx, n);
     }
-    const int q = lo;
-    int base = 0;                                    // CTAs of the items before this chunk
-    for (int i0 = 0; i0 < n_items; i0 += kThreads) {
-        const int i = i0 + tid;
-        const int n = i < n_items ? plan_tiles(len, i / nKv, capacity) : 0;
-        const int k = i < n_items ? (n + q - 1) / q : 0;
-        int x = k;                                   // inclusive scan within the warp
+    mx = block_reduce_int(mx, sh + (nb++ & 1) * kWarps, true);   // also publishes ncache
+    int q = mx;                                      // q = mx is feasible: A * nKv <= grid
+    if (A * nKv < grid) {
+        int lo = min(2, mx), hi = mx;                // the answer lies in [lo, hi]; hi is feasible
+        while (lo < hi) {
+            const int step = (hi - lo + kThreads - 1) / kThreads;
+            const int cand = lo + tid * step;
+            int best = hi;
+            if (cand < hi) {
+                const float rq = 1.f / (float)cand;
+                int cnt = 0;
+                for (int b = 0; b < A; ++b) cnt += ceil_div_small(ncache[b], cand, rq);
+                if ((int64_t)cnt * nKv <= grid) best = cand;
+            }
+            // the smallest feasible candidate; the answer is in (best - step, best]
+            best = -block_reduce_int(-best, sh + (nb++ & 1) * kWarps, true);
+            hi = best;
+            lo = max(lo, best - step + 1);
+        }
+        q = hi;
+    }
+    int base = 0;                                    // CTAs of the rows before this chunk
+    for (int b0 = 0; b0 < A; b0 += kThreads) {
+        const int b = b0 + tid;
+        const int n = b < A ? ncache[b] : 0;
+        const int k = b < A ? (n + q - 1) / q : 0;
+        int x = k * nKv;                             // inclusive scan of the rows' CTAs within the warp
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -149,9 +177,10 @@ __device__ CtaWork cta_work(const int32_t* __restrict__ len, int A, int nKv, int
             if (w < wid) wbase += wb[w];
             tot += wb[w];
         }
-        const int excl = base + wbase + x - k;
-        if (i < n_items && slot >= excl && slot < excl + k) {
-            res[0] = i; res[1] = slot - excl; res[2] = n; res[3] = k; res[4] = excl;
+        const int first = base + wbase + x - k * nKv;   // the row's first CTA
+        if (b < A && slot >= first && slot < first + k * nKv) {
+            const int rel = slot - first, g = rel / k;
+            res[0] = b * nKv + g; res[1] = rel - g * k; res[2] = n; res[3] = k; res[4] = first + g * k;
         }
         base += tot;                                 // the same in every thread
         if (base > slot) break;
@@ -289,7 +318,8 @@ __device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, v
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb, AttnTcParams P) {
+               const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
+               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmQ, AttnTcParams P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int hd = P.hd, nsub = hd / 64;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -310,7 +340,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     uint64_t* odone = pready + 2;              // [2] P V product of the tile in that P slot done (O settled)
     uint64_t* spare = odone + 2;               // teardown: MMAs in flight after an abort
     uint64_t* spare2 = spare + 1;              // teardown of the P V issuer
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(spare2 + 1);
+    uint64_t* qfull = spare2 + 1;              // the query tile landed in shared memory (TMA)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -325,9 +356,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         mbar_init(&sfree[0], kSoftThreads); mbar_init(&sfree[1], kSoftThreads);
         mbar_init(&pready[0], kSoftThreads); mbar_init(&pready[1], kSoftThreads);
         mbar_init(&odone[0], 1); mbar_init(&odone[1], 1); mbar_init(spare, 1); mbar_init(spare2, 1);
+        mbar_init(qfull, 1);
         *abort_flag = 0;
         mbar_fence_init();
-        prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmKb); prefetch_tmap(&tmVb);
+        prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmKb); prefetch_tmap(&tmVb); prefetch_tmap(&tmO);
+        prefetch_tmap(&tmQ);
     }
     if (warp == kIssuerWarp) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
@@ -340,7 +373,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 
     // this CTA's work: tiles [t_lo, t_hi) of item (b, g); an idle CTA has none
     const int slot = blockIdx.x;
-    const CtaWork W = cta_work(P.len, P.A, P.nKv, P.capacity, P.grid, slot, red);
+    const CtaWork W = cta_work(P.len, P.A, P.nKv, P.capacity, P.grid, slot, red, reinterpret_cast<int*>(sK));
     const int item = W.item;
     const int b = item >= 0 ? item / P.nKv : 0, g = item >= 0 ? item % P.nKv : 0;
     const int t_lo = W.t0, t_hi = W.t1;
@@ -358,12 +391,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         else { *row = b * P.G; *nvalid = P.G; *blk = true; }
     };
 
+    // Q tile in tensor memory (the S product's A operand): TMEM lane r holds query
+    // row r, two fp16 values per 32-bit column from column kQCol; rows past the
+    // queries are zero. The tile comes by TMA, one request per 64 head dimensions
+    // ([nq rows x 128 B], 128-byte swizzle), into V slots 1 and 2 (free until it is
+    // in tensor memory; their V tiles are requested after it), while K tiles 0..2
+    // and V tile 0 load. Softmax thread r then copies its row to tensor memory.
     const uint32_t tile_bytes = (uint32_t)nsub * KT * 128;
-    // The first kSlots K and V tiles do not depend on Q: their loads go out
-    // before the Q tile is built, so they land while it is.
+    uint8_t* sQ = sV + tile_sz;                           // nsub x [nq rows x 128 B] <= 2 tiles
+    const int qstride = (nq * 128 + 1023) & ~1023;        // chunks 1 KB aligned (the swizzle's period)
+    if (warp == kIssuerWarp && lane == 0 && item >= 0) {
+        mbar_arrive_expect_tx(qfull, (uint32_t)(nsub * nq * 128));
+        for (int c = 0; c < nsub; ++c) tma_load_5d(sQ + c * qstride, &tmQ, qfull, 0, 0, g, b * P.G, c);
+    }
     if ((warp == kIssuerWarp || warp == kIssuerWarp + 1) && lane == 0) {
         const bool v_tile = warp != kIssuerWarp;
-        for (int t = 0; t < kSlots && t < nt; ++t) {
+        for (int t = 0; t < (v_tile ? 1 : kSlots) && t < nt; ++t) {
             int row, nvalid; bool blk;
             tile_rows(t, &row, &nvalid, &blk);
             const CUtensorMap* m = blk ? (v_tile ? &tmVb : &tmKb) : (v_tile ? &tmV : &tmK);
@@ -372,41 +415,41 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             tma_load_4d((v_tile ? sV : sK) + t * tile_sz, m, bar, 0, row, g, 0);
         }
     }
-
-    // Q tile in tensor memory (the S product's A operand): TMEM lane r holds query
-    // row r, two fp16 values per 32-bit column from column kQCol; rows past the
-    // queries are zero. The softmax threads write it, thread (r, half) the row's
-    // half of the head dimensions, 16 columns per tcgen05.st.
+    bool ok = true;
     if (tid < kSoftThreads) {
-        // fp16 queries: thread r writes row r, hd / 8 contiguous 16-byte chunks (4 columns
-        // each), loaded 16 at a time before their stores
         const int r = tid;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int i = r / P.grp, h = g * P.grp + r % P.grp;
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(P.q) +
-                                                          (((int64_t)b * P.G + i) * P.nH + h) * hd);
-        const int n16 = hd / 8;                               // 16-byte chunks of the row (<= 32)
-        for (int cb = 0; cb < n16; cb += 16) {
-            uint4 u[16];
+        if (item >= 0 && !warp_wait(qfull, 0u, abort_flag, P.status)) ok = false;
+        for (int c = 0; c < nsub; ++c) {
+            const uint8_t* line = sQ + c * qstride + r * 128;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) u[c] = (cb + c < n16 && r < nq) ? src[cb + c] : make_uint4(0u, 0u, 0u, 0u);
+            for (int j0 = 0; j0 < 8; j0 += 4) {               // 4 pieces of 16 bytes = 16 columns per tcgen05.st
+                uint32_t w[16];
 #pragma unroll
-            for (int c0 = 0; c0 < 16; c0 += 4) {              // 4 chunks = 16 columns per tcgen05.st
-                if (cb + c0 >= n16) break;
-                const uint32_t w[16] = {u[c0].x, u[c0].y, u[c0].z, u[c0].w, u[c0 + 1].x, u[c0 + 1].y, u[c0 + 1].z,
-                                        u[c0 + 1].w, u[c0 + 2].x, u[c0 + 2].y, u[c0 + 2].z, u[c0 + 2].w,
-                                        u[c0 + 3].x, u[c0 + 3].y, u[c0 + 3].z, u[c0 + 3].w};
-                tmem_st_x16(tmem + (uint32_t)(kQCol + 4 * (cb + c0)) + lane_off, w);
+                for (int j = 0; j < 4; ++j) {
+                    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < nq && ok) u = *reinterpret_cast<const uint4*>(line + (((j0 + j) ^ (r & 7)) * 16));
+                    w[4 * j] = u.x; w[4 * j + 1] = u.y; w[4 * j + 2] = u.z; w[4 * j + 3] = u.w;
+                }
+                tmem_st_x16(tmem + (uint32_t)(kQCol + c * 32 + j0 * 4) + lane_off, w);
             }
         }
         tmem_st_wait();
+        fence_async_shared();                             // reads done before V tiles 1, 2 overwrite the area
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (warp == kIssuerWarp + 1 && lane == 0) {
+        for (int t = 1; t < kSlots && t < nt; ++t) {
+            int row, nvalid; bool blk;
+            tile_rows(t, &row, &nvalid, &blk);
+            mbar_arrive_expect_tx(&vfull[t], tile_bytes);
+            tma_load_4d(sV + t * tile_sz, blk ? &tmVb : &tmV, &vfull[t], 0, row, g, 0);
+        }
+    }
 
     const uint32_t tO = tmem + 2 * KT;                    // O: columns [128, 128 + hd); S buffers at 0 and 64
-    bool ok = true;
 
     if (warp == kIssuerWarp || warp == kIssuerWarp + 1) {
         // ------------------------------------------------------------ issuers
@@ -631,22 +674,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 P.part_ml[prow * 2] = any ? m_run : -INFINITY;
                 P.part_ml[prow * 2 + 1] = any ? l_run : 0.f;
             }
-            if (any && ok) {
-                float* dst = P.part_o + ((int64_t)slot * QROWS + r) * hd;
-                // 32 columns per TMEM wait: half the waits, stores of 128 contiguous bytes
+            // The unnormalised O goes through shared memory (the K / V slots are free:
+            // every product has completed): hd / 32 slices of [128 rows x 128 B], 16-byte
+            // chunks swizzled by row (the 128-byte TMA swizzle), then one TMA store per
+            // slice writes whole 128-byte lines instead of scattered 16-byte pieces.
+            const bool stage_ok = any && ok;
+            if (stage_ok) {
                 for (int c = 0; c < hd; c += 32) {
                     uint32_t o[2][16];
                     tmem_ld_x16(tO + lane_off + (uint32_t)c, o[0]);
                     tmem_ld_x16(tO + lane_off + (uint32_t)(c + 16), o[1]);
                     tmem_ld_wait();
-                    if (r < nq) {
+                    uint8_t* line = sK + (c / 32) * (QROWS * 128) + r * 128;
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<float4*>(dst + c + j) =
-                                make_float4(__uint_as_float(o[j >> 4][j & 15]), __uint_as_float(o[j >> 4][(j & 15) + 1]),
-                                            __uint_as_float(o[j >> 4][(j & 15) + 2]), __uint_as_float(o[j >> 4][(j & 15) + 3]));
-                    }
+                    for (int j4 = 0; j4 < 8; ++j4)
+                        *reinterpret_cast<uint4*>(line + ((j4 ^ (r & 7)) * 16)) =
+                            make_uint4(o[j4 >> 2][(j4 & 3) * 4], o[j4 >> 2][(j4 & 3) * 4 + 1],
+                                       o[j4 >> 2][(j4 & 3) * 4 + 2], o[j4 >> 2][(j4 & 3) * 4 + 3]);
                 }
+                fence_async_shared();                         // visible to the TMA
+            }
+            named_barrier_sync(2, kSoftThreads);
+            if (tid == 0 && stage_ok) {
+                for (int c = 0; c < hd; c += 32) tma_store_2d(&tmO, sK + (c / 32) * (QROWS * 128), c, slot * QROWS);
+                bulk_commit_group();
+                bulk_wait_all();                              // written before this CTA's shared memory goes
             }
         }
     }
@@ -681,11 +733,39 @@ bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Map over the partial outputs [rows = CTAs x 128][hd] fp32: boxes of 32 columns
+// (128 bytes, 128-byte swizzle) x 128 rows, for the TMA stores of the epilogue.
+bool make_part_map(CUtensorMap* tm, float* ptr, int64_t rows, int hd) {
+    if (!g_enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)hd, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)hd * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)QROWS};
+    cuuint32_t estr[2] = {1, 1};
+    return g_enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// Map over the queries [A * G][nKv][grp][hd] (fp16) with the head dimension split
+// into 64-element chunks: 5-D view {64 dims, grp heads, nKv, A * G rows, hd / 64
+// chunks}; a box is one chunk of one item's query tile, [G][grp][64] = [nq rows x
+// 128 B] with the 128-byte swizzle (query row r = i * grp + head-in-group).
+bool make_q_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int grp, int G, int hd) {
+    if (!g_enc) return false;
+    cuuint64_t dims[5] = {64, (cuuint64_t)grp, (cuuint64_t)nKv, (cuuint64_t)rows, (cuuint64_t)(hd / 64)};
+    cuuint64_t strides[4] = {(cuuint64_t)hd * 2, (cuuint64_t)grp * hd * 2, (cuuint64_t)nKv * grp * hd * 2, 128};
+    cuuint32_t box[5] = {64, (cuuint32_t)grp, 1, (cuuint32_t)G, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return g_enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t attn_tc_smem(int hd) {
     const int nsub = hd / 64;
     // K and V (kSlots each), P (2 slots), the plan scratch, then the barriers
-    // (5 kSlots + 10), the TMEM slot and the abort flag; 1 KB alignment slack
-    return 2 * (size_t)kSlots * nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 8 * (5 * kSlots + 10) + 16 + 1024;
+    // (5 kSlots + 11), the TMEM slot and the abort flag; 1 KB alignment slack
+    return 2 * (size_t)kSlots * nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 8 * (5 * kSlots + 11) + 16 + 1024;
 }
 
 
@@ -725,11 +805,13 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
     if (!a.item_slots || a.tc_grid < std::max(1, a.A * d.nKv) || a.q_dtype != DSPARK_DTYPE_F16 ||
         (a.out_dtype != DSPARK_DTYPE_F32 && a.out_dtype != DSPARK_DTYPE_F16))
         return cudaErrorInvalidValue;
-    CUtensorMap tk, tv, tkb, tvb;
+    CUtensorMap tk, tv, tkb, tvb, to, tq;
     const int64_t cache_rows = (int64_t)a.batch * a.capacity;   // all rows of this layer's cache
     if (!make_kv_map(&tk, a.kc, cache_rows, d.nKv, d.hd) || !make_kv_map(&tv, a.vc, cache_rows, d.nKv, d.hd) ||
         !make_kv_map(&tkb, a.kb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
-        !make_kv_map(&tvb, a.vb, (int64_t)a.A * d.gamma, d.nKv, d.hd))
+        !make_kv_map(&tvb, a.vb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
+        !make_part_map(&to, a.part_o, (int64_t)a.tc_grid * QROWS, d.hd) ||
+        !make_q_map(&tq, a.q, (int64_t)a.A * d.gamma, d.nKv, d.grp, d.gamma, d.hd))
         return cudaErrorInvalidValue;
     AttnTcParams P{};
     P.A = a.A; P.G = d.gamma; P.nH = d.nH; P.nKv = d.nKv; P.grp = d.grp; P.hd = d.hd; P.capacity = a.capacity;
@@ -739,7 +821,7 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
     const size_t smem = attn_tc_smem(d.hd);
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attn_tc_kernel, dim3(a.tc_grid), dim3(kThreads), smem, s, tk, tv, tkb, tvb, P);
+    e = launch_pdl(attn_tc_kernel, dim3(a.tc_grid), dim3(kThreads), smem, s, tk, tv, tkb, tvb, to, tq, P);
     if (e != cudaSuccess) return e;
     // with at least as many items as CTAs every item is on one CTA: nothing to merge
     if (a.A * d.nKv >= a.tc_grid) return cudaSuccess;

@@ -167,11 +167,11 @@ __global__ void __launch_bounds__(512) embed_kernel(MatRef E, int dtype, int gro
 }
 
 // ------------------------------------------------------------------ q / k / v heads
-// grid (M), block kQkWarps warps: the row's RoPE angles (hd/2 of them, one
-// position) are computed once into shared memory, then one warp per head (heads
-// warp, warp + kQkWarps, ...); lane l owns the RoPE pairs (i, i + hd/2) for
+// grid (M, ceil((nH + nKv) / kQkWarps)), block kQkWarps warps: the row's RoPE
+// angles (hd/2 of them, one position) go into shared memory first, one per
+// thread, then one warp per head; lane l owns the RoPE pairs (i, i + hd/2) for
 // i = l, l + 32, ... < hd/2.
-constexpr int kQkWarps = 8;
+constexpr int kQkWarps = 4;
 constexpr int kQkMaxPairs = 4;                // hd/2 / 32 for hd <= 256
 __global__ void __launch_bounds__(32 * kQkWarps)
 qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, int hd, const int32_t* __restrict__ block_pos,
@@ -187,7 +187,9 @@ qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, int hd, const int3
     const int half = hd / 2, np = half / 32;      // pairs per lane
     for (int i = threadIdx.x; i < half; i += blockDim.x) rope_sincos(pos, inv_freq[i], &s_sin[i], &s_cos[i]);
     __syncthreads();
-    for (int hh = warp; hh < nH + nKv; hh += kQkWarps) {
+    {
+        const int hh = blockIdx.y * kQkWarps + warp;
+        if (hh >= nH + nKv) return;
         const int64_t col = (int64_t)hh * hd;
         PartView::Pending p1[kQkMaxPairs], p2[kQkMaxPairs];
 #pragma unroll
@@ -464,7 +466,8 @@ cudaError_t launch_qk_epilogue(const dspark_model* m, int layer, const PartView&
                                const int32_t* block_pos, void* q, void* kb, void* vb, cudaStream_t s) {
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
-    return launch_pdl(qk_epilogue_kernel, dim3(A * d.gamma), dim3(32 * kQkWarps), 0, s, part, d.gamma, d.nH, d.nKv, d.hd,
+    const dim3 grid((unsigned)(A * d.gamma), (unsigned)((d.nH + d.nKv + kQkWarps - 1) / kQkWarps));
+    return launch_pdl(qk_epilogue_kernel, grid, dim3(32 * kQkWarps), 0, s, part, d.gamma, d.nH, d.nKv, d.hd,
                       block_pos, m->ws.inv_freq, m->layers[layer].q_norm, m->layers[layer].k_norm, d.eps, d.dtype,
                       d.kv_dtype, q, kb, vb);
 }
