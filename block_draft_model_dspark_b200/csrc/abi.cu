@@ -680,7 +680,9 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
     // the persistent walk's grid-barrier counter
     cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, p.ticket), 0, sizeof(uint32_t), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(at<void>(ws, p.walk_keys), 0, (size_t)d.gamma * A * 8, s);
-    if (e == cudaSuccess) e = launch_embed(m, anchors, A, h, x, m->ws.status, s);
+    ActBuf x_emb = x;
+    if (p.tc) x_emb.f32 = nullptr;                  // the first layer's GEMM reads the fp16 form
+    if (e == cudaSuccess) e = launch_embed(m, anchors, A, h, x_emb, m->ws.status, s);
     for (int l = 0; l < d.Lyr && e == cudaSuccess; ++l) {
         const LayerRef& L = m->layers[l];
         e = run_gemm(m, x, L.qk, M, Nqk, d.H, part, sc, &pv, DSPARK_TIMER_GEMM_QK, s);
@@ -688,17 +690,25 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
         if (e == cudaSuccess) {
             AttnArgs a = attn_args(m, p, ws, cache, l, A, q, kb, vb, ao.f32, d.kv_dtype, DSPARK_DTYPE_F32);
             a.out_hi = ao.hi; a.out_lo = ao.lo;
+            if (p.tc && !m->attn_dump) a.out = nullptr;    // the o GEMM reads the fp16 form only
             e = run_attention(m, a, s);
         }
         if (e == cudaSuccess && m->attn_dump)
             e = cudaMemcpyAsync(reinterpret_cast<char*>(m->attn_dump) + dump_layer * l, ao.f32, dump_layer,
                                 cudaMemcpyDeviceToDevice, s);
         if (e == cudaSuccess) e = run_gemm(m, ao, L.o, M, d.H, d.nH * d.hd, part, sc, &pv, DSPARK_TIMER_GEMM_O, s);
-        if (e == cudaSuccess) e = launch_o_epilogue(m, l, pv, M, h, x, s);
+        // on tensor cores the next GEMM reads only the fp16 forms: the fp32 ones are
+        // written only for the last layer's normed hidden (the confidence head reads it)
+        ActBuf x_out = x, act_out = act;
+        if (p.tc) act_out.f32 = nullptr;
+        if (p.tc && l + 1 < d.Lyr) x_out.f32 = nullptr;
+        ActBuf x_mid = x;
+        if (p.tc) x_mid.f32 = nullptr;
+        if (e == cudaSuccess) e = launch_o_epilogue(m, l, pv, M, h, x_mid, s);
         if (e == cudaSuccess) e = run_gemm(m, x, L.gu, M, 2 * d.I, d.H, part, sc, &pv, DSPARK_TIMER_GEMM_GU, s);
-        if (e == cudaSuccess) e = launch_gu_epilogue(m, pv, M, act, s);
+        if (e == cudaSuccess) e = launch_gu_epilogue(m, pv, M, act_out, s);
         if (e == cudaSuccess) e = run_gemm(m, act, L.down, M, d.H, d.I, part, sc, &pv, DSPARK_TIMER_GEMM_DOWN, s);
-        if (e == cudaSuccess) e = launch_down_epilogue(m, l, pv, M, h, x, s);
+        if (e == cudaSuccess) e = launch_down_epilogue(m, l, pv, M, h, x_out, s);
     }
     TileStats ts;
     ts.mx = at<float>(ws, p.st_mx); ts.arg = at<int>(ws, p.st_arg); ts.se = at<float>(ws, p.st_se);

@@ -209,8 +209,12 @@ __device__ __forceinline__ void store_out4(const AttnTcParams& P, int64_t o, flo
     uint2 hv;
     hv.x = *reinterpret_cast<const uint32_t*>(&h01);
     hv.y = *reinterpret_cast<const uint32_t*>(&h23);
-    if (P.out_dtype == DSPARK_DTYPE_F32) *reinterpret_cast<float4*>(static_cast<float*>(P.out) + o) = v;
-    else *reinterpret_cast<uint2*>(static_cast<__half*>(P.out) + o) = hv;
+    if (!P.out) {
+    } else if (P.out_dtype == DSPARK_DTYPE_F32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(P.out) + o) = v;
+    } else {
+        *reinterpret_cast<uint2*>(static_cast<__half*>(P.out) + o) = hv;
+    }
     if (P.out_hi) {
         *reinterpret_cast<uint2*>(P.out_hi + o) = hv;
         if (P.out_lo) {

@@ -95,9 +95,13 @@ __device__ __forceinline__ void rope_sincos(int pos, double inv_freq, float* s, 
 }
 
 // gelu_pytorch_tanh.
+// gelu with the tanh approximation, 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3),
+// written as x sigmoid(2u) = x / (1 + exp(-2u)) (the same function): one exponential
+// and one approximate division (x / inf -> 0 for very negative x).
 __device__ __forceinline__ float gelu_tanh(float x) {
-    const float k0 = 0.7978845608028654f;   // sqrt(2/pi)
-    return 0.5f * x * (1.f + tanhf(k0 * (x + 0.044715f * x * x * x)));
+    const float k2 = 2.f * 0.7978845608028654f;   // 2 sqrt(2/pi)
+    const float u2 = k2 * fmaf(0.044715f * x, x * x, x);
+    return __fdividef(x, 1.f + __expf(-u2));
 }
 
 // Eight consecutive weights W[n, k0 .. k0+7] of an affine 4-bit matrix

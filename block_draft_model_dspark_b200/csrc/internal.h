@@ -73,6 +73,17 @@ struct PartView {
     int BN = 16, n_mt = 1, kb = 1, P = 1;      // mode 1
     int T = 1, G = 1;                          // mode 1: stream-K partition (K blocks, CTAs)
     int wide = 0;                              // mode 1: T * G needs 64-bit arithmetic
+    // mode 1: division by T as a multiply (Granlund-Montgomery round-up method):
+    // x / T = (t + ((x - t) >> sh1)) >> sh2 with t = umulhi(x, magic), exact for every
+    // 32-bit x (set_divisor)
+    uint32_t magic = 1; int sh1 = 0, sh2 = 0;
+    void set_divisor(uint32_t d) {
+        int l = 0;
+        while (l < 32 && ((uint64_t)1 << l) < d) ++l;
+        magic = (uint32_t)((((uint64_t)1 << 32) * (((uint64_t)1 << l) - d)) / d + 1);
+        sh1 = l < 1 ? l : 1;
+        sh2 = l > 1 ? l - 1 : 0;
+    }
     struct Pending {
         float x[kMaxPartials];
         int cnt;
@@ -81,7 +92,9 @@ struct PartView {
     // the CTA whose K range holds global K block g (32-bit division unless T * G >= 2^32)
     __device__ __forceinline__ int cta_of(int g) const {
         if (wide) return (int)((((int64_t)g + 1) * G - 1) / T);
-        return (int)((((uint32_t)g + 1u) * (uint32_t)G - 1u) / (uint32_t)T);
+        const uint32_t x = ((uint32_t)g + 1u) * (uint32_t)G - 1u;
+        const uint32_t t = __umulhi(x, magic);
+        return (int)((t + ((x - t) >> sh1)) >> sh2);
     }
     __device__ __forceinline__ Pending load(int64_t m, int64_t n) const {
         Pending q;

@@ -19,8 +19,9 @@ namespace {
 
 constexpr int kMaxPer = 16;   // columns per thread in the full-row kernels
 
+// The fp32 form is written only where a consumer reads it (f32 != NULL).
 __device__ __forceinline__ void store_act(const ActBuf& a, int64_t i, float v) {
-    a.f32[i] = v;
+    if (a.f32) a.f32[i] = v;
     if (a.hi) {
         const __half h = __float2half_rn(v);
         a.hi[i] = h;
@@ -30,7 +31,7 @@ __device__ __forceinline__ void store_act(const ActBuf& a, int64_t i, float v) {
 
 // Four consecutive activation values at i .. i + 3 (i % 4 == 0).
 __device__ __forceinline__ void store_act4(const ActBuf& a, int64_t i, float4 v) {
-    *reinterpret_cast<float4*>(a.f32 + i) = v;
+    if (a.f32) *reinterpret_cast<float4*>(a.f32 + i) = v;
     if (a.hi) {
         const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
         uint2 hv;
@@ -169,10 +170,23 @@ __global__ void __launch_bounds__(512) embed_kernel(MatRef E, int dtype, int gro
 // ------------------------------------------------------------------ q / k / v heads
 // grid (M, ceil((nH + nKv) / kQkWarps)), block kQkWarps warps: the row's RoPE
 // angles (hd/2 of them, one position) go into shared memory first, one per
-// thread, then one warp per head; lane l owns the RoPE pairs (i, i + hd/2) for
-// i = l, l + 32, ... < hd/2.
+// thread, then one warp per head.
 constexpr int kQkWarps = 4;
-constexpr int kQkMaxPairs = 4;                // hd/2 / 32 for hd <= 256
+// Four consecutive values at i .. i + 3 of an fp32 or fp16 tensor (i % 4 == 0).
+__device__ __forceinline__ void store4_any(void* p, int64_t i, int dtype, float4 v) {
+    if (dtype == DSPARK_DTYPE_F32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(p) + i) = v;
+    } else if (dtype == DSPARK_DTYPE_F16) {
+        const __half2 a = __floats2half2_rn(v.x, v.y), c = __floats2half2_rn(v.z, v.w);
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t*>(&a);
+        u.y = *reinterpret_cast<const uint32_t*>(&c);
+        *reinterpret_cast<uint2*>(static_cast<__half*>(p) + i) = u;
+    } else {
+        store_any(p, i, dtype, v.x); store_any(p, i + 1, dtype, v.y);
+        store_any(p, i + 2, dtype, v.z); store_any(p, i + 3, dtype, v.w);
+    }
+}
 __global__ void __launch_bounds__(32 * kQkWarps)
 qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, int hd, const int32_t* __restrict__ block_pos,
                    const double* __restrict__ inv_freq, const void* __restrict__ q_norm,
@@ -184,53 +198,54 @@ qk_epilogue_kernel(PartView part, int gamma, int nH, int nKv, int hd, const int3
     const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int b = m / gamma, t = m % gamma;
     const int pos = block_pos[b] + t;
-    const int half = hd / 2, np = half / 32;      // pairs per lane
+    const int half = hd / 2;
     for (int i = threadIdx.x; i < half; i += blockDim.x) rope_sincos(pos, inv_freq[i], &s_sin[i], &s_cos[i]);
     __syncthreads();
-    {
-        const int hh = blockIdx.y * kQkWarps + warp;
-        if (hh >= nH + nKv) return;
-        const int64_t col = (int64_t)hh * hd;
-        PartView::Pending p1[kQkMaxPairs], p2[kQkMaxPairs];
+    const int hh = blockIdx.y * kQkWarps + warp;
+    if (hh >= nH + nKv) return;
+    // lane l: the RoPE pairs (i, i + hd/2) for the four i = 4l .. 4l + 3 (lanes past hd/8 idle)
+    const int i0 = 4 * lane;
+    const bool act = i0 < half;
+    const int64_t col = (int64_t)hh * hd;
+    float4 x1 = make_float4(0.f, 0.f, 0.f, 0.f), x2 = x1;
+    if (act) {
+        const PartView::Pending4 p1 = part.load4(m, col + i0), p2 = part.load4(m, col + i0 + half);
+        x1 = part.finish4(p1);
+        x2 = part.finish4(p2);
+    }
+    float ss = x1.x * x1.x + x1.y * x1.y + x1.z * x1.z + x1.w * x1.w + x2.x * x2.x + x2.y * x2.y + x2.z * x2.z +
+               x2.w * x2.w;
+    ss = warp_sum(ss);
+    if (!act) return;
+    const float rinv = rsqrtf(ss / (float)hd + eps);
+    const float a1[4] = {x1.x * rinv, x1.y * rinv, x1.z * rinv, x1.w * rinv};
+    const float a2[4] = {x2.x * rinv, x2.y * rinv, x2.z * rinv, x2.w * rinv};
+    float r1[4], r2[4];
+    if (hh < nH) {
 #pragma unroll
-        for (int e = 0; e < kQkMaxPairs; ++e) {
-            if (e < np) {
-                p1[e] = part.load(m, col + lane + 32 * e);
-                p2[e] = part.load(m, col + lane + 32 * e + half);
-            }
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j;
+            const float y1 = a1[j] * load_any(q_norm, i, dtype), y2 = a2[j] * load_any(q_norm, i + half, dtype);
+            r1[j] = y1 * s_cos[i] - y2 * s_sin[i];
+            r2[j] = y2 * s_cos[i] + y1 * s_sin[i];
         }
-        float x1[kQkMaxPairs], x2[kQkMaxPairs];
-        float ss = 0.f;
+        const int64_t o = ((int64_t)m * nH + hh) * hd;                // the attention's query type
+        store4_any(q, o + i0, kv_dtype, make_float4(r1[0], r1[1], r1[2], r1[3]));
+        store4_any(q, o + i0 + half, kv_dtype, make_float4(r2[0], r2[1], r2[2], r2[3]));
+    } else {
+        const int g = hh - nH;
+        const int64_t o = ((int64_t)m * nKv + g) * hd;
+        store4_any(vb, o + i0, kv_dtype, make_float4(a1[0], a1[1], a1[2], a1[3]));
+        store4_any(vb, o + i0 + half, kv_dtype, make_float4(a2[0], a2[1], a2[2], a2[3]));
 #pragma unroll
-        for (int e = 0; e < kQkMaxPairs; ++e) {
-            x1[e] = e < np ? part.finish(p1[e]) : 0.f;
-            x2[e] = e < np ? part.finish(p2[e]) : 0.f;
-            ss += x1[e] * x1[e] + x2[e] * x2[e];
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j;
+            const float k1 = a1[j] * load_any(k_norm, i, dtype), k2 = a2[j] * load_any(k_norm, i + half, dtype);
+            r1[j] = k1 * s_cos[i] - k2 * s_sin[i];
+            r2[j] = k2 * s_cos[i] + k1 * s_sin[i];
         }
-        ss = warp_sum(ss);
-        const float rinv = rsqrtf(ss / (float)hd + eps);
-#pragma unroll
-        for (int e = 0; e < kQkMaxPairs; ++e) {
-            if (e >= np) break;
-            const int i = lane + 32 * e;
-            float y1 = x1[e] * rinv, y2 = x2[e] * rinv;
-            const float sn = s_sin[i], cs = s_cos[i];
-            if (hh < nH) {
-                y1 *= load_any(q_norm, i, dtype);
-                y2 *= load_any(q_norm, i + half, dtype);
-                const int64_t o = ((int64_t)m * nH + hh) * hd;
-                store_any(q, o + i, kv_dtype, y1 * cs - y2 * sn);          // the attention's query type
-                store_any(q, o + i + half, kv_dtype, y2 * cs + y1 * sn);
-            } else {
-                const int g = hh - nH;
-                const int64_t o = ((int64_t)m * nKv + g) * hd;
-                store_any(vb, o + i, kv_dtype, y1);
-                store_any(vb, o + i + half, kv_dtype, y2);
-                const float k1 = y1 * load_any(k_norm, i, dtype), k2 = y2 * load_any(k_norm, i + half, dtype);
-                store_any(kb, o + i, kv_dtype, k1 * cs - k2 * sn);
-                store_any(kb, o + i + half, kv_dtype, k2 * cs + k1 * sn);
-            }
-        }
+        store4_any(kb, o + i0, kv_dtype, make_float4(r1[0], r1[1], r1[2], r1[3]));
+        store4_any(kb, o + i0 + half, kv_dtype, make_float4(r2[0], r2[1], r2[2], r2[3]));
     }
 }
 
@@ -332,6 +347,65 @@ __global__ void __launch_bounds__(512) residual_epilogue_kernel(PartView part, i
     if (C > 1) cluster_sync();
 }
 
+// The same epilogue with one CTA of kResThreads per row and the row's GEMM
+// result in shared memory (H / 4 float4, one per 4-column group; a thread owns
+// groups tid, tid + kResThreads, ...): few registers, so several rows share an
+// SM, for M well above the SM count. Three passes over the thread's groups:
+// the partial sums (two groups' loads in flight) and their sum of squares; h
+// and its sum of squares; x.
+constexpr int kResThreads = 256;
+__global__ void __launch_bounds__(kResThreads, 4) residual_row_kernel(PartView part, int H, const void* __restrict__ g1,
+                                                                   const void* __restrict__ g2,
+                                                                   const void* __restrict__ scalar, int mode, float eps,
+                                                                   int dtype, float* __restrict__ h, ActBuf x) {
+    extern __shared__ float4 srow[];                // [H / 4]
+    __shared__ float red[32];
+    pdl_trigger();
+    const float s = mode == 1 ? load_any(scalar, 0, dtype) : 1.f;
+    pdl_wait();
+    const int m = blockIdx.x, ng = H / 4;
+    float ss = 0.f;
+    for (int g0 = threadIdx.x; g0 < ng; g0 += 2 * kResThreads) {
+        const int ga = g0, gb = g0 + kResThreads;
+        PartView::Pending4 qa, qb;
+        qa = part.load4(m, 4 * (int64_t)ga);
+        if (gb < ng) qb = part.load4(m, 4 * (int64_t)gb);
+        const float4 va = part.finish4(qa);
+        srow[ga] = va;
+        ss += va.x * va.x + va.y * va.y + va.z * va.z + va.w * va.w;
+        if (gb < ng) {
+            const float4 vb = part.finish4(qb);
+            srow[gb] = vb;
+            ss += vb.x * vb.x + vb.y * vb.y + vb.z * vb.z + vb.w * vb.w;
+        }
+    }
+    ss = block_sum(ss, red);
+    const float r1 = rsqrtf(ss / (float)H + eps);
+    float4* hrow = reinterpret_cast<float4*>(h + (int64_t)m * H);
+    float ss2 = 0.f;
+    for (int gi = threadIdx.x; gi < ng; gi += kResThreads) {
+        const float4 a = srow[gi], hh = hrow[gi];
+        const int j = 4 * gi;
+        float4 v;
+        v.x = (hh.x + a.x * r1 * load_any(g1, j, dtype)) * s;
+        v.y = (hh.y + a.y * r1 * load_any(g1, j + 1, dtype)) * s;
+        v.z = (hh.z + a.z * r1 * load_any(g1, j + 2, dtype)) * s;
+        v.w = (hh.w + a.w * r1 * load_any(g1, j + 3, dtype)) * s;
+        hrow[gi] = v;
+        srow[gi] = v;
+        ss2 += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss2 = block_sum(ss2, red);
+    const float r2 = rsqrtf(ss2 / (float)H + eps);
+    for (int gi = threadIdx.x; gi < ng; gi += kResThreads) {
+        const float4 v = srow[gi];
+        const int j = 4 * gi;
+        store_act4(x, (int64_t)m * H + j,
+                   make_float4(v.x * r2 * load_any(g2, j, dtype), v.y * r2 * load_any(g2, j + 1, dtype),
+                               v.z * r2 * load_any(g2, j + 2, dtype), v.w * r2 * load_any(g2, j + 3, dtype)));
+    }
+}
+
 __global__ void __launch_bounds__(256) gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
     pdl_trigger();
     pdl_wait();
@@ -421,6 +495,16 @@ cudaError_t launch_residual_any(const PartView& part, int M, int H, const void* 
                                 const void* scalar, int mode, float eps, int dtype, float* h, const ActBuf& x,
                                 int num_sms, cudaStream_t s) {
     const int C = residual_cluster(M, H, num_sms);
+    if (C == 1 && M >= num_sms && H % 4 == 0) {      // rows enough to fill the SMs: a CTA per row
+        const size_t smem = (size_t)H * sizeof(float);
+        if (smem > 48 * 1024) {
+            const cudaError_t e = cudaFuncSetAttribute(residual_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        return launch_pdl(residual_row_kernel, dim3(M), dim3(kResThreads), smem, s, part, H, g1, g2, scalar, mode, eps,
+                          dtype, h, x);
+    }
     const int Hc = (H + C - 1) / C;                 // columns per CTA
     // split rows: ~4 columns a thread (each load group of 4 covers the CTA's columns)
     const int t = C > 1 ? std::min(512, std::max(32, ((Hc + 3) / 4 + 31) / 32 * 32)) : row_threads(Hc);
