@@ -97,7 +97,7 @@ void tc_view(const tc::GemmPlan& p, float* out, const GemmScratch& sc, PartView*
     *v = PartView{};
     if (p.streamk) {
         v->mode = 1; v->p = sc.part;
-        v->BN = p.BN; v->n_mt = p.n_mt; v->kb = p.kb; v->P = p.P; v->T = p.T; v->G = p.G;
+        v->BN = p.BN; v->n_mt = p.n_mt; v->kb = p.kb; v->P = p.P; v->T = p.T; v->G = p.G; v->pair = p.pair;
         v->wide = (int64_t)p.T * p.G >= ((int64_t)1 << 32) || p.T > (1 << 30);
         v->set_divisor((uint32_t)p.T);
     } else {

@@ -97,7 +97,8 @@ struct Q4Pieces {
     int n;
 };
 
-// Iterates the (tile, k-range) segments of one CTA, identically in every role.
+// Iterates the (tile, k-range) segments of one work unit (a CTA, or a CTA pair),
+// identically in every role.
 struct SegIter {
     const GemmPlan& p;
     int c;
@@ -120,7 +121,7 @@ struct SegIter {
         }
         if (t >= p.tiles) return false;
         tile = t; k0 = 0; k1 = p.kb; slot = 0;
-        t += p.grid;
+        t += p.units;
         return true;
     }
 };
@@ -156,7 +157,14 @@ __device__ __forceinline__ float tanh_fast(float x) {
 // KSUB K blocks per stage; stage layout [KSUB x W block][KSUB x (NP x BN rows of X)]
 // [the packed 4-bit blocks, for WFMT kWQ4*]. WFMT: the weight format and the MMA's
 // operand type (gemm_tc.h).
-template <int NP, int KSUB, int WFMT>
+// PAIR: the CTAs of a cluster of two form one work unit (cta_group::2): CTA rank
+// r holds weight rows [128 r, 128 r + 128) of the unit's 256-row tile and
+// activation rows [r BN / 2, (r + 1) BN / 2) of its BN, at the same shared-memory
+// offsets, and half of the accumulator (its TMEM lanes). The even CTA issues the
+// MMAs (M = 256) and commits to both CTAs' barriers; both CTAs' TMA loads count
+// on its stage barriers (the 4-bit format: each CTA's converters tell it), and
+// both CTAs' epilogues free its accumulator buffers.
+template <int NP, int KSUB, int WFMT, bool PAIR>
 __global__ void __launch_bounds__(threads_for(WFMT), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, KParams kp) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -166,7 +174,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     const GemmPlan& p = kp.p;
     const int BN = p.BN;
     const int stages = p.stages;
-    const int b_bytes = BN * BK * 2;                // one K block of one activation part
+    const int rank = PAIR ? (int)cluster_ctarank() : 0;
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int xrows = PAIR ? BN / 2 : BN;           // activation rows this CTA holds
+    const int b_bytes = xrows * BK * 2;             // one K block of one activation part
     const int x_bytes = NP * b_bytes;               // one K block of the activation (hi and lo)
     const int raw_off = KSUB * (kABytes + x_bytes); // packed 4-bit blocks of the stage
     const int stage_bytes = raw_off + (kQ4 ? q4_raw_bytes(KSUB) : 0);
@@ -190,19 +201,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1); mbar_init(&empty[s], 1);
-            if (kConv) mbar_init(&conv[s], kConvThreads);
+            if (kConv) mbar_init(&conv[s], (PAIR ? 2 : 1) * kConvThreads);
         }
-        for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 32 * kEpi); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], (PAIR ? 2 : 1) * 32 * kEpi); }
         *abort_flag = 0;
         mbar_fence_init();
         if (!kQ4) prefetch_tmap(&tmW);       // packed 4-bit weights come by bulk copy (no weight map)
         prefetch_tmap(&tmX);
     }
-    if (warp == 1) tmem_alloc(tmem_slot, tmem_cols);
+    if (warp == 1) {
+        if (PAIR) tmem_alloc_pair(tmem_slot, tmem_cols);
+        else tmem_alloc(tmem_slot, tmem_cols);
+    }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();                        // the peer's barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // PAIR: the even CTA's barriers, as shared::cluster addresses (stage s at + 8 s)
+    const uint32_t full0 = PAIR ? mapa_shared(&full[0], 0) : 0u;
+    const uint32_t conv0 = PAIR ? mapa_shared(&conv[0], 0) : 0u;
+    const uint32_t acc_empty0 = PAIR ? mapa_shared(&acc_empty[0], 0) : 0u;
+    // stage loads counted on the even CTA's barrier (not for the 4-bit format, whose
+    // converters wait for their own CTA's loads)
+    constexpr bool kRemoteFull = PAIR && !kQ4;
     // No pdl_trigger: the consumer is launched as these CTAs exit. CTAs of a
     // consumer launched at the GEMM's start would sit in griddepcontrol.wait
     // for the whole GEMM, and kernels running beside such waiting CTAs were
@@ -213,7 +235,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         if (lane == 0) {
             // one request per stage for the weights, one for the activation
             auto load_w = [&](uint8_t* dst, uint64_t* bar, int kk, int nt) {
-                if (kQ4) {
+                if (kRemoteFull) {
+                    const uint32_t fb = full0 + 8u * (uint32_t)(bar - full);
+                    if (KSUB == 1) tma_load_2d_pair(dst, &tmW, fb, kk * BK, nt * BM);
+                    else tma_load_3d_pair(dst, &tmW, fb, 0, nt * BM, kk * KSUB);
+                } else if (kQ4) {
                     // the tile's packed blocks [nt][K block] are contiguous: one bulk copy per stage
                     const uint8_t* src = static_cast<const uint8_t*>(kp.wq4) +
                                          ((int64_t)nt * (p.kb * KSUB) + (int64_t)kk * KSUB) * kQ4BlockBytes;
@@ -225,39 +251,50 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 }
             };
             auto load_x = [&](uint8_t* dst, uint64_t* bar, int kk, int mt) {
-                if (NP == 1 && KSUB == 1) tma_load_2d(dst, &tmX, bar, kk * BK, mt * BN);
-                else if (NP == 1) tma_load_3d(dst, &tmX, bar, 0, mt * BN, kk * KSUB);
+                const int xr = mt * BN + rank * xrows;         // this CTA's activation rows
+                if (kRemoteFull) {
+                    const uint32_t fb = full0 + 8u * (uint32_t)(bar - full);
+                    if (KSUB == 1) tma_load_2d_pair(dst, &tmX, fb, kk * BK, xr);
+                    else tma_load_3d_pair(dst, &tmX, fb, 0, xr, kk * KSUB);
+                } else if (NP == 1 && KSUB == 1) tma_load_2d(dst, &tmX, bar, kk * BK, xr);
+                else if (NP == 1) tma_load_3d(dst, &tmX, bar, 0, xr, kk * KSUB);
                 else if (KSUB == 1) tma_load_3d(dst, &tmX, bar, kk * BK, mt * BN, 0);
                 else tma_load_4d(dst, &tmX, bar, 0, mt * BN, 0, kk * KSUB);
             };
             // The weights do not depend on the previous kernel: the first
             // `stages` weight tiles are requested before waiting for it, so
             // the weight stream starts while the producer of X drains.
+            auto expect = [&](uint64_t* bar) {
+                if (!kRemoteFull) mbar_arrive_expect_tx(bar, tx_bytes);
+                else if (rank == 0) mbar_arrive_expect_tx(bar, 2 * tx_bytes);
+            };
+            // the 128-row weight tile of this CTA in a unit's tile
+            auto wtile = [&](int tile) { return PAIR ? (tile / p.n_mt) * 2 + rank : tile / p.n_mt; };
             int n_pre = 0;
             {
-                SegIter it(p, blockIdx.x);
+                SegIter it(p, unit);
                 int tile, k0, k1, slot;
                 while (n_pre < stages && it.next(tile, k0, k1, slot)) {
-                    const int nt = tile / p.n_mt;
+                    const int nt = wtile(tile);
                     for (int kk = k0; kk < k1 && n_pre < stages; ++kk, ++n_pre) {
-                        mbar_arrive_expect_tx(&full[n_pre], tx_bytes);
+                        expect(&full[n_pre]);
                         load_w(base + n_pre * stage_bytes, &full[n_pre], kk, nt);
                     }
                 }
             }
             pdl_wait();
-            SegIter it(p, blockIdx.x);
+            SegIter it(p, unit);
             int tile, k0, k1, slot, n = 0;
             bool ok = true;
             while (ok && it.next(tile, k0, k1, slot)) {
-                const int nt = tile / p.n_mt, mt = tile % p.n_mt;
+                const int nt = wtile(tile), mt = tile % p.n_mt;
                 for (int kk = k0; kk < k1; ++kk, ++n) {
                     const int s = n % stages;
                     uint8_t* st = base + s * stage_bytes;
                     if (n >= n_pre) {
                         const uint32_t ph = (uint32_t)(n / stages) & 1u;
                         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, kp.status)) { ok = false; break; }
-                        mbar_arrive_expect_tx(&full[s], tx_bytes);
+                        expect(&full[s]);
                         load_w(st, &full[s], kk, nt);
                     }
                     load_x(st + KSUB * kABytes, &full[s], kk, mt);
@@ -266,10 +303,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             // drain: the loads of the last `stages` slots (every issued slot
             // has its X loads too, since no wait precedes them) complete
             // before teardown, also after an abort (bounded)
+            // (the odd CTA of a pair whose loads count on the even CTA's barriers waits
+            // for the MMAs that read them instead: the commits reach its own empty barriers)
             const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
+            const bool own_full = !kRemoteFull || rank == 0;
             for (int d = 0; d < stages && d < n; ++d) {
                 const int m = n - 1 - d;
-                if (!mbar_wait_until(&full[m % stages], (uint32_t)(m / stages) & 1u, deadline)) {
+                uint64_t* bar = own_full ? &full[m % stages] : &empty[m % stages];
+                if (!mbar_wait_until(bar, (uint32_t)(m / stages) & 1u, deadline)) {
                     atomicOr(kp.status, DSPARK_DEV_WAIT_TIMEOUT);
                     break;
                 }
@@ -280,15 +321,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         pdl_wait();
-        if (lane == 0) {
+        if (lane == 0 && (!PAIR || rank == 0)) {
             // hi and lo in one MMA when both fit in N <= 256: the X_lo rows sit right
             // after the X_hi rows in the stage, so [X_hi; X_lo] is one B operand of
             // 2 BN rows and the two products land in adjacent accumulator columns
             const bool fused = NP == 2 && p.acc_cols == 2 * BN;
             constexpr bool kF16 = WFMT == kWF16 || WFMT == kWQ4AsF16;
-            const uint32_t idesc = kF16 ? idesc_f16(BM, fused ? 2 * BN : BN, 0) : idesc_bf16(BM, fused ? 2 * BN : BN);
+            constexpr int kM = PAIR ? 2 * BM : BM;         // the pair's MMA spans both CTAs' weight rows
+            const uint32_t idesc = kF16 ? idesc_f16(kM, fused ? 2 * BN : BN, 0) : idesc_bf16(kM, fused ? 2 * BN : BN);
             uint64_t* ready = kConv ? conv : full;          // the converters' barrier when they transform W
-            SegIter it(p, blockIdx.x);
+            SegIter it(p, unit);
             int tile, k0, k1, slot, n = 0, seg = 0;
             bool ok = true;
             while (ok && it.next(tile, k0, k1, slot)) {
@@ -313,14 +355,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 #pragma unroll
                             for (int j = 0; j < BK / 16; ++j) {
                                 const uint32_t accum = (kk > k0 || sub > 0 || part > 0 || j > 0) ? 1u : 0u;
-                                mma_bf16(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, accum);
+                                if (PAIR) mma_pair(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, accum);
+                                else mma_bf16(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, accum);
                             }
                         }
                     }
-                    mma_commit(&empty[s]);          // frees the stage once these MMAs have read it
+                    // frees the stage (in both CTAs of a pair) once these MMAs have read it
+                    if (PAIR) mma_commit_pair(&empty[s], 3);
+                    else mma_commit(&empty[s]);
                 }
                 if (!ok) break;
-                mma_commit(&acc_full[acc]);         // the tile's accumulator is complete
+                // the tile's accumulator is complete (both halves of a pair's)
+                if (PAIR) mma_commit_pair(&acc_full[acc], 3);
+                else mma_commit(&acc_full[acc]);
                 ++seg;
             }
         }
@@ -331,7 +378,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         // of row i at chunk c ^ (i & 7)), then the stage's barrier counts it.
         pdl_wait();
         const int i = threadIdx.x - (64 + 32 * kEpi);
-        SegIter it(p, blockIdx.x);
+        SegIter it(p, unit);
         int tile, k0, k1, slot, n = 0;
         bool ok = true;
         while (ok && it.next(tile, k0, k1, slot)) {
@@ -363,7 +410,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     }
                 }
                 fence_async_shared();            // the MMA reads these through the async proxy
-                mbar_arrive(&conv[s]);
+                if (PAIR) mbar_arrive_cluster(conv0 + 8u * (uint32_t)s);   // the even CTA's MMAs read both halves
+                else mbar_arrive(&conv[s]);
             }
         }
     } else {
@@ -380,7 +428,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         const bool with_stats = kp.stats.mx != nullptr && !p.streamk;
         const bool bounds = with_stats && kp.w2norm != nullptr;
         const float Bw1 = bounds ? __uint_as_float(*kp.w1max_bits) : 0.f;
-        SegIter it(p, blockIdx.x);
+        SegIter it(p, unit);
         int tile, k0, k1, slot, seg = 0;
         while (it.next(tile, k0, k1, slot)) {
             const int acc = seg & 1;
@@ -389,10 +437,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             // the group leaves together if any wait gave up
             if (named_barrier_or(1, 32 * kEpi, !got || *abort_flag != 0)) break;
             tc_fence_after();
-            const int nt = tile / p.n_mt, mt = tile % p.n_mt;
+            // this CTA's 128-row weight tile (a pair's CTA r holds rows 128 r .. of the unit's 256)
+            const int nt = PAIR ? (tile / p.n_mt) * 2 + rank : tile / p.n_mt, mt = tile % p.n_mt;
             const int n = nt * BM + n_local;
             const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * p.acc_cols);
-            float* part_tile = kp.part + ((int64_t)tile * p.P * BN) * BM + n_local;
+            const int64_t store = PAIR ? 2 * (int64_t)tile + rank : tile;     // the partial tiles' 128-row half
+            float* part_tile = kp.part + (store * p.P * BN) * BM + n_local;
             const bool split_acc = p.acc_cols == 2 * BN;       // X_hi and X_lo products in separate columns
             for (int c0 = 16 * grp; c0 < BN; c0 += 16 * (kEpi / 4)) {
                 uint32_t r[16];
@@ -429,7 +479,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 }
             }
             tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);
+            if (PAIR) mbar_arrive_cluster(acc_empty0 + 8u * (uint32_t)acc);   // the even CTA's MMAs reuse it
+            else mbar_arrive(&acc_empty[acc]);
             if (with_stats) {
                 // the four warps' results of every position of the tile, merged in warp order
                 asm volatile("bar.sync 2, %0;" ::"r"(32 * kEpi) : "memory");
@@ -448,8 +499,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 
     tc_fence_before();
     __syncthreads();
+    // a pair's CTAs leave together: neither frees shared memory the other's MMAs,
+    // loads or arrivals may still reach
+    if (PAIR) cluster_sync();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+    if (warp == 1) {
+        if (PAIR) tmem_dealloc_pair(tmem_base, tmem_cols);
+        else tmem_dealloc(tmem_base, tmem_cols);
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -535,6 +592,8 @@ int tmem_cols_for(int acc_cols) {
 
 }  // namespace
 
+int pair_clusters_max(int wfmt, int ksub, size_t smem, int num_sms);
+
 GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles, bool stats, int wfmt) {
     GemmPlan p{};
     p.M = M; p.N = N; p.K = K; p.np = np; p.stats = stats ? 1 : 0; p.wfmt = wfmt;
@@ -542,13 +601,21 @@ GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles, b
     const int m_pad = (M + 15) / 16 * 16;
     p.BN = m_pad <= 256 ? m_pad : 256;
     p.n_mt = (M + p.BN - 1) / p.BN;
-    p.n_nt = (N + BM - 1) / BM;
+    // CTA pairs (cta_group::2) when the shared-memory traffic of the MMAs bounds the
+    // GEMM: one activation part and >= 128 activation rows per tile. Each CTA then
+    // stages 128 weight rows and BN / 2 activation rows per K block, for an MMA of
+    // 256 x BN: a third less shared-memory traffic per flop than 128 x BN alone.
+    // (not for 4-bit weights: their converters' hand-off to the other CTA's MMAs
+    // measured slower than one CTA per tile)
+    p.pair = (np == 1 && !q4 && p.BN >= 128 && N > BM && num_sms >= 2) ? 1 : 0;
+    const int xrows = p.pair ? p.BN / 2 : p.BN;
+    p.n_nt = (N + BM * (p.pair ? 2 : 1) - 1) / (BM * (p.pair ? 2 : 1));
     p.tiles = p.n_mt * p.n_nt;
     // as many stages as shared memory holds: the bytes in flight per SM are
     // what sustains the weight stream at HBM latency under load; two K blocks
     // per stage (half the TMA requests) when K allows and >= 3 stages still fit
     auto stage_bytes_for = [&](int ksub) {
-        return ksub * (kABytes + np * p.BN * BK * 2) + (q4 ? q4_raw_bytes(ksub) : 0);
+        return ksub * (kABytes + np * xrows * BK * 2) + (q4 ? q4_raw_bytes(ksub) : 0);
     };
     const int avail = kSmemLimit - kSmemExtra(kMaxStages) - (stats ? kStatBytes(p.BN) : 0);
     p.ksub = (K % (2 * BK) == 0 && avail / stage_bytes_for(2) >= 3) ? 2 : 1;
@@ -558,44 +625,55 @@ GemmPlan plan_gemm(int num_sms, int M, int N, int K, int np, bool force_tiles, b
     // bf16 pair activation, hi and lo go through one MMA of N = 2 BN when it fits
     p.acc_cols = (np == 2 && 2 * p.BN <= 256) ? 2 * p.BN : p.BN;
     p.tmem_cols = tmem_cols_for(p.acc_cols);
-    // tile mode when whole tiles balance the SMs to >= 90%, else stream-K
-    const int waves = (p.tiles + num_sms - 1) / num_sms;
-    const bool tiles_ok = force_tiles || (p.tiles >= num_sms && 10 * p.tiles >= 9 * waves * num_sms);
+    // work units: CTAs, or as many CTA pairs as can be resident at once
+    int units_max = num_sms;
+    if (p.pair) units_max = pair_clusters_max(wfmt, p.ksub, gemm_smem_bytes(p), num_sms);
+    // tile mode when whole tiles balance the units to >= 90%, else stream-K
+    const int waves = (p.tiles + units_max - 1) / units_max;
+    const bool tiles_ok = force_tiles || (p.tiles >= units_max && 10 * p.tiles >= 9 * waves * units_max);
     if (tiles_ok) {
         p.mode = kModeTiles; p.streamk = 0;
-        p.grid = std::min(p.tiles, num_sms);
-        p.T = p.tiles * p.kb; p.G = p.grid; p.P = 1;
+        p.units = std::min(p.tiles, units_max);
+        p.T = p.tiles * p.kb; p.G = p.units; p.P = 1;
     } else {
         p.mode = kModePartials; p.streamk = 1;
         p.T = p.tiles * p.kb;
-        p.G = std::min(p.T, num_sms);
-        p.grid = p.G;
+        p.G = std::min(p.T, units_max);
+        p.units = p.G;
         int P = 1;
         for (int t = 0; t < p.tiles; ++t) P = std::max(P, p.cta_of((t + 1) * p.kb - 1) - p.cta_of(t * p.kb) + 1);
         p.P = P;
     }
+    p.grid = p.units * (p.pair ? 2 : 1);
     return p;
 }
 
 size_t gemm_partial_elems(const GemmPlan& p) {
-    return p.streamk ? (size_t)p.tiles * p.P * p.BN * BM : 0;
+    return p.streamk ? (size_t)p.tiles * (p.pair ? 2 : 1) * p.P * p.BN * BM : 0;
 }
 
 size_t gemm_smem_bytes(const GemmPlan& p) {
     const bool q4 = p.wfmt == kWQ4AsF16;
-    const int stage_bytes = p.ksub * (kABytes + p.np * p.BN * BK * 2) + (q4 ? q4_raw_bytes(p.ksub) : 0);
+    const int xrows = p.pair ? p.BN / 2 : p.BN;
+    const int stage_bytes = p.ksub * (kABytes + p.np * xrows * BK * 2) + (q4 ? q4_raw_bytes(p.ksub) : 0);
     return (size_t)p.stages * stage_bytes + kSmemExtra(p.stages) + (p.stats ? kStatBytes(p.BN) : 0);
 }
 
 namespace {
 
-template <int NP, int KSUB>
+template <int NP, int KSUB, bool PAIR>
 void* pick_kernel(int wfmt) {
     switch (wfmt) {
-        case kWF16: return (void*)gemm_tc_kernel<NP, KSUB, kWF16>;
-        case kWQ4AsF16: return (void*)gemm_tc_kernel<NP, KSUB, kWQ4AsF16>;
-        default: return (void*)gemm_tc_kernel<NP, KSUB, kWBf16>;
+        case kWF16: return (void*)gemm_tc_kernel<NP, KSUB, kWF16, PAIR>;
+        case kWQ4AsF16: return (void*)gemm_tc_kernel<NP, KSUB, kWQ4AsF16, PAIR>;
+        default: return (void*)gemm_tc_kernel<NP, KSUB, kWBf16, PAIR>;
     }
+}
+
+void* kernel_for(int np, int ksub, int pair, int wfmt) {
+    if (pair) return ksub == 2 ? pick_kernel<1, 2, true>(wfmt) : pick_kernel<1, 1, true>(wfmt);
+    return np == 2 ? (ksub == 2 ? pick_kernel<2, 2, false>(wfmt) : pick_kernel<2, 1, false>(wfmt))
+                   : (ksub == 2 ? pick_kernel<1, 2, false>(wfmt) : pick_kernel<1, 1, false>(wfmt));
 }
 
 // Packs one 128-row tile x one K block per CTA; thread i copies row i.
@@ -674,6 +752,39 @@ cudaError_t q4_pack(const Q4Piece* pieces, int npieces, int64_t n, int64_t k, vo
     return launch_pdl(q4_pack_kernel, grid, dim3(128), 0, s, pcs, n, k, static_cast<uint8_t*>(dst));
 }
 
+// CTA pairs resident at once on this device for the pair kernel of (wfmt, ksub)
+// with `smem` bytes of shared memory (clusters of two need two SMs of one GPC, so
+// this can be below num_sms / 2); cached per (device, kernel, smem).
+int pair_clusters_max(int wfmt, int ksub, size_t smem, int num_sms) {
+    static std::mutex mu;
+    struct Key { int dev; void* k; size_t smem; int v; };
+    static Key cache[32];
+    static int n_cache = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    void* kern = kernel_for(1, ksub, 1, wfmt);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n_cache; ++i)
+        if (cache[i].dev == dev && cache[i].k == kern && cache[i].smem == smem) return cache[i].v;
+    int v = num_sms / 2;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)(2 * v));
+        cfg.blockDim = dim3((unsigned)threads_for(wfmt));
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2; attr[0].val.clusterDim.y = 1; attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int c = 0;
+        if (cudaOccupancyMaxActiveClusters(&c, kern, &cfg) == cudaSuccess && c > 0) v = std::min(v, c);
+    }
+    cudaGetLastError();                               // a failed query leaves no sticky error
+    if (n_cache < 32) cache[n_cache++] = Key{dev, kern, smem, v};
+    return std::max(v, 1);
+}
+
 cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, const void* X0, const void* X1,
                            float* out, int64_t ldo, float cap, float* part, int32_t* status, cudaStream_t s,
                            const TileStats* stats, const float* w2norm, const uint32_t* w1max_bits) {
@@ -689,17 +800,20 @@ cudaError_t launch_gemm_tc(const GemmPlan& p, const void* W, int64_t w_rows, con
     memset(&tw, 0, sizeof(tw));
     // packed 4-bit weights come by bulk copy: the weight map is unused
     if (!q4 && !make_wmap(&tw, W, w_rows, p.K, p.ksub)) return cudaErrorInvalidValue;
-    if (!make_xmap(&tx, X0, p.M, p.K, p.BN, p.np, p.ksub)) return cudaErrorInvalidValue;
+    if (p.pair && (p.np != 1 || p.BN % 16)) return cudaErrorInvalidValue;
+    if (!make_xmap(&tx, X0, p.M, p.K, p.pair ? p.BN / 2 : p.BN, p.np, p.ksub)) return cudaErrorInvalidValue;
     KParams kp{};
     kp.p = p; kp.out = out; kp.ldo = ldo; kp.cap = cap; kp.cap_inv = cap > 0.f ? 1.f / cap : 0.f;
     kp.status = status; kp.part = part;
     kp.wq4 = q4 ? W : nullptr;
     if (stats) { kp.stats = *stats; kp.w2norm = w2norm; kp.w1max_bits = w1max_bits; }
     const size_t smem = gemm_smem_bytes(p);
-    void* kern = p.np == 2 ? (p.ksub == 2 ? pick_kernel<2, 2>(p.wfmt) : pick_kernel<2, 1>(p.wfmt))
-                           : (p.ksub == 2 ? pick_kernel<1, 2>(p.wfmt) : pick_kernel<1, 1>(p.wfmt));
+    void* kern = kernel_for(p.np, p.ksub, p.pair, p.wfmt);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    if (p.pair)
+        return launch_pdl_cluster(reinterpret_cast<void (*)(CUtensorMap, CUtensorMap, KParams)>(kern), dim3(p.grid),
+                                  dim3(threads_for(p.wfmt)), 2, smem, s, tw, tx, kp);
     return launch_pdl(reinterpret_cast<void (*)(CUtensorMap, CUtensorMap, KParams)>(kern), dim3(p.grid),
                       dim3(threads_for(p.wfmt)), smem, s, tw, tx, kp);
 }

@@ -12,7 +12,7 @@ struct TileStats;
 namespace tc {
 
 constexpr int kModeTiles = 0;      // whole tiles per CTA; result written directly
-constexpr int kModePartials = 1;   // stream-K; fp32 partial tiles [tile][P][BN][128]
+constexpr int kModePartials = 1;   // stream-K; fp32 partial tiles [tile][P][BN][128] ([tile][2][P][BN][128] for pairs)
 
 // Weight formats (and MMA operand types) of the GEMM:
 constexpr int kWBf16 = 0;       // bf16 weights straight from TMA; bf16 activation (the caller's context rows)
@@ -31,15 +31,17 @@ struct GemmPlan {
     int wfmt;              // weight format (kW*)
     int stats;             // tile mode: shared memory reserved for the epilogue's logit statistics
     int BN;                // activation rows per tile (MMA N)
-    int n_mt, n_nt;        // tiles along the activation rows and along the 128 weight rows
+    int n_mt, n_nt;        // tiles along the activation rows and along the weight rows (128, or 256 for pairs)
     int ksub;              // 64-wide K blocks per stage (1 or 2)
     int kb;                // stages along K: K / (64 ksub)
     int tiles;             // n_mt * n_nt; tile index t = nt * n_mt + mt
     int stages, tmem_cols;
     int acc_cols;          // TMEM columns per accumulator: 2 BN when X_hi and X_lo products share one MMA
     int mode, streamk;
+    int pair;              // CTA pairs (cta_group::2): a work unit is a 256-row weight tile on two CTAs
+    int units;             // work units: CTAs, or CTA pairs (grid = 2 units)
     int grid;              // CTAs launched
-    int T, G, P;           // stream-K: K blocks in all tiles, CTAs, most CTAs touching one tile
+    int T, G, P;           // stream-K: K blocks in all tiles, work units, most units touching one tile
     // First global K block of CTA c (stream-K partition of T blocks over G CTAs).
     __host__ __device__ int range_lo(int c) const { return (int)(((int64_t)c * T) / G); }
     // The CTA whose range holds global K block g.

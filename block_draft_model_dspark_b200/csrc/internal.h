@@ -73,6 +73,7 @@ struct PartView {
     int BN = 16, n_mt = 1, kb = 1, P = 1;      // mode 1
     int T = 1, G = 1;                          // mode 1: stream-K partition (K blocks, CTAs)
     int wide = 0;                              // mode 1: T * G needs 64-bit arithmetic
+    int pair = 0;                              // mode 1: CTA-pair tiles (256 weight rows, two 128-row halves)
     // mode 1: division by T as a multiply (Granlund-Montgomery round-up method):
     // x / T = (t + ((x - t) >> sh1)) >> sh2 with t = umulhi(x, magic), exact for every
     // 32-bit x (set_divisor)
@@ -106,9 +107,10 @@ struct PartView {
         }
         const int mi = (int)m, ni = (int)n;
         const int mt = mi / BN, ml = mi - mt * BN, nt = ni >> 7, nl = ni & 127;
-        const int tile = nt * n_mt + mt;
+        const int tile = (pair ? nt >> 1 : nt) * n_mt + mt;      // the work unit's tile
+        const int store = pair ? 2 * tile + (nt & 1) : tile;     // its 128-row half
         q.cnt = cta_of(tile * kb + kb - 1) - cta_of(tile * kb) + 1;
-        const float* base = p + (((int64_t)tile * P) * BN + ml) * 128 + nl;
+        const float* base = p + (((int64_t)store * P) * BN + ml) * 128 + nl;
 #pragma unroll
         for (int s = 0; s < kMaxPartials; ++s) q.x[s] = s < q.cnt ? base[(int64_t)s * BN * 128] : 0.f;
         q.rest = base;
@@ -141,10 +143,11 @@ struct PartView {
             base = p + (int64_t)m * ld + n;
         } else {
             const int mt = m / BN, ml = m - mt * BN, nt = (int)(n >> 7), nl = (int)(n & 127);
-            const int tile = nt * n_mt + mt;
+            const int tile = (pair ? nt >> 1 : nt) * n_mt + mt;
+            const int store = pair ? 2 * tile + (nt & 1) : tile;
             q.cnt = cta_of(tile * kb + kb - 1) - cta_of(tile * kb) + 1;
             q.step = (int64_t)BN * 128;
-            base = p + (((int64_t)tile * P) * BN + ml) * 128 + nl;
+            base = p + (((int64_t)store * P) * BN + ml) * 128 + nl;
         }
 #pragma unroll
         for (int s = 0; s < kMax4; ++s)
