@@ -232,23 +232,14 @@ __device__ __forceinline__ void store_out4(const AttnTcParams& P, int64_t o, flo
 constexpr int kMergeBatch = 8;       // slots whose rows a lane loads at once
 __device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, int r, int64_t out_row) {
     const int lane = threadIdx.x & 31, ng = P.hd / 4;
-    float M = -INFINITY;
-    for (int s = lane; s < k; s += 32) M = fmaxf(M, P.part_ml[((int64_t)(s0 + s) * QROWS + r) * 2]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float4 num[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-    float den = 0.f;
+    float den = 0.f, M = -INFINITY;
     for (int sb = 0; sb < k; sb += 32) {
-        float ws = 0.f, ls = 0.f;
-        if (sb + lane < k) {
-            const int64_t base = (int64_t)(s0 + sb + lane) * QROWS + r;
-            const float m = P.part_ml[base * 2];
-            ls = P.part_ml[base * 2 + 1];
-            ws = m == -INFINITY ? 0.f : __expf(m - M);
-        }
         const int cnt = min(32, k - sb);
-        for (int t0 = 0; t0 < cnt; t0 += kMergeBatch) {
-            float4 v[kMergeBatch][2];
+        // the first batch of rows and this chunk's (max, sum) pairs go out together: the rows'
+        // loads do not depend on the maxima
+        float4 v[kMergeBatch][2];
+        auto load_rows = [&](int t0) {
 #pragma unroll
             for (int u = 0; u < kMergeBatch; ++u) {
                 const float4* o = reinterpret_cast<const float4*>(P.part_o + ((int64_t)(s0 + sb + t0 + u) * QROWS + r) * P.hd);
@@ -258,10 +249,29 @@ __device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, 
                     v[u][q] = (t0 + u < cnt && g4 < ng) ? o[g4] : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
+        };
+        load_rows(0);
+        float2 ml = make_float2(-INFINITY, 0.f);
+        if (lane < cnt) ml = reinterpret_cast<const float2*>(P.part_ml)[(int64_t)(s0 + sb + lane) * QROWS + r];
+        float mc = ml.x;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+        // a later chunk with a larger maximum rescales what the earlier ones summed
+        const float Mn = fmaxf(M, mc);
+        if (Mn > M && M > -INFINITY) {
+            const float f = __expf(M - Mn);
+            den *= f;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) { num[q].x *= f; num[q].y *= f; num[q].z *= f; num[q].w *= f; }
+        }
+        M = Mn;
+        const float ws = ml.x == -INFINITY ? 0.f : __expf(ml.x - M);
+        for (int t0 = 0; t0 < cnt; t0 += kMergeBatch) {
+            if (t0 > 0) load_rows(t0);
 #pragma unroll
             for (int u = 0; u < kMergeBatch; ++u) {
                 const float w = __shfl_sync(0xffffffffu, ws, (t0 + u) & 31);
-                const float l = __shfl_sync(0xffffffffu, ls, (t0 + u) & 31);
+                const float l = __shfl_sync(0xffffffffu, ml.y, (t0 + u) & 31);
                 if (t0 + u >= cnt) break;
                 den += w * l;
                 if (w == 0.f) continue;                // uniform: an empty range

@@ -131,7 +131,7 @@ __global__ void commit_len_kernel(int32_t* len, const int32_t* n_new, int B) {
 }
 
 // ------------------------------------------------------------------ block embedding
-__global__ void __launch_bounds__(512) embed_kernel(MatRef E, int dtype, int group, const int32_t* __restrict__ anchors, int gamma,
+__global__ void __launch_bounds__(1024) embed_kernel(MatRef E, int dtype, int group, const int32_t* __restrict__ anchors, int gamma,
                              int mask_id, int V, int H, float scale, const void* __restrict__ w_in,
                              float eps, float* __restrict__ h, ActBuf x, int32_t* status) {
     __shared__ float red[32];
@@ -146,6 +146,40 @@ __global__ void __launch_bounds__(512) embed_kernel(MatRef E, int dtype, int gro
     }
     float vals[kMaxPer];
     float ss = 0.f;
+    if (!E.quant && dtype == DSPARK_DTYPE_BF16 && (H & 7) == 0) {
+        // bf16 rows: 8 consecutive values (16 bytes) per load, groups tid, tid + blockDim.x
+        const uint4* row = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(E.w) + (int64_t)id * E.k);
+#pragma unroll
+        for (int c8 = 0; c8 < kMaxPer / 8; ++c8) {
+            const int gi = threadIdx.x + c8 * blockDim.x;
+            uint4 u = make_uint4(0u, 0u, 0u, 0u);
+            if (gi * 8 < H) u = row[gi];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                vals[c8 * 8 + 2 * k] = __uint_as_float(w[k] << 16) * scale;
+                vals[c8 * 8 + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u) * scale;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ss += vals[c8 * 8 + k] * vals[c8 * 8 + k];
+        }
+        ss = block_sum(ss, red);
+        const float rinv = rsqrtf(ss / (float)H + eps);
+#pragma unroll
+        for (int c8 = 0; c8 < kMaxPer / 8; ++c8) {
+            const int j = (threadIdx.x + c8 * blockDim.x) * 8;
+            if (j >= H) continue;
+            float4* hp = reinterpret_cast<float4*>(h + (int64_t)m * H + j);
+            hp[0] = make_float4(vals[c8 * 8], vals[c8 * 8 + 1], vals[c8 * 8 + 2], vals[c8 * 8 + 3]);
+            hp[1] = make_float4(vals[c8 * 8 + 4], vals[c8 * 8 + 5], vals[c8 * 8 + 6], vals[c8 * 8 + 7]);
+            float y[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) y[k] = vals[c8 * 8 + k] * rinv * load_any(w_in, j + k, dtype);
+            store_act4(x, (int64_t)m * H + j, make_float4(y[0], y[1], y[2], y[3]));
+            store_act4(x, (int64_t)m * H + j + 4, make_float4(y[4], y[5], y[6], y[7]));
+        }
+        return;
+    }
 #pragma unroll
     for (int c = 0; c < kMaxPer; ++c) {
         const int j = threadIdx.x + c * blockDim.x;
@@ -406,16 +440,33 @@ __global__ void __launch_bounds__(kResThreads, 4) residual_row_kernel(PartView p
     }
 }
 
+// grid (ceil(I / (4 kGuGroups * 256)), M), 256 threads: thread t of CTA x owns the
+// kGuGroups 4-column groups x * 256 kGuGroups + t + 256 j; all their gate and up
+// loads go out before the first is used (two groups measured slower: the registers
+// of their pending partials halved the resident threads).
+constexpr int kGuGroups = 1;
 __global__ void __launch_bounds__(256) gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
     pdl_trigger();
     pdl_wait();
     const int m = blockIdx.y;
-    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-    if (i >= I) return;
-    const PartView::Pending4 qg = part.load4(m, i), qu = part.load4(m, I + i);
-    const float4 g = part.finish4(qg), u = part.finish4(qu);
-    store_act4(act, (int64_t)m * I + i,
-               make_float4(gelu_tanh(g.x) * u.x, gelu_tanh(g.y) * u.y, gelu_tanh(g.z) * u.z, gelu_tanh(g.w) * u.w));
+    const int64_t g0 = (int64_t)blockIdx.x * blockDim.x * kGuGroups + threadIdx.x;
+    PartView::Pending4 qg[kGuGroups], qu[kGuGroups];
+#pragma unroll
+    for (int j = 0; j < kGuGroups; ++j) {
+        const int64_t i = (g0 + (int64_t)j * blockDim.x) * 4;
+        if (i < I) {
+            qg[j] = part.load4(m, i);
+            qu[j] = part.load4(m, I + i);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kGuGroups; ++j) {
+        const int64_t i = (g0 + (int64_t)j * blockDim.x) * 4;
+        if (i >= I) continue;
+        const float4 g = part.finish4(qg[j]), u = part.finish4(qu[j]);
+        store_act4(act, (int64_t)m * I + i,
+                   make_float4(gelu_tanh(g.x) * u.x, gelu_tanh(g.y) * u.y, gelu_tanh(g.z) * u.z, gelu_tanh(g.w) * u.w));
+    }
 }
 
 // ------------------------------------------------------------------ confidence + truncation
@@ -542,7 +593,11 @@ cudaError_t launch_embed(const dspark_model* m, const int32_t* anchors, int A, f
                          int32_t* status, cudaStream_t s) {
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
-    return launch_pdl(embed_kernel, dim3(A * d.gamma), dim3(row_threads(d.H)), 0, s, m->embed, d.dtype, d.group, anchors,
+    // the bf16 path reads 8 values per load: H / 8 threads (two groups each above 1024 threads)
+    const bool vec = !m->embed.quant && d.dtype == DSPARK_DTYPE_BF16 && d.H % 8 == 0;
+    const int threads = vec ? ((std::min(d.H / 8, 1024) + 31) / 32 * 32) : row_threads(d.H);
+    if (vec && threads * kMaxPer < d.H) return cudaErrorInvalidValue;
+    return launch_pdl(embed_kernel, dim3(A * d.gamma), dim3(threads), 0, s, m->embed, d.dtype, d.group, anchors,
                       d.gamma, d.mask_id, d.V, d.H, sqrtf((float)d.H), m->layers[0].in_norm, d.eps, h, x, status);
 }
 
@@ -568,7 +623,7 @@ cudaError_t launch_gu_epilogue(const dspark_model* m, const PartView& part, int 
                                cudaStream_t s) {
     const Dims& d = m->d;
     KernelTimer t(DSPARK_TIMER_ROWS, s, 0.0, 0.0);
-    const dim3 grid((unsigned)((d.I / 4 + 255) / 256), (unsigned)M);
+    const dim3 grid((unsigned)((d.I / 4 + 256 * kGuGroups - 1) / (256 * kGuGroups)), (unsigned)M);
     return launch_pdl(gu_epilogue_kernel, grid, dim3(256), 0, s, part, M, d.I, act);
 }
 
