@@ -444,6 +444,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             const int64_t store = PAIR ? 2 * (int64_t)tile + rank : tile;     // the partial tiles' 128-row half
             float* part_tile = kp.part + (store * p.P * BN) * BM + n_local;
             const bool split_acc = p.acc_cols == 2 * BN;       // X_hi and X_lo products in separate columns
+            // B max |w2| over this warp's 32 entries (the group bound of the tile statistics)
+            float bwmax = 0.f;
+            if (with_stats && bounds) {
+                const float bw = n < p.N ? Bw1 * kp.w2norm[n] : 0.f;
+                bwmax = __uint_as_float(warp_max_u32(__float_as_uint(bw)));   // >= 0: bits order as floats
+            }
             for (int c0 = 16 * grp; c0 < BN; c0 += 16 * (kEpi / 4)) {
                 uint32_t r[16];
                 tmem_ld_x16(tbase + (uint32_t)c0, r);
@@ -468,8 +474,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     }
                     if (with_stats) {
                         // the 16 positions (columns) over this warp's 32 entries at once
-                        const float bw = bounds && n < p.N ? Bw1 * kp.w2norm[n] : 0.f;
-                        const WarpStat w = warp_logit_stat16(u, n, bw, bounds, kp.cap);
+                        const WarpStat w = warp_logit_stat16(u, n, bwmax, bounds, kp.cap);
                         if ((lane & 1) == 0) stat_sm[quad * BN + c0 + warp_stat16_col(lane)] = w;
                     }
                 } else {

@@ -3,12 +3,16 @@
 // 128 vocabulary entries v and for each position m,
 //   mx  = max_v U[m, v]                      arg = its lowest v
 //   se  = sum_v exp(U[m, v] - mx)            (the tile's share of the logsumexp)
-//   lo  = max_v (U[m, v] - B |w2[v]|)        hi = max_v (U[m, v] + B |w2[v]|)
-// where B |w2[v]| bounds the Markov transition bias |w2[v] . w1[p]| over
-// every previous token p (Cauchy-Schwarz). lo and hi let the walk's exact
-// pruning skip every tile that cannot hold a winner. A warp holds 32 entries
-// of a tile (one per lane) and reduces them per position; the four warps of a
-// tile then merge in warp order, so both producers give identical results.
+//   lo  = max_g (mx_g - B max_{v in g} |w2[v]|)   hi = max_g (mx_g + B max_{v in g} |w2[v]|)
+// over the tile's four 32-entry groups g (mx_g: the group's maximum), where B
+// |w2[v]| bounds the Markov transition bias |w2[v] . w1[p]| over every
+// previous token p (Cauchy-Schwarz). lo is at most max_v (U[m, v] - B |w2[v]|)
+// and hi at least max_v (U[m, v] + B |w2[v]|), so the walk's exact pruning,
+// which skips every tile whose hi is below some lo, stays exact; derived from
+// the group maxima, they add nothing to the per-position reduction. A warp
+// holds 32 entries of a tile (one per lane) and reduces them per position; the
+// four warps of a tile then merge in warp order, so both producers give
+// identical results.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -42,8 +46,8 @@ struct TileStats {
 };
 
 // One warp's part of a tile for one position: `u` is this lane's U value
-// (-inf for an entry past the vocabulary), `v` its vocabulary index and `bw`
-// its bound B |w2[v]| (0 without bounds). Returns the warp's results in every
+// (-inf for an entry past the vocabulary), `v` its vocabulary index and `bwmax`
+// the group bound B max |w2| over the warp's 32 entries (0 without bounds). Returns the warp's results in every
 // lane: keys of mx / lo / hi (0 = no entry), the lowest arg, and se relative
 // to the warp's mx.
 struct WarpStat {
@@ -51,7 +55,7 @@ struct WarpStat {
     int arg;
     float se;
 };
-__device__ __forceinline__ WarpStat warp_logit_stat(float u, int v, float bw, bool bounds) {
+__device__ __forceinline__ WarpStat warp_logit_stat(float u, int v, float bwmax, bool bounds) {
     WarpStat w;
     const bool valid = u > -INFINITY;
     w.kmx = warp_max_u32(valid ? f2ord(u) : 0u);
@@ -62,9 +66,9 @@ __device__ __forceinline__ WarpStat warp_logit_stat(float u, int v, float bw, bo
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
     w.se = e;
-    if (bounds) {
-        w.klo = warp_max_u32(valid ? f2ord(u - bw) : 0u);
-        w.khi = warp_max_u32(valid ? f2ord(u + bw) : 0u);
+    if (bounds && w.kmx) {
+        w.klo = f2ord(ord2f(w.kmx) - bwmax);
+        w.khi = f2ord(ord2f(w.kmx) + bwmax);
     } else {
         w.klo = w.khi = 0u;
     }
@@ -84,7 +88,6 @@ struct StatAcc {
     float m;     // maximum (-inf: no entry)
     int a;       // its lowest index
     float s;     // sum of exp(u - m)
-    float lo, hi;
 };
 __device__ __forceinline__ StatAcc stat_merge(const StatAcc& x, const StatAcc& y) {
     StatAcc r;
@@ -94,17 +97,13 @@ __device__ __forceinline__ StatAcc stat_merge(const StatAcc& x, const StatAcc& y
     const float small = y_wins ? x.m : y.m;
     const float s_big = y_wins ? y.s : x.s, s_small = y_wins ? x.s : y.s;
     r.s = small == -INFINITY ? s_big : s_big + s_small * __expf(small - r.m);
-    r.lo = fmaxf(x.lo, y.lo);
-    r.hi = fmaxf(x.hi, y.hi);
     return r;
 }
-__device__ __forceinline__ StatAcc stat_shfl(const StatAcc& x, int mask, bool bounds) {
+__device__ __forceinline__ StatAcc stat_shfl(const StatAcc& x, int mask) {
     StatAcc r;
     r.m = __shfl_xor_sync(0xffffffffu, x.m, mask);
     r.a = __shfl_xor_sync(0xffffffffu, x.a, mask);
     r.s = __shfl_xor_sync(0xffffffffu, x.s, mask);
-    r.lo = bounds ? __shfl_xor_sync(0xffffffffu, x.lo, mask) : -INFINITY;
-    r.hi = bounds ? __shfl_xor_sync(0xffffffffu, x.hi, mask) : -INFINITY;
     return r;
 }
 // With `cap` > 0 the values are softcapped logits, |u| <= cap: then exp(u - cap)
@@ -118,11 +117,9 @@ __device__ __forceinline__ StatAcc stat_merge_fixed(const StatAcc& x, const Stat
     r.m = y_wins ? y.m : x.m;
     r.a = y_wins ? y.a : x.a;
     r.s = x.s + y.s;
-    r.lo = fmaxf(x.lo, y.lo);
-    r.hi = fmaxf(x.hi, y.hi);
     return r;
 }
-__device__ __forceinline__ WarpStat warp_logit_stat16(const float (&u)[16], int v, float bw, bool bounds,
+__device__ __forceinline__ WarpStat warp_logit_stat16(const float (&u)[16], int v, float bwmax, bool bounds,
                                                       float cap = 0.f) {
     const int lane = threadIdx.x & 31;
     const bool fixed = cap > 0.f && cap < 43.f;
@@ -133,8 +130,6 @@ __device__ __forceinline__ WarpStat warp_logit_stat16(const float (&u)[16], int 
         x[j].m = u[j];
         x[j].a = valid ? v : 0x7fffffff;
         x[j].s = valid ? (fixed ? __expf(u[j] - cap) : 1.f) : 0.f;
-        x[j].lo = valid && bounds ? u[j] - bw : -INFINITY;
-        x[j].hi = valid && bounds ? u[j] + bw : -INFINITY;
     }
     StatAcc f;
     if (fixed) {
@@ -145,10 +140,10 @@ __device__ __forceinline__ WarpStat warp_logit_stat16(const float (&u)[16], int 
             for (int j = 0; j < half; ++j) {
                 const StatAcc give = upper ? x[j] : x[j + half];
                 const StatAcc keep = upper ? x[j + half] : x[j];
-                x[j] = stat_merge_fixed(keep, stat_shfl(give, bit, bounds));
+                x[j] = stat_merge_fixed(keep, stat_shfl(give, bit));
             }
         }
-        f = stat_merge_fixed(x[0], stat_shfl(x[0], 1, bounds));
+        f = stat_merge_fixed(x[0], stat_shfl(x[0], 1));
         if (f.m > -INFINITY) f.s *= __expf(cap - f.m);          // relative to the warp's maximum
     } else {
 #pragma unroll
@@ -158,17 +153,17 @@ __device__ __forceinline__ WarpStat warp_logit_stat16(const float (&u)[16], int 
             for (int j = 0; j < half; ++j) {
                 const StatAcc give = upper ? x[j] : x[j + half];
                 const StatAcc keep = upper ? x[j + half] : x[j];
-                x[j] = stat_merge(keep, stat_shfl(give, bit, bounds));
+                x[j] = stat_merge(keep, stat_shfl(give, bit));
             }
         }
-        f = stat_merge(x[0], stat_shfl(x[0], 1, bounds));
+        f = stat_merge(x[0], stat_shfl(x[0], 1));
     }
     WarpStat w;
     w.kmx = f.m > -INFINITY ? f2ord(f.m) : 0u;
     w.arg = f.m > -INFINITY ? f.a : 0x7fffffff;
     w.se = f.m > -INFINITY ? f.s : 0.f;
-    w.klo = f.lo > -INFINITY ? f2ord(f.lo) : 0u;
-    w.khi = f.hi > -INFINITY ? f2ord(f.hi) : 0u;
+    w.klo = bounds && f.m > -INFINITY ? f2ord(f.m - bwmax) : 0u;
+    w.khi = bounds && f.m > -INFINITY ? f2ord(f.m + bwmax) : 0u;
     return w;
 }
 

@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(128) tile_stats_kernel(const float* __restrict
         const int m = m0 + j;
         u[j] = (v < V && m < M) ? U[(int64_t)m * V + v] : -INFINITY;
     }
-    const WarpStat w = warp_logit_stat16(u, v, bw, bounds);
+    const float bwmax = bounds ? __uint_as_float(warp_max_u32(__float_as_uint(bw))) : 0.f;
+    const WarpStat w = warp_logit_stat16(u, v, bwmax, bounds);
     if ((lane & 1) == 0) q4[warp][warp_stat16_col(lane)] = w;
     __syncthreads();
     if (threadIdx.x < kStatRows && m0 + threadIdx.x < M) {
