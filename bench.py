@@ -50,8 +50,11 @@ def parse():
     ap.add_argument("--impl", default="dspark", choices=["dspark", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", default=None, choices=[None, "attention"],
-                    help="time one seam alone instead of the round (prints a case line, not the bench line)")
+    ap.add_argument("--case", default=None, choices=[None, "attention", "round"],
+                    help="attention: time the seam alone; round: run the workload's rounds (for profiling small "
+                         "cases with --layers / --vocab); both print a case line, not the bench line")
+    ap.add_argument("--layers", type=int, default=0, help="--case round: layers of the model (0: the workload's)")
+    ap.add_argument("--vocab", type=int, default=0, help="--case round: vocabulary of the model (0: the workload's)")
     return ap.parse_args()
 
 
@@ -561,12 +564,75 @@ def run_attention_case(args, wl):
                       "cache larger than L2 when its bytes exceed 126 MB"}), flush=True)
 
 
+def run_round_case(args, wl):
+    """The workload's step (append + draft rounds) on a model of the workload's shapes, with
+    the layer count and the vocabulary optionally reduced (a case small enough for a full ncu
+    capture of one launch): warm-up steps, then `--steps` steps timed together. Prints one JSON
+    case line (not the bench line: a reduced model is not the workload)."""
+    import dataclasses
+    import torch
+    import block_draft_model_dspark_b200 as dsp
+    from block_draft_model_dspark_b200 import build as libbuild
+    from synthetic import make_weights
+    libbuild.build()
+    m = wl.model
+    if args.layers:
+        m = m.replace(num_hidden_layers=args.layers)
+    if args.vocab:
+        m = m.replace(vocab_size=args.vocab, mask_token_id=args.vocab - 1)
+    wl = dataclasses.replace(wl, model=m)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    model = dsp.DsparkModel(m, {k: v.to(dev) for k, v in make_weights(m, wl.seed).items()})
+    plan = StepPlan(wl)
+    A, G = plan.A, m.block_size
+    pos0 = plan.pos0.to(dev)
+    cache = dsp.KvCache(model, A, plan.capacity)
+    init_hidden = plan.init_hidden.to(dev)
+    init_n = torch.tensor(plan.init_len, dtype=torch.int32, device=dev)
+    cache.set_lengths([0] * A)
+    model.dspark_append_context_kv(cache, init_hidden, init_n, pos0,
+                                   ws=model.workspace(model.project_workspace_bytes(A * int(init_hidden.shape[1]))))
+    del init_hidden
+    crop = torch.tensor(plan.crop, dtype=torch.int32, device=dev)
+    rounds = [{k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in r.items()} for r in plan.rounds]
+    outs = [{"tokens": torch.empty(A, G, dtype=torch.int32, device=dev),
+             "lengths": torch.empty(A, dtype=torch.int32, device=dev),
+             "conf": torch.empty(A, G, dtype=torch.float32, device=dev)} for _ in rounds]
+    aws = model.workspace(model.project_workspace_bytes(A * max(int(r["hidden"].shape[1]) for r in rounds)))
+    dws = model.workspace(model.draft_workspace_bytes(A, max(r["max_len"] for r in rounds)))
+
+    def step():
+        cache.len.copy_(crop, non_blocking=True)
+        for r, o in zip(rounds, outs):
+            model.dspark_append_context_kv(cache, r["hidden"], r["n_new"], pos0, ws=aws)
+            model.dspark_draft_rows(cache, r["anchors"], r["block_pos"], r["max_len"], o["tokens"], o["lengths"],
+                                    o["conf"], None, ws=dws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    assert model.dspark_read_device_status() == 0
+    print(json.dumps({"case": "round", "workload": wl.name, "layers": m.num_hidden_layers, "vocab": m.vocab_size,
+                      "ms_per_step": e0.elapsed_time(e1) / max(args.steps, 1), "steps": args.steps,
+                      "note": "reduced model for profiling; not the bench line"}), flush=True)
+
+
 def main():
     args = parse()
     from synthetic import WORKLOADS
     wl = WORKLOADS[args.workload]
     if args.case == "attention":
         run_attention_case(args, wl)
+        return
+    if args.case == "round":
+        run_round_case(args, wl)
         return
     if args.impl == "reference":
         run_reference(args, wl)
