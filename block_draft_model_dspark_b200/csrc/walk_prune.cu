@@ -24,6 +24,8 @@
 // win survives).
 #include <math.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "common.cuh"
 #include "logit_stats.cuh"
@@ -35,6 +37,7 @@ constexpr int kNormThreads = 256;              // 8 warps: one markov row each
 constexpr int kStatRows = 16;                  // positions per CTA of the statistics scan
 constexpr int kCandThreads = 256;
 constexpr int kMaxCandTiles = 256;             // tiles a position may scan (more: the full walk decides)
+constexpr int kHiKeep = 8;                     // tiles' hi values a candidate thread keeps in registers
 constexpr int kWalkThreads = 256;
 constexpr int kPerThread = kPruneCap / kWalkThreads;
 
@@ -136,27 +139,42 @@ __global__ void __launch_bounds__(kCandThreads) prune_candidates_kernel(const fl
     const int M = ts.M, nt = ts.n_tiles;
     if (m == 0 && tid == 0) *fail = 0;
     if (tid == 0) { s_nt = 0; s_cnt = 0; }
-    // row maximum (lowest index on ties) and T
+    // one pass over the tiles: row maximum (lowest index on ties), T, the logsumexp
+    // (tiles' sums merged online to the running maximum) and the tiles' hi kept for
+    // the candidate test (up to kHiKeep per thread; more are read again)
     uint32_t kbest = 0u, klo = 0u;
     int abest = 0x7fffffff;
-    for (int t = tid; t < nt; t += kCandThreads) {
-        const float mx = ts.mx[(int64_t)t * M + m];
+    float sm = -INFINITY, ss = 0.f;
+    float hi_keep[kHiKeep];
+#pragma unroll
+    for (int q = 0; q < kHiKeep; ++q) hi_keep[q] = -INFINITY;
+    for (int t = tid, q = 0; t < nt; t += kCandThreads, ++q) {
+        const int64_t o = (int64_t)t * M + m;
+        const float mx = ts.mx[o];
+        const int a = ts.arg[o];
+        const float se_t = ts.se[o];
+        const float lo = markov ? ts.lo[o] : -INFINITY;
+        const float hi = markov ? ts.hi[o] : -INFINITY;
         const uint32_t k = mx > -INFINITY ? f2ord(mx) : 0u;
-        const int a = ts.arg[(int64_t)t * M + m];
         if (k > kbest || (k == kbest && a < abest)) { kbest = k; abest = a; }
-        if (markov) {
-            const float lo = ts.lo[(int64_t)t * M + m];
-            if (lo > -INFINITY) klo = max(klo, f2ord(lo));
+        if (lo > -INFINITY) klo = max(klo, f2ord(lo));
+        if (mx > -INFINITY) {
+            if (mx > sm) { ss = ss * __expf(sm - mx) + se_t; sm = mx; }
+            else ss += se_t * __expf(mx - sm);
         }
+#pragma unroll
+        for (int qq = 0; qq < kHiKeep; ++qq) if (qq == q) hi_keep[qq] = hi;
     }
+    // the CTA's maximum / argmax, T and logsumexp: warps, then warp 0 over the warps
     const uint32_t wk = warp_max_u32(kbest);
     int wa = kbest == wk ? abest : 0x7fffffff;
     for (int o = 16; o > 0; o >>= 1) wa = min(wa, __shfl_xor_sync(0xffffffffu, wa, o));
-    if (lane == 0) { s_key[warp] = wk; s_arg[warp] = wa; }
-    const float Tm_partial = klo ? ord2f(klo) : -INFINITY;
-    float Tm = Tm_partial;
+    float Tm = klo ? ord2f(klo) : -INFINITY;
     for (int o = 16; o > 0; o >>= 1) Tm = fmaxf(Tm, __shfl_xor_sync(0xffffffffu, Tm, o));
-    if (lane == 0) s_red[warp] = Tm;
+    const float wmax = wk ? ord2f(wk) : -INFINITY;
+    float wsum = sm > -INFINITY ? ss * __expf(sm - wmax) : 0.f;
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    if (lane == 0) { s_key[warp] = wk; s_arg[warp] = wa; s_red[warp] = Tm; s_red[16 + warp] = wsum; }
     __syncthreads();
     uint32_t rk = 0u;
     int ra = 0x7fffffff;
@@ -166,15 +184,10 @@ __global__ void __launch_bounds__(kCandThreads) prune_candidates_kernel(const fl
     Tm = -INFINITY;
     for (int w = 0; w < kCandThreads / 32; ++w) Tm = fmaxf(Tm, s_red[w]);
     const float rmax = rk ? ord2f(rk) : -INFINITY;
-    __syncthreads();
-    // logsumexp: the tiles' sums rescaled to the row maximum
     float se = 0.f;
-    if (rk)
-        for (int t = tid; t < nt; t += kCandThreads) {
-            const float mx = ts.mx[(int64_t)t * M + m];
-            if (mx > -INFINITY) se += ts.se[(int64_t)t * M + m] * __expf(mx - rmax);
-        }
-    se = block_sum(se, s_red);
+    for (int w = 0; w < kCandThreads / 32; ++w)
+        if (s_key[w]) se += s_red[16 + w] * __expf(ord2f(s_key[w]) - rmax);
+    __syncthreads();
     if (!markov) {
         if (tid == 0) {
             tokens[m] = ra == 0x7fffffff ? 0 : ra;
@@ -192,8 +205,12 @@ __global__ void __launch_bounds__(kCandThreads) prune_candidates_kernel(const fl
         return;
     }
     const float thr = Tm - (1e-3f + 1e-3f * fabsf(Tm));   // far above the fp32 rounding of U + bias
-    for (int t = tid; t < nt; t += kCandThreads) {
-        if (ts.hi[(int64_t)t * M + m] >= thr) {
+    for (int t = tid, q = 0; t < nt; t += kCandThreads, ++q) {
+        float hi = -INFINITY;
+#pragma unroll
+        for (int qq = 0; qq < kHiKeep; ++qq) if (qq == q) hi = hi_keep[qq];
+        if (q >= kHiKeep) hi = ts.hi[(int64_t)t * M + m];
+        if (hi >= thr) {
             const int i = atomicAdd(&s_nt, 1);
             if (i < kMaxCandTiles) s_tiles[i] = t;
         }
@@ -301,6 +318,165 @@ __global__ void __launch_bounds__(kWalkThreads) prune_walk_kernel(const float* _
     }
 }
 
+// ------------------------------------------------------------------ the walk on one warp
+// The same walk for dense bf16 Markov tables, on one warp per request row: the
+// lists are short (a handful of candidates per position once the norm bound
+// has pruned the vocabulary), so every position's count and list are read once
+// and, when all of a row's candidates fit (at most `cap`), their w2 rows, w1
+// rows and U values are copied into shared memory before the first step; a step
+// is then warp-synchronous (lane i evaluates candidates i, i + 32, ...; a warp
+// argmax; the winner's w1 row becomes the next e), with no block barrier. Rows
+// whose lists do not fit read the tables from global memory at each step.
+// Values and the summation order (fp32, j ascending) are those of
+// prune_walk_kernel.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+                 "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+                 "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <int R>
+__global__ void __launch_bounds__(32) prune_walk_warp_kernel(const float* __restrict__ U, const bf16* __restrict__ w1,
+                                                             const bf16* __restrict__ w2, int r,
+                                                             const int32_t* __restrict__ anchors,
+                                                             const int* __restrict__ cnt, const int* __restrict__ list,
+                                                             int G, int V, int cap, int32_t* __restrict__ tokens,
+                                                             int* __restrict__ fail, int32_t* __restrict__ status) {
+    extern __shared__ __align__(16) uint8_t wsm[];
+    constexpr int chunks = R / 8;                   // 16-byte chunks of a row (r == R)
+    const int rowb = R * 2;
+    const int sstride = 2 * rowb;                   // a slot: w2 row, w1 row
+    int* s_cnt = reinterpret_cast<int*>(wsm);       // [G]
+    int* s_off = s_cnt + 64;                        // [G + 1] exclusive prefix of the counts
+    int* s_v = s_off + 72;                          // [cap]
+    uint8_t* s_rows = reinterpret_cast<uint8_t*>(s_v + cap);     // [cap] slots
+    float* s_u = reinterpret_cast<float*>(s_rows + (size_t)cap * sstride);   // [cap]
+    float* s_e = s_u + cap;                         // [r]
+    pdl_trigger();
+    pdl_wait();
+    const int b = blockIdx.x, lane = threadIdx.x;
+    int prev = anchors[b];
+    if (prev < 0 || prev >= V) {
+        if (lane == 0) atomicOr(status, DSPARK_DEV_BAD_TOKEN);
+        prev = min(max(prev, 0), V - 1);
+    }
+    // counts and their prefix (G <= 64: two per lane)
+    bool bad = false;
+    int c0 = 0, c1 = 0;
+    if (lane < G) { c0 = cnt[b * G + lane]; bad |= c0 <= 0 || c0 > kPruneCap; }
+    if (lane + 32 < G) { c1 = cnt[b * G + lane + 32]; bad |= c1 <= 0 || c1 > kPruneCap; }
+    if (__any_sync(0xffffffffu, bad)) {             // a list empty or too long: the full walk decides
+        if (lane == 0) atomicOr(fail, 1);
+        return;
+    }
+    int x0 = c0, x1 = c1;                           // inclusive scans of the two halves
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
+        if (lane >= o) { x0 += y0; x1 += y1; }
+    }
+    const int tot0 = __shfl_sync(0xffffffffu, x0, 31);
+    if (lane < G) { s_cnt[lane] = c0; s_off[lane] = x0 - c0; }
+    if (lane + 32 < G) { s_cnt[lane + 32] = c1; s_off[lane + 32] = tot0 + x1 - c1; }
+    const int total = tot0 + __shfl_sync(0xffffffffu, x1, 31);
+    if (lane == 0) s_off[G] = total;
+    __syncwarp();
+    const bool resident = total <= cap;
+    if (resident) {
+        // every candidate of the row, flattened (slot t = offset of its position + its list index):
+        // lane l takes slots l, l + 32, ..., so all list reads go out at once; then its rows and U
+        // value by cp.async
+        for (int t = lane; t < total; t += 32) {
+            int k = 0;
+            while (k + 1 < G && s_off[k + 1] <= t) ++k;     // the position holding slot t
+            const int i = t - s_off[k], m = b * G + k;
+            const int v = min(max(list[(int64_t)m * kPruneCap + i], 0), V - 1);   // (in range; clamped for safety)
+            s_v[t] = v;
+            uint8_t* slot = s_rows + (size_t)t * sstride;
+            const uint4* g2 = reinterpret_cast<const uint4*>(w2 + (int64_t)v * R);
+            const uint4* g1 = reinterpret_cast<const uint4*>(w1 + (int64_t)v * R);
+#pragma unroll
+            for (int ch = 0; ch < chunks; ++ch) {
+                cp_async16(slot + ch * 16, g2 + ch);
+                cp_async16(slot + rowb + ch * 16, g1 + ch);
+            }
+            cp_async4(s_u + t, U + (int64_t)m * V + v);
+        }
+    }
+    // e = w1[anchor]
+#pragma unroll
+    for (int j = lane; j < R; j += 32) s_e[j] = __bfloat162float(w1[(int64_t)prev * R + j]);
+    cp_async_wait_all();
+    __syncwarp();
+    for (int k = 0; k < G; ++k) {
+        const int m = b * G + k;
+        const int c = s_cnt[k], off = s_off[k];
+        float val = -INFINITY;
+        int idx = 0x7fffffff, slot_of = -1;
+        if (resident && c == 1) {
+            // one candidate: it is the step's argmax whatever its bias (the list keeps every entry
+            // that could win; a single valid entry wins)
+            const int v = s_v[off];
+            const float u = s_u[off];
+            if (v >= 0 && v < V && u == u) { idx = v; slot_of = off; val = 0.f; }   // (a NaN value never wins)
+        } else {
+        float ev[R];                                 // e in registers for the dot products
+#pragma unroll
+        for (int j4 = 0; j4 < R / 4; ++j4) {
+            const float4 q = reinterpret_cast<const float4*>(s_e)[j4];
+            ev[4 * j4] = q.x; ev[4 * j4 + 1] = q.y; ev[4 * j4 + 2] = q.z; ev[4 * j4 + 3] = q.w;
+        }
+        for (int i = lane; i < c; i += 32) {
+            const int v = resident ? s_v[off + i] : list[(int64_t)m * kPruneCap + i];
+            if (v < 0 || v >= V) continue;
+            const uint4* row = resident ? reinterpret_cast<const uint4*>(s_rows + (size_t)(off + i) * sstride)
+                                        : reinterpret_cast<const uint4*>(w2 + (int64_t)v * r);
+            uint4 q[chunks];
+#pragma unroll
+            for (int ch = 0; ch < chunks; ++ch) q[ch] = row[ch];
+            float acc = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < chunks; ++ch) {
+                const uint32_t w[4] = {q[ch].x, q[ch].y, q[ch].z, q[ch].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc = fmaf(__uint_as_float(w[j] << 16), ev[ch * 8 + 2 * j], acc);
+                    acc = fmaf(__uint_as_float(w[j] & 0xffff0000u), ev[ch * 8 + 2 * j + 1], acc);
+                }
+            }
+            const float x = (resident ? s_u[off + i] : U[(int64_t)m * V + v]) + acc;
+            if (x > val || (x == val && v < idx)) { val = x; idx = v; slot_of = off + i; }
+        }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, val, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, idx, o);
+            const int os = __shfl_xor_sync(0xffffffffu, slot_of, o);
+            if (ov > val || (ov == val && oi < idx)) { val = ov; idx = oi; slot_of = os; }
+        }
+        if (idx == 0x7fffffff) {                     // uniform over the warp
+            if (lane == 0) atomicOr(fail, 1);
+            return;
+        }
+        if (lane == 0) tokens[m] = idx;
+        if (k + 1 < G) {
+            __syncwarp();                            // every lane is done reading e
+            if (resident) {
+                const __nv_bfloat16* row1 = reinterpret_cast<const __nv_bfloat16*>(s_rows + (size_t)slot_of * sstride + rowb);
+                for (int j = lane; j < R; j += 32) s_e[j] = __bfloat162float(row1[j]);
+            } else {
+                for (int j = lane; j < R; j += 32) s_e[j] = __bfloat162float(w1[(int64_t)idx * R + j]);
+            }
+            __syncwarp();
+        }
+    }
+}
+
 }  // namespace
 
 bool walk_prune_model_supported(const Dims& d) { return d.r > 0 && d.r <= 256; }
@@ -334,6 +510,23 @@ cudaError_t launch_walk_prune(const dspark_model* m, const float* U, const TileS
     if (e != cudaSuccess || !markov) return e;
     MatRef w1{};
     w1.w = m->w1; w1.n = d.V; w1.k = d.r;
+    // dense bf16 tables: the walk with prefetched rows (a position's candidates in shared
+    // memory when there are at most `cap` of them)
+    const bool warp_walk = !m->w2.quant && d.dtype == DSPARK_DTYPE_BF16 && d.gamma <= 64 &&
+                           (d.r == 16 || d.r == 32 || d.r == 64 || d.r == 128);
+    if (warp_walk) {
+        // a row's candidates stay in shared memory when at most `cap` of them: 64 KB of rows
+        const size_t sstride = 4 * (size_t)d.r;
+        const int cap = std::max(32, (int)((64 * 1024) / (sstride + 8)) / 32 * 32);
+        const size_t smem = (64 + 72) * 4 + (size_t)cap * (4 + sstride + 4) + 4 * (size_t)d.r;
+        auto kern = d.r == 16 ? prune_walk_warp_kernel<16> : d.r == 32 ? prune_walk_warp_kernel<32>
+                  : d.r == 64 ? prune_walk_warp_kernel<64> : prune_walk_warp_kernel<128>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kern, dim3(A), dim3(32), smem, s, U, static_cast<const bf16*>(m->w1),
+                          static_cast<const bf16*>(m->w2.w), d.r, anchors, ps.cnt, ps.list, d.gamma, d.V, cap, tokens,
+                          ps.fail, m->ws.status);
+    }
     return launch_pdl(prune_walk_kernel, dim3(A), dim3(kWalkThreads), 0, s, U, w1, m->w2, d.dtype, d.group, d.r,
                       anchors, ps.cnt, ps.list, d.gamma, d.V, tokens, ps.fail, m->ws.status);
 }
