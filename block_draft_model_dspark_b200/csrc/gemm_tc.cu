@@ -22,10 +22,10 @@
 // rate, not HBM, bounded the weight stream at one request per 4 KB of X or
 // 16 KB of W.
 //
-// Roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
-// MMAs, warps 2-9 drain accumulators (TMEM lane quadrant = warp % 4; warps w
-// and w + 4 take alternate 16-column chunks); with 4-bit weights warps 2-5
-// drain and warps 6-9 dequantize the weight tiles.
+// Roles (448 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// MMAs, warps 2-13 drain accumulators (TMEM lane quadrant = warp % 4; warps w,
+// w + 4 and w + 8 take every third 16-column chunk); with 4-bit weights (320
+// threads) warps 2-5 drain and warps 6-9 dequantize the weight tiles.
 // Accumulators are double-buffered in TMEM so the epilogue of one tile
 // overlaps the MMAs of the next.
 //
@@ -60,11 +60,12 @@ constexpr int BM = 128;            // weight rows per tile (MMA M)
 constexpr int BK = 64;             // K elements per K block: one 128-byte swizzle row
 constexpr int kThreads = 192;      // TMA, MMA and four epilogue warps
 constexpr int kConvThreads = 128;  // the weight-transform warps (one weight row each)
-// Epilogue warps: eight (two per TMEM lane quadrant, taking alternate 16-column
-// chunks) for the 16-bit weight formats, whose drain of softcapped logits and
-// their statistics otherwise outlasted a tile's MMAs; four beside the 4-bit
-// dequantizing warps.
-__host__ __device__ constexpr int epi_warps_for(int wfmt) { return wfmt == kWQ4AsF16 ? 4 : 8; }
+// Epilogue warps: twelve (three per TMEM lane quadrant, taking every third
+// 16-column chunk) for the 16-bit weight formats, whose drain of softcapped
+// logits and their statistics otherwise outlasts a tile's MMAs (eight measured
+// 4% slower at the lm-head of 512 positions; 448 threads leave 146 registers a
+// thread); four beside the 4-bit dequantizing warps.
+__host__ __device__ constexpr int epi_warps_for(int wfmt) { return wfmt == kWQ4AsF16 ? 4 : 12; }
 constexpr int kABytes = BM * BK * 2;   // one K block of weights (16 KB)
 // threads of a launch: the weight-transform formats add the converter warps (warps 6-9)
 __host__ __device__ constexpr int threads_for(int wfmt) {

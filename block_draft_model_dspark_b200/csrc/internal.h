@@ -128,15 +128,21 @@ struct PartView {
 
     // Four consecutive columns n .. n + 3 of row m (n % 4 == 0; mode 1: within one
     // 128-column block, so they share a tile), each the sum of its partials in order.
-    static constexpr int kMax4 = 4;            // partials load4 keeps in flight (more are read in finish4)
-    struct Pending4 {
-        float4 x[kMax4];
+    // KMAX: partials load4 keeps in flight (more are read in finish4); a kernel with
+    // few columns per thread and many partials per tile raises it, one with many
+    // columns lowers it to keep its registers.
+    template <int KMAX>
+    struct Pending4T {
+        float4 x[KMAX];
         int cnt;
         const float* rest;
         int64_t step;
     };
-    __device__ __forceinline__ Pending4 load4(int m, int64_t n) const {
-        Pending4 q;
+    static constexpr int kMax4 = 4;
+    using Pending4 = Pending4T<kMax4>;
+    template <int KMAX = kMax4>
+    __device__ __forceinline__ Pending4T<KMAX> load4(int m, int64_t n) const {
+        Pending4T<KMAX> q;
         const float* base;
         if (mode == 0) {
             q.cnt = S; q.step = stride;
@@ -150,16 +156,17 @@ struct PartView {
             base = p + (((int64_t)store * P) * BN + ml) * 128 + nl;
         }
 #pragma unroll
-        for (int s = 0; s < kMax4; ++s)
+        for (int s = 0; s < KMAX; ++s)
             q.x[s] = s < q.cnt ? *reinterpret_cast<const float4*>(base + s * q.step) : make_float4(0.f, 0.f, 0.f, 0.f);
         q.rest = base;
         return q;
     }
-    __device__ __forceinline__ float4 finish4(const Pending4& q) const {
+    template <int KMAX>
+    __device__ __forceinline__ float4 finish4(const Pending4T<KMAX>& q) const {
         float4 v = q.x[0];
 #pragma unroll
-        for (int s = 1; s < kMax4; ++s) { v.x += q.x[s].x; v.y += q.x[s].y; v.z += q.x[s].z; v.w += q.x[s].w; }
-        for (int s = kMax4; s < q.cnt; ++s) {
+        for (int s = 1; s < KMAX; ++s) { v.x += q.x[s].x; v.y += q.x[s].y; v.z += q.x[s].z; v.w += q.x[s].w; }
+        for (int s = KMAX; s < q.cnt; ++s) {
             const float4 t = *reinterpret_cast<const float4*>(q.rest + s * q.step);
             v.x += t.x; v.y += t.y; v.z += t.z; v.w += t.w;
         }

@@ -337,13 +337,13 @@ __global__ void __launch_bounds__(512) residual_epilogue_kernel(PartView part, i
     constexpr int kBatch = G4 < 2 ? G4 : 2;
 #pragma unroll
     for (int g0 = 0; g0 < G4; g0 += kBatch) {
-        PartView::Pending4 q[kBatch];
+        PartView::Pending4T<(PER == 4 ? 8 : 4)> q[kBatch];   // few columns a thread (small M): the many partials at once
 #pragma unroll
         for (int gb = 0; gb < kBatch; ++gb) {
             const int g = g0 + gb;
             const int j = j0 + g * blockDim.x * 4;
             const bool in = j < H;
-            q[gb] = part.load4(m, in ? j : 0);
+            q[gb] = part.load4<(PER == 4 ? 8 : 4)>(m, in ? j : 0);
             const float4 hh = in ? *reinterpret_cast<const float4*>(h + (int64_t)m * H + j) : make_float4(0.f, 0.f, 0.f, 0.f);
             hv[g * 4] = hh.x; hv[g * 4 + 1] = hh.y; hv[g * 4 + 2] = hh.z; hv[g * 4 + 3] = hh.w;
         }
@@ -442,21 +442,22 @@ __global__ void __launch_bounds__(kResThreads, 4) residual_row_kernel(PartView p
 
 // grid (ceil(I / (4 kGuGroups * 256)), M), 256 threads: thread t of CTA x owns the
 // kGuGroups 4-column groups x * 256 kGuGroups + t + 256 j; all their gate and up
-// loads go out before the first is used (two groups measured slower: the registers
-// of their pending partials halved the resident threads).
+// loads go out before the first is used (two groups per thread, with two or four
+// partials in flight each, measured no faster at 512 rows and slower at 16).
 constexpr int kGuGroups = 1;
+constexpr int kGuPartials = 4;      // partials in flight per load
 __global__ void __launch_bounds__(256) gu_epilogue_kernel(PartView part, int M, int I, ActBuf act) {
     pdl_trigger();
     pdl_wait();
     const int m = blockIdx.y;
     const int64_t g0 = (int64_t)blockIdx.x * blockDim.x * kGuGroups + threadIdx.x;
-    PartView::Pending4 qg[kGuGroups], qu[kGuGroups];
+    PartView::Pending4T<kGuPartials> qg[kGuGroups], qu[kGuGroups];
 #pragma unroll
     for (int j = 0; j < kGuGroups; ++j) {
         const int64_t i = (g0 + (int64_t)j * blockDim.x) * 4;
         if (i < I) {
-            qg[j] = part.load4(m, i);
-            qu[j] = part.load4(m, I + i);
+            qg[j] = part.load4<kGuPartials>(m, i);
+            qu[j] = part.load4<kGuPartials>(m, I + i);
         }
     }
 #pragma unroll
