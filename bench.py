@@ -55,6 +55,9 @@ def parse():
                          "cases with --layers / --vocab); both print a case line, not the bench line")
     ap.add_argument("--layers", type=int, default=0, help="--case round: layers of the model (0: the workload's)")
     ap.add_argument("--vocab", type=int, default=0, help="--case round: vocabulary of the model (0: the workload's)")
+    ap.add_argument("--kv-cache", default="kv", choices=["kv", "v_only"],
+                    help="context cache layout: kv stores k and v (the default: the faster round); v_only stores v "
+                         "alone (half the cache; the attention rebuilds k = rope(v * k_norm))")
     return ap.parse_args()
 
 
@@ -110,6 +113,14 @@ class StepPlan:
                                 "anchors": inp["anchors"], "block_pos": inp["block_pos"], "max_len": max(lens)})
             self.append_desc = f"append {G} accepted rows per row + draft"
         self.tokens_per_step = len(self.rounds) * self.A * G
+
+
+def use_v_only(args, m) -> bool:
+    """--kv-cache v_only: needs a bf16 model on the tensor-core attention (head_dim % 64 == 0, <= 256)."""
+    ok = m.dtype == "bf16" and m.global_head_dim % 64 == 0 and m.global_head_dim <= 256
+    if args.kv_cache == "v_only" and not ok:
+        raise SystemExit(f"--kv-cache v_only: unsupported for {m}")
+    return args.kv_cache == "v_only"
 
 
 def workload_config(wl, plan=None):
@@ -323,7 +334,8 @@ def run_dspark(args, wl):
     pos0 = plan.pos0.to(dev)
 
     # the initial context, projected once into the cache (timed on its own)
-    cache = dsp.KvCache(model, A, plan.capacity)
+    v_only = use_v_only(args, m)
+    cache = dsp.KvCache(model, A, plan.capacity, v_only=v_only, pos0=pos0 if v_only else None)
     init_hidden = plan.init_hidden.to(dev)
     init_n = torch.tensor(plan.init_len, dtype=torch.int32, device=dev)
     pws = model.workspace(model.project_workspace_bytes(A * int(init_hidden.shape[1])))
@@ -489,6 +501,8 @@ def run_dspark(args, wl):
                 for k, v in kinds.items()}
         cfg = workload_config(wl, plan)
         cfg.update({"parallelism": f"dp{world} (every GPU serves the workload's rows; no collective)",
+                    "kv_cache": "v_only (v alone; the attention rebuilds k = rope(v * k_norm))" if v_only
+                    else "k and v",
                     "l2": "inputs larger than L2: 3.7 GB of dense weights (1.04 GB at 4 bits) streamed per round",
                     "round_us": round_ms * 1e3, "project_full_context_us": project_full_ms * 1e3,
                     "project_full_context_rows": project_rows,
@@ -587,7 +601,8 @@ def run_round_case(args, wl):
     plan = StepPlan(wl)
     A, G = plan.A, m.block_size
     pos0 = plan.pos0.to(dev)
-    cache = dsp.KvCache(model, A, plan.capacity)
+    v_only = use_v_only(args, m)
+    cache = dsp.KvCache(model, A, plan.capacity, v_only=v_only, pos0=pos0 if v_only else None)
     init_hidden = plan.init_hidden.to(dev)
     init_n = torch.tensor(plan.init_len, dtype=torch.int32, device=dev)
     cache.set_lengths([0] * A)
@@ -620,6 +635,7 @@ def run_round_case(args, wl):
     torch.cuda.synchronize()
     assert model.dspark_read_device_status() == 0
     print(json.dumps({"case": "round", "workload": wl.name, "layers": m.num_hidden_layers, "vocab": m.vocab_size,
+                      "kv_cache": "v_only" if v_only else "kv",
                       "ms_per_step": e0.elapsed_time(e1) / max(args.steps, 1), "steps": args.steps,
                       "note": "reduced model for profiling; not the bench line"}), flush=True)
 

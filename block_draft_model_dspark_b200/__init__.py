@@ -68,7 +68,7 @@ class dspark_weights(ctypes.Structure):
 
 class dspark_kv_cache(ctypes.Structure):
     _fields_ = [("k", c_vp), ("v", c_vp), ("len", c_i32p), ("len_host", c_i32p), ("batch", c_i32),
-                ("capacity", c_i32)]
+                ("capacity", c_i32), ("pos0", c_i32p)]
 
 
 _PROTOTYPES = {
@@ -210,14 +210,24 @@ def _matrix(tensors: Dict, name: str) -> dspark_matrix:
 
 class KvCache:
     """Caller-owned context K/V (``dspark_kv_cache``): k, v [Lyr, batch, capacity, nKv, hd] in the
-    model's KV dtype (``dspark_kv_dtype``: fp16 for a bf16 model), len [batch]."""
+    model's KV dtype (``dspark_kv_dtype``: fp16 for a bf16 model), len [batch].
 
-    def __init__(self, model: "DsparkModel", batch: int, capacity: int, k=None, v=None):
+    ``v_only=True`` keeps v alone (k is None; the attention rebuilds k = rope(v * k_norm) at the
+    positions ``pos0[b] + t``): ``pos0`` is then the int32 device tensor [batch] of the absolute
+    position of each batch row's cache row 0."""
+
+    def __init__(self, model: "DsparkModel", batch: int, capacity: int, k=None, v=None, v_only: bool = False,
+                 pos0=None):
         import torch
         s = model.shape
         shp = (s.num_hidden_layers, batch, capacity, s.num_global_key_value_heads, s.global_head_dim)
-        self.k = k if k is not None else torch.empty(shp, dtype=model.kv_torch_dtype, device=model.device)
+        self.v_only = bool(v_only)
+        if self.v_only:
+            self.k = None
+        else:
+            self.k = k if k is not None else torch.empty(shp, dtype=model.kv_torch_dtype, device=model.device)
         self.v = v if v is not None else torch.empty(shp, dtype=model.kv_torch_dtype, device=model.device)
+        self.pos0 = pos0
         self.len = torch.zeros(batch, dtype=torch.int32, device=model.device)
         self.len_host = (ctypes.c_int32 * batch)()
         self.batch, self.capacity = batch, capacity
@@ -230,7 +240,10 @@ class KvCache:
 
     def struct(self) -> dspark_kv_cache:
         c = dspark_kv_cache()
-        c.k, c.v = self.k.data_ptr(), self.v.data_ptr()
+        c.k = self.k.data_ptr() if self.k is not None else None
+        c.v = self.v.data_ptr()
+        if self.pos0 is not None:
+            c.pos0 = ctypes.cast(ctypes.c_void_p(self.pos0.data_ptr()), c_i32p)
         c.len = ctypes.cast(ctypes.c_void_p(self.len.data_ptr()), c_i32p)
         c.len_host = ctypes.cast(self.len_host, c_i32p)
         c.batch, c.capacity = self.batch, self.capacity
@@ -315,7 +328,7 @@ class DsparkModel:
         B, L = int(hidden.shape[0]), int(hidden.shape[1])
         ws = ws if ws is not None else self.workspace(self.project_workspace_bytes(B * L))
         _check(get_lib().dspark_project_context_kv(self.handle, hidden.data_ptr(), B, L, static_pos, _ptr(pos0),
-                                             k_out.data_ptr(), v_out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                             _ptr(k_out), v_out.data_ptr(), ws.data_ptr(), ws.numel(),
                                              _stream_ptr(stream)))
 
     def dspark_append_context_kv(self, cache: KvCache, hidden, n_new, pos0, ws=None, stream=None):

@@ -538,7 +538,7 @@ int dspark_project_context_kv(const dspark_model* m, const void* hidden, int32_t
     if (B < 0 || L < 0) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "B and L must be >= 0");
     if ((int64_t)B * L == 0) return DSPARK_OK;
     if ((int64_t)B * L > (int64_t)1 << 30) DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "B * L above 2^30 rows");
-    if (!hidden || !k_out || !v_out || !ws) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "hidden, k_out, v_out and ws must be non-NULL");
+    if (!hidden || !v_out || !ws) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "hidden, v_out and ws must be non-NULL");
     if (!aligned16(hidden) || !aligned16(k_out) || !aligned16(v_out)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "buffers must be 16-byte aligned");
     if (!pos0 && static_pos < 0) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "static_pos must be >= 0");
     const ProjectPlan pp = plan_project(m, (int64_t)B * L);
@@ -558,8 +558,10 @@ int dspark_append_context_kv(const dspark_model* m, const void* hidden, int32_t 
     if (B <= 0 || B > kMaxAppendBatch) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "cache.batch must be in [1, 4096]");
     if (Lnew_max < 0 || Lnew_max > cache->capacity) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "Lnew_max must be in [0, cache.capacity]");
     if ((int64_t)B * Lnew_max > (int64_t)1 << 30) DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "batch * Lnew_max above 2^30 rows");
-    if (!n_new || !pos0 || !cache->len || !cache->k || !cache->v)
-        DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "n_new, pos0 and the cache's k, v, len must be non-NULL");
+    if (!n_new || !pos0 || !cache->len || !cache->v)
+        DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "n_new, pos0 and the cache's v, len must be non-NULL");
+    if (!cache->k && !tc::vonly_attention_supported(m))
+        DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "a V-only cache (k = NULL) needs the tensor-core attention (bf16 model)");
     if (!aligned16(cache->k) || !aligned16(cache->v)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "cache k / v must be 16-byte aligned");
     if (Lnew_max == 0) return DSPARK_OK;
     if (!hidden || !ws || !aligned16(hidden)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "hidden and ws must be non-NULL, 16-byte aligned");
@@ -588,12 +590,21 @@ size_t dspark_draft_workspace_bytes(const dspark_model* m, int32_t A, int32_t ma
     return plan_draft(m, A, max_ctx_len).total;
 }
 
-static int check_cache(const dspark_model* m, const dspark_kv_cache* c, int A, int maxL, std::string* why) {
-    if (!c || !c->k || !c->v || !c->len) { *why = "cache and its k, v, len must be non-NULL"; return DSPARK_ERR_INVALID_ARGUMENT; }
+// allow_vonly: the call can read a V-only cache (k = NULL, K rebuilt from v at pos0[b] + t)
+static int check_cache(const dspark_model* m, const dspark_kv_cache* c, int A, int maxL, std::string* why,
+                       bool allow_vonly) {
+    if (!c || !c->v || !c->len) { *why = "cache and its v, len must be non-NULL"; return DSPARK_ERR_INVALID_ARGUMENT; }
+    if (!c->k) {
+        if (!allow_vonly) { *why = "the attend seam takes explicit keys: a V-only cache (k = NULL) is refused"; return DSPARK_ERR_INVALID_ARGUMENT; }
+        if (!tc::vonly_attention_supported(m)) {
+            *why = "a V-only cache (k = NULL) needs the tensor-core attention (bf16 model)";
+            return DSPARK_ERR_UNSUPPORTED;
+        }
+        if (!c->pos0) { *why = "a V-only cache (k = NULL) needs pos0"; return DSPARK_ERR_INVALID_ARGUMENT; }
+    }
     if (A <= 0 || A > c->batch) { *why = "A must be in [1, cache.batch]"; return DSPARK_ERR_INVALID_ARGUMENT; }
     if (maxL < 0 || maxL > c->capacity) { *why = "max_ctx_len must be in [0, cache.capacity]"; return DSPARK_ERR_INVALID_ARGUMENT; }
     if (!aligned16(c->k) || !aligned16(c->v)) { *why = "cache k / v must be 16-byte aligned"; return DSPARK_ERR_INVALID_ARGUMENT; }
-    (void)m;
     return DSPARK_OK;
 }
 
@@ -605,7 +616,7 @@ static AttnArgs attn_args(const dspark_model* m, const DraftPlan& p, void* ws, c
     AttnArgs a{};
     a.q = q; a.kb = kb; a.vb = vb; a.out = out;
     a.q_dtype = q_dtype; a.out_dtype = out_dtype;
-    a.kc = static_cast<const char*>(c->k) + layer_bytes * layer;
+    a.kc = c->k ? static_cast<const char*>(c->k) + layer_bytes * layer : nullptr;   // NULL: V-only
     a.vc = static_cast<const char*>(c->v) + layer_bytes * layer;
     a.len = c->len; a.capacity = c->capacity; a.batch = c->batch;
     a.part_o = at<float>(ws, p.part_o); a.part_ml = at<float>(ws, p.part_ml);
@@ -619,7 +630,7 @@ static AttnArgs attn_args(const dspark_model* m, const DraftPlan& p, void* ws, c
     else
         keys += (double)A * c->capacity;
     const double qo = (double)A * d.gamma * d.nH * d.hd * (esize(q_dtype) + esize(out_dtype));
-    a.kv_bytes = keys * d.nKv * d.hd * 2.0 * es + qo;
+    a.kv_bytes = keys * d.nKv * d.hd * (c->k ? 2.0 : 1.0) * es + qo;   // a V-only cache streams v alone
     a.flops = 4.0 * (double)d.nH * d.gamma * d.hd * keys;
     return a;
 }
@@ -628,7 +639,7 @@ int dspark_attend(const dspark_model* m, int32_t layer, const dspark_kv_cache* c
                   const void* v_blk, void* out, int32_t A, int32_t max_ctx_len, void* ws, size_t ws_bytes, void* stream) {
     if (!m) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "model is NULL");
     std::string why;
-    int rc = check_cache(m, cache, A, max_ctx_len, &why);
+    int rc = check_cache(m, cache, A, max_ctx_len, &why, false);
     if (rc) DSPARK_FAIL(rc, why);
     if (layer < 0 || layer >= m->d.Lyr) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "layer out of range");
     if (!q || !k_blk || !v_blk || !out || !ws) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "q, k_blk, v_blk, out and ws must be non-NULL");
@@ -647,7 +658,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
                       int32_t* lengths, float* base_logits, void* ws, size_t ws_bytes, void* stream) {
     if (!m) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "model is NULL");
     std::string why;
-    int rc = check_cache(m, cache, A, max_ctx_len, &why);
+    int rc = check_cache(m, cache, A, max_ctx_len, &why, true);
     if (rc) DSPARK_FAIL(rc, why);
     if (!anchors || !block_pos || !tokens || !lengths || !ws)
         DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "anchors, block_pos, tokens, lengths and ws must be non-NULL");
@@ -690,6 +701,7 @@ int dspark_draft_rows(const dspark_model* m, const dspark_kv_cache* cache, const
         if (e == cudaSuccess) {
             AttnArgs a = attn_args(m, p, ws, cache, l, A, q, kb, vb, ao.f32, d.kv_dtype, DSPARK_DTYPE_F32);
             a.out_hi = ao.hi; a.out_lo = ao.lo;
+            a.pos0 = cache->pos0; a.block_pos = block_pos; a.k_norm = L.k_norm;
             if (p.tc && !m->attn_dump) a.out = nullptr;    // the o GEMM reads the fp16 form only
             e = run_attention(m, a, s);
         }

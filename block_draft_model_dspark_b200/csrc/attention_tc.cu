@@ -21,8 +21,8 @@
 //   O += P V   -> TMEM (hd columns), P fp16 from shared memory (K-major,
 //                 128-byte swizzle), V as an MN-major operand
 // TMEM columns: S buffers [0, 128), O [128, 128 + hd), Q [384, 384 + hd / 2).
-// K and V tiles have kSlots = 3 shared-memory slots each, so three tiles' loads
-// are in flight; per 64 keys at hd = 256 the tensor cores run 16 (S) + 4 (P V) MMAs.
+// K and V tiles have 3 shared-memory slots each, so three tiles' loads are in
+// flight; per 64 keys at hd = 256 the tensor cores run 16 (S) + 4 (P V) MMAs.
 //
 // Warp roles (224 threads): warps 0-3 run the softmax, one thread per query
 // row (TMEM lane), all 64 columns of a tile, no exchange between threads; warp 4
@@ -33,6 +33,23 @@
 // -inf). Tile t + 1's S product and tile t - 1's P V product overlap tile t's
 // softmax; the softmax waits for P V of tile t - 1 only to rescale O (rare).
 // Every wait is bounded. Shared memory at hd = 256: K, V 3 x 32 KB each, P 2 x 16 KB.
+//
+// V-only cache (attention_k_eq_v: k and v come from one k_proj row and one
+// normalisation, so k = rope(v * k_norm) row by row, and the cache can hold v
+// alone): only V tiles are loaded, half the bytes, and eight more warps (6-13,
+// 448 threads) rebuild each tile's K into a K slot as it lands, in fp16:
+// x = v * k_norm, k1 = x1 cos - x2 sin, k2 = x2 cos + x1 sin for every RoPE pair
+// (i, i + hd / 2) at the key's position (pos0[b] + t for context row t,
+// block_pos[b] + i for block row i), the products and the rotation on packed
+// fp16 (the keys are rounded to fp16 anyway), the angles in fp32. A builder
+// thread owns 8 pairs of 4 keys; it starts from the angle of its first key's
+// position (reduced in double) and turns it by theta per key and by 64 theta
+// per tile (one complex product each, so the rounding of a tile's angles grows
+// with the tiles a CTA walks, a few 1e-7 per tile, far below fp16's 2^-11). The
+// V rows past the last key are zeroed by the same threads. The S product then
+// reads the rebuilt K tile as it would a loaded one. A rebuilt K tile lives
+// only from its build to its S product, so the six tile slots split 4 V + 2 K
+// (four V loads in flight, where a K+V cache keeps three of each).
 //
 // An item on one CTA writes its output straight from tensor memory. Otherwise
 // each CTA writes its unnormalised O with (max, sum) per query row into its own
@@ -55,12 +72,19 @@ namespace dspark {
 namespace tc {
 namespace {
 
-constexpr int kThreads = 224;
+// threads: warps 0-6; a V-only cache adds the K builders, warps 6-9 (warp 6 then builds too)
+constexpr int kBuildWarps = 8;       // V-only: warps 6 .. 13 rebuild K from the V tiles
+constexpr int kBuildKeys = 4;        // keys per builder thread and tile
+template <bool VONLY> struct AttnThreads { static constexpr int n = VONLY ? 192 + 32 * kBuildWarps : 224; };
 constexpr int kSoftThreads = 128;    // warps 0-3: one thread per query row
 constexpr int kIssuerWarp = 4;       // S products and K loads; warp 5: P V products and V loads
 constexpr int kFixWarp = 6;          // zeroes the V rows past the last key of a partial tile
 constexpr int KT = 64;               // keys per tile
-constexpr int kSlots = 3;            // shared-memory slots of K tiles, and of V tiles (loads in flight)
+// Shared-memory tile slots (6 tiles in all): a K+V cache loads both, 3 K and 3 V
+// slots; a V-only cache loads V alone and rebuilds each K tile just before its S
+// product, so 4 V slots keep four loads in flight and 2 K slots suffice.
+constexpr int kSlotsMax = 4;
+template <bool VONLY> struct AttnSlots { static constexpr int k = VONLY ? 2 : 3, v = VONLY ? 4 : 3; };
 constexpr int kQCol = 2 * KT + 256;  // TMEM columns: S buffers [0, 2 KT), O [2 KT, 2 KT + hd), Q from 384
 constexpr int QROWS = 128;           // MMA M
 // Natural-log headroom before the running max is raised: P = exp(s - m_run) stays
@@ -76,6 +100,11 @@ struct AttnTcParams {
     void* out; int out_dtype;        // [A, G, nH, hd] fp32 or fp16
     __half* out_hi; __half* out_lo;  // optional fp16 pair of the output (the next GEMM's input)
     int32_t* status;
+    // V-only cache: K rebuilt from the V tiles at the keys' positions
+    const int32_t* pos0;             // [A] position of cache row 0
+    const int32_t* block_pos;        // [A] position of block row 0
+    const __nv_bfloat16* k_norm;     // [hd]
+    const double* inv_freq;          // [hd / 2]
 };
 
 // The work plan (device lengths): item i = (row b, kv head g) has n_i =
@@ -88,9 +117,9 @@ __device__ __forceinline__ int plan_tiles(const int32_t* len, int b, int capacit
     const int L = min(max(len[b], 0), capacity);
     return (L + KT - 1) / KT + 1;
 }
-constexpr int kWarps = kThreads / 32;
-// Sum (or maximum) over the block; `buf` holds kWarps ints and callers
+// Sum (or maximum) over the block of NW warps; `buf` holds NW ints and callers
 // alternate two buffers, so one barrier per reduction suffices.
+template <int NW>
 __device__ __forceinline__ int block_reduce_int(int v, int* buf, bool is_max) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
@@ -101,7 +130,7 @@ __device__ __forceinline__ int block_reduce_int(int v, int* buf, bool is_max) {
     if (lane == 0) buf[wid] = v;
     __syncthreads();
     int t = is_max ? buf[0] : 0;
-    for (int w = is_max ? 1 : 0; w < kWarps; ++w) t = is_max ? max(t, buf[w]) : t + buf[w];
+    for (int w = is_max ? 1 : 0; w < NW; ++w) t = is_max ? max(t, buf[w]) : t + buf[w];
     return t;
 }
 struct CtaWork {
@@ -124,9 +153,11 @@ __device__ __forceinline__ int ceil_div_small(int n, int q, float rq) {
 // feasible q found by testing up to kThreads candidates at once (each thread
 // sums nKv * ceil(n_b / q) over the rows for its candidate; two rounds at most
 // for n up to kThreads^2), then a scan of k_b over the rows places the CTA.
-// `sh` holds 2 kWarps + 5 ints.
+// `sh` holds 2 kWarps + 5 ints. kThreads: the block's threads.
+template <int kThreads>
 __device__ CtaWork cta_work(const int32_t* __restrict__ len, int A, int nKv, int capacity, int grid, int slot,
                             int* sh, int* ncache) {
+    constexpr int kWarps = kThreads / 32;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     int* res = sh + 2 * kWarps;                      // item, index within the item, n, k, first slot
     if (tid == 0) res[0] = -1;                       // ordered before the scan by the barriers below
@@ -137,7 +168,7 @@ __device__ CtaWork cta_work(const int32_t* __restrict__ len, int A, int nKv, int
         ncache[b] = n;
         mx = max(mx, n);
     }
-    mx = block_reduce_int(mx, sh + (nb++ & 1) * kWarps, true);   // also publishes ncache
+    mx = block_reduce_int<kWarps>(mx, sh + (nb++ & 1) * kWarps, true);   // also publishes ncache
     int q = mx;                                      // q = mx is feasible: A * nKv <= grid
     if (A * nKv < grid) {
         int lo = min(2, mx), hi = mx;                // the answer lies in [lo, hi]; hi is feasible
@@ -152,7 +183,7 @@ __device__ CtaWork cta_work(const int32_t* __restrict__ len, int A, int nKv, int
                 if ((int64_t)cnt * nKv <= grid) best = cand;
             }
             // the smallest feasible candidate; the answer is in (best - step, best]
-            best = -block_reduce_int(-best, sh + (nb++ & 1) * kWarps, true);
+            best = -block_reduce_int<kWarps>(-best, sh + (nb++ & 1) * kWarps, true);
             hi = best;
             lo = max(lo, best - step + 1);
         }
@@ -330,7 +361,19 @@ __device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, v
     return __all_sync(0xffffffffu, w);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// (sin, cos) of pos * inv_freq for the K rebuild: the angle reduced to [-pi, pi] in
+// double, then the fast single-precision intrinsic (absolute error a few 1e-7 there,
+// far below the fp16 rounding of the rebuilt keys).
+__device__ __forceinline__ void rope_angle_fast(int pos, double inv_freq, float* s, float* c) {
+    const double two_pi = 6.283185307179586476925286766559;
+    const double inv_two_pi = 0.15915494309189533576888376337251;
+    double a = (double)pos * inv_freq;
+    a -= rint(a * inv_two_pi) * two_pi;
+    __sincosf((float)a, s, c);
+}
+
+template <bool VONLY>
+__global__ void __launch_bounds__(AttnThreads<VONLY>::n, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
                const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmQ, AttnTcParams P) {
@@ -338,17 +381,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     const int hd = P.hd, nsub = hd / 64;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tile_sz = nsub * KT * 128;                  // one K or V tile: nsub x [64 keys x 128 B]
-    uint8_t* sK = base;                                   // kSlots x tile
-    uint8_t* sV = sK + kSlots * tile_sz;                  // kSlots x tile
-    uint8_t* sP = sV + kSlots * tile_sz;                  // 2 slots x [128 rows x 128 B]
+    constexpr int kSK = AttnSlots<VONLY>::k, kSV = AttnSlots<VONLY>::v;
+    uint8_t* sK = base;                                   // kSK x tile
+    uint8_t* sV = sK + kSK * tile_sz;                     // kSV x tile
+    uint8_t* sP = sV + kSV * tile_sz;                     // 2 slots x [128 rows x 128 B]
     int* red = reinterpret_cast<int*>(sP + 2 * QROWS * 128);      // plan scratch (2 kWarps + 5 ints), last-CTA flag
     uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * QROWS);
-    uint64_t* kfull = bars + 0;                // [kSlots] K tile landed in the slot (TMA)
-    uint64_t* vfull = kfull + kSlots;          // [kSlots] V tile landed in the slot (TMA)
-    uint64_t* vready = vfull + kSlots;         // [kSlots] V tile of the slot ready for its product (1 arrival)
-    uint64_t* kfree = vready + kSlots;         // [kSlots] the S product that read the K slot is done
-    uint64_t* vfree = kfree + kSlots;          // [kSlots] the P V product that read the V slot is done
-    uint64_t* sdone = vfree + kSlots;          // [2] S product of the tile in that buffer done
+    uint64_t* kfull = bars + 0;                // [kSK] K tile landed in the slot (TMA)
+    uint64_t* vfull = kfull + kSlotsMax;       // [kSV] V tile landed in the slot (TMA)
+    uint64_t* vready = vfull + kSlotsMax;      // [kSV] V tile ready (V-only: and K rebuilt): 1 / kBuildWarps arrivals
+    uint64_t* kfree = vready + kSlotsMax;      // [kSK] the S product that read the K slot is done
+    uint64_t* vfree = kfree + kSlotsMax;       // [kSV] the P V product that read the V slot is done
+    uint64_t* sdone = vfree + kSlotsMax;       // [2] S product of the tile in that buffer done
     uint64_t* sfree = sdone + 2;               // [2] softmax has read the S buffer (256 arrivals)
     uint64_t* pready = sfree + 2;              // [2] P slot written (256 arrivals)
     uint64_t* odone = pready + 2;              // [2] P V product of the tile in that P slot done (O settled)
@@ -362,8 +406,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     const int nq = P.grp * P.G;
 
     if (tid == 0) {
-        for (int i = 0; i < kSlots; ++i) {
-            mbar_init(&kfull[i], 1); mbar_init(&vfull[i], 1); mbar_init(&vready[i], 1);
+        for (int i = 0; i < kSlotsMax; ++i) {
+            mbar_init(&kfull[i], 1); mbar_init(&vfull[i], 1); mbar_init(&vready[i], VONLY ? kBuildWarps : 1);
             mbar_init(&kfree[i], 1); mbar_init(&vfree[i], 1);
         }
         mbar_init(&sdone[0], 1); mbar_init(&sdone[1], 1);
@@ -387,7 +431,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 
     // this CTA's work: tiles [t_lo, t_hi) of item (b, g); an idle CTA has none
     const int slot = blockIdx.x;
-    const CtaWork W = cta_work(P.len, P.A, P.nKv, P.capacity, P.grid, slot, red, reinterpret_cast<int*>(sK));
+    const CtaWork W = cta_work<AttnThreads<VONLY>::n>(P.len, P.A, P.nKv, P.capacity, P.grid, slot, red, reinterpret_cast<int*>(sK));
     const int item = W.item;
     const int b = item >= 0 ? item / P.nKv : 0, g = item >= 0 ? item % P.nKv : 0;
     const int t_lo = W.t0, t_hi = W.t1;
@@ -412,7 +456,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     // in tensor memory; their V tiles are requested after it), while K tiles 0..2
     // and V tile 0 load. Softmax thread r then copies its row to tensor memory.
     const uint32_t tile_bytes = (uint32_t)nsub * KT * 128;
-    uint8_t* sQ = sV + tile_sz;                           // nsub x [nq rows x 128 B] <= 2 tiles
+    // V-only: the K slots are free until the builders start (after the query tile is in
+    // tensor memory), so the query tile goes there and V tiles 0..2 load at once
+    uint8_t* sQ = VONLY ? sK : sV + tile_sz;              // nsub x [nq rows x 128 B] <= 2 tiles
     const int qstride = (nq * 128 + 1023) & ~1023;        // chunks 1 KB aligned (the swizzle's period)
     if (warp == kIssuerWarp && lane == 0 && item >= 0) {
         mbar_arrive_expect_tx(qfull, (uint32_t)(nsub * nq * 128));
@@ -420,7 +466,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     }
     if ((warp == kIssuerWarp || warp == kIssuerWarp + 1) && lane == 0) {
         const bool v_tile = warp != kIssuerWarp;
-        for (int t = 0; t < (v_tile ? 1 : kSlots) && t < nt; ++t) {
+        const int n0 = v_tile ? (VONLY ? kSV : 1) : (VONLY ? 0 : kSK);
+        for (int t = 0; t < n0 && t < nt; ++t) {
             int row, nvalid; bool blk;
             tile_rows(t, &row, &nvalid, &blk);
             const CUtensorMap* m = blk ? (v_tile ? &tmVb : &tmKb) : (v_tile ? &tmV : &tmK);
@@ -454,8 +501,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kIssuerWarp + 1 && lane == 0) {
-        for (int t = 1; t < kSlots && t < nt; ++t) {
+    if (warp == kIssuerWarp + 1 && lane == 0 && !VONLY) {
+        for (int t = 1; t < kSV && t < nt; ++t) {
             int row, nvalid; bool blk;
             tile_rows(t, &row, &nvalid, &blk);
             mbar_arrive_expect_tx(&vfull[t], tile_bytes);
@@ -482,17 +529,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             uint8_t* buf = is_qk ? sK : sV;
             uint64_t* fullb = is_qk ? kfull : vfull;
             uint64_t* freeb = is_qk ? kfree : vfree;          // completion of the product that read a slot
-            int nl[kSlots] = {};                              // loads issued per slot
-            for (int t = 0; t < kSlots && t < nt; ++t) ++nl[t];   // issued before the Q tile
-            int ln = min(kSlots, nt);                         // next tile to load
+            const int ns = is_qk ? kSK : kSV;                 // this issuer's slots
+            int nl[kSlotsMax] = {};                           // loads issued per slot
+            const bool loads = !(VONLY && is_qk);             // V-only: the S issuer loads nothing
+            if (loads)
+                for (int t = 0; t < ns && t < nt; ++t) ++nl[t];   // issued before the loop
+            int ln = loads ? min(ns, nt) : nt;                // next tile to load
             int issued = 0;                                   // products issued
-            // tile ln goes into slot ln % kSlots once the product of tile ln - kSlots (the
-            // slot's previous tile, phase (ln - kSlots) / kSlots of its barrier) is done
+            // tile ln goes into slot ln % ns once the product of tile ln - ns (the slot's
+            // previous tile, phase (ln - ns) / ns of its barrier) is done
             auto service = [&]() {
-                while (ln < nt && ln - kSlots < issued &&
-                       mbar_try_wait(&freeb[ln % kSlots], (uint32_t)((ln - kSlots) / kSlots) & 1u)) {
-                    load(buf + (ln % kSlots) * tile_sz, &fullb[ln % kSlots], !is_qk, ln);
-                    ++nl[ln % kSlots];
+                while (ln < nt && ln - ns < issued &&
+                       mbar_try_wait(&freeb[ln % ns], (uint32_t)((ln - ns) / ns) & 1u)) {
+                    load(buf + (ln % ns) * tile_sz, &fullb[ln % ns], !is_qk, ln);
+                    ++nl[ln % ns];
                     ++ln;
                 }
             };
@@ -514,16 +564,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             const uint32_t qa = tmem + (uint32_t)kQCol;      // Q in tensor memory: 8 columns per 16-wide K slice
             for (int t = 0; t < nt && ok; ++t) {
                 const int sl = t & 1;                             // S buffer / P slot
-                const int ks = t % kSlots;                        // K / V slot
-                const uint32_t kph = (uint32_t)(t / kSlots) & 1u;
+                const int tk = t % kSK, tv = t % kSV;             // K slot, V slot
+                const uint32_t kph = (uint32_t)(t / kSK) & 1u, vph = (uint32_t)(t / kSV) & 1u;
                 if (is_qk) {
                     // S(t) = Q K(t)^T into buffer t % 2
-                    if (!wait_serving(&kfull[ks], kph)) { ok = false; break; }
+                    // V-only: the K tile is rebuilt from the V tile (vready), not loaded
+                    if (!(VONLY ? wait_serving(&vready[tv], vph) : wait_serving(&kfull[tk], kph))) { ok = false; break; }
                     if (t >= 2 && !wait_serving(&sfree[sl], (uint32_t)((t - 2) >> 1) & 1u)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d = tmem + (uint32_t)(sl * KT);
                     // descriptors advance by address / 16: constants per unrolled slice
-                    const uint64_t bd0 = sdesc_k_sw128(smem_u32(sK + ks * tile_sz));
+                    const uint64_t bd0 = sdesc_k_sw128(smem_u32(sK + tk * tile_sz));
                     mma_f16_ts(d, qa, bd0, idesc_qk, 0u);
 #pragma unroll
                     for (int j = 1; j < 16; ++j) {
@@ -532,22 +583,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                         mma_f16_ts(d, qa + (uint32_t)(8 * j), bd0 + boff, idesc_qk, 1u);
                     }
                     mma_commit(&sdone[sl]);
-                    mma_commit(&kfree[ks]);
+                    mma_commit(&kfree[tk]);                         // V-only: the builders wait on it
                 } else {
                     // O += P(t) V(t)
-                    if (!wait_serving(&pready[sl], (uint32_t)(t >> 1) & 1u) || !wait_serving(&vready[ks], kph)) {
+                    if (!wait_serving(&pready[sl], (uint32_t)(t >> 1) & 1u) || !wait_serving(&vready[tv], vph)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint64_t ad0 = sdesc_k_sw128(smem_u32(sP + sl * QROWS * 128));
-                    const uint64_t bd0 = sdesc_mn_sw128(smem_u32(sV + ks * tile_sz), KT * 128);
+                    const uint64_t bd0 = sdesc_mn_sw128(smem_u32(sV + tv * tile_sz), KT * 128);
 #pragma unroll
                     for (int j = 0; j < KT / 16; ++j)
                         mma_bf16(tO, ad0 + (uint64_t)((j * 32) >> 4), bd0 + (uint64_t)((j * 2048) >> 4), idesc_pv,
                                  (t > 0 || j > 0) ? 1u : 0u);
                     mma_commit(&odone[sl]);
-                    mma_commit(&vfree[ks]);
+                    mma_commit(&vfree[tv]);
                 }
                 issued = t + 1;
                 service();
@@ -556,7 +607,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             if (!ok) {
                 const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
                 bool drained = true;
-                for (int i = 0; i < kSlots; ++i)
+                for (int i = 0; i < ns; ++i)
                     if (drained && nl[i] > 0) drained = mbar_wait_until(&fullb[i], (uint32_t)(nl[i] - 1) & 1u, deadline);
                 uint64_t* sp = is_qk ? spare : spare2;
                 mma_commit(sp);
@@ -564,13 +615,112 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 if (!drained) atomicOr(P.status, DSPARK_DEV_WAIT_TIMEOUT);
             }
         }
+    } else if (VONLY && warp >= kFixWarp) {
+        // ------------------------------------------------------------ K from V (V-only cache)
+        // builder thread bt owns RoPE pairs [8 pg, 8 pg + 8) of keys [4 kr, 4 kr + 4) of
+        // every tile: dimensions d1 + m and d2 + m (d2 = d1 + hd / 2), two 16-byte
+        // pieces of each key row, read from the V slot and written to the K slot (same
+        // 128-byte swizzled layout); rows past the last key are zeroed in the V slot
+        const int bt = tid - kFixWarp * 32;
+        const int npg = hd / 16, half = hd / 2;
+        const int pg = bt % npg, kr = bt / npg;
+        const bool active = kr < KT / kBuildKeys;
+        const int d1 = pg * 8, d2 = pg * 8 + half;
+        const int o1 = (d1 / 64) * KT * 128, c1 = (d1 % 64) / 8;
+        const int o2 = (d2 / 64) * KT * 128, c2 = (d2 % 64) / 8;
+        // gains as fp16 pairs (the products and the rotation run on packed fp16: each
+        // key's k is rounded to fp16 anyway); the angles stay in fp32
+        __half2 w1h[4], w2h[4];
+        float cs[8], sn[8], cs1[8], sn1[8], cs64[8], sn64[8];
+        if (active) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                w1h[e] = __floats2half2_rn(__bfloat162float(P.k_norm[d1 + 2 * e]), __bfloat162float(P.k_norm[d1 + 2 * e + 1]));
+                w2h[e] = __floats2half2_rn(__bfloat162float(P.k_norm[d2 + 2 * e]), __bfloat162float(P.k_norm[d2 + 2 * e + 1]));
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const double f = P.inv_freq[d1 + m];
+                rope_angle_fast(1, f, &sn1[m], &cs1[m]);      // one key further
+                rope_angle_fast(KT, f, &sn64[m], &cs64[m]);   // one tile further
+                cs[m] = 1.f; sn[m] = 0.f;
+            }
+        }
+        bool anchored = false;                             // cs, sn: angles of this thread's first key of tile t
+        for (int t = 0; t < nt && ok; ++t) {
+            int row, nvalid; bool blk;
+            tile_rows(t, &row, &nvalid, &blk);
+            const int tv = t % kSV, tk = t % kSK;
+            if (!warp_wait(&vfull[tv], (uint32_t)(t / kSV) & 1u, abort_flag, P.status)) { ok = false; break; }
+            // the K slot's previous tile, t - kSK, must have had its S product
+            if (t >= kSK && !warp_wait(&kfree[tk], (uint32_t)((t - kSK) / kSK) & 1u, abort_flag, P.status)) {
+                ok = false;
+                break;
+            }
+            if (active) {
+                if (blk || !anchored) {                        // exact angles at the first context tile and the block
+                    const int p = (blk ? P.block_pos[b] : P.pos0[b] + (t_lo + t) * KT) + kr * kBuildKeys;
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) rope_angle_fast(p, P.inv_freq[d1 + m], &sn[m], &cs[m]);
+                    anchored = true;
+                }
+                uint8_t* vt = sV + tv * tile_sz;
+                uint8_t* kt = sK + tk * tile_sz;
+                float c[8], sv_[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) { c[m] = cs[m]; sv_[m] = sn[m]; }
+#pragma unroll
+                for (int kk = 0; kk < kBuildKeys; ++kk) {
+                    const int j = kr * kBuildKeys + kk;
+                    const int a1 = o1 + j * 128 + ((c1 ^ (j & 7)) * 16), a2 = o2 + j * 128 + ((c2 ^ (j & 7)) * 16);
+                    if (j < nvalid) {
+                        const uint4 x4 = *reinterpret_cast<const uint4*>(vt + a1);
+                        const uint4 y4 = *reinterpret_cast<const uint4*>(vt + a2);
+                        const __half2* xh = reinterpret_cast<const __half2*>(&x4);
+                        const __half2* yh = reinterpret_cast<const __half2*>(&y4);
+                        uint32_t k1[4], k2[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __half2 xw = __hmul2(xh[e], w1h[e]), yw = __hmul2(yh[e], w2h[e]);
+                            const __half2 ch = __floats2half2_rn(c[2 * e], c[2 * e + 1]);
+                            const __half2 sh = __floats2half2_rn(sv_[2 * e], sv_[2 * e + 1]);
+                            const __half2 r1 = __hfma2(xw, ch, __hneg2(__hmul2(yw, sh)));   // x cos - y sin
+                            const __half2 r2 = __hfma2(yw, ch, __hmul2(xw, sh));            // y cos + x sin
+                            k1[e] = *reinterpret_cast<const uint32_t*>(&r1);
+                            k2[e] = *reinterpret_cast<const uint32_t*>(&r2);
+                        }
+                        *reinterpret_cast<uint4*>(kt + a1) = make_uint4(k1[0], k1[1], k1[2], k1[3]);
+                        *reinterpret_cast<uint4*>(kt + a2) = make_uint4(k2[0], k2[1], k2[2], k2[3]);
+                    } else {
+                        // past the last key: the P V product must not meet stale bits (S masks these keys)
+                        *reinterpret_cast<uint4*>(vt + a1) = make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4*>(vt + a2) = make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {              // the next key: angle + theta
+                        const float cn = c[m] * cs1[m] - sv_[m] * sn1[m];
+                        sv_[m] = sv_[m] * cs1[m] + c[m] * sn1[m];
+                        c[m] = cn;
+                    }
+                }
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {                  // the next context tile: angle + 64 theta
+                    const float cn = cs[m] * cs64[m] - sn[m] * sn64[m];
+                    sn[m] = sn[m] * cs64[m] + cs[m] * sn64[m];
+                    cs[m] = cn;
+                }
+            }
+            fence_async_shared();                           // both tiles are read through the async proxy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&vready[tv]);
+        }
     } else if (warp == kFixWarp) {
         // ------------------------------------------------------------ V tails
         for (int t = 0; t < nt && ok; ++t) {
             int row, nvalid; bool blk;
             tile_rows(t, &row, &nvalid, &blk);
-            const int ks = t % kSlots;
-            if (!warp_wait(&vfull[ks], (uint32_t)(t / kSlots) & 1u, abort_flag, P.status)) { ok = false; break; }
+            const int ks = t % kSV;
+            if (!warp_wait(&vfull[ks], (uint32_t)(t / kSV) & 1u, abort_flag, P.status)) { ok = false; break; }
             if (nvalid < KT) {
                 zero_tail(sV + ks * tile_sz, nsub, nvalid, lane);
                 fence_async_shared();               // the P V product reads the tile through the async proxy
@@ -777,9 +927,9 @@ bool make_q_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int grp
 
 size_t attn_tc_smem(int hd) {
     const int nsub = hd / 64;
-    // K and V (kSlots each), P (2 slots), the plan scratch, then the barriers
-    // (5 kSlots + 11), the TMEM slot and the abort flag; 1 KB alignment slack
-    return 2 * (size_t)kSlots * nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 8 * (5 * kSlots + 11) + 16 + 1024;
+    // six K / V tiles, P (2 slots), the plan scratch, then the barriers
+    // (5 kSlotsMax + 11), the TMEM slot and the abort flag; 1 KB alignment slack
+    return 6 * (size_t)nsub * KT * 128 + 2 * QROWS * 128 + 2 * QROWS * 4 + 8 * (5 * kSlotsMax + 11) + 16 + 1024;
 }
 
 
@@ -806,6 +956,9 @@ bool attention_tc_supported(const dspark_model* m) {
     return d.dtype == DSPARK_DTYPE_BF16 && d.grp * d.gamma <= QROWS && d.hd % 64 == 0 && d.hd <= 256;
 }
 
+// The V-only cache: the tensor-core attention, which rebuilds K from the V tiles.
+bool vonly_attention_supported(const dspark_model* m) { return attention_tc_supported(m); }
+
 int attention_tc_key_tile() { return KT; }
 
 int attention_tc_grid(const dspark_model* m, int A) { return std::max(m->num_sms, A * m->d.nKv); }
@@ -819,10 +972,14 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
     if (!a.item_slots || a.tc_grid < std::max(1, a.A * d.nKv) || a.q_dtype != DSPARK_DTYPE_F16 ||
         (a.out_dtype != DSPARK_DTYPE_F32 && a.out_dtype != DSPARK_DTYPE_F16))
         return cudaErrorInvalidValue;
+    // V-only cache: K is rebuilt from the V tiles (the K maps repeat the V ones, unused)
+    const bool vonly = a.kc == nullptr;
+    if (vonly && (!vonly_attention_supported(m) || !a.pos0 || !a.block_pos || !a.k_norm)) return cudaErrorInvalidValue;
     CUtensorMap tk, tv, tkb, tvb, to, tq;
     const int64_t cache_rows = (int64_t)a.batch * a.capacity;   // all rows of this layer's cache
-    if (!make_kv_map(&tk, a.kc, cache_rows, d.nKv, d.hd) || !make_kv_map(&tv, a.vc, cache_rows, d.nKv, d.hd) ||
-        !make_kv_map(&tkb, a.kb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
+    if (!make_kv_map(&tk, vonly ? a.vc : a.kc, cache_rows, d.nKv, d.hd) ||
+        !make_kv_map(&tv, a.vc, cache_rows, d.nKv, d.hd) ||
+        !make_kv_map(&tkb, vonly ? a.vb : a.kb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
         !make_kv_map(&tvb, a.vb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
         !make_part_map(&to, a.part_o, (int64_t)a.tc_grid * QROWS, d.hd) ||
         !make_q_map(&tq, a.q, (int64_t)a.A * d.gamma, d.nKv, d.grp, d.gamma, d.hd))
@@ -832,10 +989,14 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
     P.q_dtype = a.q_dtype; P.grid = a.tc_grid; P.q = a.q; P.len = a.len;
     P.part_o = a.part_o; P.part_ml = a.part_ml; P.item_slots = a.item_slots; P.status = a.status;
     P.out = a.out; P.out_dtype = a.out_dtype; P.out_hi = a.out_hi; P.out_lo = a.out_lo;
+    P.pos0 = a.pos0; P.block_pos = a.block_pos;
+    P.k_norm = static_cast<const __nv_bfloat16*>(a.k_norm); P.inv_freq = m->ws.inv_freq;
     const size_t smem = attn_tc_smem(d.hd);
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = vonly ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attn_tc_kernel, dim3(a.tc_grid), dim3(kThreads), smem, s, tk, tv, tkb, tvb, to, tq, P);
+    e = launch_pdl(kern, dim3(a.tc_grid), dim3(vonly ? AttnThreads<true>::n : AttnThreads<false>::n), smem, s, tk, tv,
+                   tkb, tvb, to, tq, P);
     if (e != cudaSuccess) return e;
     // with at least as many items as CTAs every item is on one CTA: nothing to merge
     if (a.A * d.nKv >= a.tc_grid) return cudaSuccess;

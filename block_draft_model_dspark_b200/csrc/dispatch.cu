@@ -155,7 +155,7 @@ cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, c
     const Dims& d = m->d;
     const int N = d.Lyr * d.nKv * d.hd;
     const double es = d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0;
-    KernelTimer t(DSPARK_TIMER_KV_PROJECT, s, weight_bytes(m, N, d.H) + es * nrows * d.H + 2.0 * es * nrows * N,
+    KernelTimer t(DSPARK_TIMER_KV_PROJECT, s, weight_bytes(m, N, d.H) + es * nrows * d.H + (dst.k ? 2.0 : 1.0) * es * nrows * N,
                   2.0 * nrows * (double)N * d.H);
     PartView view{};
     view.p = raw;

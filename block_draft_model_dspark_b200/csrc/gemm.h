@@ -44,6 +44,8 @@ cudaError_t run_attention(const dspark_model* m, const AttnArgs& a, cudaStream_t
 int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len);
 namespace tc {
 bool attention_tc_supported(const dspark_model* m);
+// V-only caches (K rebuilt from V in the tensor-core attention).
+bool vonly_attention_supported(const dspark_model* m);
 // Tensor-core attention: CTAs of a call for A rows, ints of its work plan and floats of its
 // per-CTA partial state (one slot of 128 rows x (head_dim + 2) per CTA).
 int attention_tc_grid(const dspark_model* m, int A);

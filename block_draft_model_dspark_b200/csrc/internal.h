@@ -237,7 +237,7 @@ cudaError_t launch_simt_gemm(const void* X, int64_t ldx, int x_dtype, int w_dtyp
 // Context K/V epilogue: the K/V GEMM's result [rows, Lyr*nKv*hd] -> cache rows.
 // Row r = b*Lrows + t is valid when t < n_b.
 struct KvDest {
-    void* k; void* v;
+    void* k; void* v;        // k NULL: a V-only cache (v written alone)
     int64_t batch_stride;    // elements between batch rows   (= cap * nKv * hd)
     int64_t layer_stride;    // elements between layers       (= batch * cap * nKv * hd)
     int capacity;
@@ -294,6 +294,10 @@ struct AttnArgs {
     int S1;                                          // partial slots per (b, h): set by the kernel path
     int32_t* status;
     double kv_bytes, flops;                          // algorithmic work (for the timers)
+    // V-only cache (kc == NULL): K rebuilt in the kernel as rope(v * k_norm) at the
+    // positions pos0[b] + t (context row t) and block_pos[b] + i (block row i)
+    const int32_t* pos0; const int32_t* block_pos;
+    const void* k_norm;                              // this layer's k_norm gain [hd]
 };
 
 // Markov walk step k: tokens[:,k] from U[:,k,:] + w2 . w1[prev]; prev updated.

@@ -83,13 +83,14 @@ __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const 
     const float ss = block_sum(x1 * x1 + x2 * x2, red);
     const float rinv = rsqrtf(ss / (float)hd + eps);
     const float v1 = x1 * rinv, v2 = x2 * rinv;
+    const int64_t o = (int64_t)l * dst.layer_stride + (int64_t)b * dst.batch_stride + ((int64_t)dst_row * nKv + g) * hd;
+    store_any(dst.v, o + i, kv_dtype, v1);
+    store_any(dst.v, o + i + half, kv_dtype, v2);
+    if (!dst.k) return;                                    // a V-only cache
     const void* wk = k_norms.p[l];
     const float k1 = v1 * load_any(wk, i, dtype), k2 = v2 * load_any(wk, i + half, dtype);
     float sn, cs;
     rope_sincos(pos, inv_freq[i], &sn, &cs);
-    const int64_t o = (int64_t)l * dst.layer_stride + (int64_t)b * dst.batch_stride + ((int64_t)dst_row * nKv + g) * hd;
-    store_any(dst.v, o + i, kv_dtype, v1);
-    store_any(dst.v, o + i + half, kv_dtype, v2);
     store_any(dst.k, o + i, kv_dtype, k1 * cs - k2 * sn);
     store_any(dst.k, o + i + half, kv_dtype, k2 * cs + k1 * sn);
 }

@@ -157,6 +157,21 @@ int32_t dspark_kv_dtype(const dspark_config* cfg);
  * host copy of len when it keeps one. The library never writes it and reads
  * it only to count the attention's algorithmic bytes for the instrumentation
  * timers below.
+ * V-only cache: k = NULL. With attention_k_eq_v the keys and values come from
+ * one projection and one normalisation, so k[l,b,t] = rope(v[l,b,t] * k_norm_l,
+ * position of row t) (dspark_project_context_kv below); a V-only cache stores v
+ * alone and the attention rebuilds k from it, which halves the cache's memory
+ * and the bytes every round reads (the rebuild costs SM time: with every RoPE
+ * pair rotated, a round's attention is slower than on a K+V cache, so V-only
+ * trades speed for memory). It needs pos0 (device int32 [batch], the
+ * absolute position of cache row 0 of each batch row, so row t sits at
+ * pos0[b] + t: the positions the rows were projected at) and a bf16 model on
+ * the tensor-core attention (head_dim a multiple of 64, at most 256), and is
+ * read by dspark_draft_rows and written by
+ * dspark_append_context_kv; dspark_attend and dspark_attend_no_alloc take
+ * the seam's explicit block keys and refuse it (DSPARK_ERR_INVALID_ARGUMENT).
+ * Other calls refuse k = NULL where V-only is unsupported
+ * (DSPARK_ERR_UNSUPPORTED). pos0 is ignored when k != NULL.
  */
 typedef struct dspark_kv_cache {
     void*    k;
@@ -165,6 +180,7 @@ typedef struct dspark_kv_cache {
     int32_t* len_host;
     int32_t  batch;
     int32_t  capacity;
+    const int32_t* pos0;
 } dspark_kv_cache;
 
 typedef struct dspark_model dspark_model;
@@ -206,7 +222,8 @@ size_t dspark_project_workspace_bytes(const dspark_model* model, int64_t rows);
  *   hidden  device T [B, L, H]
  *   pos0    device int32 [B] or NULL
  *   k_out, v_out  device KV [num_hidden_layers][B][L][nKv][hd]
- * (the dspark_kv_cache layout with capacity = L).
+ * (the dspark_kv_cache layout with capacity = L). k_out = NULL writes v alone
+ * (the rows of a V-only cache).
  */
 int dspark_project_context_kv(const dspark_model* model, const void* hidden, int32_t B, int32_t L,
                               int32_t static_pos, const int32_t* pos0,
@@ -230,7 +247,8 @@ int dspark_project_context_kv(const dspark_model* model, const void* hidden, int
  * the whole append is refused -- no cache row and no len changes -- and
  * DSPARK_DEV_CAPACITY is set in the device status word (read it with
  * dspark_read_device_status). Host-side argument errors return before any
- * launch. cache.batch <= 4096.
+ * launch. cache.batch <= 4096. On a V-only cache (cache.k = NULL) only v rows
+ * are written (their values do not depend on the position).
  */
 int dspark_append_context_kv(const dspark_model* model, const void* hidden, int32_t Lnew_max,
                              const int32_t* n_new, const int32_t* pos0, dspark_kv_cache* cache,

@@ -1,7 +1,8 @@
 """GPU parity at the five workloads' full sizes, in the launch configuration the
-benchmark uses. The GPU runs every row; the oracle recomputes sampled rows
-(rows are independent in every step of the round), so it finishes in
-minutes on the host cores."""
+benchmark uses (the K+V context cache; single_bf16, quant4_bf16 and the
+incremental rounds also on the V-only cache). The GPU runs every row; the oracle
+recomputes sampled rows (rows are independent in every step of the round), so
+it finishes in minutes on the host cores."""
 import numpy as np
 import pytest
 import torch
@@ -37,10 +38,11 @@ def _check_kv(cache, kv_rows, sample, lens, dtype, name, rows_to_check=None):
     for i, b in enumerate(sample):
         L = lens[i]
         idx = np.arange(L) if rows_to_check is None else rows_to_check
-        k = cache.k[:, b, idx].float().cpu().numpy()
         v = cache.v[:, b, idx].float().cpu().numpy()
-        for l in range(k.shape[0]):
-            assert_close(k[l], kv_rows[i][l][0][idx], dtype, f"{name}: K layer {l} row {b}")
+        for l in range(v.shape[0]):
+            if cache.k is not None:                       # a V-only cache holds v alone
+                k = cache.k[l, b, idx].float().cpu().numpy()
+                assert_close(k, kv_rows[i][l][0][idx], dtype, f"{name}: K layer {l} row {b}")
             assert_close(v[l], kv_rows[i][l][1][idx], dtype, f"{name}: V layer {l} row {b}")
 
 
@@ -51,16 +53,18 @@ def _ragged_extremes():
     return sorted({0, int(lens.argmin()), int(lens.argmax())})
 
 
-@pytest.mark.parametrize("name,sample", [("single_bf16", [0]), ("ragged_bf16", _ragged_extremes()),
-                                         ("quant4_bf16", [0, 63])])
-def test_full_size_round(name, sample):
+@pytest.mark.parametrize("name,sample,v_only", [("single_bf16", [0], False), ("single_bf16", [0], True),
+                                                ("ragged_bf16", _ragged_extremes(), False),
+                                                ("quant4_bf16", [0, 63], False), ("quant4_bf16", [0, 63], True)])
+def test_full_size_round(name, sample, v_only):
     import block_draft_model_dspark_b200 as dsp
     wl = WORKLOADS[name]
     m = wl.model
     cpu, W, model = build(m, wl.seed)
     inp = make_round_inputs(wl)
     lens = inp["ctx_len"].tolist()
-    cache = dsp.KvCache(model, wl.rows, int(inp["hidden"].shape[1]))
+    cache = dsp.KvCache(model, wl.rows, int(inp["hidden"].shape[1]), v_only=v_only,
+                        pos0=inp["pos0"].cuda() if v_only else None)
     cache.set_lengths([0] * wl.rows)
     model.dspark_append_context_kv(cache, inp["hidden"].cuda(), lens, inp["pos0"].cuda())
     anchors, block_pos = inp["anchors"].tolist(), inp["block_pos"].tolist()
@@ -75,16 +79,17 @@ def test_full_size_round(name, sample):
     _compare_rows(wl, W, out, kv_rows, sample, anchors, block_pos)
 
 
-def test_long_incremental_rounds():
+@pytest.mark.parametrize("v_only", [False, True])
+def test_long_incremental_rounds(v_only):
     import block_draft_model_dspark_b200 as dsp
     wl = WORKLOADS["long_incremental_bf16"]
     m = wl.model
     cpu, W, model = build(m, wl.seed)
     inp = make_round_inputs(wl)
     A = wl.rows
-    cache = dsp.KvCache(model, A, wl.capacity)
-    cache.set_lengths([0] * A)
     pos0 = inp["pos0"].cuda()
+    cache = dsp.KvCache(model, A, wl.capacity, v_only=v_only, pos0=pos0 if v_only else None)
+    cache.set_lengths([0] * A)
     model.dspark_append_context_kv(cache, inp["hidden"].cuda(), inp["ctx_len"].tolist(), pos0)
     sample = [1]
     sub = make_round_inputs(wl, rows=sample)
