@@ -546,9 +546,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                     ++ln;
                 }
             };
+            // a waiting issuer sleeps in the barrier (woken by its completion) instead of
+            // spinning, so it takes no issue slots from the softmax and the K builders;
+            // while a load waits for its slot it looks again within 200 ns
             auto wait_serving = [&](uint64_t* bar, uint32_t parity) -> bool {
                 const uint64_t t0w = global_timer_ns();
-                while (!mbar_try_wait(bar, parity)) {
+                while (!mbar_try_wait_hint(bar, parity, ln < nt ? 200u : 2000u)) {
                     service();
                     if (*abort_flag) return false;
                     if (global_timer_ns() - t0w > kWaitLimitNs) {
@@ -739,7 +742,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             const int sl = t & 1;
             const uint32_t tS = tmem + (uint32_t)(sl * KT) + lane_off;
             // S(t) is on the critical path: poll (no suspension)
-            if (!warp_wait_spin(&sdone[sl], (uint32_t)(t >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+            // (V-only: the wait is long, behind the K rebuild, so the warp sleeps in it)
+            if (!(VONLY ? warp_wait(&sdone[sl], (uint32_t)(t >> 1) & 1u, abort_flag, P.status)
+                        : warp_wait_spin(&sdone[sl], (uint32_t)(t >> 1) & 1u, abort_flag, P.status))) { ok = false; break; }
             tc_fence_after();
             uint32_t u[4][16];
 #pragma unroll
@@ -782,7 +787,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 tmem_st_wait();
             }
             // P slot t % 2 was last read by P(t-2) V(t-2)
-            if (t >= 2 && !warp_wait_spin(&odone[sl], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, P.status)) { ok = false; break; }
+            if (t >= 2 && !(VONLY ? warp_wait(&odone[sl], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, P.status)
+                                  : warp_wait_spin(&odone[sl], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, P.status))) {
+                ok = false;
+                break;
+            }
             float ls[8];                                    // sums in 8 independent chains
 #pragma unroll
             for (int j = 0; j < 8; ++j) ls[j] = 0.f;

@@ -67,6 +67,19 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
         : "memory");
     return ok != 0;
 }
+// The same with the suspension bounded by `hint_ns` (a waiter that also has other
+// work to look after between polls).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 
 // Waits for the phase of `parity` to complete. Returns false (after flagging)
 // on timeout (`limit_ns` of polling) or when another role of the CTA has
