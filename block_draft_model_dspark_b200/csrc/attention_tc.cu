@@ -258,25 +258,31 @@ __device__ __forceinline__ void store_out4(const AttnTcParams& P, int64_t o, flo
     }
 }
 
-// Row r of item (b, g) combined over the item's k slots s0 .. s0 + k - 1 (one
-// warp): weights w_s = exp(m_s - M); lane l owns the 4-column groups l, l + 32.
-constexpr int kMergeBatch = 8;       // slots whose rows a lane loads at once
-__device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, int r, int64_t out_row) {
+// Row r of item (b, g) combined over the item's k slots s0 .. s0 + k - 1 by one
+// warp, 128 * NQ columns of it (lane l owns the 4-column groups gbase + l + 32 q,
+// q < NQ): weights w_s = exp(m_s - M) from the (max, sum) pairs. BATCH slots' loads
+// per lane are in flight at once. Items of many slots (a short call's few items)
+// take NQ = 1 and two warps per row, with twice the loads in flight; items of a
+// few slots take NQ = 2 (each warp's fixed work then counts).
+template <int NQ, int BATCH>
+__device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, int r, int64_t out_row, int gbase) {
     const int lane = threadIdx.x & 31, ng = P.hd / 4;
-    float4 num[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    float4 num[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) num[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     float den = 0.f, M = -INFINITY;
     for (int sb = 0; sb < k; sb += 32) {
         const int cnt = min(32, k - sb);
         // the first batch of rows and this chunk's (max, sum) pairs go out together: the rows'
         // loads do not depend on the maxima
-        float4 v[kMergeBatch][2];
+        float4 v[BATCH][NQ];
         auto load_rows = [&](int t0) {
 #pragma unroll
-            for (int u = 0; u < kMergeBatch; ++u) {
+            for (int u = 0; u < BATCH; ++u) {
                 const float4* o = reinterpret_cast<const float4*>(P.part_o + ((int64_t)(s0 + sb + t0 + u) * QROWS + r) * P.hd);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int g4 = lane + q * 32;
+                for (int q = 0; q < NQ; ++q) {
+                    const int g4 = gbase + lane + q * 32;
                     v[u][q] = (t0 + u < cnt && g4 < ng) ? o[g4] : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
@@ -293,21 +299,21 @@ __device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, 
             const float f = __expf(M - Mn);
             den *= f;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) { num[q].x *= f; num[q].y *= f; num[q].z *= f; num[q].w *= f; }
+            for (int q = 0; q < NQ; ++q) { num[q].x *= f; num[q].y *= f; num[q].z *= f; num[q].w *= f; }
         }
         M = Mn;
         const float ws = ml.x == -INFINITY ? 0.f : __expf(ml.x - M);
-        for (int t0 = 0; t0 < cnt; t0 += kMergeBatch) {
+        for (int t0 = 0; t0 < cnt; t0 += BATCH) {
             if (t0 > 0) load_rows(t0);
 #pragma unroll
-            for (int u = 0; u < kMergeBatch; ++u) {
+            for (int u = 0; u < BATCH; ++u) {
                 const float w = __shfl_sync(0xffffffffu, ws, (t0 + u) & 31);
                 const float l = __shfl_sync(0xffffffffu, ml.y, (t0 + u) & 31);
                 if (t0 + u >= cnt) break;
                 den += w * l;
                 if (w == 0.f) continue;                // uniform: an empty range
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q = 0; q < NQ; ++q) {
                     num[q].x += w * v[u][q].x; num[q].y += w * v[u][q].y;
                     num[q].z += w * v[u][q].z; num[q].w += w * v[u][q].w;
                 }
@@ -316,8 +322,8 @@ __device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, 
     }
     const float inv = 1.f / den;
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const int g4 = lane + q * 32;
+    for (int q = 0; q < NQ; ++q) {
+        const int g4 = gbase + lane + q * 32;
         if (g4 < ng)
             store_out4(P, out_row + g4 * 4, make_float4(num[q].x * inv, num[q].y * inv, num[q].z * inv, num[q].w * inv));
     }
@@ -945,17 +951,21 @@ size_t attn_tc_smem(int hd) {
 // One warp per output row (b, h, i) of the items on more than one CTA (an item
 // on one CTA wrote its output itself).
 constexpr int kMergeWarps = 8;
-__global__ void __launch_bounds__(kMergeWarps * 32) attn_tc_merge_kernel(AttnTcParams P, int rows) {
+// wpr warps per output row, 128 NQ columns each
+template <int NQ>
+__global__ void __launch_bounds__(kMergeWarps * 32) attn_tc_merge_kernel(AttnTcParams P, int rows, int wpr) {
     pdl_trigger();
     pdl_wait();
-    const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);   // ((b * nH) + h) * G + i
+    const int gw = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+    const int row = gw / wpr, part = gw % wpr;                      // row = ((b * nH) + h) * G + i
     if (row >= rows) return;
     const int i = row % P.G, bh = row / P.G;
     const int b = bh / P.nH, h = bh % P.nH;
     const int item = b * P.nKv + h / P.grp;
     const int k = P.item_slots[2 * item + 1];
     if (k <= 1) return;
-    merge_row(P, P.item_slots[2 * item], k, i * P.grp + h % P.grp, (((int64_t)b * P.G + i) * P.nH + h) * P.hd);
+    merge_row<NQ, NQ == 1 ? 16 : 8>(P, P.item_slots[2 * item], k, i * P.grp + h % P.grp,
+                                    (((int64_t)b * P.G + i) * P.nH + h) * P.hd, part * 32 * NQ);
 }
 
 }  // namespace
@@ -1010,8 +1020,13 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
     // with at least as many items as CTAs every item is on one CTA: nothing to merge
     if (a.A * d.nKv >= a.tc_grid) return cudaSuccess;
     const int rows = a.A * d.nH * d.gamma;
-    return launch_pdl(attn_tc_merge_kernel, dim3((rows + kMergeWarps - 1) / kMergeWarps), dim3(kMergeWarps * 32), 0,
-                      s, P, rows);
+    // items of 8 or more slots on average: two warps per row (a few items, many slots each)
+    const bool wide = a.tc_grid >= 8 * a.A * d.nKv;
+    const int wpr = wide ? (d.hd + 127) / 128 : 1;
+    const int64_t warps = (int64_t)rows * wpr;
+    return launch_pdl(wide ? attn_tc_merge_kernel<1> : attn_tc_merge_kernel<2>,
+                      dim3((unsigned)((warps + kMergeWarps - 1) / kMergeWarps)), dim3(kMergeWarps * 32), 0, s, P, rows,
+                      wpr);
 }
 
 }  // namespace tc
