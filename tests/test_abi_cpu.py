@@ -79,3 +79,32 @@ def test_null_arguments_are_rejected(dsp):
     out = ctypes.c_void_p()
     rc = lib.dspark_model_create(ctypes.byref(good), None, 256, 1 << 40, None, ctypes.byref(out))
     assert rc == dsp.DSPARK_ERR_INVALID_ARGUMENT
+
+
+def test_binding_structs_match_the_header(dsp, tmp_path):
+    """Every struct the binding passes by pointer has the header's size and field offsets
+    (compiled with the host C compiler against include/dspark.h)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    structs = {"dspark_kv_cache": dsp.dspark_kv_cache, "dspark_config": dsp.dspark_config,
+               "dspark_matrix": dsp.dspark_matrix, "dspark_layer_weights": dsp.dspark_layer_weights,
+               "dspark_weights": dsp.dspark_weights}
+    lines = ["#include <stddef.h>", "#include <stdio.h>", '#include "dspark.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
+        for f, _ in cls._fields_:
+            lines.append(f'  printf("{name} {f} %zu\\n", offsetof({name}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {(p[0], p[1]): int(p[2]) for p in (l.split() for l in out) if len(p) == 3}
+    for name, cls in structs.items():
+        assert got[(name, "size")] == ctypes.sizeof(cls), name
+        for f, _ in cls._fields_:
+            assert got[(name, f)] == getattr(cls, f).offset, (name, f)
