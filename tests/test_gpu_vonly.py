@@ -148,3 +148,31 @@ def test_vonly_refusals():
     assert e.value.code == dsp.DSPARK_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert model.dspark_read_device_status() == 0
+
+
+def test_project_without_k_writes_v_alone():
+    """dspark_project_context_kv with k_out = NULL writes the same v rows as with k_out, and a
+    round on the resulting V-only cache equals the round on the appended one."""
+    import block_draft_model_dspark_b200 as dsp
+    m = small_model(dtype="bf16")
+    cpu, W, model = build(m, 75)
+    B, L = 2, 300
+    pos0 = torch.tensor([0, 777], dtype=torch.int32, device="cuda")
+    hid = torch.randn(B, L, m.hidden_size, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16).cuda()
+    full = dsp.KvCache(model, B, L)
+    model.dspark_project_context_kv(hid, full.k, full.v, pos0=pos0)
+    vc = dsp.KvCache(model, B, L, v_only=True, pos0=pos0)
+    vc.v.fill_(float("nan"))
+    model.dspark_project_context_kv(hid, None, vc.v, pos0=pos0)
+    torch.cuda.synchronize()
+    assert torch.equal(full.v.view(torch.int16), vc.v.view(torch.int16))
+    appended = _cache(model, hid.cpu(), [L, L], pos0.tolist(), v_only=True)
+    vc.set_lengths([L, L])
+    anchors, block_pos = [3, 4], [L, 777 + L]
+    a = model.draft(vc, torch.tensor(anchors, dtype=torch.int32, device="cuda"),
+                    torch.tensor(block_pos, dtype=torch.int32, device="cuda"), L)
+    b = model.draft(appended, torch.tensor(anchors, dtype=torch.int32, device="cuda"),
+                    torch.tensor(block_pos, dtype=torch.int32, device="cuda"), L)
+    torch.cuda.synchronize()
+    assert torch.equal(a["tokens"], b["tokens"])
+    assert torch.equal(a["base_logits"], b["base_logits"])
