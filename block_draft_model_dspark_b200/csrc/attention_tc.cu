@@ -52,9 +52,9 @@
 // (four V loads in flight, where a K+V cache keeps three of each).
 //
 // An item on one CTA writes its output straight from tensor memory. Otherwise
-// each CTA writes its unnormalised O with (max, sum) per query row into its own
-// slot, and the merge kernel (one warp per output row, over the whole GPU)
-// combines the item's slots in slot order. The last range of each (b, g) also
+// each CTA writes its normalised O / l (fp16) with (max, sum) per query row into
+// its own slot, and the merge kernel (one or two warps per output row, over the
+// whole GPU) combines the item's slots in slot order. The last range of each (b, g) also
 // takes the block's own keys, as one more tile.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -62,6 +62,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "internal.h"
 #include "common.cuh"
@@ -95,7 +96,7 @@ struct AttnTcParams {
     int A, G, nH, nKv, grp, hd, capacity, q_dtype, grid;
     const void* q;                   // [A, G, nH, hd] fp16
     const int32_t* len;
-    float* part_o; float* part_ml;   // one slot per CTA: [CTA][128 rows][hd] and [CTA][128 rows][2]
+    __half* part_o; float* part_ml;  // one slot per CTA: [CTA][128 rows][hd] (O / l) and [CTA][128 rows][2] (m, l)
     int* item_slots;                 // [A * nKv][2]: the item's first slot and its number of slots
     void* out; int out_dtype;        // [A, G, nH, hd] fp32 or fp16
     __half* out_hi; __half* out_lo;  // optional fp16 pair of the output (the next GEMM's input)
@@ -259,32 +260,31 @@ __device__ __forceinline__ void store_out4(const AttnTcParams& P, int64_t o, flo
 }
 
 // Row r of item (b, g) combined over the item's k slots s0 .. s0 + k - 1 by one
-// warp, 128 * NQ columns of it (lane l owns the 4-column groups gbase + l + 32 q,
-// q < NQ): weights w_s = exp(m_s - M) from the (max, sum) pairs. BATCH slots' loads
-// per lane are in flight at once. Items of many slots (a short call's few items)
-// take NQ = 1 and two warps per row, with twice the loads in flight; items of a
-// few slots take NQ = 2 (each warp's fixed work then counts).
-template <int NQ, int BATCH>
-__device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, int r, int64_t out_row, int gbase) {
-    const int lane = threadIdx.x & 31, ng = P.hd / 4;
-    float4 num[NQ];
+// warp, lane l owning the CPL columns c0 + CPL l .. + CPL - 1: out = sum_s w_s l_s
+// O_s / sum_s w_s l_s with w_s = exp(m_s - M) and O_s the slot's normalised output
+// (fp16). BATCH slots' loads per lane are in flight at once. Items of many slots (a
+// short call's few items) take CPL = 4 and two warps per row, with twice the loads
+// in flight; items of a few slots take CPL = 8 (each warp's fixed work then counts).
+template <int CPL, int BATCH>
+__device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, int r, int64_t out_row, int c0) {
+    using Vec = typename std::conditional<CPL == 8, uint4, uint2>::type;
+    const int lane = threadIdx.x & 31, col = c0 + CPL * lane;
+    const bool mine = col < P.hd;
+    float num[CPL];
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) num[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < CPL; ++e) num[e] = 0.f;
     float den = 0.f, M = -INFINITY;
     for (int sb = 0; sb < k; sb += 32) {
         const int cnt = min(32, k - sb);
         // the first batch of rows and this chunk's (max, sum) pairs go out together: the rows'
         // loads do not depend on the maxima
-        float4 v[BATCH][NQ];
+        Vec v[BATCH];
         auto load_rows = [&](int t0) {
 #pragma unroll
             for (int u = 0; u < BATCH; ++u) {
-                const float4* o = reinterpret_cast<const float4*>(P.part_o + ((int64_t)(s0 + sb + t0 + u) * QROWS + r) * P.hd);
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    const int g4 = gbase + lane + q * 32;
-                    v[u][q] = (t0 + u < cnt && g4 < ng) ? o[g4] : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
+                const __half* o = P.part_o + ((int64_t)(s0 + sb + t0 + u) * QROWS + r) * P.hd + col;
+                Vec z{};
+                v[u] = (t0 + u < cnt && mine) ? *reinterpret_cast<const Vec*>(o) : z;
             }
         };
         load_rows(0);
@@ -299,33 +299,33 @@ __device__ __forceinline__ void merge_row(const AttnTcParams& P, int s0, int k, 
             const float f = __expf(M - Mn);
             den *= f;
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) { num[q].x *= f; num[q].y *= f; num[q].z *= f; num[q].w *= f; }
+            for (int e = 0; e < CPL; ++e) num[e] *= f;
         }
         M = Mn;
-        const float ws = ml.x == -INFINITY ? 0.f : __expf(ml.x - M);
+        const float wl = ml.x == -INFINITY ? 0.f : __expf(ml.x - M) * ml.y;   // w_s l_s
         for (int t0 = 0; t0 < cnt; t0 += BATCH) {
             if (t0 > 0) load_rows(t0);
 #pragma unroll
             for (int u = 0; u < BATCH; ++u) {
-                const float w = __shfl_sync(0xffffffffu, ws, (t0 + u) & 31);
-                const float l = __shfl_sync(0xffffffffu, ml.y, (t0 + u) & 31);
+                const float w = __shfl_sync(0xffffffffu, wl, (t0 + u) & 31);
                 if (t0 + u >= cnt) break;
-                den += w * l;
+                den += w;
                 if (w == 0.f) continue;                // uniform: an empty range
+                const __half2* h = reinterpret_cast<const __half2*>(&v[u]);
 #pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    num[q].x += w * v[u][q].x; num[q].y += w * v[u][q].y;
-                    num[q].z += w * v[u][q].z; num[q].w += w * v[u][q].w;
+                for (int e = 0; e < CPL / 2; ++e) {
+                    const float2 f = __half22float2(h[e]);
+                    num[2 * e] += w * f.x;
+                    num[2 * e + 1] += w * f.y;
                 }
             }
         }
     }
     const float inv = 1.f / den;
+    if (mine) {
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) {
-        const int g4 = gbase + lane + q * 32;
-        if (g4 < ng)
-            store_out4(P, out_row + g4 * 4, make_float4(num[q].x * inv, num[q].y * inv, num[q].z * inv, num[q].w * inv));
+        for (int e = 0; e < CPL; e += 4)
+            store_out4(P, out_row + col + e, make_float4(num[e] * inv, num[e + 1] * inv, num[e + 2] * inv, num[e + 3] * inv));
     }
 }
 
@@ -843,7 +843,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 }
             }
         } else if (item >= 0) {
-            // unnormalised O and (max, sum) per query row into this CTA's slot
+            // O / l and (max, sum) per query row into this CTA's slot
             if (tid == 0 && W.t0 == 0) {                      // the item's first CTA tells the merge its slots
                 P.item_slots[2 * item] = W.s0;
                 P.item_slots[2 * item + 1] = W.k;
@@ -853,29 +853,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 P.part_ml[prow * 2] = any ? m_run : -INFINITY;
                 P.part_ml[prow * 2 + 1] = any ? l_run : 0.f;
             }
-            // The unnormalised O goes through shared memory (the K / V slots are free:
-            // every product has completed): hd / 32 slices of [128 rows x 128 B], 16-byte
-            // chunks swizzled by row (the 128-byte TMA swizzle), then one TMA store per
-            // slice writes whole 128-byte lines instead of scattered 16-byte pieces.
+            // The normalised O = O / l (|O / l| <= max |v|: inside fp16, at fp16's relative
+            // precision; half the bytes of the fp32 sums) goes through shared memory (the K / V
+            // slots are free: every product has completed): hd / 64 slices of [128 rows x
+            // 128 B], 16-byte chunks swizzled by row (the 128-byte TMA swizzle), then one TMA
+            // store per slice writes whole 128-byte lines instead of scattered 16-byte pieces.
             const bool stage_ok = any && ok;
             if (stage_ok) {
-                for (int c = 0; c < hd; c += 32) {
-                    uint32_t o[2][16];
-                    tmem_ld_x16(tO + lane_off + (uint32_t)c, o[0]);
-                    tmem_ld_x16(tO + lane_off + (uint32_t)(c + 16), o[1]);
-                    tmem_ld_wait();
-                    uint8_t* line = sK + (c / 32) * (QROWS * 128) + r * 128;
+                const float inv = 1.f / l_run;
+                for (int c = 0; c < hd; c += 64) {
+                    uint32_t o[4][16];
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4)
-                        *reinterpret_cast<uint4*>(line + ((j4 ^ (r & 7)) * 16)) =
-                            make_uint4(o[j4 >> 2][(j4 & 3) * 4], o[j4 >> 2][(j4 & 3) * 4 + 1],
-                                       o[j4 >> 2][(j4 & 3) * 4 + 2], o[j4 >> 2][(j4 & 3) * 4 + 3]);
+                    for (int q = 0; q < 4; ++q) tmem_ld_x16(tO + lane_off + (uint32_t)(c + 16 * q), o[q]);
+                    tmem_ld_wait();
+                    uint8_t* line = sK + (c / 64) * (QROWS * 128) + r * 128;
+#pragma unroll
+                    for (int j8 = 0; j8 < 8; ++j8) {               // 16-byte chunk j8: columns c + 8 j8 .. + 7
+                        uint32_t h[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int x = 8 * j8 + 2 * e;
+                            h[e] = pack_half2(__uint_as_float(o[x >> 4][x & 15]) * inv,
+                                              __uint_as_float(o[(x + 1) >> 4][(x + 1) & 15]) * inv);
+                        }
+                        *reinterpret_cast<uint4*>(line + ((j8 ^ (r & 7)) * 16)) = make_uint4(h[0], h[1], h[2], h[3]);
+                    }
                 }
                 fence_async_shared();                         // visible to the TMA
             }
             named_barrier_sync(2, kSoftThreads);
             if (tid == 0 && stage_ok) {
-                for (int c = 0; c < hd; c += 32) tma_store_2d(&tmO, sK + (c / 32) * (QROWS * 128), c, slot * QROWS);
+                for (int c = 0; c < hd; c += 64) tma_store_2d(&tmO, sK + (c / 64) * (QROWS * 128), c, slot * QROWS);
                 bulk_commit_group();
                 bulk_wait_all();                              // written before this CTA's shared memory goes
             }
@@ -912,15 +920,15 @@ bool make_kv_map(CUtensorMap* tm, const void* ptr, int64_t rows, int nKv, int hd
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Map over the partial outputs [rows = CTAs x 128][hd] fp32: boxes of 32 columns
+// Map over the partial outputs [rows = CTAs x 128][hd] fp16: boxes of 64 columns
 // (128 bytes, 128-byte swizzle) x 128 rows, for the TMA stores of the epilogue.
-bool make_part_map(CUtensorMap* tm, float* ptr, int64_t rows, int hd) {
+bool make_part_map(CUtensorMap* tm, __half* ptr, int64_t rows, int hd) {
     if (!g_enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)hd, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)hd * 4};
-    cuuint32_t box[2] = {32, (cuuint32_t)QROWS};
+    cuuint64_t strides[1] = {(cuuint64_t)hd * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)QROWS};
     cuuint32_t estr[2] = {1, 1};
-    return g_enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    return g_enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
@@ -951,8 +959,8 @@ size_t attn_tc_smem(int hd) {
 // One warp per output row (b, h, i) of the items on more than one CTA (an item
 // on one CTA wrote its output itself).
 constexpr int kMergeWarps = 8;
-// wpr warps per output row, 128 NQ columns each
-template <int NQ>
+// wpr warps per output row, 32 CPL columns each
+template <int CPL>
 __global__ void __launch_bounds__(kMergeWarps * 32) attn_tc_merge_kernel(AttnTcParams P, int rows, int wpr) {
     pdl_trigger();
     pdl_wait();
@@ -964,8 +972,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_tc_merge_kernel(AttnTcP
     const int item = b * P.nKv + h / P.grp;
     const int k = P.item_slots[2 * item + 1];
     if (k <= 1) return;
-    merge_row<NQ, NQ == 1 ? 16 : 8>(P, P.item_slots[2 * item], k, i * P.grp + h % P.grp,
-                                    (((int64_t)b * P.G + i) * P.nH + h) * P.hd, part * 32 * NQ);
+    merge_row<CPL, CPL == 4 ? 16 : 8>(P, P.item_slots[2 * item], k, i * P.grp + h % P.grp,
+                                      (((int64_t)b * P.G + i) * P.nH + h) * P.hd, part * 32 * CPL);
 }
 
 }  // namespace
@@ -1000,13 +1008,14 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
         !make_kv_map(&tv, a.vc, cache_rows, d.nKv, d.hd) ||
         !make_kv_map(&tkb, vonly ? a.vb : a.kb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
         !make_kv_map(&tvb, a.vb, (int64_t)a.A * d.gamma, d.nKv, d.hd) ||
-        !make_part_map(&to, a.part_o, (int64_t)a.tc_grid * QROWS, d.hd) ||
+        !make_part_map(&to, reinterpret_cast<__half*>(a.part_o), (int64_t)a.tc_grid * QROWS, d.hd) ||
         !make_q_map(&tq, a.q, (int64_t)a.A * d.gamma, d.nKv, d.grp, d.gamma, d.hd))
         return cudaErrorInvalidValue;
     AttnTcParams P{};
     P.A = a.A; P.G = d.gamma; P.nH = d.nH; P.nKv = d.nKv; P.grp = d.grp; P.hd = d.hd; P.capacity = a.capacity;
     P.q_dtype = a.q_dtype; P.grid = a.tc_grid; P.q = a.q; P.len = a.len;
-    P.part_o = a.part_o; P.part_ml = a.part_ml; P.item_slots = a.item_slots; P.status = a.status;
+    P.part_o = reinterpret_cast<__half*>(a.part_o);   // the fp32 workspace holds the fp16 slots
+    P.part_ml = a.part_ml; P.item_slots = a.item_slots; P.status = a.status;
     P.out = a.out; P.out_dtype = a.out_dtype; P.out_hi = a.out_hi; P.out_lo = a.out_lo;
     P.pos0 = a.pos0; P.block_pos = a.block_pos;
     P.k_norm = static_cast<const __nv_bfloat16*>(a.k_norm); P.inv_freq = m->ws.inv_freq;
@@ -1024,7 +1033,7 @@ cudaError_t launch_attention_tc(const dspark_model* m, const AttnArgs& a, cudaSt
     const bool wide = a.tc_grid >= 8 * a.A * d.nKv;
     const int wpr = wide ? (d.hd + 127) / 128 : 1;
     const int64_t warps = (int64_t)rows * wpr;
-    return launch_pdl(wide ? attn_tc_merge_kernel<1> : attn_tc_merge_kernel<2>,
+    return launch_pdl(wide ? attn_tc_merge_kernel<4> : attn_tc_merge_kernel<8>,
                       dim3((unsigned)((warps + kMergeWarps - 1) / kMergeWarps)), dim3(kMergeWarps * 32), 0, s, P, rows,
                       wpr);
 }
