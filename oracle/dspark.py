@@ -31,7 +31,7 @@ import numpy as np
 
 __all__ = [
     "OracleWeights", "dequantize_affine4", "rope_wavelengths", "rms_norm", "apply_rope",
-    "gelu_tanh", "store_rounded", "project_context_kv", "attention_weights", "attend_concat", "attend_split",
+    "gelu_tanh", "store_rounded", "project_context", "project_context_kv", "attention_weights", "attend_concat", "attend_split",
     "embed_block", "decoder_layer", "backbone", "compute_logits", "markov_bias", "markov_walk", "teacher_forced_walk",
     "confidence", "prefix_length", "draft_rows", "block_ids",
 ]
@@ -182,6 +182,20 @@ def store_rounded(x: np.ndarray, store_dtype: Optional[str]) -> np.ndarray:
         return x
     import torch
     return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def project_context(fc, hidden_norm, target_hiddens, eps: float) -> np.ndarray:
+    """``#projectContext``: the context hidden the K/V projection reads, from the
+    target model's tap hiddens (``extract_context_feature`` concatenates them over
+    the taps, in ``target_layer_ids`` order, then ``hidden_norm(fc(.))``).
+
+    ``target_hiddens`` [..., taps * H]; ``fc`` [H, taps * H] stored [out, in]
+    (``matmulW``: x @ fc^T); ``hidden_norm`` [H], the gain of a Gemma4RMSNorm
+    over the last axis with the config's eps. Returns [..., H] in fp64.
+    """
+    x = _f64(target_hiddens)
+    proj = x @ _f64(fc).T
+    return rms_norm(proj, _f64(hidden_norm).reshape(-1), eps)
 
 
 def project_context_kv(W: OracleWeights, hidden, pos0: Sequence[int], lengths: Optional[Sequence[int]] = None,

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "ModelShape", "Workload", "WORKLOADS", "workload", "make_weights",
     "make_round_inputs", "round_meta", "make_append_schedule", "quantize_affine4", "weight_names",
-    "QUANTIZED_MATRICES",
+    "QUANTIZED_MATRICES", "make_context_projection", "make_target_hiddens",
 ]
 
 
@@ -313,3 +313,19 @@ def small_model(dtype: str = "bf16", quant_bits: int = 0, **kw) -> ModelShape:
                 quant_bits=quant_bits)
     base.update(kw)
     return ModelShape(**base)
+
+
+def make_context_projection(m: ModelShape, taps: int, seed: int) -> Dict[str, torch.Tensor]:
+    """Seeded weights of the context feature projection (deepspec.ts ``#projectContext``):
+    ``fc`` [hidden, taps * hidden] N(0, 0.02) and ``hidden_norm`` [hidden] 1 + N(0, 0.02), in the
+    model's dtype (dense: the projection's GEMM reads them as stored)."""
+    H = m.hidden_size
+    fc = _draw(seed, 10_001, (H, taps * H), std=0.02)
+    g = _draw(seed, 10_002, (H,), std=0.02, mean=1.0)
+    return {"fc": _store(fc, m.dtype), "hidden_norm": _store(g, m.dtype)}
+
+
+def make_target_hiddens(m: ModelShape, taps: int, B: int, L: int, seed: int) -> torch.Tensor:
+    """The target model's tap hiddens for B rows of L context positions, concatenated over the
+    taps: [B, L, taps * hidden], N(0, 1) in the model's dtype."""
+    return _store(_draw(seed, 10_003, (B, L, taps * m.hidden_size)), m.dtype)

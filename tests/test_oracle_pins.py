@@ -499,3 +499,63 @@ def test_store_rounded_is_round_to_nearest_even_fp16():
     assert got[4] == -3.140625                    # -3.14159 -> nearest multiple of 2^-9
     assert got[5] == 2 ** -23                     # subnormals: a multiple of 2^-24, tie -> even
     assert np.isinf(got[6])                       # past 65504
+
+
+# --------------------------------------------------------------------------- context feature projection
+
+def _ctx_case(taps=3, H=24, rows=5, seed=0):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((rows, taps * H))
+    fc = g.standard_normal((H, taps * H)) * 0.1
+    w = 1.0 + 0.05 * g.standard_normal(H)
+    return x, fc, w
+
+
+def test_context_projection_identity_fc_is_rms_norm():
+    """taps = 1 and fc = I: the projection reduces to Gemma4RMSNorm of the tap (torch's rms_norm)."""
+    x, _, w = _ctx_case(taps=1)
+    H = x.shape[-1]
+    got = O.project_context(np.eye(H), w, x, 1e-6)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (H,), torch.from_numpy(w), 1e-6).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_context_projection_vs_torch_linear_then_rms_norm():
+    """A non-symmetric fc: x @ fc^T (torch's linear, [out, in] storage) then the norm; a transposed
+    operand would fail here."""
+    x, fc, w = _ctx_case(taps=1, H=16, seed=3)
+    fc = fc + np.triu(np.ones_like(fc))               # clearly not symmetric
+    t = torch.nn.functional.linear(torch.from_numpy(x), torch.from_numpy(fc))
+    ref = torch.nn.functional.rms_norm(t, (16,), torch.from_numpy(w), 1e-6).numpy()
+    np.testing.assert_allclose(O.project_context(fc, w, x, 1e-6), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_context_projection_tap_order_and_zero_tap():
+    """Permuting the taps together with fc's column blocks changes nothing; a tap of zeros
+    drops out (the projection over the remaining taps alone)."""
+    x, fc, w = _ctx_case(taps=3, H=24, seed=5)
+    H = 24
+    blocks = lambda a: [a[..., i * H:(i + 1) * H] for i in range(3)]
+    xb, fb = blocks(x), blocks(fc)
+    perm = [2, 0, 1]
+    xp = np.concatenate([xb[i] for i in perm], -1)
+    fp = np.concatenate([fb[i] for i in perm], -1)
+    base = O.project_context(fc, w, x, 1e-6)
+    np.testing.assert_allclose(O.project_context(fp, w, xp, 1e-6), base, rtol=1e-12, atol=1e-12)
+    xz = np.concatenate([xb[0], np.zeros_like(xb[1]), xb[2]], -1)
+    two = O.project_context(np.concatenate([fb[0], fb[2]], -1), w, np.concatenate([xb[0], xb[2]], -1), 1e-6)
+    np.testing.assert_allclose(O.project_context(fc, w, xz, 1e-6), two, rtol=1e-12, atol=1e-12)
+
+
+def test_context_projection_scale_invariance_and_unit_rms():
+    """Scaling fc by c scales each output row by sqrt((ms + eps) / (ms + eps / c^2)) exactly (ms:
+    the projection's mean square; RMSNorm removes the scale but for eps), and with unit gain each
+    output row has RMS sqrt(ms / (ms + eps))."""
+    x, fc, w = _ctx_case(taps=2, H=20, seed=7)
+    eps, c = 1e-3, 7.5                                   # an eps large enough to show its term
+    base = O.project_context(fc, w, x, eps)
+    ms = np.mean((x @ fc.T) ** 2, axis=-1)
+    factor = np.sqrt((ms + eps) / (ms + eps / c ** 2))[:, None]
+    np.testing.assert_allclose(O.project_context(c * fc, w, x, eps), base * factor, rtol=1e-12, atol=1e-14)
+    out = O.project_context(fc, np.ones(20), x, 1e-6)
+    np.testing.assert_allclose(np.sqrt(np.mean(out ** 2, axis=-1)), np.sqrt(ms / (ms + 1e-6)), rtol=1e-12)
