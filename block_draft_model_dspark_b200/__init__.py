@@ -77,6 +77,9 @@ _PROTOTYPES = {
     "dspark_model_create": (c_i32, [ctypes.POINTER(dspark_config), ctypes.POINTER(dspark_weights), c_vp, c_size, c_vp,
                                     ctypes.POINTER(c_vp)]),
     "dspark_model_destroy": (c_i32, [c_vp]),
+    "dspark_context_features_workspace_bytes": (c_size, [c_vp, c_i32, ctypes.c_int64]),
+    "dspark_project_context_features": (c_i32, [c_vp, ctypes.POINTER(dspark_matrix), c_vp, c_i32, c_vp, c_i32, c_i32,
+                                                c_vp, c_vp, c_size, c_vp]),
     "dspark_project_workspace_bytes": (c_size, [c_vp, ctypes.c_int64]),
     "dspark_project_context_kv": (c_i32, [c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "dspark_append_context_kv": (c_i32, [c_vp, c_vp, c_i32, c_vp, c_vp, ctypes.POINTER(dspark_kv_cache), c_vp,
@@ -324,6 +327,27 @@ class DsparkModel:
         return get_lib().dspark_draft_workspace_bytes(self.handle, A, max_ctx_len)
 
     # -- the calls
+    def dspark_project_context_features(self, target_hiddens, fc, hidden_norm, out=None, ws=None, stream=None):
+        """The context hidden [B, L, H] from the target's tap hiddens [B, L, taps * H]
+        (deepspec.ts #projectContext): rms(target_hiddens @ fc^T, hidden_norm)."""
+        import torch
+        B, L, KT = (int(x) for x in target_hiddens.shape)
+        H = self.shape.hidden_size
+        if KT % H:
+            raise DsparkError(DSPARK_ERR_INVALID_ARGUMENT, "target_hiddens' last axis must be taps * hidden")
+        taps = KT // H
+        if out is None:
+            out = torch.empty(B, L, H, dtype=self.torch_dtype, device=self.device)
+        lib = get_lib()
+        ws = ws if ws is not None else self.workspace(lib.dspark_context_features_workspace_bytes(self.handle, taps,
+                                                                                              B * L))
+        m = dspark_matrix()
+        m.w = fc.data_ptr()
+        _check(lib.dspark_project_context_features(self.handle, ctypes.byref(m), hidden_norm.data_ptr(), taps,
+                                                   target_hiddens.data_ptr(), B, L, out.data_ptr(), ws.data_ptr(),
+                                                   ws.numel(), _stream_ptr(stream)))
+        return out
+
     def dspark_project_context_kv(self, hidden, k_out, v_out, pos0=None, static_pos: int = 0, ws=None, stream=None):
         B, L = int(hidden.shape[0]), int(hidden.shape[1])
         ws = ws if ws is not None else self.workspace(self.project_workspace_bytes(B * L))

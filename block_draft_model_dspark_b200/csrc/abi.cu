@@ -294,6 +294,31 @@ ProjectPlan plan_project(const dspark_model* m, int64_t rows) {
 
 template <typename P> P* at(void* base, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(base) + off); }
 
+// Workspace of the context feature projection: one chunk's GEMM result and its GEMM scratch.
+struct FeaturePlan {
+    int64_t chunk_rows;
+    size_t raw, gscr, gscr_bytes, total;
+};
+FeaturePlan plan_features(const dspark_model* m, int taps, int64_t rows) {
+    const Dims& d = m->d;
+    const int K = taps * d.H;
+    FeaturePlan p{};
+    rows = std::max<int64_t>(rows, 1);
+    p.chunk_rows = std::min<int64_t>(rows, kProjectChunkRows);
+    const GemmFormat f = feature_gemm_format(m);
+    size_t raw = gemm_out_elems(m, (int)p.chunk_rows, d.H, K);
+    p.gscr_bytes = gemm_scratch_bytes(m, (int)p.chunk_rows, d.H, K, f);
+    if (rows % p.chunk_rows) {
+        raw = std::max(raw, gemm_out_elems(m, (int)(rows % p.chunk_rows), d.H, K));
+        p.gscr_bytes = std::max(p.gscr_bytes, gemm_scratch_bytes(m, (int)(rows % p.chunk_rows), d.H, K, f));
+    }
+    Carve c;
+    p.raw = c.take(raw * 4);
+    p.gscr = c.take(p.gscr_bytes);
+    p.total = c.off;
+    return p;
+}
+
 int project_rows(const dspark_model* m, const void* hidden, int B, int Lrows, const int32_t* n_valid,
                  const int32_t* dst_row0, const int32_t* pos0, int static_pos, const KvDest& dst, void* ws,
                  const ProjectPlan& pp, cudaStream_t s) {
@@ -530,6 +555,50 @@ int dspark_model_destroy(dspark_model* m) {
 size_t dspark_project_workspace_bytes(const dspark_model* m, int64_t rows) {
     if (!m || rows < 0) return 0;
     return plan_project(m, rows).total;
+}
+
+size_t dspark_context_features_workspace_bytes(const dspark_model* m, int32_t taps, int64_t rows) {
+    if (!m || taps < 1 || rows < 0) return 0;
+    return plan_features(m, taps, rows).total;
+}
+
+int dspark_project_context_features(const dspark_model* m, const dspark_matrix* fc, const void* hidden_norm,
+                                    int32_t taps, const void* target_hiddens, int32_t B, int32_t L, void* out,
+                                    void* ws, size_t ws_bytes, void* stream) {
+    if (!m || !fc) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "model and fc must be non-NULL");
+    const Dims& d = m->d;
+    if (taps < 1) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "taps must be >= 1");
+    if ((int64_t)taps * d.H > (int64_t)1 << 24) DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "taps * hidden above 2^24");
+    if (fc->scales || fc->biases)
+        DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "fc must be dense (the model dtype); a 4-bit fc is not supported here");
+    if (B < 0 || L < 0) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "B and L must be >= 0");
+    if ((int64_t)B * L == 0) return DSPARK_OK;
+    if ((int64_t)B * L > (int64_t)1 << 30) DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "B * L above 2^30 rows");
+    if (!fc->w || !hidden_norm || !target_hiddens || !out || !ws)
+        DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "fc.w, hidden_norm, target_hiddens, out and ws must be non-NULL");
+    if (!aligned16(fc->w) || !aligned16(target_hiddens) || !aligned16(out) || !aligned16(ws))
+        DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "fc.w, target_hiddens, out and ws must be 16-byte aligned");
+    const int K = taps * d.H;
+    if (use_tensor_cores(m) && K % 64 != 0) DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "taps * hidden must be a multiple of 64");
+    const int64_t rows = (int64_t)B * L;
+    const FeaturePlan pp = plan_features(m, taps, rows);
+    if (ws_bytes < pp.total)
+        DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "ws smaller than dspark_context_features_workspace_bytes(): " + std::to_string(pp.total));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    MatRef fr;
+    fr.w = fc->w; fr.n = d.H; fr.k = K; fr.quant = false;
+    const size_t es = esize(d.dtype);
+    const GemmScratch sc = gemm_scratch_at(at<void>(ws, pp.gscr), pp.gscr_bytes);
+    for (int64_t r0 = 0; r0 < rows; r0 += pp.chunk_rows) {
+        const int nr = (int)std::min<int64_t>(pp.chunk_rows, rows - r0);
+        const void* X = static_cast<const char*>(target_hiddens) + (size_t)r0 * K * es;
+        PartView view;
+        cudaError_t e = run_context_features(m, X, nr, fr, at<float>(ws, pp.raw), sc, &view, s);
+        if (e == cudaSuccess)
+            e = launch_context_norm(m, view, nr, hidden_norm, static_cast<char*>(out) + (size_t)r0 * d.H * es, s);
+        if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("context feature projection launch: ") + cudaGetErrorString(e));
+    }
+    return DSPARK_OK;
 }
 
 int dspark_project_context_kv(const dspark_model* m, const void* hidden, int32_t B, int32_t L, int32_t static_pos,

@@ -51,6 +51,8 @@ GemmFormat round_gemm_format(const dspark_model* m, int M) {
 
 GemmFormat project_gemm_format(const dspark_model* m) { return {1, m->d.quant ? tc::kWQ4AsF16 : tc::kWBf16}; }
 
+GemmFormat feature_gemm_format(const dspark_model*) { return {1, tc::kWBf16}; }
+
 int attention_key_chunk(const dspark_model* m, int A, int max_ctx_len) {
     // context chunks so that A * nKv (tensor cores) or A * nH (CUDA cores) CTAs per split cover the GPU ~2x
     const Dims& d = m->d;
@@ -148,6 +150,26 @@ cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U,
     // a scan of U gives the same statistics
     KernelTimer t(DSPARK_TIMER_ROWS, s, 4.0 * M * d.V, 0.0);
     return launch_tile_stats(m, U, M, ts, s);
+}
+
+cudaError_t run_context_features(const dspark_model* m, const void* X, int nrows, const MatRef& fc, float* raw,
+                                 const GemmScratch& sc, PartView* view, cudaStream_t s) {
+    const Dims& d = m->d;
+    const int N = d.H, K = (int)fc.k;
+    const double es = d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0;
+    KernelTimer t(DSPARK_TIMER_KV_PROJECT, s, es * ((double)N * K + (double)nrows * K + (double)nrows * N),
+                  2.0 * nrows * (double)N * K);
+    if (use_tensor_cores(m)) {
+        // the caller's rows and fc in bf16, straight from TMA (products exact in fp32)
+        const tc::GemmPlan p = tc::plan_gemm(m->num_sms, nrows, N, K, 1, false, false, tc::kWBf16);
+        tc_view(p, raw, sc, view);
+        return tc::launch_gemm_tc(p, fc.w, N, X, nullptr, raw, N, 0.f, sc.part, m->ws.status, s);
+    }
+    const int S = simt_splits(m, nrows, N, K);
+    *view = PartView{};
+    view->p = raw; view->S = S; view->stride = (int64_t)nrows * N; view->ld = N;
+    return launch_simt_gemm(X, K, d.dtype, d.dtype, fc, d.group, nrows, N, K, S, raw, N, (int64_t)nrows * N, false,
+                            0.f, s);
 }
 
 cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, const RowsPlan& rp, const KvDest& dst,

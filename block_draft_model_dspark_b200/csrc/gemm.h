@@ -19,6 +19,7 @@ bool act_pair(const dspark_model* m, int M);
 struct GemmFormat { int np, wfmt; };
 GemmFormat round_gemm_format(const dspark_model* m, int M);   // the round's layer GEMMs and lm-head
 GemmFormat project_gemm_format(const dspark_model* m);        // the context K/V projection
+GemmFormat feature_gemm_format(const dspark_model* m);        // the context feature projection (dense fc)
 // Scratch of the tensor-core GEMM's stream-K partial tiles, read back by the
 // consumer through its PartView.
 struct GemmScratch {
@@ -37,6 +38,10 @@ cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, in
 cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U, const TileStats& ts, cudaStream_t s);
 // Context K/V of `nrows` rows of the caller's hidden X (model dtype) into `dst`; x16 holds
 // nrows * H fp16 values for the 4-bit GEMM's input (unused otherwise).
+// raw = X @ fc^T for `nrows` rows of the caller's tap hiddens X (model dtype, [nrows, fc.k]) and a dense
+// fc [H, fc.k] (model dtype); *view reads the result (deepspec.ts #projectContext, before its norm).
+cudaError_t run_context_features(const dspark_model* m, const void* X, int nrows, const MatRef& fc, float* raw,
+                                 const GemmScratch& sc, PartView* view, cudaStream_t s);
 cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, const RowsPlan& rp, const KvDest& dst,
                               float* raw, const GemmScratch& sc, void* x16, cudaStream_t s);
 cudaError_t run_attention(const dspark_model* m, const AttnArgs& a, cudaStream_t s);

@@ -251,6 +251,10 @@ struct RowsPlan {
     const int32_t* pos0;     // device [B] position of t = 0, or null (static_pos)
     int static_pos;
 };
+// Context features (deepspec.ts #projectContext): out[r] = rms(raw[r], gain) for `nrows` rows of H,
+// in the model's dtype.
+cudaError_t launch_context_norm(const dspark_model* m, const PartView& raw, int nrows, const void* gain, void* out,
+                                cudaStream_t s);
 cudaError_t launch_kv_epilogue(const dspark_model* m, const PartView& raw, const RowsPlan& rp, const KvDest& dst,
                                cudaStream_t s);
 // Validates an append's device counts (0 <= n_new[b] <= Lnew_max, len[b] + n_new[b] <= capacity);

@@ -95,6 +95,28 @@ __global__ void kv_epilogue_kernel(PartView raw, RowsPlan rp, KvDest dst, const 
     store_any(dst.k, o + i + half, kv_dtype, k2 * cs + k1 * sn);
 }
 
+// ------------------------------------------------------------------ context features
+// deepspec.ts #projectContext: out[r] = rms(raw[r], hidden_norm), raw = the taps' hiddens @ fc^T.
+// grid rows, block 256; the row's H values in shared memory between the two passes.
+__global__ void context_norm_kernel(PartView raw, int H, const void* __restrict__ gain, float eps, int dtype,
+                                    void* __restrict__ out) {
+    extern __shared__ float ctx_row[];
+    __shared__ float red[32];
+    pdl_trigger();
+    pdl_wait();
+    const int r = blockIdx.x;
+    float ss = 0.f;
+    for (int j = threadIdx.x; j < H; j += blockDim.x) {
+        const float x = raw.sum(r, j);
+        ctx_row[j] = x;                                   // each thread reads back only its own columns
+        ss += x * x;
+    }
+    ss = block_sum(ss, red);
+    const float rinv = rsqrtf(ss / (float)H + eps);
+    for (int j = threadIdx.x; j < H; j += blockDim.x)
+        store_any(out, (int64_t)r * H + j, dtype, ctx_row[j] * rinv * load_any(gain, j, dtype));
+}
+
 // The append's device-side validation (the accepted-row counts come from the
 // caller's device memory, so the host cannot check them): every row must have
 // 0 <= n_new[b] <= Lnew_max and len[b] + n_new[b] <= capacity. If any row
@@ -579,6 +601,14 @@ cudaError_t launch_kv_epilogue(const dspark_model* m, const PartView& raw, const
     dim3 grid(rp.nrows, d.Lyr * d.nKv);
     return launch_pdl(kv_epilogue_kernel, grid, dim3(d.hd / 2), 0, s, raw, rp, dst, m->ws.inv_freq, kn, d.nKv, d.hd,
                       d.eps, d.dtype, d.kv_dtype, m->ws.status);
+}
+
+cudaError_t launch_context_norm(const dspark_model* m, const PartView& raw, int nrows, const void* gain, void* out,
+                                cudaStream_t s) {
+    const Dims& d = m->d;
+    if (nrows <= 0) return cudaSuccess;
+    return launch_pdl(context_norm_kernel, dim3(nrows), dim3(256), (size_t)d.H * sizeof(float), s, raw, d.H, gain,
+                      d.eps, d.dtype, out);
 }
 
 cudaError_t launch_append_check(const int32_t* n_new, const int32_t* len, int B, int Lnew_max, int capacity,

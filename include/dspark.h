@@ -213,6 +213,32 @@ int dspark_model_destroy(dspark_model* model);
 size_t dspark_project_workspace_bytes(const dspark_model* model, int64_t rows);
 
 /*
+ * Context feature projection (deepspec.ts #projectContext): the context hidden
+ * the projections below read, from the target model's tap hiddens. The caller
+ * concatenates, per context row, the target's hiddens at the taps
+ * (extract_context_feature: the post-layer output of every target_layer_ids
+ * entry, in that order) into target_hiddens; then for every row
+ *   out[b,t] = rms(target_hiddens[b,t] @ fc^T, hidden_norm)
+ * with rms the Gemma4RMSNorm of the config's eps (computed in fp32).
+ *   fc              dense matrix (.w only) [hidden, taps * hidden] in the model
+ *                   dtype, stored [out, in]; a 4-bit fc (.scales set) is refused
+ *                   with DSPARK_ERR_UNSUPPORTED
+ *   hidden_norm     device T [hidden]
+ *   target_hiddens  device T [B, L, taps * hidden]
+ *   out             device T [B, L, hidden]: the `hidden` of
+ *                   dspark_project_context_kv / dspark_append_context_kv
+ *   ws              >= dspark_context_features_workspace_bytes(model, taps, B * L)
+ * fc.w, target_hiddens, out and ws must be 16-byte aligned; on a bf16 model
+ * taps * hidden must be a multiple of 64. Argument errors return before any
+ * launch. The weights are the caller's (not part of dspark_weights): the
+ * projection runs once per context row, outside the draft round.
+ */
+size_t dspark_context_features_workspace_bytes(const dspark_model* model, int32_t taps, int64_t rows);
+int dspark_project_context_features(const dspark_model* model, const dspark_matrix* fc, const void* hidden_norm,
+                                    int32_t taps, const void* target_hiddens, int32_t B, int32_t L, void* out,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Context K/V projection (deepspec.ts #projectContextKVRows; page 75
  * projectContextKV). For every layer l, batch row b < B and context row
  * t < L, with k_raw = hidden[b,t,:] @ k_proj_l^T viewed [nKv, hd]:
