@@ -329,7 +329,8 @@ class DsparkModel:
     # -- the calls
     def dspark_project_context_features(self, target_hiddens, fc, hidden_norm, out=None, ws=None, stream=None):
         """The context hidden [B, L, H] from the target's tap hiddens [B, L, taps * H]
-        (deepspec.ts #projectContext): rms(target_hiddens @ fc^T, hidden_norm)."""
+        (deepspec.ts #projectContext): rms(target_hiddens @ fc^T, hidden_norm). ``fc`` is a dense
+        tensor [H, taps * H] in the model dtype, or a 4-bit affine triple (words, scales, biases)."""
         import torch
         B, L, KT = (int(x) for x in target_hiddens.shape)
         H = self.shape.hidden_size
@@ -342,7 +343,10 @@ class DsparkModel:
         ws = ws if ws is not None else self.workspace(lib.dspark_context_features_workspace_bytes(self.handle, taps,
                                                                                               B * L))
         m = dspark_matrix()
-        m.w = fc.data_ptr()
+        if isinstance(fc, (tuple, list)):
+            m.w, m.scales, m.biases = (t.data_ptr() for t in fc)
+        else:
+            m.w = fc.data_ptr()
         _check(lib.dspark_project_context_features(self.handle, ctypes.byref(m), hidden_norm.data_ptr(), taps,
                                                    target_hiddens.data_ptr(), B, L, out.data_ptr(), ws.data_ptr(),
                                                    ws.numel(), _stream_ptr(stream)))

@@ -306,10 +306,12 @@ FeaturePlan plan_features(const dspark_model* m, int taps, int64_t rows) {
     rows = std::max<int64_t>(rows, 1);
     p.chunk_rows = std::min<int64_t>(rows, kProjectChunkRows);
     const GemmFormat f = feature_gemm_format(m);
-    size_t raw = gemm_out_elems(m, (int)p.chunk_rows, d.H, K);
+    // the larger of the model's GEMM result and the CUDA-core one (a 4-bit fc)
+    auto out_elems = [&](int M) { return std::max(gemm_out_elems(m, M, d.H, K), simt_gemm_out_elems(m, M, d.H, K)); };
+    size_t raw = out_elems((int)p.chunk_rows);
     p.gscr_bytes = gemm_scratch_bytes(m, (int)p.chunk_rows, d.H, K, f);
     if (rows % p.chunk_rows) {
-        raw = std::max(raw, gemm_out_elems(m, (int)(rows % p.chunk_rows), d.H, K));
+        raw = std::max(raw, out_elems((int)(rows % p.chunk_rows)));
         p.gscr_bytes = std::max(p.gscr_bytes, gemm_scratch_bytes(m, (int)(rows % p.chunk_rows), d.H, K, f));
     }
     Carve c;
@@ -569,8 +571,10 @@ int dspark_project_context_features(const dspark_model* m, const dspark_matrix* 
     const Dims& d = m->d;
     if (taps < 1) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "taps must be >= 1");
     if ((int64_t)taps * d.H > (int64_t)1 << 24) DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "taps * hidden above 2^24");
-    if (fc->scales || fc->biases)
-        DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "fc must be dense (the model dtype); a 4-bit fc is not supported here");
+    const bool q4 = fc->scales || fc->biases;          // a 4-bit affine fc
+    if (q4 && !(fc->scales && fc->biases)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "a 4-bit fc needs both scales and biases");
+    if (q4 && ((int64_t)taps * d.H) % d.group != 0)
+        DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "taps * hidden must be a multiple of the quantization group");
     if (B < 0 || L < 0) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "B and L must be >= 0");
     if ((int64_t)B * L == 0) return DSPARK_OK;
     if ((int64_t)B * L > (int64_t)1 << 30) DSPARK_FAIL(DSPARK_ERR_UNSUPPORTED, "B * L above 2^30 rows");
@@ -586,7 +590,8 @@ int dspark_project_context_features(const dspark_model* m, const dspark_matrix* 
         DSPARK_FAIL(DSPARK_ERR_WORKSPACE, "ws smaller than dspark_context_features_workspace_bytes(): " + std::to_string(pp.total));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     MatRef fr;
-    fr.w = fc->w; fr.n = d.H; fr.k = K; fr.quant = false;
+    fr.w = fc->w; fr.n = d.H; fr.k = K; fr.quant = q4;
+    fr.scales = static_cast<const bf16*>(fc->scales); fr.biases = static_cast<const bf16*>(fc->biases);
     const size_t es = esize(d.dtype);
     const GemmScratch sc = gemm_scratch_at(at<void>(ws, pp.gscr), pp.gscr_bytes);
     for (int64_t r0 = 0; r0 < rows; r0 += pp.chunk_rows) {

@@ -79,6 +79,10 @@ size_t gemm_out_elems(const dspark_model* m, int M, int N, int K) {
     return (size_t)simt_splits(m, M, N, K) * M * N;
 }
 
+size_t simt_gemm_out_elems(const dspark_model* m, int M, int N, int K) {
+    return M <= 0 ? 0 : (size_t)simt_splits(m, M, N, K) * M * N;
+}
+
 size_t gemm_scratch_bytes(const dspark_model* m, int M, int N, int K, const GemmFormat& f) {
     if (M <= 0 || !use_tensor_cores(m)) return 0;
     const tc::GemmPlan p = tc::plan_gemm(m->num_sms, M, N, K, f.np, false, false, f.wfmt);
@@ -159,8 +163,9 @@ cudaError_t run_context_features(const dspark_model* m, const void* X, int nrows
     const double es = d.dtype == DSPARK_DTYPE_F32 ? 4.0 : 2.0;
     KernelTimer t(DSPARK_TIMER_KV_PROJECT, s, es * ((double)N * K + (double)nrows * K + (double)nrows * N),
                   2.0 * nrows * (double)N * K);
-    if (use_tensor_cores(m)) {
-        // the caller's rows and fc in bf16, straight from TMA (products exact in fp32)
+    if (use_tensor_cores(m) && !fc.quant) {
+        // the caller's rows and fc in bf16, straight from TMA (products exact in fp32); a 4-bit
+        // fc takes the CUDA-core GEMM below (dequantized on load)
         const tc::GemmPlan p = tc::plan_gemm(m->num_sms, nrows, N, K, 1, false, false, tc::kWBf16);
         tc_view(p, raw, sc, view);
         return tc::launch_gemm_tc(p, fc.w, N, X, nullptr, raw, N, 0.f, sc.part, m->ws.status, s);

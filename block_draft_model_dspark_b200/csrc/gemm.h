@@ -29,6 +29,8 @@ struct GemmScratch {
 // [M, K] x [N, K]^T product, and bytes of GemmScratch it needs.
 size_t gemm_out_elems(const dspark_model* m, int M, int N, int K);
 size_t gemm_scratch_bytes(const dspark_model* m, int M, int N, int K, const GemmFormat& f);
+// fp32 elements of the CUDA-core GEMM's split-K result for the same product (any model).
+size_t simt_gemm_out_elems(const dspark_model* m, int M, int N, int K);
 GemmScratch gemm_scratch_at(void* base, size_t bytes);
 // out = X @ W^T for an activation X (fp32, or its bf16 pair on tensor cores); *view reads the result.
 cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, int M, int N, int K, float* out,
@@ -38,8 +40,9 @@ cudaError_t run_gemm(const dspark_model* m, const ActBuf& X, const MatRef& W, in
 cudaError_t run_lm_head(const dspark_model* m, const ActBuf& x, int M, float* U, const TileStats& ts, cudaStream_t s);
 // Context K/V of `nrows` rows of the caller's hidden X (model dtype) into `dst`; x16 holds
 // nrows * H fp16 values for the 4-bit GEMM's input (unused otherwise).
-// raw = X @ fc^T for `nrows` rows of the caller's tap hiddens X (model dtype, [nrows, fc.k]) and a dense
-// fc [H, fc.k] (model dtype); *view reads the result (deepspec.ts #projectContext, before its norm).
+// raw = X @ fc^T for `nrows` rows of the caller's tap hiddens X (model dtype, [nrows, fc.k]) and fc
+// [H, fc.k] (dense in the model dtype, or 4-bit affine: the CUDA-core GEMM); *view reads the result
+// (deepspec.ts #projectContext, before its norm).
 cudaError_t run_context_features(const dspark_model* m, const void* X, int nrows, const MatRef& fc, float* raw,
                                  const GemmScratch& sc, PartView* view, cudaStream_t s);
 cudaError_t run_kv_projection(const dspark_model* m, const void* X, int nrows, const RowsPlan& rp, const KvDest& dst,

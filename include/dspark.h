@@ -220,9 +220,13 @@ size_t dspark_project_workspace_bytes(const dspark_model* model, int64_t rows);
  * entry, in that order) into target_hiddens; then for every row
  *   out[b,t] = rms(target_hiddens[b,t] @ fc^T, hidden_norm)
  * with rms the Gemma4RMSNorm of the config's eps (computed in fp32).
- *   fc              dense matrix (.w only) [hidden, taps * hidden] in the model
- *                   dtype, stored [out, in]; a 4-bit fc (.scales set) is refused
- *                   with DSPARK_ERR_UNSUPPORTED
+ *   fc              [hidden, taps * hidden] stored [out, in]: dense in the model
+ *                   dtype (.w only; a bf16 model runs it on the tensor cores), or
+ *                   4-bit affine (.w the packed words [hidden, taps*hidden/8],
+ *                   .scales / .biases bf16 [hidden, taps*hidden/group], group the
+ *                   model's quant_group_size, 64 for a dense model: dequantized on
+ *                   load by the CUDA-core GEMM; both or neither of scales and
+ *                   biases, else DSPARK_ERR_INVALID_ARGUMENT)
  *   hidden_norm     device T [hidden]
  *   target_hiddens  device T [B, L, taps * hidden]
  *   out             device T [B, L, hidden]: the `hidden` of

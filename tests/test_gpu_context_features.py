@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from oracle import dspark as O
-from synthetic import make_context_projection, make_target_hiddens, small_model
+from synthetic import make_context_projection, make_target_hiddens, quantize_affine4, small_model
 from parity_util import as_stored, assert_close, build, ensure_built
 
 pytestmark = pytest.mark.gpu
@@ -30,6 +30,24 @@ def test_context_features_match_oracle(dtype, taps):
     ref = O.project_context(proj["fc"], proj["hidden_norm"], x, m.rms_norm_eps)
     assert out.dtype == model.torch_dtype
     assert_close(out.float().cpu().numpy(), ref, dtype, f"context features ({dtype}, {taps} taps)")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_context_features_with_a_4bit_fc(dtype):
+    """A 4-bit affine fc (group 64), dequantized on load, against the oracle on the exact
+    dequantized matrix."""
+    m = small_model(dtype=dtype)
+    cpu, W, model = build(m, 85)
+    taps = 2
+    proj = make_context_projection(m, taps, 13)
+    q, sc, bi = quantize_affine4(proj["fc"].float(), 64)
+    x = make_target_hiddens(m, taps, 2, 33, 14)
+    out = model.dspark_project_context_features(x.cuda(), (q.cuda(), sc.cuda(), bi.cuda()),
+                                                proj["hidden_norm"].cuda())
+    torch.cuda.synchronize()
+    fc = O.dequantize_affine4(q, sc, bi, 64)
+    ref = O.project_context(fc, proj["hidden_norm"], x, m.rms_norm_eps)
+    assert_close(out.float().cpu().numpy(), ref, dtype, f"context features, 4-bit fc ({dtype})")
 
 
 def test_context_features_over_two_chunks():
@@ -83,10 +101,10 @@ def test_context_features_refusals():
     ws = model.workspace(lib.dspark_context_features_workspace_bytes(model.handle, 2, 8))
     mat = dsp.dspark_matrix()
     mat.w = fc.data_ptr()
-    mat.scales = fc.data_ptr()                        # a 4-bit fc: refused
+    mat.scales = fc.data_ptr()                        # a 4-bit fc needs scales and biases
     rc = lib.dspark_project_context_features(model.handle, ctypes.byref(mat), g.data_ptr(), 2, x.data_ptr(), 1, 8,
                                              out.data_ptr(), ws.data_ptr(), ws.numel(), None)
-    assert rc == dsp.DSPARK_ERR_UNSUPPORTED
+    assert rc == dsp.DSPARK_ERR_INVALID_ARGUMENT
     mat.scales = None
     rc = lib.dspark_project_context_features(model.handle, ctypes.byref(mat), g.data_ptr(), 0, x.data_ptr(), 1, 8,
                                              out.data_ptr(), ws.data_ptr(), ws.numel(), None)
