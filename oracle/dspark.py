@@ -33,7 +33,7 @@ __all__ = [
     "OracleWeights", "dequantize_affine4", "rope_wavelengths", "rms_norm", "apply_rope",
     "gelu_tanh", "store_rounded", "project_context", "project_context_kv", "attention_weights", "attend_concat", "attend_split",
     "embed_block", "decoder_layer", "backbone", "compute_logits", "markov_bias", "markov_walk", "teacher_forced_walk",
-    "confidence", "prefix_length", "draft_rows", "block_ids",
+    "confidence", "prefix_length", "prune_lengths", "draft_rows", "block_ids",
 ]
 
 
@@ -453,6 +453,25 @@ def prefix_length(conf_row: Sequence[float], threshold: float, gamma: int) -> in
         if c < threshold:
             return k
     return gamma
+
+
+def prune_lengths(conf: np.ndarray, thresholds: Sequence[float]) -> np.ndarray:
+    """Confidence-scheduled draft-length pruning (Alg 1, the DFlash generator's
+    ``forwardInfer``, "@mlx-bun/inference 0.0.0-stage -> 1.0.0"): row b keeps
+    positions [0, k) where k is the first position >= 1 whose confidence is
+    below that position's threshold, else the whole block; position 0 always
+    survives. ``conf`` [A, gamma]; ``thresholds`` [gamma] (entry 0 unused).
+    A NaN confidence is not below any threshold.
+    """
+    conf = np.asarray(conf, dtype=np.float64)
+    A, gamma = conf.shape
+    out = np.full(A, gamma, dtype=np.int64)
+    for b in range(A):
+        for k in range(1, gamma):
+            if conf[b, k] < float(thresholds[k]):
+                out[b] = k
+                break
+    return out
 
 
 def draft_rows(W: OracleWeights, ctx_kv: List[List[tuple]], anchors: Sequence[int], block_pos: Sequence[int],

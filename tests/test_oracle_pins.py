@@ -559,3 +559,24 @@ def test_context_projection_scale_invariance_and_unit_rms():
     np.testing.assert_allclose(O.project_context(c * fc, w, x, eps), base * factor, rtol=1e-12, atol=1e-14)
     out = O.project_context(fc, np.ones(20), x, 1e-6)
     np.testing.assert_allclose(np.sqrt(np.mean(out ** 2, axis=-1)), np.sqrt(ms / (ms + 1e-6)), rtol=1e-12)
+
+
+# --------------------------------------------------------------------------- Alg 1 draft-length pruning
+
+def test_prune_lengths_hand_worked_and_special_cases():
+    """Hand-worked rows, then the rule's closed forms: position 0 survives even below its
+    threshold; a value equal to the threshold is not below it; zero thresholds never prune
+    (confidences are >= 0); thresholds above 1 prune at position 1; gamma = 1 keeps 1."""
+    conf = np.array([[0.10, 0.90, 0.20, 0.95],     # 0 below, kept; first k >= 1 below: 2
+                     [0.90, 0.80, 0.70, 0.60],     # nothing below 0.5: gamma
+                     [0.90, 0.49, 0.99, 0.10],     # 1
+                     [0.90, 0.50, 0.50, 0.50]])    # equal is not below: gamma
+    np.testing.assert_array_equal(O.prune_lengths(conf, [0.5] * 4), [2, 4, 1, 4])
+    # per-position thresholds: row 0 stops at 2 (0.20 < 0.3); rows 1-3 at 3 (0.60, 0.10, 0.50 < 0.65)
+    np.testing.assert_array_equal(O.prune_lengths(conf, [0.0, 0.3, 0.3, 0.65]), [2, 3, 3, 3])
+    g = np.random.default_rng(5).random((7, 6))
+    np.testing.assert_array_equal(O.prune_lengths(g, [0.0] * 6), [6] * 7)
+    np.testing.assert_array_equal(O.prune_lengths(g, [2.0] * 6), [1] * 7)
+    np.testing.assert_array_equal(O.prune_lengths(g[:, :1], [2.0]), [1] * 7)
+    nan = np.array([[0.9, np.nan, 0.1]])
+    np.testing.assert_array_equal(O.prune_lengths(nan, [0.5] * 3), [2])
