@@ -77,6 +77,7 @@ _PROTOTYPES = {
     "dspark_model_create": (c_i32, [ctypes.POINTER(dspark_config), ctypes.POINTER(dspark_weights), c_vp, c_size, c_vp,
                                     ctypes.POINTER(c_vp)]),
     "dspark_model_destroy": (c_i32, [c_vp]),
+    "dspark_prune_lengths": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp]),
     "dspark_context_features_workspace_bytes": (c_size, [c_vp, c_i32, ctypes.c_int64]),
     "dspark_project_context_features": (c_i32, [c_vp, ctypes.POINTER(dspark_matrix), c_vp, c_i32, c_vp, c_i32, c_i32,
                                                 c_vp, c_vp, c_size, c_vp]),
@@ -209,6 +210,19 @@ def _matrix(tensors: Dict, name: str) -> dspark_matrix:
     elif name in tensors:
         m.w = tensors[name].data_ptr()
     return m
+
+
+def prune_lengths(conf, thresholds, lengths=None, stream=None):
+    """Alg 1 draft-length pruning on the device (``dspark_prune_lengths``): the first position
+    k >= 1 of each row with conf[b, k] < thresholds[k], else gamma. ``conf`` float32 [A, gamma],
+    ``thresholds`` float32 [gamma], both CUDA tensors; returns int32 lengths [A]."""
+    import torch
+    A, gamma = int(conf.shape[0]), int(conf.shape[1])
+    if lengths is None:
+        lengths = torch.empty(A, dtype=torch.int32, device=conf.device)
+    _check(get_lib().dspark_prune_lengths(conf.data_ptr(), A, gamma, thresholds.data_ptr(), lengths.data_ptr(),
+                                          _stream_ptr(stream)))
+    return lengths
 
 
 class KvCache:

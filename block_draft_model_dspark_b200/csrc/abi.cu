@@ -559,6 +559,17 @@ size_t dspark_project_workspace_bytes(const dspark_model* m, int64_t rows) {
     return plan_project(m, rows).total;
 }
 
+int dspark_prune_lengths(const float* conf, int32_t A, int32_t gamma, const float* thresholds, int32_t* lengths,
+                         void* stream) {
+    if (A < 0 || A > (1 << 30)) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "A must be in [0, 2^30]");
+    if (gamma < 1) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "gamma must be >= 1");
+    if (A == 0) return DSPARK_OK;
+    if (!conf || !thresholds || !lengths) DSPARK_FAIL(DSPARK_ERR_INVALID_ARGUMENT, "conf, thresholds and lengths must be non-NULL");
+    cudaError_t e = launch_prune_lengths(conf, A, gamma, thresholds, lengths, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) DSPARK_FAIL(DSPARK_ERR_CUDA, std::string("prune lengths launch: ") + cudaGetErrorString(e));
+    return DSPARK_OK;
+}
+
 size_t dspark_context_features_workspace_bytes(const dspark_model* m, int32_t taps, int64_t rows) {
     if (!m || taps < 1 || rows < 0) return 0;
     return plan_features(m, taps, rows).total;

@@ -251,6 +251,9 @@ struct RowsPlan {
     const int32_t* pos0;     // device [B] position of t = 0, or null (static_pos)
     int static_pos;
 };
+// Alg 1 draft-length pruning: lengths[b] = first k >= 1 with conf[b, k] < thr[k], else gamma.
+cudaError_t launch_prune_lengths(const float* conf, int A, int gamma, const float* thr, int32_t* lengths,
+                                 cudaStream_t s);
 // Context features (deepspec.ts #projectContext): out[r] = rms(raw[r], gain) for `nrows` rows of H,
 // in the model's dtype.
 cudaError_t launch_context_norm(const dspark_model* m, const PartView& raw, int nrows, const void* gain, void* out,

@@ -530,6 +530,21 @@ __global__ void lengths_kernel(const float* __restrict__ conf, int A, int gamma,
     lengths[b] = len;
 }
 
+// Alg 1 (the DFlash generator's confidence-scheduled draft-length pruning):
+// lengths[b] = first k >= 1 with conf[b, k] < thr[k], else gamma (position 0
+// always survives; a NaN confidence is not below any threshold).
+__global__ void prune_lengths_kernel(const float* __restrict__ conf, int A, int gamma, const float* __restrict__ thr,
+                                     int32_t* __restrict__ lengths) {
+    pdl_trigger();
+    pdl_wait();
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= A) return;
+    int len = gamma;
+    for (int k = 1; k < gamma; ++k)
+        if (conf[(int64_t)b * gamma + k] < thr[k]) { len = k; break; }
+    lengths[b] = len;
+}
+
 // Threads of a full-row kernel: enough that each holds at most kMaxPer
 // columns, about 8 columns per thread, and at most 512 (the kernels use up
 // to ~80 registers a thread; 512 x 80 fits a block's register file).
@@ -609,6 +624,12 @@ cudaError_t launch_context_norm(const dspark_model* m, const PartView& raw, int 
     if (nrows <= 0) return cudaSuccess;
     return launch_pdl(context_norm_kernel, dim3(nrows), dim3(256), (size_t)d.H * sizeof(float), s, raw, d.H, gain,
                       d.eps, d.dtype, out);
+}
+
+cudaError_t launch_prune_lengths(const float* conf, int A, int gamma, const float* thr, int32_t* lengths,
+                                 cudaStream_t s) {
+    if (A <= 0) return cudaSuccess;
+    return launch_pdl(prune_lengths_kernel, dim3((A + 127) / 128), dim3(128), 0, s, conf, A, gamma, thr, lengths);
 }
 
 cudaError_t launch_append_check(const int32_t* n_new, const int32_t* len, int B, int Lnew_max, int capacity,

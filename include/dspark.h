@@ -213,6 +213,21 @@ int dspark_model_destroy(dspark_model* model);
 size_t dspark_project_workspace_bytes(const dspark_model* model, int64_t rows);
 
 /*
+ * Confidence-scheduled draft-length pruning (Alg 1 of the DFlash generator's
+ * forwardInfer, "@mlx-bun/inference 0.0.0-stage -> 1.0.0": calibrated
+ * per-position thresholds, or one minConf for every position): for row b,
+ *   lengths[b] = the first k >= 1 with conf[b, k] < thresholds[k], else gamma
+ * (position 0 always survives, unlike dspark_draft_rows' confidence_threshold
+ * rule, which can keep none; a NaN confidence is not below any threshold).
+ *   conf        device float [A, gamma] (the confidences dspark_draft_rows wrote)
+ *   thresholds  device float [gamma] (entry 0 unused)
+ *   lengths     device int32 [A]
+ * Enqueued on `stream`; argument errors return before any launch.
+ */
+int dspark_prune_lengths(const float* conf, int32_t A, int32_t gamma, const float* thresholds, int32_t* lengths,
+                         void* stream);
+
+/*
  * Context feature projection (deepspec.ts #projectContext): the context hidden
  * the projections below read, from the target model's tap hiddens. The caller
  * concatenates, per context row, the target's hiddens at the taps
